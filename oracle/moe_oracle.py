@@ -1,0 +1,462 @@
+"""Plain, slow, double-precision CPU oracle of the sparse MoE FFN layer forward.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` use it.  It shares no code with the CUDA library and never reads
+anything that the CUDA library produced, except where a test deliberately
+cross-feeds the GPU's routing decisions into the oracle's permutation step.
+
+Every step follows the source pages in their order and notation; each function
+names the page and section it restates.  Page tags used below:
+
+  [Practice]  "混合专家模型（MoE）架构实战：路由策略、负载均衡与工程实现"
+              (deepseekmodel.com blog)
+  [Compass]   "llm-compass: MoE" (brenchcc.github.io, architecture/moe)
+  [Taste]     "MoE common taste in open models" (r00kie-liu.github.io)
+  [Landscape] "MoE landscape" (cyk1337 paper-daily topic page)
+  [History]   "MoE 的工业进化：从 1.6 万亿的 Switch Transformer 到 2.8 万亿的 Kimi K3"
+              (alishangtian.com)
+
+Where the pages are silent or disagree, the reading taken is stated at the
+function.  All arithmetic is float64; integer decisions (top-k, capacity,
+positions) are made on float64 scores.  Library primitives used as single steps:
+``numpy.matmul``, ``numpy.argsort(kind="stable")``, ``numpy.exp``/``log``.
+
+Pinned by ``tests/test_oracle_pins.py`` (worked example, brute-force top-k, closed
+forms, invariants); no function here is "parity unpinned".
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Callable, Optional, Sequence
+
+import numpy as np
+
+SOFTMAX = "softmax"
+SIGMOID = "sigmoid"
+
+CAP_DROPLESS = "dropless"
+CAP_CEIL_CF_T_OVER_N = "ceil_cf_T_over_N"          # north-star / [Compass] form
+CAP_CF_K_T_OVER_N_FLOOR = "floor_cf_k_T_over_N"    # [Practice] code form
+
+
+@dataclass
+class OracleConfig:
+    """Shape and routing options of one MoE layer (oracle-side copy)."""
+
+    n_experts: int
+    top_k: int
+    score_fn: str = SOFTMAX
+    renorm: bool = True
+    n_groups: int = 1            # 1: no group-limited pre-selection
+    topk_groups: int = 1
+    group_score_topn: int = 2
+    capacity_mode: str = CAP_DROPLESS
+    capacity_factor: float = 1.0
+
+
+# ---------------------------------------------------------------------------
+# 1. Router GEMM
+# ---------------------------------------------------------------------------
+def router_logits(x: np.ndarray, w_gate: np.ndarray,
+                  logit_offset: Optional[np.ndarray] = None) -> np.ndarray:
+    """z[t, e] = sum_d x[t, d] * Wg[e, d]  (+ o[e] when a per-expert offset is given).
+
+    [Practice] section "路由的数学形式": the gate is a bias-free linear layer over the
+    flattened [T, D] tokens.  [Compass] section "稀疏门控与 Top-k 路由": affinity x·W_g.
+    The optional offset o[e] is the synthetic Zipf skew of the Switch-style stress
+    workload, added to the logits (a workload input, not a router bias).
+    """
+    z = np.asarray(x, dtype=np.float64) @ np.asarray(w_gate, dtype=np.float64).T
+    if logit_offset is not None:
+        z = z + np.asarray(logit_offset, dtype=np.float64)[None, :]
+    return z
+
+
+# ---------------------------------------------------------------------------
+# 2. Affinity
+# ---------------------------------------------------------------------------
+def softmax(z: np.ndarray) -> np.ndarray:
+    """Row softmax exp(z - max) / sum exp(z - max)  ([Practice] "路由的数学形式")."""
+    m = z.max(axis=1, keepdims=True)
+    e = np.exp(z - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def sigmoid(z: np.ndarray) -> np.ndarray:
+    """Independent per-expert score 1 / (1 + exp(-z))  ([Taste] section 7)."""
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def logsumexp(z: np.ndarray) -> np.ndarray:
+    """log sum_e exp(z[t, e]) per token, used by the router z-loss."""
+    m = z.max(axis=1)
+    return m + np.log(np.exp(z - m[:, None]).sum(axis=1))
+
+
+def affinity(z: np.ndarray, score_fn: str) -> np.ndarray:
+    if score_fn == SOFTMAX:
+        return softmax(z)
+    if score_fn == SIGMOID:
+        return sigmoid(z)
+    raise ValueError(score_fn)
+
+
+# ---------------------------------------------------------------------------
+# 3. Selection score with the choice-only bias
+# ---------------------------------------------------------------------------
+def selection_scores(s: np.ndarray, bias: Optional[np.ndarray]) -> np.ndarray:
+    """q = s + b: the bias is added to the affinity for choosing only.
+
+    [Compass] section "负载均衡：从 aux loss 到 aux-loss-free": Top-k({s_i + b_i}), with
+    the gate weights still proportional to the raw s_i.  [Practice] class
+    BiasBalancedRouter adds the bias to the softmax probabilities, not the logits.
+    """
+    if bias is None:
+        return s.copy()
+    return s + np.asarray(bias, dtype=np.float64)[None, :]
+
+
+# ---------------------------------------------------------------------------
+# 4. Group-limited pre-selection (reading: the pages give no formula)
+# ---------------------------------------------------------------------------
+def group_scores(q: np.ndarray, n_groups: int, topn: int) -> np.ndarray:
+    """Score of each contiguous expert group = sum of its `topn` largest q.
+
+    [History] part 四 and [Practice] "负载均衡损失" name node-limited routing without
+    a formula; reading: experts split into n_groups contiguous groups of N/n_groups,
+    scored by the sum of their top-`topn` selection scores (topn = 1 gives max).
+    """
+    T, N = q.shape
+    gs = N // n_groups
+    qg = q.reshape(T, n_groups, gs)
+    top = -np.sort(-qg, axis=2)[:, :, :topn]
+    return top.sum(axis=2)
+
+
+def eligible_mask(q: np.ndarray, cfg: OracleConfig) -> tuple[np.ndarray, np.ndarray]:
+    """Experts a token may pick after keeping its `topk_groups` best groups.
+
+    Returns (mask [T, N] bool, group_margin [T]).  Group ties: lower group index wins.
+    group_margin is the score of the last kept group minus the best dropped group
+    (+inf when no group is dropped).
+    """
+    T, N = q.shape
+    if cfg.n_groups <= 1:
+        return np.ones((T, N), dtype=bool), np.full(T, np.inf)
+    gsc = group_scores(q, cfg.n_groups, cfg.group_score_topn)
+    order = np.argsort(-gsc, axis=1, kind="stable")          # descending, lower index first on ties
+    kept = order[:, : cfg.topk_groups]
+    gs = N // cfg.n_groups
+    mask = np.zeros((T, N), dtype=bool)
+    for t in range(T):
+        for g in kept[t]:
+            mask[t, g * gs:(g + 1) * gs] = True
+    if cfg.topk_groups < cfg.n_groups:
+        last = np.take_along_axis(gsc, order[:, cfg.topk_groups - 1:cfg.topk_groups], axis=1)[:, 0]
+        first_out = np.take_along_axis(gsc, order[:, cfg.topk_groups:cfg.topk_groups + 1], axis=1)[:, 0]
+        gmargin = last - first_out
+    else:
+        gmargin = np.full(T, np.inf)
+    return mask, gmargin
+
+
+# ---------------------------------------------------------------------------
+# 5. Top-k
+# ---------------------------------------------------------------------------
+def select_topk(q: np.ndarray, k: int, mask: Optional[np.ndarray] = None
+                ) -> tuple[np.ndarray, np.ndarray]:
+    """The k eligible experts with the largest q, stored in descending q.
+
+    [Practice] "路由的数学形式" (probs.topk) and [Compass] "稀疏门控与 Top-k 路由".
+    Ties (pages silent): the lower expert index wins.
+    Returns (idx [T, k] int64, margin [T]) where margin = q of the k-th pick minus
+    the best eligible expert left out (+inf when none is left).
+    """
+    qq = q.copy()
+    if mask is not None:
+        qq[~mask] = -np.inf
+    order = np.argsort(-qq, axis=1, kind="stable")
+    idx = order[:, :k]
+    kth = np.take_along_axis(qq, order[:, k - 1:k], axis=1)[:, 0]
+    if qq.shape[1] > k:
+        nxt = np.take_along_axis(qq, order[:, k:k + 1], axis=1)[:, 0]
+        margin = np.where(np.isfinite(nxt), kth - nxt, np.inf)
+    else:
+        margin = np.full(q.shape[0], np.inf)
+    return idx.astype(np.int64), margin
+
+
+# ---------------------------------------------------------------------------
+# 6. Gate weights
+# ---------------------------------------------------------------------------
+def gate_weights(s: np.ndarray, idx: np.ndarray, renorm: bool = True) -> np.ndarray:
+    """w[t, j] = s[t, idx_j] / sum_j' s[t, idx_j'] (renormalised top-k weights).
+
+    [Practice] "路由的数学形式": after top-k the k probabilities are renormalised to sum
+    to one; [Compass] "负载均衡": with a bias the weights still use the raw s_i.
+    renorm=False keeps w = s (a variant; no routed scaling factor on the pages).
+    """
+    w = np.take_along_axis(s, idx, axis=1)
+    if renorm:
+        w = w / w.sum(axis=1, keepdims=True)
+    return w
+
+
+def route(x, w_gate, cfg: OracleConfig, bias=None, logit_offset=None) -> dict:
+    """Steps 1-6: logits -> affinity -> (+bias) -> group limit -> top-k -> weights."""
+    z = router_logits(x, w_gate, logit_offset)
+    s = affinity(z, cfg.score_fn)
+    q = selection_scores(s, bias)
+    mask, gmargin = eligible_mask(q, cfg)
+    idx, emargin = select_topk(q, cfg.top_k, mask)
+    w = gate_weights(s, idx, cfg.renorm)
+    return {"logits": z, "s": s, "q": q, "idx": idx, "w": w,
+            "margin": np.minimum(emargin, gmargin), "lse": logsumexp(z)}
+
+
+# ---------------------------------------------------------------------------
+# 7. Capacity
+# ---------------------------------------------------------------------------
+def capacity(cfg: OracleConfig, T: int) -> Optional[int]:
+    """Per-expert capacity C, or None when dropless.
+
+    The pages disagree ([Practice] code: max(int(cf*k*T/N), k); [Practice] prose:
+    cf*k*T/N; [Compass] "容量因子与专家并行": cf*tokens/N).  Default reading:
+    C = ceil(cf*T/N), evaluated as ceil((cf*T)/N) in double precision.
+    """
+    if cfg.capacity_mode == CAP_DROPLESS:
+        return None
+    N, k, cf = cfg.n_experts, cfg.top_k, cfg.capacity_factor
+    if cfg.capacity_mode == CAP_CEIL_CF_T_OVER_N:
+        return int(np.ceil((cf * T) / N))
+    if cfg.capacity_mode == CAP_CF_K_T_OVER_N_FLOOR:
+        expected = k * T / float(N)
+        return max(int(expected * cf), k)
+    raise ValueError(cfg.capacity_mode)
+
+
+# ---------------------------------------------------------------------------
+# 8. Token-order drop
+# ---------------------------------------------------------------------------
+def positions(idx: np.ndarray, n_experts: int) -> np.ndarray:
+    """pos[t, j] = number of earlier tokens t' < t that also chose idx[t, j].
+
+    [Practice] "路由的数学形式", third detail after the router code: the earliest
+    occupants of an expert are kept ("rank == 0" wording), so drops are reproducible.
+    The printed one_hot/cumsum code is garbled (it scans the k axis); the prose is
+    followed.  A plain running counter over tokens in order.
+    """
+    T, k = idx.shape
+    seen = np.zeros(n_experts, dtype=np.int64)
+    pos = np.zeros((T, k), dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            pos[t, j] = seen[e]
+        for j in range(k):
+            seen[idx[t, j]] += 1
+    return pos
+
+
+# ---------------------------------------------------------------------------
+# 9. Permutation into expert-contiguous rows
+# ---------------------------------------------------------------------------
+def permutation(idx: np.ndarray, n_experts: int, C: Optional[int]) -> dict:
+    """Counts, kept counts, offsets and the slot <-> row maps.
+
+    [Practice] "专家并行与 all-to-all": assignments are grouped stably by destination
+    so one grouped GEMM covers all experts.  Rows of expert e are its kept slots in
+    token order; a dropped slot (pos >= C) gets row -1 ([Practice] "容量因子、token
+    dropping": a dropped token's FFN output is zero).
+    """
+    T, k = idx.shape
+    counts = np.bincount(idx.reshape(-1), minlength=n_experts).astype(np.int64)
+    pos = positions(idx, n_experts)
+    keep = np.ones((T, k), dtype=bool) if C is None else pos < C
+    kept = counts.copy() if C is None else np.minimum(counts, C)
+    offsets = np.zeros(n_experts + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(kept)
+    R = int(offsets[-1])
+    row_of_slot = np.full((T, k), -1, dtype=np.int64)
+    token_of_row = np.full(R, -1, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            if keep[t, j]:
+                r = offsets[idx[t, j]] + pos[t, j]
+                row_of_slot[t, j] = r
+                token_of_row[r] = t
+    dropped_slots = int(T * k - R)
+    dropped_tokens = int((~keep).all(axis=1).sum())
+    return {"counts": counts, "kept": kept, "offsets": offsets, "pos": pos, "keep": keep,
+            "row_of_slot": row_of_slot, "token_of_row": token_of_row, "R": R,
+            "dropped_slots": dropped_slots, "dropped_tokens": dropped_tokens}
+
+
+def permute_rows(x: np.ndarray, token_of_row: np.ndarray) -> np.ndarray:
+    """x_perm[r] = x[token_of_row[r]], with no pre-weighting.
+
+    [Practice]'s dispatch code multiplies rows by their gate weight before the
+    experts; for a nonlinear expert that contradicts [Compass]'s y = sum g_i E_i(x),
+    so the weight is applied in the combine instead.
+    """
+    return np.asarray(x, dtype=np.float64)[token_of_row]
+
+
+# ---------------------------------------------------------------------------
+# 10-11. Expert FFN (SwiGLU) and shared experts
+# ---------------------------------------------------------------------------
+def silu(z: np.ndarray) -> np.ndarray:
+    """silu(z) = z / (1 + exp(-z))."""
+    return z / (1.0 + np.exp(-z))
+
+
+def swiglu_ffn(x_rows: np.ndarray, w1: np.ndarray, w3: np.ndarray, w2: np.ndarray) -> np.ndarray:
+    """E(x) = W2 (silu(W1 x) * (W3 x)) for each row, no biases.
+
+    The pages describe each expert as an FFN with three matrices ([Practice]
+    "推理侧的路由稳定性", E x 3D^2) without defining SwiGLU; the plain reading is the
+    gated form above with W1 [f, d] (gate), W3 [f, d] (up), W2 [d, f] (down).
+    """
+    g = x_rows @ np.asarray(w1, dtype=np.float64).T
+    u = x_rows @ np.asarray(w3, dtype=np.float64).T
+    h = silu(g) * u
+    return h @ np.asarray(w2, dtype=np.float64).T
+
+
+def swiglu_hidden(x_rows, w1, w3) -> np.ndarray:
+    """h = silu(W1 x) * (W3 x), the intermediate of swiglu_ffn."""
+    g = x_rows @ np.asarray(w1, dtype=np.float64).T
+    u = x_rows @ np.asarray(w3, dtype=np.float64).T
+    return silu(g) * u
+
+
+# ---------------------------------------------------------------------------
+# 12. Combine
+# ---------------------------------------------------------------------------
+def combine(y_rows: np.ndarray, row_of_slot: np.ndarray, w: np.ndarray,
+            shared_out: Optional[np.ndarray], T: int, d: int) -> np.ndarray:
+    """y[t] = ys[t] + sum over kept slots j of w[t, j] * E_{idx[t,j]}(x[t]).
+
+    [Compass] "稀疏门控与 Top-k 路由": y = sum_{i in T} g_i E_i(x); [Practice] "共享专家":
+    the always-on shared output is added.  Dropped slots contribute zero.
+    """
+    y = np.zeros((T, d)) if shared_out is None else np.array(shared_out, dtype=np.float64)
+    for t in range(T):
+        for j in range(row_of_slot.shape[1]):
+            r = row_of_slot[t, j]
+            if r >= 0:
+                y[t] += w[t, j] * y_rows[r]
+    return y
+
+
+# ---------------------------------------------------------------------------
+# 13. Router statistics
+# ---------------------------------------------------------------------------
+def normalised_affinity(s: np.ndarray, score_fn: str) -> np.ndarray:
+    """s-hat: the softmax probabilities, or for sigmoid s / sum_e s (reading)."""
+    if score_fn == SOFTMAX:
+        return s
+    return s / s.sum(axis=1, keepdims=True)
+
+
+def router_stats(counts, kept, s, lse, cfg: OracleConfig, T: int,
+                 dropped_slots: int, dropped_tokens: int,
+                 alpha: float, z_coef: float, bias=None) -> dict:
+    """f_i, P_i, aux, z-loss, usage CV, dead experts, drops, bias norm.
+
+    [Compass] "负载均衡": L_aux = alpha * N * sum_i f_i P_i, equal to alpha under
+    uniform routing ([Practice] "负载均衡损失" says 1 before scaling).  f_i is the
+    share of the k*T assignments (so sum f = 1); [Practice]'s printed extra
+    N*sum P^2 term contradicts its own "equals 1 when uniform" and is not used.
+    z-loss: the pages name it ([History] part 五, [Landscape] §0) without a formula;
+    reading = ST-MoE form mean_t (logsumexp_e z)^2.  CV: population std / mean of
+    the pre-capacity counts ([Landscape] 实践要点 monitoring metrics).
+    """
+    N, k = cfg.n_experts, cfg.top_k
+    counts = np.asarray(counts, dtype=np.float64)
+    kept = np.asarray(kept, dtype=np.float64)
+    f = counts / (k * T)
+    P = normalised_affinity(s, cfg.score_fn).mean(axis=0) if T > 0 else np.zeros(N)
+    aux_raw = N * float(np.sum(f * P))
+    z = float(np.mean(lse ** 2)) if T > 0 else 0.0
+    mean_c = counts.mean()
+    cv = float(np.sqrt(np.mean((counts - mean_c) ** 2)) / mean_c) if mean_c > 0 else 0.0
+    mean_k = kept.mean()
+    cv_kept = float(np.sqrt(np.mean((kept - mean_k) ** 2)) / mean_k) if mean_k > 0 else 0.0
+    return {"f": f, "P": P, "aux_raw": aux_raw, "aux": alpha * aux_raw, "z": z,
+            "z_loss": z_coef * z, "cv": cv, "cv_kept": cv_kept,
+            "dead": int(np.sum(counts == 0)), "dropped_slots": dropped_slots,
+            "dropped_tokens": dropped_tokens,
+            "bias_norm": 0.0 if bias is None else float(np.sqrt(np.sum(np.asarray(bias, np.float64) ** 2)))}
+
+
+# ---------------------------------------------------------------------------
+# 14. Aux-loss-free bias update
+# ---------------------------------------------------------------------------
+def bias_update(bias: np.ndarray, counts: np.ndarray, rate: float = 1e-3,
+                clamp: Optional[float] = None) -> np.ndarray:
+    """b[e] += rate * sign(mean(c) - c[e]) (sign(0) = 0), optional clamp to +-clamp.
+
+    [Practice] BiasBalancedRouter.update_bias (overloaded experts pushed down,
+    underloaded up, step 1e-3); [Compass] "负载均衡" describes the same direction.
+    The batch is treated as one sequence.  The +-1e-2 clamp of [Practice] is an
+    option that is off by default.
+    """
+    c = np.asarray(counts, dtype=np.float64)
+    delta = c.mean() - c
+    b = np.asarray(bias, dtype=np.float64) + rate * np.sign(delta)
+    if clamp is not None and clamp > 0:
+        b = np.clip(b, -clamp, clamp)
+    return b
+
+
+# ---------------------------------------------------------------------------
+# Whole layer
+# ---------------------------------------------------------------------------
+ExpertWeights = Callable[[int], tuple]
+
+
+def layer_forward(x: np.ndarray, w_gate: np.ndarray, cfg: OracleConfig,
+                  expert_weights: ExpertWeights,
+                  shared_weights: Optional[tuple] = None,
+                  bias=None, logit_offset=None,
+                  alpha: float = 0.0, z_coef: float = 0.0,
+                  tokens: Optional[Sequence[int]] = None,
+                  routing: Optional[dict] = None) -> dict:
+    """The layer forward in the pages' order: route, capacity/drop, permute,
+    expert FFNs (+ shared), combine, statistics.
+
+    expert_weights(e) returns (w1 [f, d], w3 [f, d], w2 [d, f]) for expert e, so
+    large layers can widen one expert at a time.  `tokens`, when given, restricts
+    the expert compute and combine to those tokens (routing, capacity and
+    statistics still see every token).  `routing` lets a test feed a fixed
+    routing decision (idx, w) instead of recomputing it.
+    """
+    T, d = x.shape
+    r = route(x, w_gate, cfg, bias, logit_offset) if routing is None else routing
+    C = capacity(cfg, T)
+    p = permutation(r["idx"], cfg.n_experts, C)
+    want = np.arange(T) if tokens is None else np.asarray(tokens)
+    want_set = set(int(t) for t in want)
+    y = np.zeros((len(want), d))
+    if shared_weights is not None:
+        y += swiglu_ffn(np.asarray(x, np.float64)[want], *shared_weights)
+    pos_in_want = {int(t): i for i, t in enumerate(want)}
+    # gather, per expert, the rows (token, slot) that belong to wanted tokens
+    for e in range(cfg.n_experts):
+        lo, hi = p["offsets"][e], p["offsets"][e + 1]
+        rows = [rr for rr in range(lo, hi) if int(p["token_of_row"][rr]) in want_set]
+        if not rows:
+            continue
+        toks = p["token_of_row"][rows]
+        ye = swiglu_ffn(np.asarray(x, np.float64)[toks], *expert_weights(e))
+        for i, rr in enumerate(rows):
+            t = int(p["token_of_row"][rr])
+            j = int(np.nonzero(p["row_of_slot"][t] == rr)[0][0])
+            y[pos_in_want[t]] += r["w"][t, j] * ye[i]
+    out = {"y": y, "tokens": want, "routing": r, "perm": p, "capacity": C}
+    if "s" in r:
+        out["stats"] = router_stats(p["counts"], p["kept"], r["s"], r["lse"], cfg, T,
+                                    p["dropped_slots"], p["dropped_tokens"], alpha, z_coef, bias)
+    return out

@@ -1,0 +1,478 @@
+"""Pins of the fp64 oracle against what the pages and mathematics fix.
+
+Each test checks the oracle against something other than itself: a worked example
+printed on the pages (tests/golden/), a brute-force search on tiny inputs, a
+closed form, a library routine, or an invariant.  CPU only.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special as sp
+
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_rows(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([float(v) for v in line.split()])
+    return rows
+
+
+# ---------------------------------------------------------------- renormalisation
+def test_renorm_worked_example():
+    for p1, p2, w1, w2 in _golden_rows("renorm_worked_example.txt"):
+        s = np.array([[p1, p2, 1.0 - p1 - p2]])
+        w = O.gate_weights(s, np.array([[0, 1]]), renorm=True)
+        assert abs(w[0, 0] - w1) < 5e-6 and abs(w[0, 1] - w2) < 5e-6
+        assert abs(w.sum() - 1.0) < 1e-12
+
+
+def test_renorm_sums_to_one_and_top1_is_one():
+    rng = np.random.default_rng(1)
+    z = rng.normal(size=(50, 16))
+    for k in (1, 2, 4, 7):
+        r = O.route(rng.normal(size=(50, 8)), rng.normal(size=(16, 8)), O.OracleConfig(16, k))
+        assert np.allclose(r["w"].sum(axis=1), 1.0, atol=1e-12)
+        if k == 1:
+            assert np.all(r["w"] == 1.0)
+    del z
+
+
+def test_renorm_off_keeps_raw_scores():
+    s = O.softmax(np.random.default_rng(2).normal(size=(5, 6)))
+    idx, _ = O.select_topk(s, 2)
+    w = O.gate_weights(s, idx, renorm=False)
+    assert np.array_equal(w, np.take_along_axis(s, idx, 1))
+
+
+# ---------------------------------------------------------------- affinity vs library
+def test_affinity_matches_scipy():
+    z = np.random.default_rng(3).normal(scale=4.0, size=(40, 33))
+    assert np.allclose(O.softmax(z), sp.softmax(z, axis=1), rtol=1e-13, atol=1e-15)
+    assert np.allclose(O.sigmoid(z), sp.expit(z), rtol=1e-13, atol=1e-15)
+    assert np.allclose(O.logsumexp(z), sp.logsumexp(z, axis=1), rtol=1e-13)
+    assert np.allclose(O.silu(z), z * sp.expit(z), rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- top-k brute force
+def _brute_topk(q, k, allowed=None):
+    """Size-k subset with max sum, lexicographically smallest among ties."""
+    n = len(q)
+    cand = range(n) if allowed is None else sorted(allowed)
+    best, best_sum = None, -math.inf
+    for sub in itertools.combinations(cand, k):
+        ssum = sum(q[i] for i in sub)
+        if ssum > best_sum:
+            best, best_sum = sub, ssum
+    return best
+
+
+def _brute_groups(q, G, keep, topn):
+    n = len(q)
+    gs = n // G
+    gscore = []
+    for g in range(G):
+        members = q[g * gs:(g + 1) * gs]
+        gscore.append(max(sum(c) for c in itertools.combinations(members, topn)))
+    best, best_sum = None, -math.inf
+    for sub in itertools.combinations(range(G), keep):
+        ssum = sum(gscore[g] for g in sub)
+        if ssum > best_sum:
+            best, best_sum = sub, ssum
+    allowed = [e for g in best for e in range(g * gs, (g + 1) * gs)]
+    return allowed
+
+
+@pytest.mark.parametrize("n,k", [(4, 1), (6, 2), (8, 3), (12, 2), (16, 3)])
+def test_topk_bruteforce_random(n, k):
+    rng = np.random.default_rng(n * 10 + k)
+    q = rng.normal(size=(60, n))
+    idx, margin = O.select_topk(q, k)
+    for t in range(q.shape[0]):
+        assert tuple(sorted(idx[t])) == _brute_topk(list(q[t]), k)
+        vals = q[t, idx[t]]
+        assert np.all(np.diff(vals) <= 0)      # stored in descending q
+        assert margin[t] >= 0
+
+
+@pytest.mark.parametrize("n,k", [(5, 2), (8, 3), (16, 3)])
+def test_topk_bruteforce_ties(n, k):
+    rng = np.random.default_rng(7 + n)
+    q = rng.integers(0, 3, size=(80, n)).astype(np.float64)   # many exact ties
+    idx, margin = O.select_topk(q, k)
+    for t in range(q.shape[0]):
+        assert tuple(sorted(idx[t])) == _brute_topk(list(q[t]), k)
+        # among equal scores the lower index is stored first
+        for a, b in zip(idx[t][:-1], idx[t][1:]):
+            assert q[t, a] > q[t, b] or (q[t, a] == q[t, b] and a < b)
+    assert np.any(margin == 0)
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_group_limited_bruteforce(ties):
+    rng = np.random.default_rng(11 + ties)
+    N, G, keep, topn, k = 16, 4, 2, 2, 3
+    cfg = O.OracleConfig(N, k, n_groups=G, topk_groups=keep, group_score_topn=topn)
+    q = (rng.integers(0, 4, size=(80, N)).astype(np.float64) if ties
+         else rng.normal(size=(80, N)))
+    mask, gmargin = O.eligible_mask(q, cfg)
+    idx, _ = O.select_topk(q, k, mask)
+    for t in range(q.shape[0]):
+        allowed = _brute_groups(list(q[t]), G, keep, topn)
+        assert sorted(np.nonzero(mask[t])[0].tolist()) == allowed
+        assert tuple(sorted(idx[t])) == _brute_topk(list(q[t]), k, allowed)
+        assert gmargin[t] >= 0
+
+
+def test_group_limit_topn1_is_group_max():
+    rng = np.random.default_rng(5)
+    q = rng.normal(size=(30, 12))
+    gs = O.group_scores(q, 3, 1)
+    assert np.array_equal(gs, q.reshape(30, 3, 4).max(axis=2))
+
+
+def test_k_distinct_experts():
+    rng = np.random.default_rng(9)
+    cfg = O.OracleConfig(64, 6)
+    r = O.route(rng.normal(size=(200, 32)), rng.normal(size=(64, 32)), cfg)
+    for t in range(200):
+        assert len(set(r["idx"][t].tolist())) == 6
+
+
+# ---------------------------------------------------------------- P4 form == P3 form
+def test_softmax_of_topk_logits_equals_renormalised_topk_probs():
+    """[Compass]'s g = softmax(TopK(xW_g)) (non-top-k logits set to -inf) equals
+    [Practice]'s renorm(topk(softmax(xW_g)))."""
+    rng = np.random.default_rng(13)
+    x, wg = rng.normal(size=(100, 16)), rng.normal(size=(10, 16)) / 4
+    for k in (1, 2, 3, 5):
+        r = O.route(x, wg, O.OracleConfig(10, k))
+        z = x @ wg.T
+        kth = -np.sort(-z, axis=1)[:, k - 1:k]
+        masked = np.where(z >= kth, z, -np.inf)
+        g = sp.softmax(masked, axis=1)
+        w_full = np.zeros_like(z)
+        np.put_along_axis(w_full, r["idx"], r["w"], axis=1)
+        assert np.allclose(w_full, g, rtol=1e-12, atol=1e-15)
+
+
+# ---------------------------------------------------------------- bias semantics
+def test_bias_zero_is_unbiased_router():
+    rng = np.random.default_rng(17)
+    x, wg = rng.normal(size=(64, 16)), rng.normal(size=(32, 16))
+    for fn in (O.SOFTMAX, O.SIGMOID):
+        cfg = O.OracleConfig(32, 4, score_fn=fn)
+        a = O.route(x, wg, cfg)
+        b = O.route(x, wg, cfg, bias=np.zeros(32))
+        assert np.array_equal(a["idx"], b["idx"]) and np.array_equal(a["w"], b["w"])
+
+
+def test_large_bias_forces_selection():
+    rng = np.random.default_rng(19)
+    x, wg = rng.normal(size=(64, 16)), rng.normal(size=(32, 16))
+    bias = np.zeros(32)
+    bias[5] = 10.0
+    r = O.route(x, wg, O.OracleConfig(32, 4, score_fn=O.SIGMOID), bias=bias)
+    assert np.all((r["idx"] == 5).any(axis=1))
+    # weights use the raw affinity, so expert 5 does not get the (huge) biased score
+    j5 = np.nonzero(r["idx"] == 5)
+    assert np.all(r["w"][j5] < 1.0)
+
+
+def test_bias_never_changes_weights_given_the_set():
+    """Two different biases that yield the same selected set give identical weights."""
+    rng = np.random.default_rng(23)
+    x, wg = rng.normal(size=(200, 16)), rng.normal(size=(16, 16))
+    cfg = O.OracleConfig(16, 3, score_fn=O.SIGMOID)
+    b1, b2 = rng.normal(scale=0.05, size=16), rng.normal(scale=0.05, size=16)
+    r1, r2 = O.route(x, wg, cfg, bias=b1), O.route(x, wg, cfg, bias=b2)
+    same = 0
+    for t in range(200):
+        if set(r1["idx"][t]) == set(r2["idx"][t]):
+            same += 1
+            m1 = dict(zip(r1["idx"][t], r1["w"][t]))
+            m2 = dict(zip(r2["idx"][t], r2["w"][t]))
+            for e in m1:
+                assert abs(m1[e] - m2[e]) < 1e-15
+    assert same > 50
+
+
+# ---------------------------------------------------------------- capacity and drop
+def test_capacity_readings():
+    T = 256
+    assert O.capacity(O.OracleConfig(8, 2, capacity_mode=O.CAP_CEIL_CF_T_OVER_N,
+                                     capacity_factor=1.25), T) == 40
+    assert O.capacity(O.OracleConfig(8, 2, capacity_mode=O.CAP_CF_K_T_OVER_N_FLOOR,
+                                     capacity_factor=1.25), T) == 80
+    assert O.capacity(O.OracleConfig(128, 1, capacity_mode=O.CAP_CEIL_CF_T_OVER_N,
+                                     capacity_factor=1.0), 65536) == 512
+    assert O.capacity(O.OracleConfig(8, 2), T) is None
+    # floor variant never goes below k
+    assert O.capacity(O.OracleConfig(64, 6, capacity_mode=O.CAP_CF_K_T_OVER_N_FLOOR,
+                                     capacity_factor=0.01), 10) == 6
+
+
+def test_drop_all_to_one_expert():
+    idx = np.zeros((10, 1), dtype=np.int64)
+    p = O.permutation(idx, 4, 3)
+    assert p["keep"][:, 0].tolist() == [True] * 3 + [False] * 7
+    assert p["row_of_slot"][:, 0].tolist() == [0, 1, 2] + [-1] * 7
+    assert p["offsets"].tolist() == [0, 3, 3, 3, 3]
+    assert p["dropped_slots"] == 7 and p["dropped_tokens"] == 7
+
+
+def test_drop_hand_case_top2():
+    idx = np.array([[0, 1], [1, 0], [0, 2], [1, 2]])
+    p = O.permutation(idx, 3, 1)
+    assert p["keep"].tolist() == [[True, True], [False, False], [False, True], [False, False]]
+    assert p["row_of_slot"].tolist() == [[0, 1], [-1, -1], [-1, 2], [-1, -1]]
+    assert p["counts"].tolist() == [3, 3, 2] and p["kept"].tolist() == [1, 1, 1]
+    assert p["dropped_slots"] == 5 and p["dropped_tokens"] == 2
+    assert p["token_of_row"].tolist() == [0, 0, 2]
+
+
+def test_positions_match_definition():
+    rng = np.random.default_rng(29)
+    N, k, T = 6, 2, 40
+    idx = np.stack([rng.choice(N, k, replace=False) for _ in range(T)])
+    pos = O.positions(idx, N)
+    for t in range(T):
+        for j in range(k):
+            e = idx[t, j]
+            assert pos[t, j] == sum(1 for tp in range(t) if e in set(idx[tp].tolist()))
+
+
+def test_drop_conservation_and_reproducible():
+    rng = np.random.default_rng(31)
+    N, k, T = 8, 2, 256
+    idx = np.stack([rng.choice(N, k, replace=False, p=np.arange(1, N + 1) / 36) for _ in range(T)])
+    for C in (1, 7, 40, 64, 1000):
+        p = O.permutation(idx, N, C)
+        assert p["kept"].sum() + p["dropped_slots"] == T * k
+        assert np.array_equal(p["kept"], np.minimum(p["counts"], C))
+        q = O.permutation(idx.copy(), N, C)
+        assert np.array_equal(p["keep"], q["keep"]) and np.array_equal(p["row_of_slot"], q["row_of_slot"])
+
+
+def test_permutation_invariants():
+    rng = np.random.default_rng(37)
+    N, k, T = 16, 3, 300
+    idx = np.stack([rng.choice(N, k, replace=False) for _ in range(T)])
+    for C in (None, 20):
+        p = O.permutation(idx, N, C)
+        off, tor, ros = p["offsets"], p["token_of_row"], p["row_of_slot"]
+        assert off[0] == 0 and off[-1] == p["R"] and np.all(np.diff(off) >= 0)
+        # bijection kept slots <-> rows
+        rows = ros[ros >= 0]
+        assert sorted(rows.tolist()) == list(range(p["R"]))
+        for t in range(T):
+            for j in range(k):
+                if ros[t, j] >= 0:
+                    r = ros[t, j]
+                    assert tor[r] == t and off[idx[t, j]] <= r < off[idx[t, j] + 1]
+        # rows of each expert in ascending token order (stable grouping)
+        for e in range(N):
+            seg = tor[off[e]:off[e + 1]]
+            assert np.all(np.diff(seg) > 0)
+
+
+# ---------------------------------------------------------------- FFN
+def test_silu_special_values():
+    assert O.silu(np.array([0.0]))[0] == 0.0
+    assert abs(O.silu(np.array([40.0]))[0] - 40.0) < 1e-12
+    assert abs(O.silu(np.array([-40.0]))[0]) < 1e-15
+
+
+def _triple_loop_swiglu(x, w1, w3, w2):
+    T, d = len(x), len(x[0])
+    f = len(w1)
+    out = []
+    for t in range(T):
+        h = []
+        for i in range(f):
+            g = sum(w1[i][c] * x[t][c] for c in range(d))
+            u = sum(w3[i][c] * x[t][c] for c in range(d))
+            h.append(g / (1.0 + math.exp(-g)) * u)
+        out.append([sum(w2[o][i] * h[i] for i in range(f)) for o in range(d)])
+    return np.array(out)
+
+
+def test_single_expert_layer_is_dense_swiglu():
+    """N=1, k=1, dropless: the MoE layer equals the dense SwiGLU FFN."""
+    rng = np.random.default_rng(41)
+    T, d, f = 5, 4, 6
+    x = rng.normal(size=(T, d))
+    w1, w3, w2 = rng.normal(size=(f, d)), rng.normal(size=(f, d)), rng.normal(size=(d, f))
+    out = O.layer_forward(x, rng.normal(size=(1, d)), O.OracleConfig(1, 1),
+                          lambda e: (w1, w3, w2))
+    ref = _triple_loop_swiglu(x.tolist(), w1.tolist(), w3.tolist(), w2.tolist())
+    assert np.allclose(out["y"], ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(out["y"], O.swiglu_ffn(x, w1, w3, w2), rtol=1e-13, atol=1e-13)
+
+
+def test_ffn_linear_in_w2():
+    rng = np.random.default_rng(43)
+    x = rng.normal(size=(7, 8))
+    w1, w3, w2 = rng.normal(size=(5, 8)), rng.normal(size=(5, 8)), rng.normal(size=(8, 5))
+    a = O.swiglu_ffn(x, w1, w3, w2)
+    assert np.allclose(O.swiglu_ffn(x, w1, w3, 2.5 * w2), 2.5 * a, rtol=1e-13)
+    assert np.allclose(O.swiglu_ffn(x, w1, w3, w2 + w2[::-1]),
+                       a + O.swiglu_ffn(x, w1, w3, w2[::-1]), rtol=1e-12, atol=1e-12)
+
+
+def test_concatenated_shared_experts_equal_their_sum():
+    rng = np.random.default_rng(47)
+    x = rng.normal(size=(6, 8))
+    a = [rng.normal(size=(5, 8)), rng.normal(size=(5, 8)), rng.normal(size=(8, 5))]
+    b = [rng.normal(size=(5, 8)), rng.normal(size=(5, 8)), rng.normal(size=(8, 5))]
+    cat = (np.concatenate([a[0], b[0]]), np.concatenate([a[1], b[1]]), np.concatenate([a[2], b[2]], axis=1))
+    assert np.allclose(O.swiglu_ffn(x, *cat), O.swiglu_ffn(x, *a) + O.swiglu_ffn(x, *b), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- combine
+def test_identical_experts_give_the_expert_output():
+    rng = np.random.default_rng(53)
+    T, d, f, N = 20, 6, 5, 8
+    x = rng.normal(size=(T, d))
+    w = (rng.normal(size=(f, d)), rng.normal(size=(f, d)), rng.normal(size=(d, f)))
+    ws = (rng.normal(size=(3, d)), rng.normal(size=(3, d)), rng.normal(size=(d, 3)))
+    for k in (1, 2, 3):
+        out = O.layer_forward(x, rng.normal(size=(N, d)), O.OracleConfig(N, k), lambda e: w, ws)
+        assert np.allclose(out["y"], O.swiglu_ffn(x, *w) + O.swiglu_ffn(x, *ws), rtol=1e-12, atol=1e-12)
+
+
+def test_dropped_token_without_shared_is_zero():
+    rng = np.random.default_rng(59)
+    T, d, N = 12, 4, 2
+    x = rng.normal(size=(T, d))
+    wg = np.zeros((N, d))
+    wg[0, 0] = 1.0
+    x[:, 0] = 5.0                   # everyone prefers expert 0
+    cfg = O.OracleConfig(N, 1, capacity_mode=O.CAP_CEIL_CF_T_OVER_N, capacity_factor=0.5)
+    w = (rng.normal(size=(3, d)), rng.normal(size=(3, d)), rng.normal(size=(d, 3)))
+    out = O.layer_forward(x, wg, cfg, lambda e: w)
+    C = out["capacity"]
+    assert C == 3
+    assert np.all(out["y"][C:] == 0.0) and np.all(np.abs(out["y"][:C]).sum(axis=1) > 0)
+
+
+def test_token_subset_matches_full_forward():
+    rng = np.random.default_rng(61)
+    T, d, f, N = 30, 8, 6, 6
+    x = rng.normal(size=(T, d))
+    W = [(rng.normal(size=(f, d)), rng.normal(size=(f, d)), rng.normal(size=(d, f))) for _ in range(N)]
+    cfg = O.OracleConfig(N, 2, capacity_mode=O.CAP_CEIL_CF_T_OVER_N, capacity_factor=1.0)
+    wg = rng.normal(size=(N, d))
+    full = O.layer_forward(x, wg, cfg, lambda e: W[e])
+    sub = [3, 17, 29]
+    part = O.layer_forward(x, wg, cfg, lambda e: W[e], tokens=sub)
+    assert np.allclose(part["y"], full["y"][sub], rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------- statistics
+def test_aux_uniform_stats_level():
+    for N, alpha, unscaled, expected in _golden_rows("aux_uniform.txt"):
+        N = int(N)
+        k, T = 2, 4 * N
+        counts = np.full(N, k * T // N)
+        s = np.full((T, N), 1.0 / N)
+        st = O.router_stats(counts, counts, s, np.zeros(T), O.OracleConfig(N, k), T, 0, 0, alpha, 0.0)
+        assert abs(st["aux_raw"] - unscaled) < 1e-12 and abs(st["aux"] - expected) < 1e-14
+
+
+def test_aux_uniform_end_to_end():
+    """k=1, T=N, x[t] = L e_t, Wg = [I | 0]: every expert gets one token and P_e = 1/N."""
+    N, d, L, alpha = 8, 12, 3.0, 0.01
+    x = np.zeros((N, d))
+    x[np.arange(N), np.arange(N)] = L
+    wg = np.zeros((N, d))
+    wg[:, :N] = np.eye(N)
+    cfg = O.OracleConfig(N, 1)
+    w = (np.ones((2, d)), np.ones((2, d)), np.ones((d, 2)))
+    out = O.layer_forward(x, wg, cfg, lambda e: w, alpha=alpha)
+    st = out["stats"]
+    assert np.array_equal(out["routing"]["idx"][:, 0], np.arange(N))
+    assert np.allclose(st["P"], 1.0 / N, rtol=1e-14) and np.allclose(st["f"], 1.0 / N)
+    assert abs(st["aux"] - alpha) < 1e-15
+
+
+def test_zloss_zero_logits():
+    N, T = 16, 10
+    st = O.router_stats(np.full(N, 1), np.full(N, 1), np.full((T, N), 1.0 / N),
+                        O.logsumexp(np.zeros((T, N))), O.OracleConfig(N, 1), T, 0, 0, 0.0, 1e-3)
+    assert abs(st["z"] - math.log(N) ** 2) < 1e-13
+    assert abs(st["z_loss"] - 1e-3 * math.log(N) ** 2) < 1e-16
+
+
+def test_cv_and_dead_constructed():
+    N, T = 8, 8
+    s = np.full((T, N), 1.0 / N)
+    eq = O.router_stats(np.full(N, 4), np.full(N, 4), s, np.zeros(T), O.OracleConfig(N, 4), T, 0, 0, 0, 0)
+    assert eq["cv"] == 0.0 and eq["dead"] == 0
+    one = np.zeros(N)
+    one[3] = 32
+    hot = O.router_stats(one, one, s, np.zeros(T), O.OracleConfig(N, 4), T, 0, 0, 0, 0)
+    assert abs(hot["cv"] - math.sqrt(N - 1)) < 1e-12 and hot["dead"] == N - 1
+
+
+def test_sum_f_is_one():
+    rng = np.random.default_rng(67)
+    cfg = O.OracleConfig(16, 4)
+    x, wg = rng.normal(size=(100, 8)), rng.normal(size=(16, 8))
+    out = O.layer_forward(x, wg, cfg, lambda e: (np.zeros((2, 8)), np.zeros((2, 8)), np.zeros((8, 2))))
+    assert abs(out["stats"]["f"].sum() - 1.0) < 1e-12
+    assert abs(out["stats"]["P"].sum() - 1.0) < 1e-12
+
+
+# ---------------------------------------------------------------- bias update
+def test_bias_update_equal_counts_no_change():
+    b = np.array([0.1, -0.2, 0.0, 0.3])
+    assert np.array_equal(O.bias_update(b, np.array([5, 5, 5, 5])), b)
+
+
+def test_bias_update_single_overloaded():
+    N, g = 8, 1e-3
+    c = np.full(N, 10)
+    c[2] = 50
+    b = O.bias_update(np.zeros(N), c, rate=g)
+    exp = np.full(N, g)
+    exp[2] = -g
+    assert np.allclose(b, exp, rtol=0, atol=1e-18)
+
+
+def test_bias_update_clamp():
+    b = O.bias_update(np.array([0.0099, -0.0099]), np.array([0, 10]), rate=1e-3, clamp=1e-2)
+    assert np.allclose(b, [0.01, -0.01])
+
+
+# ---------------------------------------------------------------- cross-batch consistency
+def test_cross_batch_consistency_dropless():
+    """Dropless routing of T tokens equals routing them in chunks ([Practice] checklist)."""
+    rng = np.random.default_rng(71)
+    x, wg = rng.normal(size=(64, 16)), rng.normal(size=(32, 16))
+    bias = rng.normal(scale=0.1, size=32)
+    cfg = O.OracleConfig(32, 4, score_fn=O.SIGMOID, n_groups=4, topk_groups=2)
+    full = O.route(x, wg, cfg, bias=bias)
+    parts = [O.route(x[i:i + 16], wg, cfg, bias=bias) for i in range(0, 64, 16)]
+    assert np.array_equal(full["idx"], np.concatenate([p["idx"] for p in parts]))
+    assert np.allclose(full["w"], np.concatenate([p["w"] for p in parts]), rtol=1e-14)
+
+
+def test_flattening_consistency():
+    """[B, S, D] inputs flattened to [T, D] route identically ([Practice] checklist)."""
+    rng = np.random.default_rng(73)
+    x3 = rng.normal(size=(4, 8, 16))
+    wg = rng.normal(size=(8, 16))
+    cfg = O.OracleConfig(8, 2)
+    flat = O.route(x3.reshape(-1, 16), wg, cfg)
+    per_b = [O.route(x3[b], wg, cfg) for b in range(4)]
+    assert np.array_equal(flat["idx"], np.concatenate([p["idx"] for p in per_b]))
