@@ -1,0 +1,243 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) sparse MoE FFN layer forward.
+ *
+ * The layer, in order (page tags as in the library's design notes):
+ *   route      router GEMM -> softmax/sigmoid affinity -> choice-only bias ->
+ *              group-limited pre-selection -> top-k -> renormalised gate weights
+ *   permute    per-expert counts -> capacity / token-order drop -> offsets ->
+ *              expert-contiguous rows (stable in token order) -> row gather
+ *   grouped_ffn SwiGLU expert FFN over variable-size row groups (also the
+ *              always-on shared experts, as one group over all tokens)
+ *   combine    gate-weighted sum of each token's expert rows (+ shared output)
+ *   router_stats / bias_update  f_i, P_i, aux, z-loss, CV, dead, drops; the
+ *              aux-loss-free sign update of the selection bias.
+ *
+ * Conventions shared by every entry point
+ *   - Return value: a moe_status_t (0 = MOE_OK).  Arguments are checked on the
+ *     host before anything is enqueued; an invalid call enqueues nothing.
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless the
+ *     comment says "host".  The library never allocates or frees device memory
+ *     and keeps no pointer after a call returns.
+ *   - All work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream).  No call synchronises the host.
+ *   - Device pointers must be 16-byte aligned; tensors are dense row-major.
+ *   - Kernel-side failures that the host cannot see (a bounded wait that ran
+ *     out) are recorded in a device status word; read it with
+ *     moe_device_status() after synchronising.
+ *   - Integer outputs are deterministic: the same inputs give the same bytes on
+ *     every run.  Floating-point outputs are deterministic too (no atomics on
+ *     any floating-point accumulation).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* bad size, null pointer, misalignment, k > N ... */
+  MOE_ERR_UNSUPPORTED = 2,        /* valid request outside what the kernels implement */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+  MOE_ERR_CUDA = 4,               /* a CUDA runtime call failed (launch, tensor map) */
+  MOE_ERR_DEVICE_TIMEOUT = 5      /* a device-side bounded wait gave up */
+} moe_status_t;
+
+enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
+enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 };
+enum {
+  MOE_CAP_DROPLESS = 0,           /* no capacity limit */
+  MOE_CAP_CEIL_CF_T_OVER_N = 1,   /* C = ceil((cf*T)/N)  (default capacity reading) */
+  MOE_CAP_CF_K_T_OVER_N_FLOOR = 2 /* C = max(floor(cf*k*T/N), k)  (the Practice page's code) */
+};
+
+/* Shape and routing options of one MoE layer.  Plain data, host memory. */
+typedef struct moe_config {
+  int64_t T;                 /* tokens (batch x sequence, flattened), >= 0          */
+  int32_t d_model;           /* d, multiple of 8                                    */
+  int32_t n_experts;         /* N routed experts, 1..512                            */
+  int32_t top_k;             /* k, 1..min(N, 16)                                    */
+  int32_t d_ff;              /* f, routed expert hidden size, multiple of 8         */
+  int32_t score_fn;          /* MOE_SCORE_*                                         */
+  int32_t renorm;            /* 1: w = s_sel / sum s_sel; 0: w = s_sel              */
+  int32_t n_groups;          /* <= 1: no group limit; else divides N, <= 32         */
+  int32_t topk_groups;       /* groups kept per token (group limit on)              */
+  int32_t group_score_topn;  /* group score = sum of its topn best scores, >= 1     */
+  int32_t capacity_mode;     /* MOE_CAP_*                                           */
+  int32_t x_dtype;           /* MOE_DTYPE_*: x, expert weights, h, y all this type  */
+  double capacity_factor;    /* cf (> 0) for the capacity modes                     */
+} moe_config_t;
+
+/* Router statistics, written by moe_router_stats (device memory). */
+typedef struct moe_stats {
+  float aux;                 /* alpha * N * sum_e f_e P_e                            */
+  float aux_raw;             /* N * sum_e f_e P_e (1 under uniform routing)          */
+  float z;                   /* mean_t (logsumexp_e z[t,e])^2                        */
+  float z_loss;              /* z_coef * z                                           */
+  float cv;                  /* population std / mean of pre-capacity counts        */
+  float cv_kept;             /* same over kept (post-capacity) counts               */
+  float bias_norm;           /* ||b||_2 (0 when no bias)                             */
+  int32_t dead;              /* experts with zero selections                        */
+  int32_t dropped_slots;     /* k*T - R                                             */
+  int32_t dropped_tokens;    /* tokens whose k slots were all dropped               */
+  int32_t R;                 /* kept rows                                           */
+  int32_t reserved[5];
+} moe_stats_t;
+
+/* ---------------------------------------------------------------------------
+ * Sizing queries (host only; no device work).
+ * ------------------------------------------------------------------------- */
+
+/* Per-expert capacity C for cfg (host out).  Dropless gives C = INT64_MAX.
+ * Capacity: "容量因子与专家并行（工程视角）" on the llm-compass MoE page
+ * (capacity = cf * tokens / N) and "容量因子、token dropping 与一笔算不清的隐形税" on the
+ * Practice page (C = cf * k * T / N; its code floors and keeps at least k). */
+int moe_capacity(const moe_config_t* cfg, int64_t* capacity);
+
+/* Rows of the p_partial buffer written by moe_route (host out). */
+int moe_route_partials(const moe_config_t* cfg, int32_t* nblk);
+
+/* Bytes of scratch `ws` needed by moe_permute for cfg (host out). */
+int moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * moe_route -- fused router GEMM + affinity + bias + group limit + top-k + renorm.
+ *
+ * Defines: "路由的数学形式：softmax、top-k 与那些必须做的小动作" (Practice page:
+ * logits -> softmax -> top-k -> renormalise; the router has no bias term), the
+ * llm-compass page's "稀疏门控与 Top-k 路由" (g = softmax(TopK(xW_g))) and its
+ * "负载均衡：从 aux loss 到 aux-loss-free" (selection on s_i + b_i, weights from s_i).
+ *
+ *   x            [T, d]   cfg->x_dtype (fp32 or bf16)
+ *   w_gate       [N, d]   fp32 router weight (kept in fp32; never quantised)
+ *   logit_offset [N] fp32 or NULL: added to every token's logits
+ *   bias         [N] fp32 or NULL: added to the affinity for selection only
+ *   topk_idx     [T, k] int32 out: experts in descending selection score;
+ *                equal scores -> lower expert index first
+ *   topk_w       [T, k] fp32 out: gate weights (raw affinity, renormalised)
+ *   lse          [T] fp32 out: logsumexp of the logits (z-loss input)
+ *   p_partial    [nblk, N] fp32 out: per-block sums over tokens of the
+ *                normalised affinity (softmax probs, or s / sum s for sigmoid);
+ *                nblk from moe_route_partials
+ *   margin       [T] fp32 out or NULL: selection score of the k-th pick minus the
+ *                best eligible expert left out, min'ed with the last-kept minus
+ *                best-dropped group score (+inf when nothing is left out)
+ * The router GEMM accumulates in fp32.  T = 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate,
+              const float* logit_offset, const float* bias,
+              int32_t* topk_idx, float* topk_w, float* lse, float* p_partial,
+              float* margin, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_permute -- counts, capacity drop in token order, offsets, row maps, gather.
+ *
+ * Defines: Practice page "容量因子、token dropping" (per-expert hard cap; the
+ * earliest occupants are kept, reproducibly) and "专家并行与 all-to-all" (stable
+ * grouping by destination so one grouped GEMM covers all experts); dropped slots
+ * contribute zero.
+ *
+ *   x            [T, d] x_dtype
+ *   topk_idx     [T, k] int32, each row k distinct experts in [0, N)
+ *   counts       [N] int32 out: selections per expert before capacity (c_e)
+ *   offsets      [N+1] int32 out: exclusive scan of kept_e = min(c_e, C)
+ *   row_of_slot  [T, k] int32 out: row of slot (t, j) in x_perm, -1 if dropped
+ *   token_of_row [T*k] int32 out: token of each row (entries >= R untouched)
+ *   x_perm       [T*k, d] x_dtype out: x_perm[row] = x[token_of_row[row]]
+ *                (rows >= R untouched); rows of expert e are its kept slots in
+ *                ascending token order
+ *   n_dropped    [2] int32 out: {dropped slots, tokens with all k slots dropped}
+ *   ws           scratch of at least moe_workspace_size() bytes (contents on
+ *                entry ignored; clobbered)
+ * ------------------------------------------------------------------------- */
+int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
+                int32_t* token_of_row, void* x_perm, int32_t* n_dropped,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_grouped_ffn -- SwiGLU FFN over G variable-size row groups in one pass.
+ *
+ * Defines: "专家并行与 all-to-all" on the Practice page (expert-contiguous rows let
+ * one grouped GEMM compute every expert) and the llm-compass "MoE 层结构" (each
+ * expert is an FFN).  The pages name three matrices per expert without spelling
+ * SwiGLU out; the form used is y = W2 (silu(W1 x) * (W3 x)), silu(z) = z/(1+e^-z).
+ *
+ *   x_rows   [rows_cap, d] x_dtype: rows offsets[g] .. offsets[g+1]-1 belong to
+ *            group g; rows_cap >= offsets[G]
+ *   offsets  [G+1] int32 (device), non-decreasing, offsets[0] = 0
+ *   w1, w3   [G, f, d] x_dtype (gate and up projections)
+ *   w2       [G, d, f] x_dtype (down projection)
+ *   h_scratch[rows_cap, f] x_dtype: the SwiGLU hidden rows (written, then read)
+ *   y_rows   [rows_cap, d] x_dtype out (rows >= offsets[G] untouched)
+ * bf16: tcgen05 tensor cores, fp32 accumulation, h rounded to bf16.
+ * fp32: fp32 FMA throughout.  Shared experts: G = 1, offsets = {0, T},
+ * x_rows = x, f = n_shared * d_ff_shared with the experts' matrices concatenated
+ * along f.
+ * ------------------------------------------------------------------------- */
+int moe_grouped_ffn(const moe_config_t* cfg, const void* x_rows, int64_t rows_cap,
+                    const int32_t* offsets, int32_t G,
+                    const void* w1, const void* w3, const void* w2, int32_t f,
+                    void* h_scratch, void* y_rows, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine -- y[t] = shared[t] + sum_{j: row >= 0} w[t,j] * y_perm[row(t,j)].
+ *
+ * Defines: llm-compass "稀疏门控与 Top-k 路由" (y = sum_i g_i E_i(x)) and the Practice
+ * page's "共享专家" (the always-on output is added).  Slots in ascending j,
+ * fp32 accumulation, no atomics.
+ *   y_perm      [R, d] x_dtype; row_of_slot [T, k]; topk_w [T, k] fp32
+ *   shared_out  [T, d] x_dtype or NULL; y [T, d] x_dtype out (may alias shared_out)
+ * ------------------------------------------------------------------------- */
+int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of_slot,
+                const float* topk_w, const void* shared_out, void* y, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_router_stats -- router statistics in fixed reduction order.
+ *
+ * Defines: llm-compass "负载均衡" (L_aux = alpha N sum f_i P_i), the Practice page's
+ * "负载均衡损失" (equals 1 unscaled under uniform routing) and "MoE 的可观测性"
+ * metrics (drop ratio, per-expert load); the landscape page's monitoring list
+ * (token drop, usage CV, dead experts, bias norm).  z-loss has no formula on the
+ * pages; mean_t (logsumexp_e z)^2 is used.
+ *   counts [N], offsets [N+1], p_partial [nblk, N], lse [T], n_dropped [2],
+ *   bias [N] or NULL  (all from the calls above)
+ *   stats  moe_stats_t out; f_out [N], p_out [N] fp32 out (either may be NULL)
+ * ------------------------------------------------------------------------- */
+int moe_router_stats(const moe_config_t* cfg, const int32_t* counts, const int32_t* offsets,
+                     const float* p_partial, const float* lse, const int32_t* n_dropped,
+                     const float* bias, float alpha, float z_coef,
+                     moe_stats_t* stats, float* f_out, float* p_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_bias_update -- b[e] += rate * sign(mean(c) - c[e]), optional clamp.
+ *
+ * Defines: the Practice page's BiasBalancedRouter.update_bias (overloaded experts
+ * down, underloaded up, step 1e-3, clamp +-1e-2) and llm-compass "负载均衡".
+ * The sign is taken exactly in integers (sum(c) - N c[e]); sign(0) = 0.
+ *   counts [N] int32; bias [N] fp32 in/out; clamp <= 0 disables clamping.
+ * ------------------------------------------------------------------------- */
+int moe_bias_update(const moe_config_t* cfg, const int32_t* counts, float* bias,
+                    float rate, float clamp, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics.
+ * ------------------------------------------------------------------------- */
+
+/* Reads (and, if reset != 0, clears) the device status word of the current
+ * device into *status (host out): MOE_OK or MOE_ERR_DEVICE_TIMEOUT.  Synchronises
+ * the current device. */
+int moe_device_status(int32_t* status, int32_t reset);
+
+/* Static string for a status code. */
+const char* moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

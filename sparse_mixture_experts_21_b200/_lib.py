@@ -1,0 +1,182 @@
+"""ctypes binding of the C ABI in include/moe_b200.h (argument marshalling only).
+
+Every function here forwards torch tensors' device pointers and the current CUDA
+stream to the library; all computation happens in the library's kernels.  There
+is no fallback: if the shared library is missing, load() raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_double, c_float, c_int, c_int32, c_int64, c_size_t, c_void_p
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_NAME = "libmoe_b200.so"
+LIB_PATH = os.path.join(_HERE, LIB_NAME)
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE_TOO_SMALL, MOE_ERR_CUDA, \
+    MOE_ERR_DEVICE_TIMEOUT = range(6)
+SCORE_SOFTMAX, SCORE_SIGMOID = 0, 1
+DTYPE_F32, DTYPE_BF16 = 0, 1
+CAP_DROPLESS, CAP_CEIL_CF_T_OVER_N, CAP_CF_K_T_OVER_N_FLOOR = 0, 1, 2
+
+EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_route", "moe_permute",
+            "moe_grouped_ffn", "moe_combine", "moe_router_stats", "moe_bias_update",
+            "moe_device_status", "moe_status_string")
+
+
+class MoeConfig(ctypes.Structure):
+    """Mirror of moe_config_t."""
+    _fields_ = [("T", c_int64), ("d_model", c_int32), ("n_experts", c_int32), ("top_k", c_int32),
+                ("d_ff", c_int32), ("score_fn", c_int32), ("renorm", c_int32), ("n_groups", c_int32),
+                ("topk_groups", c_int32), ("group_score_topn", c_int32), ("capacity_mode", c_int32),
+                ("x_dtype", c_int32), ("capacity_factor", c_double)]
+
+
+class MoeStats(ctypes.Structure):
+    """Mirror of moe_stats_t."""
+    _fields_ = [("aux", c_float), ("aux_raw", c_float), ("z", c_float), ("z_loss", c_float),
+                ("cv", c_float), ("cv_kept", c_float), ("bias_norm", c_float), ("dead", c_int32),
+                ("dropped_slots", c_int32), ("dropped_tokens", c_int32), ("R", c_int32),
+                ("reserved", c_int32 * 5)]
+
+
+STATS_BYTES = ctypes.sizeof(MoeStats)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn} failed: status {status} ({text})")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load the shared library (once).  Raises if it is absent."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise FileNotFoundError(
+            f"{p} not found: build it with `python -m sparse_mixture_experts_21_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i32p = c_void_p, POINTER(c_int32)
+    cfgp = POINTER(MoeConfig)
+    sig = {
+        "moe_capacity": [cfgp, POINTER(c_int64)],
+        "moe_route_partials": [cfgp, i32p],
+        "moe_workspace_size": [cfgp, POINTER(c_size_t)],
+        "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "moe_permute": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
+        "moe_grouped_ffn": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp],
+        "moe_combine": [cfgp, vp, vp, vp, vp, vp, vp],
+        "moe_router_stats": [cfgp, vp, vp, vp, vp, vp, vp, c_float, c_float, vp, vp, vp, vp],
+        "moe_bias_update": [cfgp, vp, vp, c_float, c_float, vp],
+        "moe_device_status": [i32p, c_int32],
+        "moe_status_string": [c_int],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = c_char_p if name == "moe_status_string" else c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+# ----------------------------------------------------------------------------- helpers
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the MoE library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check(name: str, status: int) -> None:
+    if status != MOE_OK:
+        raise MoeError(name, status, load().moe_status_string(status).decode())
+
+
+def capacity(cfg: MoeConfig) -> int:
+    out = c_int64()
+    _check("moe_capacity", load().moe_capacity(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def route_partials(cfg: MoeConfig) -> int:
+    out = c_int32()
+    _check("moe_route_partials", load().moe_route_partials(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def workspace_size(cfg: MoeConfig) -> int:
+    out = c_size_t()
+    _check("moe_workspace_size", load().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+# ----------------------------------------------------------------------------- entry points
+def moe_route(cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_partial, margin=None,
+              stream=None):
+    _check("moe_route", load().moe_route(
+        ctypes.byref(cfg), _ptr(x), _ptr(w_gate), _ptr(logit_offset), _ptr(bias), _ptr(topk_idx),
+        _ptr(topk_w), _ptr(lse), _ptr(p_partial), _ptr(margin), _stream(stream)))
+
+
+def moe_permute(cfg, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, n_dropped,
+                ws, stream=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("moe_permute", load().moe_permute(
+        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(row_of_slot),
+        _ptr(token_of_row), _ptr(x_perm), _ptr(n_dropped), _ptr(ws), nbytes, _stream(stream)))
+
+
+def moe_grouped_ffn(cfg, x_rows, rows_cap, offsets, G, w1, w3, w2, f, h_scratch, y_rows, stream=None):
+    _check("moe_grouped_ffn", load().moe_grouped_ffn(
+        ctypes.byref(cfg), _ptr(x_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1), _ptr(w3),
+        _ptr(w2), int(f), _ptr(h_scratch), _ptr(y_rows), _stream(stream)))
+
+
+def moe_combine(cfg, y_perm, row_of_slot, topk_w, shared_out, y, stream=None):
+    _check("moe_combine", load().moe_combine(
+        ctypes.byref(cfg), _ptr(y_perm), _ptr(row_of_slot), _ptr(topk_w), _ptr(shared_out), _ptr(y),
+        _stream(stream)))
+
+
+def moe_router_stats(cfg, counts, offsets, p_partial, lse, n_dropped, bias, alpha, z_coef, stats,
+                     f_out=None, p_out=None, stream=None):
+    _check("moe_router_stats", load().moe_router_stats(
+        ctypes.byref(cfg), _ptr(counts), _ptr(offsets), _ptr(p_partial), _ptr(lse), _ptr(n_dropped),
+        _ptr(bias), float(alpha), float(z_coef), _ptr(stats), _ptr(f_out), _ptr(p_out),
+        _stream(stream)))
+
+
+def moe_bias_update(cfg, counts, bias, rate, clamp=0.0, stream=None):
+    _check("moe_bias_update", load().moe_bias_update(
+        ctypes.byref(cfg), _ptr(counts), _ptr(bias), float(rate), float(clamp), _stream(stream)))
+
+
+def moe_device_status(reset: bool = True) -> int:
+    out = c_int32()
+    _check("moe_device_status", load().moe_device_status(ctypes.byref(out), 1 if reset else 0))
+    return out.value
+
+
+def stats_from_tensor(t: torch.Tensor) -> dict:
+    """Decode a moe_stats_t held in a uint8 tensor of STATS_BYTES."""
+    raw = bytes(t.detach().cpu().numpy().tobytes())
+    s = MoeStats.from_buffer_copy(raw)
+    return {name: getattr(s, name) for name, _ in MoeStats._fields_ if name != "reserved"}

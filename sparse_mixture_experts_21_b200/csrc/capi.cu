@@ -1,0 +1,215 @@
+// C ABI of the MoE layer library: host-side argument checks and launches.
+// Every check runs before anything is enqueued, so a rejected call has no effect.
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 1;
+  }
+  return cached[dev];
+}
+
+namespace capi {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_config(const moe_config_t* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d_model <= 0 || (c->d_model % 8) != 0) return MOE_ERR_INVALID_ARG;
+  if (c->n_experts < 1 || c->n_experts > 512) return MOE_ERR_INVALID_ARG;
+  if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > 16) return MOE_ERR_INVALID_ARG;
+  if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->x_dtype != MOE_DTYPE_F32 && c->x_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->capacity_mode < MOE_CAP_DROPLESS || c->capacity_mode > MOE_CAP_CF_K_T_OVER_N_FLOOR)
+    return MOE_ERR_INVALID_ARG;
+  if (c->capacity_mode != MOE_CAP_DROPLESS && !(c->capacity_factor > 0.0)) return MOE_ERR_INVALID_ARG;
+  if (c->n_groups > 1) {
+    const int G = c->n_groups;
+    if (G > 32 || c->n_experts % G != 0) return MOE_ERR_INVALID_ARG;
+    const int gs = c->n_experts / G;
+    if (c->topk_groups < 1 || c->topk_groups > G) return MOE_ERR_INVALID_ARG;
+    if (c->group_score_topn < 1 || c->group_score_topn > gs) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)c->topk_groups * gs < c->top_k) return MOE_ERR_INVALID_ARG;
+  }
+  if (c->T * (int64_t)c->top_k > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int64_t capacity_of(const moe_config_t& c) {
+  switch (c.capacity_mode) {
+    case MOE_CAP_CEIL_CF_T_OVER_N:
+      return (int64_t)ceil((c.capacity_factor * (double)c.T) / (double)c.n_experts);
+    case MOE_CAP_CF_K_T_OVER_N_FLOOR: {
+      const double expected = (double)((int64_t)c.top_k * c.T) / (double)c.n_experts;
+      const int64_t C = (int64_t)(expected * c.capacity_factor);
+      return C > c.top_k ? C : c.top_k;
+    }
+    default:
+      return INT64_MAX;
+  }
+}
+
+int route_nblk(const moe_config_t& c) {
+  const int tm = route_tokens_per_block(c.n_experts);
+  return (int)((c.T + tm - 1) / tm);
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace capi
+}  // namespace moe
+
+using namespace moe;
+using namespace moe::capi;
+
+extern "C" {
+
+int moe_capacity(const moe_config_t* cfg, int64_t* capacity) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!capacity) return MOE_ERR_INVALID_ARG;
+  *capacity = capacity_of(*cfg);
+  return MOE_OK;
+}
+
+int moe_route_partials(const moe_config_t* cfg, int32_t* nblk) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!nblk) return MOE_ERR_INVALID_ARG;
+  *nblk = route_nblk(*cfg);
+  return MOE_OK;
+}
+
+int moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = permute_workspace_bytes(*cfg);
+  return MOE_OK;
+}
+
+int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate, const float* logit_offset,
+              const float* bias, int32_t* topk_idx, float* topk_w, float* lse, float* p_partial,
+              float* margin, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_gate || !topk_idx || !topk_w || !lse || !p_partial) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_route(*cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_partial,
+                                margin, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,
+                int32_t* offsets, int32_t* row_of_slot, int32_t* token_of_row, void* x_perm,
+                int32_t* n_dropped, void* ws, size_t ws_bytes, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets || !n_dropped) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!x || !topk_idx || !row_of_slot || !token_of_row || !x_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  const size_t need = permute_workspace_bytes(*cfg);
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && !ws) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_permute(*cfg, capacity_of(*cfg), x, topk_idx, counts, offsets, row_of_slot,
+                                  token_of_row, x_perm, n_dropped, static_cast<int32_t*>(ws),
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+int moe_grouped_ffn(const moe_config_t* cfg, const void* x_rows, int64_t rows_cap,
+                    const int32_t* offsets, int32_t G, const void* w1, const void* w3, const void* w2,
+                    int32_t f, void* h_scratch, void* y_rows, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (rows_cap < 0 || G < 1 || G > 512 || f <= 0 || (f % 8) != 0) return MOE_ERR_INVALID_ARG;
+  if (!offsets) return MOE_ERR_INVALID_ARG;
+  if (rows_cap == 0) return MOE_OK;
+  if (rows_cap > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (!x_rows || !w1 || !w3 || !w2 || !h_scratch || !y_rows) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_rows) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) ||
+      !aligned16(h_scratch) || !aligned16(y_rows))
+    return MOE_ERR_INVALID_ARG;
+  const int d = cfg->d_model;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cfg->x_dtype == MOE_DTYPE_BF16)
+    return from_cuda(launch_ffn_bf16(x_rows, rows_cap, offsets, G, w1, w3, w2, d, f, h_scratch, y_rows, s));
+  return from_cuda(launch_ffn_f32(static_cast<const float*>(x_rows), rows_cap, offsets, G,
+                                  static_cast<const float*>(w1), static_cast<const float*>(w3),
+                                  static_cast<const float*>(w2), d, f, static_cast<float*>(h_scratch),
+                                  static_cast<float*>(y_rows), s));
+}
+
+int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of_slot,
+                const float* topk_w, const void* shared_out, void* y, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!row_of_slot || !topk_w || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || (y_perm && !aligned16(y_perm)) || (shared_out && !aligned16(shared_out)))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_combine(*cfg, y_perm, row_of_slot, topk_w, shared_out, y,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+int moe_router_stats(const moe_config_t* cfg, const int32_t* counts, const int32_t* offsets,
+                     const float* p_partial, const float* lse, const int32_t* n_dropped,
+                     const float* bias, float alpha, float z_coef, moe_stats_t* stats, float* f_out,
+                     float* p_out, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets || !n_dropped || !stats) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!p_partial || !lse)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_stats(*cfg, counts, offsets, p_partial, route_nblk(*cfg), lse, n_dropped,
+                                bias, alpha, z_coef, stats, f_out, p_out,
+                                static_cast<cudaStream_t>(stream)));
+}
+
+int moe_bias_update(const moe_config_t* cfg, const int32_t* counts, float* bias, float rate,
+                    float clamp, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !bias) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_bias_update(*cfg, counts, bias, rate, clamp, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_device_status(int32_t* status, int32_t reset) {
+  if (!status) return MOE_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (reset) {
+    const int32_t z = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(z)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  *status = v;
+  return MOE_OK;
+}
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

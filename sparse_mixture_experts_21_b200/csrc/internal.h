@@ -1,0 +1,49 @@
+// Host-side launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe_b200.h"
+
+namespace moe {
+
+// Padded expert count and tokens per block of the fused router kernel.
+int route_np(int n_experts);
+int route_tokens_per_block(int n_experts);
+
+cudaError_t launch_route(const moe_config_t& c, const void* x, const float* w_gate,
+                         const float* logit_offset, const float* bias, int32_t* topk_idx,
+                         float* topk_w, float* lse, float* p_partial, float* margin,
+                         cudaStream_t s);
+
+// Token-order capacity drop and permutation.
+constexpr int kPermuteTokensPerBlock = 256;
+int permute_blocks(int64_t T);
+size_t permute_workspace_bytes(const moe_config_t& c);
+cudaError_t launch_permute(const moe_config_t& c, int64_t capacity, const void* x,
+                           const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                           int32_t* row_of_slot, int32_t* token_of_row, void* x_perm,
+                           int32_t* n_dropped, int32_t* blk_counts, cudaStream_t s);
+
+// Grouped SwiGLU FFN.
+cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
+                            const void* w1, const void* w3, const void* w2, int d, int f,
+                            void* h, void* y, cudaStream_t s);
+cudaError_t launch_ffn_f32(const float* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
+                           const float* w1, const float* w3, const float* w2, int d, int f,
+                           float* h, float* y, cudaStream_t s);
+
+cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
+                           const float* topk_w, const void* shared_out, void* y, cudaStream_t s);
+cudaError_t launch_stats(const moe_config_t& c, const int32_t* counts, const int32_t* offsets,
+                         const float* p_partial, int nblk, const float* lse,
+                         const int32_t* n_dropped, const float* bias, float alpha, float z_coef,
+                         moe_stats_t* stats, float* f_out, float* p_out, cudaStream_t s);
+cudaError_t launch_bias_update(const moe_config_t& c, const int32_t* counts, float* bias,
+                               float rate, float clamp, cudaStream_t s);
+
+int sm_count();
+
+}  // namespace moe

@@ -1,0 +1,8 @@
+// Single translation unit of the library (one module, so every kernel file sees
+// the same device status word without relocatable device code).
+#include "capi.cu"
+#include "route.cu"
+#include "permute.cu"
+#include "ffn_tc.cu"
+#include "ffn_f32.cu"
+#include "combine_stats.cu"

@@ -1,0 +1,102 @@
+"""One MoE FFN layer forward through the C ABI: buffers plus the call sequence.
+
+This is orchestration only (allocation through torch, then route -> permute ->
+grouped FFN (routed, shared) -> combine -> statistics -> bias update, all on one
+stream); every step runs in the library's kernels.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+from .synth import Workload, torch_dtype
+
+CAP_MODES = {"dropless": L.CAP_DROPLESS, "ceil_cf_T_over_N": L.CAP_CEIL_CF_T_OVER_N,
+             "floor_cf_k_T_over_N": L.CAP_CF_K_T_OVER_N_FLOOR}
+
+
+def make_config(w: Workload, T: Optional[int] = None) -> L.MoeConfig:
+    c = L.MoeConfig()
+    c.T = w.T if T is None else T
+    c.d_model, c.n_experts, c.top_k, c.d_ff = w.d, w.N, w.k, w.f
+    c.score_fn = L.SCORE_SIGMOID if w.score == "sigmoid" else L.SCORE_SOFTMAX
+    c.renorm = 1 if w.renorm else 0
+    c.n_groups, c.topk_groups, c.group_score_topn = w.n_groups, w.topk_groups, w.group_topn
+    c.capacity_mode = CAP_MODES[w.capacity]
+    c.capacity_factor = w.cf
+    c.x_dtype = L.DTYPE_F32 if w.dtype == "fp32" else L.DTYPE_BF16
+    return c
+
+
+class MoELayer:
+    """Holds the weights and the per-call buffers of one layer for up to T tokens."""
+
+    def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True):
+        self.w = w
+        self.dev = torch.device(device)
+        self.weights = weights
+        self.update_bias = update_bias and weights.get("bias") is not None
+        self.cfg = make_config(w)
+        T, d, N, k = w.T, w.d, w.N, w.k
+        dt = torch_dtype(w)
+        z = lambda *s, dtype=torch.float32: torch.empty(s, dtype=dtype, device=self.dev)  # noqa: E731
+        self.nblk = L.route_partials(self.cfg)
+        self.topk_idx = z(T, k, dtype=torch.int32)
+        self.topk_w = z(T, k)
+        self.lse = z(T)
+        self.p_partial = z(max(self.nblk, 1), N)
+        self.margin = z(T)
+        self.counts = z(N, dtype=torch.int32)
+        self.offsets = z(N + 1, dtype=torch.int32)
+        self.row_of_slot = z(T, k, dtype=torch.int32)
+        self.token_of_row = z(max(T * k, 1), dtype=torch.int32)
+        self.x_perm = z(max(T * k, 1), d, dtype=dt)
+        self.n_dropped = z(2, dtype=torch.int32)
+        self.ws = z(max(L.workspace_size(self.cfg), 16), dtype=torch.uint8)
+        self.h = z(max(T * k, 1), w.f, dtype=dt)
+        self.y_perm = z(max(T * k, 1), d, dtype=dt)
+        self.fs = w.n_shared * w.f_shared
+        if self.fs > 0:
+            self.shared_offsets = torch.tensor([0, T], dtype=torch.int32, device=self.dev)
+            self.hs = z(max(T, 1), self.fs, dtype=dt)
+            self.ys = z(max(T, 1), d, dtype=dt)
+        self.y = z(max(T, 1), d, dtype=dt)
+        self.stats = torch.zeros(L.STATS_BYTES, dtype=torch.uint8, device=self.dev)
+        self.f_out = z(N)
+        self.p_out = z(N)
+
+    # the launches of one layer forward; `x` is [T, d] on the device
+    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        W, c, T = self.weights, self.cfg, self.w.T
+        L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), self.topk_idx,
+                    self.topk_w, self.lse, self.p_partial, self.margin, stream)
+        L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
+                      self.token_of_row, self.x_perm, self.n_dropped, self.ws, stream)
+        L.moe_grouped_ffn(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
+                          W["w2"], self.w.f, self.h, self.y_perm, stream)
+        shared = None
+        if self.fs > 0:
+            L.moe_grouped_ffn(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], self.fs,
+                              self.hs, self.ys, stream)
+            shared = self.ys
+        L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, self.y, stream)
+        L.moe_router_stats(c, self.counts, self.offsets, self.p_partial, self.lse, self.n_dropped,
+                           W.get("bias"), self.w.alpha, self.w.z_coef, self.stats, self.f_out,
+                           self.p_out, stream)
+        if self.update_bias:
+            L.moe_bias_update(c, self.counts, W["bias"], self.w.bias_rate, 0.0, stream)
+        return self.y
+
+    def kernel_launches(self) -> int:
+        """Number of the library's kernels one forward launches."""
+        n = 1 + 4 + 2 + 1 + 1          # route, permute (4), routed FFN (2), combine, stats
+        if self.fs > 0:
+            n += 2
+        if self.update_bias:
+            n += 1
+        return n
+
+    def stats_dict(self) -> dict:
+        return L.stats_from_tensor(self.stats)

@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol the header declares, answers sizing queries, and rejects bad arguments
+before enqueueing anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_mixture_experts_21_b200 import _lib as L
+from sparse_mixture_experts_21_b200 import layer, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if fn.endswith(".h"):
+            text = open(os.path.join(inc, fn)).read()
+            names.update(re.findall(r"^\s*(?:int|const char\*)\s+(moe_\w+)\s*\(", text, re.M))
+    return names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    declared = _declared_symbols()
+    assert declared >= set(L.EXPORTED)
+    for name in declared:
+        assert getattr(lib, name) is not None
+
+
+def test_config_struct_layout():
+    assert ctypes.sizeof(L.MoeConfig) == 64
+    assert L.MoeConfig.capacity_factor.offset == 56
+    assert ctypes.sizeof(L.MoeStats) == 64
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_sizing_queries(lib, name):
+    w = synth.WORKLOADS[name]
+    c = layer.make_config(w)
+    tm = 32 if w.N <= 32 or w.N > 256 else 64
+    assert L.route_partials(c) == (w.T + tm - 1) // tm
+    assert L.workspace_size(c) == ((w.T + 255) // 256) * w.N * 4
+    cap = L.capacity(c)
+    if w.capacity == "dropless":
+        assert cap == 2 ** 63 - 1
+    else:
+        assert cap == -(-int(w.cf * w.T) // w.N)
+
+
+def test_capacity_variants(lib):
+    c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    assert L.capacity(c) == 40                        # ceil(1.25 * 256 / 8)
+    c.capacity_mode = L.CAP_CF_K_T_OVER_N_FLOOR
+    assert L.capacity(c) == 80                        # max(int(2 * 256 / 8 * 1.25), 2)
+    c.T, c.capacity_factor = 10, 0.01
+    assert L.capacity(c) == 2                         # never below k
+
+
+def _status(fn, *args):
+    return fn(*args)
+
+
+@pytest.mark.parametrize("field,value", [
+    ("top_k", 0), ("top_k", 9), ("n_experts", 0), ("n_experts", 513), ("d_model", 12),
+    ("score_fn", 7), ("x_dtype", 5), ("capacity_mode", 9), ("n_groups", 3),
+])
+def test_invalid_config_rejected(lib, field, value):
+    c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    setattr(c, field, value)
+    out = ctypes.c_int64()
+    assert lib.moe_capacity(ctypes.byref(c), ctypes.byref(out)) == L.MOE_ERR_INVALID_ARG
+
+
+def test_group_limit_validation(lib):
+    c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    out = ctypes.c_int64()
+    assert lib.moe_capacity(ctypes.byref(c), ctypes.byref(out)) == L.MOE_OK
+    c.topk_groups = 0
+    assert lib.moe_capacity(ctypes.byref(c), ctypes.byref(out)) == L.MOE_ERR_INVALID_ARG
+    c.topk_groups, c.group_score_topn = 4, 33              # more than a group holds
+    assert lib.moe_capacity(ctypes.byref(c), ctypes.byref(out)) == L.MOE_ERR_INVALID_ARG
+    c.group_score_topn, c.n_groups, c.topk_groups = 2, 32, 1   # 1 group of 8 < k = 8? equal: ok
+    assert lib.moe_capacity(ctypes.byref(c), ctypes.byref(out)) == L.MOE_OK
+    c.top_k = 9
+    assert lib.moe_capacity(ctypes.byref(c), ctypes.byref(out)) == L.MOE_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    cp = ctypes.byref(c)
+    # null required pointers: rejected on the host, nothing launched
+    assert lib.moe_route(cp, None, None, None, None, None, None, None, None, None, None) == L.MOE_ERR_INVALID_ARG
+    bad = 0x1000008  # not 16-byte aligned
+    ok = 0x1000000
+    assert lib.moe_route(cp, bad, ok, None, None, ok, ok, ok, ok, None, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(cp, ok, ok, ok, None, bad, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_ffn(cp, ok, 10, ok, 0, ok, ok, ok, 256, ok, ok, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_ffn(cp, ok, 10, ok, 1, ok, ok, ok, 12, ok, ok, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update(cp, None, ok, 1e-3, 0.0, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_stats(cp, ok, ok, ok, ok, ok, None, 0.0, 0.0, None, None, None, None) == \
+        L.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_too_small_rejected(lib):
+    c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    ok = 0x1000000
+    st = lib.moe_permute(ctypes.byref(c), ok, ok, ok, ok, ok, ok, ok, ok, ok, 4, None)
+    assert st == L.MOE_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_empty_batch_is_a_no_op(lib):
+    c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"], T=0)
+    assert lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, None, None) == L.MOE_OK
+    assert lib.moe_combine(ctypes.byref(c), None, None, None, None, None, None) == L.MOE_OK
+    assert lib.moe_grouped_ffn(ctypes.byref(c), None, 0, 0x1000000, 1, None, None, None, 256, None, None,
+                               None) == L.MOE_OK
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.moe_status_string(s)
+    assert b"timed out" in lib.moe_status_string(L.MOE_ERR_DEVICE_TIMEOUT)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(FileNotFoundError):
+        L.load(str(tmp_path / "nope.so"))

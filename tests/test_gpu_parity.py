@@ -1,0 +1,358 @@
+"""GPU-vs-oracle parity of every step of the layer, through the C ABI.
+
+Reduced shapes of each workload family span several tiles and ragged tails and
+are checked element by element; the full-size workloads are checked on sampled
+tokens and rows plus every integer output.  Integer outputs (indices, counts,
+offsets, row maps, drops) must be bit-exact; floating outputs within
+max|a-b|/max|b| <= 2e-2 (bf16) or 1e-4 (fp32), statistics within 1e-5.  Tokens
+whose k-th vs (k+1)-th selection margin is below 1e-4 are excluded from the
+index comparison and counted; the permutation is cross-fed (the oracle permutes
+the GPU's routing) so that one near-tie cannot cascade.
+"""
+from __future__ import annotations
+
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from sparse_mixture_experts_21_b200 import _lib as L
+from sparse_mixture_experts_21_b200.layer import MoELayer, make_config
+from sparse_mixture_experts_21_b200.synth import WORKLOADS, make_inputs, random_routing, torch_dtype
+from tests.parity_util import (NEAR_TIE, TOL_STATS, expert_weights_fn, f64, i64, oracle_cfg,
+                               rel_err, shared_weights, tol_for)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny_top2_fp32": WORKLOADS["tiny_top2_fp32"],
+    "mixtral_small": replace(WORKLOADS["mixtral_8x7b"], name="mixtral_small", T=513, d=512, f=1024),
+    "dsmoe_small": replace(WORKLOADS["deepseekmoe_16b"], name="dsmoe_small", T=777, d=264, N=16,
+                           f=192, f_shared=192),
+    "v3_small": replace(WORKLOADS["deepseek_v3"], name="v3_small", T=1000, d=512, N=64, f=256,
+                        f_shared=256),
+    "switch_small": replace(WORKLOADS["switch_skewed"], name="switch_small", T=2000, d=256, N=32,
+                            f=512),
+}
+
+
+def _run(w, seed=0, update_bias=False):
+    torch.cuda.synchronize()
+    inp = make_inputs(w, "cuda", seed=seed)
+    bias0 = None if inp["bias"] is None else inp["bias"].clone()
+    lay = MoELayer(w, inp, "cuda", update_bias=update_bias)
+    lay.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    return lay, inp, bias0
+
+
+@pytest.fixture(scope="module")
+def small_runs():
+    return {name: _run(w) for name, w in SMALL.items()}
+
+
+# ----------------------------------------------------------------------------- routing
+def _check_route(w, lay, inp, tokens):
+    cfg = oracle_cfg(w)
+    x = f64(inp["x"])[tokens]
+    r = O.route(x, f64(inp["w_gate"]), cfg, bias=f64(inp["bias"]), logit_offset=f64(inp["logit_offset"]))
+    gidx = i64(lay.topk_idx)[tokens]
+    gw = f64(lay.topk_w)[tokens]
+    clear = r["margin"] >= NEAR_TIE
+    n_tie = int((~clear).sum())
+    assert np.array_equal(gidx[clear], r["idx"][clear]), "expert indices differ on a clear token"
+    assert np.max(np.abs(gw[clear] - r["w"][clear])) < 2e-5
+    assert rel_err(f64(lay.lse)[tokens], r["lse"]) < 1e-5
+    gm = f64(lay.margin)[tokens]
+    fin = np.isfinite(r["margin"]) & clear
+    assert np.all(np.abs(gm[fin] - r["margin"][fin]) < 1e-4 + 1e-4 * np.abs(r["margin"][fin]))
+    return n_tie, r
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_route_parity(small_runs, name):
+    lay, inp, _ = small_runs[name]
+    w = SMALL[name]
+    n_tie, r = _check_route(w, lay, inp, np.arange(w.T))
+    print(f"{name}: near-ties {n_tie}/{w.T}")
+    # weights sum to one, k distinct experts
+    assert np.allclose(f64(lay.topk_w).sum(1), 1.0, atol=1e-5)
+    gidx = i64(lay.topk_idx)
+    assert all(len(set(row)) == w.k for row in gidx.tolist())
+
+
+# ----------------------------------------------------------------------------- permutation
+def _check_permute(w, lay, inp):
+    idx = i64(lay.topk_idx)
+    p = O.permutation(idx, w.N, O.capacity(oracle_cfg(w), w.T))
+    assert np.array_equal(i64(lay.counts), p["counts"])
+    assert np.array_equal(i64(lay.offsets), p["offsets"])
+    assert np.array_equal(i64(lay.row_of_slot), p["row_of_slot"])
+    R = p["R"]
+    assert np.array_equal(i64(lay.token_of_row)[:R], p["token_of_row"])
+    assert i64(lay.n_dropped).tolist() == [p["dropped_slots"], p["dropped_tokens"]]
+    # the gather is a byte copy
+    tor = lay.token_of_row[:R].long()
+    assert torch.equal(lay.x_perm[:R], inp["x"][tor])
+    return p
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_permute_parity(small_runs, name):
+    lay, inp, _ = small_runs[name]
+    p = _check_permute(SMALL[name], lay, inp)
+    if SMALL[name].capacity != "dropless":
+        assert p["dropped_slots"] > 0
+
+
+# ----------------------------------------------------------------------------- expert FFN
+def _check_ffn_rows(w, lay, inp, rows_by_expert):
+    get = expert_weights_fn(inp)
+    xs, hs, ys, hr, yr = [], [], [], [], []
+    for e, rows in rows_by_expert.items():
+        if len(rows) == 0:
+            continue
+        xr = f64(lay.x_perm[rows])
+        w1, w3, w2 = get(e)
+        hr.append(O.swiglu_hidden(xr, w1, w3))
+        yr.append(O.swiglu_ffn(xr, w1, w3, w2))
+        hs.append(f64(lay.h[rows]))
+        ys.append(f64(lay.y_perm[rows]))
+    tol = tol_for(w)
+    assert rel_err(np.concatenate(hs), np.concatenate(hr)) < tol
+    assert rel_err(np.concatenate(ys), np.concatenate(yr)) < tol
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_grouped_ffn_parity(small_runs, name):
+    lay, inp, _ = small_runs[name]
+    w = SMALL[name]
+    off = i64(lay.offsets)
+    _check_ffn_rows(w, lay, inp, {e: torch.arange(off[e], off[e + 1], device="cuda") for e in range(w.N)})
+
+
+@pytest.mark.parametrize("name", [n for n in SMALL if SMALL[n].n_shared > 0])
+def test_shared_ffn_parity(small_runs, name):
+    lay, inp, _ = small_runs[name]
+    w = SMALL[name]
+    ref = O.swiglu_ffn(f64(inp["x"]), *shared_weights(inp))
+    assert rel_err(f64(lay.ys[:w.T]), ref) < tol_for(w)
+
+
+# ----------------------------------------------------------------------------- combine
+@pytest.mark.parametrize("name", list(SMALL))
+def test_combine_parity(small_runs, name):
+    lay, inp, _ = small_runs[name]
+    w = SMALL[name]
+    ys = f64(lay.ys[:w.T]) if lay.fs > 0 else None
+    ref = O.combine(f64(lay.y_perm), i64(lay.row_of_slot), f64(lay.topk_w), ys, w.T, w.d)
+    assert rel_err(f64(lay.y[:w.T]), ref) < tol_for(w)
+
+
+# ----------------------------------------------------------------------------- whole layer
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_end_to_end(small_runs, name):
+    """The layer output against the oracle's own forward (its own routing)."""
+    lay, inp, _ = small_runs[name]
+    w = SMALL[name]
+    cfg = oracle_cfg(w)
+    out = O.layer_forward(f64(inp["x"]), f64(inp["w_gate"]), cfg, expert_weights_fn(inp),
+                          shared_weights(inp), bias=f64(inp["bias"]),
+                          logit_offset=f64(inp["logit_offset"]), alpha=w.alpha, z_coef=w.z_coef)
+    margin = out["routing"]["margin"]
+    clear = margin >= NEAR_TIE
+    if np.all(clear):
+        assert rel_err(f64(lay.y[:w.T]), out["y"]) < tol_for(w)
+        st, ost = lay.stats_dict(), out["stats"]
+        for key in ("aux", "aux_raw", "z", "cv", "cv_kept"):
+            assert abs(st[key] - ost[key]) <= TOL_STATS * max(abs(ost[key]), 1e-30), key
+        for key in ("dead", "dropped_slots", "dropped_tokens"):
+            assert st[key] == ost[key], key
+    elif w.capacity == "dropless":
+        # tokens are independent when nothing is dropped: compare the clear ones
+        assert rel_err(f64(lay.y[:w.T])[clear], out["y"][clear]) < tol_for(w)
+    else:
+        # a near-tie can move a capacity cut: feed the oracle the GPU's expert choice
+        wts = O.gate_weights(out["routing"]["s"], i64(lay.topk_idx), w.renorm)
+        out2 = O.layer_forward(f64(inp["x"]), None, cfg, expert_weights_fn(inp), shared_weights(inp),
+                               routing={"idx": i64(lay.topk_idx), "w": wts})
+        assert rel_err(f64(lay.y[:w.T]), out2["y"]) < tol_for(w)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_stats_parity(small_runs, name):
+    """Statistics against the oracle, fed the GPU's integer routing decision."""
+    lay, inp, _ = small_runs[name]
+    w = SMALL[name]
+    cfg = oracle_cfg(w)
+    r = O.route(f64(inp["x"]), f64(inp["w_gate"]), cfg, bias=f64(inp["bias"]),
+                logit_offset=f64(inp["logit_offset"]))
+    p = O.permutation(i64(lay.topk_idx), w.N, O.capacity(cfg, w.T))
+    ost = O.router_stats(p["counts"], p["kept"], r["s"], r["lse"], cfg, w.T, p["dropped_slots"],
+                         p["dropped_tokens"], w.alpha, w.z_coef, f64(inp["bias"]))
+    st = lay.stats_dict()
+    for key in ("aux", "aux_raw", "z", "z_loss", "cv", "cv_kept", "bias_norm"):
+        assert abs(st[key] - ost[key]) <= TOL_STATS * max(abs(ost[key]), 1e-30) + 1e-12, key
+    for key in ("dead", "dropped_slots", "dropped_tokens"):
+        assert st[key] == ost[key], key
+    assert st["R"] == p["R"]
+    assert rel_err(f64(lay.f_out), ost["f"]) < TOL_STATS
+    assert rel_err(f64(lay.p_out), ost["P"]) < TOL_STATS
+
+
+def test_bias_update_parity():
+    w = SMALL["v3_small"]
+    lay, inp, b0 = _run(w, update_bias=True)
+    ref = O.bias_update(f64(b0), i64(lay.counts), rate=w.bias_rate)
+    assert np.max(np.abs(f64(inp["bias"]) - ref)) < 1e-7
+    # clamp variant through the C ABI
+    b = torch.full((w.N,), 0.0095, device="cuda")
+    L.moe_bias_update(make_config(w), lay.counts, b, 1e-3, 1e-2)
+    torch.cuda.synchronize()
+    refc = O.bias_update(np.full(w.N, 0.0095, dtype=np.float32).astype(np.float64), i64(lay.counts),
+                         rate=1e-3, clamp=1e-2)
+    assert np.max(np.abs(f64(b) - refc)) < 1e-7
+
+
+def test_deterministic_twice():
+    w = SMALL["dsmoe_small"]
+    inp = make_inputs(w, "cuda")
+    lay = MoELayer(w, inp, "cuda", update_bias=False)
+    lay.forward(inp["x"])
+    first = [t.clone() for t in (lay.topk_idx, lay.topk_w, lay.row_of_slot, lay.x_perm, lay.y_perm,
+                                 lay.y, lay.stats)]
+    lay.forward(inp["x"])
+    torch.cuda.synchronize()
+    second = (lay.topk_idx, lay.topk_w, lay.row_of_slot, lay.x_perm, lay.y_perm, lay.y, lay.stats)
+    for a, b in zip(first, second):
+        assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("T", [1, 31, 257])
+def test_ragged_token_counts(T):
+    w = replace(SMALL["v3_small"], T=T)
+    lay, inp, _ = _run(w)
+    _check_route(w, lay, inp, np.arange(T))
+    _check_permute(w, lay, inp)
+    off = i64(lay.offsets)
+    _check_ffn_rows(w, lay, inp, {e: torch.arange(off[e], off[e + 1], device="cuda") for e in range(w.N)})
+
+
+def test_k_equals_n():
+    w = replace(SMALL["mixtral_small"], T=100, N=4, k=4)
+    lay, inp, _ = _run(w)
+    _check_permute(w, lay, inp)
+    out = O.layer_forward(f64(inp["x"]), f64(inp["w_gate"]), oracle_cfg(w), expert_weights_fn(inp))
+    assert rel_err(f64(lay.y[:w.T]), out["y"]) < tol_for(w)
+
+
+def _permute_with(w, idx):
+    """Run moe_permute on a given routing (device) and compare with the oracle."""
+    c = make_config(w)
+    T, k, N = w.T, w.k, w.N
+    x = torch.randn(T, w.d, device="cuda").to(torch_dtype(w))
+    dev = lambda *s, dtype=torch.int32: torch.full(s, -7, dtype=dtype, device="cuda")  # noqa: E731
+    counts, offsets, ros, tor, nd = dev(N), dev(N + 1), dev(T, k), dev(T * k), dev(2)
+    xp = torch.zeros(T * k, w.d, dtype=torch_dtype(w), device="cuda")
+    ws = torch.empty(max(L.workspace_size(c), 16), dtype=torch.uint8, device="cuda")
+    L.moe_permute(c, x, idx, counts, offsets, ros, tor, xp, nd, ws)
+    torch.cuda.synchronize()
+    p = O.permutation(i64(idx), N, O.capacity(oracle_cfg(w), T))
+    assert np.array_equal(i64(counts), p["counts"]) and np.array_equal(i64(offsets), p["offsets"])
+    assert np.array_equal(i64(ros), p["row_of_slot"])
+    assert np.array_equal(i64(tor)[:p["R"]], p["token_of_row"])
+    assert i64(nd).tolist() == [p["dropped_slots"], p["dropped_tokens"]]
+    assert torch.equal(xp[:p["R"]], x[tor[:p["R"]].long()])
+    return p
+
+
+def test_permute_all_tokens_to_one_expert_with_capacity():
+    w = replace(SMALL["switch_small"], T=3000, N=16, k=2, capacity="ceil_cf_T_over_N", cf=1.0)
+    idx = random_routing(w.T, w.N, w.k, "cuda", seed=3, hot=5)
+    p = _permute_with(w, idx)
+    assert p["kept"][5] == -(-w.T // w.N) and p["dropped_slots"] > 0
+
+
+def test_permute_floor_capacity_variant_and_empty_experts():
+    w = replace(SMALL["dsmoe_small"], T=600, N=64, k=2, capacity="floor_cf_k_T_over_N", cf=0.5)
+    idx = random_routing(w.T, 8, w.k, "cuda", seed=4)          # only experts 0..7 used
+    p = _permute_with(w, idx)
+    assert (p["counts"][8:] == 0).all() and p["dropped_slots"] > 0
+
+
+def test_permute_many_blocks_dropless():
+    w = replace(SMALL["v3_small"], T=5000, N=256, k=8)
+    idx = random_routing(w.T, w.N, w.k, "cuda", seed=5)
+    _permute_with(w, idx)
+
+
+def test_grouped_ffn_empty_and_tiny_groups():
+    """Groups with 0, 1, 127, 128, 129 rows and rows_cap beyond the last row."""
+    d, f = 256, 384
+    sizes = [0, 1, 127, 0, 128, 129, 300, 0]
+    G = len(sizes)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    R, cap = int(off[-1]), int(off[-1]) + 70
+    g = torch.Generator(device="cuda").manual_seed(7)
+    xr = torch.randn(cap, d, generator=g, device="cuda").to(torch.bfloat16)
+    w1 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w3 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(G, d, f, generator=g, device="cuda") / f ** 0.5).to(torch.bfloat16)
+    h = torch.empty(cap, f, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((cap, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    wk = replace(SMALL["mixtral_small"], d=d, f=f, N=G)
+    L.moe_grouped_ffn(make_config(wk), xr, cap, torch.tensor(off, device="cuda"), G, w1, w3, w2, f, h, y)
+    torch.cuda.synchronize()
+    ref = np.zeros((R, d))
+    for e in range(G):
+        lo, hi = off[e], off[e + 1]
+        if hi > lo:
+            ref[lo:hi] = O.swiglu_ffn(f64(xr[lo:hi]), f64(w1[e]), f64(w3[e]), f64(w2[e]))
+    assert rel_err(f64(y[:R]), ref) < 2e-2
+    assert torch.all(y[R:] == 3.0)                     # rows past the last group untouched
+
+
+# ----------------------------------------------------------------------------- full size
+FULL = ["mixtral_8x7b", "deepseekmoe_16b", "deepseek_v3", "switch_skewed"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload(name):
+    w = WORKLOADS[name]
+    lay, inp, _ = _run(w)
+    rng = np.random.default_rng(0)
+    sample = np.sort(rng.choice(w.T, size=min(w.T, 512), replace=False))
+    n_tie, r = _check_route(w, lay, inp, sample)
+    print(f"{name}: near-ties {n_tie}/{len(sample)} sampled tokens")
+    p = _check_permute(w, lay, inp)
+    # expert rows: 8 experts (the most and least loaded included), up to 48 rows each
+    off = i64(lay.offsets)
+    loads = np.diff(off)
+    pick = sorted(set([int(np.argmax(loads)), int(np.argmin(np.where(loads > 0, loads, 1 << 30)))] +
+                      rng.choice(w.N, size=min(w.N, 6), replace=False).tolist()))
+    rows = {}
+    for e in pick:
+        n = int(loads[e])
+        if n:
+            sel = np.unique(np.concatenate([[0, n - 1], rng.choice(n, size=min(n, 46), replace=False)]))
+            rows[e] = torch.tensor(off[e] + sel, device="cuda")
+    _check_ffn_rows(w, lay, inp, rows)
+    # combine + whole layer on sampled tokens, oracle fed the GPU's expert choice
+    tok = sample[:24]
+    cfg = oracle_cfg(w)
+    s = O.affinity(O.router_logits(f64(inp["x"][torch.tensor(tok, device="cuda")]), f64(inp["w_gate"]),
+                                   f64(inp["logit_offset"])), cfg.score_fn)
+    wts = np.zeros((w.T, w.k))
+    wts[tok] = O.gate_weights(s, i64(lay.topk_idx)[tok], cfg.renorm)
+    out = O.layer_forward(f64(inp["x"]), None, cfg, expert_weights_fn(inp), shared_weights(inp),
+                          tokens=tok, routing={"idx": i64(lay.topk_idx), "w": wts})
+    assert rel_err(f64(lay.y[torch.tensor(tok, device="cuda")]), out["y"]) < tol_for(w)
+    st = lay.stats_dict()
+    assert st["dropped_slots"] == p["dropped_slots"] and st["R"] == p["R"]
+    assert st["dead"] == int((p["counts"] == 0).sum())
+    c = p["counts"].astype(np.float64)
+    assert abs(st["cv"] - np.std(c) / np.mean(c)) <= TOL_STATS * max(np.std(c) / np.mean(c), 1e-30)
