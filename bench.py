@@ -56,26 +56,27 @@ def _sha1(path):
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region
+    (all GPUs are sampled; lines are kept for the device's UUID)."""
+    Q = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index):
-        self.dev = device_index
+    def __init__(self, uuid):
+        self.uuid = uuid
         self.proc = None
+        self.lines = []
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200",
-                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
         return self
 
     def __exit__(self, *a):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -86,30 +87,34 @@ class ClockSampler:
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
+        rows = [[x.strip() for x in ln.split(",")] for ln in self.lines]
+        rows = [r for r in rows if len(r) >= 9]
+        mine = [r for r in rows if self.uuid and self.uuid in r[0]]
+        if not mine and len({r[0] for r in rows}) == 1:
+            mine = rows
+        sm, smax, power, reasons = [], None, [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
+        for r in mine:
             try:
-                sm.append(float(f[1]))
-                smax = float(f[2])
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                power.append(float(r[3]))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(names, r[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "power_w_median": statistics.median(power) if power else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def _nvsmi_index(dev):
+def _device_uuid(dev):
     try:
-        return torch.cuda.get_device_properties(dev).pci_bus_id
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
     except Exception:
-        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-        return vis.split(",")[dev] if vis else dev
+        return None
 
 
 # ---------------------------------------------------------------------------- reference arm
@@ -196,6 +201,10 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="reduced token count (profiling of a small case only)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="reduced routed-expert count (profiling of a small case only)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
@@ -219,6 +228,9 @@ def main():
 
     L.load()
     w = WORKLOADS[WORKLOAD]
+    if args.tokens or args.experts:
+        from dataclasses import replace
+        w = replace(w, name=WORKLOAD + "_reduced", T=args.tokens or w.T, N=args.experts or w.N)
     inp = make_inputs(w, dev, seed=rank)
     lay = MoELayer(w, inp, dev)
     x = inp["x"]
@@ -238,7 +250,7 @@ def main():
     marks = [[ev() for _ in range(7)] for _ in range(args.steps)]
     W = lay.weights
     c = lay.cfg
-    with ClockSampler(_nvsmi_index(local)) as clk:
+    with ClockSampler(_device_uuid(local)) as clk:
         barrier()
         start, end = ev(), ev()
         start.record(stream)
@@ -246,7 +258,7 @@ def main():
             m = marks[i]
             m[0].record(stream)
             L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), lay.topk_idx, lay.topk_w,
-                        lay.lse, lay.p_partial, lay.margin)
+                        lay.lse, lay.p_partial, lay.margin, lay.ws)
             m[1].record(stream)
             L.moe_permute(c, x, lay.topk_idx, lay.counts, lay.offsets, lay.row_of_slot, lay.token_of_row,
                           lay.x_perm, lay.n_dropped, lay.ws)
@@ -328,7 +340,7 @@ def main():
             "metric": METRIC, "value": world * T / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "T": T, "d_model": d, "experts": N, "top_k": k, "d_ff": f,
+            "config": {"workload": w.name, "T": T, "d_model": d, "experts": N, "top_k": k, "d_ff": f,
                        "shared_experts": w.n_shared, "score": "sigmoid+bias", "groups": "8 keep 4",
                        "capacity": "dropless", "rows_R": R, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (x 235 MB, experts 22.5 GB); no flush"},

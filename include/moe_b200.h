@@ -101,7 +101,9 @@ int moe_capacity(const moe_config_t* cfg, int64_t* capacity);
 /* Rows of the p_partial buffer written by moe_route (host out). */
 int moe_route_partials(const moe_config_t* cfg, int32_t* nblk);
 
-/* Bytes of scratch `ws` needed by moe_permute for cfg (host out). */
+/* Bytes of scratch `ws` needed by moe_route and moe_permute for cfg (host out):
+ * the larger of the two, so one buffer serves both when the calls are ordered on
+ * one stream.  Calls that share a workspace must not overlap on the GPU. */
 int moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
 
 /* ---------------------------------------------------------------------------
@@ -126,12 +128,15 @@ int moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
  *   margin       [T] fp32 out or NULL: selection score of the k-th pick minus the
  *                best eligible expert left out, min'ed with the last-kept minus
  *                best-dropped group score (+inf when nothing is left out)
- * The router GEMM accumulates in fp32.  T = 0 is a no-op.
+ *   ws           scratch of at least moe_workspace_size() bytes (clobbered)
+ * The router GEMM is fp32-equivalent: fp32 FMA, or for bf16 x and N <= 256 the
+ * tensor cores over an exact three-way bf16 split of w_gate (every product exact,
+ * fp32 accumulation).  T = 0 is a no-op.
  * ------------------------------------------------------------------------- */
 int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate,
               const float* logit_offset, const float* bias,
               int32_t* topk_idx, float* topk_w, float* lse, float* p_partial,
-              float* margin, void* stream);
+              float* margin, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_permute -- counts, capacity drop in token order, offsets, row maps, gather.
@@ -201,7 +206,7 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_
  *
  * Defines: llm-compass "负载均衡" (L_aux = alpha N sum f_i P_i), the Practice page's
  * "负载均衡损失" (equals 1 unscaled under uniform routing) and "MoE 的可观测性"
- * metrics (drop ratio, per-expert load); the landscape page's monitoring list
+ * (专家间的尺度漂移 section: drop ratio and per-expert load as the minimum metrics); the landscape page's monitoring list
  * (token drop, usage CV, dead experts, bias norm).  z-loss has no formula on the
  * pages; mean_t (logsumexp_e z)^2 is used.
  *   counts [N], offsets [N+1], p_partial [nblk, N], lse [T], n_dropped [2],

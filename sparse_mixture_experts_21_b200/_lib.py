@@ -72,7 +72,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_capacity": [cfgp, POINTER(c_int64)],
         "moe_route_partials": [cfgp, i32p],
         "moe_workspace_size": [cfgp, POINTER(c_size_t)],
-        "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
         "moe_permute": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
         "moe_grouped_ffn": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp],
         "moe_combine": [cfgp, vp, vp, vp, vp, vp, vp],
@@ -129,11 +129,12 @@ def workspace_size(cfg: MoeConfig) -> int:
 
 
 # ----------------------------------------------------------------------------- entry points
-def moe_route(cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_partial, margin=None,
+def moe_route(cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_partial, margin, ws,
               stream=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("moe_route", load().moe_route(
         ctypes.byref(cfg), _ptr(x), _ptr(w_gate), _ptr(logit_offset), _ptr(bias), _ptr(topk_idx),
-        _ptr(topk_w), _ptr(lse), _ptr(p_partial), _ptr(margin), _stream(stream)))
+        _ptr(topk_w), _ptr(lse), _ptr(p_partial), _ptr(margin), _ptr(ws), nbytes, _stream(stream)))
 
 
 def moe_permute(cfg, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, n_dropped,

@@ -64,7 +64,7 @@ int64_t capacity_of(const moe_config_t& c) {
 }
 
 int route_nblk(const moe_config_t& c) {
-  const int tm = route_tokens_per_block(c.n_experts);
+  const int tm = route_tokens_per_block(c);
   return (int)((c.T + tm - 1) / tm);
 }
 
@@ -98,20 +98,24 @@ int moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
   const int st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (!bytes) return MOE_ERR_INVALID_ARG;
-  *bytes = permute_workspace_bytes(*cfg);
+  const size_t a = permute_workspace_bytes(*cfg), b = route_workspace_bytes(*cfg);
+  *bytes = a > b ? a : b;
   return MOE_OK;
 }
 
 int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate, const float* logit_offset,
               const float* bias, int32_t* topk_idx, float* topk_w, float* lse, float* p_partial,
-              float* margin, void* stream) {
+              float* margin, void* ws, size_t ws_bytes, void* stream) {
   const int st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
   if (!x || !w_gate || !topk_idx || !topk_w || !lse || !p_partial) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+  const size_t need = route_workspace_bytes(*cfg);
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && (!ws || !aligned16(ws))) return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_route(*cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_partial,
-                                margin, static_cast<cudaStream_t>(stream)));
+                                margin, ws, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,
@@ -125,7 +129,7 @@ int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
   if (cfg->T > 0 && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
   const size_t need = permute_workspace_bytes(*cfg);
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
-  if (need > 0 && !ws) return MOE_ERR_INVALID_ARG;
+  if (need > 0 && (!ws || !aligned16(ws))) return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_permute(*cfg, capacity_of(*cfg), x, topk_idx, counts, offsets, row_of_slot,
                                   token_of_row, x_perm, n_dropped, static_cast<int32_t*>(ws),
                                   static_cast<cudaStream_t>(stream)));

@@ -12,44 +12,63 @@ namespace cs {
 // the always-on output is added).  One warp per token, fp32 accumulation in a
 // fixed order, 16-byte vectors, no atomics.
 // ---------------------------------------------------------------------------
-template <typename XT>
+template <typename XT, int K, int U>
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
                const float* __restrict__ topk_w, const uint4* __restrict__ shared_out,
                uint4* __restrict__ y, int64_t T, int k, int nvec) {
   constexpr int VN = Vec<XT>::N;
-  constexpr int KMAX = 16;
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t t = warp0; t < T; t += nwarps) {
     const int32_t mr = lane < k ? row_of_slot[t * k + lane] : -1;
     const float mw = lane < k ? topk_w[t * k + lane] : 0.f;
-    int32_t rows[KMAX];
-    float ws[KMAX];
+    // a dropped (or padding) slot reads a kept row of the same token with weight 0,
+    // so every load below is unconditional and can be issued together
+    const unsigned kept = __ballot_sync(0xffffffffu, mr >= 0);
+    const int32_t any_row = kept ? __shfl_sync(0xffffffffu, mr, __ffs(kept) - 1) : 0;
+    int32_t rows[K];
+    float ws[K];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      rows[j] = __shfl_sync(0xffffffffu, mr, j);
-      ws[j] = __shfl_sync(0xffffffffu, mw, j);
+    for (int j = 0; j < K; ++j) {
+      const int32_t r = __shfl_sync(0xffffffffu, mr, j);
+      const float wj = __shfl_sync(0xffffffffu, mw, j);
+      rows[j] = r >= 0 ? r : any_row;
+      ws[j] = r >= 0 ? wj : 0.f;
     }
-    for (int c = lane; c < nvec; c += 32) {
-      float acc[VN];
-      if (shared_out) {
-        unpack16(ldg_nc16(shared_out + t * nvec + c), acc, XT());
-      } else {
+    for (int c0 = lane; c0 < nvec; c0 += 32 * U) {
+      float acc[U][VN];
+      uint4 v[U][K];
 #pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = 0.f;
-      }
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < nvec && kept) {
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (j < k && rows[j] >= 0) {
-          float v[VN];
-          unpack16(ldg_nc16(y_perm + (int64_t)rows[j] * nvec + c), v, XT());
+          for (int j = 0; j < K; ++j) v[u][j] = ldg_nc16(y_perm + (int64_t)rows[j] * nvec + c);
+        }
+        if (c < nvec && shared_out) {
+          unpack16(ldg_nc16(shared_out + t * nvec + c), acc[u], XT());
+        } else {
 #pragma unroll
-          for (int i = 0; i < VN; ++i) acc[i] = fmaf(ws[j], v[i], acc[i]);
+          for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
         }
       }
-      y[t * nvec + c] = pack16(acc, XT());
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        if (c >= nvec) continue;
+        if (kept) {
+#pragma unroll
+          for (int j = 0; j < K; ++j) {
+            float f[VN];
+            unpack16(v[u][j], f, XT());
+#pragma unroll
+            for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(ws[j], f[i], acc[u][i]);
+          }
+        }
+        y[t * nvec + c] = pack16(acc[u], XT());
+      }
     }
   }
 }
@@ -157,6 +176,30 @@ bias_update_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias,
 }  // namespace cs
 
 
+template <typename XT>
+cudaError_t launch_combine_t(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
+                             const float* topk_w, const void* shared_out, void* y, int grid, int nvec,
+                             cudaStream_t s) {
+  auto yp = static_cast<const uint4*>(y_perm);
+  auto sh = static_cast<const uint4*>(shared_out);
+  auto yo = static_cast<uint4*>(y);
+#define MOE_COMBINE(KK, UU) \
+  cs::combine_kernel<XT, KK, UU><<<grid, 256, 0, s>>>(yp, row_of_slot, topk_w, sh, yo, c.T, c.top_k, nvec)
+  switch (c.top_k) {
+    case 1: MOE_COMBINE(1, 4); break;
+    case 2: MOE_COMBINE(2, 4); break;
+    case 3: MOE_COMBINE(3, 2); break;
+    case 4: MOE_COMBINE(4, 2); break;
+    case 5: MOE_COMBINE(5, 2); break;
+    case 6: MOE_COMBINE(6, 2); break;
+    case 7: MOE_COMBINE(7, 2); break;
+    case 8: MOE_COMBINE(8, 2); break;
+    default: MOE_COMBINE(16, 1); break;
+  }
+#undef MOE_COMBINE
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
                            const float* topk_w, const void* shared_out, void* y, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
@@ -166,14 +209,8 @@ cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int3
   const int64_t cap = (int64_t)sm_count() * 8;
   const int grid = (int)(want < cap ? want : cap);
   if (c.x_dtype == MOE_DTYPE_BF16)
-    cs::combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        static_cast<const uint4*>(y_perm), row_of_slot, topk_w,
-        static_cast<const uint4*>(shared_out), static_cast<uint4*>(y), c.T, c.top_k, nvec);
-  else
-    cs::combine_kernel<float><<<grid, 256, 0, s>>>(
-        static_cast<const uint4*>(y_perm), row_of_slot, topk_w,
-        static_cast<const uint4*>(shared_out), static_cast<uint4*>(y), c.T, c.top_k, nvec);
-  return cudaGetLastError();
+    return launch_combine_t<__nv_bfloat16>(c, y_perm, row_of_slot, topk_w, shared_out, y, grid, nvec, s);
+  return launch_combine_t<float>(c, y_perm, row_of_slot, topk_w, shared_out, y, grid, nvec, s);
 }
 
 cudaError_t launch_stats(const moe_config_t& c, const int32_t* counts, const int32_t* offsets,

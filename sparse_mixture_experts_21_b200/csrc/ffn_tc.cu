@@ -279,39 +279,6 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
   }
 }
 
-// ---------------------------------------------------------------------------
-// Host: tensor maps through the driver entry point (no libcuda link needed).
-// ---------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// Row-major bf16 matrix [rows, cols]; box = 64 columns x box_rows rows, 128 B swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int MODE>
 cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const int32_t* offsets, int G, int K, int n_out, int64_t rows_cap,
@@ -342,9 +309,9 @@ cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t*
   if (rows_cap == 0 || G == 0) return cudaSuccess;
   if (G > tc::kMaxGroups) return cudaErrorInvalidValue;
   CUtensorMap mx, m1, m3, mh, m2;
-  if (!tc::make_map(&mx, x_rows, rows_cap, d, tc::BM) || !tc::make_map(&m1, w1, (uint64_t)G * f, d, 128) ||
-      !tc::make_map(&m3, w3, (uint64_t)G * f, d, 128) || !tc::make_map(&mh, h, rows_cap, f, tc::BM) ||
-      !tc::make_map(&m2, w2, (uint64_t)G * d, f, 256))
+  if (!make_map_bf16(&mx, x_rows, rows_cap, d, tc::BM) || !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) ||
+      !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) || !make_map_bf16(&mh, h, rows_cap, f, tc::BM) ||
+      !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
     return cudaErrorInvalidValue;
   cudaError_t e = tc::launch_pass<0>(mx, m1, m3, offsets, G, d, f, rows_cap, h, s);
   if (e != cudaSuccess) return e;

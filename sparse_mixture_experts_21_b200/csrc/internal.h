@@ -1,6 +1,7 @@
 // Host-side launchers shared between the C-ABI layer and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -9,13 +10,19 @@
 
 namespace moe {
 
-// Padded expert count and tokens per block of the fused router kernel.
+// Row-major bf16 matrix [rows, cols] as a TMA tensor map: box = 64 columns x
+// box_rows rows, 128-byte swizzle, zero fill out of bounds.
+bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
+// Padded expert count, tokens per block and scratch of the fused router.
 int route_np(int n_experts);
-int route_tokens_per_block(int n_experts);
+bool route_uses_tc(const moe_config_t& c);
+int route_tokens_per_block(const moe_config_t& c);
+size_t route_workspace_bytes(const moe_config_t& c);
 
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* w_gate,
                          const float* logit_offset, const float* bias, int32_t* topk_idx,
-                         float* topk_w, float* lse, float* p_partial, float* margin,
+                         float* topk_w, float* lse, float* p_partial, float* margin, void* ws,
                          cudaStream_t s);
 
 // Token-order capacity drop and permutation.

@@ -1,5 +1,6 @@
 // Single translation unit of the library (one module, so every kernel file sees
 // the same device status word without relocatable device code).
+#include "tmap.cu"
 #include "capi.cu"
 #include "route.cu"
 #include "permute.cu"

@@ -1,5 +1,5 @@
-// Fused router: fp32 router GEMM -> affinity -> choice-only bias -> group limit
-// -> top-k (warp shuffles) -> renormalised weights, plus logsumexp and per-block
+// Fused router: router GEMM -> affinity -> choice-only bias -> group limit ->
+// top-k (warp shuffles) -> renormalised weights, plus logsumexp and per-block
 // sums of the normalised affinity for the load-balance statistics.
 //
 // Follows "路由的数学形式：softmax、top-k 与那些必须做的小动作" on the Practice page
@@ -9,10 +9,18 @@
 // pre-selection (the History page's part 四, node-limited routing, no formula
 // given): contiguous groups scored by the sum of their top-n selection scores.
 //
-// One CTA owns TM tokens and all N experts.  Phase 1 is a register-tiled fp32
-// SIMT GEMM (x widened from bf16 exactly) with an optional split of each d-chunk
-// across thread groups for small N; phase 2 gives each warp one token at a time,
-// lane l holding experts l, l+32, ...
+// Two GEMM front ends share one selection phase (one warp per token, lane l
+// holding experts l, l+32, ...):
+//  * tensor cores (bf16 x, N <= 256): the fp32 router weight is split exactly
+//    into three bf16 pieces W = W_hi + W_mid + W_lo (each piece keeps the next 8
+//    mantissa bits), so x W^T = sum over pieces of x W_p^T.  x is bf16, so every
+//    product is exact in fp32 and the MMA accumulates in fp32: fp32-equivalent
+//    logits from one tcgen05 GEMM with K = 3 d (bf16x3, Henry, Tang & Heinecke,
+//    "Leveraging the bfloat16 AI datatype for higher-precision computations",
+//    2019).  One CTA per 128 tokens; logits go TMEM -> shared memory.
+//  * fp32 FMA (fp32 x, or N > 256): register-tiled SIMT GEMM over d-chunks.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,142 +28,40 @@ namespace moe {
 
 namespace rt {
 
-constexpr int kRouteThreads = 256;
-constexpr int KC = 32;  // d-chunk staged in shared memory per iteration
-
-template <int NP, int TM, int RM, int RN, int KS>
-struct RouteShape {
-  static constexpr int NTX = NP / RN;            // thread columns (experts)
-  static constexpr int NTY = TM / RM;            // thread rows (tokens)
-  static_assert(NTX * NTY * KS == kRouteThreads, "thread layout");
-  static_assert(KC % KS == 0, "split must divide the chunk");
-  static constexpr int XS = TM + 4;              // padded smem strides (floats)
-  static constexpr int WS = NP + 4;
-  static constexpr int GEMM_FLOATS = KC * XS + KC * WS;
-  static constexpr int PART_FLOATS = KS * TM * NP;
-  static constexpr int NV = NP >= 32 ? NP / 32 : 1;   // experts per lane in phase 2
-  static constexpr int WARPS = kRouteThreads / 32;
-  static constexpr int SMEM_FLOATS =
-      (GEMM_FLOATS > PART_FLOATS ? GEMM_FLOATS : PART_FLOATS) + WARPS * NV * 32;
+struct RouteArgs {
+  const float* logit_offset;
+  const float* bias;
+  int64_t T;
+  int N, k, score_fn, renorm, n_groups, topk_groups, group_topn;
+  int32_t* topk_idx;
+  float* topk_w;
+  float* lse;
+  float* p_partial;
+  float* margin;
 };
 
-template <int N>
-__device__ __forceinline__ void lds_vec(const float* p, float* out) {
-  if constexpr (N % 4 == 0) {
-#pragma unroll
-    for (int i = 0; i < N; i += 4) {
-      float4 v = *reinterpret_cast<const float4*>(p + i);
-      out[i] = v.x; out[i + 1] = v.y; out[i + 2] = v.z; out[i + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < N; i += 2) {
-      float2 v = *reinterpret_cast<const float2*>(p + i);
-      out[i] = v.x; out[i + 1] = v.y;
-    }
-  }
-}
-
-template <int NP, int TM, int RM, int RN, int KS, typename XT>
-__global__ void __launch_bounds__(kRouteThreads)
-route_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate,
-             const float* __restrict__ logit_offset, const float* __restrict__ bias,
-             int64_t T, int d, int N, int k, int score_fn, int renorm, int n_groups,
-             int topk_groups, int group_topn, int32_t* __restrict__ topk_idx,
-             float* __restrict__ topk_w, float* __restrict__ lse_out,
-             float* __restrict__ p_partial, float* __restrict__ margin_out) {
-  using S = RouteShape<NP, TM, RM, RN, KS>;
-  extern __shared__ __align__(16) float smem[];
-  float* xs = smem;                  // [KC][XS]  x chunk, transposed
-  float* ws = smem + KC * S::XS;     // [KC][WS]  W_g chunk, transposed
-  float* part = smem;                // [KS][TM][NP] after the GEMM (aliases xs/ws)
-  float* pwarp = smem + (S::GEMM_FLOATS > S::PART_FLOATS ? S::GEMM_FLOATS : S::PART_FLOATS);
-
-  const int tid = threadIdx.x;
-  const int64_t t0 = (int64_t)blockIdx.x * TM;
-  const int split = tid / (S::NTX * S::NTY);
-  const int ty = (tid % (S::NTX * S::NTY)) / S::NTX;
-  const int tx = tid % S::NTX;
-
-  float acc[RM][RN];
-#pragma unroll
-  for (int i = 0; i < RM; ++i)
-#pragma unroll
-    for (int j = 0; j < RN; ++j) acc[i][j] = 0.f;
-
-  constexpr int XV = Vec<XT>::N;     // x elements per 16-byte vector
-  for (int k0 = 0; k0 < d; k0 += KC) {
-    // stage x[t0 : t0+TM, k0 : k0+KC] as fp32, transposed
-    for (int v = tid; v < TM * (KC / XV); v += kRouteThreads) {
-      const int r = v / (KC / XV), c = (v % (KC / XV)) * XV;
-      float vals[XV];
-      if (t0 + r < T && k0 + c < d) {
-        unpack16(ldg_nc16(x + (t0 + r) * (int64_t)d + k0 + c), vals, XT());
-      } else {
-#pragma unroll
-        for (int i = 0; i < XV; ++i) vals[i] = 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < XV; ++i) xs[(c + i) * S::XS + r] = vals[i];
-    }
-    // stage W_g[0 : NP, k0 : k0+KC], transposed
-    for (int v = tid; v < NP * (KC / 4); v += kRouteThreads) {
-      const int e = v / (KC / 4), c = (v % (KC / 4)) * 4;
-      float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < N && k0 + c < d) w4 = *reinterpret_cast<const float4*>(w_gate + (int64_t)e * d + k0 + c);
-      ws[(c + 0) * S::WS + e] = w4.x;
-      ws[(c + 1) * S::WS + e] = w4.y;
-      ws[(c + 2) * S::WS + e] = w4.z;
-      ws[(c + 3) * S::WS + e] = w4.w;
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int kk = split; kk < KC; kk += KS) {
-      float a[RM], b[RN];
-      lds_vec<RM>(xs + kk * S::XS + ty * RM, a);
-      lds_vec<RN>(ws + kk * S::WS + tx * RN, b);
-#pragma unroll
-      for (int i = 0; i < RM; ++i)
-#pragma unroll
-        for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-
-  // ---- reduce the d-splits in fixed order: logits[tm][e] in part[0]
-#pragma unroll
-  for (int i = 0; i < RM; ++i)
-#pragma unroll
-    for (int j = 0; j < RN; ++j) part[(split * TM + ty * RM + i) * NP + tx * RN + j] = acc[i][j];
-  __syncthreads();
-  if constexpr (KS > 1) {
-    for (int v = tid; v < TM * NP; v += kRouteThreads) {
-      float s = part[v];
-#pragma unroll
-      for (int q = 1; q < KS; ++q) s += part[q * TM * NP + v];
-      part[v] = s;
-    }
-    __syncthreads();
-  }
-
-  // ---- phase 2: one warp per token
-  const int warp = tid / 32, lane = tid % 32;
-  constexpr int NV = S::NV;
+// Selection phase: tokens t0 .. t0+TM-1 of the block, logits[tm * ld + e] in
+// shared memory.  Writes the per-token outputs and this block's row of p_partial.
+template <int NV, int WARPS>
+__device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, const RouteArgs& a,
+                             float* pwarp) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int N = a.N, k = a.k;
   float pacc[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) pacc[i] = 0.f;
-  const int gsz = n_groups > 1 ? N / n_groups : N;
+  const int gsz = a.n_groups > 1 ? N / a.n_groups : N;
 
-  for (int tm = warp; tm < TM; tm += S::WARPS) {
+  for (int tm = warp; tm < TM; tm += WARPS) {
     const int64_t t = t0 + tm;
-    if (t >= T) break;
+    if (t >= a.T) break;
     float z[NV], s[NV], q[NV];
     bool valid[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const int e = lane + 32 * i;
       valid[i] = e < N;
-      z[i] = valid[i] ? part[tm * NP + e] + (logit_offset ? logit_offset[e] : 0.f) : -INFINITY;
+      z[i] = valid[i] ? logits[tm * ld + e] + (a.logit_offset ? a.logit_offset[e] : 0.f) : -INFINITY;
     }
     // affinity and logsumexp
     float m = -INFINITY;
@@ -173,13 +79,13 @@ route_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate,
     float ssum = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      if (score_fn == MOE_SCORE_SOFTMAX) s[i] = valid[i] ? ex[i] / se : 0.f;
+      if (a.score_fn == MOE_SCORE_SOFTMAX) s[i] = valid[i] ? ex[i] / se : 0.f;
       else s[i] = valid[i] ? 1.f / (1.f + expf(-z[i])) : 0.f;
       ssum += s[i];
-      q[i] = valid[i] ? s[i] + (bias ? bias[lane + 32 * i] : 0.f) : -INFINITY;
+      q[i] = valid[i] ? s[i] + (a.bias ? a.bias[lane + 32 * i] : 0.f) : -INFINITY;
     }
     // load-balance statistics: normalised affinity (softmax probs or s / sum s)
-    if (score_fn == MOE_SCORE_SIGMOID) {
+    if (a.score_fn == MOE_SCORE_SIGMOID) {
       ssum = warp_sum(ssum);
 #pragma unroll
       for (int i = 0; i < NV; ++i) pacc[i] += s[i] / ssum;
@@ -191,12 +97,28 @@ route_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate,
     // group-limited pre-selection
     uint32_t group_keep = 0xffffffffu;
     float gmargin = INFINITY;
-    if (n_groups > 1) {
+    if (a.n_groups > 1) {
       float my_gscore = -INFINITY;
-      for (int g = 0; g < n_groups; ++g) {
+      if (gsz == 32 && a.group_topn <= 2) {
+        // each group is one register column: butterfly merge of (best, second) values
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          float b1 = q[i], b2 = -INFINITY;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float ob1 = __shfl_xor_sync(0xffffffffu, b1, o);
+            const float ob2 = __shfl_xor_sync(0xffffffffu, b2, o);
+            const float hi = fmaxf(b1, ob1), lo = fminf(b1, ob1);
+            b2 = fmaxf(lo, fmaxf(b2, ob2));
+            b1 = hi;
+          }
+          if (lane == i) my_gscore = a.group_topn == 1 ? b1 : b1 + b2;
+        }
+      } else
+      for (int g = 0; g < a.n_groups; ++g) {
         uint32_t taken = 0;
         float gs = 0.f;
-        for (int r = 0; r < group_topn; ++r) {
+        for (int r = 0; r < a.group_topn; ++r) {
           float v = -INFINITY;
           int bi = 0x7fffffff;
 #pragma unroll
@@ -214,11 +136,12 @@ route_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate,
       }
       uint32_t kept_mask = 0;
       float last = 0.f;
-      for (int r = 0; r <= topk_groups && r < n_groups; ++r) {
-        float v = (lane < n_groups && !((kept_mask >> lane) & 1u)) ? my_gscore : -INFINITY;
-        int gi = lane < n_groups && !((kept_mask >> lane) & 1u) ? lane : 0x7fffffff;
+      for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
+        const bool cand = lane < a.n_groups && !((kept_mask >> lane) & 1u);
+        float v = cand ? my_gscore : -INFINITY;
+        int gi = cand ? lane : 0x7fffffff;
         warp_argmax(v, gi);
-        if (r < topk_groups) {
+        if (r < a.topk_groups) {
           if (gi != 0x7fffffff) kept_mask |= 1u << gi;
           last = v;
         } else {
@@ -269,52 +192,376 @@ route_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate,
 
     const float wsum = warp_sum(lane < k ? my_s : 0.f);
     if (lane < k) {
-      topk_idx[t * k + lane] = my_idx;
-      topk_w[t * k + lane] = renorm ? my_s / wsum : my_s;
+      a.topk_idx[t * k + lane] = my_idx;
+      a.topk_w[t * k + lane] = a.renorm ? my_s / wsum : my_s;
     }
     if (lane == 0) {
-      lse_out[t] = lse;
-      if (margin_out) margin_out[t] = fminf(emargin, gmargin);
+      a.lse[t] = lse;
+      if (a.margin) a.margin[t] = fminf(emargin, gmargin);
     }
   }
 
-  // ---- per-block sums of the normalised affinity, fixed order over warps
+  // per-block sums of the normalised affinity, fixed order over warps
 #pragma unroll
   for (int i = 0; i < NV; ++i) pwarp[(warp * NV + i) * 32 + lane] = pacc[i];
   __syncthreads();
-  for (int e = tid; e < N; e += kRouteThreads) {
+  for (int e = threadIdx.x; e < N; e += WARPS * 32) {
     const int i = e / 32, l = e % 32;
     float sum = 0.f;
-    for (int w = 0; w < S::WARPS; ++w) sum += pwarp[(w * NV + i) * 32 + l];
-    p_partial[(int64_t)blockIdx.x * N + e] = sum;
+    for (int w = 0; w < WARPS; ++w) sum += pwarp[(w * NV + i) * 32 + l];
+    a.p_partial[(int64_t)blockIdx.x * N + e] = sum;
   }
 }
 
+// ============================================================================
+// fp32 FMA front end
+// ============================================================================
+constexpr int kRouteThreads = 256;
+constexpr int KC = 32;  // d-chunk staged in shared memory per iteration
+
 template <int NP, int TM, int RM, int RN, int KS>
-cudaError_t launch_shape(const moe_config_t& c, const void* x, const float* wg, const float* off,
-                         const float* bias, int32_t* idx, float* w, float* lse, float* pp,
-                         float* margin, cudaStream_t s) {
+struct RouteShape {
+  static constexpr int NTX = NP / RN;            // thread columns (experts)
+  static constexpr int NTY = TM / RM;            // thread rows (tokens)
+  static_assert(NTX * NTY * KS == kRouteThreads, "thread layout");
+  static_assert(KC % KS == 0, "split must divide the chunk");
+  static constexpr int XS = TM + 4;              // padded smem strides (floats)
+  static constexpr int WS = NP + 4;
+  static constexpr int GEMM_FLOATS = KC * XS + KC * WS;
+  static constexpr int PART_FLOATS = KS * TM * NP;
+  static constexpr int NV = NP >= 32 ? NP / 32 : 1;   // experts per lane in the selection phase
+  static constexpr int WARPS = kRouteThreads / 32;
+  static constexpr int SMEM_FLOATS =
+      (GEMM_FLOATS > PART_FLOATS ? GEMM_FLOATS : PART_FLOATS) + WARPS * NV * 32;
+};
+
+template <int N>
+__device__ __forceinline__ void lds_vec(const float* p, float* out) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      float4 v = *reinterpret_cast<const float4*>(p + i);
+      out[i] = v.x; out[i + 1] = v.y; out[i + 2] = v.z; out[i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; i += 2) {
+      float2 v = *reinterpret_cast<const float2*>(p + i);
+      out[i] = v.x; out[i + 1] = v.y;
+    }
+  }
+}
+
+template <int NP, int TM, int RM, int RN, int KS, typename XT>
+__global__ void __launch_bounds__(kRouteThreads)
+route_simt_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate, int d, RouteArgs a) {
+  using S = RouteShape<NP, TM, RM, RN, KS>;
+  extern __shared__ __align__(16) float smem[];
+  float* xs = smem;                  // [KC][XS]  x chunk, transposed
+  float* ws = smem + KC * S::XS;     // [KC][WS]  W_g chunk, transposed
+  float* part = smem;                // [KS][TM][NP] after the GEMM (aliases xs/ws)
+  float* pwarp = smem + (S::GEMM_FLOATS > S::PART_FLOATS ? S::GEMM_FLOATS : S::PART_FLOATS);
+
+  const int tid = threadIdx.x;
+  const int N = a.N;
+  const int64_t T = a.T;
+  const int64_t t0 = (int64_t)blockIdx.x * TM;
+  const int split = tid / (S::NTX * S::NTY);
+  const int ty = (tid % (S::NTX * S::NTY)) / S::NTX;
+  const int tx = tid % S::NTX;
+
+  float acc[RM][RN];
+#pragma unroll
+  for (int i = 0; i < RM; ++i)
+#pragma unroll
+    for (int j = 0; j < RN; ++j) acc[i][j] = 0.f;
+
+  constexpr int XV = Vec<XT>::N;     // x elements per 16-byte vector
+  for (int k0 = 0; k0 < d; k0 += KC) {
+    for (int v = tid; v < TM * (KC / XV); v += kRouteThreads) {
+      const int r = v / (KC / XV), c = (v % (KC / XV)) * XV;
+      float vals[XV];
+      if (t0 + r < T && k0 + c < d) {
+        unpack16(ldg_nc16(x + (t0 + r) * (int64_t)d + k0 + c), vals, XT());
+      } else {
+#pragma unroll
+        for (int i = 0; i < XV; ++i) vals[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < XV; ++i) xs[(c + i) * S::XS + r] = vals[i];
+    }
+    for (int v = tid; v < NP * (KC / 4); v += kRouteThreads) {
+      const int e = v / (KC / 4), c = (v % (KC / 4)) * 4;
+      float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < N && k0 + c < d) w4 = *reinterpret_cast<const float4*>(w_gate + (int64_t)e * d + k0 + c);
+      ws[(c + 0) * S::WS + e] = w4.x;
+      ws[(c + 1) * S::WS + e] = w4.y;
+      ws[(c + 2) * S::WS + e] = w4.z;
+      ws[(c + 3) * S::WS + e] = w4.w;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = split; kk < KC; kk += KS) {
+      float av[RM], bv[RN];
+      lds_vec<RM>(xs + kk * S::XS + ty * RM, av);
+      lds_vec<RN>(ws + kk * S::WS + tx * RN, bv);
+#pragma unroll
+      for (int i = 0; i < RM; ++i)
+#pragma unroll
+        for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+
+  // reduce the d-splits in fixed order: logits[tm][e] in part[0]
+#pragma unroll
+  for (int i = 0; i < RM; ++i)
+#pragma unroll
+    for (int j = 0; j < RN; ++j) part[(split * TM + ty * RM + i) * NP + tx * RN + j] = acc[i][j];
+  __syncthreads();
+  if constexpr (KS > 1) {
+    for (int v = tid; v < TM * NP; v += kRouteThreads) {
+      float s = part[v];
+#pragma unroll
+      for (int q = 1; q < KS; ++q) s += part[q * TM * NP + v];
+      part[v] = s;
+    }
+    __syncthreads();
+  }
+  select_phase<S::NV, S::WARPS>(part, NP, TM, t0, a, pwarp);
+}
+
+// ============================================================================
+// tensor-core (tcgen05) front end, bf16x3 split of the fp32 router weight
+// ============================================================================
+// The tensor cores' fp32 accumulation truncates, so one long accumulation over
+// K = 3 d would bias the logits towards zero (about 1e-5 relative at d = 4096).
+// Each 64-wide K block therefore starts a fresh TMEM accumulator, and drain warps
+// add the block result into fp32 registers with round-to-nearest: the truncation
+// then spans the 4 MMA steps of one block only.  K blocks run in the order
+// (d-tile, piece), so each x tile is fetched from DRAM once and reused from L2.
+constexpr int TC_TM = 128;          // tokens per CTA (MMA M)
+constexpr int TC_BK = 64;           // K per stage: one 128-byte swizzle row of bf16
+constexpr int TC_STAGES = 4;
+constexpr int TC_THREADS = 384;     // warp 0 TMA, warp 1 MMA, warps 4..11 drain; all 12 select
+constexpr int TC_WARPS = TC_THREADS / 32;
+
+template <int NP>
+struct TcRouteShape {
+  static constexpr int A_BYTES = TC_TM * TC_BK * 2;
+  static constexpr int B_BYTES = NP * TC_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int LD = NP + 1;                           // logits row stride (floats)
+  static constexpr int LOGIT_BYTES = TC_TM * LD * 4;
+  static constexpr int RING_BYTES = TC_STAGES * STAGE_BYTES;
+  static constexpr int MAIN_BYTES = RING_BYTES > LOGIT_BYTES ? RING_BYTES : LOGIT_BYTES;
+  static constexpr int NV = NP >= 32 ? NP / 32 : 1;
+  static constexpr int PWARP_BYTES = TC_WARPS * NV * 32 * 4;
+  static constexpr int ACC_COLS = NP < 32 ? 32 : NP;          // TMEM columns per accumulator
+  static constexpr int NBUF = 512 / ACC_COLS >= 4 ? 4 : 512 / ACC_COLS;
+  static constexpr int TMEM_COLS = NBUF * ACC_COLS;
+  static constexpr int DRAIN_WARPS = NP >= 32 ? 8 : 4;
+  static constexpr int CPW = NP >= 32 ? NP / 2 : NP;          // columns per drain warp
+  static constexpr size_t SMEM = 1024 + MAIN_BYTES + PWARP_BYTES + 256;
+};
+
+// Wsplit[e, p * dpad + c] = piece p of W_g[e, c] (zero past N rows / d columns).
+__global__ void __launch_bounds__(256)
+split_gate_kernel(const float* __restrict__ w_gate, int N, int d, int NP, int dpad,
+                  __nv_bfloat16* __restrict__ wsplit) {
+  const int64_t n = (int64_t)NP * dpad;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int e = (int)(i / dpad), c = (int)(i % dpad);
+    const float w = (e < N && c < d) ? w_gate[(int64_t)e * d + c] : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    __nv_bfloat16* row = wsplit + (int64_t)e * 3 * dpad;
+    row[c] = hi;
+    row[dpad + c] = mid;
+    row[2 * dpad + c] = lo;
+  }
+}
+
+template <int NP>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                int d, int dpad, RouteArgs a) {
+  using S = TcRouteShape<NP>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  float* logits = reinterpret_cast<float*>(smem);             // after the main loop
+  float* pwarp = reinterpret_cast<float*>(smem + S::MAIN_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::MAIN_BYTES + S::PWARP_BYTES);
+  uint64_t* full = bars;                            // [TC_STAGES]
+  uint64_t* empty = bars + TC_STAGES;               // [TC_STAGES]
+  uint64_t* tfull = bars + 2 * TC_STAGES;           // [NBUF]
+  uint64_t* tempty = tfull + S::NBUF;               // [NBUF]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + S::NBUF);
+  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t0 = (int64_t)blockIdx.x * TC_TM;
+  const int nkb = 3 * (dpad / TC_BK);
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < S::NBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], S::DRAIN_WARPS); }
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto bounded_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long c0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+      if (*abort_flag) return false;
+      if (clock64() - c0 > kWaitLimitCycles) { flag_timeout(); *abort_flag = 1; return false; }
+    }
+    return true;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!bounded_wait(&empty[stage], phase ^ 1u)) { ok = false; break; }
+        const int kt = kb / 3, piece = kb - 3 * kt;
+        uint8_t* sa = smem + (size_t)stage * S::STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
+        tma_load_2d(&tmX, sa, &full[stage], kt * TC_BK, (int32_t)t0);
+        tma_load_2d(&tmW, sa + S::A_BYTES, &full[stage], piece * dpad + kt * TC_BK, 0);
+        ++issued;
+        if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) {
+        for (int i = 1; i <= min(issued, TC_STAGES); ++i) {
+          const int s = ((int)stage - i + 2 * TC_STAGES) % TC_STAGES;
+          mbar_wait(&full[s], ((int)stage - i < 0) ? (phase ^ 1u) : phase);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(TC_TM, NP < 16 ? 16 : NP);
+      uint32_t stage = 0, phase = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int buf = kb % S::NBUF;
+        const uint32_t use = (uint32_t)(kb / S::NBUF) & 1u;
+        if (!bounded_wait(&tempty[buf], use ^ 1u)) break;
+        if (!bounded_wait(&full[stage], phase)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + (size_t)stage * S::STAGE_BYTES);
+        const uint32_t b_addr = a_addr + S::A_BYTES;
+        const uint32_t d_tmem = tmem_base + buf * S::ACC_COLS;
+#pragma unroll
+        for (int kk = 0; kk < TC_BK / 16; ++kk)
+          umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
+                   idesc, kk != 0 ? 1u : 0u);
+        umma_commit(&empty[stage]);
+        umma_commit(&tfull[buf]);
+        if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp >= 4 && warp < 4 + S::DRAIN_WARPS) {
+    // drain: TMEM lanes 32 (warp % 4) .. +31, columns [c0, c0 + CPW)
+    const int q = warp & 3;
+    const int c0 = ((warp - 4) / 4) * S::CPW;
+    float acc[S::CPW];
+#pragma unroll
+    for (int i = 0; i < S::CPW; ++i) acc[i] = 0.f;
+    bool ok = true;
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int buf = kb % S::NBUF;
+      const uint32_t use = (uint32_t)(kb / S::NBUF) & 1u;
+      ok = bounded_wait(&tfull[buf], use);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + buf * S::ACC_COLS + c0;
+#pragma unroll
+      for (int c = 0; c < S::CPW; c += 16) {
+        uint32_t v[16];
+        tmem_ld16(taddr + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[c + i] += __uint_as_float(v[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+    if (ok) {
+      const int r = q * 32 + lane;
+#pragma unroll
+      for (int i = 0; i < S::CPW; ++i) logits[r * S::LD + c0 + i] = acc[i];
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+  if (*abort_flag) return;
+  select_phase<S::NV, TC_WARPS>(logits, S::LD, TC_TM, t0, a, pwarp);
+}
+
+template <int NP, int TM, int RM, int RN, int KS>
+cudaError_t launch_simt(const moe_config_t& c, const void* x, const float* wg, const RouteArgs& a,
+                        cudaStream_t s) {
   using S = RouteShape<NP, TM, RM, RN, KS>;
   const size_t smem = S::SMEM_FLOATS * sizeof(float);
   const unsigned grid = (unsigned)((c.T + TM - 1) / TM);
   if (c.x_dtype == MOE_DTYPE_BF16) {
-    auto kern = route_kernel<NP, TM, RM, RN, KS, __nv_bfloat16>;
+    auto kern = route_simt_kernel<NP, TM, RM, RN, KS, __nv_bfloat16>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, kRouteThreads, smem, s>>>(
-        static_cast<const __nv_bfloat16*>(x), wg, off, bias, c.T, c.d_model, c.n_experts, c.top_k,
-        c.score_fn, c.renorm, c.n_groups, c.topk_groups, c.group_score_topn, idx, w, lse, pp, margin);
+    kern<<<grid, kRouteThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(x), wg, c.d_model, a);
   } else {
-    auto kern = route_kernel<NP, TM, RM, RN, KS, float>;
+    auto kern = route_simt_kernel<NP, TM, RM, RN, KS, float>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    kern<<<grid, kRouteThreads, smem, s>>>(
-        static_cast<const float*>(x), wg, off, bias, c.T, c.d_model, c.n_experts, c.top_k,
-        c.score_fn, c.renorm, c.n_groups, c.topk_groups, c.group_score_topn, idx, w, lse, pp, margin);
+    kern<<<grid, kRouteThreads, smem, s>>>(static_cast<const float*>(x), wg, c.d_model, a);
   }
   return cudaGetLastError();
 }
 
-}  // namespace rt
+template <int NP>
+cudaError_t launch_tc(const moe_config_t& c, const void* x, const float* wg, const RouteArgs& a,
+                      void* ws, cudaStream_t s) {
+  using S = TcRouteShape<NP>;
+  const int d = c.d_model;
+  const int dpad = (d + TC_BK - 1) / TC_BK * TC_BK;
+  __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(ws);
+  const int64_t n = (int64_t)NP * dpad;
+  const int sgrid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  split_gate_kernel<<<sgrid, 256, 0, s>>>(wg, c.n_experts, d, NP, dpad, wsplit);
+  CUtensorMap mx, mw;
+  if (!make_map_bf16(&mx, x, (uint64_t)c.T, (uint64_t)d, TC_TM) ||
+      !make_map_bf16(&mw, wsplit, (uint64_t)NP, (uint64_t)3 * dpad, NP))
+    return cudaErrorInvalidValue;
+  auto kern = route_tc_kernel<NP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)((c.T + TC_TM - 1) / TC_TM);
+  kern<<<grid, TC_THREADS, S::SMEM, s>>>(mx, mw, d, dpad, a);
+  return cudaGetLastError();
+}
 
+}  // namespace rt
 
 int route_np(int n) {
   int np = 8;
@@ -322,25 +569,63 @@ int route_np(int n) {
   return np;
 }
 
-int route_tokens_per_block(int n) {
-  switch (route_np(n)) {
+bool route_uses_tc(const moe_config_t& c) {
+  return c.x_dtype == MOE_DTYPE_BF16 && c.n_experts <= 256;
+}
+
+int route_tokens_per_block(const moe_config_t& c) {
+  if (route_uses_tc(c)) return rt::TC_TM;
+  switch (route_np(c.n_experts)) {
     case 8: case 16: case 32: case 512: return 32;
     default: return 64;
   }
 }
 
+size_t route_workspace_bytes(const moe_config_t& c) {
+  if (!route_uses_tc(c)) return 0;
+  const int np = route_np(c.n_experts) < 16 ? 16 : route_np(c.n_experts);
+  const size_t dpad = (size_t)(c.d_model + rt::TC_BK - 1) / rt::TC_BK * rt::TC_BK;
+  return (size_t)np * 3 * dpad * 2;
+}
+
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* wg, const float* off,
                          const float* bias, int32_t* idx, float* w, float* lse, float* pp,
-                         float* margin, cudaStream_t s) {
+                         float* margin, void* ws, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
+  rt::RouteArgs a;
+  a.logit_offset = off;
+  a.bias = bias;
+  a.T = c.T;
+  a.N = c.n_experts;
+  a.k = c.top_k;
+  a.score_fn = c.score_fn;
+  a.renorm = c.renorm;
+  a.n_groups = c.n_groups;
+  a.topk_groups = c.topk_groups;
+  a.group_topn = c.group_score_topn;
+  a.topk_idx = idx;
+  a.topk_w = w;
+  a.lse = lse;
+  a.p_partial = pp;
+  a.margin = margin;
+  if (route_uses_tc(c)) {
+    switch (route_np(c.n_experts)) {
+      case 8: case 16: return rt::launch_tc<16>(c, x, wg, a, ws, s);
+      case 32:  return rt::launch_tc<32>(c, x, wg, a, ws, s);
+      case 64:  return rt::launch_tc<64>(c, x, wg, a, ws, s);
+      case 128: return rt::launch_tc<128>(c, x, wg, a, ws, s);
+      case 256: return rt::launch_tc<256>(c, x, wg, a, ws, s);
+      default:  return cudaErrorInvalidValue;
+    }
+  }
   switch (route_np(c.n_experts)) {
-    case 8:   return rt::launch_shape<8, 32, 2, 8, 16>(c, x, wg, off, bias, idx, w, lse, pp, margin, s);
-    case 16:  return rt::launch_shape<16, 32, 2, 8, 8>(c, x, wg, off, bias, idx, w, lse, pp, margin, s);
-    case 32:  return rt::launch_shape<32, 32, 4, 8, 8>(c, x, wg, off, bias, idx, w, lse, pp, margin, s);
-    case 64:  return rt::launch_shape<64, 64, 4, 8, 2>(c, x, wg, off, bias, idx, w, lse, pp, margin, s);
-    case 128: return rt::launch_shape<128, 64, 8, 8, 2>(c, x, wg, off, bias, idx, w, lse, pp, margin, s);
-    case 256: return rt::launch_shape<256, 64, 8, 8, 1>(c, x, wg, off, bias, idx, w, lse, pp, margin, s);
-    case 512: return rt::launch_shape<512, 32, 4, 16, 1>(c, x, wg, off, bias, idx, w, lse, pp, margin, s);
+    case 8:   return rt::launch_simt<8, 32, 2, 8, 16>(c, x, wg, a, s);
+    case 16:  return rt::launch_simt<16, 32, 2, 8, 8>(c, x, wg, a, s);
+    case 32:  return rt::launch_simt<32, 32, 4, 8, 8>(c, x, wg, a, s);
+    case 64:  return rt::launch_simt<64, 64, 4, 8, 2>(c, x, wg, a, s);
+    case 128: return rt::launch_simt<128, 64, 8, 8, 2>(c, x, wg, a, s);
+    case 256: return rt::launch_simt<256, 64, 8, 8, 1>(c, x, wg, a, s);
+    case 512: return rt::launch_simt<512, 32, 4, 16, 1>(c, x, wg, a, s);
     default:  return cudaErrorInvalidValue;
   }
 }

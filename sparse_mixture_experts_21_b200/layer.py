@@ -71,7 +71,7 @@ class MoELayer:
     def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         W, c, T = self.weights, self.cfg, self.w.T
         L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), self.topk_idx,
-                    self.topk_w, self.lse, self.p_partial, self.margin, stream)
+                    self.topk_w, self.lse, self.p_partial, self.margin, self.ws, stream)
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
                       self.token_of_row, self.x_perm, self.n_dropped, self.ws, stream)
         L.moe_grouped_ffn(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
@@ -92,6 +92,8 @@ class MoELayer:
     def kernel_launches(self) -> int:
         """Number of the library's kernels one forward launches."""
         n = 1 + 4 + 2 + 1 + 1          # route, permute (4), routed FFN (2), combine, stats
+        if self.w.dtype == "bf16" and self.w.N <= 256:
+            n += 1                     # exact bf16 split of the router weight
         if self.fs > 0:
             n += 2
         if self.update_bias:

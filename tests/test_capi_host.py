@@ -40,9 +40,15 @@ def test_config_struct_layout():
 def test_sizing_queries(lib, name):
     w = synth.WORKLOADS[name]
     c = layer.make_config(w)
-    tm = 32 if w.N <= 32 or w.N > 256 else 64
+    if w.dtype == "bf16" and w.N <= 256:          # tensor-core router: 128 tokens per block
+        tm = 128
+        np_ = max(16, 1 << (w.N - 1).bit_length())
+        route_ws = np_ * 3 * (-(-w.d // 64) * 64) * 2
+    else:
+        tm = 32 if w.N <= 32 or w.N > 256 else 64
+        route_ws = 0
     assert L.route_partials(c) == (w.T + tm - 1) // tm
-    assert L.workspace_size(c) == ((w.T + 255) // 256) * w.N * 4
+    assert L.workspace_size(c) == max(((w.T + 255) // 256) * w.N * 4, route_ws)
     cap = L.capacity(c)
     if w.capacity == "dropless":
         assert cap == 2 ** 63 - 1
@@ -92,10 +98,11 @@ def test_null_and_misaligned_pointers_rejected(lib):
     c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
     cp = ctypes.byref(c)
     # null required pointers: rejected on the host, nothing launched
-    assert lib.moe_route(cp, None, None, None, None, None, None, None, None, None, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(cp, None, None, None, None, None, None, None, None, None, None, 0, None) == \
+        L.MOE_ERR_INVALID_ARG
     bad = 0x1000008  # not 16-byte aligned
     ok = 0x1000000
-    assert lib.moe_route(cp, bad, ok, None, None, ok, ok, ok, ok, None, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(cp, bad, ok, None, None, ok, ok, ok, ok, None, None, 0, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_combine(cp, ok, ok, ok, None, bad, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_grouped_ffn(cp, ok, 10, ok, 0, ok, ok, ok, 256, ok, ok, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_grouped_ffn(cp, ok, 10, ok, 1, ok, ok, ok, 12, ok, ok, None) == L.MOE_ERR_INVALID_ARG
@@ -109,11 +116,15 @@ def test_workspace_too_small_rejected(lib):
     ok = 0x1000000
     st = lib.moe_permute(ctypes.byref(c), ok, ok, ok, ok, ok, ok, ok, ok, ok, 4, None)
     assert st == L.MOE_ERR_WORKSPACE_TOO_SMALL
+    c3 = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    st = lib.moe_route(ctypes.byref(c3), ok, ok, None, None, ok, ok, ok, ok, None, ok, 1024, None)
+    assert st == L.MOE_ERR_WORKSPACE_TOO_SMALL
 
 
 def test_empty_batch_is_a_no_op(lib):
     c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"], T=0)
-    assert lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, None, None) == L.MOE_OK
+    assert lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, None, None, 0,
+                         None) == L.MOE_OK
     assert lib.moe_combine(ctypes.byref(c), None, None, None, None, None, None) == L.MOE_OK
     assert lib.moe_grouped_ffn(ctypes.byref(c), None, 0, 0x1000000, 1, None, None, None, 256, None, None,
                                None) == L.MOE_OK
