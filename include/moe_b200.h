@@ -230,6 +230,30 @@ int moe_bias_update(const moe_config_t* cfg, const int32_t* counts, float* bias,
                     float rate, float clamp, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_permute_noalloc -- moe_permute for callers that cannot allocate.
+ *
+ * The source pages have no counterpart to this call; it exists for deployment.
+ * Some callers cannot allocate device memory: a plugin inside a host
+ * application whose memory pool already owns the device, or a runtime with a
+ * static memory plan.  This variant computes exactly what moe_permute computes
+ * (same outputs, bit for bit) but keeps its per-block count table in a 1 MiB
+ * device array inside the library instead of a caller-provided workspace, and
+ * calls no allocator.
+ *   Arguments: as moe_permute, without ws / ws_bytes.
+ *   Limit: ceil(T / 256) * N <= 262144 (e.g. N = 256 up to T = 262144 tokens);
+ *          larger calls return MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   Every GPU that loads the library holds the array until the process exits.
+ *   All calls share the array: calls that overlap on the GPU race, so the
+ *   caller must order them (one stream, or explicit events).  Each call
+ *   rewrites the table before reading it.
+ * ------------------------------------------------------------------------- */
+int moe_permute_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                        int32_t* counts, int32_t* offsets, int32_t* row_of_slot,
+                        int32_t* token_of_row, void* x_perm, int32_t* n_dropped, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Diagnostics.
  * ------------------------------------------------------------------------- */
 

@@ -25,7 +25,7 @@ CAP_DROPLESS, CAP_CEIL_CF_T_OVER_N, CAP_CF_K_T_OVER_N_FLOOR = 0, 1, 2
 
 EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_route", "moe_permute",
             "moe_grouped_ffn", "moe_combine", "moe_router_stats", "moe_bias_update",
-            "moe_device_status", "moe_status_string")
+            "moe_device_status", "moe_status_string", "moe_permute_noalloc")
 
 
 class MoeConfig(ctypes.Structure):
@@ -74,6 +74,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_workspace_size": [cfgp, POINTER(c_size_t)],
         "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
         "moe_permute": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
+        "moe_permute_noalloc": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "moe_grouped_ffn": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp],
         "moe_combine": [cfgp, vp, vp, vp, vp, vp, vp],
         "moe_router_stats": [cfgp, vp, vp, vp, vp, vp, vp, c_float, c_float, vp, vp, vp, vp],
@@ -143,6 +144,14 @@ def moe_permute(cfg, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_
     _check("moe_permute", load().moe_permute(
         ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(row_of_slot),
         _ptr(token_of_row), _ptr(x_perm), _ptr(n_dropped), _ptr(ws), nbytes, _stream(stream)))
+
+
+def moe_permute_noalloc(cfg, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm,
+                        n_dropped, stream=None):
+    """moe_permute without a workspace (scratch kept inside the library)."""
+    _check("moe_permute_noalloc", load().moe_permute_noalloc(
+        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(row_of_slot),
+        _ptr(token_of_row), _ptr(x_perm), _ptr(n_dropped), _stream(stream)))
 
 
 def moe_grouped_ffn(cfg, x_rows, rows_cap, offsets, G, w1, w3, w2, f, h_scratch, y_rows, stream=None):

@@ -4,6 +4,7 @@
 #include "capi.cu"
 #include "route.cu"
 #include "permute.cu"
+#include "permute_noalloc.cu"
 #include "ffn_tc.cu"
 #include "ffn_f32.cu"
 #include "combine_stats.cu"
