@@ -37,7 +37,7 @@ UNIT = "tokens/s"
 
 # DRAM traffic of the dominant kernels per launch from an ncu capture, valid only
 # while the kernel source is the one that was profiled (sha1 of ffn_tc.cu).
-NCU_TRAFFIC = {"ffn_tc_sha1": None, "bytes_per_ffn_call": None}
+NCU_TRAFFIC = {"ffn_tc_sha1": "ee33c3465d5e2301f23ac7cb5772a3feff814396", "bytes_per_ffn_call": 28.6e9}
 
 
 def _peaks():
@@ -232,7 +232,7 @@ def main():
         from dataclasses import replace
         w = replace(w, name=WORKLOAD + "_reduced", T=args.tokens or w.T, N=args.experts or w.N)
     inp = make_inputs(w, dev, seed=rank)
-    lay = MoELayer(w, inp, dev)
+    lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD)
     x = inp["x"]
     stream = torch.cuda.current_stream(dev)
 
@@ -245,44 +245,22 @@ def main():
         lay.forward(x)
     barrier()
 
-    # timed region: K whole-layer steps, events between the calls for per-stage times
+    # timed region: K whole-layer steps, events between the stages for per-stage times
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
     marks = [[ev() for _ in range(7)] for _ in range(args.steps)]
-    W = lay.weights
-    c = lay.cfg
     with ClockSampler(_device_uuid(local)) as clk:
         barrier()
         start, end = ev(), ev()
         start.record(stream)
         for i in range(args.steps):
-            m = marks[i]
-            m[0].record(stream)
-            L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), lay.topk_idx, lay.topk_w,
-                        lay.lse, lay.p_partial, lay.margin, lay.ws)
-            m[1].record(stream)
-            L.moe_permute(c, x, lay.topk_idx, lay.counts, lay.offsets, lay.row_of_slot, lay.token_of_row,
-                          lay.x_perm, lay.n_dropped, lay.ws)
-            m[2].record(stream)
-            L.moe_grouped_ffn(c, lay.x_perm, w.T * w.k, lay.offsets, w.N, W["w1"], W["w3"], W["w2"], w.f,
-                              lay.h, lay.y_perm)
-            m[3].record(stream)
-            L.moe_grouped_ffn(c, x, w.T, lay.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], lay.fs,
-                              lay.hs, lay.ys)
-            m[4].record(stream)
-            L.moe_combine(c, lay.y_perm, lay.row_of_slot, lay.topk_w, lay.ys, lay.y)
-            m[5].record(stream)
-            L.moe_router_stats(c, lay.counts, lay.offsets, lay.p_partial, lay.lse, lay.n_dropped,
-                               W.get("bias"), w.alpha, w.z_coef, lay.stats, lay.f_out, lay.p_out)
-            L.moe_bias_update(c, lay.counts, W["bias"], w.bias_rate, 0.0)
-            m[6].record(stream)
+            lay.forward(x, stream, marks[i])
         end.record(stream)
         barrier()
     ms_local = start.elapsed_time(end) / args.steps
     ms = ms_local
     if pg is not None:
-        t = torch.tensor([ms_local], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+        from sparse_mixture_experts_21_b200.replicas import max_over_ranks
+        ms = max_over_ranks(ms_local, dev)
     assert L.moe_device_status() == L.MOE_OK
 
     stage = lambda a, b: statistics.mean(marks[i][a].elapsed_time(marks[i][b]) for i in range(args.steps))  # noqa: E731
@@ -324,9 +302,8 @@ def main():
         barrier()
         e2e_ms = s0.elapsed_time(s1) / args.steps
         if pg is not None:
-            t = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+            from sparse_mixture_experts_21_b200.replicas import max_over_ranks
+            e2e_ms = max_over_ranks(e2e_ms, dev)
         e2e = {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": xh.numel() * xh.element_size(),
                "d2h_bytes_per_step": yh.numel() * yh.element_size(), "ms_per_step": e2e_ms}

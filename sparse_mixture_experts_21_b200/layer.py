@@ -33,8 +33,13 @@ def make_config(w: Workload, T: Optional[int] = None) -> L.MoeConfig:
 class MoELayer:
     """Holds the weights and the per-call buffers of one layer for up to T tokens."""
 
-    def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True):
+    def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True,
+                 group=None):
+        """group: a torch.distributed process group when the layer runs as one of
+        several data-parallel replicas; the bias update then uses the counts summed
+        over the group, so all replicas keep the same selection bias."""
         self.w = w
+        self.group = group
         self.dev = torch.device(device)
         self.weights = weights
         self.update_bias = update_bias and weights.get("bias") is not None
@@ -64,29 +69,46 @@ class MoELayer:
             self.ys = z(max(T, 1), d, dtype=dt)
         self.y = z(max(T, 1), d, dtype=dt)
         self.stats = torch.zeros(L.STATS_BYTES, dtype=torch.uint8, device=self.dev)
+        self.counts_global = z(N, dtype=torch.int32)
         self.f_out = z(N)
         self.p_out = z(N)
 
-    # the launches of one layer forward; `x` is [T, d] on the device
-    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+    # the launches of one layer forward; `x` is [T, d] on the device.  `marks`, if
+    # given, is a list of 7 CUDA events recorded between the stages (route, permute,
+    # routed FFN, shared FFN, combine, statistics + bias update).
+    def forward(self, x: torch.Tensor, stream=None, marks=None) -> torch.Tensor:
         W, c, T = self.weights, self.cfg, self.w.T
+        s = stream if stream is not None else torch.cuda.current_stream(self.dev)
+        rec = (lambda i: marks[i].record(s)) if marks is not None else (lambda i: None)
+        rec(0)
         L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), self.topk_idx,
-                    self.topk_w, self.lse, self.p_partial, self.margin, self.ws, stream)
+                    self.topk_w, self.lse, self.p_partial, self.margin, self.ws, s)
+        rec(1)
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
-                      self.token_of_row, self.x_perm, self.n_dropped, self.ws, stream)
+                      self.token_of_row, self.x_perm, self.n_dropped, self.ws, s)
+        rec(2)
         L.moe_grouped_ffn(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
-                          W["w2"], self.w.f, self.h, self.y_perm, stream)
+                          W["w2"], self.w.f, self.h, self.y_perm, s)
+        rec(3)
         shared = None
         if self.fs > 0:
             L.moe_grouped_ffn(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], self.fs,
-                              self.hs, self.ys, stream)
+                              self.hs, self.ys, s)
             shared = self.ys
-        L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, self.y, stream)
+        rec(4)
+        L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, self.y, s)
+        rec(5)
         L.moe_router_stats(c, self.counts, self.offsets, self.p_partial, self.lse, self.n_dropped,
                            W.get("bias"), self.w.alpha, self.w.z_coef, self.stats, self.f_out,
-                           self.p_out, stream)
+                           self.p_out, s)
         if self.update_bias:
-            L.moe_bias_update(c, self.counts, W["bias"], self.w.bias_rate, 0.0, stream)
+            counts = self.counts
+            if self.group is not None:
+                from .replicas import all_reduce_counts
+                with torch.cuda.stream(s):
+                    counts = all_reduce_counts(self.counts, self.counts_global, self.group)
+            L.moe_bias_update(c, counts, W["bias"], self.w.bias_rate, 0.0, s)
+        rec(6)
         return self.y
 
     def kernel_launches(self) -> int:

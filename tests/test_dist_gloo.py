@@ -1,0 +1,59 @@
+"""Multi-rank host logic of the replica mode, on CPU with two gloo ranks.
+
+Each rank routes its own tokens; the per-expert counts are summed over ranks
+before the bias update, so every replica applies the same update, equal to the
+update a single process would apply to the concatenated batch.  The step time
+reported is the maximum over ranks.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from oracle import moe_oracle as O
+from sparse_mixture_experts_21_b200.replicas import all_reduce_counts, max_over_ranks
+from sparse_mixture_experts_21_b200.synth import random_routing
+
+N, K, T_PER_RANK, WORLD = 32, 4, 300, 2
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    try:
+        idx = random_routing(T_PER_RANK, N, K, "cpu", seed=100 + rank, hot=rank)
+        counts = torch.bincount(idx.reshape(-1).long(), minlength=N).to(torch.int32)
+        glob = torch.empty_like(counts)
+        all_reduce_counts(counts, glob)
+        bias = O.bias_update(np.zeros(N), glob.numpy(), rate=1e-3)
+        worst = max_over_ranks(1.5 + rank, "cpu")
+        np.savez(os.path.join(out_dir, f"r{rank}.npz"), idx=idx.numpy(), counts=counts.numpy(),
+                 glob=glob.numpy(), bias=bias, worst=worst)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replicas_share_counts_and_bias(tmp_path):
+    mp.start_processes(_worker, args=(_free_port(), str(tmp_path)), nprocs=WORLD, join=True,
+                       start_method="spawn")
+    r = [np.load(tmp_path / f"r{i}.npz") for i in range(WORLD)]
+    all_idx = np.concatenate([x["idx"] for x in r])
+    want = np.bincount(all_idx.reshape(-1), minlength=N)
+    for x in r:
+        assert np.array_equal(x["glob"], want)              # global counts on every rank
+        assert float(x["worst"]) == 2.5                     # max over ranks
+    assert not np.array_equal(r[0]["counts"], r[1]["counts"])
+    assert np.array_equal(r[0]["bias"], r[1]["bias"])       # replicas stay identical
+    single = O.bias_update(np.zeros(N), want, rate=1e-3)
+    assert np.array_equal(r[0]["bias"], single)             # same as one process on all tokens
