@@ -76,8 +76,9 @@ class MoELayer:
     # the launches of one layer forward; `x` is [T, d] on the device.  `marks`, if
     # given, is a list of 7 CUDA events recorded between the stages (route, permute,
     # routed FFN, shared FFN, combine, statistics + bias update).
-    def forward(self, x: torch.Tensor, stream=None, marks=None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, stream=None, marks=None, out=None) -> torch.Tensor:
         W, c, T = self.weights, self.cfg, self.w.T
+        y = self.y if out is None else out
         s = stream if stream is not None else torch.cuda.current_stream(self.dev)
         rec = (lambda i: marks[i].record(s)) if marks is not None else (lambda i: None)
         rec(0)
@@ -96,7 +97,7 @@ class MoELayer:
                               self.hs, self.ys, s)
             shared = self.ys
         rec(4)
-        L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, self.y, s)
+        L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, y, s)
         rec(5)
         L.moe_router_stats(c, self.counts, self.offsets, self.p_partial, self.lse, self.n_dropped,
                            W.get("bias"), self.w.alpha, self.w.z_coef, self.stats, self.f_out,
@@ -109,7 +110,49 @@ class MoELayer:
                     counts = all_reduce_counts(self.counts, self.counts_global, self.group)
             L.moe_bias_update(c, counts, W["bias"], self.w.bias_rate, 0.0, s)
         rec(6)
-        return self.y
+        return y
+
+    def forward_host(self, x_host_steps, y_host_steps, stream=None):
+        """Layer forwards on host data: for each step, copy its [T, d] input from
+        pinned host memory, run the layer, copy the result back into the matching
+        pinned host output.  Uploads, compute and downloads run on three streams
+        with two device input/output buffers, so step i+1's upload and step i-1's
+        download overlap step i's compute; every step still moves its own input
+        and result.  Returns after enqueueing; synchronise before reading outputs."""
+        comp = stream if stream is not None else torch.cuda.current_stream(self.dev)
+        if not hasattr(self, "_pipe"):
+            T, d = self.w.T, self.w.d
+            dt = self.y.dtype
+            self._pipe = {
+                "x": [torch.empty(max(T, 1), d, dtype=dt, device=self.dev) for _ in range(2)],
+                "y": [torch.empty(max(T, 1), d, dtype=dt, device=self.dev) for _ in range(2)],
+                "up": torch.cuda.Stream(self.dev), "down": torch.cuda.Stream(self.dev),
+                "x_ready": [torch.cuda.Event() for _ in range(2)],
+                "x_free": [torch.cuda.Event() for _ in range(2)],
+                "y_ready": [torch.cuda.Event() for _ in range(2)],
+                "y_free": [torch.cuda.Event() for _ in range(2)],
+            }
+        P = self._pipe
+        up, down = P["up"], P["down"]
+        # the first uploads must not overtake work already queued on the compute stream
+        up.wait_stream(comp)
+        down.wait_stream(comp)
+        for i, (xh, yh) in enumerate(zip(x_host_steps, y_host_steps)):
+            b = i % 2
+            up.wait_event(P["x_free"][b])
+            with torch.cuda.stream(up):
+                P["x"][b].copy_(xh, non_blocking=True)
+                P["x_ready"][b].record(up)
+            comp.wait_event(P["x_ready"][b])
+            comp.wait_event(P["y_free"][b])
+            self.forward(P["x"][b], comp, out=P["y"][b])
+            P["x_free"][b].record(comp)
+            P["y_ready"][b].record(comp)
+            down.wait_event(P["y_ready"][b])
+            with torch.cuda.stream(down):
+                yh.copy_(P["y"][b][: yh.shape[0]], non_blocking=True)
+                P["y_free"][b].record(down)
+        comp.wait_stream(down)
 
     def kernel_launches(self) -> int:
         """Number of the library's kernels one forward launches."""
