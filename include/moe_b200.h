@@ -69,6 +69,8 @@ typedef struct moe_config {
   int32_t group_score_topn;  /* group score = sum of its topn best scores, >= 1     */
   int32_t capacity_mode;     /* MOE_CAP_*                                           */
   int32_t x_dtype;           /* MOE_DTYPE_*: x, expert weights, h, y all this type  */
+  int32_t shared_sink;       /* 1: one shared expert joins the weight normalisation:
+                                w_gate has N+1 rows, row N scoring the shared expert */
   double capacity_factor;    /* cf (> 0) for the capacity modes                     */
 } moe_config_t;
 
@@ -128,6 +130,13 @@ int moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
  *   margin       [T] fp32 out or NULL: selection score of the k-th pick minus the
  *                best eligible expert left out, min'ed with the last-kept minus
  *                best-dropped group score (+inf when nothing is left out)
+ *   shared_w     [T] fp32 out (only with cfg->shared_sink, else NULL): weight of the
+ *                shared expert's output.  With the sink, w_gate has N+1 rows; the
+ *                affinity covers all N+1 logits (softmax over N+1, or sigmoids), top-k
+ *                chooses among the N routed experts, and the k routed weights and the
+ *                shared weight are normalised together (MoE common-taste page, section
+ *                11, shared-expert sink); lse covers the N+1 logits; p_partial uses
+ *                the routed affinities normalised over the routed experts.
  *   ws           scratch of at least moe_workspace_size() bytes (clobbered)
  * The router GEMM is fp32-equivalent: fp32 FMA, or for bf16 x and N <= 256 the
  * tensor cores over an exact three-way bf16 split of w_gate (every product exact,
@@ -136,7 +145,7 @@ int moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
 int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate,
               const float* logit_offset, const float* bias,
               int32_t* topk_idx, float* topk_w, float* lse, float* p_partial,
-              float* margin, void* ws, size_t ws_bytes, void* stream);
+              float* margin, float* shared_w, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_permute -- counts, capacity drop in token order, offsets, row maps, gather.
@@ -197,9 +206,12 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_rows, int64_t rows_ca
  * fp32 accumulation, no atomics.
  *   y_perm      [R, d] x_dtype; row_of_slot [T, k]; topk_w [T, k] fp32
  *   shared_out  [T, d] x_dtype or NULL; y [T, d] x_dtype out (may alias shared_out)
+ *   shared_w    [T] fp32 or NULL: per-token weight of shared_out (NULL: weight 1;
+ *               moe_route's shared_w output with the shared-expert sink)
  * ------------------------------------------------------------------------- */
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of_slot,
-                const float* topk_w, const void* shared_out, void* y, void* stream);
+                const float* topk_w, const void* shared_out, const float* shared_w, void* y,
+                void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_router_stats -- router statistics in fixed reduction order.
@@ -228,6 +240,35 @@ int moe_router_stats(const moe_config_t* cfg, const int32_t* counts, const int32
  * ------------------------------------------------------------------------- */
 int moe_bias_update(const moe_config_t* cfg, const int32_t* counts, float* bias,
                     float rate, float clamp, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_bias_update_ema -- the bias controller on a moving average of the loads.
+ *
+ * The landscape page names an aux-loss-free "bias EMA" controller (TL;DR, §2,
+ * 实践要点) without a formula.  Reading: ema <- beta * ema + (1 - beta) * c, then
+ * b[e] += rate * sign(mean(ema) - ema[e]) (mean and sign in double), optional
+ * clamp.  beta = 0 is moe_bias_update.
+ *   counts [N] int32; ema [N] fp32 in/out (caller-owned state, start at 0 or at
+ *   the first counts); bias [N] fp32 in/out; 0 <= beta < 1.
+ * ------------------------------------------------------------------------- */
+int moe_bias_update_ema(const moe_config_t* cfg, const int32_t* counts, float* ema, float beta,
+                        float* bias, float rate, float clamp, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_bias_update_seq -- bias update on the per-sequence (length-normalised) load.
+ *
+ * The Practice page's update_bias averages per-sequence statistics so that long
+ * sequences do not dominate (its printed mean of raw counts has the same signs as
+ * the batch counts); its long-context section suggests weighting by token count.
+ * Reading: load[e] = sum over sequences b of c_be / len_b, then
+ * b[e] += rate * sign(mean(load) - load[e]) (double), optional clamp.
+ *   topk_idx [T, k]; seq_offsets [n_seq+1] int32 (device), token ranges of the
+ *   sequences, non-decreasing, seq_offsets[n_seq] <= T; bias [N] in/out;
+ *   ws >= 8 * n_seq * N bytes (clobbered).
+ * ------------------------------------------------------------------------- */
+int moe_bias_update_seq(const moe_config_t* cfg, const int32_t* topk_idx, const int32_t* seq_offsets,
+                        int32_t n_seq, float* bias, float rate, float clamp, void* ws,
+                        size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_permute_noalloc -- moe_permute for callers that cannot allocate.

@@ -460,3 +460,77 @@ def layer_forward(x: np.ndarray, w_gate: np.ndarray, cfg: OracleConfig,
         out["stats"] = router_stats(p["counts"], p["kept"], r["s"], r["lse"], cfg, T,
                                     p["dropped_slots"], p["dropped_tokens"], alpha, z_coef, bias)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Routing variants
+# ---------------------------------------------------------------------------
+def bias_update_ema(bias: np.ndarray, counts: np.ndarray, ema: np.ndarray, beta: float,
+                    rate: float = 1e-3, clamp: Optional[float] = None) -> tuple:
+    """Bias controller on an exponential moving average of the loads.
+
+    [Landscape] (TL;DR, §2 and 实践要点) names an aux-loss-free "bias EMA" controller
+    without a formula.  Reading: the smoothed load c~ <- beta c~ + (1 - beta) c
+    replaces the current counts in the sign update of [Practice] update_bias,
+    b_e += rate * sign(mean(c~) - c~_e).  beta = 0 is the plain update.
+    Returns (new_bias, new_ema).
+    """
+    ema_new = beta * np.asarray(ema, np.float64) + (1.0 - beta) * np.asarray(counts, np.float64)
+    delta = ema_new.mean() - ema_new
+    b = np.asarray(bias, np.float64) + rate * np.sign(delta)
+    if clamp is not None and clamp > 0:
+        b = np.clip(b, -clamp, clamp)
+    return b, ema_new
+
+
+def sequence_load(idx: np.ndarray, seq_offsets: np.ndarray, n_experts: int) -> np.ndarray:
+    """Per-expert load with every sequence weighted equally: sum_b c_be / len_b.
+
+    [Practice] update_bias averages per-sequence counts "so long sequences do not
+    dominate" and its long-context section suggests weighting by token counts.
+    The printed form (mean over sequences of raw counts) equals the batch counts
+    divided by the number of sequences, so its sign update is the batch update;
+    reading for the variant: each sequence's counts are divided by its length
+    (the share of that sequence's tokens routed to e), then summed over sequences
+    (the 1/B factor does not change any sign).
+    """
+    load = np.zeros(n_experts)
+    for b in range(len(seq_offsets) - 1):
+        lo, hi = int(seq_offsets[b]), int(seq_offsets[b + 1])
+        if hi > lo:
+            load += np.bincount(idx[lo:hi].reshape(-1), minlength=n_experts) / float(hi - lo)
+    return load
+
+
+def bias_update_from_load(bias: np.ndarray, load: np.ndarray, rate: float = 1e-3,
+                          clamp: Optional[float] = None) -> np.ndarray:
+    """b_e += rate * sign(mean(load) - load_e) for a real-valued load."""
+    load = np.asarray(load, np.float64)
+    b = np.asarray(bias, np.float64) + rate * np.sign(load.mean() - load)
+    if clamp is not None and clamp > 0:
+        b = np.clip(b, -clamp, clamp)
+    return b
+
+
+def route_shared_sink(x, w_gate_ext, cfg: OracleConfig, bias=None, logit_offset=None) -> dict:
+    """Router whose single shared expert joins the weight normalisation.
+
+    [Taste] section 11 (shared-expert sink): the shared expert is normalised
+    together with the selected routed experts, so it competes for mixture weight.
+    Reading: w_gate_ext has N + 1 rows, row N scoring the shared expert; the
+    affinity covers all N + 1 logits (softmax over N + 1, or independent
+    sigmoids); top-k (and the group limit) choose among the N routed experts only;
+    w_j = s_j / (sum_sel s + s_shared) and w_shared = s_shared / (same).
+    """
+    z = router_logits(x, w_gate_ext, None)
+    if logit_offset is not None:
+        z[:, :-1] = z[:, :-1] + np.asarray(logit_offset, np.float64)[None, :]
+    s_all = affinity(z, cfg.score_fn)
+    s, s_sh = s_all[:, :-1], s_all[:, -1]
+    q = selection_scores(s, bias)
+    mask, gmargin = eligible_mask(q, cfg)
+    idx, emargin = select_topk(q, cfg.top_k, mask)
+    sel = np.take_along_axis(s, idx, axis=1)
+    den = sel.sum(axis=1) + s_sh
+    return {"logits": z, "s": s, "s_shared": s_sh, "idx": idx, "w": sel / den[:, None],
+            "w_shared": s_sh / den, "margin": np.minimum(emargin, gmargin), "lse": logsumexp(z)}

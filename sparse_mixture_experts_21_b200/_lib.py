@@ -25,7 +25,8 @@ CAP_DROPLESS, CAP_CEIL_CF_T_OVER_N, CAP_CF_K_T_OVER_N_FLOOR = 0, 1, 2
 
 EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_route", "moe_permute",
             "moe_grouped_ffn", "moe_combine", "moe_router_stats", "moe_bias_update",
-            "moe_device_status", "moe_status_string", "moe_permute_noalloc")
+            "moe_device_status", "moe_status_string", "moe_permute_noalloc", "moe_bias_update_ema",
+            "moe_bias_update_seq")
 
 
 class MoeConfig(ctypes.Structure):
@@ -33,7 +34,7 @@ class MoeConfig(ctypes.Structure):
     _fields_ = [("T", c_int64), ("d_model", c_int32), ("n_experts", c_int32), ("top_k", c_int32),
                 ("d_ff", c_int32), ("score_fn", c_int32), ("renorm", c_int32), ("n_groups", c_int32),
                 ("topk_groups", c_int32), ("group_score_topn", c_int32), ("capacity_mode", c_int32),
-                ("x_dtype", c_int32), ("capacity_factor", c_double)]
+                ("x_dtype", c_int32), ("shared_sink", c_int32), ("capacity_factor", c_double)]
 
 
 class MoeStats(ctypes.Structure):
@@ -72,13 +73,15 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_capacity": [cfgp, POINTER(c_int64)],
         "moe_route_partials": [cfgp, i32p],
         "moe_workspace_size": [cfgp, POINTER(c_size_t)],
-        "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
+        "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
         "moe_permute": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
         "moe_permute_noalloc": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "moe_grouped_ffn": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp],
-        "moe_combine": [cfgp, vp, vp, vp, vp, vp, vp],
+        "moe_combine": [cfgp, vp, vp, vp, vp, vp, vp, vp],
         "moe_router_stats": [cfgp, vp, vp, vp, vp, vp, vp, c_float, c_float, vp, vp, vp, vp],
         "moe_bias_update": [cfgp, vp, vp, c_float, c_float, vp],
+        "moe_bias_update_ema": [cfgp, vp, vp, c_float, vp, c_float, c_float, vp],
+        "moe_bias_update_seq": [cfgp, vp, vp, c_int32, vp, c_float, c_float, vp, c_size_t, vp],
         "moe_device_status": [i32p, c_int32],
         "moe_status_string": [c_int],
     }
@@ -131,11 +134,12 @@ def workspace_size(cfg: MoeConfig) -> int:
 
 # ----------------------------------------------------------------------------- entry points
 def moe_route(cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_partial, margin, ws,
-              stream=None):
+              stream=None, shared_w=None):
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("moe_route", load().moe_route(
         ctypes.byref(cfg), _ptr(x), _ptr(w_gate), _ptr(logit_offset), _ptr(bias), _ptr(topk_idx),
-        _ptr(topk_w), _ptr(lse), _ptr(p_partial), _ptr(margin), _ptr(ws), nbytes, _stream(stream)))
+        _ptr(topk_w), _ptr(lse), _ptr(p_partial), _ptr(margin), _ptr(shared_w), _ptr(ws), nbytes,
+        _stream(stream)))
 
 
 def moe_permute(cfg, x, topk_idx, counts, offsets, row_of_slot, token_of_row, x_perm, n_dropped,
@@ -160,10 +164,10 @@ def moe_grouped_ffn(cfg, x_rows, rows_cap, offsets, G, w1, w3, w2, f, h_scratch,
         _ptr(w2), int(f), _ptr(h_scratch), _ptr(y_rows), _stream(stream)))
 
 
-def moe_combine(cfg, y_perm, row_of_slot, topk_w, shared_out, y, stream=None):
+def moe_combine(cfg, y_perm, row_of_slot, topk_w, shared_out, y, stream=None, shared_w=None):
     _check("moe_combine", load().moe_combine(
-        ctypes.byref(cfg), _ptr(y_perm), _ptr(row_of_slot), _ptr(topk_w), _ptr(shared_out), _ptr(y),
-        _stream(stream)))
+        ctypes.byref(cfg), _ptr(y_perm), _ptr(row_of_slot), _ptr(topk_w), _ptr(shared_out),
+        _ptr(shared_w), _ptr(y), _stream(stream)))
 
 
 def moe_router_stats(cfg, counts, offsets, p_partial, lse, n_dropped, bias, alpha, z_coef, stats,
@@ -177,6 +181,19 @@ def moe_router_stats(cfg, counts, offsets, p_partial, lse, n_dropped, bias, alph
 def moe_bias_update(cfg, counts, bias, rate, clamp=0.0, stream=None):
     _check("moe_bias_update", load().moe_bias_update(
         ctypes.byref(cfg), _ptr(counts), _ptr(bias), float(rate), float(clamp), _stream(stream)))
+
+
+def moe_bias_update_ema(cfg, counts, ema, beta, bias, rate, clamp=0.0, stream=None):
+    _check("moe_bias_update_ema", load().moe_bias_update_ema(
+        ctypes.byref(cfg), _ptr(counts), _ptr(ema), float(beta), _ptr(bias), float(rate), float(clamp),
+        _stream(stream)))
+
+
+def moe_bias_update_seq(cfg, topk_idx, seq_offsets, n_seq, bias, rate, clamp, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    _check("moe_bias_update_seq", load().moe_bias_update_seq(
+        ctypes.byref(cfg), _ptr(topk_idx), _ptr(seq_offsets), int(n_seq), _ptr(bias), float(rate),
+        float(clamp), _ptr(ws), nbytes, _stream(stream)))
 
 
 def moe_device_status(reset: bool = True) -> int:

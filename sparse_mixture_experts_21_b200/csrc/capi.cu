@@ -34,6 +34,8 @@ int check_config(const moe_config_t* c) {
   if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > 16) return MOE_ERR_INVALID_ARG;
   if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
   if (c->x_dtype != MOE_DTYPE_F32 && c->x_dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->shared_sink != 0 && c->shared_sink != 1) return MOE_ERR_INVALID_ARG;
+  if (c->shared_sink && c->n_experts + 1 > 512) return MOE_ERR_INVALID_ARG;
   if (c->capacity_mode < MOE_CAP_DROPLESS || c->capacity_mode > MOE_CAP_CF_K_T_OVER_N_FLOOR)
     return MOE_ERR_INVALID_ARG;
   if (c->capacity_mode != MOE_CAP_DROPLESS && !(c->capacity_factor > 0.0)) return MOE_ERR_INVALID_ARG;
@@ -105,17 +107,19 @@ int moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
 
 int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate, const float* logit_offset,
               const float* bias, int32_t* topk_idx, float* topk_w, float* lse, float* p_partial,
-              float* margin, void* ws, size_t ws_bytes, void* stream) {
+              float* margin, float* shared_w, void* ws, size_t ws_bytes, void* stream) {
   const int st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
   if (!x || !w_gate || !topk_idx || !topk_w || !lse || !p_partial) return MOE_ERR_INVALID_ARG;
+  if (cfg->shared_sink && !shared_w) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
   const size_t need = route_workspace_bytes(*cfg);
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (need > 0 && (!ws || !aligned16(ws))) return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_route(*cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_partial,
-                                margin, ws, static_cast<cudaStream_t>(stream)));
+                                margin, cfg->shared_sink ? shared_w : nullptr, ws,
+                                static_cast<cudaStream_t>(stream)));
 }
 
 int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,
@@ -159,14 +163,15 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_rows, int64_t rows_ca
 }
 
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of_slot,
-                const float* topk_w, const void* shared_out, void* y, void* stream) {
+                const float* topk_w, const void* shared_out, const float* shared_w, void* y,
+                void* stream) {
   const int st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
   if (!row_of_slot || !topk_w || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y) || (y_perm && !aligned16(y_perm)) || (shared_out && !aligned16(shared_out)))
     return MOE_ERR_INVALID_ARG;
-  return from_cuda(launch_combine(*cfg, y_perm, row_of_slot, topk_w, shared_out, y,
+  return from_cuda(launch_combine(*cfg, y_perm, row_of_slot, topk_w, shared_out, shared_w, y,
                                   static_cast<cudaStream_t>(stream)));
 }
 
@@ -189,6 +194,28 @@ int moe_bias_update(const moe_config_t* cfg, const int32_t* counts, float* bias,
   if (st != MOE_OK) return st;
   if (!counts || !bias) return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_bias_update(*cfg, counts, bias, rate, clamp, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_bias_update_ema(const moe_config_t* cfg, const int32_t* counts, float* ema, float beta,
+                        float* bias, float rate, float clamp, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !ema || !bias || !(beta >= 0.f && beta < 1.f)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_bias_update_ema(*cfg, counts, ema, beta, bias, rate, clamp,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int moe_bias_update_seq(const moe_config_t* cfg, const int32_t* topk_idx, const int32_t* seq_offsets,
+                        int32_t n_seq, float* bias, float rate, float clamp, void* ws,
+                        size_t ws_bytes, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (n_seq < 0 || !seq_offsets || !bias || (n_seq > 0 && !topk_idx)) return MOE_ERR_INVALID_ARG;
+  const size_t need = (size_t)8 * (size_t)(n_seq > 0 ? n_seq : 1) * (size_t)cfg->n_experts;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 7u)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_bias_update_seq(*cfg, topk_idx, seq_offsets, n_seq, bias, rate, clamp,
+                                          static_cast<double*>(ws), static_cast<cudaStream_t>(stream)));
 }
 
 int moe_device_status(int32_t* status, int32_t reset) {

@@ -16,7 +16,8 @@ template <typename XT, int K, int U>
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
                const float* __restrict__ topk_w, const uint4* __restrict__ shared_out,
-               uint4* __restrict__ y, int64_t T, int k, int nvec) {
+               const float* __restrict__ shared_w, uint4* __restrict__ y, int64_t T, int k,
+               int nvec) {
   constexpr int VN = Vec<XT>::N;
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -27,6 +28,7 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ row
     // a dropped (or padding) slot reads a kept row of the same token with weight 0,
     // so every load below is unconditional and can be issued together
     const unsigned kept = __ballot_sync(0xffffffffu, mr >= 0);
+    const float sw = shared_w ? shared_w[t] : 1.f;
     const int32_t any_row = kept ? __shfl_sync(0xffffffffu, mr, __ffs(kept) - 1) : 0;
     int32_t rows[K];
     float ws[K];
@@ -49,6 +51,8 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ row
         }
         if (c < nvec && shared_out) {
           unpack16(ldg_nc16(shared_out + t * nvec + c), acc[u], XT());
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[u][i] *= sw;
         } else {
 #pragma unroll
           for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
@@ -173,18 +177,75 @@ bias_update_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias,
   }
 }
 
+// Moving-average controller: ema <- beta ema + (1 - beta) c; b += rate sign(mean(ema) - ema)
+// (the landscape page's "bias EMA"; reading of the formula as in the header).
+__global__ void __launch_bounds__(kStatThreads)
+bias_update_ema_kernel(const int32_t* __restrict__ counts, float* __restrict__ ema, float beta,
+                       float* __restrict__ bias, int N, float rate, float clamp) {
+  __shared__ double buf[kStatThreads];
+  const int e = threadIdx.x;
+  double v = 0.0;
+  if (e < N) {
+    v = (double)beta * (double)ema[e] + (1.0 - (double)beta) * (double)counts[e];
+    ema[e] = (float)v;
+  }
+  const double mean = block_sum<kStatThreads>(e < N ? v : 0.0, buf) / N;
+  if (e < N) {
+    const double delta = mean - v;
+    const float sgn = delta > 0 ? 1.f : (delta < 0 ? -1.f : 0.f);
+    float b = bias[e] + rate * sgn;
+    if (clamp > 0.f) b = fminf(fmaxf(b, -clamp), clamp);
+    bias[e] = b;
+  }
+}
+
+// Per-sequence share of each expert: part[b, e] = c_be / len_b (one CTA per sequence).
+__global__ void __launch_bounds__(256)
+seq_load_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ seq_offsets,
+                int k, int N, double* __restrict__ part) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < N; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int64_t lo = seq_offsets[blockIdx.x], hi = seq_offsets[blockIdx.x + 1];
+  for (int64_t sl = lo * k + threadIdx.x; sl < hi * k; sl += blockDim.x) atomicAdd(&hist[topk_idx[sl]], 1);
+  __syncthreads();
+  const double inv = hi > lo ? 1.0 / (double)(hi - lo) : 0.0;
+  for (int e = threadIdx.x; e < N; e += blockDim.x)
+    part[(int64_t)blockIdx.x * N + e] = hist[e] * inv;
+}
+
+// load_e = sum_b part[b, e] in sequence order; b += rate sign(mean(load) - load_e).
+__global__ void __launch_bounds__(kStatThreads)
+bias_update_seq_kernel(const double* __restrict__ part, int n_seq, float* __restrict__ bias, int N,
+                       float rate, float clamp) {
+  __shared__ double buf[kStatThreads];
+  const int e = threadIdx.x;
+  double load = 0.0;
+  if (e < N)
+    for (int b = 0; b < n_seq; ++b) load += part[(int64_t)b * N + e];
+  const double mean = block_sum<kStatThreads>(e < N ? load : 0.0, buf) / N;
+  if (e < N) {
+    const double delta = mean - load;
+    const float sgn = delta > 0 ? 1.f : (delta < 0 ? -1.f : 0.f);
+    float b = bias[e] + rate * sgn;
+    if (clamp > 0.f) b = fminf(fmaxf(b, -clamp), clamp);
+    bias[e] = b;
+  }
+}
+
 }  // namespace cs
 
 
 template <typename XT>
 cudaError_t launch_combine_t(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
-                             const float* topk_w, const void* shared_out, void* y, int grid, int nvec,
-                             cudaStream_t s) {
+                             const float* topk_w, const void* shared_out, const float* shared_w,
+                             void* y, int grid, int nvec, cudaStream_t s) {
   auto yp = static_cast<const uint4*>(y_perm);
   auto sh = static_cast<const uint4*>(shared_out);
   auto yo = static_cast<uint4*>(y);
 #define MOE_COMBINE(KK, UU) \
-  cs::combine_kernel<XT, KK, UU><<<grid, 256, 0, s>>>(yp, row_of_slot, topk_w, sh, yo, c.T, c.top_k, nvec)
+  cs::combine_kernel<XT, KK, UU><<<grid, 256, 0, s>>>(yp, row_of_slot, topk_w, sh, shared_w, yo, c.T, \
+                                                      c.top_k, nvec)
   switch (c.top_k) {
     case 1: MOE_COMBINE(1, 4); break;
     case 2: MOE_COMBINE(2, 4); break;
@@ -201,7 +262,8 @@ cudaError_t launch_combine_t(const moe_config_t& c, const void* y_perm, const in
 }
 
 cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
-                           const float* topk_w, const void* shared_out, void* y, cudaStream_t s) {
+                           const float* topk_w, const void* shared_out, const float* shared_w,
+                           void* y, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   const size_t eb = c.x_dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const int nvec = (int)((size_t)c.d_model * eb / 16);
@@ -209,8 +271,9 @@ cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int3
   const int64_t cap = (int64_t)sm_count() * 8;
   const int grid = (int)(want < cap ? want : cap);
   if (c.x_dtype == MOE_DTYPE_BF16)
-    return launch_combine_t<__nv_bfloat16>(c, y_perm, row_of_slot, topk_w, shared_out, y, grid, nvec, s);
-  return launch_combine_t<float>(c, y_perm, row_of_slot, topk_w, shared_out, y, grid, nvec, s);
+    return launch_combine_t<__nv_bfloat16>(c, y_perm, row_of_slot, topk_w, shared_out, shared_w, y, grid,
+                                           nvec, s);
+  return launch_combine_t<float>(c, y_perm, row_of_slot, topk_w, shared_out, shared_w, y, grid, nvec, s);
 }
 
 cudaError_t launch_stats(const moe_config_t& c, const int32_t* counts, const int32_t* offsets,
@@ -226,6 +289,27 @@ cudaError_t launch_stats(const moe_config_t& c, const int32_t* counts, const int
 cudaError_t launch_bias_update(const moe_config_t& c, const int32_t* counts, float* bias, float rate,
                                float clamp, cudaStream_t s) {
   cs::bias_update_kernel<<<1, cs::kStatThreads, 0, s>>>(counts, bias, c.n_experts, rate, clamp);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
+
+namespace moe {
+
+cudaError_t launch_bias_update_ema(const moe_config_t& c, const int32_t* counts, float* ema, float beta,
+                                   float* bias, float rate, float clamp, cudaStream_t s) {
+  cs::bias_update_ema_kernel<<<1, cs::kStatThreads, 0, s>>>(counts, ema, beta, bias, c.n_experts, rate,
+                                                            clamp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bias_update_seq(const moe_config_t& c, const int32_t* topk_idx,
+                                   const int32_t* seq_offsets, int n_seq, float* bias, float rate,
+                                   float clamp, double* ws, cudaStream_t s) {
+  if (n_seq > 0)
+    cs::seq_load_kernel<<<n_seq, 256, c.n_experts * sizeof(int32_t), s>>>(topk_idx, seq_offsets, c.top_k,
+                                                                         c.n_experts, ws);
+  cs::bias_update_seq_kernel<<<1, cs::kStatThreads, 0, s>>>(ws, n_seq, bias, c.n_experts, rate, clamp);
   return cudaGetLastError();
 }
 

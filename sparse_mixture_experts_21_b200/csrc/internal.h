@@ -22,8 +22,8 @@ size_t route_workspace_bytes(const moe_config_t& c);
 
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* w_gate,
                          const float* logit_offset, const float* bias, int32_t* topk_idx,
-                         float* topk_w, float* lse, float* p_partial, float* margin, void* ws,
-                         cudaStream_t s);
+                         float* topk_w, float* lse, float* p_partial, float* margin,
+                         float* shared_w, void* ws, cudaStream_t s);
 
 // Token-order capacity drop and permutation.
 constexpr int kPermuteTokensPerBlock = 256;
@@ -43,13 +43,19 @@ cudaError_t launch_ffn_f32(const float* x_rows, int64_t rows_cap, const int32_t*
                            float* h, float* y, cudaStream_t s);
 
 cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
-                           const float* topk_w, const void* shared_out, void* y, cudaStream_t s);
+                           const float* topk_w, const void* shared_out, const float* shared_w,
+                           void* y, cudaStream_t s);
 cudaError_t launch_stats(const moe_config_t& c, const int32_t* counts, const int32_t* offsets,
                          const float* p_partial, int nblk, const float* lse,
                          const int32_t* n_dropped, const float* bias, float alpha, float z_coef,
                          moe_stats_t* stats, float* f_out, float* p_out, cudaStream_t s);
 cudaError_t launch_bias_update(const moe_config_t& c, const int32_t* counts, float* bias,
                                float rate, float clamp, cudaStream_t s);
+cudaError_t launch_bias_update_ema(const moe_config_t& c, const int32_t* counts, float* ema, float beta,
+                                   float* bias, float rate, float clamp, cudaStream_t s);
+cudaError_t launch_bias_update_seq(const moe_config_t& c, const int32_t* topk_idx,
+                                   const int32_t* seq_offsets, int n_seq, float* bias, float rate,
+                                   float clamp, double* ws, cudaStream_t s);
 
 int sm_count();
 

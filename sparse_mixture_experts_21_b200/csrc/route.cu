@@ -38,6 +38,8 @@ struct RouteArgs {
   float* lse;
   float* p_partial;
   float* margin;
+  int sink;            // 1: logit column N scores the shared expert (shared-expert sink)
+  float* shared_w;     // [T] weight of the shared expert when sink
 };
 
 // Selection phase: tokens t0 .. t0+TM-1 of the block, logits[tm * ld + e] in
@@ -63,8 +65,9 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
       valid[i] = e < N;
       z[i] = valid[i] ? logits[tm * ld + e] + (a.logit_offset ? a.logit_offset[e] : 0.f) : -INFINITY;
     }
-    // affinity and logsumexp
-    float m = -INFINITY;
+    // affinity and logsumexp (with the sink, over the N routed logits and the shared one)
+    const float z_sh = a.sink ? logits[tm * ld + N] : -INFINITY;
+    float m = z_sh;
 #pragma unroll
     for (int i = 0; i < NV; ++i) m = fmaxf(m, z[i]);
     m = warp_max(m);
@@ -75,7 +78,11 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
       se += ex[i];
     }
     se = warp_sum(se);
+    const float ex_sh = a.sink ? expf(z_sh - m) : 0.f;
+    se += ex_sh;
     const float lse = m + logf(se);
+    float s_sh = 0.f;
+    if (a.sink) s_sh = a.score_fn == MOE_SCORE_SOFTMAX ? ex_sh / se : 1.f / (1.f + expf(-z_sh));
     float ssum = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
@@ -84,8 +91,9 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
       ssum += s[i];
       q[i] = valid[i] ? s[i] + (a.bias ? a.bias[lane + 32 * i] : 0.f) : -INFINITY;
     }
-    // load-balance statistics: normalised affinity (softmax probs or s / sum s)
-    if (a.score_fn == MOE_SCORE_SIGMOID) {
+    // load-balance statistics: routed affinities normalised over the routed experts
+    // (softmax probs as they are, or s / sum s)
+    if (a.score_fn == MOE_SCORE_SIGMOID || a.sink) {
       ssum = warp_sum(ssum);
 #pragma unroll
       for (int i = 0; i < NV; ++i) pacc[i] += s[i] / ssum;
@@ -190,7 +198,7 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
     warp_argmax(nv, ni);
     const float emargin = (nv == -INFINITY) ? INFINITY : kth_q - nv;
 
-    const float wsum = warp_sum(lane < k ? my_s : 0.f);
+    const float wsum = warp_sum(lane < k ? my_s : 0.f) + s_sh;
     if (lane < k) {
       a.topk_idx[t * k + lane] = my_idx;
       a.topk_w[t * k + lane] = a.renorm ? my_s / wsum : my_s;
@@ -198,6 +206,7 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
     if (lane == 0) {
       a.lse[t] = lse;
       if (a.margin) a.margin[t] = fminf(emargin, gmargin);
+      if (a.sink) a.shared_w[t] = a.renorm ? s_sh / wsum : s_sh;
     }
   }
 
@@ -263,7 +272,7 @@ route_simt_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate, in
   float* pwarp = smem + (S::GEMM_FLOATS > S::PART_FLOATS ? S::GEMM_FLOATS : S::PART_FLOATS);
 
   const int tid = threadIdx.x;
-  const int N = a.N;
+  const int N = a.N + a.sink;     // gate rows (the shared expert's row last)
   const int64_t T = a.T;
   const int64_t t0 = (int64_t)blockIdx.x * TM;
   const int split = tid / (S::NTX * S::NTY);
@@ -548,7 +557,8 @@ cudaError_t launch_tc(const moe_config_t& c, const void* x, const float* wg, con
   __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(ws);
   const int64_t n = (int64_t)NP * dpad;
   const int sgrid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  split_gate_kernel<<<sgrid, 256, 0, s>>>(wg, c.n_experts, d, NP, dpad, wsplit);
+  split_gate_kernel<<<sgrid, 256, 0, s>>>(wg, c.n_experts + (c.shared_sink ? 1 : 0), d, NP, dpad,
+                                          wsplit);
   CUtensorMap mx, mw;
   if (!make_map_bf16(&mx, x, (uint64_t)c.T, (uint64_t)d, TC_TM) ||
       !make_map_bf16(&mw, wsplit, (uint64_t)NP, (uint64_t)3 * dpad, NP))
@@ -569,13 +579,15 @@ int route_np(int n) {
   return np;
 }
 
+static int gate_rows(const moe_config_t& c) { return c.n_experts + (c.shared_sink ? 1 : 0); }
+
 bool route_uses_tc(const moe_config_t& c) {
-  return c.x_dtype == MOE_DTYPE_BF16 && c.n_experts <= 256;
+  return c.x_dtype == MOE_DTYPE_BF16 && gate_rows(c) <= 256;
 }
 
 int route_tokens_per_block(const moe_config_t& c) {
   if (route_uses_tc(c)) return rt::TC_TM;
-  switch (route_np(c.n_experts)) {
+  switch (route_np(gate_rows(c))) {
     case 8: case 16: case 32: case 512: return 32;
     default: return 64;
   }
@@ -583,14 +595,14 @@ int route_tokens_per_block(const moe_config_t& c) {
 
 size_t route_workspace_bytes(const moe_config_t& c) {
   if (!route_uses_tc(c)) return 0;
-  const int np = route_np(c.n_experts) < 16 ? 16 : route_np(c.n_experts);
+  const int np = route_np(gate_rows(c)) < 16 ? 16 : route_np(gate_rows(c));
   const size_t dpad = (size_t)(c.d_model + rt::TC_BK - 1) / rt::TC_BK * rt::TC_BK;
   return (size_t)np * 3 * dpad * 2;
 }
 
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* wg, const float* off,
                          const float* bias, int32_t* idx, float* w, float* lse, float* pp,
-                         float* margin, void* ws, cudaStream_t s) {
+                         float* margin, float* shared_w, void* ws, cudaStream_t s) {
   if (c.T == 0) return cudaSuccess;
   rt::RouteArgs a;
   a.logit_offset = off;
@@ -608,8 +620,10 @@ cudaError_t launch_route(const moe_config_t& c, const void* x, const float* wg, 
   a.lse = lse;
   a.p_partial = pp;
   a.margin = margin;
+  a.sink = c.shared_sink ? 1 : 0;
+  a.shared_w = shared_w;
   if (route_uses_tc(c)) {
-    switch (route_np(c.n_experts)) {
+    switch (route_np(gate_rows(c))) {
       case 8: case 16: return rt::launch_tc<16>(c, x, wg, a, ws, s);
       case 32:  return rt::launch_tc<32>(c, x, wg, a, ws, s);
       case 64:  return rt::launch_tc<64>(c, x, wg, a, ws, s);
@@ -618,7 +632,7 @@ cudaError_t launch_route(const moe_config_t& c, const void* x, const float* wg, 
       default:  return cudaErrorInvalidValue;
     }
   }
-  switch (route_np(c.n_experts)) {
+  switch (route_np(gate_rows(c))) {
     case 8:   return rt::launch_simt<8, 32, 2, 8, 16>(c, x, wg, a, s);
     case 16:  return rt::launch_simt<16, 32, 2, 8, 8>(c, x, wg, a, s);
     case 32:  return rt::launch_simt<32, 32, 4, 8, 8>(c, x, wg, a, s);

@@ -27,6 +27,7 @@ def make_config(w: Workload, T: Optional[int] = None) -> L.MoeConfig:
     c.capacity_mode = CAP_MODES[w.capacity]
     c.capacity_factor = w.cf
     c.x_dtype = L.DTYPE_F32 if w.dtype == "fp32" else L.DTYPE_BF16
+    c.shared_sink = 1 if w.shared_sink else 0
     return c
 
 
@@ -72,6 +73,7 @@ class MoELayer:
         self.counts_global = z(N, dtype=torch.int32)
         self.f_out = z(N)
         self.p_out = z(N)
+        self.shared_w = z(max(T, 1)) if w.shared_sink else None
 
     # the launches of one layer forward; `x` is [T, d] on the device.  `marks`, if
     # given, is a list of 7 CUDA events recorded between the stages (route, permute,
@@ -83,7 +85,8 @@ class MoELayer:
         rec = (lambda i: marks[i].record(s)) if marks is not None else (lambda i: None)
         rec(0)
         L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), self.topk_idx,
-                    self.topk_w, self.lse, self.p_partial, self.margin, self.ws, s)
+                    self.topk_w, self.lse, self.p_partial, self.margin, self.ws, s,
+                    shared_w=self.shared_w)
         rec(1)
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
                       self.token_of_row, self.x_perm, self.n_dropped, self.ws, s)
@@ -97,7 +100,8 @@ class MoELayer:
                               self.hs, self.ys, s)
             shared = self.ys
         rec(4)
-        L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, y, s)
+        L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, y, s,
+                      shared_w=self.shared_w)
         rec(5)
         L.moe_router_stats(c, self.counts, self.offsets, self.p_partial, self.lse, self.n_dropped,
                            W.get("bias"), self.w.alpha, self.w.z_coef, self.stats, self.f_out,

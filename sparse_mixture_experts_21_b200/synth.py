@@ -12,6 +12,7 @@ and fan_in = f for W2; the selection bias b ~ N(0, 0.01) read as variance 0.01
 temporary) and rounded to the storage dtype.  The Switch-style workload adds the
 fixed per-expert logit offset o[e] = -1.1 * ln(e + 1), the log of an unnormalised
 Zipf(s = 1.1) weight, so expert 0 is the hottest.
+With the shared-expert sink, W_g has one extra (last) row scoring the shared expert.
 """
 from __future__ import annotations
 
@@ -45,6 +46,7 @@ class Workload:
     z_coef: float = 1e-3                # z-loss coefficient reported in the stats
     bias_rate: float = 1e-3             # aux-loss-free bias update step
     renorm: bool = True
+    shared_sink: bool = False           # the (single) shared expert joins the weight normalisation
 
     def with_tokens(self, T: int) -> "Workload":
         return replace(self, T=T)
@@ -83,7 +85,7 @@ def make_inputs(w: Workload, device="cuda", seed: int = 0, experts: bool = True)
         return (torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * std)
 
     out = {"x": randn((w.T, w.d), 1.0).to(dt).contiguous(),
-           "w_gate": randn((w.N, w.d), 1.0 / math.sqrt(w.d)).contiguous()}
+           "w_gate": randn((w.N + (1 if w.shared_sink else 0), w.d), 1.0 / math.sqrt(w.d)).contiguous()}
     out["bias"] = randn((w.N,), w.bias_std).contiguous() if w.bias_std > 0 else None
     out["logit_offset"] = zipf_offset(w.N, w.zipf_s).to(dev) if w.zipf_s > 0 else None
     if not experts:

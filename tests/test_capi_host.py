@@ -98,12 +98,12 @@ def test_null_and_misaligned_pointers_rejected(lib):
     c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
     cp = ctypes.byref(c)
     # null required pointers: rejected on the host, nothing launched
-    assert lib.moe_route(cp, None, None, None, None, None, None, None, None, None, None, 0, None) == \
+    assert lib.moe_route(cp, None, None, None, None, None, None, None, None, None, None, None, 0, None) == \
         L.MOE_ERR_INVALID_ARG
     bad = 0x1000008  # not 16-byte aligned
     ok = 0x1000000
-    assert lib.moe_route(cp, bad, ok, None, None, ok, ok, ok, ok, None, None, 0, None) == L.MOE_ERR_INVALID_ARG
-    assert lib.moe_combine(cp, ok, ok, ok, None, bad, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(cp, bad, ok, None, None, ok, ok, ok, ok, None, None, None, 0, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(cp, ok, ok, ok, None, None, bad, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_grouped_ffn(cp, ok, 10, ok, 0, ok, ok, ok, 256, ok, ok, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_grouped_ffn(cp, ok, 10, ok, 1, ok, ok, ok, 12, ok, ok, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_bias_update(cp, None, ok, 1e-3, 0.0, None) == L.MOE_ERR_INVALID_ARG
@@ -117,17 +117,31 @@ def test_workspace_too_small_rejected(lib):
     st = lib.moe_permute(ctypes.byref(c), ok, ok, ok, ok, ok, ok, ok, ok, ok, 4, None)
     assert st == L.MOE_ERR_WORKSPACE_TOO_SMALL
     c3 = layer.make_config(synth.WORKLOADS["deepseek_v3"])
-    st = lib.moe_route(ctypes.byref(c3), ok, ok, None, None, ok, ok, ok, ok, None, ok, 1024, None)
+    st = lib.moe_route(ctypes.byref(c3), ok, ok, None, None, ok, ok, ok, ok, None, None, ok, 1024, None)
     assert st == L.MOE_ERR_WORKSPACE_TOO_SMALL
 
 
 def test_empty_batch_is_a_no_op(lib):
     c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"], T=0)
-    assert lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, None, None, 0,
+    assert lib.moe_route(ctypes.byref(c), None, None, None, None, None, None, None, None, None, None, None, 0,
                          None) == L.MOE_OK
-    assert lib.moe_combine(ctypes.byref(c), None, None, None, None, None, None) == L.MOE_OK
+    assert lib.moe_combine(ctypes.byref(c), None, None, None, None, None, None, None) == L.MOE_OK
     assert lib.moe_grouped_ffn(ctypes.byref(c), None, 0, 0x1000000, 1, None, None, None, 256, None, None,
                                None) == L.MOE_OK
+
+
+def test_variant_argument_checks(lib):
+    c = layer.make_config(synth.WORKLOADS["deepseekmoe_16b"])
+    ok = 0x1000000
+    c.shared_sink = 1          # the sink needs its shared-weight output
+    assert lib.moe_route(ctypes.byref(c), ok, ok, None, None, ok, ok, ok, ok, None, None, ok, 1 << 30,
+                         None) == L.MOE_ERR_INVALID_ARG
+    c.shared_sink = 2
+    assert lib.moe_capacity(ctypes.byref(c), ctypes.byref(ctypes.c_int64())) == L.MOE_ERR_INVALID_ARG
+    c.shared_sink = 0
+    assert lib.moe_bias_update_ema(ctypes.byref(c), ok, ok, 1.0, ok, 1e-3, 0.0, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_bias_update_seq(ctypes.byref(c), ok, ok, 4, ok, 1e-3, 0.0, ok, 8, None) == \
+        L.MOE_ERR_WORKSPACE_TOO_SMALL
 
 
 def test_status_strings(lib):

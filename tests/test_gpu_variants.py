@@ -1,0 +1,106 @@
+"""GPU-vs-oracle parity of the routing variants, through the C ABI:
+non-renormalised weights, the shared-expert sink, the moving-average bias
+controller and the per-sequence (length-normalised) bias update."""
+from __future__ import annotations
+
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from sparse_mixture_experts_21_b200 import _lib as L
+from sparse_mixture_experts_21_b200.layer import MoELayer, make_config
+from sparse_mixture_experts_21_b200.synth import WORKLOADS, make_inputs, random_routing
+from tests.parity_util import (NEAR_TIE, expert_weights_fn, f64, i64, oracle_cfg, rel_err,
+                               shared_weights, tol_for)
+
+pytestmark = pytest.mark.gpu
+
+DS_SMALL = replace(WORKLOADS["deepseekmoe_16b"], name="dsmoe_small", T=777, d=264, N=16, f=192,
+                   f_shared=192)
+
+
+def _run(w):
+    inp = make_inputs(w, "cuda")
+    lay = MoELayer(w, inp, "cuda", update_bias=False)
+    lay.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    return lay, inp
+
+
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+def test_renorm_off(score):
+    w = replace(DS_SMALL, renorm=False, score=score)
+    lay, inp = _run(w)
+    r = O.route(f64(inp["x"]), f64(inp["w_gate"]), oracle_cfg(w))
+    clear = r["margin"] >= NEAR_TIE
+    assert np.array_equal(i64(lay.topk_idx)[clear], r["idx"][clear])
+    assert np.max(np.abs(f64(lay.topk_w)[clear] - r["w"][clear])) < 2e-5
+    wts = O.gate_weights(r["s"], i64(lay.topk_idx), False)
+    out = O.layer_forward(f64(inp["x"]), None, oracle_cfg(w), expert_weights_fn(inp), shared_weights(inp),
+                          routing={"idx": i64(lay.topk_idx), "w": wts})
+    assert rel_err(f64(lay.y[:w.T]), out["y"]) < tol_for(w)
+
+
+@pytest.mark.parametrize("score,N,dtype", [("softmax", 16, "bf16"), ("sigmoid", 64, "bf16"),
+                                           ("sigmoid", 300, "bf16"), ("softmax", 8, "fp32")])
+def test_shared_expert_sink(score, N, dtype):
+    """N + 1 <= 256 runs the tensor-core router, 301 gate rows and fp32 the FMA one."""
+    d = 128 if dtype == "fp32" else 264
+    w = replace(DS_SMALL, score=score, N=N, n_shared=1, shared_sink=True, dtype=dtype, d=d,
+                k=2 if N == 8 else 6)
+    lay, inp = _run(w)
+    cfg = oracle_cfg(w)
+    r = O.route_shared_sink(f64(inp["x"]), f64(inp["w_gate"]), cfg)
+    clear = r["margin"] >= NEAR_TIE
+    assert np.array_equal(i64(lay.topk_idx)[clear], r["idx"][clear])
+    assert np.max(np.abs(f64(lay.topk_w)[clear] - r["w"][clear])) < 2e-5
+    assert np.max(np.abs(f64(lay.shared_w[:w.T])[clear] - r["w_shared"][clear])) < 2e-5
+    assert np.allclose(f64(lay.topk_w).sum(1) + f64(lay.shared_w[:w.T]), 1.0, atol=1e-5)
+    assert rel_err(f64(lay.lse), r["lse"]) < 1e-5
+    # whole layer, oracle fed the GPU's expert choice
+    sel = np.take_along_axis(r["s"], i64(lay.topk_idx), 1)
+    den = sel.sum(1) + r["s_shared"]
+    out = O.layer_forward(f64(inp["x"]), None, cfg, expert_weights_fn(inp), None,
+                          routing={"idx": i64(lay.topk_idx), "w": sel / den[:, None]})
+    y_ref = out["y"] + (r["s_shared"] / den)[:, None] * O.swiglu_ffn(f64(inp["x"]), *shared_weights(inp))
+    assert rel_err(f64(lay.y[:w.T]), y_ref) < tol_for(w)
+
+
+def test_bias_update_ema_steps():
+    w = WORKLOADS["deepseek_v3"]
+    c = make_config(w)
+    rng = np.random.default_rng(3)
+    b0 = rng.normal(scale=0.05, size=w.N).astype(np.float32)
+    bias = torch.tensor(b0, device="cuda")
+    ema = torch.zeros(w.N, device="cuda")
+    b_ref, e_ref = b0.astype(np.float64), np.zeros(w.N)
+    for step in range(4):
+        counts = rng.integers(0, 2000, size=w.N).astype(np.int32)
+        L.moe_bias_update_ema(c, torch.tensor(counts, device="cuda"), ema, 0.8, bias, 1e-3, 0.0)
+        b_ref, e_ref = O.bias_update_ema(b_ref, counts, e_ref, 0.8, 1e-3)
+    torch.cuda.synchronize()
+    assert np.max(np.abs(f64(ema) - e_ref)) <= 1e-6 * np.max(np.abs(e_ref))
+    assert np.max(np.abs(f64(bias) - b_ref)) < 1e-7
+
+
+def test_bias_update_seq():
+    w = WORKLOADS["deepseek_v3"]
+    T, N, k = 5000, w.N, w.k
+    c = make_config(w, T=T)
+    rng = np.random.default_rng(4)
+    cuts = np.sort(rng.choice(np.arange(1, T), size=11, replace=False))
+    off = np.concatenate([[0], cuts, [T]]).astype(np.int32)
+    off[5] = off[4]                                         # one empty sequence
+    idx = random_routing(T, N, k, "cuda", seed=9)
+    bias = torch.zeros(N, device="cuda")
+    ws = torch.empty(8 * (len(off) - 1) * N, dtype=torch.uint8, device="cuda")
+    L.moe_bias_update_seq(c, idx, torch.tensor(off, device="cuda"), len(off) - 1, bias, 1e-3, 0.0, ws)
+    torch.cuda.synchronize()
+    load = O.sequence_load(i64(idx), off, N)
+    ref = O.bias_update_from_load(np.zeros(N), load, 1e-3)
+    assert np.array_equal(f64(bias) != 0, ref != 0)
+    assert np.max(np.abs(f64(bias) - ref)) < 1e-9

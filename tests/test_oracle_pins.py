@@ -476,3 +476,69 @@ def test_flattening_consistency():
     flat = O.route(x3.reshape(-1, 16), wg, cfg)
     per_b = [O.route(x3[b], wg, cfg) for b in range(4)]
     assert np.array_equal(flat["idx"], np.concatenate([p["idx"] for p in per_b]))
+
+
+# ---------------------------------------------------------------- routing variants
+def test_ema_controller_beta_zero_is_plain_update():
+    rng = np.random.default_rng(79)
+    c = rng.integers(0, 50, size=16)
+    b0 = rng.normal(scale=0.01, size=16)
+    b, e = O.bias_update_ema(b0, c, np.zeros(16), beta=0.0, rate=1e-3)
+    assert np.array_equal(b, O.bias_update(b0, c, rate=1e-3)) and np.array_equal(e, c)
+
+
+def test_ema_controller_geometric_closed_form():
+    """Constant loads c from a zero state: c~_n = c (1 - beta^n)."""
+    c = np.array([4.0, 10.0, 1.0, 5.0])
+    beta, ema = 0.9, np.zeros(4)
+    for n in range(1, 8):
+        _, ema = O.bias_update_ema(np.zeros(4), c, ema, beta)
+        assert np.allclose(ema, c * (1 - beta ** n), rtol=1e-14)
+
+
+def test_sequence_load_equal_lengths_matches_batch_sign_update():
+    rng = np.random.default_rng(83)
+    idx = np.stack([rng.choice(12, 3, replace=False) for _ in range(40)])
+    off = np.arange(0, 41, 10)
+    load = O.sequence_load(idx, off, 12)
+    counts = np.bincount(idx.reshape(-1), minlength=12)
+    assert np.allclose(load, counts / 10.0)
+    assert np.array_equal(O.bias_update_from_load(np.zeros(12), load),
+                          O.bias_update(np.zeros(12), counts))
+
+
+def test_printed_per_sequence_mean_is_the_batch_update():
+    """[Practice]'s per_seq_counts.mean(0) sign update equals the batch update."""
+    rng = np.random.default_rng(89)
+    idx = np.stack([rng.choice(8, 2, replace=False) for _ in range(30)])
+    off = [0, 4, 19, 30]
+    per_seq = np.stack([np.bincount(idx[a:b].reshape(-1), minlength=8) for a, b in zip(off[:-1], off[1:])])
+    score = per_seq.astype(np.float64).mean(axis=0)
+    printed = np.zeros(8) + 1e-3 * np.sign(score.mean() - score)
+    assert np.array_equal(printed, O.bias_update(np.zeros(8), np.bincount(idx.reshape(-1), minlength=8)))
+
+
+def test_sequence_load_hand_case():
+    # sequence 0 = 1 token choosing {0, 1}; sequence 1 = 3 tokens choosing {0,2},{0,2},{1,2}
+    idx = np.array([[0, 1], [0, 2], [0, 2], [1, 2]])
+    load = O.sequence_load(idx, np.array([0, 1, 4]), 3)
+    assert np.allclose(load, [1 + 2 / 3, 1 + 1 / 3, 1.0])
+
+
+def test_shared_sink_reduces_to_plain_router_and_weights_sum_to_one():
+    rng = np.random.default_rng(97)
+    x, wg = rng.normal(size=(50, 16)), rng.normal(size=(12, 16)) / 4
+    for fn in (O.SOFTMAX, O.SIGMOID):
+        cfg = O.OracleConfig(12, 3, score_fn=fn)
+        ext = np.concatenate([wg, rng.normal(size=(1, 16))])
+        r = O.route_shared_sink(x, ext, cfg)
+        assert np.allclose(r["w"].sum(1) + r["w_shared"], 1.0, atol=1e-12)
+        # a shared gate that is never active (score -> 0) leaves the plain router
+        x2 = np.concatenate([x, np.ones((50, 1))], axis=1)
+        ext2 = np.concatenate([np.concatenate([wg, np.zeros((12, 1))], 1),
+                               np.concatenate([np.zeros((1, 16)), [[-1e3]]], 1)])
+        r2 = O.route_shared_sink(x2, ext2, cfg)
+        plain = O.route(x, wg, cfg)
+        assert np.array_equal(r2["idx"], plain["idx"])
+        if fn == O.SIGMOID:       # sigmoid scores of the routed experts are unchanged
+            assert np.allclose(r2["w"], plain["w"], rtol=1e-12) and np.all(r2["w_shared"] < 1e-300)
