@@ -201,6 +201,8 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="workload name from synth.WORKLOADS (default: the DeepSeek-V3-shaped layer)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="reduced token count (profiling of a small case only)")
     ap.add_argument("--experts", type=int, default=None,
@@ -227,10 +229,10 @@ def main():
         pg = dist
 
     L.load()
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
     if args.tokens or args.experts:
         from dataclasses import replace
-        w = replace(w, name=WORKLOAD + "_reduced", T=args.tokens or w.T, N=args.experts or w.N)
+        w = replace(w, name=w.name + "_reduced", T=args.tokens or w.T, N=args.experts or w.N)
     inp = make_inputs(w, dev, seed=rank)
     lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD)
     x = inp["x"]
@@ -275,6 +277,10 @@ def main():
     bytes_route = T * d * eb + 4 * N * d + 8 * T * k
     bytes_perm = T * d * eb + R * d * eb + 12 * T * k
     bytes_comb = R * d * eb + 2 * T * d * eb + 8 * T * k
+    if w.expert_choice:        # scores [N, T] written; rows gathered per row; combine reads the maps
+        bytes_route = T * d * eb + 4 * N * d + 4 * N * T
+        bytes_perm = 2 * R * d * eb + 12 * N * T
+        bytes_comb = R * d * eb + 2 * T * d * eb + 8 * N * T
     peaks = _peaks()
     tflops_ffn = flops_routed / (t_ffn * 1e-3) / 1e12
     traffic = None
@@ -316,8 +322,11 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "T": T, "d_model": d, "experts": N, "top_k": k, "d_ff": f,
-                       "shared_experts": w.n_shared, "score": "sigmoid+bias", "groups": "8 keep 4",
-                       "capacity": "dropless", "rows_R": R, "parallelism": f"replicas x{world}",
+                       "shared_experts": w.n_shared,
+                       "score": w.score + ("+bias" if w.bias_std > 0 else ""),
+                       "groups": f"{w.n_groups} keep {w.topk_groups}" if w.n_groups > 1 else "none",
+                       "routing": "expert-choice" if w.expert_choice else "token-choice top-k",
+                       "capacity": w.capacity, "rows_R": R, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (x 235 MB, experts 22.5 GB); no flush"},
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
             "roofline": {"kernel": "grouped SwiGLU FFN, routed experts (gate/up + down passes)",

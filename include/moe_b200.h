@@ -271,6 +271,43 @@ int moe_bias_update_seq(const moe_config_t* cfg, const int32_t* topk_idx, const 
                         size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Expert-choice routing: moe_route_scores -> moe_expert_choice -> moe_grouped_ffn
+ * (G = N, offsets from moe_expert_choice) -> moe_combine_ec.
+ *
+ * Defines: the Practice page ("路由的数学形式", last paragraphs: each expert picks its
+ * top-C tokens by its own capacity; perfectly balanced, no capacity drops; not
+ * causal) and the landscape page §0.  Readings: the affinity is the token-choice
+ * router's (softmax or sigmoid of x W_g, no bias, no group limit); equal scores go
+ * to the lower token index; a picked pair's gate weight is its affinity (no
+ * renormalisation); an expert's rows are its picked tokens in ascending order;
+ * the caller chooses C (the plain reading is ceil(cf * k * T / N), k being the
+ * average number of experts per token).
+ * ------------------------------------------------------------------------- */
+
+/* Affinity matrix of the router, expert-major.  scores [N, T] fp32 out;
+ * lse [T] and p_partial [nblk, N] as in moe_route; ws as in moe_route.
+ * cfg->shared_sink must be 0. */
+int moe_route_scores(const moe_config_t* cfg, const void* x, const float* w_gate,
+                     const float* logit_offset, float* scores, float* lse, float* p_partial,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Every expert takes its `capacity` (C, 0 <= C <= T) best tokens.
+ *   scores [N, T] (from moe_route_scores); row_of [N, T] int32 out: row of (e, t)
+ *   in x_perm or -1; token_of_row [N*C] out; offsets [N+1] out (= e*C);
+ *   x_perm [N*C, d] out (x_dtype); n_unpicked [1] int32 or NULL: zeroed here and
+ *   counted by moe_combine_ec (tokens no expert picked). */
+int moe_expert_choice(const moe_config_t* cfg, const void* x, const float* scores, int32_t capacity,
+                      int32_t* row_of, int32_t* token_of_row, int32_t* offsets, void* x_perm,
+                      int32_t* n_unpicked, void* stream);
+
+/* y[t] = shared[t] + sum over experts e that picked t (ascending e) of
+ * scores[e, t] * y_perm[row_of[e, t]]; fp32 accumulation, no atomics on floats.
+ * shared_out [T, d] or NULL; n_unpicked as in moe_expert_choice (or NULL). */
+int moe_combine_ec(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of,
+                   const float* scores, const void* shared_out, void* y, int32_t* n_unpicked,
+                   void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_permute_noalloc -- moe_permute for callers that cannot allocate.
  *
  * The source pages have no counterpart to this call; it exists for deployment.

@@ -534,3 +534,51 @@ def route_shared_sink(x, w_gate_ext, cfg: OracleConfig, bias=None, logit_offset=
     den = sel.sum(axis=1) + s_sh
     return {"logits": z, "s": s, "s_shared": s_sh, "idx": idx, "w": sel / den[:, None],
             "w_shared": s_sh / den, "margin": np.minimum(emargin, gmargin), "lse": logsumexp(z)}
+
+
+# ---------------------------------------------------------------------------
+# Expert-choice routing
+# ---------------------------------------------------------------------------
+def expert_choice_capacity(n_experts: int, top_k: int, T: int, cf: float) -> int:
+    """C = ceil(cf * k * T / N): each expert takes its share of the k T assignments
+    ([Practice] "容量因子、token dropping": C = capacity_factor * k * T / n_experts),
+    at most T."""
+    return min(T, int(np.ceil((cf * top_k * T) / n_experts)))
+
+
+def expert_choice(s: np.ndarray, C: int) -> dict:
+    """Every expert takes the C tokens with the largest affinity.
+
+    [Practice] "路由的数学形式" (last paragraphs) and [Landscape] §0: in expert-choice
+    routing each expert picks its top-C tokens by its own capacity, so every expert
+    is exactly full and no token is dropped by capacity (a token may be picked by no
+    expert, or by several).  Readings: the affinity is the token-choice router's
+    (softmax over experts); equal scores go to the lower token index; the gate weight
+    of a picked pair is its affinity (no renormalisation); an expert's rows are its
+    picked tokens in ascending token order.
+    """
+    T, N = s.shape
+    row_of = np.full((N, T), -1, dtype=np.int64)
+    token_of_row = np.zeros(N * C, dtype=np.int64)
+    for e in range(N):
+        order = np.argsort(-s[:, e], kind="stable")[:C]       # descending, lower token first on ties
+        picked = np.sort(order)
+        for i, t in enumerate(picked):
+            row_of[e, t] = e * C + i
+            token_of_row[e * C + i] = t
+    picks = (row_of >= 0).sum(axis=0)
+    return {"row_of": row_of, "token_of_row": token_of_row, "offsets": np.arange(N + 1) * C,
+            "picks": picks, "unpicked": int((picks == 0).sum())}
+
+
+def expert_choice_combine(y_rows: np.ndarray, row_of: np.ndarray, s: np.ndarray,
+                          shared_out: Optional[np.ndarray]) -> np.ndarray:
+    """y[t] = shared[t] + sum over experts e that picked t of s[t, e] * E_e(x[t])."""
+    N, T = row_of.shape
+    y = np.zeros((T, y_rows.shape[1])) if shared_out is None else np.array(shared_out, np.float64)
+    for t in range(T):
+        for e in range(N):
+            r = row_of[e, t]
+            if r >= 0:
+                y[t] += s[t, e] * y_rows[r]
+    return y

@@ -26,7 +26,7 @@ CAP_DROPLESS, CAP_CEIL_CF_T_OVER_N, CAP_CF_K_T_OVER_N_FLOOR = 0, 1, 2
 EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_route", "moe_permute",
             "moe_grouped_ffn", "moe_combine", "moe_router_stats", "moe_bias_update",
             "moe_device_status", "moe_status_string", "moe_permute_noalloc", "moe_bias_update_ema",
-            "moe_bias_update_seq")
+            "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec")
 
 
 class MoeConfig(ctypes.Structure):
@@ -82,6 +82,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_bias_update": [cfgp, vp, vp, c_float, c_float, vp],
         "moe_bias_update_ema": [cfgp, vp, vp, c_float, vp, c_float, c_float, vp],
         "moe_bias_update_seq": [cfgp, vp, vp, c_int32, vp, c_float, c_float, vp, c_size_t, vp],
+        "moe_route_scores": [cfgp, vp, vp, vp, vp, vp, vp, vp, c_size_t, vp],
+        "moe_expert_choice": [cfgp, vp, vp, c_int32, vp, vp, vp, vp, vp, vp],
+        "moe_combine_ec": [cfgp, vp, vp, vp, vp, vp, vp, vp],
         "moe_device_status": [i32p, c_int32],
         "moe_status_string": [c_int],
     }
@@ -194,6 +197,26 @@ def moe_bias_update_seq(cfg, topk_idx, seq_offsets, n_seq, bias, rate, clamp, ws
     _check("moe_bias_update_seq", load().moe_bias_update_seq(
         ctypes.byref(cfg), _ptr(topk_idx), _ptr(seq_offsets), int(n_seq), _ptr(bias), float(rate),
         float(clamp), _ptr(ws), nbytes, _stream(stream)))
+
+
+def moe_route_scores(cfg, x, w_gate, logit_offset, scores, lse, p_partial, ws, stream=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("moe_route_scores", load().moe_route_scores(
+        ctypes.byref(cfg), _ptr(x), _ptr(w_gate), _ptr(logit_offset), _ptr(scores), _ptr(lse),
+        _ptr(p_partial), _ptr(ws), nbytes, _stream(stream)))
+
+
+def moe_expert_choice(cfg, x, scores, capacity, row_of, token_of_row, offsets, x_perm, n_unpicked=None,
+                      stream=None):
+    _check("moe_expert_choice", load().moe_expert_choice(
+        ctypes.byref(cfg), _ptr(x), _ptr(scores), int(capacity), _ptr(row_of), _ptr(token_of_row),
+        _ptr(offsets), _ptr(x_perm), _ptr(n_unpicked), _stream(stream)))
+
+
+def moe_combine_ec(cfg, y_perm, row_of, scores, shared_out, y, n_unpicked=None, stream=None):
+    _check("moe_combine_ec", load().moe_combine_ec(
+        ctypes.byref(cfg), _ptr(y_perm), _ptr(row_of), _ptr(scores), _ptr(shared_out), _ptr(y),
+        _ptr(n_unpicked), _stream(stream)))
 
 
 def moe_device_status(reset: bool = True) -> int:

@@ -218,6 +218,52 @@ int moe_bias_update_seq(const moe_config_t* cfg, const int32_t* topk_idx, const 
                                           static_cast<double*>(ws), static_cast<cudaStream_t>(stream)));
 }
 
+int moe_route_scores(const moe_config_t* cfg, const void* x, const float* w_gate,
+                     const float* logit_offset, float* scores, float* lse, float* p_partial, void* ws,
+                     size_t ws_bytes, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->shared_sink) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_gate || !scores || !lse || !p_partial) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+  const size_t need = route_workspace_bytes(*cfg);
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && (!ws || !aligned16(ws))) return MOE_ERR_INVALID_ARG;
+  moe_config_t c = *cfg;
+  c.n_groups = 1;
+  return from_cuda(launch_route(c, x, w_gate, logit_offset, nullptr, nullptr, nullptr, lse, p_partial,
+                                nullptr, nullptr, ws, static_cast<cudaStream_t>(stream), scores));
+}
+
+int moe_expert_choice(const moe_config_t* cfg, const void* x, const float* scores, int32_t capacity,
+                      int32_t* row_of, int32_t* token_of_row, int32_t* offsets, void* x_perm,
+                      int32_t* n_unpicked, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (capacity < 0 || (int64_t)capacity > cfg->T) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)capacity * cfg->n_experts > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (!scores || !row_of || !offsets || (capacity > 0 && (!token_of_row || !x_perm || !x)))
+    return MOE_ERR_INVALID_ARG;
+  if (cfg->T == 0) return MOE_ERR_INVALID_ARG;
+  if ((x && !aligned16(x)) || (x_perm && !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_expert_choice(*cfg, x, scores, capacity, row_of, token_of_row, offsets, x_perm,
+                                        n_unpicked, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_combine_ec(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of,
+                   const float* scores, const void* shared_out, void* y, int32_t* n_unpicked,
+                   void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!row_of || !scores || !y || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(y_perm) || (shared_out && !aligned16(shared_out)))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_combine_ec(*cfg, y_perm, row_of, scores, shared_out, y, n_unpicked,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 int moe_device_status(int32_t* status, int32_t reset) {
   if (!status) return MOE_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;

@@ -23,7 +23,15 @@ size_t route_workspace_bytes(const moe_config_t& c);
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* w_gate,
                          const float* logit_offset, const float* bias, int32_t* topk_idx,
                          float* topk_w, float* lse, float* p_partial, float* margin,
-                         float* shared_w, void* ws, cudaStream_t s);
+                         float* shared_w, void* ws, cudaStream_t s, float* scores = nullptr);
+
+// Expert-choice routing (selection + gather, and the per-token combine).
+cudaError_t launch_expert_choice(const moe_config_t& c, const void* x, const float* scores, int C,
+                                 int32_t* row_of, int32_t* token_of_row, int32_t* offsets, void* x_perm,
+                                 int32_t* n_unpicked, cudaStream_t s);
+cudaError_t launch_combine_ec(const moe_config_t& c, const void* y_perm, const int32_t* row_of,
+                              const float* scores, const void* shared_out, void* y, int32_t* n_unpicked,
+                              cudaStream_t s);
 
 // Token-order capacity drop and permutation.
 constexpr int kPermuteTokensPerBlock = 256;

@@ -8,3 +8,4 @@
 #include "ffn_tc.cu"
 #include "ffn_f32.cu"
 #include "combine_stats.cu"
+#include "expert_choice.cu"

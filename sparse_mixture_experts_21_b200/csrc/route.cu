@@ -40,6 +40,7 @@ struct RouteArgs {
   float* margin;
   int sink;            // 1: logit column N scores the shared expert (shared-expert sink)
   float* shared_w;     // [T] weight of the shared expert when sink
+  float* scores;       // [N, T] affinities, expert-major (expert-choice routing); no top-k
 };
 
 // Selection phase: tokens t0 .. t0+TM-1 of the block, logits[tm * ld + e] in
@@ -100,6 +101,14 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
     } else {
 #pragma unroll
       for (int i = 0; i < NV; ++i) pacc[i] += s[i];
+    }
+
+    if (a.scores) {      // expert-choice routing: the affinity matrix, expert-major
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        if (valid[i]) a.scores[(int64_t)(lane + 32 * i) * a.T + t] = s[i];
+      if (lane == 0) a.lse[t] = lse;
+      continue;
     }
 
     // group-limited pre-selection
@@ -602,7 +611,7 @@ size_t route_workspace_bytes(const moe_config_t& c) {
 
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* wg, const float* off,
                          const float* bias, int32_t* idx, float* w, float* lse, float* pp,
-                         float* margin, float* shared_w, void* ws, cudaStream_t s) {
+                         float* margin, float* shared_w, void* ws, cudaStream_t s, float* scores) {
   if (c.T == 0) return cudaSuccess;
   rt::RouteArgs a;
   a.logit_offset = off;
@@ -622,6 +631,7 @@ cudaError_t launch_route(const moe_config_t& c, const void* x, const float* wg, 
   a.margin = margin;
   a.sink = c.shared_sink ? 1 : 0;
   a.shared_w = shared_w;
+  a.scores = scores;
   if (route_uses_tc(c)) {
     switch (route_np(gate_rows(c))) {
       case 8: case 16: return rt::launch_tc<16>(c, x, wg, a, ws, s);

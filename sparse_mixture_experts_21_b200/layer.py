@@ -6,6 +6,7 @@ stream); every step runs in the library's kernels.
 """
 from __future__ import annotations
 
+import math
 from typing import Optional
 
 import torch
@@ -29,6 +30,12 @@ def make_config(w: Workload, T: Optional[int] = None) -> L.MoeConfig:
     c.x_dtype = L.DTYPE_F32 if w.dtype == "fp32" else L.DTYPE_BF16
     c.shared_sink = 1 if w.shared_sink else 0
     return c
+
+
+def ec_capacity(w: Workload, T: Optional[int] = None) -> int:
+    """Expert-choice capacity C = ceil(cf * k * T / N), at most T."""
+    T = w.T if T is None else T
+    return min(T, math.ceil((w.cf * w.k * T) / w.N))
 
 
 class MoELayer:
@@ -74,6 +81,15 @@ class MoELayer:
         self.f_out = z(N)
         self.p_out = z(N)
         self.shared_w = z(max(T, 1)) if w.shared_sink else None
+        if w.expert_choice:
+            C = self.C = ec_capacity(w)
+            self.scores = z(N, max(T, 1))
+            self.row_of = z(N, max(T, 1), dtype=torch.int32)
+            self.token_of_row = z(max(N * C, 1), dtype=torch.int32)
+            self.x_perm = z(max(N * C, 1), d, dtype=dt)
+            self.h = z(max(N * C, 1), w.f, dtype=dt)
+            self.y_perm = z(max(N * C, 1), d, dtype=dt)
+            self.n_unpicked = z(1, dtype=torch.int32)
 
     # the launches of one layer forward; `x` is [T, d] on the device.  `marks`, if
     # given, is a list of 7 CUDA events recorded between the stages (route, permute,
@@ -83,6 +99,8 @@ class MoELayer:
         y = self.y if out is None else out
         s = stream if stream is not None else torch.cuda.current_stream(self.dev)
         rec = (lambda i: marks[i].record(s)) if marks is not None else (lambda i: None)
+        if self.w.expert_choice:
+            return self._forward_ec(x, s, rec, y)
         rec(0)
         L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), self.topk_idx,
                     self.topk_w, self.lse, self.p_partial, self.margin, self.ws, s,
@@ -113,6 +131,30 @@ class MoELayer:
                 with torch.cuda.stream(s):
                     counts = all_reduce_counts(self.counts, self.counts_global, self.group)
             L.moe_bias_update(c, counts, W["bias"], self.w.bias_rate, 0.0, s)
+        rec(6)
+        return y
+
+    def _forward_ec(self, x, s, rec, y):
+        """Expert-choice routing: scores -> per-expert top-C -> grouped FFN -> combine."""
+        W, c, w = self.weights, self.cfg, self.w
+        rec(0)
+        L.moe_route_scores(c, x, W["w_gate"], W.get("logit_offset"), self.scores, self.lse,
+                           self.p_partial, self.ws, s)
+        rec(1)
+        L.moe_expert_choice(c, x, self.scores, self.C, self.row_of, self.token_of_row, self.offsets,
+                            self.x_perm, self.n_unpicked, s)
+        rec(2)
+        L.moe_grouped_ffn(c, self.x_perm, w.N * self.C, self.offsets, w.N, W["w1"], W["w3"], W["w2"],
+                          w.f, self.h, self.y_perm, s)
+        rec(3)
+        shared = None
+        if self.fs > 0:
+            L.moe_grouped_ffn(c, x, w.T, self.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], self.fs,
+                              self.hs, self.ys, s)
+            shared = self.ys
+        rec(4)
+        L.moe_combine_ec(c, self.y_perm, self.row_of, self.scores, shared, y, self.n_unpicked, s)
+        rec(5)
         rec(6)
         return y
 
@@ -160,6 +202,9 @@ class MoELayer:
 
     def kernel_launches(self) -> int:
         """Number of the library's kernels one forward launches."""
+        if self.w.expert_choice:       # scores (+ split), select, gather, FFN (2), combine
+            n = 1 + 2 + 2 + 1 + (1 if self.w.dtype == "bf16" and self.w.N <= 256 else 0)
+            return n + (2 if self.fs > 0 else 0)
         n = 1 + 4 + 2 + 1 + 1          # route, permute (4), routed FFN (2), combine, stats
         if self.w.dtype == "bf16" and self.w.N <= 256:
             n += 1                     # exact bf16 split of the router weight

@@ -47,6 +47,7 @@ class Workload:
     bias_rate: float = 1e-3             # aux-loss-free bias update step
     renorm: bool = True
     shared_sink: bool = False           # the (single) shared expert joins the weight normalisation
+    expert_choice: bool = False         # experts pick their top-C tokens (C = ceil(cf k T / N))
 
     def with_tokens(self, T: int) -> "Workload":
         return replace(self, T=T)
@@ -63,6 +64,10 @@ WORKLOADS = {
                             group_topn=2, bias_std=0.1),
     "switch_skewed": Workload("switch_skewed", T=65536, d=1024, N=128, k=1, f=4096,
                               capacity="ceil_cf_T_over_N", cf=1.0, zipf_s=1.1),
+    # expert-choice routing on the DeepSeekMoE-16B shape: k = 6 experts per token on
+    # average, so each of the 64 experts takes C = 768 tokens
+    "ec_deepseekmoe_16b": Workload("ec_deepseekmoe_16b", T=8192, d=2048, N=64, k=6, f=1408,
+                                   n_shared=2, f_shared=1408, expert_choice=True),
 }
 
 

@@ -104,3 +104,55 @@ def test_bias_update_seq():
     ref = O.bias_update_from_load(np.zeros(N), load, 1e-3)
     assert np.array_equal(f64(bias) != 0, ref != 0)
     assert np.max(np.abs(f64(bias) - ref)) < 1e-9
+
+
+# ----------------------------------------------------------------------------- expert choice
+from sparse_mixture_experts_21_b200.layer import ec_capacity  # noqa: E402
+
+
+@pytest.mark.parametrize("score,dtype", [("softmax", "bf16"), ("sigmoid", "bf16"), ("softmax", "fp32")])
+def test_expert_choice_layer(score, dtype):
+    d = 128 if dtype == "fp32" else 264
+    w = replace(DS_SMALL, score=score, dtype=dtype, d=d, expert_choice=True)
+    lay, inp = _run(w)
+    C = ec_capacity(w)
+    cfg = oracle_cfg(w)
+    s_ref = O.affinity(O.router_logits(f64(inp["x"]), f64(inp["w_gate"])), cfg.score_fn)
+    s_gpu = f64(lay.scores).T                                   # [T, N]
+    assert np.max(np.abs(s_gpu - s_ref)) < 1e-5
+    # the selection, decided on the GPU's own fp32 scores on both sides
+    ec = O.expert_choice(s_gpu, C)
+    assert np.array_equal(i64(lay.row_of), ec["row_of"])
+    assert np.array_equal(i64(lay.token_of_row)[: w.N * C], ec["token_of_row"])
+    assert np.array_equal(i64(lay.offsets), ec["offsets"])
+    assert int(lay.n_unpicked.item()) == ec["unpicked"]
+    # expert rows and the combine against the oracle (fp64 affinities, same selection)
+    off = ec["offsets"]
+    get = expert_weights_fn(inp)
+    y_rows = np.zeros((w.N * C, w.d))
+    for e in range(w.N):
+        y_rows[off[e]:off[e + 1]] = O.swiglu_ffn(f64(inp["x"])[ec["token_of_row"][off[e]:off[e + 1]]], *get(e))
+    assert rel_err(f64(lay.y_perm[: w.N * C]), y_rows) < tol_for(w)
+    ys = O.swiglu_ffn(f64(inp["x"]), *shared_weights(inp))
+    y_ref = O.expert_choice_combine(y_rows, ec["row_of"], s_ref, ys)
+    assert rel_err(f64(lay.y[:w.T]), y_ref) < tol_for(w)
+
+
+def test_expert_choice_ties_and_capacity_edges():
+    """Quantised scores with many exact ties; C = 1 and C = T."""
+    w = replace(DS_SMALL, T=700, N=12, expert_choice=True)
+    c = make_config(w)
+    rng = np.random.default_rng(11)
+    s = (rng.integers(0, 5, size=(w.T, w.N)) / 8.0).astype(np.float32)
+    scores = torch.tensor(s.T.copy(), device="cuda")
+    x = torch.randn(w.T, w.d, device="cuda").to(torch.bfloat16)
+    for C in (1, 37, w.T):
+        row_of = torch.empty(w.N, w.T, dtype=torch.int32, device="cuda")
+        tor = torch.empty(w.N * C, dtype=torch.int32, device="cuda")
+        off = torch.empty(w.N + 1, dtype=torch.int32, device="cuda")
+        xp = torch.empty(w.N * C, w.d, dtype=torch.bfloat16, device="cuda")
+        L.moe_expert_choice(c, x, scores, C, row_of, tor, off, xp)
+        torch.cuda.synchronize()
+        ec = O.expert_choice(s.astype(np.float64), C)
+        assert np.array_equal(i64(row_of), ec["row_of"]) and np.array_equal(i64(tor), ec["token_of_row"])
+        assert torch.equal(xp, x[tor.long()])

@@ -542,3 +542,54 @@ def test_shared_sink_reduces_to_plain_router_and_weights_sum_to_one():
         assert np.array_equal(r2["idx"], plain["idx"])
         if fn == O.SIGMOID:       # sigmoid scores of the routed experts are unchanged
             assert np.allclose(r2["w"], plain["w"], rtol=1e-12) and np.all(r2["w_shared"] < 1e-300)
+
+
+# ---------------------------------------------------------------- expert choice
+def _brute_expert_pick(col, C):
+    """The C-subset of tokens with max score sum, lexicographically smallest."""
+    best, best_sum = None, -math.inf
+    for sub in itertools.combinations(range(len(col)), C):
+        ssum = sum(col[i] for i in sub)
+        if ssum > best_sum:
+            best, best_sum = sub, ssum
+    return list(best)
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_expert_choice_bruteforce(ties):
+    rng = np.random.default_rng(101 + ties)
+    T, N, C = 9, 4, 3
+    s = rng.integers(0, 3, size=(T, N)).astype(np.float64) if ties else rng.random((T, N))
+    ec = O.expert_choice(s, C)
+    for e in range(N):
+        picked = ec["token_of_row"][e * C:(e + 1) * C].tolist()
+        assert picked == _brute_expert_pick(list(s[:, e]), C)
+        assert picked == sorted(picked)
+
+
+def test_expert_choice_balance_and_capacity():
+    rng = np.random.default_rng(103)
+    T, N, k = 200, 8, 2
+    C = O.expert_choice_capacity(N, k, T, 1.0)
+    assert C == 50 and O.expert_choice_capacity(N, k, 10, 8.0) == 10
+    s = O.softmax(rng.normal(size=(T, N)))
+    ec = O.expert_choice(s, C)
+    per_expert = (ec["row_of"] >= 0).sum(axis=1)
+    assert np.all(per_expert == C)                       # perfectly balanced
+    assert ec["picks"].sum() == N * C == k * T
+    assert sorted(ec["row_of"][ec["row_of"] >= 0].tolist()) == list(range(N * C))
+
+
+def test_expert_choice_identical_experts_give_weighted_output():
+    """Identical experts: y_t = (sum of t's picked affinities) * E(x_t)."""
+    rng = np.random.default_rng(107)
+    T, d, f, N = 30, 6, 5, 4
+    x = rng.normal(size=(T, d))
+    w = (rng.normal(size=(f, d)), rng.normal(size=(f, d)), rng.normal(size=(d, f)))
+    s = O.softmax(rng.normal(size=(T, N)))
+    ec = O.expert_choice(s, 12)
+    y_rows = O.swiglu_ffn(x[ec["token_of_row"]], *w)
+    y = O.expert_choice_combine(y_rows, ec["row_of"], s, None)
+    mass = np.where(ec["row_of"].T >= 0, s, 0.0).sum(axis=1)
+    assert np.allclose(y, mass[:, None] * O.swiglu_ffn(x, *w), rtol=1e-12, atol=1e-12)
+    assert np.all(y[ec["picks"] == 0] == 0)
