@@ -284,7 +284,7 @@ def main():
     peaks = _peaks()
     tflops_ffn = flops_routed / (t_ffn * 1e-3) / 1e12
     traffic = None
-    if NCU_TRAFFIC["ffn_tc_sha1"] == _sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc",
+    if w.name == WORKLOAD and NCU_TRAFFIC["ffn_tc_sha1"] == _sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc",
                                                         "ffn_tc.cu")):
         traffic = NCU_TRAFFIC["bytes_per_ffn_call"]
 
@@ -327,7 +327,8 @@ def main():
                        "groups": f"{w.n_groups} keep {w.topk_groups}" if w.n_groups > 1 else "none",
                        "routing": "expert-choice" if w.expert_choice else "token-choice top-k",
                        "capacity": w.capacity, "rows_R": R, "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (x 235 MB, experts 22.5 GB); no flush"},
+                       "l2": (f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "
+                              f"{3 * N * d * f * eb / 1e9:.1f} GB); no flush")},
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
             "roofline": {"kernel": "grouped SwiGLU FFN, routed experts (gate/up + down passes)",
                          "bound": "tensor", "achieved": tflops_ffn,
