@@ -340,6 +340,15 @@ int moe_permute_noalloc(const moe_config_t* cfg, const void* x, const int32_t* t
  * the current device. */
 int moe_device_status(int32_t* status, int32_t reset);
 
+/* Self-test of the device-side failure detection: launches one thread that waits,
+ * through the library's bounded wait, on an mbarrier that can never complete.  The
+ * wait gives up after limit_cycles SM clock cycles (1 .. about 2e9), records
+ * MOE_ERR_DEVICE_TIMEOUT in the device status word (read it with
+ * moe_device_status) and the kernel returns normally, so the context stays usable.
+ * completed [1] int32 device out or NULL: 0 when the wait gave up.  No page defines
+ * this call: it tests the bounded waits every tensor-core kernel uses. */
+int moe_selftest_wait_timeout(int64_t limit_cycles, int32_t* completed, void* stream);
+
 /* Static string for a status code. */
 const char* moe_status_string(int status);
 

@@ -26,7 +26,8 @@ CAP_DROPLESS, CAP_CEIL_CF_T_OVER_N, CAP_CF_K_T_OVER_N_FLOOR = 0, 1, 2
 EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_route", "moe_permute",
             "moe_grouped_ffn", "moe_combine", "moe_router_stats", "moe_bias_update",
             "moe_device_status", "moe_status_string", "moe_permute_noalloc", "moe_bias_update_ema",
-            "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec")
+            "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec",
+            "moe_selftest_wait_timeout")
 
 
 class MoeConfig(ctypes.Structure):
@@ -86,6 +87,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_expert_choice": [cfgp, vp, vp, c_int32, vp, vp, vp, vp, vp, vp],
         "moe_combine_ec": [cfgp, vp, vp, vp, vp, vp, vp, vp],
         "moe_device_status": [i32p, c_int32],
+        "moe_selftest_wait_timeout": [c_int64, vp, vp],
         "moe_status_string": [c_int],
     }
     for name, args in sig.items():
@@ -217,6 +219,11 @@ def moe_combine_ec(cfg, y_perm, row_of, scores, shared_out, y, n_unpicked=None, 
     _check("moe_combine_ec", load().moe_combine_ec(
         ctypes.byref(cfg), _ptr(y_perm), _ptr(row_of), _ptr(scores), _ptr(shared_out), _ptr(y),
         _ptr(n_unpicked), _stream(stream)))
+
+
+def moe_selftest_wait_timeout(limit_cycles, completed=None, stream=None):
+    _check("moe_selftest_wait_timeout", load().moe_selftest_wait_timeout(
+        int(limit_cycles), _ptr(completed), _stream(stream)))
 
 
 def moe_device_status(reset: bool = True) -> int:

@@ -72,6 +72,20 @@ int route_nblk(const moe_config_t& c) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// ever arrives on (its own arrival count is 2 and it arrives once), gives up after
+// `limit` cycles, records MOE_ERR_DEVICE_TIMEOUT and returns normally.
+__global__ void wait_timeout_selftest_kernel(long long limit, int32_t* waited_out) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 2);
+    fence_barrier_init();
+    mbar_arrive(&bar);                        // one of two arrivals: the phase never completes
+    const bool ok = mbar_wait(&bar, 0, limit);
+    if (waited_out) *waited_out = ok ? 1 : 0;
+  }
+}
+
 }  // namespace capi
 }  // namespace moe
 
@@ -262,6 +276,13 @@ int moe_combine_ec(const moe_config_t* cfg, const void* y_perm, const int32_t* r
     return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_combine_ec(*cfg, y_perm, row_of, scores, shared_out, y, n_unpicked,
                                      static_cast<cudaStream_t>(stream)));
+}
+
+int moe_selftest_wait_timeout(int64_t limit_cycles, int32_t* completed, void* stream) {
+  if (limit_cycles <= 0 || limit_cycles > kWaitLimitCycles) return MOE_ERR_INVALID_ARG;
+  capi::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles,
+                                                                                      completed);
+  return from_cuda(cudaGetLastError());
 }
 
 int moe_device_status(int32_t* status, int32_t reset) {
