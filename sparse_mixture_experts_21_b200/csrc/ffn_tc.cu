@@ -373,8 +373,10 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     // ---------------- epilogue: TMEM -> registers -> global
     const int q = warp & 3;                   // TMEM lane quarter of this warp
     if constexpr (PAIR) {
+      // Each warp copies its 32 lanes x 128 columns of an accumulator into registers
+      // behind one wait, releases the accumulator, and only then converts and stores,
+      // so the MMA warp waits for the TMEM copy, not for the global stores.
       const int half = (warp - 2) >> 2;       // column half handled by this warp
-      constexpr int CW = MODE == 0 ? 64 : 128;
       uint32_t use0 = 0, use1 = 0;
       for (int L = blockIdx.x; L < total; L += gridDim.x) {
         const Tile t = decode_tile<PAIR>(L, sh, G, tiles_n, BN);
@@ -383,14 +385,44 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
           uint32_t& use = sub == 0 ? use0 : use1;
           if (!wait_or_abort(&sh->tfull[sub], use & 1u, sh)) { ok = false; break; }
           tc_fence_after();
-          const int r = sub * SUB + q * 32 + lane;
-          const int64_t grow = (int64_t)t.row0 + r;
-          drain<MODE>(tmem_base + ((uint32_t)(q * 32) << 16) + sub * 256u, half * CW, half * CW + CW,
-                      r < t.rows && grow < rows_cap, out + grow * (int64_t)n_out + t.n0, t.n0, n_out);
+          const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + sub * 256u;
+          uint32_t v[128];
+          if (MODE == 0) {             // gate columns [64 h, 64 h + 64) and the matching up columns
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              tmem_ld16(tbase + half * 64 + 16 * j, v + 16 * j);
+              tmem_ld16(tbase + 128 + half * 64 + 16 * j, v + 64 + 16 * j);
+            }
+          } else {                     // output columns [128 h, 128 h + 128)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) tmem_ld16(tbase + half * 128 + 16 * j, v + 16 * j);
+          }
+          tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh->tempty[sub]);
           ++use;
+          const int r = sub * SUB + q * 32 + lane;
+          const int64_t grow = (int64_t)t.row0 + r;
+          if (r < t.rows && grow < rows_cap) {
+            __nv_bfloat16* orow = out + grow * (int64_t)n_out + t.n0;
+            constexpr int NC = MODE == 0 ? 64 : 128;     // output columns of this thread
+            const int c0 = half * NC;
+#pragma unroll
+            for (int j = 0; j < NC; j += 8) {
+              float o[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o[i] = MODE == 0 ? silu_f(__uint_as_float(v[j + i])) * __uint_as_float(v[64 + j + i])
+                                 : __uint_as_float(v[j + i]);
+              if (t.n0 + c0 + j + 8 <= n_out) {
+                uint4 pk;
+                pk.x = pack_bf16x2(o[0], o[1]); pk.y = pack_bf16x2(o[2], o[3]);
+                pk.z = pack_bf16x2(o[4], o[5]); pk.w = pack_bf16x2(o[6], o[7]);
+                stg16(orow + c0 + j, pk);
+              }
+            }
+          }
         }
         if (!ok) break;
       }
