@@ -593,3 +593,65 @@ def test_expert_choice_identical_experts_give_weighted_output():
     mass = np.where(ec["row_of"].T >= 0, s, 0.0).sum(axis=1)
     assert np.allclose(y, mass[:, None] * O.swiglu_ffn(x, *w), rtol=1e-12, atol=1e-12)
     assert np.all(y[ec["picks"] == 0] == 0)
+
+
+# ---------------------------------------------------------------- FP8 (E4M3)
+def test_e4m3_grid_values():
+    # every representable magnitude, built from the definition independently
+    grid = {0.0}
+    for m in range(1, 8):
+        grid.add(m * 2.0 ** -9)                                  # subnormals
+    for e in range(-6, 9):
+        for m in range(8):
+            v = (1 + m / 8) * 2.0 ** e
+            if v <= 448:
+                grid.add(v)
+    grid = np.array(sorted(grid))
+    assert grid[-1] == 448.0 and len(grid) == 127               # 0 + 7 subnormals + 119 normals
+    assert np.array_equal(O.round_e4m3(grid), grid)             # the grid is fixed by rounding
+    assert np.array_equal(O.round_e4m3(-grid), -grid)
+    # midpoints round to the even neighbour (even = last mantissa bit zero)
+    mids = (grid[1:] + grid[:-1]) / 2
+    r = O.round_e4m3(mids)
+    for lo, hi, v in zip(grid[:-1], grid[1:], r):
+        assert v in (lo, hi)
+    assert O.round_e4m3(np.array([1.0625]))[0] == 1.0            # tie between 1 and 1.125 -> even
+    assert O.round_e4m3(np.array([1.1875]))[0] == 1.25           # tie between 1.125 and 1.25 -> even
+    assert O.round_e4m3(np.array([1e6, -500.0]))[0] == 448.0 and O.round_e4m3(np.array([-500.0]))[0] == -448.0
+
+
+def test_e4m3_rounding_error_bound():
+    rng = np.random.default_rng(109)
+    v = rng.normal(scale=30, size=20000)
+    v = v[np.abs(v) <= 448]
+    r = O.round_e4m3(v)
+    normal = np.abs(v) >= 2.0 ** -6
+    assert np.all(np.abs(r - v)[normal] <= 2.0 ** -4 * np.abs(v)[normal] * (1 + 1e-12))
+    assert np.all(np.abs(r - v)[~normal] <= 2.0 ** -10)
+
+
+def test_fp8_block_quantisation():
+    rng = np.random.default_rng(113)
+    x = rng.normal(size=(5, 256)).astype(np.float32)
+    x[2, 128:] = 0.0                                             # an all-zero block -> scale 1
+    q, s = O.quantize_fp8_blocks(x, 1)
+    assert s.shape == (5, 2) and s[2, 1] == 1.0
+    assert np.all(np.abs(q) <= 448) and np.max(np.abs(q[0, :128])) == 448.0
+    xd = O.dequantize_fp8_blocks(q, s, 1)
+    assert np.all(np.abs(xd - x) <= 2.0 ** -4 * np.abs(x) + 2.0 ** -9 * np.repeat(s, 128, axis=1))
+    w = rng.normal(size=(256, 384)).astype(np.float32)
+    qw, sw = O.quantize_fp8_blocks(w, 128)
+    assert sw.shape == (2, 3)
+    assert np.allclose(sw, [[np.max(np.abs(w[i:i + 128, j:j + 128])) / 448 for j in (0, 128, 256)]
+                            for i in (0, 128)], rtol=1e-6)
+
+
+def test_fp8_ffn_close_to_exact():
+    """FP8 expert output within a few percent of the exact one (E4M3 keeps 3 bits)."""
+    rng = np.random.default_rng(127)
+    x = rng.normal(size=(16, 256))
+    w1, w3 = rng.normal(size=(256, 256)) / 16, rng.normal(size=(256, 256)) / 16
+    w2 = rng.normal(size=(256, 256)) / 16
+    exact = O.swiglu_ffn(x, w1, w3, w2)
+    err = np.max(np.abs(O.swiglu_ffn_fp8(x, w1, w3, w2) - exact)) / np.max(np.abs(exact))
+    assert 1e-4 < err < 0.08
