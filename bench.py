@@ -117,6 +117,14 @@ def _device_uuid(dev):
         return None
 
 
+def _oracle_cfg(O, w):
+    cap = {"dropless": O.CAP_DROPLESS, "ceil_cf_T_over_N": O.CAP_CEIL_CF_T_OVER_N,
+           "floor_cf_k_T_over_N": O.CAP_CF_K_T_OVER_N_FLOOR}[w.capacity]
+    return O.OracleConfig(n_experts=w.N, top_k=w.k, score_fn=O.SIGMOID if w.score == "sigmoid" else O.SOFTMAX,
+                          renorm=w.renorm, n_groups=w.n_groups, topk_groups=w.topk_groups,
+                          group_score_topn=w.group_topn, capacity_mode=cap, capacity_factor=w.cf)
+
+
 # ---------------------------------------------------------------------------- reference arm
 def run_reference(args, rank):
     """The fp64 CPU oracle on a bounded sample of the workload, host cores."""
@@ -125,15 +133,15 @@ def run_reference(args, rank):
     from oracle import moe_oracle as O
     from sparse_mixture_experts_21_b200.synth import WORKLOADS, make_inputs
 
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
     sample = args.ref_tokens
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(w, dev)
-    cfg = O.OracleConfig(n_experts=w.N, top_k=w.k, score_fn=O.SIGMOID, n_groups=w.n_groups,
-                         topk_groups=w.topk_groups, group_score_topn=w.group_topn)
+    cfg = _oracle_cfg(O, w)
     f64 = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
-    wg, bias = f64(inp["w_gate"]), f64(inp["bias"])
-    shared = (f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"]))
+    wg, bias, off = f64(inp["w_gate"]), f64(inp["bias"]), f64(inp["logit_offset"])
+    shared = (f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"])) if w.n_shared else None
+    ffn = O.swiglu_ffn_fp8 if w.fp8 else None
 
     def experts(e):
         return f64(inp["w1"][e]), f64(inp["w3"][e]), f64(inp["w2"][e])
@@ -141,7 +149,8 @@ def run_reference(args, rank):
     def step(i):
         t0 = (i * sample) % w.T
         x = f64(inp["x"][t0:t0 + sample])
-        O.layer_forward(x, wg, cfg, experts, shared, bias=bias, alpha=w.alpha, z_coef=w.z_coef)
+        O.layer_forward(x, wg, cfg, experts, shared, bias=bias, logit_offset=off, alpha=w.alpha,
+                        z_coef=w.z_coef, expert_ffn=ffn)
 
     for i in range(args.warmup):
         step(i)
@@ -155,10 +164,10 @@ def run_reference(args, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "T": w.T, "d_model": w.d, "experts": w.N, "top_k": w.k,
+            "config": {"workload": w.name, "T": w.T, "d_model": w.d, "experts": w.N, "top_k": w.k,
                        "d_ff": w.f, "shared": w.n_shared, "sample_tokens_per_step": sample},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{sample} tokens per step of the {WORKLOAD} workload "
+                             "sample": f"{sample} tokens per step of the {w.name} workload "
                                        f"(full routing, experts, shared expert, combine, stats)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -169,11 +178,11 @@ def run_reference(args, rank):
 def cpu_baseline(inp, w, seconds_target=20.0):
     """Oracle timed on a bounded sample (a few tokens of the same workload)."""
     from oracle import moe_oracle as O
-    cfg = O.OracleConfig(n_experts=w.N, top_k=w.k, score_fn=O.SIGMOID, n_groups=w.n_groups,
-                         topk_groups=w.topk_groups, group_score_topn=w.group_topn)
+    cfg = _oracle_cfg(O, w)
     f64 = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
-    wg, bias = f64(inp["w_gate"]), f64(inp["bias"])
-    shared = (f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"]))
+    wg, bias, off = f64(inp["w_gate"]), f64(inp["bias"]), f64(inp["logit_offset"])
+    shared = (f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"])) if w.n_shared else None
+    ffn = O.swiglu_ffn_fp8 if w.fp8 else None
 
     def experts(e):
         return f64(inp["w1"][e]), f64(inp["w3"][e]), f64(inp["w2"][e])
@@ -182,13 +191,14 @@ def cpu_baseline(inp, w, seconds_target=20.0):
     chunk = 4
     while True:
         x = f64(inp["x"][done:done + chunk])
-        O.layer_forward(x, wg, cfg, experts, shared, bias=bias, alpha=w.alpha, z_coef=w.z_coef)
+        O.layer_forward(x, wg, cfg, experts, shared, bias=bias, logit_offset=off, alpha=w.alpha,
+                        z_coef=w.z_coef, expert_ffn=ffn)
         done += chunk
         el = time.perf_counter() - t0
         if el > seconds_target or done >= 64:
             break
     return {"value": done / el, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-            "sample": f"first {done} tokens of the {WORKLOAD} workload, {chunk} per oracle call "
+            "sample": f"first {done} tokens of the {w.name} workload, {chunk} per oracle call "
                       f"(routing, experts, shared expert, combine, stats), {el:.1f} s"}
 
 
@@ -277,11 +287,16 @@ def main():
     bytes_route = T * d * eb + 4 * N * d + 8 * T * k
     bytes_perm = T * d * eb + R * d * eb + 12 * T * k
     bytes_comb = R * d * eb + 2 * T * d * eb + 8 * T * k
+    if w.fp8:                  # bf16 x read once; E4M3 codes + 1x128 scales written per row (+ token order)
+        bytes_perm = T * d * eb + (R + (T if lay.fs else 0)) * d * (1 + 4 / 128) + 12 * T * k
     if w.expert_choice:        # scores [N, T] written; rows gathered per row; combine reads the maps
         bytes_route = T * d * eb + 4 * N * d + 4 * N * T
         bytes_perm = 2 * R * d * eb + 12 * N * T
         bytes_comb = R * d * eb + 2 * T * d * eb + 8 * N * T
     peaks = _peaks()
+    # E4M3 operands: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    ffn_peak = peaks["bf16_tflops_sustained"] * (2.0 if w.fp8 else 1.0)
+    ffn_peak_src = peaks["source"] + (" sustained bf16 x 2 (nominal fp8/bf16 ratio)" if w.fp8 else " sustained bf16")
     tflops_ffn = flops_routed / (t_ffn * 1e-3) / 1e12
     traffic = None
     if w.name == WORKLOAD and NCU_TRAFFIC["ffn_tc_sha1"] == _sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc",
@@ -320,21 +335,23 @@ def main():
         line = {
             "metric": METRIC, "value": world * T / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 experts, fp32 router" if w.fp8 else "bf16",
+            "data": "synthetic",
             "config": {"workload": w.name, "T": T, "d_model": d, "experts": N, "top_k": k, "d_ff": f,
                        "shared_experts": w.n_shared,
                        "score": w.score + ("+bias" if w.bias_std > 0 else ""),
                        "groups": f"{w.n_groups} keep {w.topk_groups}" if w.n_groups > 1 else "none",
                        "routing": "expert-choice" if w.expert_choice else "token-choice top-k",
                        "capacity": w.capacity, "rows_R": R, "parallelism": f"replicas x{world}",
+                       "experts_precision": "E4M3, 1x128 / 128x128 block scales" if w.fp8 else "bf16",
                        "l2": (f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "
-                              f"{3 * N * d * f * eb / 1e9:.1f} GB); no flush")},
+                              f"{3 * N * d * f * (1 if w.fp8 else eb) / 1e9:.1f} GB); no flush")},
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
             "roofline": {"kernel": "grouped SwiGLU FFN, routed experts (gate/up + down passes)",
                          "bound": "tensor", "achieved": tflops_ffn,
-                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": tflops_ffn / peaks["bf16_tflops_sustained"], "traffic": traffic,
-                         "peak_source": peaks["source"] + " sustained bf16"},
+                         "peak": ffn_peak, "unit": "TFLOP/s",
+                         "frac": tflops_ffn / ffn_peak, "traffic": traffic,
+                         "peak_source": ffn_peak_src},
             "stages_ms": {"route": t_route, "permute": t_perm, "routed_ffn": t_ffn,
                           "shared_ffn": t_shared, "combine": t_comb, "stats_bias": t_stats},
             "hbm": {"route_gbs": bytes_route / (t_route * 1e-3) / 1e9,

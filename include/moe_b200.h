@@ -163,7 +163,8 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate,
  *   token_of_row [T*k] int32 out: token of each row (entries >= R untouched)
  *   x_perm       [T*k, d] x_dtype out: x_perm[row] = x[token_of_row[row]]
  *                (rows >= R untouched); rows of expert e are its kept slots in
- *                ascending token order
+ *                ascending token order.  NULL skips the gather (x may then be
+ *                NULL too), e.g. when moe_permute_fp8 fills FP8 rows instead
  *   n_dropped    [2] int32 out: {dropped slots, tokens with all k slots dropped}
  *   ws           scratch of at least moe_workspace_size() bytes (contents on
  *                entry ignored; clobbered)
@@ -197,6 +198,62 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_rows, int64_t rows_ca
                     const int32_t* offsets, int32_t G,
                     const void* w1, const void* w3, const void* w2, int32_t f,
                     void* h_scratch, void* y_rows, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * FP8 expert compute with fine-grained block scaling.
+ *
+ * Defines: the MoE common-taste page, section 2 (its table lists FP8 / MXFP8 expert
+ * compute as a strong candidate), and the Practice page "精度怎么定" (matmuls in
+ * FP8 with fine-grained precision assignment, the router kept at higher
+ * precision).  The pages give no scheme; the reading used is the DeepSeek-V3 one:
+ * E4M3 codes (OCP FP8, bias 7, max 448, no infinities), one fp32 scale per 1 x 128
+ * block of activations and per 128 x 128 block of weights, scale = amax / 448
+ * (1 for an all-zero block), code = E4M3(x / scale) rounded to nearest even with
+ * saturation, x / scale in fp32.  The router (moe_route) is unchanged.
+ * ------------------------------------------------------------------------- */
+
+/* moe_quantize_fp8 -- block-quantise a bf16 matrix.
+ *   x          [rows, cols] bf16 (device), cols % 128 == 0
+ *   block_rows 1 (activations: 1 x 128 blocks) or 128 (weights: 128 x 128 blocks)
+ *   q          [rows, cols] uint8 E4M3 codes out
+ *   scales     [ceil(rows / block_rows), cols / 128] fp32 out
+ * Stacked expert weights [G, f, d] are passed as rows = G * f; with f % 128 == 0
+ * no block spans two experts.  Errors: MOE_ERR_INVALID_ARG for a bad shape, a
+ * NULL or misaligned pointer (x, q 16-byte; scales 4-byte). */
+int moe_quantize_fp8(const void* x, int64_t rows, int32_t cols, int32_t block_rows, uint8_t* q,
+                     float* scales, void* stream);
+
+/* moe_permute_fp8 -- quantise x (1 x 128 blocks) and scatter it into expert rows.
+ * Each token's row is read and quantised once; its codes and scales are written
+ * to every row the permutation gave it (row_of_slot from moe_permute, which may
+ * be called with x_perm = NULL to skip its own bf16 gather) and, when xq is not
+ * NULL, to row t of token-order buffers (the shared experts' input).
+ *   x           [T, d] bf16, d % 128 == 0
+ *   row_of_slot [T, k] int32 or NULL (token-order output only)
+ *   xq_perm     [rows, d] uint8 out, xs_perm [rows, d / 128] fp32 out
+ *   xq, xs      [T, d] uint8 and [T, d / 128] fp32 out, or NULL
+ * Errors: MOE_ERR_UNSUPPORTED unless x is bf16 with d % 128 == 0;
+ * MOE_ERR_INVALID_ARG for NULL or misaligned buffers. */
+int moe_permute_fp8(const moe_config_t* cfg, const void* x, const int32_t* row_of_slot, uint8_t* xq_perm,
+                    float* xs_perm, uint8_t* xq, float* xs, void* stream);
+
+/* moe_grouped_ffn_fp8 -- the grouped SwiGLU FFN of moe_grouped_ffn on E4M3 codes.
+ *   xq_rows, xs_rows  [rows_cap, d] codes, [rows_cap, d / 128] scales
+ *   offsets           [G+1] int32 (device), as for moe_grouped_ffn
+ *   w1q/w1s, w3q/w3s  [G f, d] codes, [G f / 128, d / 128] scales
+ *   w2q/w2s           [G d, f] codes, [G d / 128, f / 128] scales
+ *   hq/hs_scratch     [rows_cap, f] codes, [rows_cap, f / 128] scales (written, read)
+ *   y_rows            [rows_cap, d] bf16 out (rows >= offsets[G] untouched)
+ * Tensor cores (E4M3 x E4M3, fp32 accumulation) over one 128-wide K block at a
+ * time; the two block scales are applied in fp32 as each block is accumulated.
+ * h = silu(W1 x) * (W3 x) is computed in fp32 and re-quantised in 1 x 128 blocks.
+ * Errors: MOE_ERR_UNSUPPORTED unless bf16 config with d % 128 == f % 128 == 0;
+ * MOE_ERR_INVALID_ARG for G outside [1, 512], NULL or misaligned buffers. */
+int moe_grouped_ffn_fp8(const moe_config_t* cfg, const uint8_t* xq_rows, const float* xs_rows,
+                        int64_t rows_cap, const int32_t* offsets, int32_t G, const uint8_t* w1q,
+                        const float* w1s, const uint8_t* w3q, const float* w3s, const uint8_t* w2q,
+                        const float* w2s, int32_t f, uint8_t* hq_scratch, float* hs_scratch, void* y_rows,
+                        void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_combine -- y[t] = shared[t] + sum_{j: row >= 0} w[t,j] * y_perm[row(t,j)].

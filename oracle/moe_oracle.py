@@ -423,7 +423,7 @@ def layer_forward(x: np.ndarray, w_gate: np.ndarray, cfg: OracleConfig,
                   bias=None, logit_offset=None,
                   alpha: float = 0.0, z_coef: float = 0.0,
                   tokens: Optional[Sequence[int]] = None,
-                  routing: Optional[dict] = None) -> dict:
+                  routing: Optional[dict] = None, expert_ffn=None) -> dict:
     """The layer forward in the pages' order: route, capacity/drop, permute,
     expert FFNs (+ shared), combine, statistics.
 
@@ -431,9 +431,11 @@ def layer_forward(x: np.ndarray, w_gate: np.ndarray, cfg: OracleConfig,
     large layers can widen one expert at a time.  `tokens`, when given, restricts
     the expert compute and combine to those tokens (routing, capacity and
     statistics still see every token).  `routing` lets a test feed a fixed
-    routing decision (idx, w) instead of recomputing it.
+    routing decision (idx, w) instead of recomputing it.  `expert_ffn(x_rows, w1,
+    w3, w2)` replaces the exact SwiGLU expert (e.g. swiglu_ffn_fp8).
     """
     T, d = x.shape
+    ffn = swiglu_ffn if expert_ffn is None else expert_ffn
     r = route(x, w_gate, cfg, bias, logit_offset) if routing is None else routing
     C = capacity(cfg, T)
     p = permutation(r["idx"], cfg.n_experts, C)
@@ -441,7 +443,7 @@ def layer_forward(x: np.ndarray, w_gate: np.ndarray, cfg: OracleConfig,
     want_set = set(int(t) for t in want)
     y = np.zeros((len(want), d))
     if shared_weights is not None:
-        y += swiglu_ffn(np.asarray(x, np.float64)[want], *shared_weights)
+        y += ffn(np.asarray(x, np.float64)[want], *shared_weights)
     pos_in_want = {int(t): i for i, t in enumerate(want)}
     # gather, per expert, the rows (token, slot) that belong to wanted tokens
     for e in range(cfg.n_experts):
@@ -450,7 +452,7 @@ def layer_forward(x: np.ndarray, w_gate: np.ndarray, cfg: OracleConfig,
         if not rows:
             continue
         toks = p["token_of_row"][rows]
-        ye = swiglu_ffn(np.asarray(x, np.float64)[toks], *expert_weights(e))
+        ye = ffn(np.asarray(x, np.float64)[toks], *expert_weights(e))
         for i, rr in enumerate(rows):
             t = int(p["token_of_row"][rr])
             j = int(np.nonzero(p["row_of_slot"][t] == rr)[0][0])
@@ -611,7 +613,8 @@ def round_e4m3(v: np.ndarray) -> np.ndarray:
 def quantize_fp8_blocks(x: np.ndarray, block_rows: int, block_cols: int = 128) -> tuple:
     """Fine-grained FP8 quantisation: one scale per block_rows x block_cols block.
 
-    [Taste] §3 lists FP8 / MXFP8 expert compute as a strong candidate and [Practice]
+    [Taste] §2 (table of common taste vs frontier) lists FP8 / MXFP8 expert compute
+    as a strong candidate and [Practice]
     "精度怎么定" says DeepSeek-V3 trains in FP8 with fine-grained precision assignment,
     without giving the scheme.  Reading (the DeepSeek-V3 one): 1 x 128 blocks for
     activations, 128 x 128 for weights; scale s = amax / 448 computed in fp32

@@ -27,7 +27,7 @@ EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_rou
             "moe_grouped_ffn", "moe_combine", "moe_router_stats", "moe_bias_update",
             "moe_device_status", "moe_status_string", "moe_permute_noalloc", "moe_bias_update_ema",
             "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec",
-            "moe_selftest_wait_timeout")
+            "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8")
 
 
 class MoeConfig(ctypes.Structure):
@@ -89,6 +89,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_device_status": [i32p, c_int32],
         "moe_selftest_wait_timeout": [c_int64, vp, vp],
         "moe_status_string": [c_int],
+        "moe_quantize_fp8": [vp, c_int64, c_int32, c_int32, vp, vp, vp],
+        "moe_permute_fp8": [cfgp, vp, vp, vp, vp, vp, vp, vp],
+        "moe_grouped_ffn_fp8": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, c_int32, vp, vp,
+                                vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -167,6 +171,27 @@ def moe_grouped_ffn(cfg, x_rows, rows_cap, offsets, G, w1, w3, w2, f, h_scratch,
     _check("moe_grouped_ffn", load().moe_grouped_ffn(
         ctypes.byref(cfg), _ptr(x_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1), _ptr(w3),
         _ptr(w2), int(f), _ptr(h_scratch), _ptr(y_rows), _stream(stream)))
+
+
+def moe_quantize_fp8(x, block_rows, q, scales, stream=None):
+    """Block-quantise a bf16 matrix [rows, cols] to E4M3 codes (uint8) and fp32 scales."""
+    rows, cols = x.shape
+    _check("moe_quantize_fp8", load().moe_quantize_fp8(
+        _ptr(x), int(rows), int(cols), int(block_rows), _ptr(q), _ptr(scales), _stream(stream)))
+
+
+def moe_permute_fp8(cfg, x, row_of_slot, xq_perm, xs_perm, xq=None, xs=None, stream=None):
+    _check("moe_permute_fp8", load().moe_permute_fp8(
+        ctypes.byref(cfg), _ptr(x), _ptr(row_of_slot), _ptr(xq_perm), _ptr(xs_perm), _ptr(xq), _ptr(xs),
+        _stream(stream)))
+
+
+def moe_grouped_ffn_fp8(cfg, xq_rows, xs_rows, rows_cap, offsets, G, w1q, w1s, w3q, w3s, w2q, w2s, f,
+                        hq_scratch, hs_scratch, y_rows, stream=None):
+    _check("moe_grouped_ffn_fp8", load().moe_grouped_ffn_fp8(
+        ctypes.byref(cfg), _ptr(xq_rows), _ptr(xs_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1q),
+        _ptr(w1s), _ptr(w3q), _ptr(w3s), _ptr(w2q), _ptr(w2s), int(f), _ptr(hq_scratch), _ptr(hs_scratch),
+        _ptr(y_rows), _stream(stream)))
 
 
 def moe_combine(cfg, y_perm, row_of_slot, topk_w, shared_out, y, stream=None, shared_w=None):

@@ -142,9 +142,9 @@ int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
   const int st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (!counts || !offsets || !n_dropped) return MOE_ERR_INVALID_ARG;
-  if (cfg->T > 0 && (!x || !topk_idx || !row_of_slot || !token_of_row || !x_perm))
+  if (cfg->T > 0 && (!topk_idx || !row_of_slot || !token_of_row || (x_perm && !x)))
     return MOE_ERR_INVALID_ARG;
-  if (cfg->T > 0 && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && x_perm && (!aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
   const size_t need = permute_workspace_bytes(*cfg);
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (need > 0 && (!ws || !aligned16(ws))) return MOE_ERR_INVALID_ARG;
@@ -174,6 +174,60 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_rows, int64_t rows_ca
                                   static_cast<const float*>(w1), static_cast<const float*>(w3),
                                   static_cast<const float*>(w2), d, f, static_cast<float*>(h_scratch),
                                   static_cast<float*>(y_rows), s));
+}
+
+int moe_quantize_fp8(const void* x, int64_t rows, int32_t cols, int32_t block_rows, uint8_t* q,
+                     float* scales, void* stream) {
+  if (rows < 0 || cols <= 0 || (cols % 128) != 0 || (block_rows != 1 && block_rows != 128))
+    return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!x || !q || !scales || !aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+    return MOE_ERR_INVALID_ARG;
+  if (block_rows == 128 && (rows + 127) / 128 * (cols / 128) > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  return from_cuda(launch_quantize_fp8(x, rows, cols, block_rows, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_permute_fp8(const moe_config_t* cfg, const void* x, const int32_t* row_of_slot, uint8_t* xq_perm,
+                    float* xs_perm, uint8_t* xq, float* xs, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->x_dtype != MOE_DTYPE_BF16 || (cfg->d_model % 128) != 0) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (row_of_slot && (!xq_perm || !xs_perm)) return MOE_ERR_INVALID_ARG;
+  if (!row_of_slot && !xq) return MOE_ERR_INVALID_ARG;
+  if ((xq && !xs) || (xq_perm && !aligned16(xq_perm)) || (xq && !aligned16(xq)))
+    return MOE_ERR_INVALID_ARG;
+  if ((xs_perm && (reinterpret_cast<uintptr_t>(xs_perm) & 3u)) || (xs && (reinterpret_cast<uintptr_t>(xs) & 3u)))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_quant_scatter(x, cfg->T, row_of_slot ? cfg->top_k : 0, cfg->d_model, row_of_slot,
+                                        xq_perm, xs_perm, xq, xs, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_grouped_ffn_fp8(const moe_config_t* cfg, const uint8_t* xq_rows, const float* xs_rows,
+                        int64_t rows_cap, const int32_t* offsets, int32_t G, const uint8_t* w1q,
+                        const float* w1s, const uint8_t* w3q, const float* w3s, const uint8_t* w2q,
+                        const float* w2s, int32_t f, uint8_t* hq_scratch, float* hs_scratch, void* y_rows,
+                        void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (rows_cap < 0 || G < 1 || G > 512 || f <= 0) return MOE_ERR_INVALID_ARG;
+  if (cfg->x_dtype != MOE_DTYPE_BF16 || (cfg->d_model % 128) != 0 || (f % 128) != 0)
+    return MOE_ERR_UNSUPPORTED;
+  if (!offsets) return MOE_ERR_INVALID_ARG;
+  if (rows_cap == 0) return MOE_OK;
+  if (rows_cap > (int64_t)INT32_MAX || (int64_t)G * cfg->d_model > (int64_t)INT32_MAX ||
+      (int64_t)G * f > (int64_t)INT32_MAX)
+    return MOE_ERR_UNSUPPORTED;
+  if (!xq_rows || !xs_rows || !w1q || !w1s || !w3q || !w3s || !w2q || !w2s || !hq_scratch || !hs_scratch ||
+      !y_rows)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq_rows) || !aligned16(w1q) || !aligned16(w3q) || !aligned16(w2q) || !aligned16(hq_scratch) ||
+      !aligned16(y_rows))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_ffn_fp8(xq_rows, xs_rows, rows_cap, offsets, G, w1q, w1s, w3q, w3s, w2q, w2s,
+                                  cfg->d_model, f, hq_scratch, hs_scratch, y_rows,
+                                  static_cast<cudaStream_t>(stream)));
 }
 
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of_slot,

@@ -13,6 +13,7 @@ namespace moe {
 // Row-major bf16 matrix [rows, cols] as a TMA tensor map: box = 64 columns x
 // box_rows rows, 128-byte swizzle, zero fill out of bounds.
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // Padded expert count, tokens per block and scratch of the fused router.
 int route_np(int n_experts);
@@ -65,6 +66,15 @@ cudaError_t launch_bias_update_seq(const moe_config_t& c, const int32_t* topk_id
                                    const int32_t* seq_offsets, int n_seq, float* bias, float rate,
                                    float clamp, double* ws, cudaStream_t s);
 
+cudaError_t launch_quantize_fp8(const void* x, int64_t rows, int cols, int block_rows, uint8_t* q,
+                                float* scales, cudaStream_t s);
+cudaError_t launch_quant_scatter(const void* x, int64_t T, int k, int d, const int32_t* row_of_slot,
+                                 uint8_t* xq_perm, float* xs_perm, uint8_t* xq_tok, float* xs_tok,
+                                 cudaStream_t s);
+cudaError_t launch_ffn_fp8(const uint8_t* xq, const float* xs, int64_t rows_cap, const int32_t* offsets, int G,
+                           const uint8_t* w1q, const float* w1s, const uint8_t* w3q, const float* w3s,
+                           const uint8_t* w2q, const float* w2s, int d, int f, uint8_t* hq, float* hs,
+                           void* y, cudaStream_t s);
 int sm_count();
 
 }  // namespace moe

@@ -9,3 +9,4 @@
 #include "ffn_f32.cu"
 #include "combine_stats.cu"
 #include "expert_choice.cu"
+#include "ffn_fp8.cu"

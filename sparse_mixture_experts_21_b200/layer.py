@@ -76,6 +76,8 @@ class MoELayer:
             self.hs = z(max(T, 1), self.fs, dtype=dt)
             self.ys = z(max(T, 1), d, dtype=dt)
         self.y = z(max(T, 1), d, dtype=dt)
+        if w.fp8:
+            self._init_fp8(z)
         self.stats = torch.zeros(L.STATS_BYTES, dtype=torch.uint8, device=self.dev)
         self.counts_global = z(N, dtype=torch.int32)
         self.f_out = z(N)
@@ -90,6 +92,35 @@ class MoELayer:
             self.h = z(max(N * C, 1), w.f, dtype=dt)
             self.y_perm = z(max(N * C, 1), d, dtype=dt)
             self.n_unpicked = z(1, dtype=torch.int32)
+
+    def _init_fp8(self, z):
+        """FP8 experts: quantise the weights once (128 x 128 blocks) and hold E4M3
+        buffers for the permuted rows, the hidden rows and the shared experts' input
+        in place of the bf16 ones."""
+        w, W, T, d, N, k = self.w, self.weights, self.w.T, self.w.d, self.w.N, self.w.k
+        u8 = torch.uint8
+
+        def quant_w(t):
+            m = t.reshape(-1, t.shape[-1])
+            q = z(m.shape[0], m.shape[1], dtype=u8)
+            sc = z((m.shape[0] + 127) // 128, m.shape[1] // 128)
+            L.moe_quantize_fp8(m, 128, q, sc)
+            return q, sc
+
+        self.wq = {name: quant_w(W[name]) for name in ("w1", "w3", "w2")}
+        rows = max(T * k, 1)
+        self.x_perm = self.h = None
+        self.xq_perm, self.xs_perm = z(rows, d, dtype=u8), z(rows, d // 128)
+        self.hq, self.hsc = z(rows, w.f, dtype=u8), z(rows, w.f // 128)
+        if self.fs > 0:
+            self.wq.update({name: quant_w(W[name]) for name in ("ws1", "ws3", "ws2")})
+            self.xq, self.xs = z(max(T, 1), d, dtype=u8), z(max(T, 1), d // 128)
+            self.hq_sh, self.hsc_sh = z(max(T, 1), self.fs, dtype=u8), z(max(T, 1), self.fs // 128)
+            self.hs = None
+
+    def _ffn_fp8(self, c, xq, xs, rows, offsets, G, names, f, hq, hsc, y, s):
+        (w1q, w1s), (w3q, w3s), (w2q, w2s) = (self.wq[n] for n in names)
+        L.moe_grouped_ffn_fp8(c, xq, xs, rows, offsets, G, w1q, w1s, w3q, w3s, w2q, w2s, f, hq, hsc, y, s)
 
     # the launches of one layer forward; `x` is [T, d] on the device.  `marks`, if
     # given, is a list of 7 CUDA events recorded between the stages (route, permute,
@@ -106,16 +137,28 @@ class MoELayer:
                     self.topk_w, self.lse, self.p_partial, self.margin, self.ws, s,
                     shared_w=self.shared_w)
         rec(1)
+        fp8 = self.w.fp8
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
                       self.token_of_row, self.x_perm, self.n_dropped, self.ws, s)
+        if fp8:
+            L.moe_permute_fp8(c, x, self.row_of_slot, self.xq_perm, self.xs_perm,
+                              self.xq if self.fs > 0 else None, self.xs if self.fs > 0 else None, s)
         rec(2)
-        L.moe_grouped_ffn(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
-                          W["w2"], self.w.f, self.h, self.y_perm, s)
+        if fp8:
+            self._ffn_fp8(c, self.xq_perm, self.xs_perm, T * self.w.k, self.offsets, self.w.N,
+                          ("w1", "w3", "w2"), self.w.f, self.hq, self.hsc, self.y_perm, s)
+        else:
+            L.moe_grouped_ffn(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
+                              W["w2"], self.w.f, self.h, self.y_perm, s)
         rec(3)
         shared = None
         if self.fs > 0:
-            L.moe_grouped_ffn(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], self.fs,
-                              self.hs, self.ys, s)
+            if fp8:
+                self._ffn_fp8(c, self.xq, self.xs, T, self.shared_offsets, 1, ("ws1", "ws3", "ws2"),
+                              self.fs, self.hq_sh, self.hsc_sh, self.ys, s)
+            else:
+                L.moe_grouped_ffn(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"],
+                                  self.fs, self.hs, self.ys, s)
             shared = self.ys
         rec(4)
         L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, y, s,
@@ -206,6 +249,7 @@ class MoELayer:
             n = 1 + 2 + 2 + 1 + (1 if self.w.dtype == "bf16" and self.w.N <= 256 else 0)
             return n + (2 if self.fs > 0 else 0)
         n = 1 + 4 + 2 + 1 + 1          # route, permute (4), routed FFN (2), combine, stats
+        # FP8: the permutation's bf16 gather is replaced by the quantising scatter
         if self.w.dtype == "bf16" and self.w.N <= 256:
             n += 1                     # exact bf16 split of the router weight
         if self.fs > 0:

@@ -13,6 +13,7 @@ temporary) and rounded to the storage dtype.  The Switch-style workload adds the
 fixed per-expert logit offset o[e] = -1.1 * ln(e + 1), the log of an unnormalised
 Zipf(s = 1.1) weight, so expert 0 is the hottest.
 With the shared-expert sink, W_g has one extra (last) row scoring the shared expert.
+FP8 workloads draw the same bf16 tensors; the layer quantises them.
 """
 from __future__ import annotations
 
@@ -48,6 +49,7 @@ class Workload:
     renorm: bool = True
     shared_sink: bool = False           # the (single) shared expert joins the weight normalisation
     expert_choice: bool = False         # experts pick their top-C tokens (C = ceil(cf k T / N))
+    fp8: bool = False                   # expert matmuls on E4M3 codes with fine-grained block scales
 
     def with_tokens(self, T: int) -> "Workload":
         return replace(self, T=T)
@@ -68,6 +70,11 @@ WORKLOADS = {
     # average, so each of the 64 experts takes C = 768 tokens
     "ec_deepseekmoe_16b": Workload("ec_deepseekmoe_16b", T=8192, d=2048, N=64, k=6, f=1408,
                                    n_shared=2, f_shared=1408, expert_choice=True),
+    # the DeepSeek-V3 shape with every expert matmul (routed and shared) in FP8: bf16
+    # x and weights drawn as above, quantised by the layer (1 x 128 / 128 x 128 blocks)
+    "deepseek_v3_fp8": Workload("deepseek_v3_fp8", T=16384, d=7168, N=256, k=8, f=2048, n_shared=1,
+                                f_shared=2048, score="sigmoid", n_groups=8, topk_groups=4,
+                                group_topn=2, bias_std=0.1, fp8=True),
 }
 
 
