@@ -37,7 +37,7 @@ UNIT = "tokens/s"
 
 # DRAM traffic of the dominant kernels per launch from an ncu capture, valid only
 # while the kernel source is the one that was profiled (sha1 of ffn_tc.cu).
-NCU_TRAFFIC = {"ffn_tc_sha1": "8d1acdedbd6775bb2d08630abb529ca4d3b07a7e", "bytes_per_ffn_call": 35.8e9}
+NCU_TRAFFIC = {"ffn_tc_sha1": "20e1efc02dee7b5fd27a4663f5e984a52ae4205d", "bytes_per_ffn_call": 35.7e9}
 
 
 def _peaks():
