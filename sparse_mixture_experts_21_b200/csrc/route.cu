@@ -354,13 +354,16 @@ route_simt_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate, in
 // ============================================================================
 // The tensor cores' fp32 accumulation truncates, so one long accumulation over
 // K = 3 d would bias the logits towards zero (about 1e-5 relative at d = 4096).
-// Each 64-wide K block therefore starts a fresh TMEM accumulator, and drain warps
-// add the block result into fp32 registers with round-to-nearest: the truncation
-// then spans the 4 MMA steps of one block only.  K blocks run in the order
-// (d-tile, piece), so each x tile is fetched from DRAM once and reused from L2.
+// Each group of TC_ACC_GROUP 64-wide K blocks therefore starts a fresh TMEM
+// accumulator, and drain warps add the group's result into fp32 registers with
+// round-to-nearest: the truncation then spans the 16 MMA steps of one group only
+// (a bias of order 16 / (3 d / 16) of the single-accumulator one).  K blocks run in
+// the order (d-tile, piece), so each x tile is fetched from DRAM once and reused
+// from L2.
 constexpr int TC_TM = 128;          // tokens per CTA (MMA M)
 constexpr int TC_BK = 64;           // K per stage: one 128-byte swizzle row of bf16
 constexpr int TC_STAGES = 4;
+constexpr int TC_ACC_GROUP = 4;     // K blocks per fresh accumulator
 constexpr int TC_THREADS = 384;     // warp 0 TMA, warp 1 MMA, warps 4..11 drain; all 12 select
 constexpr int TC_WARPS = TC_THREADS / 32;
 
@@ -479,9 +482,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
       constexpr uint32_t idesc = umma_idesc_bf16(TC_TM, NP < 16 ? 16 : NP);
       uint32_t stage = 0, phase = 0;
       for (int kb = 0; kb < nkb; ++kb) {
-        const int buf = kb % S::NBUF;
-        const uint32_t use = (uint32_t)(kb / S::NBUF) & 1u;
-        if (!bounded_wait(&tempty[buf], use ^ 1u)) break;
+        const int grp = kb / TC_ACC_GROUP;
+        const bool first = kb % TC_ACC_GROUP == 0;
+        const bool last = kb % TC_ACC_GROUP == TC_ACC_GROUP - 1 || kb == nkb - 1;
+        const int buf = grp % S::NBUF;
+        const uint32_t use = (uint32_t)(grp / S::NBUF) & 1u;
+        if (first && !bounded_wait(&tempty[buf], use ^ 1u)) break;
         if (!bounded_wait(&full[stage], phase)) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + (size_t)stage * S::STAGE_BYTES);
@@ -490,9 +496,9 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
         for (int kk = 0; kk < TC_BK / 16; ++kk)
           umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
-                   idesc, kk != 0 ? 1u : 0u);
+                   idesc, (kk != 0 || !first) ? 1u : 0u);
         umma_commit(&empty[stage]);
-        umma_commit(&tfull[buf]);
+        if (last) umma_commit(&tfull[buf]);
         if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
       }
     }
@@ -504,9 +510,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
 #pragma unroll
     for (int i = 0; i < S::CPW; ++i) acc[i] = 0.f;
     bool ok = true;
-    for (int kb = 0; kb < nkb && ok; ++kb) {
-      const int buf = kb % S::NBUF;
-      const uint32_t use = (uint32_t)(kb / S::NBUF) & 1u;
+    const int ngrp = (nkb + TC_ACC_GROUP - 1) / TC_ACC_GROUP;
+    for (int grp = 0; grp < ngrp && ok; ++grp) {
+      const int buf = grp % S::NBUF;
+      const uint32_t use = (uint32_t)(grp / S::NBUF) & 1u;
       ok = bounded_wait(&tfull[buf], use);
       if (!ok) break;
       tc_fence_after();
