@@ -653,3 +653,53 @@ def swiglu_ffn_fp8(x_rows, w1, w3, w2, hidden_out: bool = False):
     hq, hs = quantize_fp8_blocks(h, 1)
     y = dequantize_fp8_blocks(hq, hs, 1) @ wd[2].T
     return (y, h) if hidden_out else y
+
+
+# ---------------------------------------------------------------------------
+# MXFP8 (OCP Microscaling) experts
+# ---------------------------------------------------------------------------
+MX_BLOCK = 32
+E4M3_EMAX = 8          # exponent of E4M3's largest normal (448 = 1.75 * 2^8)
+
+
+def quantize_mxfp8(x: np.ndarray, block: int = MX_BLOCK) -> tuple:
+    """MXFP8 quantisation along each row: every `block` consecutive elements share
+    one E8M0 scale 2^e.
+
+    [Taste] §2 (table) names MXFP8 expert compute.  The format is the OCP
+    Microscaling (MX) one: scale exponent e = floor(log2(amax)) - emax(E4M3), with
+    emax(E4M3) = 8, clamped to the E8M0 range [-127, 127]; elements are
+    E4M3(x / 2^e), saturating at 448 (a block's largest magnitude lands in
+    [256, 512), so it may saturate).  An all-zero block takes e = -127.
+    floor(log2(amax)) comes from frexp, which is exact.
+    Returns (dequantisable codes as float64 values, exponents e [rows, cols/block] int).
+    """
+    x = np.asarray(x, np.float64)
+    R, C = x.shape
+    nb = C // block
+    q = np.zeros((R, C))
+    e = np.full((R, nb), -127, np.int64)
+    for i in range(R):
+        for j in range(nb):
+            blk = x[i, j * block:(j + 1) * block]
+            amax = np.max(np.abs(blk))
+            if amax > 0:
+                _, ex = np.frexp(amax)                 # amax = m 2^ex, m in [0.5, 1)
+                e[i, j] = min(127, max(-127, int(ex) - 1 - E4M3_EMAX))
+            q[i, j * block:(j + 1) * block] = round_e4m3(blk / 2.0 ** e[i, j])
+    return q, e
+
+
+def dequantize_mxfp8(q: np.ndarray, e: np.ndarray, block: int = MX_BLOCK) -> np.ndarray:
+    return np.asarray(q, np.float64) * np.repeat(2.0 ** np.asarray(e, np.float64), block, axis=1)
+
+
+def swiglu_ffn_mxfp8(x_rows, w1, w3, w2, hidden_out: bool = False):
+    """The SwiGLU expert with MXFP8 operands: x, W1, W3 quantised along d and W2
+    and h along d_ff (the contraction dimension, 1 x 32 blocks); fp64 products of
+    the dequantised values."""
+    xd = dequantize_mxfp8(*quantize_mxfp8(x_rows))
+    w1d, w3d, w2d = (dequantize_mxfp8(*quantize_mxfp8(w)) for w in (w1, w3, w2))
+    h = silu(xd @ w1d.T) * (xd @ w3d.T)
+    y = dequantize_mxfp8(*quantize_mxfp8(h)) @ w2d.T
+    return (y, h) if hidden_out else y

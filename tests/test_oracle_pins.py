@@ -655,3 +655,65 @@ def test_fp8_ffn_close_to_exact():
     exact = O.swiglu_ffn(x, w1, w3, w2)
     err = np.max(np.abs(O.swiglu_ffn_fp8(x, w1, w3, w2) - exact)) / np.max(np.abs(exact))
     assert 1e-4 < err < 0.08
+
+
+# ----------------------------------------------------------------------------- MXFP8
+def _e4m3_grid():
+    g = {0.0}
+    for m in range(1, 8):
+        g.add(m * 2.0 ** -9)
+    for ex in range(-6, 9):
+        for m in range(8):
+            v = (1 + m / 8) * 2.0 ** ex
+            if v <= 448:
+                g.add(v)
+    return np.array(sorted(g))
+
+
+def test_mxfp8_scale_hand_cases():
+    x = np.zeros((4, 64))
+    x[0, :32] = 1.0                       # amax 1 -> e = -8, codes 256
+    x[0, 32:] = 448.0                     # amax 448 -> e = 0, codes 448
+    x[1, :32] = np.linspace(-3.0, 3.0, 32)  # amax 3 -> floor(log2 3) = 1 -> e = -7
+    x[1, 32] = 500.0                      # amax 500 -> e = 0, 500 saturates to 448
+    x[2, 5] = 2.0 ** -130                 # tiny amax -> e clamps at -127
+    # row 3 all zero -> e = -127
+    q, e = O.quantize_mxfp8(x)
+    assert e.tolist() == [[-8, 0], [-7, 0], [-127, -127], [-127, -127]]
+    assert np.all(q[0, :32] == 256.0) and np.all(q[0, 32:] == 448.0)
+    assert q[1, 32] == 448.0
+    assert np.all(O.dequantize_mxfp8(q, e)[3] == 0.0)
+    # amax / 2^e lies in [256, 512) for every non-zero, unclamped block
+    rng = np.random.default_rng(131)
+    y = rng.normal(scale=rng.uniform(1e-3, 1e3, size=(40, 1)), size=(40, 128))
+    qy, ey = O.quantize_mxfp8(y)
+    amax = np.abs(y).reshape(40, 4, 32).max(axis=2)
+    ratio = amax / 2.0 ** ey
+    assert np.all((ratio >= 256.0) & (ratio < 512.0))
+
+
+def test_mxfp8_codes_on_grid_and_error_bound():
+    rng = np.random.default_rng(137)
+    x = rng.standard_t(3, size=(64, 256)) * rng.uniform(0.01, 100, size=(64, 1))
+    q, e = O.quantize_mxfp8(x)
+    grid = _e4m3_grid()
+    assert np.all(np.isin(np.abs(q), grid))        # every code is an E4M3 value
+    xs = np.abs(x) / np.repeat(2.0 ** e, 32, axis=1)
+    ok = xs <= 448.0                               # not saturated
+    err = np.abs(O.dequantize_mxfp8(q, e) - x)
+    bound = 2.0 ** -4 * np.abs(x) + np.repeat(2.0 ** (e - 10), 32, axis=1)
+    assert np.all(err[ok] <= bound[ok] * (1 + 1e-12))
+    # saturated elements are clamped to 448 with the sign kept
+    assert np.all(np.abs(q[~ok]) == 448.0) and np.all(np.sign(q[~ok]) == np.sign(x[~ok]))
+
+
+def test_mxfp8_ffn_close_to_exact():
+    rng = np.random.default_rng(139)
+    x = rng.normal(size=(16, 256))
+    w1, w3 = rng.normal(scale=256 ** -0.5, size=(2, 128, 256))
+    w2 = rng.normal(scale=128 ** -0.5, size=(256, 128))
+    y, h = O.swiglu_ffn_mxfp8(x, w1, w3, w2, hidden_out=True)
+    y0 = O.swiglu_ffn(x, w1, w3, w2)
+    assert np.max(np.abs(y - y0)) / np.max(np.abs(y0)) < 0.1
+    h0 = O.silu(x @ w1.T) * (x @ w3.T)
+    assert np.max(np.abs(h - h0)) / np.max(np.abs(h0)) < 0.1
