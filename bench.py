@@ -141,7 +141,7 @@ def run_reference(args, rank):
     f64 = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
     wg, bias, off = f64(inp["w_gate"]), f64(inp["bias"]), f64(inp["logit_offset"])
     shared = (f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"])) if w.n_shared else None
-    ffn = O.swiglu_ffn_fp8 if w.fp8 else None
+    ffn = O.swiglu_ffn_fp8 if w.fp8 else (O.swiglu_ffn_mxfp8 if w.mxfp8 else None)
 
     def experts(e):
         return f64(inp["w1"][e]), f64(inp["w3"][e]), f64(inp["w2"][e])
@@ -182,7 +182,7 @@ def cpu_baseline(inp, w, seconds_target=20.0):
     f64 = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
     wg, bias, off = f64(inp["w_gate"]), f64(inp["bias"]), f64(inp["logit_offset"])
     shared = (f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"])) if w.n_shared else None
-    ffn = O.swiglu_ffn_fp8 if w.fp8 else None
+    ffn = O.swiglu_ffn_fp8 if w.fp8 else (O.swiglu_ffn_mxfp8 if w.mxfp8 else None)
 
     def experts(e):
         return f64(inp["w1"][e]), f64(inp["w3"][e]), f64(inp["w2"][e])
@@ -287,16 +287,18 @@ def main():
     bytes_route = T * d * eb + 4 * N * d + 8 * T * k
     bytes_perm = T * d * eb + R * d * eb + 12 * T * k
     bytes_comb = R * d * eb + 2 * T * d * eb + 8 * T * k
-    if w.fp8:                  # bf16 x read once; E4M3 codes + 1x128 scales written per row (+ token order)
-        bytes_perm = T * d * eb + (R + (T if lay.fs else 0)) * d * (1 + 4 / 128) + 12 * T * k
+    lowp = w.fp8 or w.mxfp8
+    if lowp:                   # bf16 x read once; E4M3 codes + scales written per row (+ token order)
+        sf_per_elem = 4 / 128 if w.fp8 else 1 / 32
+        bytes_perm = T * d * eb + (R + (T if lay.fs else 0)) * d * (1 + sf_per_elem) + 12 * T * k
     if w.expert_choice:        # scores [N, T] written; rows gathered per row; combine reads the maps
         bytes_route = T * d * eb + 4 * N * d + 4 * N * T
         bytes_perm = 2 * R * d * eb + 12 * N * T
         bytes_comb = R * d * eb + 2 * T * d * eb + 8 * N * T
     peaks = _peaks()
     # E4M3 operands: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
-    ffn_peak = peaks["bf16_tflops_sustained"] * (2.0 if w.fp8 else 1.0)
-    ffn_peak_src = peaks["source"] + (" sustained bf16 x 2 (nominal fp8/bf16 ratio)" if w.fp8 else " sustained bf16")
+    ffn_peak = peaks["bf16_tflops_sustained"] * (2.0 if lowp else 1.0)
+    ffn_peak_src = peaks["source"] + (" sustained bf16 x 2 (nominal fp8/bf16 ratio)" if lowp else " sustained bf16")
     tflops_ffn = flops_routed / (t_ffn * 1e-3) / 1e12
     traffic = None
     if w.name == WORKLOAD and NCU_TRAFFIC["ffn_tc_sha1"] == _sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc",
@@ -335,7 +337,8 @@ def main():
         line = {
             "metric": METRIC, "value": world * T / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 experts, fp32 router" if w.fp8 else "bf16",
+            "scaling": "weak", "vs_baseline": None, "dtype": ("mxfp8-e4m3 experts, fp32 router" if w.mxfp8 else
+                                                              "fp8-e4m3 experts, fp32 router" if w.fp8 else "bf16"),
             "data": "synthetic",
             "config": {"workload": w.name, "T": T, "d_model": d, "experts": N, "top_k": k, "d_ff": f,
                        "shared_experts": w.n_shared,
@@ -343,9 +346,10 @@ def main():
                        "groups": f"{w.n_groups} keep {w.topk_groups}" if w.n_groups > 1 else "none",
                        "routing": "expert-choice" if w.expert_choice else "token-choice top-k",
                        "capacity": w.capacity, "rows_R": R, "parallelism": f"replicas x{world}",
-                       "experts_precision": "E4M3, 1x128 / 128x128 block scales" if w.fp8 else "bf16",
+                       "experts_precision": ("E4M3, 1x128 / 128x128 block scales" if w.fp8 else
+                                             "MXFP8: E4M3, E8M0 scale per 32 along K" if w.mxfp8 else "bf16"),
                        "l2": (f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "
-                              f"{3 * N * d * f * (1 if w.fp8 else eb) / 1e9:.1f} GB); no flush")},
+                              f"{3 * N * d * f * (1 if lowp else eb) / 1e9:.1f} GB); no flush")},
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
             "roofline": {"kernel": "grouped SwiGLU FFN, routed experts (gate/up + down passes)",
                          "bound": "tensor", "achieved": tflops_ffn,

@@ -256,6 +256,70 @@ int moe_grouped_ffn_fp8(const moe_config_t* cfg, const uint8_t* xq_rows, const f
                         void* stream);
 
 /* ---------------------------------------------------------------------------
+ * MXFP8 expert compute (OCP Microscaling FP8).
+ *
+ * Defines: the MoE common-taste page, section 2 (its table names MXFP8 expert
+ * compute).  Format: E4M3 codes; every 32 consecutive elements along a row (the
+ * contraction dimension of the GEMM operand) share one E8M0 scale byte b, value
+ * 2^(b - 127), with b - 127 = floor(log2 amax) - 8 clamped to [-127, 127]
+ * (b = 0 for an all-zero block); code = E4M3(x / 2^(b - 127)), round to nearest
+ * even, saturating at 448.  The tensor cores apply the scales inside the MMA
+ * (block-scaled MMA).
+ *
+ * Scale layout ("tile atoms", the order the GEMM consumes them in): the rows of
+ * an operand are cut into tiles of 128 -- for rows grouped by expert (offsets),
+ * tile i of group g starts at row offsets[g] + 128 i and the tiles are numbered
+ * in group order; a plain matrix is one group.  The scales of tile t and 128-wide
+ * K block kb fill the 512-byte atom at byte (t * (cols / 128) + kb) * 512; row m
+ * of the tile, scale j of the K block (elements 128 kb + 32 j .. + 31) is at byte
+ * 16 (m mod 32) + 4 floor(m / 32) + j of the atom.  A buffer for `rows` rows in G
+ * groups needs (ceil(rows / 128) + G) * (cols / 128) * 512 bytes (plain matrix:
+ * ceil(rows / 128) * (cols / 128) * 512); bytes of rows past a group's end are
+ * unspecified.
+ * ------------------------------------------------------------------------- */
+
+/* moe_quantize_mxfp8 -- quantise a bf16 matrix along its rows.
+ *   x   [rows, cols] bf16 (device, 16-byte aligned), cols % 128 == 0
+ *   q   [rows, cols] uint8 E4M3 codes out (8-byte aligned)
+ *   sf  E8M0 scales out, tile atoms of the plain matrix (layout above)
+ * Expert weights [G, f, d] are quantised as rows = G * f (blocks never span rows).
+ * Errors: MOE_ERR_INVALID_ARG for a bad shape or a NULL or misaligned pointer. */
+int moe_quantize_mxfp8(const void* x, int64_t rows, int32_t cols, uint8_t* q, uint8_t* sf, void* stream);
+
+/* moe_permute_mxfp8 -- moe_permute_fp8 with MXFP8 rows: each token's row is read
+ * and quantised once and written (codes and scales) to every kept row given by
+ * row_of_slot and, when q is not NULL, to row t of token-order buffers.
+ *   x            [T, d] bf16, d % 128 == 0
+ *   topk_idx     [T, k] int32 (the experts of the slots)
+ *   row_of_slot  [T, k] int32 from moe_permute, or NULL (token order only)
+ *   offsets      [N+1] int32 from moe_permute (the groups of the tile-atom layout)
+ *   q_perm       [T*k, d] codes out; sf_perm: scales out, tile atoms grouped by offsets
+ *   q, sf        [T, d] codes and plain-matrix tile atoms out, or NULL
+ * Errors: MOE_ERR_UNSUPPORTED unless bf16 with d % 128 == 0 and N <= 1024;
+ * MOE_ERR_INVALID_ARG for NULL or misaligned buffers. */
+int moe_permute_mxfp8(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const int32_t* row_of_slot,
+                      const int32_t* offsets, uint8_t* q_perm, uint8_t* sf_perm, uint8_t* q, uint8_t* sf,
+                      void* stream);
+
+/* moe_grouped_ffn_mxfp8 -- the grouped SwiGLU FFN of moe_grouped_ffn on MXFP8 operands.
+ *   xq_rows, xsf_rows  [rows_cap, d] codes; scales as tile atoms grouped by offsets
+ *   offsets            [G+1] int32 (device), as for moe_grouped_ffn
+ *   w1q/w1sf, w3q/w3sf [G f, d] codes; scales as plain-matrix tile atoms
+ *   w2q/w2sf           [G d, f] codes; scales as plain-matrix tile atoms
+ *   hq/hsf_scratch     [rows_cap, f] codes; scales as tile atoms grouped by offsets
+ *                      (written by the first pass, read by the second)
+ *   y_rows             [rows_cap, d] bf16 out (rows >= offsets[G] untouched)
+ * One fp32 TMEM accumulator over the whole K range (block-scaled tcgen05 MMA);
+ * h = silu(W1 x) * (W3 x) in fp32, re-quantised to MXFP8 along f.
+ * Errors: MOE_ERR_UNSUPPORTED unless a bf16 config with d % 128 == f % 128 == 0;
+ * MOE_ERR_INVALID_ARG for G outside [1, 512], NULL or misaligned (16-byte) buffers. */
+int moe_grouped_ffn_mxfp8(const moe_config_t* cfg, const uint8_t* xq_rows, const uint8_t* xsf_rows,
+                          int64_t rows_cap, const int32_t* offsets, int32_t G, const uint8_t* w1q,
+                          const uint8_t* w1sf, const uint8_t* w3q, const uint8_t* w3sf, const uint8_t* w2q,
+                          const uint8_t* w2sf, int32_t f, uint8_t* hq_scratch, uint8_t* hsf_scratch,
+                          void* y_rows, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_combine -- y[t] = shared[t] + sum_{j: row >= 0} w[t,j] * y_perm[row(t,j)].
  *
  * Defines: llm-compass "稀疏门控与 Top-k 路由" (y = sum_i g_i E_i(x)) and the Practice

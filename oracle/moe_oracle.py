@@ -676,17 +676,12 @@ def quantize_mxfp8(x: np.ndarray, block: int = MX_BLOCK) -> tuple:
     """
     x = np.asarray(x, np.float64)
     R, C = x.shape
-    nb = C // block
-    q = np.zeros((R, C))
-    e = np.full((R, nb), -127, np.int64)
-    for i in range(R):
-        for j in range(nb):
-            blk = x[i, j * block:(j + 1) * block]
-            amax = np.max(np.abs(blk))
-            if amax > 0:
-                _, ex = np.frexp(amax)                 # amax = m 2^ex, m in [0.5, 1)
-                e[i, j] = min(127, max(-127, int(ex) - 1 - E4M3_EMAX))
-            q[i, j * block:(j + 1) * block] = round_e4m3(blk / 2.0 ** e[i, j])
+    blocks = x.reshape(R, C // block, block)
+    amax = np.max(np.abs(blocks), axis=2)
+    _, ex = np.frexp(amax)                         # amax = m 2^ex, m in [0.5, 1)
+    e = np.where(amax > 0, ex.astype(np.int64) - 1 - E4M3_EMAX, -127)
+    e = np.clip(e, -127, 127)
+    q = round_e4m3(blocks / (2.0 ** e)[:, :, None]).reshape(R, C)
     return q, e
 
 

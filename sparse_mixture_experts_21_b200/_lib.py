@@ -27,7 +27,8 @@ EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_rou
             "moe_grouped_ffn", "moe_combine", "moe_router_stats", "moe_bias_update",
             "moe_device_status", "moe_status_string", "moe_permute_noalloc", "moe_bias_update_ema",
             "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec",
-            "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8")
+            "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
+            "moe_quantize_mxfp8", "moe_permute_mxfp8", "moe_grouped_ffn_mxfp8")
 
 
 class MoeConfig(ctypes.Structure):
@@ -93,6 +94,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_permute_fp8": [cfgp, vp, vp, vp, vp, vp, vp, vp],
         "moe_grouped_ffn_fp8": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, c_int32, vp, vp,
                                 vp, vp],
+        "moe_quantize_mxfp8": [vp, c_int64, c_int32, vp, vp, vp],
+        "moe_permute_mxfp8": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "moe_grouped_ffn_mxfp8": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, c_int32, vp, vp,
+                                  vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +196,57 @@ def moe_grouped_ffn_fp8(cfg, xq_rows, xs_rows, rows_cap, offsets, G, w1q, w1s, w
     _check("moe_grouped_ffn_fp8", load().moe_grouped_ffn_fp8(
         ctypes.byref(cfg), _ptr(xq_rows), _ptr(xs_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1q),
         _ptr(w1s), _ptr(w3q), _ptr(w3s), _ptr(w2q), _ptr(w2s), int(f), _ptr(hq_scratch), _ptr(hs_scratch),
+        _ptr(y_rows), _stream(stream)))
+
+
+def mx_scales(rows: int, cols: int, device, groups: int = 0) -> torch.Tensor:
+    """Buffer for MXFP8 scales in tile-atom order: rows cut into 128-row tiles (per group
+    when `groups` > 0), one 512-byte atom per (tile, 128-wide K block)."""
+    tiles = (rows + 127) // 128 + groups
+    return torch.empty(max(tiles, 1) * (cols // 128) * 512, dtype=torch.uint8, device=device)
+
+
+def mx_scales_rowmajor(sf, rows: int, cols: int, offsets=None):
+    """Tile atoms -> numpy [rows, cols / 32] scale bytes (rows grouped by `offsets`, a
+    sequence of G + 1 row offsets, or one plain group)."""
+    import numpy as np
+    a = sf.cpu().numpy() if hasattr(sf, "cpu") else np.asarray(sf)
+    nkb = cols // 128
+    off = [0, rows] if offsets is None else [int(o) for o in offsets]
+    out = np.zeros((rows, cols // 32), np.uint8)
+    tile = 0
+    m = np.arange(128)
+    pos = 16 * (m % 32) + 4 * (m // 32)
+    for g in range(len(off) - 1):
+        for r0 in range(off[g], off[g + 1], 128):
+            n = min(128, off[g + 1] - r0)
+            for kb in range(nkb):
+                atom = a[(tile * nkb + kb) * 512:(tile * nkb + kb + 1) * 512]
+                for j in range(4):
+                    out[r0:r0 + n, 4 * kb + j] = atom[pos[:n] + j]
+            tile += 1
+    return out
+
+
+def moe_quantize_mxfp8(x, q, sf, stream=None):
+    """MXFP8-quantise a bf16 matrix [rows, cols] along its rows: E4M3 codes and E8M0 scales
+    (sf from mx_scales(rows, cols))."""
+    rows, cols = x.shape
+    _check("moe_quantize_mxfp8", load().moe_quantize_mxfp8(
+        _ptr(x), int(rows), int(cols), _ptr(q), _ptr(sf), _stream(stream)))
+
+
+def moe_permute_mxfp8(cfg, x, topk_idx, row_of_slot, offsets, q_perm, sf_perm, q=None, sf=None, stream=None):
+    _check("moe_permute_mxfp8", load().moe_permute_mxfp8(
+        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(row_of_slot), _ptr(offsets), _ptr(q_perm),
+        _ptr(sf_perm), _ptr(q), _ptr(sf), _stream(stream)))
+
+
+def moe_grouped_ffn_mxfp8(cfg, xq_rows, xsf_rows, rows_cap, offsets, G, w1q, w1sf, w3q, w3sf, w2q, w2sf, f,
+                          hq_scratch, hsf_scratch, y_rows, stream=None):
+    _check("moe_grouped_ffn_mxfp8", load().moe_grouped_ffn_mxfp8(
+        ctypes.byref(cfg), _ptr(xq_rows), _ptr(xsf_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1q),
+        _ptr(w1sf), _ptr(w3q), _ptr(w3sf), _ptr(w2q), _ptr(w2sf), int(f), _ptr(hq_scratch), _ptr(hsf_scratch),
         _ptr(y_rows), _stream(stream)))
 
 

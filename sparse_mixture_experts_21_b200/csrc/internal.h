@@ -75,6 +75,15 @@ cudaError_t launch_ffn_fp8(const uint8_t* xq, const float* xs, int64_t rows_cap,
                            const uint8_t* w1q, const float* w1s, const uint8_t* w3q, const float* w3s,
                            const uint8_t* w2q, const float* w2s, int d, int f, uint8_t* hq, float* hs,
                            void* y, cudaStream_t s);
+cudaError_t launch_mx_quant_rows(const void* x, int64_t rows, int cols, uint8_t* q, uint8_t* sf,
+                                 cudaStream_t s);
+cudaError_t launch_mx_quant_scatter(const void* x, int64_t T, int k, int d, int N, const int32_t* topk_idx,
+                                    const int32_t* row_of_slot, const int32_t* offsets, uint8_t* q_perm,
+                                    uint8_t* sf_perm, uint8_t* q_tok, uint8_t* sf_tok, cudaStream_t s);
+cudaError_t launch_ffn_mx(const uint8_t* xq, const uint8_t* xsf, int64_t rows_cap, const int32_t* offsets, int G,
+                          const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w3q, const uint8_t* w3sf,
+                          const uint8_t* w2q, const uint8_t* w2sf, int d, int f, uint8_t* hq, uint8_t* hsf,
+                          void* y, cudaStream_t s);
 int sm_count();
 
 }  // namespace moe

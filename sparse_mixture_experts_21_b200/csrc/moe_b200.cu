@@ -10,3 +10,4 @@
 #include "combine_stats.cu"
 #include "expert_choice.cu"
 #include "ffn_fp8.cu"
+#include "ffn_mx.cu"

@@ -76,7 +76,7 @@ class MoELayer:
             self.hs = z(max(T, 1), self.fs, dtype=dt)
             self.ys = z(max(T, 1), d, dtype=dt)
         self.y = z(max(T, 1), d, dtype=dt)
-        if w.fp8:
+        if w.fp8 or w.mxfp8:
             self._init_fp8(z)
         self.stats = torch.zeros(L.STATS_BYTES, dtype=torch.uint8, device=self.dev)
         self.counts_global = z(N, dtype=torch.int32)
@@ -94,33 +94,43 @@ class MoELayer:
             self.n_unpicked = z(1, dtype=torch.int32)
 
     def _init_fp8(self, z):
-        """FP8 experts: quantise the weights once (128 x 128 blocks) and hold E4M3
+        """FP8 experts: quantise the weights once (fine-grained: 128 x 128 blocks with
+        fp32 scales; MXFP8: 1 x 32 blocks along K with E8M0 scales) and hold E4M3
         buffers for the permuted rows, the hidden rows and the shared experts' input
         in place of the bf16 ones."""
         w, W, T, d, N, k = self.w, self.weights, self.w.T, self.w.d, self.w.N, self.w.k
         u8 = torch.uint8
+        mx = w.mxfp8
+        # scales of grouped (permuted) rows: MXFP8 tile atoms need one spare tile per group
+        sfa = (lambda rows, cols, groups=0: L.mx_scales(rows, cols, self.dev, groups)) if mx else \
+            (lambda rows, cols, groups=0: z(rows, cols // 128))
 
         def quant_w(t):
             m = t.reshape(-1, t.shape[-1])
             q = z(m.shape[0], m.shape[1], dtype=u8)
-            sc = z((m.shape[0] + 127) // 128, m.shape[1] // 128)
-            L.moe_quantize_fp8(m, 128, q, sc)
+            if mx:
+                sc = L.mx_scales(m.shape[0], m.shape[1], self.dev)
+                L.moe_quantize_mxfp8(m, q, sc)
+            else:
+                sc = z((m.shape[0] + 127) // 128, m.shape[1] // 128)
+                L.moe_quantize_fp8(m, 128, q, sc)
             return q, sc
 
         self.wq = {name: quant_w(W[name]) for name in ("w1", "w3", "w2")}
         rows = max(T * k, 1)
         self.x_perm = self.h = None
-        self.xq_perm, self.xs_perm = z(rows, d, dtype=u8), z(rows, d // 128)
-        self.hq, self.hsc = z(rows, w.f, dtype=u8), z(rows, w.f // 128)
+        self.xq_perm, self.xs_perm = z(rows, d, dtype=u8), sfa(rows, d, N)
+        self.hq, self.hsc = z(rows, w.f, dtype=u8), sfa(rows, w.f, N)
         if self.fs > 0:
             self.wq.update({name: quant_w(W[name]) for name in ("ws1", "ws3", "ws2")})
-            self.xq, self.xs = z(max(T, 1), d, dtype=u8), z(max(T, 1), d // 128)
-            self.hq_sh, self.hsc_sh = z(max(T, 1), self.fs, dtype=u8), z(max(T, 1), self.fs // 128)
+            self.xq, self.xs = z(max(T, 1), d, dtype=u8), sfa(max(T, 1), d)
+            self.hq_sh, self.hsc_sh = z(max(T, 1), self.fs, dtype=u8), sfa(max(T, 1), self.fs)
             self.hs = None
 
     def _ffn_fp8(self, c, xq, xs, rows, offsets, G, names, f, hq, hsc, y, s):
         (w1q, w1s), (w3q, w3s), (w2q, w2s) = (self.wq[n] for n in names)
-        L.moe_grouped_ffn_fp8(c, xq, xs, rows, offsets, G, w1q, w1s, w3q, w3s, w2q, w2s, f, hq, hsc, y, s)
+        fn = L.moe_grouped_ffn_mxfp8 if self.w.mxfp8 else L.moe_grouped_ffn_fp8
+        fn(c, xq, xs, rows, offsets, G, w1q, w1s, w3q, w3s, w2q, w2s, f, hq, hsc, y, s)
 
     # the launches of one layer forward; `x` is [T, d] on the device.  `marks`, if
     # given, is a list of 7 CUDA events recorded between the stages (route, permute,
@@ -137,10 +147,13 @@ class MoELayer:
                     self.topk_w, self.lse, self.p_partial, self.margin, self.ws, s,
                     shared_w=self.shared_w)
         rec(1)
-        fp8 = self.w.fp8
+        fp8 = self.w.fp8 or self.w.mxfp8
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
                       self.token_of_row, self.x_perm, self.n_dropped, self.ws, s)
-        if fp8:
+        if self.w.mxfp8:
+            L.moe_permute_mxfp8(c, x, self.topk_idx, self.row_of_slot, self.offsets, self.xq_perm, self.xs_perm,
+                                self.xq if self.fs > 0 else None, self.xs if self.fs > 0 else None, s)
+        elif fp8:
             L.moe_permute_fp8(c, x, self.row_of_slot, self.xq_perm, self.xs_perm,
                               self.xq if self.fs > 0 else None, self.xs if self.fs > 0 else None, s)
         rec(2)

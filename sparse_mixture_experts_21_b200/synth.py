@@ -50,6 +50,7 @@ class Workload:
     shared_sink: bool = False           # the (single) shared expert joins the weight normalisation
     expert_choice: bool = False         # experts pick their top-C tokens (C = ceil(cf k T / N))
     fp8: bool = False                   # expert matmuls on E4M3 codes with fine-grained block scales
+    mxfp8: bool = False                 # expert matmuls in MXFP8 (E4M3, E8M0 scale per 32 along K)
 
     def with_tokens(self, T: int) -> "Workload":
         return replace(self, T=T)
@@ -75,6 +76,10 @@ WORKLOADS = {
     "deepseek_v3_fp8": Workload("deepseek_v3_fp8", T=16384, d=7168, N=256, k=8, f=2048, n_shared=1,
                                 f_shared=2048, score="sigmoid", n_groups=8, topk_groups=4,
                                 group_topn=2, bias_std=0.1, fp8=True),
+    # the same with MXFP8 experts (scales applied by the tensor cores)
+    "deepseek_v3_mxfp8": Workload("deepseek_v3_mxfp8", T=16384, d=7168, N=256, k=8, f=2048, n_shared=1,
+                                  f_shared=2048, score="sigmoid", n_groups=8, topk_groups=4,
+                                  group_topn=2, bias_std=0.1, mxfp8=True),
 }
 
 
