@@ -35,9 +35,13 @@ WORKLOAD = "deepseek_v3"
 METRIC = "MoE layer fwd tokens/s"
 UNIT = "tokens/s"
 
-# DRAM traffic of the dominant kernels per launch from an ncu capture, valid only
-# while the kernel source is the one that was profiled (sha1 of ffn_tc.cu).
-NCU_TRAFFIC = {"ffn_tc_sha1": "20e1efc02dee7b5fd27a4663f5e984a52ae4205d", "bytes_per_ffn_call": 35.7e9}
+# DRAM bytes (read + write) of one routed grouped-FFN call (both passes) from a
+# full-size ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass),
+# valid only while the kernel source is the one that was profiled (sha1).
+NCU_TRAFFIC = {
+    "deepseek_v3": ("ffn_tc.cu", "20e1efc02dee7b5fd27a4663f5e984a52ae4205d", 32.3e9),
+    "deepseek_v3_mxfp8": ("ffn_mx.cu", "709e9d80185da2b81c3d48f20340d1eabb0fd4e9", 15.07e9),
+}
 
 
 def _peaks():
@@ -301,9 +305,10 @@ def main():
     ffn_peak_src = peaks["source"] + (" sustained bf16 x 2 (nominal fp8/bf16 ratio)" if lowp else " sustained bf16")
     tflops_ffn = flops_routed / (t_ffn * 1e-3) / 1e12
     traffic = None
-    if w.name == WORKLOAD and NCU_TRAFFIC["ffn_tc_sha1"] == _sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc",
-                                                        "ffn_tc.cu")):
-        traffic = NCU_TRAFFIC["bytes_per_ffn_call"]
+    if w.name in NCU_TRAFFIC:
+        src, sha, nbytes = NCU_TRAFFIC[w.name]
+        if _sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc", src)) == sha:
+            traffic = nbytes
 
     # end to end through the public API: every step copies its input from pinned host
     # memory and its result back to pinned host memory (MoELayer.forward_host, which
