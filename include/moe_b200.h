@@ -320,6 +320,43 @@ int moe_grouped_ffn_mxfp8(const moe_config_t* cfg, const uint8_t* xq_rows, const
                           void* y_rows, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Expert parallelism: the data path around the all-to-all exchange.
+ *
+ * Defines: the Practice page, "专家并行与 all-to-all": experts are sharded over W
+ * ranks (rank of expert e = e / (N / W), N % W == 0); the ranks exchange their
+ * per-expert counts before the all-to-all, send each kept (token, expert) row to
+ * the rank holding its expert, compute there, and send the results back for the
+ * weighted combine.  After moe_permute a rank's rows are ordered by expert, hence
+ * by destination rank, so they are the dispatch send buffer as they stand.  The
+ * exchange itself (count all-gather, two all-to-alls) is the caller's (NCCL).
+ * ------------------------------------------------------------------------- */
+
+/* moe_ep_plan -- split sizes and regroup map of one rank.
+ *   offsets_all   [W, N+1] int32 (device): every rank's expert offsets from
+ *                 moe_permute (the all-gather of offsets); rank s keeps
+ *                 offsets_all[s, e+1] - offsets_all[s, e] rows of expert e
+ *   send_splits   [W] int32 out: rows this rank sends to each rank
+ *   recv_splits   [W] int32 out: rows this rank receives from each rank
+ *   local_offsets [N/W + 1] int32 out: exclusive scan, over this rank's experts, of
+ *                 the rows all ranks send it (the groups of the local grouped FFN)
+ *   regroup_map   [recv_cap] int32 out: received row q (source-rank major, then
+ *                 expert, then row) -> its local row (expert major, then source
+ *                 rank, then row); entries past the received total are untouched
+ * Errors: MOE_ERR_INVALID_ARG for W < 1, rank outside [0, W), N % W != 0, NULL. */
+int moe_ep_plan(const int32_t* offsets_all, int32_t world, int32_t rank, int32_t n_experts, int32_t* send_splits,
+                int32_t* recv_splits, int32_t* local_offsets, int32_t* regroup_map, int64_t recv_cap, void* stream);
+
+/* moe_rows_move -- move rows through an index map (no counterpart on the pages:
+ * the regroup step of the exchange above).
+ *   src, dst   row-major buffers of row_bytes per row (row_bytes % 16 == 0, 16-byte aligned)
+ *   map        [rows_cap] int32 (device)
+ *   n_rows     device int32 scalar: rows to move (min with rows_cap), or NULL for rows_cap
+ *   scatter    0: dst[r] = src[map[r]];  1: dst[map[r]] = src[r]
+ * Errors: MOE_ERR_INVALID_ARG for a bad size, flag, NULL or misaligned buffer. */
+int moe_rows_move(const void* src, int64_t row_bytes, const int32_t* map, const int32_t* n_rows, int64_t rows_cap,
+                  int32_t scatter, void* dst, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_combine -- y[t] = shared[t] + sum_{j: row >= 0} w[t,j] * y_perm[row(t,j)].
  *
  * Defines: llm-compass "稀疏门控与 Top-k 路由" (y = sum_i g_i E_i(x)) and the Practice

@@ -698,3 +698,39 @@ def swiglu_ffn_mxfp8(x_rows, w1, w3, w2, hidden_out: bool = False):
     h = silu(xd @ w1d.T) * (xd @ w3d.T)
     y = dequantize_mxfp8(*quantize_mxfp8(h)) @ w2d.T
     return (y, h) if hidden_out else y
+
+
+# ---------------------------------------------------------------------------
+# Expert parallelism: the exchange plan
+# ---------------------------------------------------------------------------
+def ep_plan(offsets_all: np.ndarray, rank: int) -> dict:
+    """The bookkeeping of [Practice] "专家并行与 all-to-all" for rank `rank` of W:
+    experts are sharded contiguously (rank of expert e = e // (N / W)); each rank
+    knows every rank's per-expert kept counts (exchanged before the rows).
+
+    offsets_all [W, N+1]: every rank's expert offsets (rows kept per expert are
+    their differences).  Returns
+      send[r]       rows this rank sends to rank r (its kept rows of r's experts),
+      recv[s]       rows it receives from rank s,
+      local_offsets exclusive scan over its experts of the rows received for each,
+      regroup[q]    received row q -> local row, where received rows come source
+                    rank major, then expert, then row (the all-to-all order) and
+                    local rows come expert major, then source rank, then row.
+    Written as explicit loops over (source, expert, row).
+    """
+    off = np.asarray(offsets_all, np.int64)
+    W, N = off.shape[0], off.shape[1] - 1
+    El = N // W
+    kept = off[:, 1:] - off[:, :-1]
+    mine = range(rank * El, (rank + 1) * El)
+    send = [int(sum(kept[rank, r * El + j] for j in range(El))) for r in range(W)]
+    recv = [int(sum(kept[s, e] for e in mine)) for s in range(W)]
+    local_counts = [int(sum(kept[s, e] for s in range(W))) for e in mine]
+    local_offsets = np.concatenate([[0], np.cumsum(local_counts)]).astype(np.int64)
+    regroup = []
+    for s in range(W):
+        for j, e in enumerate(mine):
+            before = sum(kept[s2, e] for s2 in range(s))
+            for i in range(kept[s, e]):
+                regroup.append(int(local_offsets[j] + before + i))
+    return {"send": send, "recv": recv, "local_offsets": local_offsets, "regroup": np.array(regroup, np.int64)}

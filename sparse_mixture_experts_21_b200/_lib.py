@@ -28,7 +28,8 @@ EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_rou
             "moe_device_status", "moe_status_string", "moe_permute_noalloc", "moe_bias_update_ema",
             "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec",
             "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
-            "moe_quantize_mxfp8", "moe_permute_mxfp8", "moe_grouped_ffn_mxfp8")
+            "moe_quantize_mxfp8", "moe_permute_mxfp8", "moe_grouped_ffn_mxfp8", "moe_ep_plan",
+            "moe_rows_move")
 
 
 class MoeConfig(ctypes.Structure):
@@ -95,6 +96,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_grouped_ffn_fp8": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, c_int32, vp, vp,
                                 vp, vp],
         "moe_quantize_mxfp8": [vp, c_int64, c_int32, vp, vp, vp],
+        "moe_ep_plan": [vp, c_int32, c_int32, c_int32, vp, vp, vp, vp, c_int64, vp],
+        "moe_rows_move": [vp, c_int64, vp, vp, c_int64, c_int32, vp, vp],
         "moe_permute_mxfp8": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "moe_grouped_ffn_mxfp8": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, c_int32, vp, vp,
                                   vp, vp],
@@ -248,6 +251,22 @@ def moe_grouped_ffn_mxfp8(cfg, xq_rows, xsf_rows, rows_cap, offsets, G, w1q, w1s
         ctypes.byref(cfg), _ptr(xq_rows), _ptr(xsf_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1q),
         _ptr(w1sf), _ptr(w3q), _ptr(w3sf), _ptr(w2q), _ptr(w2sf), int(f), _ptr(hq_scratch), _ptr(hsf_scratch),
         _ptr(y_rows), _stream(stream)))
+
+
+def moe_ep_plan(offsets_all, world, rank, send_splits, recv_splits, local_offsets, regroup_map, stream=None):
+    """Split sizes, local expert offsets and the regroup map of one rank (offsets_all [W, N + 1])."""
+    _check("moe_ep_plan", load().moe_ep_plan(
+        _ptr(offsets_all), int(world), int(rank), int(offsets_all.shape[1]) - 1, _ptr(send_splits), _ptr(recv_splits),
+        _ptr(local_offsets), _ptr(regroup_map), int(regroup_map.shape[0]), _stream(stream)))
+
+
+def moe_rows_move(src, map_, n_rows, dst, scatter=False, rows_cap=None, stream=None):
+    """dst[r] = src[map[r]] (gather) or dst[map[r]] = src[r] (scatter) for r < n_rows
+    (a device int32 scalar, or None for rows_cap = len(map))."""
+    row_bytes = src.stride(0) * src.element_size()
+    _check("moe_rows_move", load().moe_rows_move(
+        _ptr(src), int(row_bytes), _ptr(map_), _ptr(n_rows), int(map_.shape[0] if rows_cap is None else rows_cap),
+        1 if scatter else 0, _ptr(dst), _stream(stream)))
 
 
 def moe_combine(cfg, y_perm, row_of_slot, topk_w, shared_out, y, stream=None, shared_w=None):

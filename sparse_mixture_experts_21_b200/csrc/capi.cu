@@ -282,6 +282,26 @@ int moe_grouped_ffn_mxfp8(const moe_config_t* cfg, const uint8_t* xq_rows, const
                                  static_cast<cudaStream_t>(stream)));
 }
 
+int moe_ep_plan(const int32_t* offsets_all, int32_t world, int32_t rank, int32_t n_experts, int32_t* send_splits,
+                int32_t* recv_splits, int32_t* local_offsets, int32_t* regroup_map, int64_t recv_cap, void* stream) {
+  if (world < 1 || n_experts < 1 || rank < 0 || rank >= world || (n_experts % world) != 0 || recv_cap < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!offsets_all || !send_splits || !recv_splits || !local_offsets || (recv_cap > 0 && !regroup_map))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_ep_plan(offsets_all, world, rank, n_experts, send_splits, recv_splits, local_offsets,
+                                  regroup_map, recv_cap, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_rows_move(const void* src, int64_t row_bytes, const int32_t* map, const int32_t* n_rows, int64_t rows_cap,
+                  int32_t scatter, void* dst, void* stream) {
+  if (row_bytes <= 0 || (row_bytes % 16) != 0 || rows_cap < 0 || (scatter != 0 && scatter != 1))
+    return MOE_ERR_INVALID_ARG;
+  if (rows_cap == 0) return MOE_OK;
+  if (!src || !map || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_rows_move(src, row_bytes, map, n_rows, rows_cap, scatter, dst,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of_slot,
                 const float* topk_w, const void* shared_out, const float* shared_w, void* y,
                 void* stream) {

@@ -84,6 +84,11 @@ cudaError_t launch_ffn_mx(const uint8_t* xq, const uint8_t* xsf, int64_t rows_ca
                           const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w3q, const uint8_t* w3sf,
                           const uint8_t* w2q, const uint8_t* w2sf, int d, int f, uint8_t* hq, uint8_t* hsf,
                           void* y, cudaStream_t s);
+cudaError_t launch_ep_plan(const int32_t* offsets_all, int W, int rank, int N, int32_t* send_splits,
+                           int32_t* recv_splits, int32_t* local_offsets, int32_t* regroup_map, int64_t recv_cap,
+                           cudaStream_t s);
+cudaError_t launch_rows_move(const void* src, int64_t row_bytes, const int32_t* map, const int32_t* n_rows,
+                             int64_t rows_cap, int scatter, void* dst, cudaStream_t s);
 int sm_count();
 
 }  // namespace moe

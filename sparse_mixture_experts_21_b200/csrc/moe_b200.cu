@@ -11,3 +11,4 @@
 #include "expert_choice.cu"
 #include "ffn_fp8.cu"
 #include "ffn_mx.cu"
+#include "ep.cu"

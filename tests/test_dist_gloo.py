@@ -57,3 +57,61 @@ def test_replicas_share_counts_and_bias(tmp_path):
     assert np.array_equal(r[0]["bias"], r[1]["bias"])       # replicas stay identical
     single = O.bias_update(np.zeros(N), want, rate=1e-3)
     assert np.array_equal(r[0]["bias"], single)             # same as one process on all tokens
+
+
+# ----------------------------------------------------------------------------- expert parallelism
+EP_N, EP_WORLD, EP_D = 8, 2, 16
+
+
+def _ep_worker(rank, port, out_dir):
+    """Rank `rank` exchanges rows with TorchDistExchange on CPU (gloo): the offsets
+    all-gather, the dispatch all-to-all in the plan's split sizes, and the return
+    all-to-all.  Each row carries (source rank, source row) so the receiver can
+    check where it came from."""
+    from sparse_mixture_experts_21_b200.ep import TorchDistExchange
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=EP_WORLD)
+    try:
+        ex = TorchDistExchange()
+        rng = np.random.default_rng(300 + rank)
+        kept = rng.integers(0, 6, size=EP_N)
+        kept[rank * 3] = 0                                    # an empty expert on each rank
+        offsets = torch.tensor(np.concatenate([[0], np.cumsum(kept)]), dtype=torch.int32)
+        offsets_all = ex.all_gather(offsets)
+        plan = O.ep_plan(offsets_all.numpy(), rank)
+        R = int(kept.sum())
+        send = torch.zeros(R, EP_D)
+        send[:, 0] = rank
+        send[:, 1] = torch.arange(R, dtype=torch.float32)
+        recv = torch.full((sum(plan["recv"]), EP_D), -1.0)
+        ex.all_to_all(recv, send, plan["recv"], plan["send"])
+        # the "expert" here: add 1000 to every received row, then send it back
+        back = torch.empty_like(send)
+        ex.all_to_all(back, recv + 1000.0, plan["send"], plan["recv"])
+        np.savez(os.path.join(out_dir, f"ep{rank}.npz"), offsets_all=offsets_all.numpy(), recv=recv.numpy(),
+                 back=back.numpy(), send=send.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ep_exchange_two_ranks(tmp_path):
+    mp.start_processes(_ep_worker, args=(_free_port(), str(tmp_path)), nprocs=EP_WORLD, join=True,
+                       start_method="spawn")
+    r = [np.load(tmp_path / f"ep{i}.npz") for i in range(EP_WORLD)]
+    assert np.array_equal(r[0]["offsets_all"], r[1]["offsets_all"])
+    off = r[0]["offsets_all"]
+    El = EP_N // EP_WORLD
+    for rank in range(EP_WORLD):
+        recv = r[rank]["recv"]
+        # received rows: source-rank major, each source's rows of this rank's experts in order
+        q = 0
+        for s in range(EP_WORLD):
+            lo, hi = off[s, rank * El], off[s, (rank + 1) * El]
+            n = hi - lo
+            assert np.all(recv[q:q + n, 0] == s)
+            assert np.array_equal(recv[q:q + n, 1], np.arange(lo, hi))
+            q += n
+        assert q == len(recv)
+        # every row comes home, in place, transformed once
+        assert np.array_equal(r[rank]["back"], r[rank]["send"] + 1000.0)

@@ -717,3 +717,47 @@ def test_mxfp8_ffn_close_to_exact():
     assert np.max(np.abs(y - y0)) / np.max(np.abs(y0)) < 0.1
     h0 = O.silu(x @ w1.T) * (x @ w3.T)
     assert np.max(np.abs(h - h0)) / np.max(np.abs(h0)) < 0.1
+
+
+# ----------------------------------------------------------------------------- expert parallelism plan
+def test_ep_plan_hand_case():
+    # W = 2 ranks, N = 4 experts (rank 0 holds 0, 1; rank 1 holds 2, 3)
+    # rank 0 keeps [2, 1, 0, 3] rows, rank 1 keeps [1, 0, 2, 2] rows per expert
+    off = np.array([[0, 2, 3, 3, 6], [0, 1, 1, 3, 5]])
+    p0 = O.ep_plan(off, 0)
+    assert p0["send"] == [3, 3] and p0["recv"] == [3, 1]
+    assert p0["local_offsets"].tolist() == [0, 3, 4]
+    # received: from rank 0 expert 0 (2 rows), expert 1 (1), then rank 1 expert 0 (1), expert 1 (0)
+    # local: expert 0 = [r0 row0, r0 row1, r1 row0], expert 1 = [r0 row0]
+    assert p0["regroup"].tolist() == [0, 1, 3, 2]
+    p1 = O.ep_plan(off, 1)
+    assert p1["send"] == [1, 4] and p1["recv"] == [3, 4]
+    assert p1["local_offsets"].tolist() == [0, 2, 7]
+    # received: r0 e2 (0), r0 e3 (3 rows), r1 e2 (2), r1 e3 (2); local e2 = [r1 x2], e3 = [r0 x3, r1 x2]
+    assert p1["regroup"].tolist() == [2, 3, 4, 0, 1, 5, 6]
+
+
+def test_ep_plan_invariants():
+    rng = np.random.default_rng(149)
+    W, N = 4, 16
+    kept = rng.integers(0, 7, size=(W, N))
+    off = np.concatenate([np.zeros((W, 1), np.int64), np.cumsum(kept, axis=1)], axis=1)
+    plans = [O.ep_plan(off, r) for r in range(W)]
+    for r, p in enumerate(plans):
+        R = sum(p["recv"])
+        assert p["local_offsets"][-1] == R
+        assert sorted(p["regroup"].tolist()) == list(range(R))          # a permutation
+        assert sum(p["send"]) == kept[r].sum()                           # every kept row leaves once
+        for s in range(W):
+            assert p["recv"][s] == plans[s]["send"][r]                   # both ends agree
+    # regroup keeps the order of a source's rows within an expert
+    p = plans[1]
+    El = N // W
+    q = 0
+    for s in range(W):
+        for j in range(El):
+            n = kept[s, 1 * El + j]
+            loc = p["regroup"][q:q + n]
+            assert np.all(np.diff(loc) == 1)
+            assert p["local_offsets"][j] <= (loc.min() if n else p["local_offsets"][j]) < p["local_offsets"][j + 1] + 1
+            q += n
