@@ -283,7 +283,7 @@ def main():
     t_route, t_perm, t_ffn, t_shared, t_comb, t_stats = (stage(0, 1), stage(1, 2), stage(2, 3),
                                                          stage(3, 4), stage(4, 5), stage(5, 6))
     R = int(lay.offsets[-1].item())
-    eb = 2
+    eb = 4 if w.dtype == "fp32" else 2
     T, d, N, k, f = w.T, w.d, w.N, w.k, w.f
     flops_routed = 6.0 * R * d * f
     flops_shared = 6.0 * T * d * lay.fs
@@ -303,6 +303,11 @@ def main():
     # E4M3 operands: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
     ffn_peak = peaks["bf16_tflops_sustained"] * (2.0 if lowp else 1.0)
     ffn_peak_src = peaks["source"] + (" sustained bf16 x 2 (nominal fp8/bf16 ratio)" if lowp else " sustained bf16")
+    ffn_bound = "tensor"
+    if w.dtype == "fp32":
+        # fp32 experts run on the FMA pipes: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
+        ffn_peak, ffn_bound = 148 * 128 * 2 * 1.965e9 / 1e12, "alu"
+        ffn_peak_src = "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"
     tflops_ffn = flops_routed / (t_ffn * 1e-3) / 1e12
     traffic = None
     if w.name in NCU_TRAFFIC:
@@ -343,7 +348,8 @@ def main():
             "metric": METRIC, "value": world * T / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": ("mxfp8-e4m3 experts, fp32 router" if w.mxfp8 else
-                                                              "fp8-e4m3 experts, fp32 router" if w.fp8 else "bf16"),
+                                                              "fp8-e4m3 experts, fp32 router" if w.fp8 else
+                                                              "fp32" if w.dtype == "fp32" else "bf16"),
             "data": "synthetic",
             "config": {"workload": w.name, "T": T, "d_model": d, "experts": N, "top_k": k, "d_ff": f,
                        "shared_experts": w.n_shared,
@@ -357,7 +363,7 @@ def main():
                               f"{3 * N * d * f * (1 if lowp else eb) / 1e9:.1f} GB); no flush")},
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
             "roofline": {"kernel": "grouped SwiGLU FFN, routed experts (gate/up + down passes)",
-                         "bound": "tensor", "achieved": tflops_ffn,
+                         "bound": ffn_bound, "achieved": tflops_ffn,
                          "peak": ffn_peak, "unit": "TFLOP/s",
                          "frac": tflops_ffn / ffn_peak, "traffic": traffic,
                          "peak_source": ffn_peak_src},
