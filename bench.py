@@ -215,6 +215,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay measurement")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload name from synth.WORKLOADS (default: the DeepSeek-V3-shaped layer)")
     ap.add_argument("--tokens", type=int, default=None,
@@ -315,6 +316,21 @@ def main():
         if _sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc", src)) == sha:
             traffic = nbytes
 
+    # the same step replayed from a CUDA graph (one capture, K replays): launch overhead out
+    graph = None
+    if pg is None and not args.no_graph:
+        lay.capture(x)
+        barrier()
+        g0, g1 = ev(), ev()
+        g0.record(stream)
+        for _ in range(args.steps):
+            lay.replay()
+        g1.record(stream)
+        barrier()
+        gms = g0.elapsed_time(g1) / args.steps
+        graph = {"value": T / (gms * 1e-3), "unit": UNIT, "ms_per_step": gms}
+        assert L.moe_device_status() == L.MOE_OK
+
     # end to end through the public API: every step copies its input from pinned host
     # memory and its result back to pinned host memory (MoELayer.forward_host, which
     # overlaps one step's copies with the neighbouring steps' compute)
@@ -378,6 +394,7 @@ def main():
             "gpu_launches": lay.kernel_launches() * args.steps,
             "clocks": clk.summary(),
             "e2e": e2e,
+            "cuda_graph": graph,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

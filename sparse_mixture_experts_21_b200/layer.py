@@ -214,6 +214,28 @@ class MoELayer:
         rec(6)
         return y
 
+    def capture(self, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.cuda.CUDAGraph:
+        """Record one whole forward on the fixed input buffer `x` into a CUDA graph
+        (after one eager forward on the capture stream, which sets the kernels' launch
+        attributes); `replay()` then reruns every launch of the step, the bias update
+        included, without host launch overhead.  Not for the replica mode (its counts
+        all-reduce is a collective)."""
+        if self.group is not None:
+            raise ValueError("capture is for a single-process layer")
+        s = torch.cuda.Stream(self.dev)
+        s.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(s):
+            self.forward(x, s, out=out)
+        torch.cuda.current_stream(self.dev).wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            self.forward(x, s, out=out)
+        self._graph = g
+        return g
+
+    def replay(self):
+        self._graph.replay()
+
     def forward_host(self, x_host_steps, y_host_steps, stream=None):
         """Layer forwards on host data: for each step, copy its [T, d] input from
         pinned host memory, run the layer, copy the result back into the matching

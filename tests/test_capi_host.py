@@ -153,3 +153,42 @@ def test_status_strings(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(FileNotFoundError):
         L.load(str(tmp_path / "nope.so"))
+
+
+def test_low_precision_argument_checks(lib):
+    """FP8 / MXFP8 entry points reject bad shapes and pointers before touching the GPU."""
+    ok = 0x1000000
+    IA, UN = L.MOE_ERR_INVALID_ARG, L.MOE_ERR_UNSUPPORTED
+    # block quantisation: cols must be a multiple of 128, block rows 1 or 128
+    assert lib.moe_quantize_fp8(ok, 10, 100, 1, ok, ok, None) == IA
+    assert lib.moe_quantize_fp8(ok, 10, 128, 64, ok, ok, None) == IA
+    assert lib.moe_quantize_fp8(ok + 8, 10, 128, 1, ok, ok, None) == IA       # misaligned x
+    assert lib.moe_quantize_fp8(ok, 0, 128, 1, None, None, None) == L.MOE_OK  # nothing to do
+    assert lib.moe_quantize_mxfp8(ok, 10, 96, ok, ok, None) == IA             # MXFP8 wants cols % 128
+    assert lib.moe_quantize_mxfp8(ok, 10, 128, ok + 4, ok, None) == IA        # codes not 8-byte aligned
+    c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    # grouped FFNs: f % 128, G range, fp32 configs unsupported
+    args = (ok, ok, 1024, ok, 4, ok, ok, ok, ok, ok, ok)
+    assert lib.moe_grouped_ffn_fp8(ctypes.byref(c), *args, 2000, ok, ok, ok, None) == UN
+    assert lib.moe_grouped_ffn_mxfp8(ctypes.byref(c), *args, 2000, ok, ok, ok, None) == UN
+    assert lib.moe_grouped_ffn_mxfp8(ctypes.byref(c), ok, ok, 1024, ok, 0, ok, ok, ok, ok, ok, ok, 2048, ok, ok,
+                                     ok, None) == IA
+    assert lib.moe_grouped_ffn_mxfp8(ctypes.byref(c), ok, ok + 4, 1024, ok, 4, ok, ok, ok, ok, ok, ok, 2048, ok,
+                                     ok, ok, None) == IA                      # scale atoms 16-byte aligned
+    c32 = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    assert lib.moe_grouped_ffn_fp8(ctypes.byref(c32), ok, ok, 64, ok, 1, ok, ok, ok, ok, ok, ok, 256, ok, ok, ok,
+                                   None) == UN
+    # the quantising permutations need their row maps
+    assert lib.moe_permute_mxfp8(ctypes.byref(c), ok, None, ok, ok, ok, ok, None, None, None) == IA
+    assert lib.moe_permute_fp8(ctypes.byref(c), ok, ok, None, ok, None, None, None) == IA
+
+
+def test_expert_parallel_argument_checks(lib):
+    ok = 0x1000000
+    IA = L.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_plan(ok, 3, 0, 256, ok, ok, ok, ok, 10, None) == IA    # 256 experts over 3 ranks
+    assert lib.moe_ep_plan(ok, 4, 4, 256, ok, ok, ok, ok, 10, None) == IA    # rank out of range
+    assert lib.moe_ep_plan(None, 4, 0, 256, ok, ok, ok, ok, 10, None) == IA
+    assert lib.moe_rows_move(ok, 24, ok, None, 10, 0, ok, None) == IA        # rows of 24 bytes
+    assert lib.moe_rows_move(ok, 32, ok, None, 10, 2, ok, None) == IA        # bad direction flag
+    assert lib.moe_rows_move(ok, 32, ok, None, 0, 0, ok, None) == L.MOE_OK   # no rows

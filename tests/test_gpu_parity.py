@@ -374,3 +374,23 @@ def test_forward_host_pipeline_matches_forward():
     torch.cuda.synchronize()
     for a, b in zip(want, yh):
         assert torch.equal(a.cpu(), b)
+
+
+def test_cuda_graph_replay_matches_eager():
+    """A captured forward replays the same launches: outputs and the bias after the
+    same number of steps are bit-identical to eager execution."""
+    w = replace(SMALL["v3_small"], T=513)
+    inp_a = make_inputs(w, "cuda")
+    inp_b = make_inputs(w, "cuda")
+    eager = MoELayer(w, inp_a, "cuda", update_bias=True)
+    graph = MoELayer(w, inp_b, "cuda", update_bias=True)
+    graph.capture(inp_b["x"])                  # one eager forward + the capture
+    eager.forward(inp_a["x"])
+    for _ in range(3):
+        eager.forward(inp_a["x"])
+        graph.replay()
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(eager.y, graph.y)
+    assert torch.equal(inp_a["bias"], inp_b["bias"])
+    assert torch.equal(eager.stats, graph.stats)
