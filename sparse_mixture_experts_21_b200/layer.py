@@ -46,6 +46,10 @@ class MoELayer:
         """group: a torch.distributed process group when the layer runs as one of
         several data-parallel replicas; the bias update then uses the counts summed
         over the group, so all replicas keep the same selection bias."""
+        if w.expert_choice and (w.fp8 or w.mxfp8):
+            raise ValueError("expert-choice routing runs bf16 or fp32 experts")
+        if (w.fp8 or w.mxfp8) and (w.dtype != "bf16" or w.d % 128 or w.f % 128 or w.f_shared % 128):
+            raise ValueError("FP8 experts need bf16 inputs and d, d_ff multiples of 128")
         self.w = w
         self.group = group
         self.dev = torch.device(device)

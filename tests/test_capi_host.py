@@ -192,3 +192,12 @@ def test_expert_parallel_argument_checks(lib):
     assert lib.moe_rows_move(ok, 24, ok, None, 10, 0, ok, None) == IA        # rows of 24 bytes
     assert lib.moe_rows_move(ok, 32, ok, None, 10, 2, ok, None) == IA        # bad direction flag
     assert lib.moe_rows_move(ok, 32, ok, None, 0, 0, ok, None) == L.MOE_OK   # no rows
+
+
+def test_layer_rejects_unsupported_combinations():
+    from dataclasses import replace
+    w = synth.WORKLOADS["ec_deepseekmoe_16b"]
+    with pytest.raises(ValueError):
+        layer.MoELayer(replace(w, mxfp8=True), {}, "cpu")
+    with pytest.raises(ValueError):
+        layer.MoELayer(replace(synth.WORKLOADS["deepseek_v3"], fp8=True, f=1000), {}, "cpu")
