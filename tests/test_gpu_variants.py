@@ -156,3 +156,36 @@ def test_expert_choice_ties_and_capacity_edges():
         ec = O.expert_choice(s.astype(np.float64), C)
         assert np.array_equal(i64(row_of), ec["row_of"]) and np.array_equal(i64(tor), ec["token_of_row"])
         assert torch.equal(xp, x[tor.long()])
+
+
+def test_expert_choice_full_size():
+    """The DeepSeekMoE-16B-shaped expert-choice workload (T = 8192, 64 experts, C = 768):
+    the selection bit for bit on the GPU's own affinities, sampled expert rows, and the
+    combine on sampled tokens."""
+    w = WORKLOADS["ec_deepseekmoe_16b"]
+    lay, inp = _run(w)
+    C = ec_capacity(w)
+    assert C == 768
+    s_gpu = f64(lay.scores).T                                   # [T, N]
+    ec = O.expert_choice(s_gpu, C)
+    assert np.array_equal(i64(lay.row_of), ec["row_of"])
+    assert np.array_equal(i64(lay.token_of_row)[: w.N * C], ec["token_of_row"])
+    assert int(lay.n_unpicked.item()) == ec["unpicked"]
+    rng = np.random.default_rng(5)
+    get = expert_weights_fn(inp)
+    x64 = f64(inp["x"])
+    for e in rng.choice(w.N, size=4, replace=False):
+        rows = np.sort(rng.choice(C, size=24, replace=False)) + e * C
+        toks = ec["token_of_row"][rows]
+        ref = O.swiglu_ffn(x64[toks], *get(int(e)))
+        assert rel_err(f64(lay.y_perm[torch.tensor(rows, device="cuda")]), ref) < tol_for(w)
+    # combine on sampled tokens: shared experts + picked experts weighted by their affinity
+    tok = np.sort(rng.choice(w.T, size=16, replace=False))
+    ys = O.swiglu_ffn(x64[tok], *shared_weights(inp))
+    # the GPU's expert rows (checked above by sampling) fed to the oracle's combine
+    y_rows = np.zeros((w.N * C, w.d))
+    need = sorted({int(ec["row_of"][t, e]) for t in tok for e in range(w.N) if ec["row_of"][t, e] >= 0})
+    y_rows[need] = f64(lay.y_perm[torch.tensor(need, device="cuda")])
+    y_ref = np.stack([ys[i] + sum(s_gpu[t, e] * y_rows[ec["row_of"][t, e]] for e in range(w.N)
+                                  if ec["row_of"][t, e] >= 0) for i, t in enumerate(tok)])
+    assert rel_err(f64(lay.y[torch.tensor(tok, device="cuda")]), y_ref) < tol_for(w)
