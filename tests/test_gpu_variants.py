@@ -184,8 +184,9 @@ def test_expert_choice_full_size():
     ys = O.swiglu_ffn(x64[tok], *shared_weights(inp))
     # the GPU's expert rows (checked above by sampling) fed to the oracle's combine
     y_rows = np.zeros((w.N * C, w.d))
-    need = sorted({int(ec["row_of"][t, e]) for t in tok for e in range(w.N) if ec["row_of"][t, e] >= 0})
+    ro = ec["row_of"]                                           # [N, T]: row of (expert, token) or -1
+    need = sorted({int(ro[e, t]) for t in tok for e in range(w.N) if ro[e, t] >= 0})
     y_rows[need] = f64(lay.y_perm[torch.tensor(need, device="cuda")])
-    y_ref = np.stack([ys[i] + sum(s_gpu[t, e] * y_rows[ec["row_of"][t, e]] for e in range(w.N)
-                                  if ec["row_of"][t, e] >= 0) for i, t in enumerate(tok)])
+    y_ref = np.stack([ys[i] + sum(s_gpu[t, e] * y_rows[ro[e, t]] for e in range(w.N) if ro[e, t] >= 0)
+                      for i, t in enumerate(tok)])
     assert rel_err(f64(lay.y[torch.tensor(tok, device="cuda")]), y_ref) < tol_for(w)
