@@ -39,7 +39,7 @@ UNIT = "tokens/s"
 # full-size ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass),
 # valid only while the kernel source is the one that was profiled (sha1).
 NCU_TRAFFIC = {
-    "deepseek_v3": ("ffn_tc.cu", "20e1efc02dee7b5fd27a4663f5e984a52ae4205d", 32.3e9),
+    "deepseek_v3": ("ffn_tc.cu", "6c3608e44a457edba78d671673af093dfd68799d", 32.3e9),
     "deepseek_v3_mxfp8": ("ffn_mx.cu", "709e9d80185da2b81c3d48f20340d1eabb0fd4e9", 15.07e9),
 }
 

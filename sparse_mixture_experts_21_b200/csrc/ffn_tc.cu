@@ -218,7 +218,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
               int G, int K, int n_out, int64_t rows_cap, __nv_bfloat16* __restrict__ out) {
   using S = Shape<PAIR>;
   using SH = TcShared<S::STAGES>;
-  constexpr int STAGES = S::STAGES, STAGE_BYTES = S::STAGE_BYTES, BM = S::BM;
+  constexpr int STAGES = S::STAGES, STAGE_BYTES = S::STAGE_BYTES;
   constexpr int BN = MODE == 0 ? 128 : 256;    // output columns per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
