@@ -201,3 +201,21 @@ def test_layer_rejects_unsupported_combinations():
         layer.MoELayer(replace(w, mxfp8=True), {}, "cpu")
     with pytest.raises(ValueError):
         layer.MoELayer(replace(synth.WORKLOADS["deepseek_v3"], fp8=True, f=1000), {}, "cpu")
+
+
+def test_expert_parallel_layer_validation():
+    from dataclasses import replace
+    from sparse_mixture_experts_21_b200.ep import EPMoELayer
+    w = synth.WORKLOADS["deepseek_v3"]
+    with pytest.raises(ValueError):
+        EPMoELayer(w, {}, 0, 3, "cpu")                       # 256 experts over 3 ranks
+    with pytest.raises(ValueError):
+        EPMoELayer(replace(w, mxfp8=True), {}, 0, 2, "cpu")  # the exchange carries bf16 rows
+    with pytest.raises(ValueError):
+        EPMoELayer(synth.WORKLOADS["ec_deepseekmoe_16b"], {}, 0, 2, "cpu")
+
+
+def test_capture_refuses_replica_mode():
+    lay = layer.MoELayer(synth.WORKLOADS["tiny_top2_fp32"], {}, "cpu", group=object())
+    with pytest.raises(ValueError):
+        lay.capture(None)
