@@ -140,6 +140,78 @@ def test_group_limit_topn1_is_group_max():
     assert np.array_equal(gs, q.reshape(30, 3, 4).max(axis=2))
 
 
+# ---------------------------------------------------------------- near-tie margins (values)
+def test_topk_margin_hand_case():
+    """margin = q of the k-th pick minus the best eligible expert left out."""
+    q = np.array([[0.9, 0.5, 0.7, 0.1]])
+    idx, m = O.select_topk(q, 2)
+    assert idx.tolist() == [[0, 2]] and m[0] == 0.7 - 0.5
+    # expert 1 ineligible: the best expert left out is expert 3
+    idx, m = O.select_topk(q, 2, np.array([[True, False, True, True]]))
+    assert idx.tolist() == [[0, 2]] and m[0] == 0.7 - 0.1
+    # nothing eligible is left out
+    _, m = O.select_topk(q, 4)
+    assert np.isinf(m[0])
+    _, m = O.select_topk(q, 2, np.array([[True, False, True, False]]))
+    assert np.isinf(m[0])
+
+
+@pytest.mark.parametrize("n,k,ties", [(6, 2, False), (8, 3, False), (12, 4, False), (8, 3, True), (16, 2, True)])
+def test_topk_margin_bruteforce(n, k, ties):
+    """The margin value equals min(q over the brute-force best set) - max(q over the
+    eligible experts outside it), with random eligibility masks."""
+    rng = np.random.default_rng(100 + n * 7 + k + ties)
+    T = 80
+    q = rng.integers(0, 4, size=(T, n)).astype(np.float64) if ties else rng.normal(size=(T, n))
+    mask = rng.random((T, n)) < 0.75
+    for t in range(T):                          # at least k eligible experts
+        off = np.nonzero(~mask[t])[0]
+        need = k - int(mask[t].sum())
+        if need > 0:
+            mask[t, off[:need]] = True
+    idx, margin = O.select_topk(q, k, mask)
+    for t in range(T):
+        allowed = np.nonzero(mask[t])[0].tolist()
+        best = _brute_topk(list(q[t]), k, allowed)
+        assert tuple(sorted(idx[t])) == best
+        left = [q[t, e] for e in allowed if e not in best]
+        want = min(q[t, e] for e in best) - max(left) if left else math.inf
+        assert margin[t] == want
+    if ties:
+        assert np.any(margin == 0)
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_group_margin_bruteforce(ties):
+    """The group margin equals the smallest kept group score minus the largest dropped
+    one (brute force over group subsets), and route() reports min(expert, group) margin."""
+    rng = np.random.default_rng(211 + ties)
+    N, G, keep, topn, k = 16, 4, 2, 2, 3
+    cfg = O.OracleConfig(N, k, n_groups=G, topk_groups=keep, group_score_topn=topn)
+    T = 60
+    q = rng.integers(0, 4, size=(T, N)).astype(np.float64) if ties else rng.normal(size=(T, N))
+    mask, gmargin = O.eligible_mask(q, cfg)
+    idx, emargin = O.select_topk(q, k, mask)
+    gs = N // G
+    for t in range(T):
+        gscore = [max(sum(c) for c in itertools.combinations(q[t, g * gs:(g + 1) * gs], topn))
+                  for g in range(G)]
+        kept = max(itertools.combinations(range(G), keep), key=lambda sub: sum(gscore[g] for g in sub))
+        want = min(gscore[g] for g in kept) - max(gscore[g] for g in range(G) if g not in kept)
+        assert abs(gmargin[t] - want) <= 1e-12
+    # the router's margin is the smaller of the two; a config with every group kept has
+    # only the expert margin
+    x = rng.normal(size=(T, 8))
+    wg = rng.normal(size=(N, 8))
+    r = O.route(x, wg, cfg)
+    m, gm = O.eligible_mask(O.affinity(x @ wg.T, cfg.score_fn), cfg)
+    _, em = O.select_topk(O.affinity(x @ wg.T, cfg.score_fn), k, m)
+    assert np.array_equal(r["margin"], np.minimum(em, gm))
+    all_kept = O.OracleConfig(N, k, n_groups=G, topk_groups=G, group_score_topn=topn)
+    _, gm_all = O.eligible_mask(q, all_kept)
+    assert np.all(np.isinf(gm_all))
+
+
 def test_k_distinct_experts():
     rng = np.random.default_rng(9)
     cfg = O.OracleConfig(64, 6)
@@ -431,6 +503,56 @@ def test_sum_f_is_one():
     out = O.layer_forward(x, wg, cfg, lambda e: (np.zeros((2, 8)), np.zeros((2, 8)), np.zeros((8, 2))))
     assert abs(out["stats"]["f"].sum() - 1.0) < 1e-12
     assert abs(out["stats"]["P"].sum() - 1.0) < 1e-12
+    sig = O.layer_forward(x, wg, O.OracleConfig(16, 4, score_fn=O.SIGMOID),
+                          lambda e: (np.zeros((2, 8)), np.zeros((2, 8)), np.zeros((8, 2))))
+    assert abs(sig["stats"]["P"].sum() - 1.0) < 1e-12
+
+
+# ---------------------------------------------------------------- sigmoid load-balance probabilities
+def test_sigmoid_p_hand_case():
+    """P_e under sigmoid scores = token mean of s / sum_e s, worked by hand with
+    sigmoid(0) = 1/2 and sigmoid(ln 3) = 3/4: token 0 has logits (0, ln 3), so
+    s = (1/2, 3/4) -> (2/5, 3/5); token 1 has (ln 3, ln 3) -> (1/2, 1/2).  P =
+    (9/20, 11/20); with counts (2, 0), k = 1, T = 2: f = (1, 0) and aux_raw = N f.P = 0.9.
+    (The mean of the raw s would give P = (5/8, 3/4) and aux_raw = 1.25.)"""
+    z = np.array([[0.0, math.log(3.0)], [math.log(3.0), math.log(3.0)]])
+    cfg = O.OracleConfig(2, 1, score_fn=O.SIGMOID)
+    counts = np.array([2, 0])
+    st = O.router_stats(counts, counts, O.sigmoid(z), O.logsumexp(z), cfg, 2, 0, 0, alpha=0.01, z_coef=0.0)
+    assert np.allclose(st["P"], [0.45, 0.55], rtol=0, atol=1e-15)
+    assert abs(st["aux_raw"] - 0.9) < 1e-15 and abs(st["aux"] - 0.009) < 1e-16
+
+
+def test_sigmoid_aux_uniform_is_alpha():
+    """All logits 0 under sigmoid: every s = 1/2, so s / sum s = 1/N and, with equal
+    counts, aux = alpha exactly (the mean raw s = 1/2 would give alpha N / 2)."""
+    N, k, T, alpha = 16, 4, 32, 0.01
+    z = np.zeros((T, N))
+    counts = np.full(N, k * T // N)
+    st = O.router_stats(counts, counts, O.sigmoid(z), O.logsumexp(z), O.OracleConfig(N, k, score_fn=O.SIGMOID),
+                        T, 0, 0, alpha, 0.0)
+    assert np.allclose(st["P"], 1.0 / N, rtol=0, atol=1e-16)
+    assert abs(st["aux"] - alpha) < 1e-16
+
+
+def test_sigmoid_aux_uniform_end_to_end():
+    """k = 1, T = N, x_t = L e_t, W_g = [I | 0] under sigmoid: token t scores sigmoid(L)
+    on expert t and 1/2 elsewhere, so it picks expert t (f = 1/N); each row of s / sum s
+    sums to 1 and the construction is symmetric, so P_e = 1/N and aux = alpha."""
+    N, d, L, alpha = 8, 12, 2.5, 0.01
+    x = np.zeros((N, d))
+    x[np.arange(N), np.arange(N)] = L
+    wg = np.zeros((N, d))
+    wg[:, :N] = np.eye(N)
+    out = O.layer_forward(x, wg, O.OracleConfig(N, 1, score_fn=O.SIGMOID),
+                          lambda e: (np.ones((2, d)), np.ones((2, d)), np.ones((d, 2))), alpha=alpha)
+    st = out["stats"]
+    assert np.array_equal(out["routing"]["idx"][:, 0], np.arange(N))
+    assert np.allclose(out["routing"]["w"], 1.0)
+    sL = 1.0 / (1.0 + math.exp(-L))
+    assert abs(out["routing"]["s"][0, 0] - sL) < 1e-15
+    assert np.allclose(st["P"], 1.0 / N, rtol=1e-14) and np.allclose(st["f"], 1.0 / N)
+    assert abs(st["aux"] - alpha) < 1e-15
 
 
 # ---------------------------------------------------------------- bias update
@@ -761,3 +883,55 @@ def test_ep_plan_invariants():
             assert np.all(np.diff(loc) == 1)
             assert p["local_offsets"][j] <= (loc.min() if n else p["local_offsets"][j]) < p["local_offsets"][j + 1] + 1
             q += n
+
+
+# ----------------------------------------------------------------------------- fp32 against double
+def _tiny_layer_fp32(x, wg, w1, w3, w2, k, C):
+    """The tiny top-2 layer computed a second way, in float32 with torch CPU library
+    steps (softmax, topk, a stable sort for the token-order capacity, index_add for
+    the combine): an independent route to the same definition."""
+    import torch
+    f = lambda a: torch.tensor(a, dtype=torch.float32)  # noqa: E731
+    x, wg, w1, w3, w2 = f(x), f(wg), f(w1), f(w3), f(w2)
+    T, N = x.shape[0], wg.shape[0]
+    z = x @ wg.T
+    p = torch.softmax(z, dim=1)
+    val, idx = torch.topk(p, k, dim=1)
+    w = val / val.sum(dim=1, keepdim=True)
+    flat = idx.reshape(-1)                                   # slot order = token order
+    order = torch.sort(flat, stable=True).indices
+    first = torch.searchsorted(flat[order], torch.arange(N))
+    pos = torch.empty_like(flat)
+    pos[order] = torch.arange(flat.numel()) - first[flat[order]]
+    keep = pos < C
+    y = torch.zeros(T, x.shape[1])
+    for e in range(N):
+        slots = torch.nonzero((flat == e) & keep).reshape(-1)
+        tok = slots // k
+        xe = x[tok]
+        ye = (torch.nn.functional.silu(xe @ w1[e].T) * (xe @ w3[e].T)) @ w2[e].T
+        y.index_add_(0, tok, ye * w.reshape(-1)[slots][:, None])
+    return {"y": y.double().numpy(), "idx": idx.long().numpy(), "lse": torch.logsumexp(z, 1).double().numpy(),
+            "keep": keep.reshape(T, k).numpy()}
+
+
+def test_fp32_and_double_agree_on_the_tiny_workload():
+    """The tiny fp32 workload's forward agrees between float32 and double arithmetic:
+    expert choices and drops equal on every clear token, outputs within 1e-6 of max |y|
+    (the double oracle, against an independent float32 computation), so an fp32 GPU
+    path can be held to 1e-4."""
+    from sparse_mixture_experts_21_b200.synth import WORKLOADS, make_inputs
+    w = WORKLOADS["tiny_top2_fp32"]
+    inp = make_inputs(w, "cpu", seed=0)
+    a = {key: (None if v is None else v.double().numpy()) for key, v in inp.items()}
+    cfg = O.OracleConfig(w.N, w.k, capacity_mode=O.CAP_CEIL_CF_T_OVER_N, capacity_factor=w.cf)
+    ref = O.layer_forward(a["x"], a["w_gate"], cfg, lambda e: (a["w1"][e], a["w3"][e], a["w2"][e]))
+    C = O.capacity(cfg, w.T)
+    got = _tiny_layer_fp32(a["x"], a["w_gate"], a["w1"], a["w3"], a["w2"], w.k, C)
+    clear = ref["routing"]["margin"] >= 1e-4
+    assert clear.mean() > 0.98
+    assert np.array_equal(got["idx"][clear], ref["routing"]["idx"][clear])
+    if clear.all():
+        assert np.array_equal(got["keep"], ref["perm"]["keep"])
+        assert np.max(np.abs(got["y"] - ref["y"])) / np.max(np.abs(ref["y"])) < 1e-6
+    assert np.max(np.abs(got["lse"] - ref["routing"]["lse"])) / np.max(np.abs(ref["routing"]["lse"])) < 1e-6
