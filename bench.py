@@ -279,6 +279,7 @@ def main():
         from sparse_mixture_experts_21_b200.replicas import max_over_ranks
         ms = max_over_ranks(ms_local, dev)
     assert L.moe_device_status() == L.MOE_OK
+    st = lay.stats_dict()          # the last timed step's router statistics
 
     stage = lambda a, b: statistics.mean(marks[i][a].elapsed_time(marks[i][b]) for i in range(args.steps))  # noqa: E731
     t_route, t_perm, t_ffn, t_shared, t_comb, t_stats = (stage(0, 1), stage(1, 2), stage(2, 3),
@@ -391,6 +392,10 @@ def main():
                     "peak_gbs": peaks["hbm_gbs"]},
             "shared_ffn_tflops": flops_shared / (t_shared * 1e-3) / 1e12,
             "router_tflops_fp32": flops_router / (t_route * 1e-3) / 1e12,
+            "router_stats": {"aux": st["aux"], "z_loss": st["z_loss"], "cv": st["cv"], "dead": st["dead"],
+                             "dropped_slots": st["dropped_slots"], "dropped_tokens": st["dropped_tokens"]},
+            "near_ties": {"count": st["near_ties"], "tokens": st["T"], "threshold": L.NEAR_TIE,
+                          "frac": st["near_ties"] / max(st["T"], 1)},
             "gpu_launches": lay.kernel_launches() * args.steps,
             "clocks": clk.summary(),
             "e2e": e2e,

@@ -87,8 +87,14 @@ typedef struct moe_stats {
   int32_t dropped_slots;     /* k*T - R                                             */
   int32_t dropped_tokens;    /* tokens whose k slots were all dropped               */
   int32_t R;                 /* kept rows                                           */
-  int32_t reserved[5];
+  int32_t near_ties;         /* tokens whose selection margin (moe_route's margin) is
+                                below the near-tie threshold; -1 when not counted   */
+  int64_t T;                 /* tokens covered (summed over ranks after a reduction) */
+  int32_t reserved[2];
 } moe_stats_t;
+
+/* Length, in doubles, of the sufficient-statistics vector of moe_router_stats_partial. */
+#define MOE_STATS_PARTIAL_LEN(n_experts) (3 * (n_experts) + 5)
 
 /* ---------------------------------------------------------------------------
  * Sizing queries (host only; no device work).
@@ -156,7 +162,10 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate,
  * contribute zero.
  *
  *   x            [T, d] x_dtype
- *   topk_idx     [T, k] int32, each row k distinct experts in [0, N)
+ *   topk_idx     [T, k] int32, each row k distinct experts in [0, N); a slot whose
+ *                id is outside [0, N) or repeats an earlier slot of its token is
+ *                treated as dropped (row -1) and recorded as MOE_ERR_INVALID_ARG
+ *                in the device status word (see moe_device_status)
  *   counts       [N] int32 out: selections per expert before capacity (c_e)
  *   offsets      [N+1] int32 out: exclusive scan of kept_e = min(c_e, C)
  *   row_of_slot  [T, k] int32 out: row of slot (t, j) in x_perm, -1 if dropped
@@ -381,12 +390,36 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_
  * pages; mean_t (logsumexp_e z)^2 is used.
  *   counts [N], offsets [N+1], p_partial [nblk, N], lse [T], n_dropped [2],
  *   bias [N] or NULL  (all from the calls above)
+ *   margin [T] fp32 or NULL (moe_route's margin): tokens with margin < near_tie are
+ *          counted in stats->near_ties (-1 when margin is NULL)
  *   stats  moe_stats_t out; f_out [N], p_out [N] fp32 out (either may be NULL)
  * ------------------------------------------------------------------------- */
 int moe_router_stats(const moe_config_t* cfg, const int32_t* counts, const int32_t* offsets,
                      const float* p_partial, const float* lse, const int32_t* n_dropped,
-                     const float* bias, float alpha, float z_coef,
-                     moe_stats_t* stats, float* f_out, float* p_out, void* stream);
+                     const float* margin, float near_tie, const float* bias, float alpha,
+                     float z_coef, moe_stats_t* stats, float* f_out, float* p_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Global statistics over data-parallel ranks: moe_router_stats_partial on every
+ * rank -> element-wise sum of the vectors over ranks (the caller's all-reduce) ->
+ * moe_router_stats_finalize.  The result equals moe_router_stats on the
+ * concatenated batch (the landscape page's TL;DR and 实践要点: balance statistics
+ * should be global, not per micro-batch; the Practice page's load-balance section
+ * on the batch the statistics are taken over).
+ *
+ * moe_router_stats_partial: arguments as moe_router_stats; partial
+ *   [MOE_STATS_PARTIAL_LEN(N)] fp64 out: c_e, kept_e, sum_t s-hat_te for every
+ *   expert, then sum_t lse_t^2, T, dropped slots, dropped tokens, near-ties.
+ * moe_router_stats_finalize: partial as above (summed over ranks); stats, f_out,
+ *   p_out as in moe_router_stats; counts_out [N] int32 out or NULL: the summed
+ *   c_e (input of moe_bias_update, so every rank applies the same update).
+ * ------------------------------------------------------------------------- */
+int moe_router_stats_partial(const moe_config_t* cfg, const int32_t* counts, const int32_t* offsets,
+                             const float* p_partial, const float* lse, const int32_t* n_dropped,
+                             const float* margin, float near_tie, double* partial, void* stream);
+int moe_router_stats_finalize(const moe_config_t* cfg, const double* partial, const float* bias,
+                              float alpha, float z_coef, moe_stats_t* stats, float* f_out,
+                              float* p_out, int32_t* counts_out, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_bias_update -- b[e] += rate * sign(mean(c) - c[e]), optional clamp.
@@ -449,6 +482,12 @@ int moe_route_scores(const moe_config_t* cfg, const void* x, const float* w_gate
                      const float* logit_offset, float* scores, float* lse, float* p_partial,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* Expert-choice capacity (host out): C = min(T, ceil(cf * k * T / N)) with
+ * cf = cfg->capacity_factor (> 0) and k = cfg->top_k read as the average number of
+ * experts per token (the Practice page's C = capacity_factor * k * T / n_experts in
+ * "容量因子、token dropping"), evaluated as ceil((cf * k * T) / N) in double. */
+int moe_expert_choice_capacity(const moe_config_t* cfg, int32_t* capacity);
+
 /* Every expert takes its `capacity` (C, 0 <= C <= T) best tokens.
  *   scores [N, T] (from moe_route_scores); row_of [N, T] int32 out: row of (e, t)
  *   in x_perm or -1; token_of_row [N*C] out; offsets [N+1] out (= e*C);
@@ -475,11 +514,13 @@ int moe_combine_ec(const moe_config_t* cfg, const void* y_perm, const int32_t* r
  * (same outputs, bit for bit) but keeps its per-block count table in a 1 MiB
  * device array inside the library instead of a caller-provided workspace, and
  * calls no allocator.
- *   Arguments: as moe_permute, without ws / ws_bytes.
+ *   Arguments: as moe_permute, without ws / ws_bytes (x_perm = NULL skips the
+ *   gather, as there).
  *   Limit: ceil(T / 256) * N <= 262144 (e.g. N = 256 up to T = 262144 tokens);
  *          larger calls return MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
  *   The first call on a device looks up the array's device address (with that
- *   device current); make that first call before any stream capture.
+ *   device current), and so does the first call after the device's context has
+ *   been replaced (cudaDeviceReset); make those calls before any stream capture.
  *   Every GPU that loads the library holds the array until the process exits.
  *   All calls share the array: calls that overlap on the GPU race, so the
  *   caller must order them (one stream, or explicit events).  Each call
@@ -494,8 +535,11 @@ int moe_permute_noalloc(const moe_config_t* cfg, const void* x, const int32_t* t
  * ------------------------------------------------------------------------- */
 
 /* Reads (and, if reset != 0, clears) the device status word of the current
- * device into *status (host out): MOE_OK or MOE_ERR_DEVICE_TIMEOUT.  Synchronises
- * the current device. */
+ * device into *status (host out): MOE_OK, MOE_ERR_DEVICE_TIMEOUT (a bounded wait
+ * gave up) or MOE_ERR_INVALID_ARG (a kernel met a caller-supplied index outside its
+ * range -- an expert id outside [0, N) or repeated within a token, a sequence range
+ * outside [0, T] -- and skipped that slot: it is treated as dropped and never
+ * dereferenced).  Synchronises the current device. */
 int moe_device_status(int32_t* status, int32_t reset);
 
 /* Self-test of the device-side failure detection: launches one thread that waits,

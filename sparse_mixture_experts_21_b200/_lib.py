@@ -29,7 +29,10 @@ EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_rou
             "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec",
             "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
             "moe_quantize_mxfp8", "moe_permute_mxfp8", "moe_grouped_ffn_mxfp8", "moe_ep_plan",
-            "moe_rows_move")
+            "moe_rows_move", "moe_router_stats_partial", "moe_router_stats_finalize",
+            "moe_expert_choice_capacity")
+
+NEAR_TIE = 1e-4        # margin below which a token counts as a near-tie
 
 
 class MoeConfig(ctypes.Structure):
@@ -45,10 +48,15 @@ class MoeStats(ctypes.Structure):
     _fields_ = [("aux", c_float), ("aux_raw", c_float), ("z", c_float), ("z_loss", c_float),
                 ("cv", c_float), ("cv_kept", c_float), ("bias_norm", c_float), ("dead", c_int32),
                 ("dropped_slots", c_int32), ("dropped_tokens", c_int32), ("R", c_int32),
-                ("reserved", c_int32 * 5)]
+                ("near_ties", c_int32), ("T", c_int64), ("reserved", c_int32 * 2)]
 
 
 STATS_BYTES = ctypes.sizeof(MoeStats)
+
+
+def stats_partial_len(n_experts: int) -> int:
+    """Doubles in the sufficient-statistics vector (MOE_STATS_PARTIAL_LEN)."""
+    return 3 * n_experts + 5
 
 
 class MoeError(RuntimeError):
@@ -81,7 +89,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_permute_noalloc": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "moe_grouped_ffn": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp],
         "moe_combine": [cfgp, vp, vp, vp, vp, vp, vp, vp],
-        "moe_router_stats": [cfgp, vp, vp, vp, vp, vp, vp, c_float, c_float, vp, vp, vp, vp],
+        "moe_router_stats": [cfgp, vp, vp, vp, vp, vp, vp, c_float, vp, c_float, c_float, vp, vp, vp, vp],
+        "moe_router_stats_partial": [cfgp, vp, vp, vp, vp, vp, vp, c_float, vp, vp],
+        "moe_router_stats_finalize": [cfgp, vp, vp, c_float, c_float, vp, vp, vp, vp, vp],
+        "moe_expert_choice_capacity": [cfgp, i32p],
         "moe_bias_update": [cfgp, vp, vp, c_float, c_float, vp],
         "moe_bias_update_ema": [cfgp, vp, vp, c_float, vp, c_float, c_float, vp],
         "moe_bias_update_seq": [cfgp, vp, vp, c_int32, vp, c_float, c_float, vp, c_size_t, vp],
@@ -209,28 +220,6 @@ def mx_scales(rows: int, cols: int, device, groups: int = 0) -> torch.Tensor:
     return torch.empty(max(tiles, 1) * (cols // 128) * 512, dtype=torch.uint8, device=device)
 
 
-def mx_scales_rowmajor(sf, rows: int, cols: int, offsets=None):
-    """Tile atoms -> numpy [rows, cols / 32] scale bytes (rows grouped by `offsets`, a
-    sequence of G + 1 row offsets, or one plain group)."""
-    import numpy as np
-    a = sf.cpu().numpy() if hasattr(sf, "cpu") else np.asarray(sf)
-    nkb = cols // 128
-    off = [0, rows] if offsets is None else [int(o) for o in offsets]
-    out = np.zeros((rows, cols // 32), np.uint8)
-    tile = 0
-    m = np.arange(128)
-    pos = 16 * (m % 32) + 4 * (m // 32)
-    for g in range(len(off) - 1):
-        for r0 in range(off[g], off[g + 1], 128):
-            n = min(128, off[g + 1] - r0)
-            for kb in range(nkb):
-                atom = a[(tile * nkb + kb) * 512:(tile * nkb + kb + 1) * 512]
-                for j in range(4):
-                    out[r0:r0 + n, 4 * kb + j] = atom[pos[:n] + j]
-            tile += 1
-    return out
-
-
 def moe_quantize_mxfp8(x, q, sf, stream=None):
     """MXFP8-quantise a bf16 matrix [rows, cols] along its rows: E4M3 codes and E8M0 scales
     (sf from mx_scales(rows, cols))."""
@@ -276,11 +265,27 @@ def moe_combine(cfg, y_perm, row_of_slot, topk_w, shared_out, y, stream=None, sh
 
 
 def moe_router_stats(cfg, counts, offsets, p_partial, lse, n_dropped, bias, alpha, z_coef, stats,
-                     f_out=None, p_out=None, stream=None):
+                     f_out=None, p_out=None, stream=None, margin=None, near_tie=NEAR_TIE):
     _check("moe_router_stats", load().moe_router_stats(
         ctypes.byref(cfg), _ptr(counts), _ptr(offsets), _ptr(p_partial), _ptr(lse), _ptr(n_dropped),
-        _ptr(bias), float(alpha), float(z_coef), _ptr(stats), _ptr(f_out), _ptr(p_out),
-        _stream(stream)))
+        _ptr(margin), float(near_tie), _ptr(bias), float(alpha), float(z_coef), _ptr(stats), _ptr(f_out),
+        _ptr(p_out), _stream(stream)))
+
+
+def moe_router_stats_partial(cfg, counts, offsets, p_partial, lse, n_dropped, partial, margin=None,
+                             near_tie=NEAR_TIE, stream=None):
+    """This batch's sufficient statistics (fp64 [3N + 5]) for a sum over ranks."""
+    _check("moe_router_stats_partial", load().moe_router_stats_partial(
+        ctypes.byref(cfg), _ptr(counts), _ptr(offsets), _ptr(p_partial), _ptr(lse), _ptr(n_dropped),
+        _ptr(margin), float(near_tie), _ptr(partial), _stream(stream)))
+
+
+def moe_router_stats_finalize(cfg, partial, bias, alpha, z_coef, stats, f_out=None, p_out=None,
+                              counts_out=None, stream=None):
+    """Statistics of the (summed) sufficient-statistics vector."""
+    _check("moe_router_stats_finalize", load().moe_router_stats_finalize(
+        ctypes.byref(cfg), _ptr(partial), _ptr(bias), float(alpha), float(z_coef), _ptr(stats), _ptr(f_out),
+        _ptr(p_out), _ptr(counts_out), _stream(stream)))
 
 
 def moe_bias_update(cfg, counts, bias, rate, clamp=0.0, stream=None):
@@ -306,6 +311,13 @@ def moe_route_scores(cfg, x, w_gate, logit_offset, scores, lse, p_partial, ws, s
     _check("moe_route_scores", load().moe_route_scores(
         ctypes.byref(cfg), _ptr(x), _ptr(w_gate), _ptr(logit_offset), _ptr(scores), _ptr(lse),
         _ptr(p_partial), _ptr(ws), nbytes, _stream(stream)))
+
+
+def expert_choice_capacity(cfg: MoeConfig) -> int:
+    """Expert-choice capacity C = min(T, ceil(cf k T / N)) computed by the library."""
+    out = c_int32()
+    _check("moe_expert_choice_capacity", load().moe_expert_choice_capacity(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
 
 
 def moe_expert_choice(cfg, x, scores, capacity, row_of, token_of_row, offsets, x_perm, n_unpicked=None,

@@ -3,12 +3,27 @@
 #include <math.h>
 
 #include <mutex>
+#include <set>
+#include <tuple>
 
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
+cudaError_t ensure_smem_attr(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::set<std::tuple<const void*, int, int>> done;   // (kernel, device, bytes)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(func, dev, bytes);
+  if (done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return e;
+}
 
 int sm_count() {
   static int cached[64] = {0};
@@ -317,14 +332,38 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_
 
 int moe_router_stats(const moe_config_t* cfg, const int32_t* counts, const int32_t* offsets,
                      const float* p_partial, const float* lse, const int32_t* n_dropped,
-                     const float* bias, float alpha, float z_coef, moe_stats_t* stats, float* f_out,
-                     float* p_out, void* stream) {
+                     const float* margin, float near_tie, const float* bias, float alpha, float z_coef,
+                     moe_stats_t* stats, float* f_out, float* p_out, void* stream) {
   const int st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (!counts || !offsets || !n_dropped || !stats) return MOE_ERR_INVALID_ARG;
   if (cfg->T > 0 && (!p_partial || !lse)) return MOE_ERR_INVALID_ARG;
-  return from_cuda(launch_stats(*cfg, counts, offsets, p_partial, route_nblk(*cfg), lse, n_dropped,
-                                bias, alpha, z_coef, stats, f_out, p_out,
+  return from_cuda(launch_stats(*cfg, 0, counts, offsets, p_partial, route_nblk(*cfg), lse, n_dropped, margin,
+                                near_tie, nullptr, nullptr, bias, alpha, z_coef, stats, f_out, p_out, nullptr,
+                                static_cast<cudaStream_t>(stream)));
+}
+
+int moe_router_stats_partial(const moe_config_t* cfg, const int32_t* counts, const int32_t* offsets,
+                             const float* p_partial, const float* lse, const int32_t* n_dropped,
+                             const float* margin, float near_tie, double* partial, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets || !n_dropped || !partial) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && (!p_partial || !lse)) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(partial) & 7u) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_stats(*cfg, 1, counts, offsets, p_partial, route_nblk(*cfg), lse, n_dropped, margin,
+                                near_tie, nullptr, partial, nullptr, 0.f, 0.f, nullptr, nullptr, nullptr,
+                                nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_router_stats_finalize(const moe_config_t* cfg, const double* partial, const float* bias,
+                              float alpha, float z_coef, moe_stats_t* stats, float* f_out, float* p_out,
+                              int32_t* counts_out, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!partial || !stats || (reinterpret_cast<uintptr_t>(partial) & 7u)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_stats(*cfg, 2, nullptr, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0.f, partial,
+                                nullptr, bias, alpha, z_coef, stats, f_out, p_out, counts_out,
                                 static_cast<cudaStream_t>(stream)));
 }
 
@@ -374,6 +413,17 @@ int moe_route_scores(const moe_config_t* cfg, const void* x, const float* w_gate
   c.n_groups = 1;
   return from_cuda(launch_route(c, x, w_gate, logit_offset, nullptr, nullptr, nullptr, lse, p_partial,
                                 nullptr, nullptr, ws, static_cast<cudaStream_t>(stream), scores));
+}
+
+int moe_expert_choice_capacity(const moe_config_t* cfg, int32_t* capacity) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!capacity || !(cfg->capacity_factor > 0.0)) return MOE_ERR_INVALID_ARG;
+  const double c = ceil((cfg->capacity_factor * (double)cfg->top_k * (double)cfg->T) / (double)cfg->n_experts);
+  const double C = c < (double)cfg->T ? c : (double)cfg->T;
+  if (C > (double)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  *capacity = (int32_t)C;
+  return MOE_OK;
 }
 
 int moe_expert_choice(const moe_config_t* cfg, const void* x, const float* scores, int32_t capacity,

@@ -96,40 +96,96 @@ __device__ double block_sum(double v, double* buf) {
 
 constexpr int kStatThreads = 512;
 
+// Sufficient statistics of one batch, fp64 [3N + 5]: c_e, kept_e, sum_t s-hat_te
+// for every expert, then sum_t lse_t^2, T, dropped slots, dropped tokens, near-ties.
+// Summing these vectors over data-parallel ranks gives the statistics of the
+// concatenated batch.
+enum { ST_SUM_Z = 0, ST_T = 1, ST_DROP_SLOTS = 2, ST_DROP_TOKENS = 3, ST_NEAR = 4, ST_TAIL = 5 };
+
+struct StatsArgs {
+  const int32_t* counts;
+  const int32_t* offsets;
+  const float* p_partial;
+  int nblk;
+  const float* lse;
+  const int32_t* n_dropped;
+  const float* margin;        // NULL: near-ties not counted (reported as -1)
+  float near_tie;
+  const double* part_in;      // mode 2
+  double* part_out;           // mode 1
+  const float* bias;
+  int64_t T;
+  int k, N;
+  float alpha, z_coef;
+  moe_stats_t* st;
+  float* f_out;
+  float* p_out;
+  int32_t* counts_out;        // mode 2: the summed counts as int32 (bias update input)
+};
+
 // Router statistics (llm-compass "负载均衡": L_aux = alpha N sum f_i P_i; the
 // Practice page's load-balance section: 1 before scaling under uniform routing;
 // monitoring metrics from the landscape page's 实践要点).  z-loss reading:
-// mean_t (logsumexp_e z)^2.
-__global__ void __launch_bounds__(kStatThreads)
-stats_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
-             const float* __restrict__ p_partial, int nblk, const float* __restrict__ lse,
-             const int32_t* __restrict__ n_dropped, const float* __restrict__ bias, int64_t T,
-             int k, int N, float alpha, float z_coef, moe_stats_t* __restrict__ st,
-             float* __restrict__ f_out, float* __restrict__ p_out) {
+// mean_t (logsumexp_e z)^2.  MODE 0: this batch's inputs -> moe_stats_t;
+// MODE 1: this batch's inputs -> the sufficient-statistics vector; MODE 2: a
+// (summed) vector -> moe_stats_t.  One CTA, fixed-order fp64 reductions.
+template <int MODE>
+__global__ void __launch_bounds__(kStatThreads) stats_kernel(StatsArgs a) {
   __shared__ double buf[kStatThreads];
-  const int e = threadIdx.x;
-  double c = 0, kept = 0, fP = 0, b2 = 0, dead = 0;
-  if (e < N) {
-    c = counts[e];
-    kept = offsets[e + 1] - offsets[e];
-    double P = 0;
-    for (int b = 0; b < nblk; ++b) P += p_partial[(int64_t)b * N + e];
-    P = T > 0 ? P / (double)T : 0.0;
-    const double f = T > 0 ? c / ((double)k * (double)T) : 0.0;
-    fP = f * P;
-    dead = counts[e] == 0 ? 1.0 : 0.0;
-    if (bias) b2 = (double)bias[e] * bias[e];
-    if (f_out) f_out[e] = (float)f;
-    if (p_out) p_out[e] = (float)P;
+  const int e = threadIdx.x, N = a.N;
+  double c = 0, kept = 0, psum = 0;
+  double zs = 0, near = 0;
+  if (MODE != 2) {
+    if (e < N) {
+      c = a.counts[e];
+      kept = a.offsets[e + 1] - a.offsets[e];
+      for (int b = 0; b < a.nblk; ++b) psum += a.p_partial[(int64_t)b * N + e];
+    }
+    for (int64_t t = threadIdx.x; t < a.T; t += kStatThreads) {
+      zs += (double)a.lse[t] * a.lse[t];
+      if (a.margin) near += a.margin[t] < a.near_tie ? 1.0 : 0.0;
+    }
+  } else if (e < N) {
+    c = a.part_in[e];
+    kept = a.part_in[N + e];
+    psum = a.part_in[2 * N + e];
   }
-  double zs = 0;
-  for (int64_t t = threadIdx.x; t < T; t += kStatThreads) zs += (double)lse[t] * lse[t];
+  const double sum_z = MODE == 2 ? 0.0 : block_sum<kStatThreads>(zs, buf);
+  const double n_near = MODE == 2 ? 0.0 : block_sum<kStatThreads>(near, buf);
+  if (MODE == 1) {
+    if (e < N) {
+      a.part_out[e] = c;
+      a.part_out[N + e] = kept;
+      a.part_out[2 * N + e] = psum;
+    }
+    if (threadIdx.x == 0) {
+      double* tail = a.part_out + 3 * N;
+      tail[ST_SUM_Z] = sum_z;
+      tail[ST_T] = (double)a.T;
+      tail[ST_DROP_SLOTS] = a.n_dropped[0];
+      tail[ST_DROP_TOKENS] = a.n_dropped[1];
+      tail[ST_NEAR] = a.margin ? n_near : -1.0;
+    }
+    return;
+  }
+  const double* tail = MODE == 2 ? a.part_in + 3 * N : nullptr;
+  const double T = MODE == 2 ? tail[ST_T] : (double)a.T;
+  double fP = 0, b2 = 0, dead = 0;
+  if (e < N) {
+    const double P = T > 0 ? psum / T : 0.0;
+    const double f = T > 0 ? c / ((double)a.k * T) : 0.0;
+    fP = f * P;
+    dead = c == 0 ? 1.0 : 0.0;
+    if (a.bias) b2 = (double)a.bias[e] * a.bias[e];
+    if (a.f_out) a.f_out[e] = (float)f;
+    if (a.p_out) a.p_out[e] = (float)P;
+    if (a.counts_out) a.counts_out[e] = (int32_t)c;
+  }
   const double sum_fP = block_sum<kStatThreads>(fP, buf);
   const double sum_c = block_sum<kStatThreads>(c, buf);
   const double sum_k = block_sum<kStatThreads>(kept, buf);
   const double sum_b2 = block_sum<kStatThreads>(b2, buf);
   const double n_dead = block_sum<kStatThreads>(dead, buf);
-  const double sum_z = block_sum<kStatThreads>(zs, buf);
   const double mean_c = sum_c / N, mean_k = sum_k / N;
   const double dc = e < N ? (c - mean_c) * (c - mean_c) : 0.0;
   const double dk = e < N ? (kept - mean_k) * (kept - mean_k) : 0.0;
@@ -137,20 +193,21 @@ stats_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ off
   const double var_k = block_sum<kStatThreads>(dk, buf) / N;
   if (threadIdx.x == 0) {
     const double aux_raw = (double)N * sum_fP;
-    const double z = T > 0 ? sum_z / (double)T : 0.0;
+    const double z = T > 0 ? (MODE == 2 ? tail[ST_SUM_Z] : sum_z) / T : 0.0;
+    moe_stats_t* st = a.st;
     st->aux_raw = (float)aux_raw;
-    st->aux = (float)(alpha * aux_raw);
+    st->aux = (float)(a.alpha * aux_raw);
     st->z = (float)z;
-    st->z_loss = (float)(z_coef * z);
+    st->z_loss = (float)(a.z_coef * z);
     st->cv = mean_c > 0 ? (float)(sqrt(var_c) / mean_c) : 0.f;
     st->cv_kept = mean_k > 0 ? (float)(sqrt(var_k) / mean_k) : 0.f;
     st->bias_norm = (float)sqrt(sum_b2);
     st->dead = (int32_t)n_dead;
-    st->dropped_slots = n_dropped[0];
-    st->dropped_tokens = n_dropped[1];
-    st->R = offsets[N];
-#pragma unroll
-    for (int i = 0; i < 5; ++i) st->reserved[i] = 0;
+    st->dropped_slots = MODE == 2 ? (int32_t)tail[ST_DROP_SLOTS] : a.n_dropped[0];
+    st->dropped_tokens = MODE == 2 ? (int32_t)tail[ST_DROP_TOKENS] : a.n_dropped[1];
+    st->R = (int32_t)sum_k;
+    st->near_ties = MODE == 2 ? (int32_t)tail[ST_NEAR] : (a.margin ? (int32_t)n_near : -1);
+    st->T = MODE == 2 ? (int64_t)T : a.T;
   }
 }
 
@@ -202,12 +259,20 @@ bias_update_ema_kernel(const int32_t* __restrict__ counts, float* __restrict__ e
 // Per-sequence share of each expert: part[b, e] = c_be / len_b (one CTA per sequence).
 __global__ void __launch_bounds__(256)
 seq_load_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ seq_offsets,
-                int k, int N, double* __restrict__ part) {
+                int64_t T, int k, int N, double* __restrict__ part) {
   extern __shared__ int32_t hist[];
   for (int e = threadIdx.x; e < N; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int64_t lo = seq_offsets[blockIdx.x], hi = seq_offsets[blockIdx.x + 1];
-  for (int64_t sl = lo * k + threadIdx.x; sl < hi * k; sl += blockDim.x) atomicAdd(&hist[topk_idx[sl]], 1);
+  int64_t lo = seq_offsets[blockIdx.x], hi = seq_offsets[blockIdx.x + 1];
+  if (lo < 0 || hi > T || lo > hi) {     // a sequence range outside [0, T]: skipped
+    if (threadIdx.x == 0) flag_invalid_index();
+    lo = hi = 0;
+  }
+  for (int64_t sl = lo * k + threadIdx.x; sl < hi * k; sl += blockDim.x) {
+    const int64_t t = sl / k;
+    const int e = checked_expert(topk_idx + t * k, (int)(sl - t * k), N);
+    if (e >= 0) atomicAdd(&hist[e], 1);
+  }
   __syncthreads();
   const double inv = hi > lo ? 1.0 / (double)(hi - lo) : 0.0;
   for (int e = threadIdx.x; e < N; e += blockDim.x)
@@ -276,13 +341,35 @@ cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int3
   return launch_combine_t<float>(c, y_perm, row_of_slot, topk_w, shared_out, shared_w, y, grid, nvec, s);
 }
 
-cudaError_t launch_stats(const moe_config_t& c, const int32_t* counts, const int32_t* offsets,
-                         const float* p_partial, int nblk, const float* lse,
-                         const int32_t* n_dropped, const float* bias, float alpha, float z_coef,
-                         moe_stats_t* stats, float* f_out, float* p_out, cudaStream_t s) {
-  cs::stats_kernel<<<1, cs::kStatThreads, 0, s>>>(counts, offsets, p_partial, nblk, lse, n_dropped, bias,
-                                          c.T, c.top_k, c.n_experts, alpha, z_coef, stats, f_out,
-                                          p_out);
+cudaError_t launch_stats(const moe_config_t& c, int mode, const int32_t* counts, const int32_t* offsets,
+                         const float* p_partial, int nblk, const float* lse, const int32_t* n_dropped,
+                         const float* margin, float near_tie, const double* part_in, double* part_out,
+                         const float* bias, float alpha, float z_coef, moe_stats_t* stats, float* f_out,
+                         float* p_out, int32_t* counts_out, cudaStream_t s) {
+  cs::StatsArgs a;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.p_partial = p_partial;
+  a.nblk = nblk;
+  a.lse = lse;
+  a.n_dropped = n_dropped;
+  a.margin = margin;
+  a.near_tie = near_tie;
+  a.part_in = part_in;
+  a.part_out = part_out;
+  a.bias = bias;
+  a.T = c.T;
+  a.k = c.top_k;
+  a.N = c.n_experts;
+  a.alpha = alpha;
+  a.z_coef = z_coef;
+  a.st = stats;
+  a.f_out = f_out;
+  a.p_out = p_out;
+  a.counts_out = counts_out;
+  if (mode == 0) cs::stats_kernel<0><<<1, cs::kStatThreads, 0, s>>>(a);
+  else if (mode == 1) cs::stats_kernel<1><<<1, cs::kStatThreads, 0, s>>>(a);
+  else cs::stats_kernel<2><<<1, cs::kStatThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -307,8 +394,8 @@ cudaError_t launch_bias_update_seq(const moe_config_t& c, const int32_t* topk_id
                                    const int32_t* seq_offsets, int n_seq, float* bias, float rate,
                                    float clamp, double* ws, cudaStream_t s) {
   if (n_seq > 0)
-    cs::seq_load_kernel<<<n_seq, 256, c.n_experts * sizeof(int32_t), s>>>(topk_idx, seq_offsets, c.top_k,
-                                                                         c.n_experts, ws);
+    cs::seq_load_kernel<<<n_seq, 256, c.n_experts * sizeof(int32_t), s>>>(topk_idx, seq_offsets, c.T,
+                                                                         c.top_k, c.n_experts, ws);
   cs::bias_update_seq_kernel<<<1, cs::kStatThreads, 0, s>>>(ws, n_seq, bias, c.n_experts, rate, clamp);
   return cudaGetLastError();
 }

@@ -21,6 +21,24 @@ __device__ int32_t g_device_status = 0;
 __device__ __forceinline__ void flag_timeout() {
   atomicExch(&g_device_status, (int32_t)MOE_ERR_DEVICE_TIMEOUT);
 }
+// A caller-supplied index outside its range (an expert id, a sequence offset):
+// the offending slot is skipped, never dereferenced, and MOE_ERR_INVALID_ARG is
+// recorded unless an error is already recorded.
+__device__ __forceinline__ void flag_invalid_index() {
+  atomicCAS(&g_device_status, (int32_t)MOE_OK, (int32_t)MOE_ERR_INVALID_ARG);
+}
+// Expert of slot j in one token's row of k ids, or -1 (and the status flag) when the
+// id is outside [0, N) or repeats an earlier slot of the same token.
+__device__ __forceinline__ int checked_expert(const int32_t* __restrict__ row, int j, int N) {
+  const int e = row[j];
+  bool ok = (unsigned)e < (unsigned)N;
+  for (int i = 0; i < j && ok; ++i) ok = row[i] != e;
+  if (!ok) {
+    flag_invalid_index();
+    return -1;
+  }
+  return e;
+}
 
 // About one second at the B200 boost clock; a healthy wait ends in microseconds.
 constexpr long long kWaitLimitCycles = 2000000000LL;

@@ -470,13 +470,8 @@ cudaError_t launch_f8(const CUtensorMap& a, const CUtensorMap& b0, const CUtenso
                       const float* sb0, const float* sb1, const int32_t* offsets, int G, int K, int n_out,
                       int64_t rows_cap, uint8_t* out_q, float* out_s, void* out, cudaStream_t s) {
   constexpr int BN = MODE == 0 ? 128 : 256;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_fp8_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  const cudaError_t e = ensure_smem_attr((const void*)ffn_fp8_kernel<MODE>, (int)kSmem);
+  if (e != cudaSuccess) return e;
   const int64_t tiles_n = (n_out + BN - 1) / BN;
   const int64_t max_tiles = ((rows_cap + BM - 1) / BM + G) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());

@@ -143,8 +143,12 @@ mx_quant_scatter_kernel(const uint4* __restrict__ x, int64_t T, int k, int d, in
     int32_t my_row = -1;
     if (row_of_slot && lane < k) {
       my_row = row_of_slot[t * k + lane];
+      const int e = my_row >= 0 ? topk_idx[t * k + lane] : -1;
+      if ((unsigned)e >= (unsigned)N && my_row >= 0) {
+        flag_invalid_index();           // a kept slot with an expert id outside [0, N)
+        my_row = -1;
+      }
       if (my_row >= 0) {
-        const int e = topk_idx[t * k + lane];
         const int within = my_row - off[e];
         my_tile = tp[e] + within / 128;
         my_m = within & 127;
@@ -515,13 +519,8 @@ cudaError_t launch_mx(const CUtensorMap& a, const CUtensorMap& b0, const CUtenso
                       const uint8_t* sfb0, const uint8_t* sfb1, const int32_t* offsets, int G, int K, int n_out,
                       int64_t rows_cap, uint8_t* out_q, uint8_t* out_sf, void* out, cudaStream_t s) {
   constexpr int BN = MODE == 0 ? 128 : 256;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_mx_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  const cudaError_t e = ensure_smem_attr((const void*)ffn_mx_kernel<MODE>, (int)kSmem);
+  if (e != cudaSuccess) return e;
   const int64_t tiles_n = (n_out + BN - 1) / BN;
   const int64_t max_tiles = ((rows_cap + BM - 1) / BM + G) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());

@@ -460,13 +460,8 @@ cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& b0, const CUten
                         void* out, cudaStream_t s) {
   constexpr int BN = MODE == 0 ? 128 : 256;
   constexpr size_t SMEM = smem_bytes<PAIR>();
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ffn_tc_kernel<MODE, PAIR>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<MODE, PAIR>, (int)SMEM);
+  if (e != cudaSuccess) return e;
   const int64_t tiles_n = (n_out + BN - 1) / BN;
   const int64_t max_tiles = ((rows_cap + Shape<PAIR>::BM - 1) / Shape<PAIR>::BM + G) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());

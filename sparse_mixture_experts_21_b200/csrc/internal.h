@@ -54,10 +54,15 @@ cudaError_t launch_ffn_f32(const float* x_rows, int64_t rows_cap, const int32_t*
 cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
                            const float* topk_w, const void* shared_out, const float* shared_w,
                            void* y, cudaStream_t s);
-cudaError_t launch_stats(const moe_config_t& c, const int32_t* counts, const int32_t* offsets,
-                         const float* p_partial, int nblk, const float* lse,
-                         const int32_t* n_dropped, const float* bias, float alpha, float z_coef,
-                         moe_stats_t* stats, float* f_out, float* p_out, cudaStream_t s);
+// mode 0: this batch -> stats; 1: this batch -> sufficient statistics (part_out);
+// 2: sufficient statistics (part_in, possibly summed over ranks) -> stats.
+cudaError_t launch_stats(const moe_config_t& c, int mode, const int32_t* counts, const int32_t* offsets,
+                         const float* p_partial, int nblk, const float* lse, const int32_t* n_dropped,
+                         const float* margin, float near_tie, const double* part_in, double* part_out,
+                         const float* bias, float alpha, float z_coef, moe_stats_t* stats, float* f_out,
+                         float* p_out, int32_t* counts_out, cudaStream_t s);
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device, size).
+cudaError_t ensure_smem_attr(const void* func, int bytes);
 cudaError_t launch_bias_update(const moe_config_t& c, const int32_t* counts, float* bias,
                                float rate, float clamp, cudaStream_t s);
 cudaError_t launch_bias_update_ema(const moe_config_t& c, const int32_t* counts, float* ema, float beta,

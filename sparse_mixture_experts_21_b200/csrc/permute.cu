@@ -7,6 +7,10 @@
 //   pos(t, j) = #{t' < t : e in idx[t']},  kept iff pos < C,
 //   row = offsets[e] + pos,  offsets = exclusive scan of min(c_e, C).
 //
+// A slot whose expert id is outside [0, N), or repeats an earlier slot of the same
+// token, is treated as dropped (row -1, counted in the dropped slots) and never
+// indexes anything; the device status word then reads MOE_ERR_INVALID_ARG.
+//
 // Four launches, all deterministic (integer atomics only, whose result does not
 // depend on order):
 //   1. hist    per block of kPermuteTokensPerBlock tokens: selections per expert
@@ -34,7 +38,11 @@ permute_hist_kernel(const int32_t* __restrict__ topk_idx, int64_t T, int k, int 
   __syncthreads();
   const int64_t s0 = (int64_t)blockIdx.x * TB * k;
   const int64_t s1 = min((int64_t)(blockIdx.x + 1) * TB, T) * k;
-  for (int64_t sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) atomicAdd(&hist[topk_idx[sl]], 1);
+  for (int64_t sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) {
+    const int64_t t = sl / k;
+    const int e = checked_expert(topk_idx + t * k, (int)(sl - t * k), N);
+    if (e >= 0) atomicAdd(&hist[e], 1);
+  }
   __syncthreads();
   for (int e = threadIdx.x; e < N; e += blockDim.x) blk_counts[(int64_t)blockIdx.x * N + e] = hist[e];
 }
@@ -103,8 +111,8 @@ permute_place_kernel(const int32_t* __restrict__ topk_idx, int64_t T, int k, int
   const int ntok = (int)min((int64_t)TB, T - tb0);
   for (int i = threadIdx.x; i < ntok * k; i += blockDim.x) {
     const int tl = i / k;
-    const int e = topk_idx[(tb0 + tl) * k + i % k];
-    atomicOr(&bits[e * kWordsPerExpert + (tl >> 5)], 1u << (tl & 31));
+    const int e = checked_expert(topk_idx + (tb0 + tl) * k, i % k, N);
+    if (e >= 0) atomicOr(&bits[e * kWordsPerExpert + (tl >> 5)], 1u << (tl & 31));
   }
   __syncthreads();
   // one thread per token of the block: its k slots
@@ -112,7 +120,11 @@ permute_place_kernel(const int32_t* __restrict__ topk_idx, int64_t T, int k, int
     const int64_t t = tb0 + tl;
     bool any_kept = false;
     for (int j = 0; j < k; ++j) {
-      const int e = topk_idx[t * k + j];
+      const int e = checked_expert(topk_idx + t * k, j, N);
+      if (e < 0) {                     // invalid or repeated id: a dropped slot
+        row_of_slot[t * k + j] = -1;
+        continue;
+      }
       const uint32_t* be = bits + e * kWordsPerExpert;
       int rank = __popc(be[tl >> 5] & ((1u << (tl & 31)) - 1u));
       for (int w = 0; w < (tl >> 5); ++w) rank += __popc(be[w]);

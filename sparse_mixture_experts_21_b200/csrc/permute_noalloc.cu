@@ -29,23 +29,53 @@ constexpr int64_t kNoallocScratchInts = 262144;  // 1 MiB of int32
 
 static __device__ __align__(256) int32_t g_permute_scratch[kNoallocScratchInts];
 
-// Device address of the array, looked up once per device with that device
-// current.  (In host code the array's name is only a host-side stand-in.)
+// Device address of the array, looked up with the device current once per device
+// and context.  (In host code the array's name is only a host-side stand-in.)  The
+// cache is keyed by the context's unique id, so after a device reset (a new
+// primary context, in which the module and the array are loaded again) the next
+// call looks the address up again instead of using a stale one.
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int32_t* g_addr[kMaxDevices] = {nullptr};
+unsigned long long g_ctx_id[kMaxDevices] = {0};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+template <class Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess && q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<Fn>(p);
+  return nullptr;
+}
+
+// Unique id of the current context (0 if it cannot be read).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx) get_id(ctx, &id);
+  return id;
+}
 
 cudaError_t scratch_address(int32_t** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // 0 until the runtime has made the device's context current: the lookup below
+  // does that, and the next call then records the context's id
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
+  if (!g_addr[dev] || ctx == 0 || ctx != g_ctx_id[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_permute_scratch);
     if (e != cudaSuccess) return e;
     g_addr[dev] = static_cast<int32_t*>(p);
+    g_ctx_id[dev] = ctx;
   }
   *out = g_addr[dev];
   return cudaSuccess;
@@ -62,9 +92,9 @@ extern "C" int moe_permute_noalloc(const moe_config_t* cfg, const void* x, const
   const int st = capi::check_config(cfg);
   if (st != MOE_OK) return st;
   if (!counts || !offsets || !n_dropped) return MOE_ERR_INVALID_ARG;
-  if (cfg->T > 0 && (!x || !topk_idx || !row_of_slot || !token_of_row || !x_perm))
+  if (cfg->T > 0 && (!topk_idx || !row_of_slot || !token_of_row || (x_perm && !x)))
     return MOE_ERR_INVALID_ARG;
-  if (cfg->T > 0 && (!capi::aligned16(x) || !capi::aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (cfg->T > 0 && x_perm && (!capi::aligned16(x) || !capi::aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
   if ((int64_t)permute_blocks(cfg->T) * cfg->n_experts > noalloc::kNoallocScratchInts)
     return MOE_ERR_WORKSPACE_TOO_SMALL;
   int32_t* scratch = nullptr;

@@ -554,11 +554,13 @@ cudaError_t launch_simt(const moe_config_t& c, const void* x, const float* wg, c
   const unsigned grid = (unsigned)((c.T + TM - 1) / TM);
   if (c.x_dtype == MOE_DTYPE_BF16) {
     auto kern = route_simt_kernel<NP, TM, RM, RN, KS, __nv_bfloat16>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t e = ensure_smem_attr((const void*)kern, (int)smem);
+    if (e != cudaSuccess) return e;
     kern<<<grid, kRouteThreads, smem, s>>>(static_cast<const __nv_bfloat16*>(x), wg, c.d_model, a);
   } else {
     auto kern = route_simt_kernel<NP, TM, RM, RN, KS, float>;
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t e = ensure_smem_attr((const void*)kern, (int)smem);
+    if (e != cudaSuccess) return e;
     kern<<<grid, kRouteThreads, smem, s>>>(static_cast<const float*>(x), wg, c.d_model, a);
   }
   return cudaGetLastError();
@@ -580,7 +582,7 @@ cudaError_t launch_tc(const moe_config_t& c, const void* x, const float* wg, con
       !make_map_bf16(&mw, wsplit, (uint64_t)NP, (uint64_t)3 * dpad, NP))
     return cudaErrorInvalidValue;
   auto kern = route_tc_kernel<NP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+  cudaError_t e = ensure_smem_attr((const void*)kern, (int)S::SMEM);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((c.T + TC_TM - 1) / TC_TM);
   kern<<<grid, TC_THREADS, S::SMEM, s>>>(mx, mw, d, dpad, a);

@@ -11,8 +11,9 @@ Orchestration only; every data-path step runs in the library's kernels:
   4. all-to-all of the rows; moe_rows_move regroups them by local expert;
   5. grouped SwiGLU FFN over the local experts;
   6. moe_rows_move back to arrival order; all-to-all back to the owning ranks;
-  7. shared experts, combine, router statistics and the bias update as in the
-     single-rank layer (the bias update uses the counts summed over ranks).
+  7. shared experts, combine; router statistics of the whole batch (every rank's
+     sufficient statistics summed over ranks) and the bias update on the counts
+     summed over ranks, so every rank keeps the same selection bias.
 
 The exchange is an object with all_gather(t) -> [W, *t.shape],
 all_to_all(out, inp, out_splits, in_splits) and all_reduce_sum(t); TorchDistExchange
@@ -121,9 +122,18 @@ class EPMoELayer:
                           self.w1, self.w3, self.w2, w.f, self.h_loc, self.y_loc, stream)
         L.moe_rows_move(self.y_loc, self.regroup_map, n, self.recv_y, scatter=False, stream=stream)
 
-    def finish(self, x: torch.Tensor, stream=None, counts_global: Optional[torch.Tensor] = None) -> torch.Tensor:
-        """Shared experts, combine (base.y_perm holds the returned rows), statistics,
-        bias update (with the counts summed over ranks when given)."""
+    def stats_partial(self, stream=None) -> torch.Tensor:
+        """This rank's sufficient statistics (fp64 [3N + 5]), to be summed over ranks."""
+        b = self.base
+        L.moe_router_stats_partial(b.cfg, b.counts, b.offsets, b.p_partial, b.lse, b.n_dropped, b.stats_part,
+                                   margin=b.margin, stream=stream)
+        return b.stats_part
+
+    def finish(self, x: torch.Tensor, stream=None, partial_sum: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Shared experts, combine (base.y_perm holds the returned rows), statistics
+        and bias update.  With partial_sum (the sum over ranks of stats_partial())
+        the statistics are the whole batch's and the bias update uses the summed
+        counts; without it, this rank's statistics and no bias update."""
         b, c, w = self.base, self.base.cfg, self.w
         W = b.weights
         shared = None
@@ -132,10 +142,14 @@ class EPMoELayer:
                               stream)
             shared = b.ys
         L.moe_combine(c, b.y_perm, b.row_of_slot, b.topk_w, shared, b.y, stream, shared_w=b.shared_w)
-        L.moe_router_stats(c, b.counts, b.offsets, b.p_partial, b.lse, b.n_dropped, W.get("bias"), w.alpha,
-                           w.z_coef, b.stats, b.f_out, b.p_out, stream)
-        if self.update_bias and counts_global is not None:
-            L.moe_bias_update(c, counts_global, W["bias"], w.bias_rate, 0.0, stream)
+        if partial_sum is None:
+            L.moe_router_stats(c, b.counts, b.offsets, b.p_partial, b.lse, b.n_dropped, W.get("bias"), w.alpha,
+                               w.z_coef, b.stats, b.f_out, b.p_out, stream, margin=b.margin)
+        else:
+            L.moe_router_stats_finalize(c, partial_sum, W.get("bias"), w.alpha, w.z_coef, b.stats, b.f_out,
+                                        b.p_out, self.counts_global, stream)
+            if self.update_bias:
+                L.moe_bias_update(c, self.counts_global, W["bias"], w.bias_rate, 0.0, stream)
         return b.y
 
     # ---------------------------------------------------------------- one rank, real exchange
@@ -146,14 +160,11 @@ class EPMoELayer:
         ex.all_to_all(self.recv_x[:sum(recv)], self.base.x_perm[:sum(send)], recv, send)
         self.local_compute(stream)
         ex.all_to_all(self.base.y_perm[:sum(send)], self.recv_y[:sum(recv)], send, recv)
-        counts_global = None
-        if self.update_bias:
-            self.counts_global.copy_(self.base.counts)
-            counts_global = ex.all_reduce_sum(self.counts_global)
-        return self.finish(x, stream, counts_global)
+        part = ex.all_reduce_sum(self.stats_partial(stream))
+        return self.finish(x, stream, part)
 
     def kernel_launches(self) -> int:
-        # route (+ split), permute (4), plan, two row moves, local FFN (2), shared (2), combine, stats, bias
-        n = 1 + 1 + 4 + 1 + 2 + 2 + 1 + 1
+        # route (+ split), permute (4), plan, two row moves, local FFN (2), combine, stats (2), bias
+        n = 1 + 1 + 4 + 1 + 2 + 2 + 1 + 2
         n += 2 if self.base.fs > 0 else 0
         return n + (1 if self.update_bias else 0)

@@ -6,7 +6,6 @@ stream); every step runs in the library's kernels.
 """
 from __future__ import annotations
 
-import math
 from typing import Optional
 
 import torch
@@ -32,20 +31,16 @@ def make_config(w: Workload, T: Optional[int] = None) -> L.MoeConfig:
     return c
 
 
-def ec_capacity(w: Workload, T: Optional[int] = None) -> int:
-    """Expert-choice capacity C = ceil(cf * k * T / N), at most T."""
-    T = w.T if T is None else T
-    return min(T, math.ceil((w.cf * w.k * T) / w.N))
-
-
 class MoELayer:
     """Holds the weights and the per-call buffers of one layer for up to T tokens."""
 
     def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True,
                  group=None):
         """group: a torch.distributed process group when the layer runs as one of
-        several data-parallel replicas; the bias update then uses the counts summed
-        over the group, so all replicas keep the same selection bias."""
+        several data-parallel replicas; the router statistics are then those of the
+        whole group's batch (each rank's sufficient statistics summed over the
+        group) and the bias update uses the counts summed over the group, so all
+        replicas keep the same selection bias."""
         if w.expert_choice and (w.fp8 or w.mxfp8):
             raise ValueError("expert-choice routing runs bf16 or fp32 experts")
         if (w.fp8 or w.mxfp8) and (w.dtype != "bf16" or w.d % 128 or w.f % 128 or w.f_shared % 128):
@@ -84,11 +79,12 @@ class MoELayer:
             self._init_fp8(z)
         self.stats = torch.zeros(L.STATS_BYTES, dtype=torch.uint8, device=self.dev)
         self.counts_global = z(N, dtype=torch.int32)
+        self.stats_part = z(L.stats_partial_len(N), dtype=torch.float64)
         self.f_out = z(N)
         self.p_out = z(N)
         self.shared_w = z(max(T, 1)) if w.shared_sink else None
         if w.expert_choice:
-            C = self.C = ec_capacity(w)
+            C = self.C = L.expert_choice_capacity(self.cfg)
             self.scores = z(N, max(T, 1))
             self.row_of = z(N, max(T, 1), dtype=torch.int32)
             self.token_of_row = z(max(N * C, 1), dtype=torch.int32)
@@ -181,15 +177,22 @@ class MoELayer:
         L.moe_combine(c, self.y_perm, self.row_of_slot, self.topk_w, shared, y, s,
                       shared_w=self.shared_w)
         rec(5)
-        L.moe_router_stats(c, self.counts, self.offsets, self.p_partial, self.lse, self.n_dropped,
-                           W.get("bias"), self.w.alpha, self.w.z_coef, self.stats, self.f_out,
-                           self.p_out, s)
+        counts = self.counts
+        if self.group is None:
+            L.moe_router_stats(c, self.counts, self.offsets, self.p_partial, self.lse, self.n_dropped,
+                               W.get("bias"), self.w.alpha, self.w.z_coef, self.stats, self.f_out,
+                               self.p_out, s, margin=self.margin)
+        else:
+            # statistics of the whole group's batch: sum the sufficient statistics
+            from .replicas import all_reduce_sum
+            L.moe_router_stats_partial(c, self.counts, self.offsets, self.p_partial, self.lse, self.n_dropped,
+                                       self.stats_part, margin=self.margin, stream=s)
+            with torch.cuda.stream(s):
+                all_reduce_sum(self.stats_part, self.group)
+            L.moe_router_stats_finalize(c, self.stats_part, W.get("bias"), self.w.alpha, self.w.z_coef,
+                                        self.stats, self.f_out, self.p_out, self.counts_global, s)
+            counts = self.counts_global
         if self.update_bias:
-            counts = self.counts
-            if self.group is not None:
-                from .replicas import all_reduce_counts
-                with torch.cuda.stream(s):
-                    counts = all_reduce_counts(self.counts, self.counts_global, self.group)
             L.moe_bias_update(c, counts, W["bias"], self.w.bias_rate, 0.0, s)
         rec(6)
         return y
@@ -288,6 +291,8 @@ class MoELayer:
             n = 1 + 2 + 2 + 1 + (1 if self.w.dtype == "bf16" and self.w.N <= 256 else 0)
             return n + (2 if self.fs > 0 else 0)
         n = 1 + 4 + 2 + 1 + 1          # route, permute (4), routed FFN (2), combine, stats
+        if self.group is not None:
+            n += 1                     # statistics in two launches around the all-reduce
         # FP8: the permutation's bf16 gather is replaced by the quantising scatter
         if self.w.dtype == "bf16" and self.w.N <= 256:
             n += 1                     # exact bf16 split of the router weight

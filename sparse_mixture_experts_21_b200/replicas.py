@@ -1,10 +1,12 @@
 """Host-side plumbing for running the layer as data-parallel replicas.
 
 Each rank routes and computes its own tokens against replicated experts; the
-only exchange is the per-expert selection counts, summed over ranks before the
-aux-loss-free bias update so every replica applies the same update and the
-selection bias stays identical everywhere (the landscape page's point that the
-balancing statistics should be global, not per micro-batch).
+only exchange is each rank's vector of router sufficient statistics (per-expert
+counts, kept counts and affinity sums, sum of lse^2, tokens, drops, near-ties),
+summed over ranks so the statistics and the aux-loss-free bias update are those
+of the whole batch and every replica applies the same update (the landscape
+page's point that the balancing statistics should be global, not per
+micro-batch).
 """
 from __future__ import annotations
 
@@ -17,6 +19,12 @@ def all_reduce_counts(counts: torch.Tensor, out: torch.Tensor, group=None) -> to
     out.copy_(counts)
     dist.all_reduce(out, op=dist.ReduceOp.SUM, group=group)
     return out
+
+
+def all_reduce_sum(t: torch.Tensor, group=None) -> torch.Tensor:
+    """t <- sum over ranks of t, in place."""
+    dist.all_reduce(t, op=dist.ReduceOp.SUM, group=group)
+    return t
 
 
 def max_over_ranks(value: float, device, group=None) -> float:

@@ -56,3 +56,24 @@ def shared_weights(inp: dict):
     if "ws1" not in inp:
         return None
     return f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"])
+
+
+def mx_scales_rowmajor(sf, rows: int, cols: int, offsets=None):
+    """Tile atoms -> numpy [rows, cols / 32] scale bytes (rows grouped by `offsets`, a
+    sequence of G + 1 row offsets, or one plain group)."""
+    a = sf.cpu().numpy() if hasattr(sf, "cpu") else np.asarray(sf)
+    nkb = cols // 128
+    off = [0, rows] if offsets is None else [int(o) for o in offsets]
+    out = np.zeros((rows, cols // 32), np.uint8)
+    tile = 0
+    m = np.arange(128)
+    pos = 16 * (m % 32) + 4 * (m // 32)
+    for g in range(len(off) - 1):
+        for r0 in range(off[g], off[g + 1], 128):
+            n = min(128, off[g + 1] - r0)
+            for kb in range(nkb):
+                atom = a[(tile * nkb + kb) * 512:(tile * nkb + kb + 1) * 512]
+                for j in range(4):
+                    out[r0:r0 + n, 4 * kb + j] = atom[pos[:n] + j]
+            tile += 1
+    return out

@@ -34,6 +34,22 @@ def test_config_struct_layout():
     assert ctypes.sizeof(L.MoeConfig) == 64
     assert L.MoeConfig.capacity_factor.offset == 56
     assert ctypes.sizeof(L.MoeStats) == 64
+    assert L.MoeStats.near_ties.offset == 44 and L.MoeStats.T.offset == 48
+
+
+@pytest.mark.parametrize("T,N,k,cf", [(8192, 64, 6, 1.0), (1000, 7, 3, 1.25), (5, 64, 6, 1.0), (300, 4, 4, 2.0),
+                                      (4097, 96, 2, 0.8)])
+def test_expert_choice_capacity_matches_oracle(lib, T, N, k, cf):
+    """The library's expert-choice capacity (host only) against the oracle's reading,
+    C = min(T, ceil(cf k T / N))."""
+    from oracle import moe_oracle as O
+    w = synth.WORKLOADS["ec_deepseekmoe_16b"]
+    c = layer.make_config(w, T=T)
+    c.n_experts, c.top_k, c.capacity_factor = N, k, cf
+    assert L.expert_choice_capacity(c) == O.expert_choice_capacity(N, k, T, cf)
+    c.capacity_factor = 0.0
+    out = ctypes.c_int32()
+    assert lib.moe_expert_choice_capacity(ctypes.byref(c), ctypes.byref(out)) == L.MOE_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("name", list(synth.WORKLOADS))
@@ -107,7 +123,11 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert lib.moe_grouped_ffn(cp, ok, 10, ok, 0, ok, ok, ok, 256, ok, ok, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_grouped_ffn(cp, ok, 10, ok, 1, ok, ok, ok, 12, ok, ok, None) == L.MOE_ERR_INVALID_ARG
     assert lib.moe_bias_update(cp, None, ok, 1e-3, 0.0, None) == L.MOE_ERR_INVALID_ARG
-    assert lib.moe_router_stats(cp, ok, ok, ok, ok, ok, None, 0.0, 0.0, None, None, None, None) == \
+    assert lib.moe_router_stats(cp, ok, ok, ok, ok, ok, None, 1e-4, None, 0.0, 0.0, None, None, None, None) == \
+        L.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_stats_partial(cp, ok, ok, ok, ok, ok, None, 1e-4, None, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_stats_partial(cp, ok, ok, ok, ok, ok, None, 1e-4, ok + 4, None) == L.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_stats_finalize(cp, None, None, 0.0, 0.0, ok, None, None, None, None) == \
         L.MOE_ERR_INVALID_ARG
 
 

@@ -115,3 +115,59 @@ def test_ep_exchange_two_ranks(tmp_path):
         assert q == len(recv)
         # every row comes home, in place, transformed once
         assert np.array_equal(r[rank]["back"], r[rank]["send"] + 1000.0)
+
+
+# ----------------------------------------------------------------------------- global router statistics
+ST_N, ST_K, ST_T, ST_D = 16, 3, 120, 12
+
+
+def _stats_vector(x, wg, cfg):
+    """The sufficient-statistics layout of moe_router_stats_partial, from the oracle:
+    c_e, kept_e, sum_t s-hat_te, then sum_t lse^2, T, dropped slots, dropped tokens,
+    near-ties (margin < 1e-4)."""
+    r = O.route(x, wg, cfg)
+    p = O.permutation(r["idx"], cfg.n_experts, O.capacity(cfg, x.shape[0]))
+    shat = O.normalised_affinity(r["s"], cfg.score_fn)
+    return np.concatenate([p["counts"], p["kept"], shat.sum(axis=0),
+                           [np.sum(r["lse"] ** 2), x.shape[0], p["dropped_slots"], p["dropped_tokens"],
+                            np.sum(r["margin"] < 1e-4)]])
+
+
+def _stats_worker(rank, port, out_dir):
+    from sparse_mixture_experts_21_b200.replicas import all_reduce_sum
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    try:
+        rng = np.random.default_rng(500)
+        wg = rng.normal(size=(ST_N, ST_D))
+        x = np.random.default_rng(600 + rank).normal(size=(ST_T, ST_D))
+        cfg = O.OracleConfig(ST_N, ST_K, score_fn=O.SIGMOID)
+        v = torch.tensor(_stats_vector(x, wg, cfg), dtype=torch.float64)
+        all_reduce_sum(v)
+        np.savez(os.path.join(out_dir, f"st{rank}.npz"), v=v.numpy(), x=x, wg=wg)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_global_stats_vector_is_the_concatenated_batch(tmp_path):
+    """Every rank's sufficient statistics summed over two gloo ranks equal those of the
+    concatenated batch (dropless, so routing is per token), and the statistics
+    computed from them are the oracle's statistics of the concatenated batch."""
+    mp.start_processes(_stats_worker, args=(_free_port(), str(tmp_path)), nprocs=WORLD, join=True,
+                       start_method="spawn")
+    r = [np.load(tmp_path / f"st{i}.npz") for i in range(WORLD)]
+    assert np.array_equal(r[0]["v"], r[1]["v"])
+    cfg = O.OracleConfig(ST_N, ST_K, score_fn=O.SIGMOID)
+    x_all = np.concatenate([r[i]["x"] for i in range(WORLD)])
+    want = _stats_vector(x_all, r[0]["wg"], cfg)
+    n = ST_N
+    assert np.array_equal(r[0]["v"][:2 * n], want[:2 * n])                       # integer counts exact
+    assert np.allclose(r[0]["v"][2 * n:], want[2 * n:], rtol=1e-13, atol=0)
+    # aux from the summed vector = the oracle's aux on the concatenated batch
+    v, T = r[0]["v"], WORLD * ST_T
+    aux_raw = n * np.sum((v[:n] / (ST_K * T)) * (v[2 * n:3 * n] / T))
+    out = O.layer_forward(x_all, r[0]["wg"], cfg, lambda e: (np.zeros((2, ST_D)), np.zeros((2, ST_D)),
+                                                             np.zeros((ST_D, 2))))
+    assert abs(aux_raw - out["stats"]["aux_raw"]) < 1e-12
+    assert abs(v[3 * n] / T - out["stats"]["z"]) < 1e-12

@@ -5,7 +5,9 @@
 * W = 2 and 4 ranks driven in lock step on one GPU, the all-to-alls done by the
   test with plain copies (no kernel of one rank waits for another): every rank's
   output equals the single-rank layer's on its tokens, bit for bit -- a row's
-  expert result does not depend on which rows share its GEMM tile;
+  expert result does not depend on which rows share its GEMM tile -- and the
+  oracle's layer forward on its tokens within the bf16 bar; the router statistics,
+  summed over ranks, equal the oracle's on the concatenated batch;
 * one rank with a real NCCL exchange (world size 1).
 """
 from __future__ import annotations
@@ -23,6 +25,8 @@ from sparse_mixture_experts_21_b200 import _lib as L
 from sparse_mixture_experts_21_b200.ep import EPMoELayer, TorchDistExchange
 from sparse_mixture_experts_21_b200.layer import MoELayer
 from sparse_mixture_experts_21_b200.synth import WORKLOADS, make_inputs
+from tests.parity_util import (NEAR_TIE, TOL_BF16, TOL_STATS, expert_weights_fn, f64, i64, oracle_cfg, rel_err,
+                               shared_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -100,15 +104,39 @@ def test_ep_lock_step_matches_single_rank(W):
             off_in_d = sum(recv[d][:s])                     # where s's rows sit among d's arrivals
             start, n = sum(send[s][:d]), send[s][d]
             layers[s].base.y_perm[start:start + n] = layers[d].recv_y[off_in_d:off_in_d + n]
-    ys = [lay.finish(x) for lay, x in zip(layers, xs)]
+    # the statistics all-reduce, by a sum
+    psum = torch.stack([lay.stats_partial().clone() for lay in layers]).sum(0)
+    ys = [lay.finish(x, partial_sum=psum) for lay, x in zip(layers, xs)]
     torch.cuda.synchronize()
     assert L.moe_device_status() == L.MOE_OK
+    cfg = oracle_cfg(w)
     for r in range(W):
         single = MoELayer(w, dict(shared, x=xs[r]), "cuda", update_bias=False)
         y_ref = single.forward(xs[r])
         torch.cuda.synchronize()
         assert torch.equal(ys[r][:w.T], y_ref[:w.T]), r
-        assert torch.equal(layers[r].base.stats, single.stats)
+        assert torch.equal(layers[r].base.stats, layers[0].base.stats)     # global: the same on every rank
+        # the oracle's forward on this rank's tokens (dropless: tokens are independent)
+        out = O.layer_forward(f64(xs[r]), f64(shared["w_gate"]), cfg, expert_weights_fn(shared),
+                              shared_weights(shared), bias=f64(shared["bias"]))
+        clear = out["routing"]["margin"] >= NEAR_TIE
+        assert clear.mean() > 0.95
+        assert np.array_equal(i64(layers[r].base.topk_idx)[clear], out["routing"]["idx"][clear])
+        assert rel_err(f64(ys[r][:w.T])[clear], out["y"][clear]) < TOL_BF16, r
+    # global statistics against the oracle on the concatenated batch (counts and drops
+    # from the GPU's expert choice, affinities and lse the oracle's own)
+    x_all = torch.cat(xs)
+    rall = O.route(f64(x_all), f64(shared["w_gate"]), cfg, bias=f64(shared["bias"]))
+    idx_all = np.concatenate([i64(lay.base.topk_idx) for lay in layers])
+    p = O.permutation(idx_all, w.N, None)
+    ost = O.router_stats(p["counts"], p["kept"], rall["s"], rall["lse"], cfg, W * w.T, p["dropped_slots"],
+                         p["dropped_tokens"], w.alpha, w.z_coef, f64(shared["bias"]))
+    st = layers[0].base.stats_dict()
+    for key in ("aux", "aux_raw", "z", "z_loss", "cv", "cv_kept", "bias_norm"):
+        assert abs(st[key] - ost[key]) <= TOL_STATS * max(abs(ost[key]), 1e-30) + 1e-12, key
+    assert st["T"] == W * w.T and st["R"] == p["R"] and st["dead"] == ost["dead"]
+    assert torch.equal(layers[0].counts_global.cpu(), torch.tensor(p["counts"], dtype=torch.int32))
+    assert rel_err(f64(layers[0].base.p_out), ost["P"]) < TOL_STATS
 
 
 def _free_port():

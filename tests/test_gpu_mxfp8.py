@@ -19,7 +19,8 @@ from oracle import moe_oracle as O
 from sparse_mixture_experts_21_b200 import _lib as L
 from sparse_mixture_experts_21_b200.layer import MoELayer, make_config
 from sparse_mixture_experts_21_b200.synth import WORKLOADS, make_inputs
-from tests.parity_util import NEAR_TIE, expert_weights_fn, f64, i64, oracle_cfg, rel_err, shared_weights
+from tests.parity_util import (NEAR_TIE, expert_weights_fn, f64, i64, mx_scales_rowmajor, oracle_cfg, rel_err,
+                               shared_weights)
 from tests.test_gpu_fp8 import decode_e4m3
 
 pytestmark = pytest.mark.gpu
@@ -43,7 +44,7 @@ def gpu_mx(x: torch.Tensor):
 
 def exps(sf: torch.Tensor, rows: int, cols: int, offsets=None) -> np.ndarray:
     """GPU scale bytes (tile atoms) -> exponents [rows, cols / 32]."""
-    return L.mx_scales_rowmajor(sf, rows, cols, offsets).astype(np.int64) - 127
+    return mx_scales_rowmajor(sf, rows, cols, offsets).astype(np.int64) - 127
 
 
 def deq_mx(q: torch.Tensor, sf: torch.Tensor, offsets=None) -> np.ndarray:

@@ -198,9 +198,24 @@ def test_stats_parity(small_runs, name):
         assert abs(st[key] - ost[key]) <= TOL_STATS * max(abs(ost[key]), 1e-30) + 1e-12, key
     for key in ("dead", "dropped_slots", "dropped_tokens"):
         assert st[key] == ost[key], key
-    assert st["R"] == p["R"]
+    assert st["R"] == p["R"] and st["T"] == w.T
     assert rel_err(f64(lay.f_out), ost["f"]) < TOL_STATS
     assert rel_err(f64(lay.p_out), ost["P"]) < TOL_STATS
+    _check_near_ties(st, lay, r["margin"])
+
+
+def _check_near_ties(st, lay, oracle_margin, max_frac=0.05):
+    """The reported near-tie count is the number of the GPU's margins below the
+    threshold, it agrees with the oracle's count up to tokens whose margin sits within
+    a factor 2 of the threshold (where fp32 and fp64 may fall on different sides),
+    and near-ties stay a small fraction of the tokens."""
+    gm = f64(lay.margin)[:len(oracle_margin)]
+    assert st["near_ties"] == int((gm < NEAR_TIE).sum())
+    n_oracle = int((oracle_margin < NEAR_TIE).sum())
+    border = int(((oracle_margin >= NEAR_TIE / 2) & (oracle_margin < 2 * NEAR_TIE)).sum())
+    assert abs(st["near_ties"] - n_oracle) <= border
+    assert n_oracle <= max_frac * len(oracle_margin)
+    return n_oracle
 
 
 def test_bias_update_parity():
@@ -290,6 +305,83 @@ def test_permute_many_blocks_dropless():
     _permute_with(w, idx)
 
 
+def test_permute_invalid_expert_ids_are_dropped_and_flagged():
+    """Expert ids outside [0, N) and repeats within a token: those slots are treated
+    as dropped (row -1) and never dereferenced, the rest is the oracle's permutation
+    of the valid slots, and the device status word reports MOE_ERR_INVALID_ARG."""
+    assert L.moe_device_status() == L.MOE_OK
+    for capacity in ("dropless", "ceil_cf_T_over_N"):
+        w = replace(SMALL["v3_small"], T=700, N=16, k=4, capacity=capacity, cf=1.5)
+        idx = random_routing(w.T, w.N, w.k, "cpu", seed=21).numpy().astype(np.int32)
+        idx[3, 1] = w.N + 5                       # out of range
+        idx[10, 0] = -1                           # negative
+        idx[11, 3] = 1 << 30                      # far out of range
+        idx[20, 2] = idx[20, 0]                   # a repeat within the token
+        idx[40, :] = w.N                          # every slot invalid: a dropped token
+        bad = (idx < 0) | (idx >= w.N)
+        bad[20, 2] = True
+        clean = np.where(bad, w.N, idx).astype(np.int64)       # invalid slots -> a dummy last expert
+        C = O.capacity(oracle_cfg(w), w.T)
+        ref = O.permutation(clean, w.N + 1, C)
+        c = make_config(w)
+        dev = lambda *s_, dtype=torch.int32: torch.full(s_, -7, dtype=dtype, device="cuda")  # noqa: E731
+        counts, offsets, ros, tor, nd = dev(w.N), dev(w.N + 1), dev(w.T, w.k), dev(w.T * w.k), dev(2)
+        x = torch.randn(w.T, w.d, device="cuda").to(torch.bfloat16)
+        xp = torch.zeros(w.T * w.k, w.d, dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(max(L.workspace_size(c), 16), dtype=torch.uint8, device="cuda")
+        L.moe_permute(c, x, torch.tensor(idx, device="cuda"), counts, offsets, ros, tor, xp, nd, ws)
+        torch.cuda.synchronize()
+        assert L.moe_device_status() == L.MOE_ERR_INVALID_ARG      # read and cleared
+        assert L.moe_device_status() == L.MOE_OK
+        R = int(ref["offsets"][w.N])
+        assert np.array_equal(i64(counts), ref["counts"][:w.N])
+        assert np.array_equal(i64(offsets), ref["offsets"][:w.N + 1])
+        assert np.array_equal(i64(ros), np.where(bad, -1, ref["row_of_slot"]))
+        assert np.array_equal(i64(tor)[:R], ref["token_of_row"][:R])
+        keep_valid = (~bad) & ref["keep"]
+        assert i64(nd).tolist() == [w.T * w.k - R, int((~keep_valid).all(axis=1).sum())]
+        assert torch.equal(xp[:R], x[tor[:R].long()])
+
+
+def test_stats_summed_over_split_batches_equal_whole_batch():
+    """Sufficient statistics of two halves of a batch, summed (what the all-reduce
+    over data-parallel ranks does) and finalised, equal the statistics of the whole
+    batch and the oracle's on all tokens (dropless routing is per token)."""
+    w = SMALL["v3_small"]
+    inp = make_inputs(w, "cuda")
+    whole = MoELayer(w, inp, "cuda", update_bias=False)
+    whole.forward(inp["x"])
+    half = w.T // 2
+    parts = []
+    for lo, hi in ((0, half), (half, w.T)):
+        wh = replace(w, T=hi - lo)
+        lay = MoELayer(wh, dict(inp, x=inp["x"][lo:hi].contiguous()), "cuda", update_bias=False)
+        lay.forward(lay.weights["x"])
+        L.moe_router_stats_partial(lay.cfg, lay.counts, lay.offsets, lay.p_partial, lay.lse, lay.n_dropped,
+                                   lay.stats_part, margin=lay.margin)
+        parts.append(lay.stats_part.clone())
+    total = parts[0] + parts[1]
+    stats = torch.zeros(L.STATS_BYTES, dtype=torch.uint8, device="cuda")
+    f_out = torch.empty(w.N, device="cuda")
+    p_out = torch.empty(w.N, device="cuda")
+    cglob = torch.empty(w.N, dtype=torch.int32, device="cuda")
+    L.moe_router_stats_finalize(whole.cfg, total, inp["bias"], w.alpha, w.z_coef, stats, f_out, p_out, cglob)
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    st, st_whole = L.stats_from_tensor(stats), whole.stats_dict()
+    assert torch.equal(cglob, whole.counts)
+    for key in ("dead", "dropped_slots", "dropped_tokens", "R", "near_ties", "T"):
+        assert st[key] == st_whole[key], key
+    cfg = oracle_cfg(w)
+    r = O.route(f64(inp["x"]), f64(inp["w_gate"]), cfg, bias=f64(inp["bias"]))
+    p = O.permutation(i64(whole.topk_idx), w.N, O.capacity(cfg, w.T))
+    ost = O.router_stats(p["counts"], p["kept"], r["s"], r["lse"], cfg, w.T, p["dropped_slots"],
+                         p["dropped_tokens"], w.alpha, w.z_coef, f64(inp["bias"]))
+    for key in ("aux", "aux_raw", "z", "z_loss", "cv", "cv_kept", "bias_norm"):
+        assert abs(st[key] - ost[key]) <= TOL_STATS * max(abs(ost[key]), 1e-30) + 1e-12, key
+    assert rel_err(f64(f_out), ost["f"]) < TOL_STATS and rel_err(f64(p_out), ost["P"]) < TOL_STATS
+
+
 def test_grouped_ffn_empty_and_tiny_groups():
     """Groups with 0, 1, 127, 128, 129 rows and rows_cap beyond the last row."""
     d, f = 256, 384
@@ -351,11 +443,22 @@ def test_full_size_workload(name):
     out = O.layer_forward(f64(inp["x"]), None, cfg, expert_weights_fn(inp), shared_weights(inp),
                           tokens=tok, routing={"idx": i64(lay.topk_idx), "w": wts})
     assert rel_err(f64(lay.y[torch.tensor(tok, device="cuda")]), out["y"]) < tol_for(w)
+    # statistics on every token: the oracle routes all T tokens in fp64 (its own
+    # affinities and lse), counts and drops from the GPU's expert choice (cross-fed)
+    rall = O.route(f64(inp["x"]), f64(inp["w_gate"]), cfg, bias=f64(inp["bias"]),
+                   logit_offset=f64(inp["logit_offset"]))
+    ost = O.router_stats(p["counts"], p["kept"], rall["s"], rall["lse"], cfg, w.T, p["dropped_slots"],
+                         p["dropped_tokens"], w.alpha, w.z_coef, f64(inp["bias"]))
     st = lay.stats_dict()
-    assert st["dropped_slots"] == p["dropped_slots"] and st["R"] == p["R"]
-    assert st["dead"] == int((p["counts"] == 0).sum())
-    c = p["counts"].astype(np.float64)
-    assert abs(st["cv"] - np.std(c) / np.mean(c)) <= TOL_STATS * max(np.std(c) / np.mean(c), 1e-30)
+    for key in ("aux", "aux_raw", "z", "z_loss", "cv", "cv_kept", "bias_norm"):
+        assert abs(st[key] - ost[key]) <= TOL_STATS * max(abs(ost[key]), 1e-30) + 1e-12, key
+    for key in ("dead", "dropped_slots", "dropped_tokens"):
+        assert st[key] == ost[key], key
+    assert st["R"] == p["R"] and st["T"] == w.T
+    assert rel_err(f64(lay.f_out), ost["f"]) < TOL_STATS
+    assert rel_err(f64(lay.p_out), ost["P"]) < TOL_STATS
+    n_oracle = _check_near_ties(st, lay, rall["margin"])
+    print(f"{name}: near-ties {st['near_ties']} (oracle {n_oracle}) of {w.T} tokens")
 
 
 def test_forward_host_pipeline_matches_forward():

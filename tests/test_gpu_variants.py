@@ -107,7 +107,8 @@ def test_bias_update_seq():
 
 
 # ----------------------------------------------------------------------------- expert choice
-from sparse_mixture_experts_21_b200.layer import ec_capacity  # noqa: E402
+def ec_capacity(w):
+    return L.expert_choice_capacity(make_config(w))
 
 
 @pytest.mark.parametrize("score,dtype", [("softmax", "bf16"), ("sigmoid", "bf16"), ("softmax", "fp32")])

@@ -9,9 +9,11 @@ is collected last so that a failure here cannot hide the other tests.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+from oracle import moe_oracle as O
 from sparse_mixture_experts_21_b200 import _lib as L
 from sparse_mixture_experts_21_b200.layer import make_config
 from sparse_mixture_experts_21_b200.synth import WORKLOADS, random_routing
@@ -45,6 +47,28 @@ def test_noalloc_matches_permute_twice(name, T, seed):
         torch.cuda.synchronize()
         for key in ref:
             assert torch.equal(ref[key], got[key]), f"call {call}: {key} differs"
+        # and against the oracle's permutation of the same routing
+        p = O.permutation(idx.cpu().numpy().astype(np.int64), w.N, None)
+        assert np.array_equal(got["counts"].cpu().numpy(), p["counts"])
+        assert np.array_equal(got["offsets"].cpu().numpy(), p["offsets"])
+        assert np.array_equal(got["ros"].cpu().numpy(), p["row_of_slot"])
+        assert np.array_equal(got["tor"].cpu().numpy()[:p["R"]], p["token_of_row"])
+
+
+def test_noalloc_without_gather():
+    """x_perm = NULL skips the row gather, as in moe_permute (x may then be NULL)."""
+    from dataclasses import replace
+    w = replace(WORKLOADS["deepseek_v3"], T=3000, d=256)
+    c = make_config(w)
+    idx = random_routing(w.T, w.N, w.k, "cuda", seed=13)
+    ws = torch.empty(max(L.workspace_size(c), 16), dtype=torch.uint8, device="cuda")
+    ref, got = _buffers(w), _buffers(w)
+    L.moe_permute(c, None, idx, ref["counts"], ref["offsets"], ref["ros"], ref["tor"], None, ref["nd"], ws)
+    L.moe_permute_noalloc(c, None, idx, got["counts"], got["offsets"], got["ros"], got["tor"], None, got["nd"])
+    torch.cuda.synchronize()
+    for key in ("counts", "offsets", "ros", "tor", "nd"):
+        assert torch.equal(ref[key], got[key]), key
+    assert torch.all(got["xp"] == 0)
 
 
 def test_noalloc_rejects_sizes_beyond_its_array():
