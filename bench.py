@@ -179,8 +179,13 @@ def run_reference(args, rank):
 
 
 # ---------------------------------------------------------------------------- our arm
-def cpu_baseline(inp, w, seconds_target=20.0):
-    """Oracle timed on a bounded sample (a few tokens of the same workload)."""
+def cpu_baseline(inp, w, seconds_target=20.0, chunk=4, max_tokens=64, threads=None):
+    """Oracle timed on a bounded sample (the first tokens of the same workload, `chunk`
+    tokens per oracle call, until `seconds_target` or `max_tokens`; a workload smaller
+    than the sample is run again from its first token).  threads: cap on the BLAS
+    threads (None: every host core)."""
+    from threadpoolctl import threadpool_limits
+
     from oracle import moe_oracle as O
     cfg = _oracle_cfg(O, w)
     f64 = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
@@ -191,19 +196,43 @@ def cpu_baseline(inp, w, seconds_target=20.0):
     def experts(e):
         return f64(inp["w1"][e]), f64(inp["w3"][e]), f64(inp["w2"][e])
 
+    cores = len(os.sched_getaffinity(0)) if threads is None else threads
     done, t0 = 0, time.perf_counter()
-    chunk = 4
-    while True:
-        x = f64(inp["x"][done:done + chunk])
-        O.layer_forward(x, wg, cfg, experts, shared, bias=bias, logit_offset=off, alpha=w.alpha,
-                        z_coef=w.z_coef, expert_ffn=ffn)
-        done += chunk
-        el = time.perf_counter() - t0
-        if el > seconds_target or done >= 64:
-            break
-    return {"value": done / el, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
-            "sample": f"first {done} tokens of the {w.name} workload, {chunk} per oracle call "
+    with threadpool_limits(limits=cores):
+        while True:
+            t0_ = done % w.T                       # wraps around small workloads
+            x = f64(inp["x"][t0_:t0_ + chunk])
+            O.layer_forward(x, wg, cfg, experts, shared, bias=bias, logit_offset=off, alpha=w.alpha,
+                            z_coef=w.z_coef, expert_ffn=ffn)
+            done += chunk
+            el = time.perf_counter() - t0
+            if el > seconds_target or done >= max_tokens:
+                break
+    return {"value": done / el, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} tokens of the {w.name} workload from its first, {chunk} per oracle call "
                       f"(routing, experts, shared expert, combine, stats), {el:.1f} s"}
+
+
+def run_cpu_baselines(args):
+    """The oracle on every workload of the task (host cores; also one core for the
+    three smaller ones): one JSON line per (workload, cores).  Inputs are drawn on the
+    GPU with the workload's seed, so they are the bytes the GPU path sees."""
+    from sparse_mixture_experts_21_b200.synth import WORKLOADS, make_inputs
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    plan = [("tiny_top2_fp32", 256, 256 * 1000, (None, 1)), ("mixtral_8x7b", 8, 64, (None, 1)),
+            ("deepseekmoe_16b", 32, 256, (None, 1)), ("deepseek_v3", 4, 64, (None,)),
+            ("switch_skewed", 64, 1024, (None,))]
+    for name, chunk, max_tokens, cores in plan:
+        w = WORKLOADS[name]
+        inp = make_inputs(w, dev)
+        for c in cores:
+            r = cpu_baseline(inp, w, seconds_target=args.cpu_seconds, chunk=chunk, max_tokens=max_tokens,
+                             threads=c)
+            print(json.dumps({"workload": name, **r}), flush=True)
+        del inp
+        if dev == "cuda":
+            torch.cuda.empty_cache()
+    return 0
 
 
 def main():
@@ -214,6 +243,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-baselines", action="store_true",
+                    help="time the oracle on every workload (host cores, and one core for the smaller ones)")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay measurement")
     ap.add_argument("--workload", default=WORKLOAD,
@@ -230,6 +262,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.cpu_baselines:
+        return run_cpu_baselines(args) if rank == 0 else 0
 
     from sparse_mixture_experts_21_b200 import _lib as L
     from sparse_mixture_experts_21_b200.layer import MoELayer

@@ -382,10 +382,16 @@ def test_stats_summed_over_split_batches_equal_whole_batch():
     assert rel_err(f64(f_out), ost["f"]) < TOL_STATS and rel_err(f64(p_out), ost["P"]) < TOL_STATS
 
 
-def test_grouped_ffn_empty_and_tiny_groups():
-    """Groups with 0, 1, 127, 128, 129 rows and rows_cap beyond the last row."""
-    d, f = 256, 384
-    sizes = [0, 1, 127, 0, 128, 129, 300, 0]
+@pytest.mark.parametrize("d,f,sizes", [
+    (256, 384, [0, 1, 127, 0, 128, 129, 300, 0]),
+    # every tile kind: tails of 1..127 rows alone, after one full 128-row tile, after
+    # full pairs; partial last n-tiles in both passes (f = 320, d = 384)
+    (384, 320, [16, 17, 112, 113, 255, 256, 257, 383, 384, 385, 511, 640, 5, 0, 31]),
+])
+def test_grouped_ffn_empty_and_tiny_groups(d, f, sizes):
+    """Groups with 0, 1, 127, 128, 129 ... rows (every kind of tile: two full 128-row
+    sub-tiles, one, one with the group's ragged tail computed transposed, the tail
+    alone) and rows_cap beyond the last row."""
     G = len(sizes)
     off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     R, cap = int(off[-1]), int(off[-1]) + 70
@@ -405,6 +411,10 @@ def test_grouped_ffn_empty_and_tiny_groups():
         if hi > lo:
             ref[lo:hi] = O.swiglu_ffn(f64(xr[lo:hi]), f64(w1[e]), f64(w3[e]), f64(w2[e]))
     assert rel_err(f64(y[:R]), ref) < 2e-2
+    for e in range(G):                                 # each group on its own scale
+        lo, hi = off[e], off[e + 1]
+        if hi > lo:
+            assert rel_err(f64(y[lo:hi]), ref[lo:hi]) < 2e-2, (e, sizes[e])
     assert torch.all(y[R:] == 3.0)                     # rows past the last group untouched
 
 
