@@ -235,6 +235,109 @@ def run_cpu_baselines(args):
     return 0
 
 
+def run_ep(args, w, world, rank, local, dev, pg):
+    """Expert parallelism: every rank routes its own T tokens, holds N / W experts, and
+    exchanges rows with the others (all-to-all dispatch and return, in rounds bounded
+    by the receive buffer).  Weak scaling: T tokens per rank."""
+    from sparse_mixture_experts_21_b200 import _lib as L
+    from sparse_mixture_experts_21_b200.ep import EPMoELayer, TorchDistExchange
+    from sparse_mixture_experts_21_b200.replicas import max_over_ranks
+    from sparse_mixture_experts_21_b200.synth import make_inputs
+
+    if pg is None:
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29531")
+        dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    inp = make_inputs(w, dev, seed=0)                       # router and experts: the same on every rank
+    x = make_inputs(w, dev, seed=100 + rank, experts=False)["x"]  # this rank's tokens
+    lay = EPMoELayer(w, inp, rank, world, dev, exchange=TorchDistExchange(), recv_factor=args.recv_factor)
+    for name in ("w1", "w3", "w2"):                         # only this rank's experts stay resident
+        inp[name] = None
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        pg.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        lay.forward(x)
+    barrier()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    marks = [[ev() for _ in range(4)] for _ in range(args.steps)]
+    rounds = []
+    with ClockSampler(_device_uuid(local)) as clk:
+        barrier()
+        start, end = ev(), ev()
+        start.record(stream)
+        for i in range(args.steps):
+            lay.forward(x, stream, marks[i])
+            rounds.append(len(lay.plans) if world > 1 else 1)
+        end.record(stream)
+        barrier()
+    ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
+    assert L.moe_device_status() == L.MOE_OK
+    stage = lambda a, b: statistics.mean(marks[i][a].elapsed_time(marks[i][b]) for i in range(args.steps))  # noqa: E731
+    t_route_perm, t_expert, t_finish = stage(0, 1), stage(1, 2), stage(2, 3)
+    t_expert_max = max_over_ranks(t_expert, dev)
+    # rows this rank's experts computed in the last step, and their FLOPs
+    R_local = int(lay.base.offsets[-1].item()) if world == 1 else \
+        sum(sum(p.recv_count) for p in lay.plans)
+    flops_local = 6.0 * R_local * w.d * w.f
+    peaks = _peaks()
+    tflops = flops_local / (t_expert * 1e-3) / 1e12
+    st = lay.base.stats_dict()
+
+    # end to end: each step copies its tokens from pinned host memory and its output back
+    xh = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    xh.copy_(x)
+    yh = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    xd = torch.empty_like(x)
+    barrier()
+    s0, s1 = ev(), ev()
+    s0.record(stream)
+    for _ in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        y = lay.forward(xd)
+        yh.copy_(y[: w.T], non_blocking=True)
+    s1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1) / args.steps, dev)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * w.T / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "T_per_rank": w.T, "d_model": w.d, "experts": w.N, "top_k": w.k,
+                       "d_ff": w.f, "shared_experts": w.n_shared, "parallelism": f"ep{world}",
+                       "experts_per_rank": w.N // world, "recv_factor": args.recv_factor,
+                       "rounds_per_step": max(rounds) if rounds else 1,
+                       "l2": "inputs larger than L2 (x 235 MB per rank, local expert weights "
+                             f"{3 * (w.N // world) * w.d * w.f * 2 / 1e9:.1f} GB); no flush"},
+            "roofline": {"kernel": "exchange + local grouped SwiGLU FFN (rank 0)", "bound": "tensor",
+                         "achieved": tflops, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops_sustained"], "traffic": None,
+                         "peak_source": peaks["source"] + " sustained bf16"},
+            "stages_ms": {"route_permute": t_route_perm, "exchange_and_experts": t_expert,
+                          "exchange_and_experts_max_over_ranks": t_expert_max, "shared_combine_stats": t_finish},
+            "near_ties": {"count": st["near_ties"], "tokens": st["T"], "threshold": L.NEAR_TIE},
+            "gpu_launches": lay.kernel_launches() * args.steps,
+            "clocks": clk.summary(),
+            "e2e": {"value": world * w.T / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+                    "d2h_bytes_per_step": yh.numel() * yh.element_size(), "ms_per_step": e2e_ms,
+                    "api": "EPMoELayer.forward (pinned host in/out per step)"},
+            "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    pg.barrier()
+    pg.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -254,6 +357,11 @@ def main():
                     help="reduced token count (profiling of a small case only)")
     ap.add_argument("--experts", type=int, default=None,
                     help="reduced routed-expert count (profiling of a small case only)")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
+                    help="replicas: every rank holds every expert; ep: expert parallelism (N / W experts per "
+                         "rank, all-to-all dispatch and return)")
+    ap.add_argument("--recv-factor", type=float, default=1.0,
+                    help="ep: receive buffer rows as a multiple of T * k (rounds bound it)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
@@ -282,6 +390,8 @@ def main():
     if args.tokens or args.experts:
         from dataclasses import replace
         w = replace(w, name=w.name + "_reduced", T=args.tokens or w.T, N=args.experts or w.N)
+    if args.parallel == "ep":
+        return run_ep(args, w, world, rank, local, dev, pg)
     inp = make_inputs(w, dev, seed=rank)
     lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD)
     x = inp["x"]

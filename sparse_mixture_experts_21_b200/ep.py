@@ -5,30 +5,53 @@ Orchestration only; every data-path step runs in the library's kernels:
   1. route and permute the rank's own tokens over all N experts (rows ordered by
      expert, hence by destination rank: they are the dispatch send buffer);
   2. exchange the expert offsets (all-gather) -- the counts travel before the rows;
-  3. moe_ep_plan: split sizes, local expert offsets, regroup map (on the device);
-     the split sizes are copied to the host for the all-to-all (the one
-     synchronisation of the exchange);
-  4. all-to-all of the rows; moe_rows_move regroups them by local expert;
-  5. grouped SwiGLU FFN over the local experts;
-  6. moe_rows_move back to arrival order; all-to-all back to the owning ranks;
-  7. shared experts, combine; router statistics of the whole batch (every rank's
+  3. plan the exchange on the host (the one synchronisation of a forward): every
+     rank derives the same plan from the all-gathered offsets.  The rows a rank
+     receives are bounded by its receive buffer (recv_factor * T * k rows, at
+     least T): a destination's (source, expert) pieces are packed, in expert then
+     source order, into rounds that each fit the buffer, and every rank runs as
+     many rounds as the busiest destination needs;
+  4. per round: all-to-all of the round's rows; moe_ep_plan + moe_rows_move regroup
+     them by local expert; grouped SwiGLU FFN over the local experts; moe_rows_move
+     back to arrival order; all-to-all back into the owning ranks' y_perm;
+  5. shared experts, combine; router statistics of the whole batch (every rank's
      sufficient statistics summed over ranks) and the bias update on the counts
      summed over ranks, so every rank keeps the same selection bias.
 
+With a real exchange (forward) rounds use two buffer sets: round r + 1's dispatch
+is issued before round r's expert compute and round r's return right after it, so
+the transfers overlap the grouped GEMMs ([Practice] "通信优化按什么顺序做": overlap
+the dispatch with expert compute).
+
 The exchange is an object with all_gather(t) -> [W, *t.shape],
-all_to_all(out, inp, out_splits, in_splits) and all_reduce_sum(t); TorchDistExchange
-runs them with torch.distributed (NCCL over NVLink on GPUs).  The phases are
-separate methods so a caller can drive several ranks' layers in lock step.
+all_to_all(out_list, in_list, async_op) (lists of per-rank tensors; async_op returns
+a handle with wait()) and all_reduce_sum(t); TorchDistExchange runs them with
+torch.distributed (NCCL over NVLink on GPUs).  The phases are separate methods so a
+caller can drive several ranks' layers in lock step.
 """
 from __future__ import annotations
 
-from typing import Optional
+import math
+from dataclasses import dataclass
+from typing import List, Optional
 
+import numpy as np
 import torch
 
 from . import _lib as L
 from .layer import MoELayer
 from .synth import Workload
+
+
+class _Works:
+    """Handle of a batch of point-to-point operations."""
+
+    def __init__(self, works):
+        self.works = works
+
+    def wait(self):
+        for w in self.works:
+            w.wait()
 
 
 class TorchDistExchange:
@@ -44,29 +67,116 @@ class TorchDistExchange:
         self.dist.all_gather_into_tensor(out, t.contiguous().reshape(-1), group=self.group)
         return out.view((self.world,) + tuple(t.shape))
 
-    def all_to_all(self, out, inp, out_splits, in_splits):
-        self.dist.all_to_all_single(out, inp, output_split_sizes=list(out_splits),
-                                    input_split_sizes=list(in_splits), group=self.group)
+    def all_to_all(self, out_list, in_list, async_op: bool = False):
+        """out_list[s] <- what rank s sends here; in_list[d] -> rank d.  Batched
+        point-to-point sends and receives (one grouped call under NCCL); a rank's own
+        slice is a local copy and empty slices are skipped on both ends."""
+        dist = self.dist
+        ops = []
+        for peer in range(self.world):
+            gpeer = peer if self.group is None else dist.get_global_rank(self.group, peer)
+            if peer == self.rank:
+                if out_list[peer].numel():
+                    out_list[peer].copy_(in_list[peer])
+                continue
+            if in_list[peer].numel():
+                ops.append(dist.P2POp(dist.isend, in_list[peer], gpeer, self.group))
+            if out_list[peer].numel():
+                ops.append(dist.P2POp(dist.irecv, out_list[peer], gpeer, self.group))
+        handle = _Works(dist.batch_isend_irecv(ops) if ops else [])
+        if async_op:
+            return handle
+        handle.wait()
+        return None
 
     def all_reduce_sum(self, t: torch.Tensor) -> torch.Tensor:
         self.dist.all_reduce(t, group=self.group)
         return t
 
 
+# ----------------------------------------------------------------------------- host plan
+def plan_rounds(kept: np.ndarray, world: int, cap: int):
+    """Pack every destination's (source, expert) pieces into rounds of at most `cap`
+    received rows.  kept [W, N]: rows source s keeps for expert e.  A destination
+    takes its experts in order and, for each, the sources in order; a piece opens a
+    new round when it does not fit the current one (a piece never exceeds T <= cap
+    rows, since a token picks an expert at most once).  Returns (round_of [W, N], R):
+    the round of each piece at its destination, and the number of rounds every rank
+    runs (that of the busiest destination, at least 1).  Deterministic, so every
+    rank computes the same plan."""
+    W, N = kept.shape
+    El = N // world
+    round_of = np.zeros((W, N), np.int64)
+    R = 1
+    for d in range(world):
+        cur, r = 0, 0
+        for e in range(d * El, (d + 1) * El):
+            for s in range(W):
+                n = int(kept[s, e])
+                if n > cap:
+                    raise ValueError(f"a piece of {n} rows exceeds the receive capacity {cap}")
+                if n and cur + n > cap:
+                    r, cur = r + 1, 0
+                round_of[s, e] = r
+                cur += n
+        R = max(R, r + 1)
+    return round_of, R
+
+
+@dataclass
+class RoundPlan:
+    offsets_all: np.ndarray        # [W, N + 1] offsets of the round's pieces only (moe_ep_plan input)
+    send_start: List[int]          # per destination: first row of this rank's x_perm it sends
+    send_count: List[int]          # per destination: rows sent
+    recv_count: List[int]          # per source: rows received
+
+
+def round_plans(offsets_all: np.ndarray, rank: int, world: int, cap: int) -> List[RoundPlan]:
+    """The per-round exchange of rank `rank` (host side).  A source's pieces for one
+    destination in one round cover a contiguous range of its experts (the round index
+    never decreases along a destination's experts), hence a contiguous slice of its
+    expert-ordered rows."""
+    off = np.asarray(offsets_all, np.int64)
+    W, N = off.shape[0], off.shape[1] - 1
+    El = N // world
+    kept = off[:, 1:] - off[:, :-1]
+    round_of, R = plan_rounds(kept, world, cap)
+    plans = []
+    for r in range(R):
+        kr = np.where(round_of == r, kept, 0)
+        off_r = np.concatenate([np.zeros((W, 1), np.int64), np.cumsum(kr, axis=1)], axis=1)
+        start, count = [], []
+        for d in range(world):
+            es = [e for e in range(d * El, (d + 1) * El) if round_of[rank, e] == r and kept[rank, e] > 0]
+            start.append(int(off[rank, es[0]]) if es else 0)
+            count.append(int(sum(kept[rank, e] for e in es)))
+        recv = [int(kr[s, rank * El:(rank + 1) * El].sum()) for s in range(W)]
+        plans.append(RoundPlan(off_r.astype(np.int32), start, count, recv))
+    return plans
+
+
+# ----------------------------------------------------------------------------- layer
 class EPMoELayer:
     """Rank `rank` of `world`: routes its own T tokens over all N experts and computes
-    the experts rank * N / W .. (rank + 1) * N / W - 1 for every rank's tokens."""
+    the experts rank * N / W .. (rank + 1) * N / W - 1 for every rank's tokens.
+
+    recv_factor: the receive buffer holds ceil(recv_factor * T * k) rows (at least T);
+    1.0 is what a rank receives on average.  Skewed routing costs more rounds, never
+    a failure."""
 
     def __init__(self, w: Workload, weights: dict, rank: int, world: int, device="cuda",
-                 exchange=None, update_bias: bool = True, recv_factor: Optional[float] = None):
+                 exchange=None, update_bias: bool = True, recv_factor: float = 1.0):
         if w.N % world != 0:
             raise ValueError(f"{w.N} experts do not divide over {world} ranks")
         if w.fp8 or w.mxfp8 or w.expert_choice or w.dtype != "bf16":
             raise ValueError("the expert-parallel layer runs bf16 token-choice routing")
+        if not recv_factor > 0:
+            raise ValueError("recv_factor must be positive")
         self.w, self.rank, self.world = w, rank, world
         self.El = w.N // world
         self.exchange = exchange
         dev = torch.device(device)
+        self.dev = dev
         lo, hi = rank * self.El, (rank + 1) * self.El
         # the single-rank layer supplies routing, permutation, shared experts, combine, stats;
         # it keeps only this rank's experts
@@ -74,20 +184,21 @@ class EPMoELayer:
         self.base = MoELayer(w, local, dev, update_bias=False)
         self.w1, self.w3, self.w2 = (weights[n][lo:hi].contiguous() for n in ("w1", "w3", "w2"))
         self.update_bias = update_bias and weights.get("bias") is not None
-        # received rows: at most every rank's T * k rows (dropless, all to this rank's experts)
-        cap = world * w.T * w.k if recv_factor is None else int(recv_factor * w.T * w.k)
-        self.recv_cap = max(cap, 1)
+        self.recv_cap = max(int(math.ceil(recv_factor * w.T * w.k)), w.T, 1)
         z = lambda *s, dtype=torch.bfloat16: torch.empty(s, dtype=dtype, device=dev)  # noqa: E731
-        self.recv_x = z(self.recv_cap, w.d)
-        self.x_loc = z(self.recv_cap, w.d)
-        self.h_loc = z(self.recv_cap, w.f)
-        self.y_loc = z(self.recv_cap, w.d)
-        self.recv_y = z(self.recv_cap, w.d)
+        # two buffer sets (rounds alternate): received rows (later the results in arrival
+        # order), rows regrouped by local expert (later their results), hidden rows;
+        # a single rank exchanges nothing and needs none
+        nset = 2 if world > 1 else 0
+        self.recv = [z(self.recv_cap, w.d) for _ in range(nset)]
+        self.loc = [z(self.recv_cap, w.d) for _ in range(nset)]
+        self.h_loc = [z(self.recv_cap, w.f) for _ in range(nset)]
+        self.regroup_map = [z(self.recv_cap, dtype=torch.int32) for _ in range(nset)]
+        self.local_offsets = [z(self.El + 1, dtype=torch.int32) for _ in range(nset)]
         self.send_splits = z(world, dtype=torch.int32)
         self.recv_splits = z(world, dtype=torch.int32)
-        self.local_offsets = z(self.El + 1, dtype=torch.int32)
-        self.regroup_map = z(self.recv_cap, dtype=torch.int32)
         self.counts_global = z(w.N, dtype=torch.int32)
+        self.plans: List[RoundPlan] = []
 
     # ---------------------------------------------------------------- phases
     def dispatch_prepare(self, x: torch.Tensor, stream=None) -> torch.Tensor:
@@ -100,27 +211,51 @@ class EPMoELayer:
                       b.n_dropped, b.ws, stream)
         return b.offsets
 
-    def plan(self, offsets_all: torch.Tensor, stream=None):
-        """Split sizes (host lists: send, receive) from every rank's offsets."""
-        L.moe_ep_plan(offsets_all, self.world, self.rank, self.send_splits, self.recv_splits,
-                      self.local_offsets, self.regroup_map, stream)
-        send, recv = self.send_splits.cpu().tolist(), self.recv_splits.cpu().tolist()
-        if sum(recv) > self.recv_cap:
-            raise RuntimeError(f"{sum(recv)} rows received, capacity {self.recv_cap}")
-        return send, recv
+    def plan(self, offsets_all: torch.Tensor, stream=None) -> int:
+        """Plan the rounds from every rank's offsets (copied to the host: the one
+        synchronisation) and upload every round's offsets at once.  Returns the
+        number of rounds."""
+        off = offsets_all.cpu().numpy()
+        self.plans = round_plans(off, self.rank, self.world, self.recv_cap)
+        stacked = np.stack([p.offsets_all for p in self.plans])
+        host = torch.from_numpy(stacked).pin_memory() if self.dev.type == "cuda" else torch.from_numpy(stacked)
+        self.round_offsets = host.to(self.dev, non_blocking=True)
+        return len(self.plans)
 
-    def send_rows(self) -> torch.Tensor:
-        return self.base.x_perm
+    def round_begin(self, r: int, stream=None):
+        """The device plan of round r (regroup map, local expert offsets) into buffer set r % 2."""
+        i = r % 2
+        L.moe_ep_plan(self.round_offsets[r], self.world, self.rank, self.send_splits, self.recv_splits,
+                      self.local_offsets[i], self.regroup_map[i], stream)
 
-    def local_compute(self, stream=None):
-        """Regroup the received rows by local expert, run the local experts' grouped
-        FFN, and put the results back in arrival order (self.recv_y)."""
-        w = self.w
-        n = self.local_offsets[self.El:]                      # device scalar: rows received
-        L.moe_rows_move(self.recv_x, self.regroup_map, n, self.x_loc, scatter=True, stream=stream)
-        L.moe_grouped_ffn(self.base.cfg, self.x_loc, self.recv_cap, self.local_offsets, self.El,
-                          self.w1, self.w3, self.w2, w.f, self.h_loc, self.y_loc, stream)
-        L.moe_rows_move(self.y_loc, self.regroup_map, n, self.recv_y, scatter=False, stream=stream)
+    def send_slices(self, r: int) -> List[torch.Tensor]:
+        p, x = self.plans[r], self.base.x_perm
+        return [x[s:s + n] for s, n in zip(p.send_start, p.send_count)]
+
+    def recv_slices(self, r: int) -> List[torch.Tensor]:
+        """Per source, where its rows of round r land (source-major arrival order)."""
+        p, buf = self.plans[r], self.recv[r % 2]
+        q = np.concatenate([[0], np.cumsum(p.recv_count)]).astype(np.int64)
+        return [buf[q[s]:q[s + 1]] for s in range(self.world)]
+
+    def local_compute(self, r: int, stream=None):
+        """Regroup round r's received rows by local expert, run the local experts'
+        grouped FFN, and put the results back in arrival order (in the receive buffer)."""
+        i, w = r % 2, self.w
+        n_rows = self.local_offsets[i][self.El:]             # device scalar: rows received
+        L.moe_rows_move(self.recv[i], self.regroup_map[i], n_rows, self.loc[i], scatter=True, stream=stream)
+        L.moe_grouped_ffn(self.base.cfg, self.loc[i], self.recv_cap, self.local_offsets[i], self.El,
+                          self.w1, self.w3, self.w2, w.f, self.h_loc[i], self.loc[i], stream)
+        L.moe_rows_move(self.loc[i], self.regroup_map[i], n_rows, self.recv[i], scatter=False, stream=stream)
+
+    def return_send_slices(self, r: int) -> List[torch.Tensor]:
+        """Per source, the results of its rows (arrival order), to send back."""
+        return self.recv_slices(r)
+
+    def return_recv_slices(self, r: int) -> List[torch.Tensor]:
+        """Per destination, where its results land in this rank's y_perm."""
+        p, y = self.plans[r], self.base.y_perm
+        return [y[s:s + n] for s, n in zip(p.send_start, p.send_count)]
 
     def stats_partial(self, stream=None) -> torch.Tensor:
         """This rank's sufficient statistics (fp64 [3N + 5]), to be summed over ranks."""
@@ -153,18 +288,72 @@ class EPMoELayer:
         return b.y
 
     # ---------------------------------------------------------------- one rank, real exchange
-    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, stream=None, marks=None) -> torch.Tensor:
+        """One layer forward with the real exchange.  `marks`, if given, is a list of 4
+        CUDA events recorded on the compute stream: start, after route + permute, after
+        the exchange and the local experts (all rounds), at the end."""
         ex = self.exchange
-        offsets_all = ex.all_gather(self.dispatch_prepare(x, stream))
-        send, recv = self.plan(offsets_all, stream)
-        ex.all_to_all(self.recv_x[:sum(recv)], self.base.x_perm[:sum(send)], recv, send)
-        self.local_compute(stream)
-        ex.all_to_all(self.base.y_perm[:sum(send)], self.recv_y[:sum(recv)], send, recv)
-        part = ex.all_reduce_sum(self.stats_partial(stream))
-        return self.finish(x, stream, part)
+        comp = stream if stream is not None else torch.cuda.current_stream(self.dev)
+        rec = (lambda i: marks[i].record(comp)) if marks is not None else (lambda i: None)
+        rec(0)
+        if self.world == 1:
+            # nothing to exchange: every row stays, already grouped by expert
+            b, w = self.base, self.w
+            self.dispatch_prepare(x, comp)
+            rec(1)
+            L.moe_grouped_ffn(b.cfg, b.x_perm, w.T * w.k, b.offsets, self.El, self.w1, self.w3, self.w2, w.f,
+                              b.h, b.y_perm, comp)
+            rec(2)
+            with torch.cuda.stream(comp):
+                part = ex.all_reduce_sum(self.stats_partial(comp))
+            y = self.finish(x, comp, part)
+            rec(3)
+            return y
+        self.dispatch_prepare(x, comp)
+        rec(1)
+        offsets_all = ex.all_gather(self.base.offsets)
+        R = self.plan(offsets_all, comp)
+        # collectives are issued from a side stream, so waiting for a transfer holds
+        # back only the transfers queued behind it, never the expert compute
+        if not hasattr(self, "_comm"):
+            self._comm = torch.cuda.Stream(self.dev)
+        comm = self._comm
 
-    def kernel_launches(self) -> int:
-        # route (+ split), permute (4), plan, two row moves, local FFN (2), combine, stats (2), bias
-        n = 1 + 1 + 4 + 1 + 2 + 2 + 1 + 2
+        def dispatch(r):
+            self.round_begin(r, comp)
+            comm.wait_stream(comp)            # the plan and this round's rows are ready
+            with torch.cuda.stream(comm):
+                return ex.all_to_all(self.recv_slices(r), self.send_slices(r), async_op=True)
+
+        back = []
+        nxt = dispatch(0)
+        for r in range(R):
+            with torch.cuda.stream(comp):
+                nxt.wait()                    # round r's rows have arrived
+            if r + 1 < R:
+                if r >= 1:
+                    with torch.cuda.stream(comm):
+                        back[r - 1].wait()    # buffer set (r + 1) % 2 is free once round r - 1 returned
+                nxt = dispatch(r + 1)
+            self.local_compute(r, comp)
+            comm.wait_stream(comp)            # round r's results are ready
+            with torch.cuda.stream(comm):
+                back.append(ex.all_to_all(self.return_recv_slices(r), self.return_send_slices(r), async_op=True))
+        with torch.cuda.stream(comp):
+            for h in back:                    # every round's results are home
+                h.wait()
+        rec(2)
+        with torch.cuda.stream(comp):
+            part = ex.all_reduce_sum(self.stats_partial(comp))
+        y = self.finish(x, comp, part)
+        rec(3)
+        return y
+
+    def kernel_launches(self, rounds: Optional[int] = None) -> int:
+        # route (+ split), permute (4), shared FFN (2), combine, stats (2), bias
+        n = 1 + 1 + 4 + 1 + 2 + (1 if self.update_bias else 0)
         n += 2 if self.base.fs > 0 else 0
-        return n + (1 if self.update_bias else 0)
+        if self.world == 1:
+            return n + 2                                      # local FFN (2)
+        R = len(self.plans) if rounds is None else rounds
+        return n + R * (1 + 2 + 2)                            # per round: plan, two row moves, FFN (2)

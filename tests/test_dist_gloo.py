@@ -85,10 +85,10 @@ def _ep_worker(rank, port, out_dir):
         send[:, 0] = rank
         send[:, 1] = torch.arange(R, dtype=torch.float32)
         recv = torch.full((sum(plan["recv"]), EP_D), -1.0)
-        ex.all_to_all(recv, send, plan["recv"], plan["send"])
+        ex.all_to_all(list(torch.split(recv, plan["recv"])), list(torch.split(send, plan["send"])))
         # the "expert" here: add 1000 to every received row, then send it back
         back = torch.empty_like(send)
-        ex.all_to_all(back, recv + 1000.0, plan["send"], plan["recv"])
+        ex.all_to_all(list(torch.split(back, plan["send"])), list(torch.split(recv + 1000.0, plan["recv"])))
         np.savez(os.path.join(out_dir, f"ep{rank}.npz"), offsets_all=offsets_all.numpy(), recv=recv.numpy(),
                  back=back.numpy(), send=send.numpy())
     finally:
@@ -171,3 +171,87 @@ def test_global_stats_vector_is_the_concatenated_batch(tmp_path):
                                                              np.zeros((ST_D, 2))))
     assert abs(aux_raw - out["stats"]["aux_raw"]) < 1e-12
     assert abs(v[3 * n] / T - out["stats"]["z"]) < 1e-12
+
+
+# ----------------------------------------------------------------------------- bounded EP exchange rounds
+def test_round_plan_invariants():
+    """Every (source, expert) piece goes to exactly one round, no destination receives
+    more than the capacity in a round, and both ends agree on every split size."""
+    from sparse_mixture_experts_21_b200.ep import plan_rounds, round_plans
+    rng = np.random.default_rng(77)
+    for W, N, cap in [(2, 8, 40), (4, 16, 60), (4, 16, 10 ** 6), (8, 64, 150)]:
+        kept = rng.integers(0, 30, size=(W, N))
+        kept[:, 3] = 0
+        kept[0, N - 1] = cap                              # one piece exactly at the capacity
+        off = np.concatenate([np.zeros((W, 1), np.int64), np.cumsum(kept, axis=1)], axis=1)
+        round_of, R = plan_rounds(kept, W, cap)
+        plans = [round_plans(off, r, W, cap) for r in range(W)]
+        El = N // W
+        for r in range(R):
+            for d in range(W):
+                assert sum(plans[d][r].recv_count) <= cap
+                for s in range(W):
+                    assert plans[s][r].send_count[d] == plans[d][r].recv_count[s]
+                    # the slice a source sends is its rows of exactly this round's pieces
+                    es = [e for e in range(d * El, (d + 1) * El) if round_of[s, e] == r]
+                    assert plans[s][r].send_count[d] == sum(kept[s, e] for e in es)
+        for s in range(W):                                # every row leaves once over the rounds
+            assert sum(sum(p.send_count) for p in plans[s]) == kept[s].sum()
+        if cap >= kept.sum():
+            assert R == 1
+
+
+EPR_N, EPR_WORLD, EPR_D, EPR_CAP = 8, 2, 4, 7
+
+
+def _ep_round_worker(rank, port, out_dir):
+    """The round protocol of EPMoELayer on CPU (gloo): per round the dispatch all-to-all
+    of the plan's slices, an "expert" (+1000, then regroup by local expert is not needed
+    for this check), and the return all-to-all into the source's slots."""
+    from sparse_mixture_experts_21_b200.ep import TorchDistExchange, round_plans
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=EPR_WORLD)
+    try:
+        ex = TorchDistExchange()
+        rng = np.random.default_rng(900 + rank)
+        kept = rng.integers(0, 6, size=EPR_N)
+        offsets = torch.tensor(np.concatenate([[0], np.cumsum(kept)]), dtype=torch.int32)
+        off_all = ex.all_gather(offsets).numpy()
+        plans = round_plans(off_all, rank, EPR_WORLD, EPR_CAP)
+        R = int(kept.sum())
+        x = torch.zeros(R, EPR_D)
+        x[:, 0] = rank
+        x[:, 1] = torch.arange(R, dtype=torch.float32)
+        y = torch.full((R, EPR_D), -1.0)
+        got = []
+        for p in plans:
+            recv = torch.full((sum(p.recv_count), EPR_D), -5.0)
+            q = np.concatenate([[0], np.cumsum(p.recv_count)])
+            ex.all_to_all([recv[q[s]:q[s + 1]] for s in range(EPR_WORLD)],
+                          [x[a:a + n] for a, n in zip(p.send_start, p.send_count)])
+            got.append(recv.clone())
+            out = recv + 1000.0
+            ex.all_to_all([y[a:a + n] for a, n in zip(p.send_start, p.send_count)],
+                          [out[q[s]:q[s + 1]] for s in range(EPR_WORLD)])
+        np.savez(os.path.join(out_dir, f"epr{rank}.npz"), x=x.numpy(), y=y.numpy(), n_rounds=len(plans),
+                 recv=np.concatenate(got) if got else np.zeros((0, EPR_D)), off_all=off_all)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ep_round_exchange_two_ranks(tmp_path):
+    """With a receive capacity of 7 rows the exchange takes several rounds; every row
+    reaches the rank that owns its expert exactly once and comes back, transformed
+    once, to its own slot."""
+    mp.start_processes(_ep_round_worker, args=(_free_port(), str(tmp_path)), nprocs=EPR_WORLD, join=True,
+                       start_method="spawn")
+    r = [np.load(tmp_path / f"epr{i}.npz") for i in range(EPR_WORLD)]
+    assert int(r[0]["n_rounds"]) == int(r[1]["n_rounds"]) > 1
+    off = r[0]["off_all"]
+    El = EPR_N // EPR_WORLD
+    for rank in range(EPR_WORLD):
+        assert np.array_equal(r[rank]["y"], r[rank]["x"] + 1000.0)
+        recv = r[rank]["recv"]
+        want = sorted((s, i) for s in range(EPR_WORLD) for i in range(off[s, rank * El], off[s, (rank + 1) * El]))
+        assert sorted(zip(recv[:, 0].astype(int).tolist(), recv[:, 1].astype(int).tolist())) == want

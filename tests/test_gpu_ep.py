@@ -77,33 +77,31 @@ def _case(T=300):
                    topk_groups=2, n_shared=1, f_shared=256)
 
 
-@pytest.mark.parametrize("W", [2, 4])
-def test_ep_lock_step_matches_single_rank(W):
+@pytest.mark.parametrize("W,recv_factor", [(2, 1.0), (4, 1.0), (4, 0.3)])
+def test_ep_lock_step_matches_single_rank(W, recv_factor):
     w = _case()
     shared = make_inputs(w, "cuda", seed=0)                 # router, bias, experts: the same on every rank
     xs = [make_inputs(w, "cuda", seed=10 + r, experts=False)["x"] for r in range(W)]
-    layers = [EPMoELayer(w, shared, r, W, "cuda", update_bias=False) for r in range(W)]
-    # phase 1: route and permute; the offsets all-gather
+    layers = [EPMoELayer(w, shared, r, W, "cuda", update_bias=False, recv_factor=recv_factor) for r in range(W)]
+    # phase 1: route and permute; the offsets all-gather; every rank's plan
     offsets_all = torch.stack([lay.dispatch_prepare(x).clone() for lay, x in zip(layers, xs)])
-    plans = [lay.plan(offsets_all) for lay in layers]
-    send = [p[0] for p in plans]
-    recv = [p[1] for p in plans]
-    # the dispatch all-to-all, by copies: rank d receives from s the rows s sends to d
-    for d in range(W):
-        q = 0
-        for s in range(W):
-            start = sum(send[s][:d])
-            n = send[s][d]
-            layers[d].recv_x[q:q + n] = layers[s].base.x_perm[start:start + n]
-            q += n
-    for lay in layers:
-        lay.local_compute()
-    # the return all-to-all
-    for s in range(W):
+    R = [lay.plan(offsets_all) for lay in layers]
+    assert len(set(R)) == 1                                 # every rank runs the same rounds
+    if recv_factor < 1.0:
+        assert R[0] > 1
+    for r in range(R[0]):
+        for lay in layers:
+            lay.round_begin(r)
+        # the dispatch all-to-all, by copies: rank d receives from s what s sends to d
         for d in range(W):
-            off_in_d = sum(recv[d][:s])                     # where s's rows sit among d's arrivals
-            start, n = sum(send[s][:d]), send[s][d]
-            layers[s].base.y_perm[start:start + n] = layers[d].recv_y[off_in_d:off_in_d + n]
+            for s_ in range(W):
+                layers[d].recv_slices(r)[s_].copy_(layers[s_].send_slices(r)[d])
+        for lay in layers:
+            lay.local_compute(r)
+        # the return all-to-all
+        for s_ in range(W):
+            for d in range(W):
+                layers[s_].return_recv_slices(r)[d].copy_(layers[d].return_send_slices(r)[s_])
     # the statistics all-reduce, by a sum
     psum = torch.stack([lay.stats_partial().clone() for lay in layers]).sum(0)
     ys = [lay.finish(x, partial_sum=psum) for lay, x in zip(layers, xs)]
@@ -167,3 +165,109 @@ def test_ep_one_rank_nccl():
         assert L.moe_device_status() == L.MOE_OK
     finally:
         dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- forward() with rounds, W threads
+class _Hub:
+    """Meeting point of W in-process ranks: a barrier and one slot per rank."""
+
+    def __init__(self, world):
+        import threading
+        self.world = world
+        self.barrier = threading.Barrier(world, timeout=120)
+        self.slot = [None] * world
+
+
+class _ThreadExchange:
+    """The exchange interface of EPMoELayer for W ranks run as threads on one GPU.
+    Data moves by device copies on the receiving rank's current stream, ordered after
+    the sender's data by CUDA events recorded before a host barrier; no kernel waits
+    for another rank's kernel."""
+
+    def __init__(self, hub, rank):
+        self.hub, self.rank, self.world = hub, rank, hub.world
+
+    def _post(self, item):
+        ev = torch.cuda.Event()
+        ev.record()
+        self.hub.barrier.wait()
+        self.hub.slot[self.rank] = (item, ev)
+        self.hub.barrier.wait()
+        got = list(self.hub.slot)
+        self.hub.barrier.wait()
+        for _, e in got:
+            torch.cuda.current_stream().wait_event(e)
+        return [g[0] for g in got]
+
+    def all_gather(self, t):
+        return torch.stack([x.clone() for x in self._post(t)])
+
+    def all_to_all(self, out_list, in_list, async_op=False):
+        ins = self._post(list(in_list))
+        for s in range(self.world):
+            out_list[s].copy_(ins[s][self.rank])
+        arrived = torch.cuda.Event()
+        arrived.record()
+        self._post(None)                               # senders may reuse their buffers after this
+
+        class _H:
+            def wait(self_inner):                      # the caller's stream waits for the data
+                torch.cuda.current_stream().wait_event(arrived)
+        if async_op:
+            return _H()
+        _H().wait()
+        return None
+
+    def all_reduce_sum(self, t):
+        parts = self._post(t)
+        total = torch.stack([p.clone() for p in parts]).sum(0)
+        self._post(None)
+        t.copy_(total)
+        return t
+
+
+@pytest.mark.parametrize("W,recv_factor", [(2, 0.4), (4, 1.0)])
+def test_ep_forward_threads_matches_single_rank(W, recv_factor):
+    """EPMoELayer.forward (rounds on two buffer sets, collectives from a side stream)
+    for W ranks run as threads on one GPU: each rank's output equals the single-rank
+    layer's on its tokens, and the bias update uses the counts of all ranks."""
+    import threading
+    w = _case()
+    shared = make_inputs(w, "cuda", seed=0)
+    xs = [make_inputs(w, "cuda", seed=30 + r, experts=False)["x"] for r in range(W)]
+    bias0 = shared["bias"].clone()
+    hub = _Hub(W)
+    weights = [dict(shared, bias=bias0.clone()) for _ in range(W)]
+    layers = [EPMoELayer(w, weights[r], r, W, "cuda", exchange=_ThreadExchange(hub, r), update_bias=True,
+                         recv_factor=recv_factor) for r in range(W)]
+    ys, errs = [None] * W, []
+
+    def run(r):
+        try:
+            with torch.cuda.stream(torch.cuda.Stream()):
+                ys[r] = layers[r].forward(xs[r]).clone()
+                torch.cuda.current_stream().synchronize()
+        except Exception as e:          # reported below
+            errs.append(e)
+            hub.barrier.abort()
+
+    th = [threading.Thread(target=run, args=(r,)) for r in range(W)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errs, errs
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    if recv_factor < 1.0:
+        assert len(layers[0].plans) > 1
+    counts = torch.zeros(w.N, dtype=torch.int64, device="cuda")
+    for r in range(W):
+        single = MoELayer(w, dict(shared, x=xs[r], bias=bias0.clone()), "cuda", update_bias=False)
+        y_ref = single.forward(xs[r])
+        torch.cuda.synchronize()
+        assert torch.equal(ys[r][:w.T], y_ref[:w.T]), r
+        counts += single.counts.long()
+    ref_bias = O.bias_update(f64(bias0), counts.cpu().numpy(), rate=w.bias_rate)
+    for r in range(W):
+        assert np.max(np.abs(f64(weights[r]["bias"]) - ref_bias)) < 1e-7
