@@ -352,29 +352,35 @@ route_simt_kernel(const XT* __restrict__ x, const float* __restrict__ w_gate, in
 // ============================================================================
 // tensor-core (tcgen05) front end, bf16x3 split of the fp32 router weight
 // ============================================================================
+// One CTA per 128 tokens.  For every 64-wide slice kt of d, the x tile (16 KB) is
+// loaded once and multiplied by the three weight pieces (3 x 4 MMAs of K = 16),
+// so x crosses L2 -> shared memory once instead of once per piece.  x tiles and
+// weight tiles have rings of their own, each fed by its own producer warp, so an
+// x tile (a DRAM miss, the only operand not shared by every CTA) is requested
+// A_STAGES slices ahead, independently of the weight tiles (which every CTA reads,
+// and which therefore stay in L2).
+//
 // The tensor cores' fp32 accumulation truncates, so one long accumulation over
 // K = 3 d would bias the logits towards zero (about 1e-5 relative at d = 4096).
-// Each group of TC_ACC_GROUP 64-wide K blocks therefore starts a fresh TMEM
+// Each group of TC_ACC_KT slices (24 MMA steps) therefore starts a fresh TMEM
 // accumulator, and drain warps add the group's result into fp32 registers with
-// round-to-nearest: the truncation then spans the 16 MMA steps of one group only
-// (a bias of order 16 / (3 d / 16) of the single-accumulator one).  K blocks run in
-// the order (d-tile, piece), so each x tile is fetched from DRAM once and reused
-// from L2.
+// round-to-nearest: the truncation spans the 24 MMA steps of one group only.
 constexpr int TC_TM = 128;          // tokens per CTA (MMA M)
-constexpr int TC_BK = 64;           // K per stage: one 128-byte swizzle row of bf16
-constexpr int TC_STAGES = 4;
-constexpr int TC_ACC_GROUP = 4;     // K blocks per fresh accumulator
-constexpr int TC_THREADS = 384;     // warp 0 TMA, warp 1 MMA, warps 4..11 drain; all 12 select
+constexpr int TC_BK = 64;           // K per slice: one 128-byte swizzle row of bf16
+constexpr int TC_A_STAGES = 4;      // x tiles in flight
+constexpr int TC_B_RING = 128 * 1024;   // bytes of weight-tile ring
+constexpr int TC_ACC_KT = 2;        // slices per fresh accumulator
+constexpr int TC_THREADS = 384;     // warp 0 x loads, 1 MMA, 2 weight loads, 4..11 drain; all 12 select
 constexpr int TC_WARPS = TC_THREADS / 32;
 
 template <int NP>
 struct TcRouteShape {
   static constexpr int A_BYTES = TC_TM * TC_BK * 2;
   static constexpr int B_BYTES = NP * TC_BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int B_STAGES = TC_B_RING / B_BYTES > 8 ? 8 : TC_B_RING / B_BYTES;
+  static constexpr int RING_BYTES = TC_A_STAGES * A_BYTES + B_STAGES * B_BYTES;
   static constexpr int LD = NP + 1;                           // logits row stride (floats)
   static constexpr int LOGIT_BYTES = TC_TM * LD * 4;
-  static constexpr int RING_BYTES = TC_STAGES * STAGE_BYTES;
   static constexpr int MAIN_BYTES = RING_BYTES > LOGIT_BYTES ? RING_BYTES : LOGIT_BYTES;
   static constexpr int NV = NP >= 32 ? NP / 32 : 1;
   static constexpr int PWARP_BYTES = TC_WARPS * NV * 32 * 4;
@@ -383,7 +389,7 @@ struct TcRouteShape {
   static constexpr int TMEM_COLS = NBUF * ACC_COLS;
   static constexpr int DRAIN_WARPS = NP >= 32 ? 8 : 4;
   static constexpr int CPW = NP >= 32 ? NP / 2 : NP;          // columns per drain warp
-  static constexpr size_t SMEM = 1024 + MAIN_BYTES + PWARP_BYTES + 256;
+  static constexpr size_t SMEM = 1024 + MAIN_BYTES + PWARP_BYTES + 512;
 };
 
 // Wsplit[e, p * dpad + c] = piece p of W_g[e, c] (zero past N rows / d columns).
@@ -406,31 +412,49 @@ split_gate_kernel(const float* __restrict__ w_gate, int N, int d, int NP, int dp
   }
 }
 
+// After an abort, wait (bounded) for the copies this producer issued into the last
+// min(issued, STAGES) stages, so none is still writing shared memory at exit.
+__device__ __forceinline__ void drain_own_copies(uint64_t* full, int STAGES, uint32_t stage, uint32_t phase,
+                                                 int issued) {
+  for (int i = 1; i <= min(issued, STAGES); ++i) {
+    const int st = ((int)stage - i + 2 * STAGES) % STAGES;
+    mbar_wait(&full[st], ((int)stage - i < 0) ? (phase ^ 1u) : phase);
+  }
+}
+
 template <int NP>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                 int d, int dpad, RouteArgs a) {
   using S = TcRouteShape<NP>;
+  constexpr int AS = TC_A_STAGES, BS = S::B_STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* a_ring = smem;                                     // [AS][A_BYTES]
+  uint8_t* b_ring = smem + AS * S::A_BYTES;                   // [BS][B_BYTES]
   float* logits = reinterpret_cast<float*>(smem);             // after the main loop
   float* pwarp = reinterpret_cast<float*>(smem + S::MAIN_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::MAIN_BYTES + S::PWARP_BYTES);
-  uint64_t* full = bars;                            // [TC_STAGES]
-  uint64_t* empty = bars + TC_STAGES;               // [TC_STAGES]
-  uint64_t* tfull = bars + 2 * TC_STAGES;           // [NBUF]
+  uint64_t* afull = bars;                           // [AS]
+  uint64_t* aempty = afull + AS;                    // [AS]
+  uint64_t* bfull = aempty + AS;                    // [BS]
+  uint64_t* bempty = bfull + BS;                    // [BS]
+  uint64_t* tfull = bempty + BS;                    // [NBUF]
   uint64_t* tempty = tfull + S::NBUF;               // [NBUF]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + S::NBUF);
+  uint64_t* mma_done = tempty + S::NBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t0 = (int64_t)blockIdx.x * TC_TM;
-  const int nkb = 3 * (dpad / TC_BK);
+  const int nkt = dpad / TC_BK;
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < AS; ++s) { mbar_init(&afull[s], 1); mbar_init(&aempty[s], 1); }
+    for (int s = 0; s < BS; ++s) { mbar_init(&bfull[s], 1); mbar_init(&bempty[s], 1); }
     for (int b = 0; b < S::NBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], S::DRAIN_WARPS); }
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tmX);
@@ -456,61 +480,87 @@ route_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__
   };
 
   if (warp == 0) {
+    // ---------------- x tiles: one per slice
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int issued = 0;
+      for (int kt = 0; kt < nkt; ++kt) {
+        if (!bounded_wait(&aempty[stage], phase ^ 1u)) {
+          drain_own_copies(afull, AS, stage, phase, issued);
+          break;
+        }
+        mbar_arrive_expect_tx(&afull[stage], S::A_BYTES);
+        tma_load_2d(&tmX, a_ring + (size_t)stage * S::A_BYTES, &afull[stage], kt * TC_BK, (int32_t)t0);
+        ++issued;
+        if (++stage == AS) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 2) {
+    // ---------------- weight tiles: three pieces per slice
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
-        if (!bounded_wait(&empty[stage], phase ^ 1u)) { ok = false; break; }
-        const int kt = kb / 3, piece = kb - 3 * kt;
-        uint8_t* sa = smem + (size_t)stage * S::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[stage], S::STAGE_BYTES);
-        tma_load_2d(&tmX, sa, &full[stage], kt * TC_BK, (int32_t)t0);
-        tma_load_2d(&tmW, sa + S::A_BYTES, &full[stage], piece * dpad + kt * TC_BK, 0);
-        ++issued;
-        if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) {
-        for (int i = 1; i <= min(issued, TC_STAGES); ++i) {
-          const int s = ((int)stage - i + 2 * TC_STAGES) % TC_STAGES;
-          mbar_wait(&full[s], ((int)stage - i < 0) ? (phase ^ 1u) : phase);
+      for (int kt = 0; kt < nkt && ok; ++kt) {
+        for (int p = 0; p < 3; ++p) {
+          if (!bounded_wait(&bempty[stage], phase ^ 1u)) {
+            drain_own_copies(bfull, BS, stage, phase, issued);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bfull[stage], S::B_BYTES);
+          tma_load_2d(&tmW, b_ring + (size_t)stage * S::B_BYTES, &bfull[stage], p * dpad + kt * TC_BK, 0);
+          ++issued;
+          if (++stage == BS) { stage = 0; phase ^= 1u; }
         }
       }
     }
   } else if (warp == 1) {
+    // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(TC_TM, NP < 16 ? 16 : NP);
-      uint32_t stage = 0, phase = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int grp = kb / TC_ACC_GROUP;
-        const bool first = kb % TC_ACC_GROUP == 0;
-        const bool last = kb % TC_ACC_GROUP == TC_ACC_GROUP - 1 || kb == nkb - 1;
+      uint32_t as = 0, aph = 0, bs = 0, bph = 0;
+      bool ok = true;
+      for (int kt = 0; kt < nkt && ok; ++kt) {
+        const int grp = kt / TC_ACC_KT;
+        const bool first = kt % TC_ACC_KT == 0;
+        const bool last = kt % TC_ACC_KT == TC_ACC_KT - 1 || kt == nkt - 1;
         const int buf = grp % S::NBUF;
         const uint32_t use = (uint32_t)(grp / S::NBUF) & 1u;
         if (first && !bounded_wait(&tempty[buf], use ^ 1u)) break;
-        if (!bounded_wait(&full[stage], phase)) break;
+        if (!bounded_wait(&afull[as], aph)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + (size_t)stage * S::STAGE_BYTES);
-        const uint32_t b_addr = a_addr + S::A_BYTES;
+        const uint32_t a_addr = smem_u32(a_ring + (size_t)as * S::A_BYTES);
         const uint32_t d_tmem = tmem_base + buf * S::ACC_COLS;
+        for (int p = 0; p < 3; ++p) {
+          if (!bounded_wait(&bfull[bs], bph)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t b_addr = smem_u32(b_ring + (size_t)bs * S::B_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < TC_BK / 16; ++kk)
-          umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
-                   idesc, (kk != 0 || !first) ? 1u : 0u);
-        umma_commit(&empty[stage]);
+          for (int kk = 0; kk < TC_BK / 16; ++kk)
+            umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), idesc,
+                     (first && p == 0 && kk == 0) ? 0u : 1u);
+          umma_commit(&bempty[bs]);
+          if (++bs == BS) { bs = 0; bph ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&aempty[as]);
+        if (++as == AS) { as = 0; aph ^= 1u; }
         if (last) umma_commit(&tfull[buf]);
-        if (++stage == TC_STAGES) { stage = 0; phase ^= 1u; }
       }
+      // every MMA of this CTA has finished once this barrier flips
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0);
     }
   } else if (warp >= 4 && warp < 4 + S::DRAIN_WARPS) {
-    // drain: TMEM lanes 32 (warp % 4) .. +31, columns [c0, c0 + CPW)
+    // ---------------- drain: TMEM lanes 32 (warp % 4) .. +31, columns [c0, c0 + CPW)
     const int q = warp & 3;
     const int c0 = ((warp - 4) / 4) * S::CPW;
     float acc[S::CPW];
 #pragma unroll
     for (int i = 0; i < S::CPW; ++i) acc[i] = 0.f;
     bool ok = true;
-    const int ngrp = (nkb + TC_ACC_GROUP - 1) / TC_ACC_GROUP;
+    const int ngrp = (nkt + TC_ACC_KT - 1) / TC_ACC_KT;
     for (int grp = 0; grp < ngrp && ok; ++grp) {
       const int buf = grp % S::NBUF;
       const uint32_t use = (uint32_t)(grp / S::NBUF) & 1u;

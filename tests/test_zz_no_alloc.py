@@ -17,6 +17,7 @@ from oracle import moe_oracle as O
 from sparse_mixture_experts_21_b200 import _lib as L
 from sparse_mixture_experts_21_b200.layer import make_config
 from sparse_mixture_experts_21_b200.synth import WORKLOADS, random_routing
+from tests.parity_util import oracle_cfg
 
 pytestmark = pytest.mark.gpu
 
@@ -48,11 +49,12 @@ def test_noalloc_matches_permute_twice(name, T, seed):
         for key in ref:
             assert torch.equal(ref[key], got[key]), f"call {call}: {key} differs"
         # and against the oracle's permutation of the same routing
-        p = O.permutation(idx.cpu().numpy().astype(np.int64), w.N, None)
+        p = O.permutation(idx.cpu().numpy().astype(np.int64), w.N, O.capacity(oracle_cfg(w), T))
         assert np.array_equal(got["counts"].cpu().numpy(), p["counts"])
         assert np.array_equal(got["offsets"].cpu().numpy(), p["offsets"])
         assert np.array_equal(got["ros"].cpu().numpy(), p["row_of_slot"])
         assert np.array_equal(got["tor"].cpu().numpy()[:p["R"]], p["token_of_row"])
+        assert got["nd"].cpu().tolist() == [p["dropped_slots"], p["dropped_tokens"]]
 
 
 def test_noalloc_without_gather():
