@@ -123,7 +123,10 @@ int moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
  * "负载均衡：从 aux loss 到 aux-loss-free" (selection on s_i + b_i, weights from s_i).
  *
  *   x            [T, d]   cfg->x_dtype (fp32 or bf16)
- *   w_gate       [N, d]   fp32 router weight (kept in fp32; never quantised)
+ *   w_gate       [N, d]   fp32 router weight (kept in fp32; never quantised), or NULL
+ *                on the tensor-core path (bf16 x, N <= 256) when `ws` holds the split
+ *                written by moe_route_prepare for this cfg and weight (`ws` must then
+ *                not be shared with moe_permute)
  *   logit_offset [N] fp32 or NULL: added to every token's logits
  *   bias         [N] fp32 or NULL: added to the affinity for selection only
  *   topk_idx     [T, k] int32 out: experts in descending selection score;
@@ -152,6 +155,23 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate,
               const float* logit_offset, const float* bias,
               int32_t* topk_idx, float* topk_w, float* lse, float* p_partial,
               float* margin, float* shared_w, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_route_prepare -- the router weight's exact three-way bf16 split, once per weight.
+ *
+ * The tensor-core router (bf16 x, N <= 256; see moe_route) multiplies x by the
+ * split W_g = W_hi + W_mid + W_lo (each piece the next 8 significant bits, so every
+ * product is exact).  moe_route computes the split on every call; a caller whose
+ * router weight changes less often than it routes writes it once here and then
+ * calls moe_route with w_gate = NULL and ws = this buffer.  No page defines this
+ * call: it is the reuse of a pure function of the weight.
+ *   w_gate    [N, d] fp32 (N + 1 rows with cfg->shared_sink)
+ *   prepared  device out, at least moe_route_prepare_size() bytes, 16-byte aligned
+ * Errors: MOE_ERR_UNSUPPORTED off the tensor-core path; MOE_ERR_WORKSPACE_TOO_SMALL.
+ * ------------------------------------------------------------------------- */
+int moe_route_prepare_size(const moe_config_t* cfg, size_t* bytes);
+int moe_route_prepare(const moe_config_t* cfg, const float* w_gate, void* prepared, size_t bytes,
+                      void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_permute -- counts, capacity drop in token order, offsets, row maps, gather.
@@ -553,6 +573,12 @@ int moe_selftest_wait_timeout(int64_t limit_cycles, int32_t* completed, void* st
 
 /* Static string for a status code. */
 const char* moe_status_string(int status);
+
+/* The CUDA runtime error (cudaError_t value, and its name) behind the last
+ * MOE_ERR_CUDA returned to the calling host thread; cudaSuccess / "cudaSuccess" if
+ * none.  Host only. */
+int moe_last_cuda_error(void);
+const char* moe_last_cuda_error_string(void);
 
 #ifdef __cplusplus
 }

@@ -30,7 +30,8 @@ EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_rou
             "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
             "moe_quantize_mxfp8", "moe_permute_mxfp8", "moe_grouped_ffn_mxfp8", "moe_ep_plan",
             "moe_rows_move", "moe_router_stats_partial", "moe_router_stats_finalize",
-            "moe_expert_choice_capacity")
+            "moe_expert_choice_capacity", "moe_route_prepare_size", "moe_route_prepare",
+            "moe_last_cuda_error", "moe_last_cuda_error_string")
 
 NEAR_TIE = 1e-4        # margin below which a token counts as a near-tie
 
@@ -93,6 +94,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_router_stats_partial": [cfgp, vp, vp, vp, vp, vp, vp, c_float, vp, vp],
         "moe_router_stats_finalize": [cfgp, vp, vp, c_float, c_float, vp, vp, vp, vp, vp],
         "moe_expert_choice_capacity": [cfgp, i32p],
+        "moe_route_prepare_size": [cfgp, POINTER(c_size_t)],
+        "moe_route_prepare": [cfgp, vp, vp, c_size_t, vp],
         "moe_bias_update": [cfgp, vp, vp, c_float, c_float, vp],
         "moe_bias_update_ema": [cfgp, vp, vp, c_float, vp, c_float, c_float, vp],
         "moe_bias_update_seq": [cfgp, vp, vp, c_int32, vp, c_float, c_float, vp, c_size_t, vp],
@@ -102,6 +105,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_device_status": [i32p, c_int32],
         "moe_selftest_wait_timeout": [c_int64, vp, vp],
         "moe_status_string": [c_int],
+        "moe_last_cuda_error": [],
+        "moe_last_cuda_error_string": [],
         "moe_quantize_fp8": [vp, c_int64, c_int32, c_int32, vp, vp, vp],
         "moe_permute_fp8": [cfgp, vp, vp, vp, vp, vp, vp, vp],
         "moe_grouped_ffn_fp8": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, c_int32, vp, vp,
@@ -116,7 +121,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     for name, args in sig.items():
         fn = getattr(lib, name)
         fn.argtypes = args
-        fn.restype = c_char_p if name == "moe_status_string" else c_int
+        fn.restype = c_char_p if name in ("moe_status_string", "moe_last_cuda_error_string") else c_int
     if path is None:
         _lib = lib
     return lib
@@ -139,7 +144,10 @@ def _stream(stream=None) -> Optional[int]:
 
 def _check(name: str, status: int) -> None:
     if status != MOE_OK:
-        raise MoeError(name, status, load().moe_status_string(status).decode())
+        text = load().moe_status_string(status).decode()
+        if status == MOE_ERR_CUDA:
+            text += ": " + load().moe_last_cuda_error_string().decode()
+        raise MoeError(name, status, text)
 
 
 def capacity(cfg: MoeConfig) -> int:
@@ -167,6 +175,19 @@ def moe_route(cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_parti
     _check("moe_route", load().moe_route(
         ctypes.byref(cfg), _ptr(x), _ptr(w_gate), _ptr(logit_offset), _ptr(bias), _ptr(topk_idx),
         _ptr(topk_w), _ptr(lse), _ptr(p_partial), _ptr(margin), _ptr(shared_w), _ptr(ws), nbytes,
+        _stream(stream)))
+
+
+def route_prepare_size(cfg: MoeConfig) -> int:
+    out = c_size_t()
+    _check("moe_route_prepare_size", load().moe_route_prepare_size(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def moe_route_prepare(cfg, w_gate, prepared, stream=None):
+    """Write the router weight's exact bf16 split into `prepared` (a uint8 tensor)."""
+    _check("moe_route_prepare", load().moe_route_prepare(
+        ctypes.byref(cfg), _ptr(w_gate), _ptr(prepared), prepared.numel() * prepared.element_size(),
         _stream(stream)))
 
 

@@ -85,7 +85,14 @@ int route_nblk(const moe_config_t& c) {
   return (int)((c.T + tm - 1) / tm);
 }
 
-int from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+// The CUDA error behind the last MOE_ERR_CUDA returned to this host thread.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+int from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  g_last_cuda_error = e;
+  return MOE_ERR_CUDA;
+}
 
 // Self-test of the bounded wait: one thread waits on an mbarrier that nothing
 // ever arrives on (its own arrival count is 2 and it arrives once), gives up after
@@ -140,15 +147,34 @@ int moe_route(const moe_config_t* cfg, const void* x, const float* w_gate, const
   const int st = check_config(cfg);
   if (st != MOE_OK) return st;
   if (cfg->T == 0) return MOE_OK;
-  if (!x || !w_gate || !topk_idx || !topk_w || !lse || !p_partial) return MOE_ERR_INVALID_ARG;
+  if (!x || !topk_idx || !topk_w || !lse || !p_partial) return MOE_ERR_INVALID_ARG;
+  if (!w_gate && !route_uses_tc(*cfg)) return MOE_ERR_INVALID_ARG;   // no prepared form on this path
   if (cfg->shared_sink && !shared_w) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w_gate)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || (w_gate && !aligned16(w_gate))) return MOE_ERR_INVALID_ARG;
   const size_t need = route_workspace_bytes(*cfg);
   if (ws_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (need > 0 && (!ws || !aligned16(ws))) return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_route(*cfg, x, w_gate, logit_offset, bias, topk_idx, topk_w, lse, p_partial,
                                 margin, cfg->shared_sink ? shared_w : nullptr, ws,
                                 static_cast<cudaStream_t>(stream)));
+}
+
+int moe_route_prepare_size(const moe_config_t* cfg, size_t* bytes) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = route_workspace_bytes(*cfg);
+  return MOE_OK;
+}
+
+int moe_route_prepare(const moe_config_t* cfg, const float* w_gate, void* prepared, size_t bytes,
+                      void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!route_uses_tc(*cfg)) return MOE_ERR_UNSUPPORTED;
+  if (!w_gate || !prepared || !aligned16(w_gate) || !aligned16(prepared)) return MOE_ERR_INVALID_ARG;
+  if (bytes < route_workspace_bytes(*cfg)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return from_cuda(launch_route_prepare(*cfg, w_gate, prepared, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_permute(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,
@@ -473,6 +499,10 @@ int moe_device_status(int32_t* status, int32_t reset) {
   *status = v;
   return MOE_OK;
 }
+
+int moe_last_cuda_error(void) { return (int)g_last_cuda_error; }
+
+const char* moe_last_cuda_error_string(void) { return cudaGetErrorName(g_last_cuda_error); }
 
 const char* moe_status_string(int status) {
   switch (status) {

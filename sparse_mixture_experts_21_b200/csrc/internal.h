@@ -21,6 +21,9 @@ bool route_uses_tc(const moe_config_t& c);
 int route_tokens_per_block(const moe_config_t& c);
 size_t route_workspace_bytes(const moe_config_t& c);
 
+// Exact three-way bf16 split of the router weight into ws (tensor-core router only).
+cudaError_t launch_route_prepare(const moe_config_t& c, const float* w_gate, void* ws, cudaStream_t s);
+// w_gate == NULL: ws already holds the split (tensor-core router only).
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* w_gate,
                          const float* logit_offset, const float* bias, int32_t* topk_idx,
                          float* topk_w, float* lse, float* p_partial, float* margin,

@@ -45,27 +45,43 @@ struct RouteArgs {
 
 // Selection phase: tokens t0 .. t0+TM-1 of the block, logits[tm * ld + e] in
 // shared memory.  Writes the per-token outputs and this block's row of p_partial.
+//
+// One warp per token; lane l holds experts l, l+32, ... (register column i holds
+// expert l + 32 i).  Per token: affinity and logsumexp; the group limit (when every
+// group is one register column, each lane finds the top groups itself from the
+// butterfly-merged column maxima); then each lane sorts its eligible experts by
+// selection score once (stable, so the lower expert index stays first on ties), and
+// each of the k picks is one warp arg-max over the lanes' list heads, after which
+// the winning lane drops its head.  The margin is one more such round.
 template <int NV, int WARPS>
 __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, const RouteArgs& a,
                              float* pwarp) {
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int N = a.N, k = a.k;
   float pacc[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) pacc[i] = 0.f;
+  // per-lane constants: validity, group of each column, bias and logit offset
+  float bias_r[NV], off_r[NV];
+  int gid[NV];
+  uint32_t valid_m = 0;
   const int gsz = a.n_groups > 1 ? N / a.n_groups : N;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int e = lane + 32 * i;
+    pacc[i] = 0.f;
+    if (e < N) valid_m |= 1u << i;
+    gid[i] = e < N ? e / gsz : 0;
+    bias_r[i] = (e < N && a.bias) ? a.bias[e] : 0.f;
+    off_r[i] = (e < N && a.logit_offset) ? a.logit_offset[e] : 0.f;
+  }
+  const bool col_groups = a.n_groups > 1 && gsz == 32 && a.group_topn <= 2;
 
   for (int tm = warp; tm < TM; tm += WARPS) {
     const int64_t t = t0 + tm;
     if (t >= a.T) break;
     float z[NV], s[NV], q[NV];
-    bool valid[NV];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int e = lane + 32 * i;
-      valid[i] = e < N;
-      z[i] = valid[i] ? logits[tm * ld + e] + (a.logit_offset ? a.logit_offset[e] : 0.f) : -INFINITY;
-    }
+    for (int i = 0; i < NV; ++i)
+      z[i] = ((valid_m >> i) & 1u) ? logits[tm * ld + lane + 32 * i] + off_r[i] : -INFINITY;
     // affinity and logsumexp (with the sink, over the N routed logits and the shared one)
     const float z_sh = a.sink ? logits[tm * ld + N] : -INFINITY;
     float m = z_sh;
@@ -75,7 +91,7 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
     float ex[NV], se = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      ex[i] = valid[i] ? expf(z[i] - m) : 0.f;
+      ex[i] = ((valid_m >> i) & 1u) ? expf(z[i] - m) : 0.f;
       se += ex[i];
     }
     se = warp_sum(se);
@@ -87,10 +103,11 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
     float ssum = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      if (a.score_fn == MOE_SCORE_SOFTMAX) s[i] = valid[i] ? ex[i] / se : 0.f;
-      else s[i] = valid[i] ? 1.f / (1.f + expf(-z[i])) : 0.f;
+      const bool v = (valid_m >> i) & 1u;
+      if (a.score_fn == MOE_SCORE_SOFTMAX) s[i] = v ? ex[i] / se : 0.f;
+      else s[i] = v ? 1.f / (1.f + expf(-z[i])) : 0.f;
       ssum += s[i];
-      q[i] = valid[i] ? s[i] + (a.bias ? a.bias[lane + 32 * i] : 0.f) : -INFINITY;
+      q[i] = v ? s[i] + bias_r[i] : -INFINITY;
     }
     // load-balance statistics: routed affinities normalised over the routed experts
     // (softmax probs as they are, or s / sum s)
@@ -106,18 +123,21 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
     if (a.scores) {      // expert-choice routing: the affinity matrix, expert-major
 #pragma unroll
       for (int i = 0; i < NV; ++i)
-        if (valid[i]) a.scores[(int64_t)(lane + 32 * i) * a.T + t] = s[i];
+        if ((valid_m >> i) & 1u) a.scores[(int64_t)(lane + 32 * i) * a.T + t] = s[i];
       if (lane == 0) a.lse[t] = lse;
       continue;
     }
 
-    // group-limited pre-selection
+    // group-limited pre-selection: group_keep bit g = group g kept; gmargin = score of
+    // the last kept group minus the best dropped one (ties: lower group index first)
     uint32_t group_keep = 0xffffffffu;
     float gmargin = INFINITY;
     if (a.n_groups > 1) {
-      float my_gscore = -INFINITY;
-      if (gsz == 32 && a.group_topn <= 2) {
-        // each group is one register column: butterfly merge of (best, second) values
+      uint32_t kept_mask = 0;
+      if (col_groups) {
+        // each group is one register column: butterfly merge of (best, second) gives
+        // every lane every group's score, and each lane selects the groups itself
+        float gsc[NV];
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
           float b1 = q[i], b2 = -INFINITY;
@@ -129,83 +149,108 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
             b2 = fmaxf(lo, fmaxf(b2, ob2));
             b1 = hi;
           }
-          if (lane == i) my_gscore = a.group_topn == 1 ? b1 : b1 + b2;
+          gsc[i] = a.group_topn == 1 ? b1 : b1 + b2;
         }
-      } else
-      for (int g = 0; g < a.n_groups; ++g) {
-        uint32_t taken = 0;
-        float gs = 0.f;
-        for (int r = 0; r < a.group_topn; ++r) {
+        float last = 0.f;
+        for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
           float v = -INFINITY;
-          int bi = 0x7fffffff;
+          int gi = -1;
 #pragma unroll
-          for (int i = 0; i < NV; ++i) {
-            const int e = lane + 32 * i;
-            if (valid[i] && e / gsz == g && !((taken >> i) & 1u) && (q[i] > v || (q[i] == v && e < bi))) {
-              v = q[i]; bi = e;
-            }
+          for (int i = 0; i < NV; ++i)
+            if (i < a.n_groups && !((kept_mask >> i) & 1u) && (gi < 0 || gsc[i] > v)) { v = gsc[i]; gi = i; }
+          if (r < a.topk_groups) {
+            kept_mask |= 1u << gi;
+            last = v;
+          } else {
+            gmargin = last - v;
           }
-          warp_argmax(v, bi);
-          gs += v;
-          if (bi != 0x7fffffff && (bi & 31) == lane) taken |= 1u << (bi >> 5);
         }
-        if (lane == g) my_gscore = gs;
-      }
-      uint32_t kept_mask = 0;
-      float last = 0.f;
-      for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
-        const bool cand = lane < a.n_groups && !((kept_mask >> lane) & 1u);
-        float v = cand ? my_gscore : -INFINITY;
-        int gi = cand ? lane : 0x7fffffff;
-        warp_argmax(v, gi);
-        if (r < a.topk_groups) {
-          if (gi != 0x7fffffff) kept_mask |= 1u << gi;
-          last = v;
-        } else {
-          gmargin = last - v;
+      } else {
+        float my_gscore = -INFINITY;
+        for (int g = 0; g < a.n_groups; ++g) {
+          uint32_t taken = 0;
+          float gs = 0.f;
+          for (int r = 0; r < a.group_topn; ++r) {
+            float v = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+              const int e = lane + 32 * i;
+              if (((valid_m >> i) & 1u) && gid[i] == g && !((taken >> i) & 1u) && (q[i] > v || (q[i] == v && e < bi))) {
+                v = q[i]; bi = e;
+              }
+            }
+            warp_argmax(v, bi);
+            gs += v;
+            if (bi != 0x7fffffff && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+          }
+          if (lane == g) my_gscore = gs;
+        }
+        float last = 0.f;
+        for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
+          const bool cand = lane < a.n_groups && !((kept_mask >> lane) & 1u);
+          float v = cand ? my_gscore : -INFINITY;
+          int gi = cand ? lane : 0x7fffffff;
+          warp_argmax(v, gi);
+          if (r < a.topk_groups) {
+            if (gi != 0x7fffffff) kept_mask |= 1u << gi;
+            last = v;
+          } else {
+            gmargin = last - v;
+          }
         }
       }
       group_keep = kept_mask;
     }
 
-    // top-k over eligible experts, descending, ties to the lower index
-    uint32_t taken = 0;
-    int my_idx = 0;
-    float my_s = 0.f, kth_q = 0.f;
-    for (int j = 0; j < k; ++j) {
-      float v = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const int e = lane + 32 * i;
-        if (valid[i] && ((group_keep >> (e / gsz)) & 1u) && !((taken >> i) & 1u) &&
-            (q[i] > v || (q[i] == v && e < bi))) {
-          v = q[i]; bi = e;
-        }
-      }
-      warp_argmax(v, bi);
-      float mine = 0.f;
-#pragma unroll
-      for (int i = 0; i < NV; ++i)
-        if ((bi >> 5) == i) mine = s[i];
-      const float sv = __shfl_sync(0xffffffffu, mine, bi & 31);
-      if (bi != 0x7fffffff && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (lane == j) { my_idx = bi; my_s = sv; }
-      kth_q = v;
-    }
-    // margin to the best eligible expert left out
-    float nv = -INFINITY;
-    int ni = 0x7fffffff;
+    // this lane's eligible experts, sorted by selection score (stable: the lower
+    // column, hence the lower expert, first among equal scores)
+    float cv[NV];
+    int ci[NV];
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
-      const int e = lane + 32 * i;
-      if (valid[i] && ((group_keep >> (e / gsz)) & 1u) && !((taken >> i) & 1u) &&
-          (q[i] > nv || (q[i] == nv && e < ni))) {
-        nv = q[i]; ni = e;
+      const bool el = ((valid_m >> i) & 1u) && ((group_keep >> gid[i]) & 1u);
+      cv[i] = el ? q[i] : -INFINITY;
+      ci[i] = i;
+    }
+#pragma unroll
+    for (int x = 1; x < NV; ++x) {
+#pragma unroll
+      for (int y = x; y > 0; --y) {
+        const bool sw = cv[y] > cv[y - 1];
+        const float tv = cv[y];
+        const int ti = ci[y];
+        cv[y] = sw ? cv[y - 1] : cv[y];
+        ci[y] = sw ? ci[y - 1] : ci[y];
+        cv[y - 1] = sw ? tv : cv[y - 1];
+        ci[y - 1] = sw ? ti : ci[y - 1];
       }
     }
-    warp_argmax(nv, ni);
+    // k picks, descending, ties to the lower expert index; then the margin
+    int my_idx = 0;
+    float kth_q = 0.f, nv = -INFINITY;
+    for (int j = 0; j <= k; ++j) {
+      float v = cv[0];
+      int e = v == -INFINITY ? 0x7fffffff : lane + 32 * ci[0];
+      warp_argmax(v, e);
+      if (j == k) { nv = v; break; }
+      if (e != 0x7fffffff && (e & 31) == lane) {       // the winning lane drops its head
+#pragma unroll
+        for (int i = 0; i + 1 < NV; ++i) { cv[i] = cv[i + 1]; ci[i] = ci[i + 1]; }
+        cv[NV - 1] = -INFINITY;
+      }
+      if (lane == j) my_idx = e;
+      kth_q = v;
+    }
     const float emargin = (nv == -INFINITY) ? INFINITY : kth_q - nv;
+    // the affinity of each lane's pick (lanes j < k)
+    float my_s = 0.f;
+    const int src = lane < k ? (my_idx & 31) : 0;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const float v = __shfl_sync(0xffffffffu, s[i], src);
+      if (lane < k && (my_idx >> 5) == i) my_s = v;
+    }
 
     const float wsum = warp_sum(lane < k ? my_s : 0.f) + s_sh;
     if (lane < k) {
@@ -617,16 +662,26 @@ cudaError_t launch_simt(const moe_config_t& c, const void* x, const float* wg, c
 }
 
 template <int NP>
+cudaError_t launch_split(const moe_config_t& c, const float* wg, __nv_bfloat16* wsplit, cudaStream_t s) {
+  const int d = c.d_model;
+  const int dpad = (d + TC_BK - 1) / TC_BK * TC_BK;
+  const int64_t n = (int64_t)NP * dpad;
+  const int sgrid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  split_gate_kernel<<<sgrid, 256, 0, s>>>(wg, c.n_experts + (c.shared_sink ? 1 : 0), d, NP, dpad, wsplit);
+  return cudaGetLastError();
+}
+
+template <int NP>
 cudaError_t launch_tc(const moe_config_t& c, const void* x, const float* wg, const RouteArgs& a,
                       void* ws, cudaStream_t s) {
   using S = TcRouteShape<NP>;
   const int d = c.d_model;
   const int dpad = (d + TC_BK - 1) / TC_BK * TC_BK;
   __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(ws);
-  const int64_t n = (int64_t)NP * dpad;
-  const int sgrid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  split_gate_kernel<<<sgrid, 256, 0, s>>>(wg, c.n_experts + (c.shared_sink ? 1 : 0), d, NP, dpad,
-                                          wsplit);
+  if (wg) {                        // else ws holds the split written by moe_route_prepare
+    const cudaError_t e = launch_split<NP>(c, wg, wsplit, s);
+    if (e != cudaSuccess) return e;
+  }
   CUtensorMap mx, mw;
   if (!make_map_bf16(&mx, x, (uint64_t)c.T, (uint64_t)d, TC_TM) ||
       !make_map_bf16(&mw, wsplit, (uint64_t)NP, (uint64_t)3 * dpad, NP))
@@ -666,6 +721,18 @@ size_t route_workspace_bytes(const moe_config_t& c) {
   const int np = route_np(gate_rows(c)) < 16 ? 16 : route_np(gate_rows(c));
   const size_t dpad = (size_t)(c.d_model + rt::TC_BK - 1) / rt::TC_BK * rt::TC_BK;
   return (size_t)np * 3 * dpad * 2;
+}
+
+cudaError_t launch_route_prepare(const moe_config_t& c, const float* wg, void* ws, cudaStream_t s) {
+  __nv_bfloat16* wsplit = static_cast<__nv_bfloat16*>(ws);
+  switch (route_np(gate_rows(c))) {
+    case 8: case 16: return rt::launch_split<16>(c, wg, wsplit, s);
+    case 32:  return rt::launch_split<32>(c, wg, wsplit, s);
+    case 64:  return rt::launch_split<64>(c, wg, wsplit, s);
+    case 128: return rt::launch_split<128>(c, wg, wsplit, s);
+    case 256: return rt::launch_split<256>(c, wg, wsplit, s);
+    default:  return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_route(const moe_config_t& c, const void* x, const float* wg, const float* off,

@@ -204,9 +204,7 @@ class EPMoELayer:
     def dispatch_prepare(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         """Route and permute this rank's tokens; returns the offsets to all-gather."""
         b, c = self.base, self.base.cfg
-        W = b.weights
-        L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), b.topk_idx, b.topk_w, b.lse,
-                    b.p_partial, b.margin, b.ws, stream, shared_w=b.shared_w)
+        b.route(x, stream)
         L.moe_permute(c, x, b.topk_idx, b.counts, b.offsets, b.row_of_slot, b.token_of_row, b.x_perm,
                       b.n_dropped, b.ws, stream)
         return b.offsets
@@ -350,8 +348,8 @@ class EPMoELayer:
         return y
 
     def kernel_launches(self, rounds: Optional[int] = None) -> int:
-        # route (+ split), permute (4), shared FFN (2), combine, stats (2), bias
-        n = 1 + 1 + 4 + 1 + 2 + (1 if self.update_bias else 0)
+        # route, permute (4), combine, stats (2), bias; shared FFN (2)
+        n = 1 + 4 + 1 + 2 + (1 if self.update_bias else 0)
         n += 2 if self.base.fs > 0 else 0
         if self.world == 1:
             return n + 2                                      # local FFN (2)

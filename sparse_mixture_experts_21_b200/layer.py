@@ -67,6 +67,11 @@ class MoELayer:
         self.x_perm = z(max(T * k, 1), d, dtype=dt)
         self.n_dropped = z(2, dtype=torch.int32)
         self.ws = z(max(L.workspace_size(self.cfg), 16), dtype=torch.uint8)
+        # the tensor-core router's exact bf16 split of W_g, written once (prepare_router)
+        self.route_split = None
+        if L.route_prepare_size(self.cfg) > 0 and not w.expert_choice:
+            self.route_split = z(L.route_prepare_size(self.cfg), dtype=torch.uint8)
+            self.prepare_router()
         self.h = z(max(T * k, 1), w.f, dtype=dt)
         self.y_perm = z(max(T * k, 1), d, dtype=dt)
         self.fs = w.n_shared * w.f_shared
@@ -92,6 +97,22 @@ class MoELayer:
             self.h = z(max(N * C, 1), w.f, dtype=dt)
             self.y_perm = z(max(N * C, 1), d, dtype=dt)
             self.n_unpicked = z(1, dtype=torch.int32)
+
+    def prepare_router(self, stream=None):
+        """Split the router weight for the tensor-core router; call again after changing
+        weights["w_gate"] in place."""
+        if self.route_split is not None:
+            L.moe_route_prepare(self.cfg, self.weights["w_gate"], self.route_split, stream)
+
+    def route(self, x, stream=None):
+        """moe_route on x into this layer's routing buffers."""
+        W = self.weights
+        if self.route_split is not None:
+            wg, ws = None, self.route_split
+        else:
+            wg, ws = W["w_gate"], self.ws
+        L.moe_route(self.cfg, x, wg, W.get("logit_offset"), W.get("bias"), self.topk_idx, self.topk_w, self.lse,
+                    self.p_partial, self.margin, ws, stream, shared_w=self.shared_w)
 
     def _init_fp8(self, z):
         """FP8 experts: quantise the weights once (fine-grained: 128 x 128 blocks with
@@ -143,9 +164,7 @@ class MoELayer:
         if self.w.expert_choice:
             return self._forward_ec(x, s, rec, y)
         rec(0)
-        L.moe_route(c, x, W["w_gate"], W.get("logit_offset"), W.get("bias"), self.topk_idx,
-                    self.topk_w, self.lse, self.p_partial, self.margin, self.ws, s,
-                    shared_w=self.shared_w)
+        self.route(x, s)
         rec(1)
         fp8 = self.w.fp8 or self.w.mxfp8
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
@@ -293,9 +312,8 @@ class MoELayer:
         n = 1 + 4 + 2 + 1 + 1          # route, permute (4), routed FFN (2), combine, stats
         if self.group is not None:
             n += 1                     # statistics in two launches around the all-reduce
-        # FP8: the permutation's bf16 gather is replaced by the quantising scatter
-        if self.w.dtype == "bf16" and self.w.N <= 256:
-            n += 1                     # exact bf16 split of the router weight
+        # FP8: the permutation's bf16 gather is replaced by the quantising scatter;
+        # the router weight's split is written once, outside the forward
         if self.fs > 0:
             n += 2
         if self.update_bias:

@@ -131,6 +131,20 @@ def test_null_and_misaligned_pointers_rejected(lib):
         L.MOE_ERR_INVALID_ARG
 
 
+def test_route_prepare_checks(lib):
+    ok = 0x1000000
+    c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    assert L.route_prepare_size(c) == L.workspace_size(c) or L.route_prepare_size(c) <= L.workspace_size(c)
+    assert lib.moe_route_prepare(ctypes.byref(c), ok, ok, 16, None) == L.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert lib.moe_route_prepare(ctypes.byref(c), None, ok, 1 << 30, None) == L.MOE_ERR_INVALID_ARG
+    cf = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])          # fp32 router: no split
+    assert L.route_prepare_size(cf) == 0
+    assert lib.moe_route_prepare(ctypes.byref(cf), ok, ok, 1 << 30, None) == L.MOE_ERR_UNSUPPORTED
+    # a NULL router weight is only accepted where a prepared split exists
+    assert lib.moe_route(ctypes.byref(cf), ok, None, None, None, ok, ok, ok, ok, None, None, None, 0, None) == \
+        L.MOE_ERR_INVALID_ARG
+
+
 def test_workspace_too_small_rejected(lib):
     c = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
     ok = 0x1000000

@@ -507,3 +507,25 @@ def test_cuda_graph_replay_matches_eager():
     assert torch.equal(eager.y, graph.y)
     assert torch.equal(inp_a["bias"], inp_b["bias"])
     assert torch.equal(eager.stats, graph.stats)
+
+
+def test_route_with_prepared_split_equals_route_with_weight():
+    """moe_route on the split written once by moe_route_prepare (w_gate = NULL) gives
+    the same bytes as moe_route splitting w_gate itself."""
+    w = SMALL["v3_small"]
+    inp = make_inputs(w, "cuda")
+    c = make_config(w)
+    T, N, k = w.T, w.N, w.k
+    nblk = L.route_partials(c)
+    outs = []
+    for prepared in (False, True):
+        z = lambda *s, dtype=torch.float32: torch.full(s, -3, dtype=dtype, device="cuda")  # noqa: E731
+        o = [z(T, k, dtype=torch.int32), z(T, k), z(T), z(nblk, N), z(T)]
+        ws = torch.zeros(max(L.workspace_size(c), 16), dtype=torch.uint8, device="cuda")
+        if prepared:
+            L.moe_route_prepare(c, inp["w_gate"], ws)
+        L.moe_route(c, inp["x"], None if prepared else inp["w_gate"], None, inp["bias"], *o, ws)
+        outs.append(o)
+    torch.cuda.synchronize()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
