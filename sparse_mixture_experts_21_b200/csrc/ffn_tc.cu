@@ -6,35 +6,59 @@
 // in its "推理侧的路由稳定性" parameter count E x 3D^2).
 //
 // Two persistent launches over a tile list built on the device from `offsets`:
-//   pass 0 (gate/up): H[r, n0:n0+128] = silu(X W1[g]^T) * (X W3[g]^T); the B tile
-//          stacks 128 rows of W1 over 128 rows of W3, so one N = 256 MMA gives gate
-//          and up for 128 hidden units and SwiGLU runs in the epilogue from TMEM.
+//   pass 0 (gate/up): H[r, n0:n0+128] = silu(X W1[g]^T) * (X W3[g]^T); the weight
+//          tile stacks 128 rows of W1 over 128 rows of W3, so one N = 256 MMA gives
+//          gate and up for 128 hidden units and SwiGLU runs in the epilogue from TMEM.
 //   pass 1 (down):    Y[r, n0:n0+256] = H W2[g]^T.
-// Every MMA is tcgen05.mma.cta_group::1.kind::f16, M 128, N 256, K 16, bf16 in,
-// fp32 accumulate in TMEM; operands come by TMA (128-byte swizzle, no multicast).
+// Every MMA is tcgen05.mma.cta_group::1.kind::f16 (bf16 in, fp32 accumulate in
+// TMEM); operands come by TMA (128-byte swizzle, no multicast).
 //
-// Two tile shapes, one per pass:
-//  * PAIR (pass 0, long K = d): a CTA tile is 256 rows of one group as two M = 128
-//    sub-tiles sharing each B stage: per 64-wide K step it loads A0 16 KB + A1 16 KB
-//    + B 32 KB and issues 2 x 4 MMAs, 64 bytes of operand traffic per MMA cycle
-//    (96 with one 128-row tile), 3-stage ring.  A group's last tile with at most
-//    128 rows loads and computes sub-tile 0 only, so padding stays at 128 rows.
-//    TMEM holds both accumulators (2 x 256 columns); to hide the epilogue, the 8
-//    epilogue warps drain accumulator 0 first, and as soon as it is free the MMA
-//    warp computes sub-tile 0 of the next tile over the first resident K stages,
-//    then waits for accumulator 1 and catches up sub-tile 1 on the same stages.
-//  * SINGLE (pass 1, short K = f): 128-row tiles, 4-stage ring of 48 KB, two TMEM
-//    accumulators used alternately so one tile's epilogue (4 warps) overlaps the
-//    next tile's MMAs completely — with K = 2048 a tile is too short to absorb the
-//    paired shape's epilogue bubble.
+// Gate/up pass (long K = d): a CTA tile is up to two sub-tiles of one group sharing
+// each weight stage.  Per 64-wide K step a stage holds A0 16 KB + A1 16 KB + W 32 KB
+// (the weight tile), 64 bytes of operand traffic per MMA cycle for two full
+// sub-tiles (96 with one 128-row tile); 3-stage ring; TMEM holds two 256-column fp32
+// accumulators, one per sub-tile.  To hide the epilogue, the 8 epilogue warps drain
+// accumulator 0 first, and as soon as it is free the MMA warp computes sub-tile 0 of
+// the next tile over the first resident stages, then waits for accumulator 1 and
+// catches up sub-tile 1 on the same stages.
 //
-// Warp roles: 0 = TMA producer, 1 = TMEM allocator + MMA issuer, 2.. = epilogue
-// (TMEM lane quarter = warp % 4).  Tiles are ordered group, n-tile, m-tile, so
-// CTAs running together share weight tiles through L2.  Rows past a group's end
-// are computed from whatever follows and never stored.  Every mbarrier wait is
-// bounded; on timeout the kernel records MOE_ERR_DEVICE_TIMEOUT, drains its own
-// copies and MMAs, frees TMEM and returns.
+// No padding rows in the gate/up pass.  A group of R rows is cut into floor(R / 128)
+// full 128-row sub-tiles (paired two by two) and a ragged tail of r = R mod 128 rows.
+// The tail is computed transposed ("swapped"): the weight tile already in shared
+// memory is the MMA's A operand (M = 128 weight rows, i.e. output columns) and the r
+// tail rows are its B operand (N = r rounded up to 16), so the tail costs its own MMA
+// work, not that of a 128-row tile, and reuses the weight stages of the group's last
+// full sub-tile.  Kinds of tile:
+//   PAIR   two full sub-tiles;
+//   SINGLE one full sub-tile (an odd count of full sub-tiles), no tail;
+//   ST     one full sub-tile + the group's tail as sub-tile 1 (swapped);
+//   T      the tail alone (an even count of full sub-tiles, or R < 128).
+// The swapped sub-tile writes D^T into accumulator 1: weight rows 0..127 (W1, gate)
+// into columns [0, n) and rows 128..255 (W3, up) into columns [128, 128 + n), so gate
+// and up of one hidden unit share a TMEM lane.
+//
+// Tile order and scheduling (gate/up): group, n-tile, then that (group, n-tile)'s
+// PAIR tiles followed by its extra tile.  Tiles are claimed dynamically -- the
+// producer warp takes the next index from a per-launch global counter and hands it
+// to the MMA and epilogue warps through a small shared-memory queue -- so the tiles
+// in flight are always a contiguous window of the list and the CTAs that share a
+// weight tile run together, whatever the tiles' lengths (a static round-robin
+// assignment lets CTAs drift apart and stream weight tiles from DRAM again).  The
+// last CTA to finish resets the counter.
+//
+// Down pass (short K = f): 128-row tiles of one group (group, n-tile, m-tile order,
+// static: every tile has the same length), 4-stage ring of 48 KB, two TMEM
+// accumulators used alternately so one tile's epilogue (4 warps) overlaps the next
+// tile's MMAs completely.  Rows past a group's end are computed from whatever
+// follows and never stored.
+//
+// Warp roles: 0 = TMA producer (and tile claims), 1 = TMEM allocator + MMA issuer,
+// 2.. = epilogue (TMEM lane quarter = warp % 4).  Every mbarrier wait is bounded; on
+// timeout the kernel records MOE_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs,
+// frees TMEM and returns.
 #include <cuda.h>
+
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -43,44 +67,46 @@ namespace moe {
 
 namespace tc {
 
-constexpr int SUB = 128;                      // rows per MMA
+constexpr int SUB = 128;                      // rows per MMA (full sub-tile)
 constexpr int BK = 64;
 constexpr int A_BYTES = SUB * BK * 2;         // 16 KB per 128-row A tile
-constexpr int B_BYTES = 256 * BK * 2;         // 32 KB
+constexpr int W_BYTES = 256 * BK * 2;         // 32 KB weight tile
+constexpr int STAGES = 3;
+constexpr int STAGE_BYTES = 2 * A_BYTES + W_BYTES;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int TMEM_COLS = 512;                // two 256-column fp32 accumulators
+constexpr int TAIL_BOX = 16;                  // rows per TMA box of a tail (swapped) operand
 constexpr int kMaxGroups = 512;
 
-template <bool PAIR>
-struct Shape {
-  static constexpr int BM = PAIR ? 2 * SUB : SUB;
-  static constexpr int STAGES = PAIR ? 3 : 4;
-  static constexpr int STAGE_BYTES = (PAIR ? 2 : 1) * A_BYTES + B_BYTES;
-  static constexpr int EPI_WARPS = PAIR ? 8 : 4;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-};
+enum TileKind { K_PAIR = 0, K_SINGLE = 1, K_ST = 2, K_T = 3 };
 
-template <int STAGES>
+constexpr int TQ = 4;                         // tile indices in flight from the producer
+constexpr int kCtrSlots = 64;                 // per-launch tile counters (rotating)
+
 struct __align__(8) TcShared {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t tq_full[TQ];
+  uint64_t tq_empty[TQ];
   uint64_t mma_done;
   uint32_t tmem_base;
   volatile int32_t abort;
+  volatile int32_t tq[TQ];        // claimed tile indices (>= total: no more tiles)
   int32_t goff[kMaxGroups + 1];   // group row offsets
-  int32_t tpre[kMaxGroups + 1];   // prefix of full tiles (BM rows, or two sub-tiles) per group
-  int32_t spre[kMaxGroups + 1];   // paired shape: prefix of tail tiles of at most 128 rows
+  int32_t tpre[kMaxGroups + 1];   // prefix over groups of (PAIR tiles + extra tile) per n-tile
 };
 
-template <bool PAIR>
-constexpr size_t smem_bytes() {
-  return 1024 + (size_t)Shape<PAIR>::STAGES * Shape<PAIR>::STAGE_BYTES +
-         sizeof(TcShared<Shape<PAIR>::STAGES>);
-}
+// Per-launch tile counters: [slot][0] = next tile to claim, [slot][1] = CTAs done.
+// Each launch takes the next slot; its last CTA puts both back to 0.  Launches more
+// than kCtrSlots apart may share a slot (the earlier one has long finished).
+__device__ int32_t g_tile_ctr[kCtrSlots][2];
 
-template <class SH>
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, SH* sh) {
+constexpr size_t kSmem = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(TcShared);
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, TcShared* sh) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
@@ -95,16 +121,15 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, SH
 }
 
 struct Tile {
-  int g, row0, rows, n0;
-  bool two;        // (paired shape) sub-tile 1 has rows
+  int g, n0, kind;
+  int row0;          // first row of the full sub-tile(s)
+  int trow0, tr;     // tail: first row and row count (kinds ST, T)
+  int tn;            // tail rows rounded up to TAIL_BOX (the swapped MMA's N)
+  __device__ bool has0() const { return kind != K_T; }
+  __device__ bool has1() const { return kind != K_SINGLE; }
+  __device__ bool swap1() const { return kind >= K_ST; }
 };
 
-// Tile list.  Single shape: (group, n-tile, m-tile) over 128-row tiles.  Paired
-// shape, in two phases so that tiles running side by side take the same time
-// (CTAs that share a weight tile through L2 must stay in step, and a weight tile
-// stays in L2 only for microseconds): first every tile with two sub-tiles
-// (group, n-tile, m-tile), then every tail of at most 128 rows (group, n-tile).
-template <bool PAIR, class SH>
 __device__ __forceinline__ int find_group(const int32_t* pre, int G, int tiles_n, int L) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {  // largest g with pre[g] * tiles_n <= L
@@ -114,116 +139,119 @@ __device__ __forceinline__ int find_group(const int32_t* pre, int G, int tiles_n
   return lo;
 }
 
-template <bool PAIR, class SH>
-__device__ __forceinline__ Tile decode_tile(int L, const SH* sh, int G, int tiles_n, int BN) {
-  constexpr int BM = PAIR ? 2 * SUB : SUB;
+__device__ __forceinline__ Tile decode_tile(int L, const TcShared* sh, int G, int tiles_n, int BN) {
   Tile t;
-  const int na = sh->tpre[G] * tiles_n;
-  if (L < na) {
-    const int g = find_group<PAIR, SH>(sh->tpre, G, tiles_n, L);
-    const int local = L - sh->tpre[g] * tiles_n;
-    const int mt = sh->tpre[g + 1] - sh->tpre[g];
-    const int n_tile = local / mt, m_tile = local - n_tile * mt;
-    t.g = g;
-    t.row0 = sh->goff[g] + m_tile * BM;
-    t.rows = min(BM, sh->goff[g + 1] - t.row0);
-    t.n0 = n_tile * BN;
+  const int g = find_group(sh->tpre, G, tiles_n, L);
+  const int per = sh->tpre[g + 1] - sh->tpre[g];          // tiles of group g per n-tile
+  const int local = L - sh->tpre[g] * tiles_n;
+  const int n_tile = local / per, j = local - n_tile * per;
+  const int rows = sh->goff[g + 1] - sh->goff[g];
+  const int full = rows / SUB, r = rows - full * SUB;
+  t.g = g;
+  t.n0 = n_tile * BN;
+  if (j < full / 2) {
+    t.kind = K_PAIR;
+    t.row0 = sh->goff[g] + j * 2 * SUB;
+    t.trow0 = 0;
+    t.tr = 0;
+    t.tn = 0;
   } else {
-    const int Lb = L - na;
-    const int g = find_group<PAIR, SH>(sh->spre, G, tiles_n, Lb);
-    const int rows_g = sh->goff[g + 1] - sh->goff[g];
-    t.g = g;
-    t.rows = rows_g % BM;
-    t.row0 = sh->goff[g + 1] - t.rows;
-    t.n0 = (Lb - sh->spre[g] * tiles_n) * BN;
+    t.kind = (full & 1) ? (r > 0 ? K_ST : K_SINGLE) : K_T;
+    t.row0 = sh->goff[g] + (full & ~1) * SUB;
+    t.trow0 = sh->goff[g + 1] - r;
+    t.tr = r;
+    t.tn = (r + TAIL_BOX - 1) / TAIL_BOX * TAIL_BOX;
   }
-  t.two = t.rows > SUB;
   return t;
 }
 
-// Per-group tile prefixes, one warp.
-template <bool PAIR, class SH>
-__device__ void build_tile_table(SH* sh, const int32_t* offsets, int G, int lane) {
-  constexpr int BM = PAIR ? 2 * SUB : SUB;
-  int carry = 0, carry_s = 0;
+// Per-group tile prefixes (PAIR tiles + at most one extra tile, per n-tile), one warp.
+__device__ void build_tile_table(TcShared* sh, const int32_t* offsets, int G, int lane) {
+  int carry = 0;
   for (int base = 0; base < G; base += 32) {
     const int g = base + lane;
-    int mt = 0, st = 0;
+    int mt = 0;
     if (g < G) {
       const int o0 = offsets[g], o1 = offsets[g + 1];
       sh->goff[g] = o0;
       const int rows = o1 > o0 ? o1 - o0 : 0;
-      if (PAIR) {
-        const int rem = rows % BM;
-        mt = rows / BM + (rem > SUB ? 1 : 0);
-        st = (rem > 0 && rem <= SUB) ? 1 : 0;
-      } else {
-        mt = (rows + BM - 1) / BM;
-      }
+      const int full = rows / SUB;
+      mt = full / 2 + (((full & 1) || rows % SUB) ? 1 : 0);
     }
-    int incl = mt, incl_s = st;
+    int incl = mt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      const int u = __shfl_up_sync(0xffffffffu, incl_s, o);
-      if (lane >= o) { incl += v; incl_s += u; }
+      if (lane >= o) incl += v;
     }
-    if (g < G) { sh->tpre[g + 1] = carry + incl; sh->spre[g + 1] = carry_s + incl_s; }
+    if (g < G) sh->tpre[g + 1] = carry + incl;
     carry += __shfl_sync(0xffffffffu, incl, 31);
-    carry_s += __shfl_sync(0xffffffffu, incl_s, 31);
   }
   if (lane == 0) {
     sh->tpre[0] = 0;
-    sh->spre[0] = 0;
     sh->goff[G] = offsets[G];
   }
 }
 
+// Consumer side of the tile queue: the i-th claimed tile index (>= total: done).
+__device__ __forceinline__ bool next_tile(TcShared* sh, uint32_t i, int* L) {
+  const uint32_t slot = i % TQ, ph = (i / TQ) & 1u;
+  if (!wait_or_abort(&sh->tq_full[slot], ph, sh)) return false;
+  *L = sh->tq[slot];
+  return true;
+}
+
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
-// Epilogue of one accumulator: TMEM columns [c_begin, c_end) of this warp's 32
-// lanes -> bf16 rows of `out`.  MODE 0 pairs gate column c with up column 128 + c.
+// Swapped (tail) epilogue.  The epilogue loads the same TMEM columns for a normal
+// and for a swapped sub-tile (pass 0: columns [64 h, 64 h + 64) and 128 + those;
+// pass 1: [128 h, 128 h + 128)); only their meaning differs.  Normal: the lane is a
+// row and the columns are output columns.  Swapped: the lane is an output column
+// and the columns are tail rows -- pass 0: warp half h holds tail rows
+// [64 h, 64 h + 64) of hidden unit n0 + 32 q + lane (gate at v[i], up at v[64 + i]);
+// pass 1: warp half h holds every tail row of output column n0 + 128 h + 32 q + lane.
+// Columns past the tail hold stale values and are never stored.
 template <int MODE>
-__device__ __forceinline__ void drain(uint32_t tbase, int c_begin, int c_end, bool row_ok,
-                                      __nv_bfloat16* orow, int col0, int n_out) {
-#pragma unroll 1
-  for (int c = c_begin; c < c_end; c += 16) {
-    float o[16];
-    if (MODE == 0) {
-      uint32_t gv[16], uv[16];
-      tmem_ld16(tbase + c, gv);
-      tmem_ld16(tbase + 128 + c, uv);
-      tmem_ld_wait();
+__device__ __forceinline__ void store_swapped(const uint32_t* v, const Tile& t, int half, int q, int lane,
+                                              int n_out, int64_t rows_cap, __nv_bfloat16* out) {
+  const int col = t.n0 + (MODE == 0 ? 0 : 128 * half) + 32 * q + lane;
+  const int64_t lim64 = rows_cap - t.trow0;
+  const int lim = (int)(lim64 < t.tr ? lim64 : t.tr);        // tail rows to store
+  if (col >= n_out) return;
+  const int64_t ld = n_out;
+  __nv_bfloat16* p = out + (int64_t)t.trow0 * ld + col;
+  // one running pointer (a chain of adds), so the unrolled loop does not keep an
+  // address per row live
+  if (MODE == 0) {
+    const int n = lim - half * 64;
+    p += (int64_t)(half * 64) * ld;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) o[i] = silu_f(__uint_as_float(gv[i])) * __uint_as_float(uv[i]);
-    } else {
-      uint32_t v[16];
-      tmem_ld16(tbase + c, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) o[i] = __uint_as_float(v[i]);
+    for (int i = 0; i < 64; ++i) {
+      if (i < n) *p = __float2bfloat16_rn(silu_f(__uint_as_float(v[i])) * __uint_as_float(v[64 + i]));
+      asm volatile("" : "+l"(p));
+      p += ld;
     }
-    if (row_ok) {
-      const int col = col0 + c;
-      if (col + 8 <= n_out) stg16(orow + c, pack16(o, __nv_bfloat16()));
-      if (col + 16 <= n_out) stg16(orow + c + 8, pack16(o + 8, __nv_bfloat16()));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 128; ++i) {
+      if (i < lim) *p = __float2bfloat16_rn(__uint_as_float(v[i]));
+      asm volatile("" : "+l"(p));
+      p += ld;
     }
   }
 }
 
-template <int MODE, bool PAIR>
-__global__ void __launch_bounds__(Shape<PAIR>::THREADS, 1)
-ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-              const __grid_constant__ CUtensorMap tmB1, const int32_t* __restrict__ offsets,
-              int G, int K, int n_out, int64_t rows_cap, __nv_bfloat16* __restrict__ out) {
-  using S = Shape<PAIR>;
-  using SH = TcShared<S::STAGES>;
-  constexpr int STAGES = S::STAGES, STAGE_BYTES = S::STAGE_BYTES;
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1)
+ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAt,
+              const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+              const int32_t* __restrict__ offsets, int G, int K, int n_out, int64_t rows_cap,
+              __nv_bfloat16* __restrict__ out, int ctr_slot) {
   constexpr int BN = MODE == 0 ? 128 : 256;    // output columns per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  SH* sh = reinterpret_cast<SH*>(smem + (size_t)STAGES * STAGE_BYTES);
+  TcShared* sh = reinterpret_cast<TcShared*>(smem + (size_t)STAGES * STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_n = (n_out + BN - 1) / BN;
@@ -231,11 +259,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&sh->full[s], 1); mbar_init(&sh->empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&sh->tfull[a], 1); mbar_init(&sh->tempty[a], S::EPI_WARPS); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&sh->tfull[a], 1); mbar_init(&sh->tempty[a], EPI_WARPS); }
+    for (int q = 0; q < TQ; ++q) { mbar_init(&sh->tq_full[q], 1); mbar_init(&sh->tq_empty[q], 1 + EPI_WARPS); }
     mbar_init(&sh->mma_done, 1);
     sh->abort = 0;
     fence_barrier_init();
     prefetch_tmap(&tmA);
+    prefetch_tmap(&tmAt);
     prefetch_tmap(&tmB0);
     if (MODE == 0) prefetch_tmap(&tmB1);
   }
@@ -243,34 +273,46 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     tmem_alloc(&sh->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 2) build_tile_table<PAIR>(sh, offsets, G, lane);
+  if (warp == 2) build_tile_table(sh, offsets, G, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sh->tmem_base;
-  const int total = (sh->tpre[G] + (PAIR ? sh->spre[G] : 0)) * tiles_n;
+  const int total = sh->tpre[G] * tiles_n;
+  int32_t* ctr = g_tile_ctr[ctr_slot];
 
   if (warp == 0) {
-    // ---------------- TMA producer
+    // ---------------- tile claims + TMA producer
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-        const Tile t = decode_tile<PAIR>(L, sh, G, tiles_n, BN);
-        const bool two = PAIR && t.two;
+      for (uint32_t i = 0; ok; ++i) {
+        // claim the next tile and hand its index to the MMA and epilogue warps
+        const uint32_t qs = i % TQ, qph = (i / TQ) & 1u;
+        if (!wait_or_abort(&sh->tq_empty[qs], qph ^ 1u, sh)) { ok = false; break; }
+        const int L = atomicAdd(&ctr[0], 1);
+        sh->tq[qs] = L;
+        mbar_arrive(&sh->tq_full[qs]);
+        if (L >= total) break;
+        const Tile t = decode_tile(L, sh, G, tiles_n, BN);
         const int brow = t.g * n_out + t.n0;
-        const uint32_t bytes = two ? STAGE_BYTES : A_BYTES + B_BYTES;
+        const uint32_t bytes = (t.has0() ? A_BYTES : 0) + (t.kind == K_PAIR ? A_BYTES : 0) +
+                               (t.swap1() ? t.tn * BK * 2 : 0) + W_BYTES;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!wait_or_abort(&sh->empty[stage], phase ^ 1u, sh)) { ok = false; break; }
           uint8_t* a = smem + (size_t)stage * STAGE_BYTES;
-          uint8_t* b = a + (PAIR ? 2 : 1) * A_BYTES;
+          uint8_t* b = a + 2 * A_BYTES;
           mbar_arrive_expect_tx(&sh->full[stage], bytes);
-          tma_load_2d(&tmA, a, &sh->full[stage], kb * BK, t.row0);
-          if (two) tma_load_2d(&tmA, a + A_BYTES, &sh->full[stage], kb * BK, t.row0 + SUB);
+          if (t.has0()) tma_load_2d(&tmA, a, &sh->full[stage], kb * BK, t.row0);
+          if (t.kind == K_PAIR) tma_load_2d(&tmA, a + A_BYTES, &sh->full[stage], kb * BK, t.row0 + SUB);
+          if (t.swap1())
+            for (int j = 0; j < t.tn / TAIL_BOX; ++j)
+              tma_load_2d(&tmAt, a + A_BYTES + j * TAIL_BOX * BK * 2, &sh->full[stage], kb * BK,
+                          t.trow0 + j * TAIL_BOX);
           if (MODE == 0) {
             tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
-            tma_load_2d(&tmB1, b + B_BYTES / 2, &sh->full[stage], kb * BK, brow);
+            tma_load_2d(&tmB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
           } else {
             tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
           }
@@ -293,77 +335,78 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       constexpr uint32_t idesc = umma_idesc_bf16(SUB, 256);
       uint32_t stage = 0, phase = 0;
       bool ok = true;
-      // MMAs of one K stage into accumulator `acc` from A sub-tile `sub`
-      auto issue = [&](uint32_t st, int sub, uint32_t acc, bool first_kb) {
+      // normal sub-tile: D[128 rows, 256] (+)= A_sub . W^T into accumulator `sub`
+      auto issue = [&](uint32_t st, int sub, bool first_kb) {
         const uint32_t base = smem_u32(smem + (size_t)st * STAGE_BYTES);
         const uint32_t a_addr = base + sub * A_BYTES;
-        const uint32_t b_addr = base + (PAIR ? 2 : 1) * A_BYTES;
-        const uint32_t d_tmem = tmem_base + acc * 256u;
+        const uint32_t b_addr = base + 2 * A_BYTES;
+        const uint32_t d_tmem = tmem_base + sub * 256u;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
           umma_f16(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
                    idesc, (!first_kb || kk != 0) ? 1u : 0u);
       };
-      if constexpr (PAIR) {
-        uint32_t use0 = 0, use1 = 0;       // completed uses of each accumulator
-        for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-          const Tile t = decode_tile<PAIR>(L, sh, G, tiles_n, BN);
+      // swapped tail in sub-tile 1: D^T[128 weight rows, tn] (+)= W_half . Tail^T, the two
+      // 128-row halves of the weight tile into columns [0, tn) and [128, 128 + tn) of
+      // accumulator 1
+      auto issue_swapped = [&](uint32_t st, int tn, bool first_kb) {
+        const uint32_t base = smem_u32(smem + (size_t)st * STAGE_BYTES);
+        const uint32_t tail_addr = base + A_BYTES;
+        const uint32_t w_addr = base + 2 * A_BYTES;
+        const uint32_t idesc_t = umma_idesc_bf16(SUB, tn);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t d_tmem = tmem_base + 256u + h * 128u;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_f16(d_tmem, umma_desc_sw128(w_addr + h * (W_BYTES / 2) + kk * 32),
+                     umma_desc_sw128(tail_addr + kk * 32), idesc_t, (!first_kb || kk != 0) ? 1u : 0u);
+        }
+      };
+      uint32_t use0 = 0, use1 = 0;       // completed uses of each accumulator
+      for (uint32_t i = 0; ok; ++i) {
+        int L = 0;
+        if (!next_tile(sh, i, &L)) break;
+        mbar_arrive(&sh->tq_empty[i % TQ]);
+        if (L >= total) break;
+        const Tile t = decode_tile(L, sh, G, tiles_n, BN);
+        const bool h0 = t.has0(), h1 = t.has1(), sw = t.swap1();
+        if (h0) {
           if (!wait_or_abort(&sh->tempty[0], (use0 & 1u) ^ 1u, sh)) { ok = false; break; }
           tc_fence_after();
-          // sub-tile 0 over the first P stages while accumulator 1 may still drain
-          const int P = nkb < STAGES ? nkb : STAGES;
-          const uint32_t st0 = stage;
-          for (int j = 0; j < P; ++j) {
-            if (!wait_or_abort(&sh->full[stage], phase, sh)) { ok = false; break; }
-            tc_fence_after();
-            issue(stage, 0, 0, j == 0);
-            if (!t.two) umma_commit(&sh->empty[stage]);
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          }
-          if (!ok) break;
-          if (t.two) {
-            if (!wait_or_abort(&sh->tempty[1], (use1 & 1u) ^ 1u, sh)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t s2 = st0;
-            for (int j = 0; j < P; ++j) {
-              issue(s2, 1, 1, j == 0);
-              umma_commit(&sh->empty[s2]);
-              if (++s2 == STAGES) s2 = 0;
-            }
-          }
-          for (int kb = P; kb < nkb; ++kb) {
-            if (!wait_or_abort(&sh->full[stage], phase, sh)) { ok = false; break; }
-            tc_fence_after();
-            issue(stage, 0, 0, false);
-            if (t.two) issue(stage, 1, 1, false);
-            umma_commit(&sh->empty[stage]);
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          }
-          if (!ok) break;
-          umma_commit(&sh->tfull[0]);
-          ++use0;
-          if (t.two) {
-            umma_commit(&sh->tfull[1]);
-            ++use1;
-          }
         }
-      } else {
-        uint32_t acc = 0, acc_phase = 0;
-        for (int L = blockIdx.x; L < total && ok; L += gridDim.x) {
-          if (!wait_or_abort(&sh->tempty[acc], acc_phase ^ 1u, sh)) { ok = false; break; }
+        // sub-tile 0 over the first P stages while accumulator 1 may still drain
+        const int P = nkb < STAGES ? nkb : STAGES;
+        const uint32_t st0 = stage;
+        for (int j = 0; j < P; ++j) {
+          if (!wait_or_abort(&sh->full[stage], phase, sh)) { ok = false; break; }
           tc_fence_after();
-          for (int kb = 0; kb < nkb; ++kb) {
-            if (!wait_or_abort(&sh->full[stage], phase, sh)) { ok = false; break; }
-            tc_fence_after();
-            issue(stage, 0, acc, kb == 0);
-            umma_commit(&sh->empty[stage]);
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          }
-          if (!ok) break;
-          umma_commit(&sh->tfull[acc]);
-          acc ^= 1u;
-          if (acc == 0) acc_phase ^= 1u;
+          if (h0) issue(stage, 0, j == 0);
+          if (!h1) umma_commit(&sh->empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        if (!ok) break;
+        if (h1) {
+          if (!wait_or_abort(&sh->tempty[1], (use1 & 1u) ^ 1u, sh)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t s2 = st0;
+          for (int j = 0; j < P; ++j) {
+            if (sw) issue_swapped(s2, t.tn, j == 0); else issue(s2, 1, j == 0);
+            umma_commit(&sh->empty[s2]);
+            if (++s2 == STAGES) s2 = 0;
+          }
+        }
+        for (int kb = P; kb < nkb; ++kb) {
+          if (!wait_or_abort(&sh->full[stage], phase, sh)) { ok = false; break; }
+          tc_fence_after();
+          if (h0) issue(stage, 0, false);
+          if (h1) { if (sw) issue_swapped(stage, t.tn, false); else issue(stage, 1, false); }
+          umma_commit(&sh->empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        if (h0) { umma_commit(&sh->tfull[0]); ++use0; }
+        if (h1) { umma_commit(&sh->tfull[1]); ++use1; }
       }
       // every MMA of this CTA has finished once this barrier flips
       umma_commit(&sh->mma_done);
@@ -371,78 +414,72 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     }
   } else {
     // ---------------- epilogue: TMEM -> registers -> global
+    // Each warp copies its 32 lanes x 128 columns of an accumulator into registers
+    // behind one wait, releases the accumulator, and only then converts and stores,
+    // so the MMA warp waits for the TMEM copy, not for the global stores.
     const int q = warp & 3;                   // TMEM lane quarter of this warp
-    if constexpr (PAIR) {
-      // Each warp copies its 32 lanes x 128 columns of an accumulator into registers
-      // behind one wait, releases the accumulator, and only then converts and stores,
-      // so the MMA warp waits for the TMEM copy, not for the global stores.
-      const int half = (warp - 2) >> 2;       // column half handled by this warp
-      uint32_t use0 = 0, use1 = 0;
-      for (int L = blockIdx.x; L < total; L += gridDim.x) {
-        const Tile t = decode_tile<PAIR>(L, sh, G, tiles_n, BN);
-        bool ok = true;
-        for (int sub = 0; sub < (t.two ? 2 : 1); ++sub) {
-          uint32_t& use = sub == 0 ? use0 : use1;
-          if (!wait_or_abort(&sh->tfull[sub], use & 1u, sh)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + sub * 256u;
-          uint32_t v[128];
-          if (MODE == 0) {             // gate columns [64 h, 64 h + 64) and the matching up columns
+    const int half = (warp - 2) >> 2;         // column half (normal) / row or W half (swapped)
+    uint32_t use0 = 0, use1 = 0;
+    for (uint32_t i = 0;; ++i) {
+      // every lane waits (and acquires); the outcome is made warp-uniform
+      int L = 0;
+      const bool okq = __all_sync(0xffffffffu, next_tile(sh, i, &L));
+      if (!okq) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh->tq_empty[i % TQ]);
+      if (L >= total) break;
+      const Tile t = decode_tile(L, sh, G, tiles_n, BN);
+      bool ok = true;
+      for (int sub = 0; sub < 2; ++sub) {
+        if (sub == 0 ? !t.has0() : !t.has1()) continue;
+        uint32_t& use = sub == 0 ? use0 : use1;
+        if (!__all_sync(0xffffffffu, wait_or_abort(&sh->tfull[sub], use & 1u, sh))) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + sub * 256u;
+        uint32_t v[128];
+        const bool swapped = sub == 1 && t.swap1();
+        if (MODE == 0) {               // gate columns [64 h, 64 h + 64) and the matching up columns
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              tmem_ld16(tbase + half * 64 + 16 * j, v + 16 * j);
-              tmem_ld16(tbase + 128 + half * 64 + 16 * j, v + 64 + 16 * j);
-            }
-          } else {                     // output columns [128 h, 128 h + 128)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) tmem_ld16(tbase + half * 128 + 16 * j, v + 16 * j);
+          for (int j = 0; j < 4; ++j) {
+            tmem_ld16(tbase + half * 64 + 16 * j, v + 16 * j);
+            tmem_ld16(tbase + 128 + half * 64 + 16 * j, v + 64 + 16 * j);
           }
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh->tempty[sub]);
-          ++use;
-          const int r = sub * SUB + q * 32 + lane;
-          const int64_t grow = (int64_t)t.row0 + r;
-          if (r < t.rows && grow < rows_cap) {
-            __nv_bfloat16* orow = out + grow * (int64_t)n_out + t.n0;
-            constexpr int NC = MODE == 0 ? 64 : 128;     // output columns of this thread
-            const int c0 = half * NC;
+        } else {                       // output columns [128 h, 128 h + 128)
 #pragma unroll
-            for (int j = 0; j < NC; j += 8) {
-              float o[8];
+          for (int j = 0; j < 8; ++j) tmem_ld16(tbase + half * 128 + 16 * j, v + 16 * j);
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->tempty[sub]);
+        ++use;
+        if (swapped) {
+          store_swapped<MODE>(v, t, half, q, lane, n_out, rows_cap, out);
+          continue;
+        }
+        const int r = sub * SUB + q * 32 + lane;
+        const int64_t grow = (int64_t)t.row0 + r;
+        if (grow < rows_cap) {
+          __nv_bfloat16* orow = out + grow * (int64_t)n_out + t.n0;
+          constexpr int NC = MODE == 0 ? 64 : 128;     // output columns of this thread
+          const int c0 = half * NC;
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                o[i] = MODE == 0 ? silu_f(__uint_as_float(v[j + i])) * __uint_as_float(v[64 + j + i])
-                                 : __uint_as_float(v[j + i]);
-              if (t.n0 + c0 + j + 8 <= n_out) {
-                uint4 pk;
-                pk.x = pack_bf16x2(o[0], o[1]); pk.y = pack_bf16x2(o[2], o[3]);
-                pk.z = pack_bf16x2(o[4], o[5]); pk.w = pack_bf16x2(o[6], o[7]);
-                stg16(orow + c0 + j, pk);
-              }
+          for (int j = 0; j < NC; j += 8) {
+            float o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              o[i] = MODE == 0 ? silu_f(__uint_as_float(v[j + i])) * __uint_as_float(v[64 + j + i])
+                               : __uint_as_float(v[j + i]);
+            if (t.n0 + c0 + j + 8 <= n_out) {
+              uint4 pk;
+              pk.x = pack_bf16x2(o[0], o[1]); pk.y = pack_bf16x2(o[2], o[3]);
+              pk.z = pack_bf16x2(o[4], o[5]); pk.w = pack_bf16x2(o[6], o[7]);
+              stg16(orow + c0 + j, pk);
             }
           }
         }
-        if (!ok) break;
       }
-    } else {
-      constexpr int CW = MODE == 0 ? 128 : 256;
-      uint32_t acc = 0, acc_phase = 0;
-      for (int L = blockIdx.x; L < total; L += gridDim.x) {
-        const Tile t = decode_tile<PAIR>(L, sh, G, tiles_n, BN);
-        if (!wait_or_abort(&sh->tfull[acc], acc_phase, sh)) break;
-        tc_fence_after();
-        const int r = q * 32 + lane;
-        const int64_t grow = (int64_t)t.row0 + r;
-        drain<MODE>(tmem_base + ((uint32_t)(q * 32) << 16) + acc * 256u, 0, CW,
-                    r < t.rows && grow < rows_cap, out + grow * (int64_t)n_out + t.n0, t.n0, n_out);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->tempty[acc]);
-        acc ^= 1u;
-        if (acc == 0) acc_phase ^= 1u;
-      }
+      if (!ok) break;
     }
   }
 
@@ -452,22 +489,32 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
+  // the last CTA to finish puts the launch's tile counter back to 0 (every CTA has
+  // stopped claiming by now)
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&ctr[1], 1) == (int)gridDim.x - 1) {
+      atomicExch(&ctr[0], 0);
+      atomicExch(&ctr[1], 0);
+    }
+  }
 }
 
-template <int MODE, bool PAIR>
-cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const int32_t* offsets, int G, int K, int n_out, int64_t rows_cap,
-                        void* out, cudaStream_t s) {
+template <int MODE>
+cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
+                        const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
+                        int64_t rows_cap, void* out, cudaStream_t s) {
+  static std::atomic<unsigned> next_slot{0};
   constexpr int BN = MODE == 0 ? 128 : 256;
-  constexpr size_t SMEM = smem_bytes<PAIR>();
-  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<MODE, PAIR>, (int)SMEM);
+  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<MODE>, (int)kSmem);
   if (e != cudaSuccess) return e;
   const int64_t tiles_n = (n_out + BN - 1) / BN;
-  const int64_t max_tiles = ((rows_cap + Shape<PAIR>::BM - 1) / Shape<PAIR>::BM + G) * tiles_n;
+  const int64_t max_tiles = ((rows_cap + SUB - 1) / SUB + G) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
-  ffn_tc_kernel<MODE, PAIR><<<grid, Shape<PAIR>::THREADS, SMEM, s>>>(
-      a, b0, b1, offsets, G, K, n_out, rows_cap, static_cast<__nv_bfloat16*>(out));
+  const int slot = (int)(next_slot.fetch_add(1) % kCtrSlots);
+  ffn_tc_kernel<MODE><<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
+                                                   static_cast<__nv_bfloat16*>(out), slot);
   return cudaGetLastError();
 }
 
@@ -478,14 +525,15 @@ cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t*
                             void* y, cudaStream_t s) {
   if (rows_cap == 0 || G == 0) return cudaSuccess;
   if (G > tc::kMaxGroups) return cudaErrorInvalidValue;
-  CUtensorMap mx, m1, m3, mh, m2;
-  if (!make_map_bf16(&mx, x_rows, rows_cap, d, tc::SUB) || !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) ||
-      !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) || !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) ||
-      !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
+  CUtensorMap mx, mxt, m1, m3, mh, m2;
+  if (!make_map_bf16(&mx, x_rows, rows_cap, d, tc::SUB) ||
+      !make_map_bf16(&mxt, x_rows, rows_cap, d, tc::TAIL_BOX) ||
+      !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) || !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) ||
+      !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) || !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
     return cudaErrorInvalidValue;
-  cudaError_t e = tc::launch_pass<0, true>(mx, m1, m3, offsets, G, d, f, rows_cap, h, s);
+  cudaError_t e = tc::launch_pass<0>(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, s);
   if (e != cudaSuccess) return e;
-  return tc::launch_pass<1, false>(mh, m2, m2, offsets, G, f, d, rows_cap, y, s);
+  return launch_ffn_down(mh, m2, offsets, G, f, d, rows_cap, y, s);
 }
 
 }  // namespace moe

@@ -1,6 +1,9 @@
 // TMA tensor maps, encoded through the driver entry point (no libcuda link).
 #include <cuda.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "internal.h"
 
 namespace moe {
@@ -12,16 +15,29 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once per process (any host thread may
+// be the first to ask).  The device's primary context is made current in the asking
+// thread first, so the lookup does not depend on which thread initialised CUDA; a
+// failed lookup is retried by the next call.
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  static std::mutex mu;
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f) return f;
+  std::lock_guard<std::mutex> lock(mu);
+  f = fn.load(std::memory_order_relaxed);
+  if (f) return f;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaSetDevice(dev);
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess && p) {
+    f = reinterpret_cast<EncodeTiledFn>(p);
+    fn.store(f, std::memory_order_release);
   }
-  return fn;
+  cudaGetLastError();   // a failed lookup must not surface as a later launch's error
+  return f;
 }
 
 }  // namespace
