@@ -35,12 +35,12 @@ WORKLOAD = "deepseek_v3"
 METRIC = "MoE layer fwd tokens/s"
 UNIT = "tokens/s"
 
-# DRAM bytes (read + write) of one routed grouped-FFN call (both passes) from a
-# full-size ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass),
-# valid only while the kernel source is the one that was profiled (sha1).
+# DRAM bytes (read + write) of one routed grouped-FFN call (its kernels' launches of
+# one forward) from an ncu capture of those kernels alone with the one-pass metrics
+# dram__bytes_read.sum, dram__bytes_write.sum, gpu__time_duration.sum; valid only
+# while every listed kernel source is the one that was profiled (sha1), else null.
 NCU_TRAFFIC = {
-    "deepseek_v3": ("ffn_tc.cu", "6c3608e44a457edba78d671673af093dfd68799d", 32.3e9),
-    "deepseek_v3_mxfp8": ("ffn_mx.cu", "709e9d80185da2b81c3d48f20340d1eabb0fd4e9", 15.07e9),
+    "deepseek_v3_mxfp8": ({"ffn_mx.cu": "709e9d80185da2b81c3d48f20340d1eabb0fd4e9"}, 15.07e9),
 }
 
 
@@ -360,6 +360,9 @@ def main():
     ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
                     help="replicas: every rank holds every expert; ep: expert parallelism (N / W experts per "
                          "rank, all-to-all dispatch and return)")
+    ap.add_argument("--no-overlap-shared", action="store_true",
+                    help="run the shared experts on the main stream after the routed experts (default: on a "
+                         "side stream, concurrently with route and permute)")
     ap.add_argument("--recv-factor", type=float, default=1.0,
                     help="ep: receive buffer rows as a multiple of T * k (rounds bound it)")
     args = ap.parse_args()
@@ -393,7 +396,7 @@ def main():
     if args.parallel == "ep":
         return run_ep(args, w, world, rank, local, dev, pg)
     inp = make_inputs(w, dev, seed=rank)
-    lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD)
+    lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD, overlap_shared=not args.no_overlap_shared)
     x = inp["x"]
     stream = torch.cuda.current_stream(dev)
 
@@ -457,8 +460,8 @@ def main():
     tflops_ffn = flops_routed / (t_ffn * 1e-3) / 1e12
     traffic = None
     if w.name in NCU_TRAFFIC:
-        src, sha, nbytes = NCU_TRAFFIC[w.name]
-        if _sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc", src)) == sha:
+        srcs, nbytes = NCU_TRAFFIC[w.name]
+        if all(_sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc", f)) == h for f, h in srcs.items()):
             traffic = nbytes
 
     # the same step replayed from a CUDA graph (one capture, K replays): launch overhead out
@@ -534,7 +537,10 @@ def main():
                     "permute_gbs": bytes_perm / (t_perm * 1e-3) / 1e9,
                     "combine_gbs": bytes_comb / (t_comb * 1e-3) / 1e9,
                     "peak_gbs": peaks["hbm_gbs"]},
-            "shared_ffn_tflops": flops_shared / (t_shared * 1e-3) / 1e12,
+            # on a side stream the shared experts overlap route, permute and the routed
+            # experts; the main stream's "shared_ffn" stage is then only the join
+            "shared_ffn_tflops": None if lay.overlap_shared else flops_shared / (t_shared * 1e-3) / 1e12,
+            "shared_experts_stream": "side (overlapped)" if lay.overlap_shared else "main",
             "router_tflops_fp32": flops_router / (t_route * 1e-3) / 1e12,
             "router_stats": {"aux": st["aux"], "z_loss": st["z_loss"], "cv": st["cv"], "dead": st["dead"],
                              "dropped_slots": st["dropped_slots"], "dropped_tokens": st["dropped_tokens"]},

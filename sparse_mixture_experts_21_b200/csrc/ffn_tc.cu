@@ -5,11 +5,11 @@
 // expert itself is E(x) = W2 (silu(W1 x) * (W3 x)) (three matrices per expert, as
 // in its "推理侧的路由稳定性" parameter count E x 3D^2).
 //
-// Two persistent launches over a tile list built on the device from `offsets`:
-//   pass 0 (gate/up): H[r, n0:n0+128] = silu(X W1[g]^T) * (X W3[g]^T); the weight
+// Two persistent launches over tile lists built on the device from `offsets`:
+//   gate/up (this file): H[r, n0:n0+128] = silu(X W1[g]^T) * (X W3[g]^T); the weight
 //          tile stacks 128 rows of W1 over 128 rows of W3, so one N = 256 MMA gives
 //          gate and up for 128 hidden units and SwiGLU runs in the epilogue from TMEM.
-//   pass 1 (down):    Y[r, n0:n0+256] = H W2[g]^T.
+//   down (ffn_down.cu): Y[r, n0:n0+256] = H W2[g]^T.
 // Every MMA is tcgen05.mma.cta_group::1.kind::f16 (bf16 in, fp32 accumulate in
 // TMEM); operands come by TMA (128-byte swizzle, no multicast).
 //
@@ -204,17 +204,14 @@ __device__ __forceinline__ bool next_tile(TcShared* sh, uint32_t i, int* L) {
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
 // Swapped (tail) epilogue.  The epilogue loads the same TMEM columns for a normal
-// and for a swapped sub-tile (pass 0: columns [64 h, 64 h + 64) and 128 + those;
-// pass 1: [128 h, 128 h + 128)); only their meaning differs.  Normal: the lane is a
-// row and the columns are output columns.  Swapped: the lane is an output column
-// and the columns are tail rows -- pass 0: warp half h holds tail rows
-// [64 h, 64 h + 64) of hidden unit n0 + 32 q + lane (gate at v[i], up at v[64 + i]);
-// pass 1: warp half h holds every tail row of output column n0 + 128 h + 32 q + lane.
-// Columns past the tail hold stale values and are never stored.
-template <int MODE>
+// and for a swapped sub-tile (columns [64 h, 64 h + 64) and 128 + those); only their
+// meaning differs.  Normal: the lane is a row and the columns are hidden units.
+// Swapped: the lane is a hidden unit (n0 + 32 q + lane) and warp half h holds tail
+// rows [64 h, 64 h + 64) (gate at v[i], up at v[64 + i]).  Columns past the tail
+// hold stale values and are never stored.
 __device__ __forceinline__ void store_swapped(const uint32_t* v, const Tile& t, int half, int q, int lane,
                                               int n_out, int64_t rows_cap, __nv_bfloat16* out) {
-  const int col = t.n0 + (MODE == 0 ? 0 : 128 * half) + 32 * q + lane;
+  const int col = t.n0 + 32 * q + lane;
   const int64_t lim64 = rows_cap - t.trow0;
   const int lim = (int)(lim64 < t.tr ? lim64 : t.tr);        // tail rows to store
   if (col >= n_out) return;
@@ -222,32 +219,22 @@ __device__ __forceinline__ void store_swapped(const uint32_t* v, const Tile& t, 
   __nv_bfloat16* p = out + (int64_t)t.trow0 * ld + col;
   // one running pointer (a chain of adds), so the unrolled loop does not keep an
   // address per row live
-  if (MODE == 0) {
-    const int n = lim - half * 64;
-    p += (int64_t)(half * 64) * ld;
+  const int n = lim - half * 64;
+  p += (int64_t)(half * 64) * ld;
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      if (i < n) *p = __float2bfloat16_rn(silu_f(__uint_as_float(v[i])) * __uint_as_float(v[64 + i]));
-      asm volatile("" : "+l"(p));
-      p += ld;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 128; ++i) {
-      if (i < lim) *p = __float2bfloat16_rn(__uint_as_float(v[i]));
-      asm volatile("" : "+l"(p));
-      p += ld;
-    }
+  for (int i = 0; i < 64; ++i) {
+    if (i < n) *p = __float2bfloat16_rn(silu_f(__uint_as_float(v[i])) * __uint_as_float(v[64 + i]));
+    asm volatile("" : "+l"(p));
+    p += ld;
   }
 }
 
-template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAt,
               const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
               const int32_t* __restrict__ offsets, int G, int K, int n_out, int64_t rows_cap,
               __nv_bfloat16* __restrict__ out, int ctr_slot) {
-  constexpr int BN = MODE == 0 ? 128 : 256;    // output columns per tile
+  constexpr int BN = 128;                      // hidden units per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -267,7 +254,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmAt);
     prefetch_tmap(&tmB0);
-    if (MODE == 0) prefetch_tmap(&tmB1);
+    prefetch_tmap(&tmB1);
   }
   if (warp == 1) {
     tmem_alloc(&sh->tmem_base, TMEM_COLS);
@@ -310,12 +297,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             for (int j = 0; j < t.tn / TAIL_BOX; ++j)
               tma_load_2d(&tmAt, a + A_BYTES + j * TAIL_BOX * BK * 2, &sh->full[stage], kb * BK,
                           t.trow0 + j * TAIL_BOX);
-          if (MODE == 0) {
-            tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
-            tma_load_2d(&tmB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
-          } else {
-            tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
-          }
+          tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
+          tma_load_2d(&tmB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -438,15 +421,11 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + sub * 256u;
         uint32_t v[128];
         const bool swapped = sub == 1 && t.swap1();
-        if (MODE == 0) {               // gate columns [64 h, 64 h + 64) and the matching up columns
+        // gate columns [64 h, 64 h + 64) and the matching up columns
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_ld16(tbase + half * 64 + 16 * j, v + 16 * j);
-            tmem_ld16(tbase + 128 + half * 64 + 16 * j, v + 64 + 16 * j);
-          }
-        } else {                       // output columns [128 h, 128 h + 128)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) tmem_ld16(tbase + half * 128 + 16 * j, v + 16 * j);
+        for (int j = 0; j < 4; ++j) {
+          tmem_ld16(tbase + half * 64 + 16 * j, v + 16 * j);
+          tmem_ld16(tbase + 128 + half * 64 + 16 * j, v + 64 + 16 * j);
         }
         tmem_ld_wait();
         tc_fence_before();
@@ -454,22 +433,19 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         if (lane == 0) mbar_arrive(&sh->tempty[sub]);
         ++use;
         if (swapped) {
-          store_swapped<MODE>(v, t, half, q, lane, n_out, rows_cap, out);
+          store_swapped(v, t, half, q, lane, n_out, rows_cap, out);
           continue;
         }
         const int r = sub * SUB + q * 32 + lane;
         const int64_t grow = (int64_t)t.row0 + r;
         if (grow < rows_cap) {
           __nv_bfloat16* orow = out + grow * (int64_t)n_out + t.n0;
-          constexpr int NC = MODE == 0 ? 64 : 128;     // output columns of this thread
-          const int c0 = half * NC;
+          const int c0 = half * 64;                    // this thread's 64 hidden units
 #pragma unroll
-          for (int j = 0; j < NC; j += 8) {
+          for (int j = 0; j < 64; j += 8) {
             float o[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              o[i] = MODE == 0 ? silu_f(__uint_as_float(v[j + i])) * __uint_as_float(v[64 + j + i])
-                               : __uint_as_float(v[j + i]);
+            for (int i = 0; i < 8; ++i) o[i] = silu_f(__uint_as_float(v[j + i])) * __uint_as_float(v[64 + j + i]);
             if (t.n0 + c0 + j + 8 <= n_out) {
               uint4 pk;
               pk.x = pack_bf16x2(o[0], o[1]); pk.y = pack_bf16x2(o[2], o[3]);
@@ -500,21 +476,20 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
   }
 }
 
-template <int MODE>
-cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
-                        const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
-                        int64_t rows_cap, void* out, cudaStream_t s) {
+cudaError_t launch_gate_up(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
+                           const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
+                           int64_t rows_cap, void* out, cudaStream_t s) {
   static std::atomic<unsigned> next_slot{0};
-  constexpr int BN = MODE == 0 ? 128 : 256;
-  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<MODE>, (int)kSmem);
+  constexpr int BN = 128;
+  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel, (int)kSmem);
   if (e != cudaSuccess) return e;
   const int64_t tiles_n = (n_out + BN - 1) / BN;
   const int64_t max_tiles = ((rows_cap + SUB - 1) / SUB + G) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
   const int slot = (int)(next_slot.fetch_add(1) % kCtrSlots);
-  ffn_tc_kernel<MODE><<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
-                                                   static_cast<__nv_bfloat16*>(out), slot);
+  ffn_tc_kernel<<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
+                                             static_cast<__nv_bfloat16*>(out), slot);
   return cudaGetLastError();
 }
 
@@ -531,7 +506,7 @@ cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t*
       !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) || !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) ||
       !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) || !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
     return cudaErrorInvalidValue;
-  cudaError_t e = tc::launch_pass<0>(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, s);
+  cudaError_t e = tc::launch_gate_up(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, s);
   if (e != cudaSuccess) return e;
   return launch_ffn_down(mh, m2, offsets, G, f, d, rows_cap, y, s);
 }

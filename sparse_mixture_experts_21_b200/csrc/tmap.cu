@@ -16,9 +16,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 // The driver's tensor-map encoder, looked up once per process (any host thread may
-// be the first to ask).  The device's primary context is made current in the asking
-// thread first, so the lookup does not depend on which thread initialised CUDA; a
-// failed lookup is retried by the next call.
+// be the first to ask); a failed lookup is retried by the next call.
 EncodeTiledFn encode_fn() {
   static std::atomic<EncodeTiledFn> fn{nullptr};
   static std::mutex mu;
@@ -27,8 +25,6 @@ EncodeTiledFn encode_fn() {
   std::lock_guard<std::mutex> lock(mu);
   f = fn.load(std::memory_order_relaxed);
   if (f) return f;
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaSetDevice(dev);
   void* p = nullptr;
   cudaDriverEntryPointQueryResult q;
   if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
@@ -40,9 +36,20 @@ EncodeTiledFn encode_fn() {
   return f;
 }
 
+// cuTensorMapEncodeTiled is a driver call and needs a current context in the calling
+// thread; a host thread whose only CUDA use so far went through pooled streams may
+// have none.  Make the current device's primary context current, once per thread.
+void bind_context() {
+  thread_local bool bound = false;
+  if (bound) return;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess) bound = true;
+}
+
 }  // namespace
 
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  bind_context();
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows == 0 || cols == 0) return false;
   const cuuint64_t dims[2] = {cols, rows};
@@ -56,6 +63,7 @@ bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t col
 
 // Byte (E4M3 code) matrices: a box is 128 codes (128 B, one swizzle row) by box_rows.
 bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  bind_context();
   EncodeTiledFn fn = encode_fn();
   if (!fn || rows == 0 || cols == 0) return false;
   const cuuint64_t dims[2] = {cols, rows};

@@ -35,7 +35,7 @@ class MoELayer:
     """Holds the weights and the per-call buffers of one layer for up to T tokens."""
 
     def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True,
-                 group=None):
+                 group=None, overlap_shared: bool = True):
         """group: a torch.distributed process group when the layer runs as one of
         several data-parallel replicas; the router statistics are then those of the
         whole group's batch (each rank's sufficient statistics summed over the
@@ -47,6 +47,9 @@ class MoELayer:
             raise ValueError("FP8 experts need bf16 inputs and d, d_ff multiples of 128")
         self.w = w
         self.group = group
+        # bf16 shared experts on a side stream, concurrently with route and permute (they
+        # do not depend on the routing); joined before the combine
+        self.overlap_shared = overlap_shared and not (w.fp8 or w.mxfp8) and w.n_shared > 0
         self.dev = torch.device(device)
         self.weights = weights
         self.update_bias = update_bias and weights.get("bias") is not None
@@ -164,7 +167,21 @@ class MoELayer:
         if self.w.expert_choice:
             return self._forward_ec(x, s, rec, y)
         rec(0)
+        join = None
+        if self.overlap_shared:
+            fork = torch.cuda.Event()
+            fork.record(s)
         self.route(x, s)
+        if self.overlap_shared:
+            if not hasattr(self, "_side"):
+                self._side = torch.cuda.Stream(self.dev)
+            side = self._side
+            side.wait_event(fork)
+            with torch.cuda.stream(side):
+                L.moe_grouped_ffn(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], self.fs, self.hs,
+                                  self.ys, side)
+            join = torch.cuda.Event()
+            join.record(side)
         rec(1)
         fp8 = self.w.fp8 or self.w.mxfp8
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
@@ -185,7 +202,9 @@ class MoELayer:
         rec(3)
         shared = None
         if self.fs > 0:
-            if fp8:
+            if join is not None:
+                s.wait_event(join)
+            elif fp8:
                 self._ffn_fp8(c, self.xq, self.xs, T, self.shared_offsets, 1, ("ws1", "ws3", "ws2"),
                               self.fs, self.hq_sh, self.hsc_sh, self.ys, s)
             else:
