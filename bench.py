@@ -363,6 +363,9 @@ def main():
     ap.add_argument("--no-overlap-shared", action="store_true",
                     help="run the shared experts on the main stream after the routed experts (default: on a "
                          "side stream, concurrently with route and permute)")
+    ap.add_argument("--gather-rows", action="store_true",
+                    help="bf16: the grouped FFN gathers its rows from x (TMA gather4) instead of reading the "
+                         "expert-ordered copy that the permutation writes")
     ap.add_argument("--recv-factor", type=float, default=1.0,
                     help="ep: receive buffer rows as a multiple of T * k (rounds bound it)")
     args = ap.parse_args()
@@ -396,7 +399,8 @@ def main():
     if args.parallel == "ep":
         return run_ep(args, w, world, rank, local, dev, pg)
     inp = make_inputs(w, dev, seed=rank)
-    lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD, overlap_shared=not args.no_overlap_shared)
+    lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD, overlap_shared=not args.no_overlap_shared,
+                   gather_rows=args.gather_rows)
     x = inp["x"]
     stream = torch.cuda.current_stream(dev)
 
@@ -439,6 +443,8 @@ def main():
     flops_router = 2.0 * T * d * N
     bytes_route = T * d * eb + 4 * N * d + 8 * T * k
     bytes_perm = T * d * eb + R * d * eb + 12 * T * k
+    if lay.gather_rows:        # no row gather: index maps only (the grouped FFN reads x itself)
+        bytes_perm = 12 * T * k
     bytes_comb = R * d * eb + 2 * T * d * eb + 8 * T * k
     lowp = w.fp8 or w.mxfp8
     if lowp:                   # bf16 x read once; E4M3 codes + scales written per row (+ token order)
@@ -521,6 +527,8 @@ def main():
                        "groups": f"{w.n_groups} keep {w.topk_groups}" if w.n_groups > 1 else "none",
                        "routing": "expert-choice" if w.expert_choice else "token-choice top-k",
                        "capacity": w.capacity, "rows_R": R, "parallelism": f"replicas x{world}",
+                       "expert_rows": ("read from x by the first grouped GEMM (TMA gather4)" if lay.gather_rows
+                                       else "expert-ordered copy of x written by the permutation"),
                        "experts_precision": ("E4M3, 1x128 / 128x128 block scales" if w.fp8 else
                                              "MXFP8: E4M3, E8M0 scale per 32 along K" if w.mxfp8 else "bf16"),
                        "l2": (f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "

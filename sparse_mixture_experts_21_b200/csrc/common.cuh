@@ -175,6 +175,17 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, void* smem_d
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+// Four rows chosen by index (TMA tile::gather4): rows y0..y3 of a 2-D map whose box
+// is one row high, columns [x, x + box width), land as four consecutive box rows at
+// smem_dst (swizzled by their shared-memory address like a 4-row box load).
+__device__ __forceinline__ void tma_gather4(const CUtensorMap* map, void* smem_dst, uint64_t* bar, int32_t x,
+                                            int32_t y0, int32_t y1, int32_t y2, int32_t y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -52,6 +52,12 @@
 // tile's MMAs completely.  Rows past a group's end are computed from whatever
 // follows and never stored.
 //
+// Gathering form (ffn_tc_kernel<true>): the A rows come from x by token index
+// (TMA tile::gather4, four one-row boxes per copy, every lane of warp 0 issuing its
+// own four rows), so the expert-ordered copy of x is never written.  Same MMAs, same
+// shared-memory layout, bit-identical output; measured at about 76 cycles per
+// 512-byte gather4 copy per SM, it is slower than the row copy it saves.
+//
 // Warp roles: 0 = TMA producer (and tile claims), 1 = TMEM allocator + MMA issuer,
 // 2.. = epilogue (TMEM lane quarter = warp % 4).  Every mbarrier wait is bounded; on
 // timeout the kernel records MOE_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs,
@@ -229,11 +235,28 @@ __device__ __forceinline__ void store_swapped(const uint32_t* v, const Tile& t, 
   }
 }
 
+// Token of permuted row `row` for the gathering producer: an id outside [0, T) is
+// recorded as MOE_ERR_INVALID_ARG and replaced by token 0.
+__device__ __forceinline__ int32_t token_at(const int32_t* __restrict__ token_of_row, int64_t row, int T) {
+  const int32_t v = token_of_row[row];
+  if ((uint32_t)v >= (uint32_t)T) {
+    flag_invalid_index();
+    return 0;
+  }
+  return v;
+}
+
+// GATHER = false: A rows come from the expert-ordered rows X (map tmA, 128-row boxes;
+// tmAt, 16-row boxes for the tails).  GATHER = true: row r of group g is token
+// token_of_row[r] of x [T, K], fetched with tile::gather4 (tmA over x, one-row
+// boxes; tmAt unused), so the expert-ordered copy of x is never written.
+template <bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAt,
               const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
               const int32_t* __restrict__ offsets, int G, int K, int n_out, int64_t rows_cap,
-              __nv_bfloat16* __restrict__ out, int ctr_slot) {
+              __nv_bfloat16* __restrict__ out, int ctr_slot, const int32_t* __restrict__ token_of_row,
+              int T) {
   constexpr int BN = 128;                      // hidden units per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -268,7 +291,71 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
   const int total = sh->tpre[G] * tiles_n;
   int32_t* ctr = g_tile_ctr[ctr_slot];
 
-  if (warp == 0) {
+  if (warp == 0 && GATHER) {
+    // ---------------- tile claims + gathering TMA producer (whole warp)
+    // Lane l gathers rows 4l .. 4l+3 of each 128-row operand of the tile (the tail:
+    // of its first tn rows), 32 gather4 copies per full sub-tile and K step; the
+    // token ids are read once per tile.  Lane 0 claims tiles, waits for free stages,
+    // arms the stage barrier and loads the weight tile.
+    uint32_t stage = 0, phase = 0;
+    int issued = 0;
+    bool ok = true;
+    for (uint32_t i = 0; ok; ++i) {
+      const uint32_t qs = i % TQ, qph = (i / TQ) & 1u;
+      int L = -1;
+      if (lane == 0 && wait_or_abort(&sh->tq_empty[qs], qph ^ 1u, sh)) {
+        L = atomicAdd(&ctr[0], 1);
+        sh->tq[qs] = L;
+        mbar_arrive(&sh->tq_full[qs]);
+      }
+      L = __shfl_sync(0xffffffffu, L, 0);
+      if (L < 0) { ok = false; break; }
+      if (L >= total) break;
+      const Tile t = decode_tile(L, sh, G, tiles_n, BN);
+      const int brow = t.g * n_out + t.n0;
+      const uint32_t bytes = (t.has0() ? A_BYTES : 0) + (t.kind == K_PAIR ? A_BYTES : 0) +
+                             (t.swap1() ? t.tn * BK * 2 : 0) + W_BYTES;
+      // token ids of this lane's rows; a row at or past `lim` (past the group's tail,
+      // or past rows_cap) reads token 0 and feeds output that is never stored
+      auto ids = [&](int64_t first, int64_t lim, int32_t* r) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int64_t row = first + 4 * lane + j;
+          r[j] = row < lim ? token_at(token_of_row, row, T) : 0;
+        }
+      };
+      int32_t r0[4] = {0, 0, 0, 0}, r1[4] = {0, 0, 0, 0};
+      const bool g1 = t.kind == K_PAIR || (t.swap1() && 4 * lane < t.tn);
+      if (t.has0()) ids(t.row0, rows_cap, r0);
+      if (t.kind == K_PAIR) ids((int64_t)t.row0 + SUB, rows_cap, r1);
+      else if (g1) ids(t.trow0, min((int64_t)t.trow0 + t.tr, rows_cap), r1);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const bool w = lane == 0 ? wait_or_abort(&sh->empty[stage], phase ^ 1u, sh) : true;
+        if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        uint8_t* a = smem + (size_t)stage * STAGE_BYTES;
+        uint8_t* b = a + 2 * A_BYTES;
+        if (lane == 0) mbar_arrive_expect_tx(&sh->full[stage], bytes);
+        __syncwarp();
+        if (t.has0()) tma_gather4(&tmA, a + lane * 512, &sh->full[stage], kb * BK, r0[0], r0[1], r0[2], r0[3]);
+        if (g1)
+          tma_gather4(&tmA, a + A_BYTES + lane * 512, &sh->full[stage], kb * BK, r1[0], r1[1], r1[2], r1[3]);
+        if (lane == 0) {
+          tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
+          tma_load_2d(&tmB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
+        }
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok && lane == 0) {
+      // drain this CTA's own copies still in flight before leaving
+      for (int i = 1; i <= min(issued, STAGES); ++i) {
+        const int s = ((int)stage - i + 2 * STAGES) % STAGES;
+        const uint32_t ph = ((int)stage - i < 0) ? (phase ^ 1u) : phase;
+        mbar_wait(&sh->full[s], ph);
+      }
+    }
+  } else if (warp == 0) {
     // ---------------- tile claims + TMA producer
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
@@ -476,21 +563,32 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
   }
 }
 
-cudaError_t launch_gate_up(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
-                           const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
-                           int64_t rows_cap, void* out, cudaStream_t s) {
-  static std::atomic<unsigned> next_slot{0};
+// One counter for every launch of either form, so launches in flight on different
+// streams never share a tile-counter slot.
+static std::atomic<unsigned> g_next_slot{0};
+
+template <bool GATHER>
+static cudaError_t launch_gate_up_t(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
+                                    const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
+                                    int64_t rows_cap, void* out, const int32_t* token_of_row, int T,
+                                    cudaStream_t s) {
   constexpr int BN = 128;
-  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel, (int)kSmem);
+  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<GATHER>, (int)kSmem);
   if (e != cudaSuccess) return e;
   const int64_t tiles_n = (n_out + BN - 1) / BN;
   const int64_t max_tiles = ((rows_cap + SUB - 1) / SUB + G) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
-  const int slot = (int)(next_slot.fetch_add(1) % kCtrSlots);
-  ffn_tc_kernel<<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
-                                             static_cast<__nv_bfloat16*>(out), slot);
+  const int slot = (int)(g_next_slot.fetch_add(1) % kCtrSlots);
+  ffn_tc_kernel<GATHER><<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
+                                                     static_cast<__nv_bfloat16*>(out), slot, token_of_row, T);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gate_up(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
+                           const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
+                           int64_t rows_cap, void* out, cudaStream_t s) {
+  return launch_gate_up_t<false>(a, at, b0, b1, offsets, G, K, n_out, rows_cap, out, nullptr, 0, s);
 }
 
 }  // namespace tc
@@ -507,6 +605,21 @@ cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t*
       !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) || !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
     return cudaErrorInvalidValue;
   cudaError_t e = tc::launch_gate_up(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, s);
+  if (e != cudaSuccess) return e;
+  return launch_ffn_down(mh, m2, offsets, G, f, d, rows_cap, y, s);
+}
+
+cudaError_t launch_ffn_bf16_gather(const void* x, int T, const int32_t* token_of_row, int64_t rows_cap,
+                                   const int32_t* offsets, int G, const void* w1, const void* w3, const void* w2,
+                                   int d, int f, void* h, void* y, cudaStream_t s) {
+  if (rows_cap == 0 || G == 0 || T == 0) return cudaSuccess;
+  if (G > tc::kMaxGroups) return cudaErrorInvalidValue;
+  CUtensorMap mx, m1, m3, mh, m2;
+  if (!make_map_bf16(&mx, x, (uint64_t)T, d, 1) || !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) ||
+      !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) || !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) ||
+      !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
+    return cudaErrorInvalidValue;
+  cudaError_t e = tc::launch_gate_up_t<true>(mx, mx, m1, m3, offsets, G, d, f, rows_cap, h, token_of_row, T, s);
   if (e != cudaSuccess) return e;
   return launch_ffn_down(mh, m2, offsets, G, f, d, rows_cap, y, s);
 }

@@ -50,6 +50,10 @@ cudaError_t launch_permute(const moe_config_t& c, int64_t capacity, const void* 
 cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
                             const void* w1, const void* w3, const void* w2, int d, int f,
                             void* h, void* y, cudaStream_t s);
+// The same FFN with row r of group g read from x[token_of_row[r]] (x [T, d] bf16).
+cudaError_t launch_ffn_bf16_gather(const void* x, int T, const int32_t* token_of_row, int64_t rows_cap,
+                                   const int32_t* offsets, int G, const void* w1, const void* w3, const void* w2,
+                                   int d, int f, void* h, void* y, cudaStream_t s);
 // Down projection over row groups: H (map `mh`, 128-row boxes) times W2 (map `m2`,
 // 256-row boxes) -> Y [rows_cap, d] bf16.
 cudaError_t launch_ffn_down(const CUtensorMap& mh, const CUtensorMap& m2, const int32_t* offsets, int G, int f,

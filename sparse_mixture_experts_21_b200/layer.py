@@ -35,7 +35,7 @@ class MoELayer:
     """Holds the weights and the per-call buffers of one layer for up to T tokens."""
 
     def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True,
-                 group=None, overlap_shared: bool = True):
+                 group=None, overlap_shared: bool = True, gather_rows: bool = False):
         """group: a torch.distributed process group when the layer runs as one of
         several data-parallel replicas; the router statistics are then those of the
         whole group's batch (each rank's sufficient statistics summed over the
@@ -50,6 +50,11 @@ class MoELayer:
         # bf16 shared experts on a side stream, concurrently with route and permute (they
         # do not depend on the routing); joined before the combine
         self.overlap_shared = overlap_shared and not (w.fp8 or w.mxfp8) and w.n_shared > 0
+        # gather_rows: bf16 experts read their rows straight from x (moe_grouped_ffn_gather),
+        # so the permutation writes no expert-ordered copy of x (T k d elements less
+        # memory); off by default: the gathering copies are slower than the copy they save
+        self.gather_rows = (gather_rows and w.dtype == "bf16" and w.d % 64 == 0
+                            and not (w.fp8 or w.mxfp8 or w.expert_choice))
         self.dev = torch.device(device)
         self.weights = weights
         self.update_bias = update_bias and weights.get("bias") is not None
@@ -67,7 +72,7 @@ class MoELayer:
         self.offsets = z(N + 1, dtype=torch.int32)
         self.row_of_slot = z(T, k, dtype=torch.int32)
         self.token_of_row = z(max(T * k, 1), dtype=torch.int32)
-        self.x_perm = z(max(T * k, 1), d, dtype=dt)
+        self.x_perm = None if self.gather_rows else z(max(T * k, 1), d, dtype=dt)
         self.n_dropped = z(2, dtype=torch.int32)
         self.ws = z(max(L.workspace_size(self.cfg), 16), dtype=torch.uint8)
         # the tensor-core router's exact bf16 split of W_g, written once (prepare_router)
@@ -196,6 +201,9 @@ class MoELayer:
         if fp8:
             self._ffn_fp8(c, self.xq_perm, self.xs_perm, T * self.w.k, self.offsets, self.w.N,
                           ("w1", "w3", "w2"), self.w.f, self.hq, self.hsc, self.y_perm, s)
+        elif self.gather_rows:
+            L.moe_grouped_ffn_gather(c, x, T, self.token_of_row, T * self.w.k, self.offsets, self.w.N, W["w1"],
+                                     W["w3"], W["w2"], self.w.f, self.h, self.y_perm, s)
         else:
             L.moe_grouped_ffn(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
                               W["w2"], self.w.f, self.h, self.y_perm, s)
@@ -333,6 +341,8 @@ class MoELayer:
             n += 1                     # statistics in two launches around the all-reduce
         # FP8: the permutation's bf16 gather is replaced by the quantising scatter;
         # the router weight's split is written once, outside the forward
+        if self.gather_rows:
+            n -= 1                     # no row gather: the grouped FFN reads x itself
         if self.fs > 0:
             n += 2
         if self.update_bias:

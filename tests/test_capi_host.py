@@ -131,6 +131,27 @@ def test_null_and_misaligned_pointers_rejected(lib):
         L.MOE_ERR_INVALID_ARG
 
 
+def test_gathering_ffn_checks(lib):
+    """moe_grouped_ffn_gather: bf16 with d % 64 == 0 only; its row map is required;
+    no rows or no tokens is a no-op.  Nothing here reaches the GPU."""
+    ok, UN, IA = 0x1000000, L.MOE_ERR_UNSUPPORTED, L.MOE_ERR_INVALID_ARG
+    c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    cp = ctypes.byref(c)
+    f = lib.moe_grouped_ffn_gather
+    assert f(cp, ok, 100, None, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == IA      # token_of_row
+    assert f(cp, ok, 100, ok + 2, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == IA    # misaligned map
+    assert f(cp, ok + 8, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == IA    # misaligned x
+    assert f(cp, ok, -1, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == IA
+    assert f(cp, ok, 100, ok, 800, ok, 0, ok, ok, ok, 2048, ok, ok, None) == IA          # G
+    assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2047, ok, ok, None) == IA        # f % 8
+    assert f(cp, None, 0, ok, 800, ok, 256, None, None, None, 2048, None, None, None) == L.MOE_OK
+    assert f(cp, None, 100, ok, 0, ok, 256, None, None, None, 2048, None, None, None) == L.MOE_OK
+    c32 = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    assert f(ctypes.byref(c32), ok, 10, ok, 20, ok, 8, ok, ok, ok, 256, ok, ok, None) == UN
+    c.d_model = 7168 + 8                                                                    # d % 64 != 0
+    assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == UN
+
+
 def test_route_prepare_checks(lib):
     ok = 0x1000000
     c = layer.make_config(synth.WORKLOADS["deepseek_v3"])

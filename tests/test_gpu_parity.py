@@ -94,9 +94,10 @@ def _check_permute(w, lay, inp):
     R = p["R"]
     assert np.array_equal(i64(lay.token_of_row)[:R], p["token_of_row"])
     assert i64(lay.n_dropped).tolist() == [p["dropped_slots"], p["dropped_tokens"]]
-    # the gather is a byte copy
-    tor = lay.token_of_row[:R].long()
-    assert torch.equal(lay.x_perm[:R], inp["x"][tor])
+    # the gather is a byte copy (layers whose grouped FFN reads x itself write none)
+    if lay.x_perm is not None:
+        tor = lay.token_of_row[:R].long()
+        assert torch.equal(lay.x_perm[:R], inp["x"][tor])
     return p
 
 
@@ -115,7 +116,7 @@ def _check_ffn_rows(w, lay, inp, rows_by_expert):
     for e, rows in rows_by_expert.items():
         if len(rows) == 0:
             continue
-        xr = f64(lay.x_perm[rows])
+        xr = f64(inp["x"][lay.token_of_row[rows].long()])
         w1, w3, w2 = get(e)
         hr.append(O.swiglu_hidden(xr, w1, w3))
         yr.append(O.swiglu_ffn(xr, w1, w3, w2))
@@ -237,11 +238,11 @@ def test_deterministic_twice():
     inp = make_inputs(w, "cuda")
     lay = MoELayer(w, inp, "cuda", update_bias=False)
     lay.forward(inp["x"])
-    first = [t.clone() for t in (lay.topk_idx, lay.topk_w, lay.row_of_slot, lay.x_perm, lay.y_perm,
+    first = [t.clone() for t in (lay.topk_idx, lay.topk_w, lay.row_of_slot, lay.token_of_row, lay.y_perm,
                                  lay.y, lay.stats)]
     lay.forward(inp["x"])
     torch.cuda.synchronize()
-    second = (lay.topk_idx, lay.topk_w, lay.row_of_slot, lay.x_perm, lay.y_perm, lay.y, lay.stats)
+    second = (lay.topk_idx, lay.topk_w, lay.row_of_slot, lay.token_of_row, lay.y_perm, lay.y, lay.stats)
     for a, b in zip(first, second):
         assert torch.equal(a, b)
 
@@ -416,6 +417,88 @@ def test_grouped_ffn_empty_and_tiny_groups(d, f, sizes):
         if hi > lo:
             assert rel_err(f64(y[lo:hi]), ref[lo:hi]) < 2e-2, (e, sizes[e])
     assert torch.all(y[R:] == 3.0)                     # rows past the last group untouched
+
+
+@pytest.mark.parametrize("d,f,sizes", [
+    (256, 384, [0, 1, 127, 0, 128, 129, 300, 0]),
+    (384, 320, [16, 17, 112, 113, 255, 256, 257, 383, 384, 385, 511, 640, 5, 0, 31]),
+])
+def test_grouped_ffn_gather_equals_grouped_ffn_on_gathered_rows(d, f, sizes):
+    """moe_grouped_ffn_gather (rows fetched from x by index inside the first GEMM) gives
+    bit for bit what moe_grouped_ffn gives on the gathered rows x[token_of_row], over
+    every tile kind; rows past the last group stay untouched."""
+    G = len(sizes)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    R, cap = int(off[-1]), int(off[-1]) + 70
+    T = 613
+    g = torch.Generator(device="cuda").manual_seed(11)
+    x = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+    # repeats and arbitrary order, as a permutation's row map has; entries >= R are
+    # never read, so they hold an out-of-range id
+    tor = torch.randint(0, T, (cap,), generator=g, device="cuda", dtype=torch.int32)
+    tor[R:] = T + 5
+    w1 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w3 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(G, d, f, generator=g, device="cuda") / f ** 0.5).to(torch.bfloat16)
+    offs = torch.tensor(off, device="cuda")
+    cfg = make_config(replace(SMALL["mixtral_small"], d=d, f=f, N=G, T=T))
+    xr = torch.zeros(cap, d, dtype=torch.bfloat16, device="cuda")
+    xr[:R] = x[tor[:R].long()]
+    h0, h1 = (torch.empty(cap, f, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    y0, y1 = (torch.full((cap, d), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    L.moe_device_status()
+    L.moe_grouped_ffn(cfg, xr, cap, offs, G, w1, w3, w2, f, h0, y0)
+    L.moe_grouped_ffn_gather(cfg, x, T, tor, cap, offs, G, w1, w3, w2, f, h1, y1)
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(h1[:R], h0[:R])
+    assert torch.equal(y1, y0)
+
+
+def test_grouped_ffn_gather_flags_out_of_range_token_ids():
+    """A token id outside [0, T) in a read row is replaced by token 0 and recorded
+    as MOE_ERR_INVALID_ARG; the call itself completes."""
+    d, f, sizes = 256, 256, [130, 5]
+    G = len(sizes)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    R, T = int(off[-1]), 50
+    g = torch.Generator(device="cuda").manual_seed(3)
+    x = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+    tor = torch.randint(0, T, (R,), generator=g, device="cuda", dtype=torch.int32)
+    tor[7], tor[R - 1] = T, -1
+    w1 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w3 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(G, d, f, generator=g, device="cuda") / f ** 0.5).to(torch.bfloat16)
+    cfg = make_config(replace(SMALL["mixtral_small"], d=d, f=f, N=G, T=T))
+    h = torch.empty(R, f, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(R, d, dtype=torch.bfloat16, device="cuda")
+    L.moe_device_status()
+    L.moe_grouped_ffn_gather(cfg, x, T, tor, R, torch.tensor(off, device="cuda"), G, w1, w3, w2, f, h, y)
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_ERR_INVALID_ARG
+    fixed = tor.clone()
+    fixed[7], fixed[R - 1] = 0, 0
+    y_ok = torch.empty_like(y)
+    L.moe_grouped_ffn_gather(cfg, x, T, fixed, R, torch.tensor(off, device="cuda"), G, w1, w3, w2, f, h, y_ok)
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(y, y_ok)
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "v3_small", "switch_small"])
+def test_layer_gathering_ffn_equals_permuted_copy(name):
+    """The layer's output is bit-identical whether the grouped FFN reads the permuted
+    copy of x or gathers its rows from x."""
+    w = SMALL[name]
+    inp = make_inputs(w, "cuda")
+    a = MoELayer(w, inp, "cuda", update_bias=False, gather_rows=False)
+    b = MoELayer(w, inp, "cuda", update_bias=False, gather_rows=True)
+    assert a.x_perm is not None and b.x_perm is None
+    ya = a.forward(inp["x"]).clone()
+    yb = b.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert torch.equal(ya, yb)
+    assert torch.equal(a.y_perm[:int(a.offsets[-1])], b.y_perm[:int(b.offsets[-1])])
 
 
 # ----------------------------------------------------------------------------- full size
