@@ -701,6 +701,82 @@ def swiglu_ffn_mxfp8(x_rows, w1, w3, w2, hidden_out: bool = False):
 
 
 # ---------------------------------------------------------------------------
+# NVFP4 experts
+# ---------------------------------------------------------------------------
+NVFP4_BLOCK = 16
+E2M1_MAX = 6.0
+
+
+def round_e2m1(v: np.ndarray) -> np.ndarray:
+    """Round to the nearest FP4 E2M1 value (ties to even), saturating at +-6.
+
+    E2M1: 1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit; normal values
+    (1 + m/2) 2^(e-1) for e in 1..3 (1, 1.5, 2, 3, 4, 6), subnormals m/2 (0, 0.5);
+    no infinities or NaN.  The spacing is 0.5 below 2, then doubles per binade.
+    Written from that definition.
+    """
+    v = np.asarray(v, np.float64)
+    a = np.abs(v)
+    step = np.where(a >= 1.0, 2.0 ** (np.floor(np.log2(np.where(a >= 1.0, a, 1.0))) - 1.0), 0.5)
+    r = np.rint(a / step) * step                       # np.rint: round half to even
+    return np.sign(v) * np.minimum(r, E2M1_MAX)
+
+
+def nvfp4_tensor_scale(x: np.ndarray) -> np.float32:
+    """Per-tensor fp32 scale of the two-level NVFP4 scheme: amax / (6 * 448), so the
+    block scales amax_b / (6 g) stay inside UE4M3's range; 1 for an all-zero tensor."""
+    amax = np.float32(np.max(np.abs(np.asarray(x, np.float32)))) if np.size(x) else np.float32(0)
+    return np.float32(amax / np.float32(E2M1_MAX * E4M3_MAX)) if amax > 0 else np.float32(1.0)
+
+
+def quantize_nvfp4(x: np.ndarray, g: float = 1.0, block: int = NVFP4_BLOCK) -> tuple:
+    """NVFP4 quantisation along each row with tensor scale g.
+
+    [Taste] §2 (table) names NVFP4 expert compute without spelling it out.  Reading
+    (NVIDIA's NVFP4): E2M1 elements, one unsigned E4M3 scale per 16 consecutive
+    elements of the contraction dimension and one fp32 scale g per tensor.  In fp32,
+    in this order: b = E4M3(amax_b / fp32(6 g)) (round to nearest even, saturating at
+    448), s = fp32(b g), code = E2M1(fp32(x / s)); a block with b = 0 has all codes 0.
+    Dequantised value: code * b * g.  Reading of the tensor scale: weights take
+    nvfp4_tensor_scale (one per expert matrix); activations (x rows and the hidden h)
+    take g = 1, their block maxima already lying in E4M3's normal range.
+    Returns (codes as float64 values [R, C], block scales b [R, C / block] float64).
+    """
+    x32 = np.asarray(x, np.float32)
+    R, C = x32.shape
+    g = np.float32(g)
+    blocks = x32.reshape(R, C // block, block)
+    amax = np.max(np.abs(blocks), axis=2).astype(np.float32)
+    denom = np.float32(np.float32(E2M1_MAX) * g)
+    b = round_e4m3((amax / denom).astype(np.float32))
+    s = (b.astype(np.float32) * g).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = (blocks / s[:, :, None]).astype(np.float32)
+    q = np.where(b[:, :, None] > 0, round_e2m1(v), 0.0).reshape(R, C)
+    return q, b
+
+
+def dequantize_nvfp4(q: np.ndarray, b: np.ndarray, g: float = 1.0, block: int = NVFP4_BLOCK) -> np.ndarray:
+    return np.asarray(q, np.float64) * np.repeat(np.asarray(b, np.float64), block, axis=1) * float(np.float32(g))
+
+
+def swiglu_ffn_nvfp4(x_rows, w1, w3, w2, hidden_out: bool = False):
+    """The SwiGLU expert with NVFP4 operands: x (g = 1), W1, W3 (each its own tensor
+    scale) quantised along d, h (g = 1) and W2 along d_ff; fp64 products of the
+    dequantised values."""
+    xd = dequantize_nvfp4(*quantize_nvfp4(x_rows))
+
+    def wq(w):
+        g = nvfp4_tensor_scale(w)
+        return dequantize_nvfp4(*quantize_nvfp4(w, g), g)
+
+    w1d, w3d, w2d = wq(w1), wq(w3), wq(w2)
+    h = silu(xd @ w1d.T) * (xd @ w3d.T)
+    y = dequantize_nvfp4(*quantize_nvfp4(h)) @ w2d.T
+    return (y, h) if hidden_out else y
+
+
+# ---------------------------------------------------------------------------
 # Expert parallelism: the exchange plan
 # ---------------------------------------------------------------------------
 def ep_plan(offsets_all: np.ndarray, rank: int) -> dict:

@@ -841,6 +841,99 @@ def test_mxfp8_ffn_close_to_exact():
     assert np.max(np.abs(h - h0)) / np.max(np.abs(h0)) < 0.1
 
 
+# ----------------------------------------------------------------------------- NVFP4
+def _e2m1_codes():
+    """All 16 E2M1 bit patterns decoded from the format (sign, 2 exponent bits with
+    bias 1, 1 mantissa bit; exponent 0 is subnormal), with the mantissa bit."""
+    out = []
+    for code in range(16):
+        sgn, ex, m = code >> 3, (code >> 1) & 3, code & 1
+        mag = (m / 2.0) if ex == 0 else (1 + m / 2.0) * 2.0 ** (ex - 1)
+        out.append(((-1.0) ** sgn * mag, m))
+    return out
+
+
+def test_e2m1_grid_and_ties():
+    codes = _e2m1_codes()
+    mags = sorted({abs(v) for v, _ in codes})
+    assert mags == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    vals = np.array([v for v, _ in codes])
+    assert np.array_equal(O.round_e2m1(vals), vals)             # representable values are fixed
+    # midpoints go to the neighbour whose mantissa bit is 0
+    mbit = {abs(v): m for v, m in codes}
+    for lo, hi in zip(mags[:-1], mags[1:]):
+        mid = (lo + hi) / 2
+        want = lo if mbit[lo] == 0 else hi
+        assert O.round_e2m1(np.array([mid]))[0] == want, (lo, hi)
+        assert O.round_e2m1(np.array([-mid]))[0] == -want
+    assert O.round_e2m1(np.array([6.5, 1e9, -7.0])).tolist() == [6.0, 6.0, -6.0]   # saturation
+
+
+def test_e2m1_rounding_is_nearest():
+    """Brute force: the rounded value is the nearest grid value (ties: even bit)."""
+    codes = _e2m1_codes()
+    grid = np.array(sorted({v for v, _ in codes}))
+    mbit = {v: m for v, m in codes}
+    rng = np.random.default_rng(149)
+    v = np.concatenate([rng.uniform(-6, 6, 4000), np.arange(-24, 25) / 4.0])
+    r = O.round_e2m1(v)
+    for x, got in zip(v, r):
+        d = np.abs(grid - x)
+        near = grid[d == d.min()]
+        want = near[0] if len(near) == 1 else [g for g in near if mbit[g] == 0][0]
+        assert got == want, (x, got, want)
+
+
+def test_nvfp4_block_scale_hand_cases():
+    x = np.zeros((3, 32))
+    x[0, :16] = 3.0                 # amax 3, g = 1 -> b = E4M3(0.5) = 0.5, codes 6
+    x[0, 16:] = np.linspace(-1.2, 1.2, 16)   # amax 1.2 -> b = E4M3(0.2) = 0.203125
+    x[1, :16] = 3000.0              # amax 3000 -> b saturates at 448, codes saturate at 6
+    # row 2 all zero -> b = 0 and codes 0
+    q, b = O.quantize_nvfp4(x)
+    assert b[0].tolist() == [0.5, 0.203125] and b[1, 0] == 448.0 and np.all(b[2] == 0)
+    assert np.all(q[0, :16] == 6.0) and np.all(q[1, :16] == 6.0) and np.all(q[2] == 0)
+    # the second block: codes are E2M1(x / 0.203125) computed in fp32
+    want = O.round_e2m1((np.float32(1.0) * x[0, 16:].astype(np.float32) / np.float32(0.203125)))
+    assert np.array_equal(q[0, 16:], want)
+    # with a tensor scale: g = amax / 2688 maps the tensor's largest block to b = 448
+    w = np.random.default_rng(151).normal(scale=0.01, size=(8, 64))
+    g = O.nvfp4_tensor_scale(w)
+    assert g == np.float32(np.float32(np.max(np.abs(w.astype(np.float32)))) / np.float32(2688.0))
+    qw, bw = O.quantize_nvfp4(w, g)
+    assert bw.max() == 448.0 and np.all(bw <= 448.0)
+
+
+def test_nvfp4_codes_are_the_nearest_grid_point():
+    """Every dequantised element is the grid point nearest x / s (s = b g), found by
+    brute force over the 15 values; requantising the dequantised rows is exact."""
+    rng = np.random.default_rng(157)
+    x = rng.standard_t(3, size=(16, 64)) * rng.uniform(0.01, 10, size=(16, 1))
+    for g in (1.0, O.nvfp4_tensor_scale(x)):
+        q, b = O.quantize_nvfp4(x, g)
+        s = np.repeat((b.astype(np.float32) * np.float32(g)).astype(np.float32), 16, axis=1)
+        grid = np.array(sorted({v for v, _ in _e2m1_codes()}))
+        v = (x.astype(np.float32) / s).astype(np.float64)
+        nearest = grid[np.argmin(np.abs(grid[None, None, :] - np.clip(v, -6, 6)[:, :, None]), axis=2)]
+        tie = np.isclose(np.sort(np.abs(grid[None, None, :] - np.clip(v, -6, 6)[:, :, None]), axis=2)[:, :, 0],
+                         np.sort(np.abs(grid[None, None, :] - np.clip(v, -6, 6)[:, :, None]), axis=2)[:, :, 1])
+        assert np.array_equal(q[~tie], nearest[~tie])
+        xd = O.dequantize_nvfp4(q, b, g)
+        q2, b2 = O.quantize_nvfp4(xd.astype(np.float32), g)
+        assert np.array_equal(b2, b) and np.array_equal(q2, q)
+
+
+def test_nvfp4_ffn_close_to_exact():
+    rng = np.random.default_rng(163)
+    x = rng.normal(size=(16, 256))
+    w1, w3 = rng.normal(scale=256 ** -0.5, size=(2, 128, 256))
+    w2 = rng.normal(scale=128 ** -0.5, size=(256, 128))
+    y, h = O.swiglu_ffn_nvfp4(x, w1, w3, w2, hidden_out=True)
+    y0 = O.swiglu_ffn(x, w1, w3, w2)
+    err = np.max(np.abs(y - y0)) / np.max(np.abs(y0))
+    assert 0.01 < err < 0.35                       # E2M1 keeps one mantissa bit
+
+
 # ----------------------------------------------------------------------------- expert parallelism plan
 def test_ep_plan_hand_case():
     # W = 2 ranks, N = 4 experts (rank 0 holds 0, 1; rank 1 holds 2, 3)
