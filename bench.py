@@ -363,6 +363,9 @@ def main():
     ap.add_argument("--no-overlap-shared", action="store_true",
                     help="run the shared experts on the main stream after the routed experts (default: on a "
                          "side stream, concurrently with route and permute)")
+    ap.add_argument("--no-fuse-shared", action="store_true",
+                    help="run the shared expert in launches of its own instead of as one more group of the "
+                         "routed grouped-FFN launches")
     ap.add_argument("--gather-rows", action="store_true",
                     help="bf16: the grouped FFN gathers its rows from x (TMA gather4) instead of reading the "
                          "expert-ordered copy that the permutation writes")
@@ -400,7 +403,7 @@ def main():
         return run_ep(args, w, world, rank, local, dev, pg)
     inp = make_inputs(w, dev, seed=rank)
     lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD, overlap_shared=not args.no_overlap_shared,
-                   gather_rows=args.gather_rows)
+                   gather_rows=args.gather_rows, fuse_shared=not args.no_fuse_shared)
     x = inp["x"]
     stream = torch.cuda.current_stream(dev)
 
@@ -463,7 +466,9 @@ def main():
         # fp32 experts run on the FMA pipes: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
         ffn_peak, ffn_bound = 148 * 128 * 2 * 1.965e9 / 1e12, "alu"
         ffn_peak_src = "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"
-    tflops_ffn = flops_routed / (t_ffn * 1e-3) / 1e12
+    # with the shared expert fused into the routed launches, the stage does both
+    flops_ffn = flops_routed + (flops_shared if lay.fuse_shared else 0.0)
+    tflops_ffn = flops_ffn / (t_ffn * 1e-3) / 1e12
     traffic = None
     if w.name in NCU_TRAFFIC:
         srcs, nbytes = NCU_TRAFFIC[w.name]
@@ -534,7 +539,9 @@ def main():
                        "l2": (f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "
                               f"{3 * N * d * f * (1 if lowp else eb) / 1e9:.1f} GB); no flush")},
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
-            "roofline": {"kernel": "grouped SwiGLU FFN, routed experts (gate/up + down passes)",
+            "roofline": {"kernel": ("grouped SwiGLU FFN, routed + shared experts in one tile list (gate/up + "
+                                    "down passes)" if lay.fuse_shared else
+                                    "grouped SwiGLU FFN, routed experts (gate/up + down passes)"),
                          "bound": ffn_bound, "achieved": tflops_ffn,
                          "peak": ffn_peak, "unit": "TFLOP/s",
                          "frac": tflops_ffn / ffn_peak, "traffic": traffic,
@@ -547,8 +554,11 @@ def main():
                     "peak_gbs": peaks["hbm_gbs"]},
             # on a side stream the shared experts overlap route, permute and the routed
             # experts; the main stream's "shared_ffn" stage is then only the join
-            "shared_ffn_tflops": None if lay.overlap_shared else flops_shared / (t_shared * 1e-3) / 1e12,
-            "shared_experts_stream": "side (overlapped)" if lay.overlap_shared else "main",
+            "shared_ffn_tflops": (None if (lay.overlap_shared or lay.fuse_shared or lay.fs == 0)
+                                  else flops_shared / (t_shared * 1e-3) / 1e12),
+            "shared_experts": ("fused into the routed grouped-FFN launches" if lay.fuse_shared else
+                               "side stream (overlapped)" if lay.overlap_shared else
+                               "main stream" if lay.fs > 0 else "none"),
             "router_tflops_fp32": flops_router / (t_route * 1e-3) / 1e12,
             "router_stats": {"aux": st["aux"], "z_loss": st["z_loss"], "cv": st["cv"], "dead": st["dead"],
                              "dropped_slots": st["dropped_slots"], "dropped_tokens": st["dropped_tokens"]},

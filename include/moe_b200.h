@@ -229,6 +229,36 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_rows, int64_t rows_ca
                     void* h_scratch, void* y_rows, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_grouped_ffn_shared -- moe_grouped_ffn with the shared expert in the same launches.
+ *
+ * The shared expert (the Practice page's and the llm-compass "MoE 层结构" always-on
+ * expert) is the same SwiGLU FFN applied to every token: here it is one more group,
+ * of all T tokens with its own weights, scheduled with the routed groups inside the
+ * two grouped-GEMM launches (one tile list, no second pair of launches, no launch
+ * tails between them).  Same arithmetic as moe_grouped_ffn on each part: the routed
+ * outputs equal moe_grouped_ffn's and the shared outputs equal moe_grouped_ffn with
+ * G = 1, offsets = {0, T}, bit for bit.
+ *   x_rows, rows_cap, offsets, G, w1, w3, w2, f  the routed groups, as for
+ *                     moe_grouped_ffn
+ *   h_scratch         [rows_cap + T, f] bf16 (written, then read): the groups' hidden
+ *                     rows, then the shared expert's (row rows_cap + t for token t)
+ *   y_rows            [rows_cap + T, d] bf16 out: the groups' rows (rows >= offsets[G]
+ *                     and < rows_cap untouched), then the shared expert's output for
+ *                     token t at row rows_cap + t
+ *   x                 [T, d] bf16: the shared expert's input (token order)
+ *   ws1, ws3          [f, d] bf16; ws2 [d, f] bf16: the shared expert, hidden width f
+ *                     (the routed experts' f; shared experts of another total width
+ *                     take moe_grouped_ffn with G = 1)
+ * Errors: MOE_ERR_UNSUPPORTED unless bf16, or when rows_cap + T exceeds INT32_MAX;
+ * MOE_ERR_INVALID_ARG as for moe_grouped_ffn, for G > 511, T < 0, or a NULL or
+ * misaligned buffer.  T = 0 is moe_grouped_ffn.
+ * ------------------------------------------------------------------------- */
+int moe_grouped_ffn_shared(const moe_config_t* cfg, const void* x_rows, int64_t rows_cap,
+                           const int32_t* offsets, int32_t G, const void* w1, const void* w3, const void* w2,
+                           int32_t f, void* h_scratch, void* y_rows, const void* x, int64_t T, const void* ws1,
+                           const void* ws3, const void* ws2, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_grouped_ffn_gather -- moe_grouped_ffn reading each row straight from x.
  *
  * The same grouped SwiGLU FFN (same sources, same arithmetic, bit-identical

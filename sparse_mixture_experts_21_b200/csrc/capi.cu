@@ -217,6 +217,28 @@ int moe_grouped_ffn(const moe_config_t* cfg, const void* x_rows, int64_t rows_ca
                                   static_cast<float*>(y_rows), s));
 }
 
+int moe_grouped_ffn_shared(const moe_config_t* cfg, const void* x_rows, int64_t rows_cap,
+                           const int32_t* offsets, int32_t G, const void* w1, const void* w3, const void* w2,
+                           int32_t f, void* h_scratch, void* y_rows, const void* x, int64_t T, const void* ws1,
+                           const void* ws3, const void* ws2, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->x_dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (T == 0)
+    return moe_grouped_ffn(cfg, x_rows, rows_cap, offsets, G, w1, w3, w2, f, h_scratch, y_rows, stream);
+  if (rows_cap < 0 || G < 1 || G > 511 || f <= 0 || (f % 8) != 0 || !offsets) return MOE_ERR_INVALID_ARG;
+  if (rows_cap + T > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (!w1 || !w3 || !w2 || !x || !ws1 || !ws3 || !ws2 || !h_scratch || !y_rows) return MOE_ERR_INVALID_ARG;
+  if (rows_cap > 0 && !x_rows) return MOE_ERR_INVALID_ARG;
+  if ((x_rows && !aligned16(x_rows)) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) ||
+      !aligned16(h_scratch) || !aligned16(y_rows) || !aligned16(x) || !aligned16(ws1) || !aligned16(ws3) ||
+      !aligned16(ws2))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_ffn_bf16_shared(x_rows, rows_cap, offsets, G, w1, w3, w2, cfg->d_model, f, h_scratch,
+                                          y_rows, x, (int)T, ws1, ws3, ws2, static_cast<cudaStream_t>(stream)));
+}
+
 int moe_grouped_ffn_gather(const moe_config_t* cfg, const void* x, int64_t T, const int32_t* token_of_row,
                            int64_t rows_cap, const int32_t* offsets, int32_t G, const void* w1, const void* w3,
                            const void* w2, int32_t f, void* h_scratch, void* y_rows, void* stream) {

@@ -5,58 +5,48 @@
 // expert itself is E(x) = W2 (silu(W1 x) * (W3 x)) (three matrices per expert, as
 // in its "推理侧的路由稳定性" parameter count E x 3D^2).
 //
-// Two persistent launches over tile lists built on the device from `offsets`:
-//   gate/up (this file): H[r, n0:n0+128] = silu(X W1[g]^T) * (X W3[g]^T); the weight
+// Two persistent launches of one kernel over tile lists built on the device from
+// `offsets`:
+//   gate/up (MODE 0): H[r, n0:n0+128] = silu(X W1[g]^T) * (X W3[g]^T); the weight
 //          tile stacks 128 rows of W1 over 128 rows of W3, so one N = 256 MMA gives
 //          gate and up for 128 hidden units and SwiGLU runs in the epilogue from TMEM.
-//   down (ffn_down.cu): Y[r, n0:n0+256] = H W2[g]^T.
+//   down (MODE 1):    Y[r, n0:n0+256] = H W2[g]^T.
 // Every MMA is tcgen05.mma.cta_group::1.kind::f16 (bf16 in, fp32 accumulate in
 // TMEM); operands come by TMA (128-byte swizzle, no multicast).
 //
-// Gate/up pass (long K = d): a CTA tile is up to two sub-tiles of one group sharing
-// each weight stage.  Per 64-wide K step a stage holds A0 16 KB + A1 16 KB + W 32 KB
-// (the weight tile), 64 bytes of operand traffic per MMA cycle for two full
-// sub-tiles (96 with one 128-row tile); 3-stage ring; TMEM holds two 256-column fp32
-// accumulators, one per sub-tile.  To hide the epilogue, the 8 epilogue warps drain
-// accumulator 0 first, and as soon as it is free the MMA warp computes sub-tile 0 of
-// the next tile over the first resident stages, then waits for accumulator 1 and
-// catches up sub-tile 1 on the same stages.
+// A CTA tile is up to two 128-row sub-tiles of one group sharing each weight stage.
+// Per 64-wide K step a stage holds A0 16 KB + A1 16 KB + W 32 KB (the weight tile),
+// 64 bytes of operand traffic per MMA cycle for two full sub-tiles (96 with one
+// 128-row tile); 3-stage ring; TMEM holds two 256-column fp32 accumulators, one per
+// sub-tile.  To hide the epilogue, the 8 epilogue warps drain accumulator 0 first,
+// and as soon as it is free the MMA warp computes sub-tile 0 of the next tile over
+// the first resident stages, then waits for accumulator 1 and catches up sub-tile 1
+// on the same stages.
 //
-// No padding rows in the gate/up pass.  A group of R rows is cut into floor(R / 128)
-// full 128-row sub-tiles (paired two by two) and a ragged tail of r = R mod 128 rows.
-// The tail is computed transposed ("swapped"): the weight tile already in shared
-// memory is the MMA's A operand (M = 128 weight rows, i.e. output columns) and the r
-// tail rows are its B operand (N = r rounded up to 16), so the tail costs its own MMA
-// work, not that of a 128-row tile, and reuses the weight stages of the group's last
-// full sub-tile.  Kinds of tile:
+// No padding rows.  A group of R rows is cut into floor(R / 128) full 128-row
+// sub-tiles (paired two by two) and a ragged tail of r = R mod 128 rows.  The tail
+// is computed transposed ("swapped"): the weight tile already in shared memory is
+// the MMA's A operand (M = 128 weight rows, i.e. output columns) and the r tail rows
+// are its B operand (N = r rounded up to 16), so the tail costs its own MMA work,
+// not that of a 128-row tile, and reuses the weight stages of the group's last full
+// sub-tile.  Kinds of tile:
 //   PAIR   two full sub-tiles;
 //   SINGLE one full sub-tile (an odd count of full sub-tiles), no tail;
 //   ST     one full sub-tile + the group's tail as sub-tile 1 (swapped);
 //   T      the tail alone (an even count of full sub-tiles, or R < 128).
-// The swapped sub-tile writes D^T into accumulator 1: weight rows 0..127 (W1, gate)
-// into columns [0, n) and rows 128..255 (W3, up) into columns [128, 128 + n), so gate
-// and up of one hidden unit share a TMEM lane.
+// The swapped sub-tile writes D^T into accumulator 1: weight rows 0..127 into
+// columns [0, n) and rows 128..255 into columns [128, 128 + n) (gate/up: W1 and W3,
+// so gate and up of one hidden unit share a TMEM lane; down: the two 128-column
+// halves of the output tile).
 //
-// Tile order and scheduling (gate/up): group, n-tile, then that (group, n-tile)'s
-// PAIR tiles followed by its extra tile.  Tiles are claimed dynamically -- the
-// producer warp takes the next index from a per-launch global counter and hands it
-// to the MMA and epilogue warps through a small shared-memory queue -- so the tiles
-// in flight are always a contiguous window of the list and the CTAs that share a
-// weight tile run together, whatever the tiles' lengths (a static round-robin
-// assignment lets CTAs drift apart and stream weight tiles from DRAM again).  The
-// last CTA to finish resets the counter.
-//
-// Down pass (short K = f): 128-row tiles of one group (group, n-tile, m-tile order,
-// static: every tile has the same length), 4-stage ring of 48 KB, two TMEM
-// accumulators used alternately so one tile's epilogue (4 warps) overlaps the next
-// tile's MMAs completely.  Rows past a group's end are computed from whatever
-// follows and never stored.
-//
-// Gathering form (ffn_tc_kernel<true>): the A rows come from x by token index
-// (TMA tile::gather4, four one-row boxes per copy, every lane of warp 0 issuing its
-// own four rows), so the expert-ordered copy of x is never written.  Same MMAs, same
-// shared-memory layout, bit-identical output; measured at about 76 cycles per
-// 512-byte gather4 copy per SM, it is slower than the row copy it saves.
+// Tile order and scheduling: group, n-tile, then that (group, n-tile)'s PAIR tiles
+// followed by its extra tile.  Tiles are claimed dynamically -- the producer warp
+// takes the next index from a per-launch global counter and hands it to the MMA
+// and epilogue warps through a small shared-memory queue -- so the tiles in flight
+// are always a contiguous window of the list and the CTAs that share a weight tile
+// run together, whatever the tiles' lengths (a static round-robin assignment lets
+// CTAs drift apart and stream weight tiles from DRAM again).  The last CTA to
+// finish resets the counter.
 //
 // Warp roles: 0 = TMA producer (and tile claims), 1 = TMEM allocator + MMA issuer,
 // 2.. = epilogue (TMEM lane quarter = warp % 4).  Every mbarrier wait is bounded; on
@@ -101,8 +91,8 @@ struct __align__(8) TcShared {
   uint32_t tmem_base;
   volatile int32_t abort;
   volatile int32_t tq[TQ];        // claimed tile indices (>= total: no more tiles)
-  int32_t goff[kMaxGroups + 1];   // group row offsets
-  int32_t tpre[kMaxGroups + 1];   // prefix over groups of (PAIR tiles + extra tile) per n-tile
+  int32_t goff[kMaxGroups + 3];   // group row offsets (then an empty gap and the extra group)
+  int32_t tpre[kMaxGroups + 3];   // prefix over groups of (PAIR tiles + extra tile) per n-tile
 };
 
 // Per-launch tile counters: [slot][0] = next tile to claim, [slot][1] = CTAs done.
@@ -171,8 +161,18 @@ __device__ __forceinline__ Tile decode_tile(int L, const TcShared* sh, int G, in
   return t;
 }
 
-// Per-group tile prefixes (PAIR tiles + at most one extra tile, per n-tile), one warp.
-__device__ void build_tile_table(TcShared* sh, const int32_t* offsets, int G, int lane) {
+// Tiles of a group of `rows` rows per n-tile: its PAIR tiles + at most one more.
+__device__ __forceinline__ int group_tiles(int rows) {
+  const int full = rows / SUB;
+  return full / 2 + (((full & 1) || rows % SUB) ? 1 : 0);
+}
+
+// Per-group tile prefixes, one warp.  With a dense extra group (rows_x > 0) the
+// list goes on with an empty group over rows [offsets[G], rows_cap) and the extra
+// group G + 1 over rows [rows_cap, rows_cap + rows_x): its rows are numbered as its
+// output rows.
+__device__ void build_tile_table(TcShared* sh, const int32_t* offsets, int G, int rows_x, int rows_cap,
+                                 int lane) {
   int carry = 0;
   for (int base = 0; base < G; base += 32) {
     const int g = base + lane;
@@ -180,9 +180,7 @@ __device__ void build_tile_table(TcShared* sh, const int32_t* offsets, int G, in
     if (g < G) {
       const int o0 = offsets[g], o1 = offsets[g + 1];
       sh->goff[g] = o0;
-      const int rows = o1 > o0 ? o1 - o0 : 0;
-      const int full = rows / SUB;
-      mt = full / 2 + (((full & 1) || rows % SUB) ? 1 : 0);
+      mt = group_tiles(o1 > o0 ? o1 - o0 : 0);
     }
     int incl = mt;
 #pragma unroll
@@ -196,6 +194,12 @@ __device__ void build_tile_table(TcShared* sh, const int32_t* offsets, int G, in
   if (lane == 0) {
     sh->tpre[0] = 0;
     sh->goff[G] = offsets[G];
+    if (rows_x > 0) {
+      sh->goff[G + 1] = rows_cap;
+      sh->goff[G + 2] = rows_cap + rows_x;
+      sh->tpre[G + 1] = carry;
+      sh->tpre[G + 2] = carry + group_tiles(rows_x);
+    }
   }
 }
 
@@ -210,14 +214,17 @@ __device__ __forceinline__ bool next_tile(TcShared* sh, uint32_t i, int* L) {
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
 
 // Swapped (tail) epilogue.  The epilogue loads the same TMEM columns for a normal
-// and for a swapped sub-tile (columns [64 h, 64 h + 64) and 128 + those); only their
-// meaning differs.  Normal: the lane is a row and the columns are hidden units.
-// Swapped: the lane is a hidden unit (n0 + 32 q + lane) and warp half h holds tail
-// rows [64 h, 64 h + 64) (gate at v[i], up at v[64 + i]).  Columns past the tail
-// hold stale values and are never stored.
+// and for a swapped sub-tile (gate/up: columns [64 h, 64 h + 64) and 128 + those;
+// down: [128 h, 128 h + 128)); only their meaning differs.  Normal: the lane is a
+// row and the columns are output columns.  Swapped: the lane is an output column
+// and the columns are tail rows -- gate/up: warp half h holds tail rows
+// [64 h, 64 h + 64) of hidden unit n0 + 32 q + lane (gate at v[i], up at v[64 + i]);
+// down: warp half h holds every tail row of output column n0 + 128 h + 32 q + lane.
+// Columns past the tail hold stale values and are never stored.
+template <int MODE>
 __device__ __forceinline__ void store_swapped(const uint32_t* v, const Tile& t, int half, int q, int lane,
                                               int n_out, int64_t rows_cap, __nv_bfloat16* out) {
-  const int col = t.n0 + 32 * q + lane;
+  const int col = t.n0 + (MODE == 0 ? 0 : 128 * half) + 32 * q + lane;
   const int64_t lim64 = rows_cap - t.trow0;
   const int lim = (int)(lim64 < t.tr ? lim64 : t.tr);        // tail rows to store
   if (col >= n_out) return;
@@ -225,13 +232,22 @@ __device__ __forceinline__ void store_swapped(const uint32_t* v, const Tile& t, 
   __nv_bfloat16* p = out + (int64_t)t.trow0 * ld + col;
   // one running pointer (a chain of adds), so the unrolled loop does not keep an
   // address per row live
-  const int n = lim - half * 64;
-  p += (int64_t)(half * 64) * ld;
+  if (MODE == 0) {
+    const int n = lim - half * 64;
+    p += (int64_t)(half * 64) * ld;
 #pragma unroll
-  for (int i = 0; i < 64; ++i) {
-    if (i < n) *p = __float2bfloat16_rn(silu_f(__uint_as_float(v[i])) * __uint_as_float(v[64 + i]));
-    asm volatile("" : "+l"(p));
-    p += ld;
+    for (int i = 0; i < 64; ++i) {
+      if (i < n) *p = __float2bfloat16_rn(silu_f(__uint_as_float(v[i])) * __uint_as_float(v[64 + i]));
+      asm volatile("" : "+l"(p));
+      p += ld;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 128; ++i) {
+      if (i < lim) *p = __float2bfloat16_rn(__uint_as_float(v[i]));
+      asm volatile("" : "+l"(p));
+      p += ld;
+    }
   }
 }
 
@@ -246,18 +262,33 @@ __device__ __forceinline__ int32_t token_at(const int32_t* __restrict__ token_of
   return v;
 }
 
-// GATHER = false: A rows come from the expert-ordered rows X (map tmA, 128-row boxes;
-// tmAt, 16-row boxes for the tails).  GATHER = true: row r of group g is token
-// token_of_row[r] of x [T, K], fetched with tile::gather4 (tmA over x, one-row
-// boxes; tmAt unused), so the expert-ordered copy of x is never written.
-template <bool GATHER>
+// MODE 0: gate/up (B = W1 rows over W3 rows, maps tmB0 / tmB1, 128-row boxes; the
+// epilogue applies SwiGLU); MODE 1: down (B = one 256-row W2 box, map tmB0).
+// GATHER = false: A rows come from the expert-ordered rows (map tmA, 128-row boxes;
+// tmAt, 16-row boxes for the tails).  GATHER = true (gate/up only): row r of group g
+// is token token_of_row[r] of x [T, K], fetched with tile::gather4 (tmA over x,
+// one-row boxes; tmAt unused), so the expert-ordered copy of x is never written.
+// The dense extra group (the shared expert run inside the same launches): its
+// input rows are rows a_base .. a_base + rows - 1 of map a (128-row boxes; at: the
+// tail boxes), its weights b0 / b1 (as for the groups); its outputs are rows
+// rows_cap .. rows_cap + rows - 1 of the pass's output.  rows = 0: none.  Only the
+// non-gathering form takes one.  In the tile list it is group G + 1, after an
+// empty group G over the unused rows [offsets[G], rows_cap).
+struct ExtraGroup {
+  CUtensorMap a, at, b0, b1;
+  int a_base;
+  int rows;
+};
+
+template <int MODE, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAt,
               const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
               const int32_t* __restrict__ offsets, int G, int K, int n_out, int64_t rows_cap,
               __nv_bfloat16* __restrict__ out, int ctr_slot, const int32_t* __restrict__ token_of_row,
-              int T) {
-  constexpr int BN = 128;                      // hidden units per tile
+              int T, const __grid_constant__ ExtraGroup xg) {
+  static_assert(MODE == 0 || !GATHER, "only the gate/up pass gathers its rows");
+  constexpr int BN = MODE == 0 ? 128 : 256;    // output columns per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -277,18 +308,26 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmAt);
     prefetch_tmap(&tmB0);
-    prefetch_tmap(&tmB1);
+    if (MODE == 0) prefetch_tmap(&tmB1);
+    if (xg.rows > 0) {
+      prefetch_tmap(&xg.a);
+      prefetch_tmap(&xg.at);
+      prefetch_tmap(&xg.b0);
+      if (MODE == 0) prefetch_tmap(&xg.b1);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&sh->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 2) build_tile_table(sh, offsets, G, lane);
+  const int rows_x = GATHER ? 0 : xg.rows;
+  if (warp == 2) build_tile_table(sh, offsets, G, rows_x, (int)rows_cap, lane);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sh->tmem_base;
-  const int total = sh->tpre[G] * tiles_n;
+  const int Gt = G + (rows_x > 0 ? 2 : 0);     // groups in the tile list
+  const int total = sh->tpre[Gt] * tiles_n;
   int32_t* ctr = g_tile_ctr[ctr_slot];
 
   if (warp == 0 && GATHER) {
@@ -311,7 +350,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       L = __shfl_sync(0xffffffffu, L, 0);
       if (L < 0) { ok = false; break; }
       if (L >= total) break;
-      const Tile t = decode_tile(L, sh, G, tiles_n, BN);
+      const Tile t = decode_tile(L, sh, Gt, tiles_n, BN);
       const int brow = t.g * n_out + t.n0;
       const uint32_t bytes = (t.has0() ? A_BYTES : 0) + (t.kind == K_PAIR ? A_BYTES : 0) +
                              (t.swap1() ? t.tn * BK * 2 : 0) + W_BYTES;
@@ -341,7 +380,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
           tma_gather4(&tmA, a + A_BYTES + lane * 512, &sh->full[stage], kb * BK, r1[0], r1[1], r1[2], r1[3]);
         if (lane == 0) {
           tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
-          tma_load_2d(&tmB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
+          if (MODE == 0) tma_load_2d(&tmB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
         }
         ++issued;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -369,8 +408,15 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         sh->tq[qs] = L;
         mbar_arrive(&sh->tq_full[qs]);
         if (L >= total) break;
-        const Tile t = decode_tile(L, sh, G, tiles_n, BN);
-        const int brow = t.g * n_out + t.n0;
+        Tile t = decode_tile(L, sh, Gt, tiles_n, BN);
+        // the extra group reads its own maps, rows counted from its first row
+        const bool ex = t.g == G + 1;
+        const CUtensorMap* mA = ex ? &xg.a : &tmA;
+        const CUtensorMap* mAt = ex ? &xg.at : &tmAt;
+        const CUtensorMap* mB0 = ex ? &xg.b0 : &tmB0;
+        const CUtensorMap* mB1 = ex ? &xg.b1 : &tmB1;
+        if (ex) { t.row0 += xg.a_base - (int)rows_cap; t.trow0 += xg.a_base - (int)rows_cap; }
+        const int brow = (ex ? 0 : t.g * n_out) + t.n0;
         const uint32_t bytes = (t.has0() ? A_BYTES : 0) + (t.kind == K_PAIR ? A_BYTES : 0) +
                                (t.swap1() ? t.tn * BK * 2 : 0) + W_BYTES;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -378,14 +424,14 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
           uint8_t* a = smem + (size_t)stage * STAGE_BYTES;
           uint8_t* b = a + 2 * A_BYTES;
           mbar_arrive_expect_tx(&sh->full[stage], bytes);
-          if (t.has0()) tma_load_2d(&tmA, a, &sh->full[stage], kb * BK, t.row0);
-          if (t.kind == K_PAIR) tma_load_2d(&tmA, a + A_BYTES, &sh->full[stage], kb * BK, t.row0 + SUB);
+          if (t.has0()) tma_load_2d(mA, a, &sh->full[stage], kb * BK, t.row0);
+          if (t.kind == K_PAIR) tma_load_2d(mA, a + A_BYTES, &sh->full[stage], kb * BK, t.row0 + SUB);
           if (t.swap1())
             for (int j = 0; j < t.tn / TAIL_BOX; ++j)
-              tma_load_2d(&tmAt, a + A_BYTES + j * TAIL_BOX * BK * 2, &sh->full[stage], kb * BK,
+              tma_load_2d(mAt, a + A_BYTES + j * TAIL_BOX * BK * 2, &sh->full[stage], kb * BK,
                           t.trow0 + j * TAIL_BOX);
-          tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
-          tma_load_2d(&tmB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
+          tma_load_2d(mB0, b, &sh->full[stage], kb * BK, brow);
+          if (MODE == 0) tma_load_2d(mB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -439,7 +485,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         if (!next_tile(sh, i, &L)) break;
         mbar_arrive(&sh->tq_empty[i % TQ]);
         if (L >= total) break;
-        const Tile t = decode_tile(L, sh, G, tiles_n, BN);
+        const Tile t = decode_tile(L, sh, Gt, tiles_n, BN);
         const bool h0 = t.has0(), h1 = t.has1(), sw = t.swap1();
         if (h0) {
           if (!wait_or_abort(&sh->tempty[0], (use0 & 1u) ^ 1u, sh)) { ok = false; break; }
@@ -498,41 +544,52 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->tq_empty[i % TQ]);
       if (L >= total) break;
-      const Tile t = decode_tile(L, sh, G, tiles_n, BN);
+      // only the kind here; the rest of the tile is decoded again after the TMEM
+      // loads, so it is not held in registers across them
+      const int kind = decode_tile(L, sh, Gt, tiles_n, BN).kind;
       bool ok = true;
       for (int sub = 0; sub < 2; ++sub) {
-        if (sub == 0 ? !t.has0() : !t.has1()) continue;
+        if (sub == 0 ? kind == K_T : kind == K_SINGLE) continue;
         uint32_t& use = sub == 0 ? use0 : use1;
         if (!__all_sync(0xffffffffu, wait_or_abort(&sh->tfull[sub], use & 1u, sh))) { ok = false; break; }
         tc_fence_after();
         const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + sub * 256u;
         uint32_t v[128];
-        const bool swapped = sub == 1 && t.swap1();
-        // gate columns [64 h, 64 h + 64) and the matching up columns
+        const bool swapped = sub == 1 && kind >= K_ST;
+        if (MODE == 0) {               // gate columns [64 h, 64 h + 64) and the matching up columns
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          tmem_ld16(tbase + half * 64 + 16 * j, v + 16 * j);
-          tmem_ld16(tbase + 128 + half * 64 + 16 * j, v + 64 + 16 * j);
+          for (int j = 0; j < 4; ++j) {
+            tmem_ld16(tbase + half * 64 + 16 * j, v + 16 * j);
+            tmem_ld16(tbase + 128 + half * 64 + 16 * j, v + 64 + 16 * j);
+          }
+        } else {                       // output columns [128 h, 128 h + 128)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) tmem_ld16(tbase + half * 128 + 16 * j, v + 16 * j);
         }
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh->tempty[sub]);
         ++use;
+        const Tile t = decode_tile(L, sh, Gt, tiles_n, BN);
         if (swapped) {
-          store_swapped(v, t, half, q, lane, n_out, rows_cap, out);
+          store_swapped<MODE>(v, t, half, q, lane, n_out, rows_cap + (GATHER ? 0 : xg.rows), out);
           continue;
         }
         const int r = sub * SUB + q * 32 + lane;
         const int64_t grow = (int64_t)t.row0 + r;
-        if (grow < rows_cap) {
+        // output rows: the groups' rows_cap rows, then the extra group's
+        if (grow < rows_cap + (GATHER ? 0 : xg.rows)) {
           __nv_bfloat16* orow = out + grow * (int64_t)n_out + t.n0;
-          const int c0 = half * 64;                    // this thread's 64 hidden units
+          constexpr int NC = MODE == 0 ? 64 : 128;     // output columns of this thread
+          const int c0 = half * NC;
 #pragma unroll
-          for (int j = 0; j < 64; j += 8) {
+          for (int j = 0; j < NC; j += 8) {
             float o[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) o[i] = silu_f(__uint_as_float(v[j + i])) * __uint_as_float(v[64 + j + i]);
+            for (int i = 0; i < 8; ++i)
+              o[i] = MODE == 0 ? silu_f(__uint_as_float(v[j + i])) * __uint_as_float(v[64 + j + i])
+                               : __uint_as_float(v[j + i]);
             if (t.n0 + c0 + j + 8 <= n_out) {
               uint4 pk;
               pk.x = pack_bf16x2(o[0], o[1]); pk.y = pack_bf16x2(o[2], o[3]);
@@ -567,28 +624,22 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 // streams never share a tile-counter slot.
 static std::atomic<unsigned> g_next_slot{0};
 
-template <bool GATHER>
-static cudaError_t launch_gate_up_t(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
-                                    const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
-                                    int64_t rows_cap, void* out, const int32_t* token_of_row, int T,
-                                    cudaStream_t s) {
-  constexpr int BN = 128;
-  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<GATHER>, (int)kSmem);
+template <int MODE, bool GATHER>
+static cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
+                               const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
+                               int64_t rows_cap, void* out, const int32_t* token_of_row, int T,
+                               const ExtraGroup& xg, cudaStream_t s) {
+  constexpr int BN = MODE == 0 ? 128 : 256;
+  const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<MODE, GATHER>, (int)kSmem);
   if (e != cudaSuccess) return e;
   const int64_t tiles_n = (n_out + BN - 1) / BN;
-  const int64_t max_tiles = ((rows_cap + SUB - 1) / SUB + G) * tiles_n;
+  const int64_t max_tiles = ((rows_cap + xg.rows + SUB - 1) / SUB + G + 1) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
   const int slot = (int)(g_next_slot.fetch_add(1) % kCtrSlots);
-  ffn_tc_kernel<GATHER><<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
-                                                     static_cast<__nv_bfloat16*>(out), slot, token_of_row, T);
+  ffn_tc_kernel<MODE, GATHER><<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
+                                                           static_cast<__nv_bfloat16*>(out), slot, token_of_row, T, xg);
   return cudaGetLastError();
-}
-
-cudaError_t launch_gate_up(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
-                           const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
-                           int64_t rows_cap, void* out, cudaStream_t s) {
-  return launch_gate_up_t<false>(a, at, b0, b1, offsets, G, K, n_out, rows_cap, out, nullptr, 0, s);
 }
 
 }  // namespace tc
@@ -598,15 +649,49 @@ cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t*
                             void* y, cudaStream_t s) {
   if (rows_cap == 0 || G == 0) return cudaSuccess;
   if (G > tc::kMaxGroups) return cudaErrorInvalidValue;
-  CUtensorMap mx, mxt, m1, m3, mh, m2;
+  CUtensorMap mx, mxt, m1, m3, mh, mht, m2;
   if (!make_map_bf16(&mx, x_rows, rows_cap, d, tc::SUB) ||
       !make_map_bf16(&mxt, x_rows, rows_cap, d, tc::TAIL_BOX) ||
       !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) || !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) ||
-      !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) || !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
+      !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) || !make_map_bf16(&mht, h, rows_cap, f, tc::TAIL_BOX) ||
+      !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
     return cudaErrorInvalidValue;
-  cudaError_t e = tc::launch_gate_up(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, s);
+  tc::ExtraGroup none{};
+  none.a = none.at = none.b0 = none.b1 = mx;
+  cudaError_t e = tc::launch_pass<0, false>(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, nullptr, 0, none, s);
   if (e != cudaSuccess) return e;
-  return launch_ffn_down(mh, m2, offsets, G, f, d, rows_cap, y, s);
+  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, none, s);
+}
+
+cudaError_t launch_ffn_bf16_shared(const void* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
+                                   const void* w1, const void* w3, const void* w2, int d, int f, void* h, void* y,
+                                   const void* xs, int Ts, const void* ws1, const void* ws3, const void* ws2,
+                                   cudaStream_t s) {
+  if (G > tc::kMaxGroups - 1) return cudaErrorInvalidValue;
+  if (Ts == 0) return launch_ffn_bf16(x_rows, rows_cap, offsets, G, w1, w3, w2, d, f, h, y, s);
+  // h and y hold the groups' rows_cap rows followed by the shared expert's Ts rows;
+  // with no routed rows the routed input map points at xs (never read)
+  const int64_t hr = rows_cap + Ts;
+  const void* xr = rows_cap > 0 ? x_rows : xs;
+  const int64_t xrows = rows_cap > 0 ? rows_cap : Ts;
+  CUtensorMap mx, mxt, m1, m3, mh, mht, m2;
+  tc::ExtraGroup g0{}, g1{};
+  if (!make_map_bf16(&mx, xr, xrows, d, tc::SUB) || !make_map_bf16(&mxt, xr, xrows, d, tc::TAIL_BOX) ||
+      !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) || !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) ||
+      !make_map_bf16(&mh, h, hr, f, tc::SUB) || !make_map_bf16(&mht, h, hr, f, tc::TAIL_BOX) ||
+      !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256) || !make_map_bf16(&g0.a, xs, Ts, d, tc::SUB) ||
+      !make_map_bf16(&g0.at, xs, Ts, d, tc::TAIL_BOX) || !make_map_bf16(&g0.b0, ws1, f, d, 128) ||
+      !make_map_bf16(&g0.b1, ws3, f, d, 128) || !make_map_bf16(&g1.b0, ws2, d, f, 256))
+    return cudaErrorInvalidValue;
+  g0.a_base = 0;
+  g1.a = mh;
+  g1.at = mht;
+  g1.b1 = g1.b0;
+  g1.a_base = (int)rows_cap;
+  g0.rows = g1.rows = Ts;
+  cudaError_t e = tc::launch_pass<0, false>(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, nullptr, 0, g0, s);
+  if (e != cudaSuccess) return e;
+  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, g1, s);
 }
 
 cudaError_t launch_ffn_bf16_gather(const void* x, int T, const int32_t* token_of_row, int64_t rows_cap,
@@ -614,14 +699,16 @@ cudaError_t launch_ffn_bf16_gather(const void* x, int T, const int32_t* token_of
                                    int d, int f, void* h, void* y, cudaStream_t s) {
   if (rows_cap == 0 || G == 0 || T == 0) return cudaSuccess;
   if (G > tc::kMaxGroups) return cudaErrorInvalidValue;
-  CUtensorMap mx, m1, m3, mh, m2;
+  CUtensorMap mx, m1, m3, mh, mht, m2;
   if (!make_map_bf16(&mx, x, (uint64_t)T, d, 1) || !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) ||
       !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) || !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) ||
-      !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
+      !make_map_bf16(&mht, h, rows_cap, f, tc::TAIL_BOX) || !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
     return cudaErrorInvalidValue;
-  cudaError_t e = tc::launch_gate_up_t<true>(mx, mx, m1, m3, offsets, G, d, f, rows_cap, h, token_of_row, T, s);
+  tc::ExtraGroup none{};
+  none.a = none.at = none.b0 = none.b1 = mh;
+  cudaError_t e = tc::launch_pass<0, true>(mx, mx, m1, m3, offsets, G, d, f, rows_cap, h, token_of_row, T, none, s);
   if (e != cudaSuccess) return e;
-  return launch_ffn_down(mh, m2, offsets, G, f, d, rows_cap, y, s);
+  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, none, s);
 }
 
 }  // namespace moe

@@ -50,14 +50,17 @@ cudaError_t launch_permute(const moe_config_t& c, int64_t capacity, const void* 
 cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
                             const void* w1, const void* w3, const void* w2, int d, int f,
                             void* h, void* y, cudaStream_t s);
+// The same FFN plus one dense group of Ts rows (xs [Ts, d], its own ws1/ws3 [f, d],
+// ws2 [d, f]) in the same two launches; h [rows_cap + Ts, f] and y [rows_cap + Ts, d]
+// hold its rows after the groups' rows_cap rows.
+cudaError_t launch_ffn_bf16_shared(const void* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
+                                   const void* w1, const void* w3, const void* w2, int d, int f, void* h, void* y,
+                                   const void* xs, int Ts, const void* ws1, const void* ws3, const void* ws2,
+                                   cudaStream_t s);
 // The same FFN with row r of group g read from x[token_of_row[r]] (x [T, d] bf16).
 cudaError_t launch_ffn_bf16_gather(const void* x, int T, const int32_t* token_of_row, int64_t rows_cap,
                                    const int32_t* offsets, int G, const void* w1, const void* w3, const void* w2,
                                    int d, int f, void* h, void* y, cudaStream_t s);
-// Down projection over row groups: H (map `mh`, 128-row boxes) times W2 (map `m2`,
-// 256-row boxes) -> Y [rows_cap, d] bf16.
-cudaError_t launch_ffn_down(const CUtensorMap& mh, const CUtensorMap& m2, const int32_t* offsets, int G, int f,
-                            int d, int64_t rows_cap, void* y, cudaStream_t s);
 cudaError_t launch_ffn_f32(const float* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
                            const float* w1, const float* w3, const float* w2, int d, int f,
                            float* h, float* y, cudaStream_t s);

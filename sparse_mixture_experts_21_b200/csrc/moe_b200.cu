@@ -5,7 +5,6 @@
 #include "route.cu"
 #include "permute.cu"
 #include "permute_noalloc.cu"
-#include "ffn_down.cu"
 #include "ffn_tc.cu"
 #include "ffn_f32.cu"
 #include "combine_stats.cu"

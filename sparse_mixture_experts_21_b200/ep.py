@@ -181,7 +181,7 @@ class EPMoELayer:
         # the single-rank layer supplies routing, permutation, shared experts, combine, stats;
         # it keeps only this rank's experts
         local = {k: v for k, v in weights.items() if k not in ("w1", "w3", "w2")}
-        self.base = MoELayer(w, local, dev, update_bias=False, gather_rows=False)
+        self.base = MoELayer(w, local, dev, update_bias=False, gather_rows=False, fuse_shared=False)
         self.w1, self.w3, self.w2 = (weights[n][lo:hi].contiguous() for n in ("w1", "w3", "w2"))
         self.update_bias = update_bias and weights.get("bias") is not None
         self.recv_cap = max(int(math.ceil(recv_factor * w.T * w.k)), w.T, 1)

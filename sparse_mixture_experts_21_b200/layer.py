@@ -35,7 +35,8 @@ class MoELayer:
     """Holds the weights and the per-call buffers of one layer for up to T tokens."""
 
     def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True,
-                 group=None, overlap_shared: bool = True, gather_rows: bool = False):
+                 group=None, overlap_shared: bool = True, gather_rows: bool = False,
+                 fuse_shared: bool = True):
         """group: a torch.distributed process group when the layer runs as one of
         several data-parallel replicas; the router statistics are then those of the
         whole group's batch (each rank's sufficient statistics summed over the
@@ -55,6 +56,13 @@ class MoELayer:
         # memory); off by default: the gathering copies are slower than the copy they save
         self.gather_rows = (gather_rows and w.dtype == "bf16" and w.d % 64 == 0
                             and not (w.fp8 or w.mxfp8 or w.expert_choice))
+        # fuse_shared: a bf16 shared expert of the routed experts' width runs as one more
+        # group inside the routed grouped-FFN launches (moe_grouped_ffn_shared); its rows
+        # follow the routed rows in h and y_perm
+        self.fuse_shared = (fuse_shared and w.dtype == "bf16" and not (w.fp8 or w.mxfp8 or w.expert_choice)
+                            and not self.gather_rows and w.n_shared * w.f_shared == w.f and w.N < 512)
+        if self.fuse_shared:
+            self.overlap_shared = False
         self.dev = torch.device(device)
         self.weights = weights
         self.update_bias = update_bias and weights.get("bias") is not None
@@ -80,13 +88,17 @@ class MoELayer:
         if L.route_prepare_size(self.cfg) > 0 and not w.expert_choice:
             self.route_split = z(L.route_prepare_size(self.cfg), dtype=torch.uint8)
             self.prepare_router()
-        self.h = z(max(T * k, 1), w.f, dtype=dt)
-        self.y_perm = z(max(T * k, 1), d, dtype=dt)
         self.fs = w.n_shared * w.f_shared
+        extra = T if self.fuse_shared else 0         # the fused shared expert's rows
+        self.h = z(max(T * k + extra, 1), w.f, dtype=dt)
+        self.y_perm = z(max(T * k + extra, 1), d, dtype=dt)
         if self.fs > 0:
             self.shared_offsets = torch.tensor([0, T], dtype=torch.int32, device=self.dev)
-            self.hs = z(max(T, 1), self.fs, dtype=dt)
-            self.ys = z(max(T, 1), d, dtype=dt)
+            if self.fuse_shared:
+                self.hs, self.ys = self.h[T * k:], self.y_perm[T * k:]
+            else:
+                self.hs = z(max(T, 1), self.fs, dtype=dt)
+                self.ys = z(max(T, 1), d, dtype=dt)
         self.y = z(max(T, 1), d, dtype=dt)
         if w.fp8 or w.mxfp8:
             self._init_fp8(z)
@@ -201,6 +213,9 @@ class MoELayer:
         if fp8:
             self._ffn_fp8(c, self.xq_perm, self.xs_perm, T * self.w.k, self.offsets, self.w.N,
                           ("w1", "w3", "w2"), self.w.f, self.hq, self.hsc, self.y_perm, s)
+        elif self.fuse_shared:
+            L.moe_grouped_ffn_shared(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
+                                     W["w2"], self.w.f, self.h, self.y_perm, x, T, W["ws1"], W["ws3"], W["ws2"], s)
         elif self.gather_rows:
             L.moe_grouped_ffn_gather(c, x, T, self.token_of_row, T * self.w.k, self.offsets, self.w.N, W["w1"],
                                      W["w3"], W["w2"], self.w.f, self.h, self.y_perm, s)
@@ -212,6 +227,8 @@ class MoELayer:
         if self.fs > 0:
             if join is not None:
                 s.wait_event(join)
+            elif self.fuse_shared:
+                pass                   # computed with the routed experts
             elif fp8:
                 self._ffn_fp8(c, self.xq, self.xs, T, self.shared_offsets, 1, ("ws1", "ws3", "ws2"),
                               self.fs, self.hq_sh, self.hsc_sh, self.ys, s)
@@ -343,7 +360,7 @@ class MoELayer:
         # the router weight's split is written once, outside the forward
         if self.gather_rows:
             n -= 1                     # no row gather: the grouped FFN reads x itself
-        if self.fs > 0:
+        if self.fs > 0 and not self.fuse_shared:
             n += 2
         if self.update_bias:
             n += 1

@@ -152,6 +152,33 @@ def test_gathering_ffn_checks(lib):
     assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == UN
 
 
+def test_fused_shared_ffn_checks(lib):
+    """moe_grouped_ffn_shared: bf16 only, G <= 511, every buffer present and aligned;
+    no shared rows is moe_grouped_ffn.  Nothing here reaches the GPU."""
+    ok, UN, IA = 0x1000000, L.MOE_ERR_UNSUPPORTED, L.MOE_ERR_INVALID_ARG
+    c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    cp = ctypes.byref(c)
+    f = lib.moe_grouped_ffn_shared
+    good = [ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, ok, 100, ok, ok, ok, None]
+    def call(**kw):
+        a = list(good)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(cp, *a)
+    assert call(a3=512) == IA                       # G: one slot is the shared group
+    assert call(a3=0) == IA
+    assert call(a11=-1) == IA                       # T
+    assert call(a12=None) == IA                     # ws1
+    assert call(a10=ok + 4) == IA                   # x misaligned
+    assert call(a8=None) == IA                      # h_scratch
+    assert call(a1=(1 << 31) - 50) == UN            # rows_cap + T past INT32_MAX
+    assert call(a7=2047) == IA                      # f % 8
+    c32 = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    assert f(ctypes.byref(c32), *good) == UN
+    # T = 0 with nothing to do: the plain grouped FFN's no-op
+    assert f(cp, None, 0, ok, 1, None, None, None, 256, None, None, None, 0, None, None, None, None) == L.MOE_OK
+
+
 def test_route_prepare_checks(lib):
     ok = 0x1000000
     c = layer.make_config(synth.WORKLOADS["deepseek_v3"])

@@ -419,6 +419,65 @@ def test_grouped_ffn_empty_and_tiny_groups(d, f, sizes):
     assert torch.all(y[R:] == 3.0)                     # rows past the last group untouched
 
 
+@pytest.mark.parametrize("d,f,sizes,Ts,gap", [
+    (256, 384, [0, 1, 127, 0, 128, 129, 300, 0], 300, 70),
+    (384, 320, [16, 17, 112, 113, 255, 256, 257, 383, 384, 385, 511, 640, 5, 0, 31], 513, 0),
+    (256, 256, [0, 0, 0], 129, 5),                       # no routed rows at all
+    (256, 256, [40, 200], 16, 1),                        # shared rows: a tail alone
+])
+def test_grouped_ffn_shared_equals_separate_calls(d, f, sizes, Ts, gap):
+    """moe_grouped_ffn_shared (the shared expert as one more group of the same two
+    launches) gives bit for bit moe_grouped_ffn on the routed groups plus
+    moe_grouped_ffn with G = 1 over x; the shared rows follow the routed rows_cap
+    rows, and rows between the last group and rows_cap stay untouched."""
+    G = len(sizes)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    R = int(off[-1])
+    cap = R + gap
+    g = torch.Generator(device="cuda").manual_seed(5)
+    xr = torch.randn(max(cap, 1), d, generator=g, device="cuda").to(torch.bfloat16)
+    x = torch.randn(Ts, d, generator=g, device="cuda").to(torch.bfloat16)
+    mk = lambda *s, sc: (torch.randn(*s, generator=g, device="cuda") * sc).to(torch.bfloat16)  # noqa: E731
+    w1, w3, w2 = mk(G, f, d, sc=d ** -0.5), mk(G, f, d, sc=d ** -0.5), mk(G, d, f, sc=f ** -0.5)
+    ws1, ws3, ws2 = mk(f, d, sc=d ** -0.5), mk(f, d, sc=d ** -0.5), mk(d, f, sc=f ** -0.5)
+    offs = torch.tensor(off, device="cuda")
+    cfg = make_config(replace(SMALL["mixtral_small"], d=d, f=f, N=G, T=Ts))
+    h = torch.full((cap + Ts, f), 7.0, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((cap + Ts, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    L.moe_device_status()
+    L.moe_grouped_ffn_shared(cfg, xr, cap, offs, G, w1, w3, w2, f, h, y, x, Ts, ws1, ws3, ws2)
+    h0 = torch.empty(max(cap, 1), f, dtype=torch.bfloat16, device="cuda")
+    y0 = torch.empty(max(cap, 1), d, dtype=torch.bfloat16, device="cuda")
+    if cap > 0:
+        L.moe_grouped_ffn(cfg, xr, cap, offs, G, w1, w3, w2, f, h0, y0)
+    hs = torch.empty(Ts, f, dtype=torch.bfloat16, device="cuda")
+    ys = torch.empty(Ts, d, dtype=torch.bfloat16, device="cuda")
+    L.moe_grouped_ffn(cfg, x, Ts, torch.tensor([0, Ts], dtype=torch.int32, device="cuda"), 1, ws1, ws3, ws2, f,
+                      hs, ys)
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(h[:R], h0[:R]) and torch.equal(y[:R], y0[:R])
+    assert torch.equal(h[cap:], hs) and torch.equal(y[cap:], ys)
+    assert torch.all(y[R:cap] == 3.0)
+
+
+@pytest.mark.parametrize("name", ["v3_small"])
+def test_layer_fused_shared_expert_equals_separate(name):
+    """The layer's output is bit-identical with the shared expert fused into the
+    routed launches and with it in launches of its own."""
+    w = SMALL[name]
+    inp = make_inputs(w, "cuda")
+    a = MoELayer(w, inp, "cuda", update_bias=False, fuse_shared=False, overlap_shared=False)
+    b = MoELayer(w, inp, "cuda", update_bias=False, fuse_shared=True)
+    assert b.fuse_shared and not a.fuse_shared
+    ya = a.forward(inp["x"]).clone()
+    yb = b.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(ya, yb)
+    assert torch.equal(a.ys[:w.T], b.ys[:w.T])
+
+
 @pytest.mark.parametrize("d,f,sizes", [
     (256, 384, [0, 1, 127, 0, 128, 129, 300, 0]),
     (384, 320, [16, 17, 112, 113, 255, 256, 257, 383, 384, 385, 511, 640, 5, 0, 31]),
