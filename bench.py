@@ -40,6 +40,10 @@ UNIT = "tokens/s"
 # dram__bytes_read.sum, dram__bytes_write.sum, gpu__time_duration.sum; valid only
 # while every listed kernel source is the one that was profiled (sha1), else null.
 NCU_TRAFFIC = {
+    # reduced case (T = 4096, 64 experts, shared expert in launches of its own), scaled to
+    # the full layer: routed bytes x 4, the shared expert's rows x 4 plus its 88 MB of
+    # weights once; profiles/ffn_deepseek_v3_reduced.md
+    "deepseek_v3": ({"ffn_tc.cu": "454b3a2c199fd06c22d7bd11968154aa96b151b5"}, 28.6e9),
     "deepseek_v3_mxfp8": ({"ffn_mx.cu": "709e9d80185da2b81c3d48f20340d1eabb0fd4e9"}, 15.07e9),
 }
 
@@ -145,7 +149,8 @@ def run_reference(args, rank):
     f64 = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
     wg, bias, off = f64(inp["w_gate"]), f64(inp["bias"]), f64(inp["logit_offset"])
     shared = (f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"])) if w.n_shared else None
-    ffn = O.swiglu_ffn_fp8 if w.fp8 else (O.swiglu_ffn_mxfp8 if w.mxfp8 else None)
+    ffn = (O.swiglu_ffn_fp8 if w.fp8 else O.swiglu_ffn_mxfp8 if w.mxfp8 else
+           O.swiglu_ffn_nvfp4 if w.nvfp4 else None)
 
     def experts(e):
         return f64(inp["w1"][e]), f64(inp["w3"][e]), f64(inp["w2"][e])
@@ -191,7 +196,8 @@ def cpu_baseline(inp, w, seconds_target=20.0, chunk=4, max_tokens=64, threads=No
     f64 = lambda t: None if t is None else t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
     wg, bias, off = f64(inp["w_gate"]), f64(inp["bias"]), f64(inp["logit_offset"])
     shared = (f64(inp["ws1"]), f64(inp["ws3"]), f64(inp["ws2"])) if w.n_shared else None
-    ffn = O.swiglu_ffn_fp8 if w.fp8 else (O.swiglu_ffn_mxfp8 if w.mxfp8 else None)
+    ffn = (O.swiglu_ffn_fp8 if w.fp8 else O.swiglu_ffn_mxfp8 if w.mxfp8 else
+           O.swiglu_ffn_nvfp4 if w.nvfp4 else None)
 
     def experts(e):
         return f64(inp["w1"][e]), f64(inp["w3"][e]), f64(inp["w2"][e])
@@ -449,18 +455,21 @@ def main():
     if lay.gather_rows:        # no row gather: index maps only (the grouped FFN reads x itself)
         bytes_perm = 12 * T * k
     bytes_comb = R * d * eb + 2 * T * d * eb + 8 * T * k
-    lowp = w.fp8 or w.mxfp8
-    if lowp:                   # bf16 x read once; E4M3 codes + scales written per row (+ token order)
-        sf_per_elem = 4 / 128 if w.fp8 else 1 / 32
-        bytes_perm = T * d * eb + (R + (T if lay.fs else 0)) * d * (1 + sf_per_elem) + 12 * T * k
+    lowp = w.fp8 or w.mxfp8 or w.nvfp4
+    if lowp:                   # bf16 x read once; codes + scales written per row (+ token order)
+        per_elem = 0.5 + 1 / 16 if w.nvfp4 else 1 + (4 / 128 if w.fp8 else 1 / 32)
+        bytes_perm = T * d * eb + (R + (T if lay.fs else 0)) * d * per_elem + 12 * T * k
     if w.expert_choice:        # scores [N, T] written; rows gathered per row; combine reads the maps
         bytes_route = T * d * eb + 4 * N * d + 4 * N * T
         bytes_perm = 2 * R * d * eb + 12 * N * T
         bytes_comb = R * d * eb + 2 * T * d * eb + 8 * N * T
     peaks = _peaks()
-    # E4M3 operands: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
-    ffn_peak = peaks["bf16_tflops_sustained"] * (2.0 if lowp else 1.0)
-    ffn_peak_src = peaks["source"] + (" sustained bf16 x 2 (nominal fp8/bf16 ratio)" if lowp else " sustained bf16")
+    # E4M3 operands: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25);
+    # E2M1 operands: times the nominal fp4 / bf16 ratio (9 / 2.25)
+    ratio = 4.0 if w.nvfp4 else 2.0 if lowp else 1.0
+    ffn_peak = peaks["bf16_tflops_sustained"] * ratio
+    ffn_peak_src = peaks["source"] + (" sustained bf16 x 4 (nominal fp4/bf16 ratio)" if w.nvfp4 else
+                                      " sustained bf16 x 2 (nominal fp8/bf16 ratio)" if lowp else " sustained bf16")
     ffn_bound = "tensor"
     if w.dtype == "fp32":
         # fp32 experts run on the FMA pipes: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
@@ -522,7 +531,8 @@ def main():
         line = {
             "metric": METRIC, "value": world * T / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": ("mxfp8-e4m3 experts, fp32 router" if w.mxfp8 else
+            "scaling": "weak", "vs_baseline": None, "dtype": ("nvfp4-e2m1 experts, fp32 router" if w.nvfp4 else
+                                                              "mxfp8-e4m3 experts, fp32 router" if w.mxfp8 else
                                                               "fp8-e4m3 experts, fp32 router" if w.fp8 else
                                                               "fp32" if w.dtype == "fp32" else "bf16"),
             "data": "synthetic",
@@ -535,9 +545,11 @@ def main():
                        "expert_rows": ("read from x by the first grouped GEMM (TMA gather4)" if lay.gather_rows
                                        else "expert-ordered copy of x written by the permutation"),
                        "experts_precision": ("E4M3, 1x128 / 128x128 block scales" if w.fp8 else
-                                             "MXFP8: E4M3, E8M0 scale per 32 along K" if w.mxfp8 else "bf16"),
+                                             "MXFP8: E4M3, E8M0 scale per 32 along K" if w.mxfp8 else
+                                             "NVFP4: E2M1, E4M3 scale per 16 along K, fp32 per expert matrix"
+                                             if w.nvfp4 else "bf16"),
                        "l2": (f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "
-                              f"{3 * N * d * f * (1 if lowp else eb) / 1e9:.1f} GB); no flush")},
+                              f"{3 * N * d * f * (0.5 if w.nvfp4 else 1 if lowp else eb) / 1e9:.1f} GB); no flush")},
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
             "roofline": {"kernel": ("grouped SwiGLU FFN, routed + shared experts in one tile list (gate/up + "
                                     "down passes)" if lay.fuse_shared else

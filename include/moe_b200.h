@@ -403,6 +403,69 @@ int moe_grouped_ffn_mxfp8(const moe_config_t* cfg, const uint8_t* xq_rows, const
                           void* y_rows, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * NVFP4 expert compute.
+ *
+ * Defines: the MoE common-taste page, section 2 (its table names NVFP4 beside FP8 /
+ * MXFP8 expert compute, without the scheme).  Reading (NVIDIA's two-level NVFP4):
+ * E2M1 codes (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), one unsigned E4M3 scale b per
+ * 16 consecutive elements of a row (the GEMM's contraction dimension) and one fp32
+ * scale g per tensor.  In fp32, in this order: b = E4M3(amax_16 / fp32(6 g)) (round
+ * to nearest even, saturating at 448), s = fp32(b g), code = E2M1(fp32(x / s)) (round
+ * to nearest even, saturating at 6); b = 0 gives zero codes.  Weights take
+ * g = amax / (6 * 448) per expert matrix; activations (x rows, h) take g = 1.
+ * Codes are packed two per byte, element 2i in the low nibble: a [rows, cols] matrix
+ * takes rows * cols / 2 bytes.  Scales are stored as tile atoms: rows cut into tiles
+ * of 128 (per group for grouped rows: tile i of group g starts at offsets[g] + 128 i,
+ * tiles numbered in group order); the 512-byte atom of tile t and 64-wide K chunk c
+ * sits at (t * (cols / 64) + c) * 512 and holds scale j (elements 64 c + 16 j ..
+ * 64 c + 16 j + 15) of the tile's row m at byte 16 (m % 32) + 4 (m / 32) + j.  A
+ * buffer for R rows in G groups takes (ceil(R / 128) + G) * (cols / 64) * 512 bytes.
+ * The tensor cores apply the E4M3 block scales inside the MMA
+ * (tcgen05.mma.kind::mxf4nvf4.block_scale.scale_vec::4X); the epilogue multiplies by
+ * the weights' tensor scales.
+ * ------------------------------------------------------------------------- */
+
+/* moe_quantize_nvfp4 -- quantise a bf16 matrix along its rows.
+ *   x            [rows, cols] bf16 (device, 16-byte aligned), cols % 64 == 0
+ *   tensor_rows  0: tensor scale 1 (activations); else rows per tensor (rows %
+ *                tensor_rows == 0), each tensor's g = amax / (6 * 448) written to g
+ *   q            [rows, cols / 2] uint8 out (4-byte aligned); sf tile atoms out
+ *   g            [rows / tensor_rows] fp32 out (unused when tensor_rows == 0)
+ * Errors: MOE_ERR_INVALID_ARG for a bad shape or a NULL or misaligned pointer. */
+int moe_quantize_nvfp4(const void* x, int64_t rows, int32_t cols, int32_t tensor_rows, uint8_t* q, uint8_t* sf,
+                       float* g, void* stream);
+
+/* moe_permute_nvfp4 -- moe_permute_mxfp8 with NVFP4 rows (tensor scale 1): each
+ * token's row is read and quantised once and written to every kept row it has
+ * (row_of_slot from moe_permute, called with x_perm = NULL), and, when q is not
+ * NULL, to row t of token-order buffers (the shared experts' input).
+ *   q_perm [rows, d / 2], sf_perm tile atoms of the grouped rows (groups: offsets)
+ *   q [T, d / 2], sf tile atoms of the T token rows (one group)
+ * Errors: MOE_ERR_UNSUPPORTED unless bf16 with d % 256 == 0 and N <= 1024;
+ * MOE_ERR_INVALID_ARG for missing or misaligned buffers. */
+int moe_permute_nvfp4(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const int32_t* row_of_slot,
+                      const int32_t* offsets, uint8_t* q_perm, uint8_t* sf_perm, uint8_t* q, uint8_t* sf,
+                      void* stream);
+
+/* moe_grouped_ffn_nvfp4 -- the grouped SwiGLU FFN of moe_grouped_ffn on NVFP4 operands.
+ *   xq_rows, xsf_rows  [rows_cap, d / 2] codes, grouped tile atoms (tensor scale 1)
+ *   offsets            [G+1] int32 (device), as for moe_grouped_ffn
+ *   w1q/w1sf/g1, w3q/w3sf/g3  [G f, d / 2] codes, atoms, [G] tensor scales
+ *   w2q/w2sf/g2        [G d, f / 2] codes, atoms, [G] tensor scales
+ *   hq/hsf_scratch     [rows_cap, f / 2] codes and grouped atoms of h (written, read)
+ *   y_rows             [rows_cap, d] bf16 out (rows >= offsets[G] untouched)
+ * Tensor cores (E2M1 x E2M1, fp32 accumulation, E4M3 scales applied per 16 elements
+ * inside the MMA); h = silu(g1 W1 x) * (g3 W3 x) in fp32, re-quantised with tensor
+ * scale 1; y = g2 (W2 h).
+ * Errors: MOE_ERR_UNSUPPORTED unless bf16 with d % 256 == 0 and f % 256 == 0;
+ * MOE_ERR_INVALID_ARG for G outside [1, 512] or NULL or misaligned buffers. */
+int moe_grouped_ffn_nvfp4(const moe_config_t* cfg, const uint8_t* xq_rows, const uint8_t* xsf_rows,
+                          int64_t rows_cap, const int32_t* offsets, int32_t G, const uint8_t* w1q,
+                          const uint8_t* w1sf, const float* g1, const uint8_t* w3q, const uint8_t* w3sf,
+                          const float* g3, const uint8_t* w2q, const uint8_t* w2sf, const float* g2, int32_t f,
+                          uint8_t* hq_scratch, uint8_t* hsf_scratch, void* y_rows, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Expert parallelism: the data path around the all-to-all exchange.
  *
  * Defines: the Practice page, "专家并行与 all-to-all": experts are sharded over W

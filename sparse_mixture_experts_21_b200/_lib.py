@@ -28,7 +28,8 @@ EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_rou
             "moe_device_status", "moe_status_string", "moe_permute_noalloc", "moe_bias_update_ema",
             "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec",
             "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
-            "moe_quantize_mxfp8", "moe_permute_mxfp8", "moe_grouped_ffn_mxfp8", "moe_ep_plan",
+            "moe_quantize_mxfp8", "moe_permute_mxfp8", "moe_grouped_ffn_mxfp8", "moe_quantize_nvfp4",
+            "moe_permute_nvfp4", "moe_grouped_ffn_nvfp4", "moe_ep_plan",
             "moe_rows_move", "moe_router_stats_partial", "moe_router_stats_finalize",
             "moe_expert_choice_capacity", "moe_route_prepare_size", "moe_route_prepare",
             "moe_last_cuda_error", "moe_last_cuda_error_string")
@@ -120,6 +121,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_permute_mxfp8": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "moe_grouped_ffn_mxfp8": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, c_int32, vp, vp,
                                   vp, vp],
+        "moe_quantize_nvfp4": [vp, c_int64, c_int32, c_int32, vp, vp, vp, vp],
+        "moe_permute_nvfp4": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "moe_grouped_ffn_nvfp4": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, vp, vp, vp, c_int32,
+                                  vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -281,6 +286,36 @@ def moe_grouped_ffn_mxfp8(cfg, xq_rows, xsf_rows, rows_cap, offsets, G, w1q, w1s
         ctypes.byref(cfg), _ptr(xq_rows), _ptr(xsf_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1q),
         _ptr(w1sf), _ptr(w3q), _ptr(w3sf), _ptr(w2q), _ptr(w2sf), int(f), _ptr(hq_scratch), _ptr(hsf_scratch),
         _ptr(y_rows), _stream(stream)))
+
+
+def nv_scales(rows: int, cols: int, device, groups: int = 0) -> torch.Tensor:
+    """Buffer for NVFP4 scales in tile-atom order: rows cut into 128-row tiles (per group
+    when `groups` > 0), one 512-byte atom per (tile, 64-wide K chunk)."""
+    tiles = (rows + 127) // 128 + groups
+    return torch.empty(max(tiles, 1) * (cols // 64) * 512, dtype=torch.uint8, device=device)
+
+
+def moe_quantize_nvfp4(x, q, sf, g=None, tensor_rows=0, stream=None):
+    """NVFP4-quantise a bf16 matrix [rows, cols] along its rows: packed E2M1 codes
+    (q: rows x cols / 2 bytes), E4M3 block scales (sf from nv_scales(rows, cols)) and,
+    with tensor_rows > 0, one tensor scale per tensor_rows rows into g."""
+    rows, cols = x.shape
+    _check("moe_quantize_nvfp4", load().moe_quantize_nvfp4(
+        _ptr(x), int(rows), int(cols), int(tensor_rows), _ptr(q), _ptr(sf), _ptr(g), _stream(stream)))
+
+
+def moe_permute_nvfp4(cfg, x, topk_idx, row_of_slot, offsets, q_perm, sf_perm, q=None, sf=None, stream=None):
+    _check("moe_permute_nvfp4", load().moe_permute_nvfp4(
+        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(row_of_slot), _ptr(offsets), _ptr(q_perm),
+        _ptr(sf_perm), _ptr(q), _ptr(sf), _stream(stream)))
+
+
+def moe_grouped_ffn_nvfp4(cfg, xq_rows, xsf_rows, rows_cap, offsets, G, w1q, w1sf, g1, w3q, w3sf, g3, w2q, w2sf,
+                          g2, f, hq_scratch, hsf_scratch, y_rows, stream=None):
+    _check("moe_grouped_ffn_nvfp4", load().moe_grouped_ffn_nvfp4(
+        ctypes.byref(cfg), _ptr(xq_rows), _ptr(xsf_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1q),
+        _ptr(w1sf), _ptr(g1), _ptr(w3q), _ptr(w3sf), _ptr(g3), _ptr(w2q), _ptr(w2sf), _ptr(g2), int(f),
+        _ptr(hq_scratch), _ptr(hsf_scratch), _ptr(y_rows), _stream(stream)))
 
 
 def moe_ep_plan(offsets_all, world, rank, send_splits, recv_splits, local_offsets, regroup_map, stream=None):

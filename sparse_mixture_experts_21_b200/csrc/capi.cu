@@ -364,6 +364,64 @@ int moe_grouped_ffn_mxfp8(const moe_config_t* cfg, const uint8_t* xq_rows, const
                                  static_cast<cudaStream_t>(stream)));
 }
 
+int moe_quantize_nvfp4(const void* x, int64_t rows, int32_t cols, int32_t tensor_rows, uint8_t* q, uint8_t* sf,
+                       float* g, void* stream) {
+  if (rows < 0 || cols <= 0 || (cols % 64) != 0 || tensor_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (tensor_rows > 0 && (rows % tensor_rows) != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (rows * (int64_t)cols / 8 > ((int64_t)1 << 40)) return MOE_ERR_UNSUPPORTED;
+  if (!x || !q || !sf || !aligned16(x) || (reinterpret_cast<uintptr_t>(q) & 3u)) return MOE_ERR_INVALID_ARG;
+  if (tensor_rows > 0 && (!g || (reinterpret_cast<uintptr_t>(g) & 3u))) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_nv_quant_rows(x, rows, cols, tensor_rows, q, sf, tensor_rows > 0 ? g : nullptr,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int moe_permute_nvfp4(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const int32_t* row_of_slot,
+                      const int32_t* offsets, uint8_t* q_perm, uint8_t* sf_perm, uint8_t* q, uint8_t* sf,
+                      void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->x_dtype != MOE_DTYPE_BF16 || (cfg->d_model % 256) != 0 || cfg->n_experts > 1024)
+    return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !aligned16(x)) return MOE_ERR_INVALID_ARG;
+  if (row_of_slot && (!q_perm || !sf_perm || !topk_idx || !offsets)) return MOE_ERR_INVALID_ARG;
+  if (!row_of_slot && !q) return MOE_ERR_INVALID_ARG;
+  if ((q && !sf) || (q_perm && !aligned16(q_perm)) || (q && !aligned16(q))) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_nv_quant_scatter(x, cfg->T, row_of_slot ? cfg->top_k : 0, cfg->d_model,
+                                           cfg->n_experts, topk_idx, row_of_slot, offsets, q_perm, sf_perm, q,
+                                           sf, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_grouped_ffn_nvfp4(const moe_config_t* cfg, const uint8_t* xq_rows, const uint8_t* xsf_rows,
+                          int64_t rows_cap, const int32_t* offsets, int32_t G, const uint8_t* w1q,
+                          const uint8_t* w1sf, const float* g1, const uint8_t* w3q, const uint8_t* w3sf,
+                          const float* g3, const uint8_t* w2q, const uint8_t* w2sf, const float* g2, int32_t f,
+                          uint8_t* hq_scratch, uint8_t* hsf_scratch, void* y_rows, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (rows_cap < 0 || G < 1 || G > 512 || f <= 0) return MOE_ERR_INVALID_ARG;
+  if (cfg->x_dtype != MOE_DTYPE_BF16 || (cfg->d_model % 256) != 0 || (f % 256) != 0) return MOE_ERR_UNSUPPORTED;
+  if (!offsets) return MOE_ERR_INVALID_ARG;
+  if (rows_cap == 0) return MOE_OK;
+  if (rows_cap > (int64_t)INT32_MAX || (int64_t)G * cfg->d_model > (int64_t)INT32_MAX ||
+      (int64_t)G * f > (int64_t)INT32_MAX)
+    return MOE_ERR_UNSUPPORTED;
+  if (!xq_rows || !xsf_rows || !w1q || !w1sf || !g1 || !w3q || !w3sf || !g3 || !w2q || !w2sf || !g2 ||
+      !hq_scratch || !hsf_scratch || !y_rows)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq_rows) || !aligned16(w1q) || !aligned16(w3q) || !aligned16(w2q) || !aligned16(hq_scratch) ||
+      !aligned16(y_rows))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xsf_rows) || !aligned16(w1sf) || !aligned16(w3sf) || !aligned16(w2sf) || !aligned16(hsf_scratch))
+    return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(g1) | reinterpret_cast<uintptr_t>(g3) | reinterpret_cast<uintptr_t>(g2)) & 3u)
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_ffn_nv(xq_rows, xsf_rows, rows_cap, offsets, G, w1q, w1sf, g1, w3q, w3sf, g3, w2q, w2sf,
+                                 g2, cfg->d_model, f, hq_scratch, hsf_scratch, y_rows,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
 int moe_ep_plan(const int32_t* offsets_all, int32_t world, int32_t rank, int32_t n_experts, int32_t* send_splits,
                 int32_t* recv_splits, int32_t* local_offsets, int32_t* regroup_map, int64_t recv_cap, void* stream) {
   if (world < 1 || n_experts < 1 || rank < 0 || rank >= world || (n_experts % world) != 0 || recv_cap < 0)

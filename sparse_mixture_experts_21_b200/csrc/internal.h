@@ -103,6 +103,15 @@ cudaError_t launch_ffn_mx(const uint8_t* xq, const uint8_t* xsf, int64_t rows_ca
                           const uint8_t* w1q, const uint8_t* w1sf, const uint8_t* w3q, const uint8_t* w3sf,
                           const uint8_t* w2q, const uint8_t* w2sf, int d, int f, uint8_t* hq, uint8_t* hsf,
                           void* y, cudaStream_t s);
+cudaError_t launch_nv_quant_rows(const void* x, int64_t rows, int cols, int tensor_rows, uint8_t* q, uint8_t* sf,
+                                 float* g, cudaStream_t s);
+cudaError_t launch_nv_quant_scatter(const void* x, int64_t T, int k, int d, int N, const int32_t* topk_idx,
+                                    const int32_t* row_of_slot, const int32_t* offsets, uint8_t* q_perm,
+                                    uint8_t* sf_perm, uint8_t* q_tok, uint8_t* sf_tok, cudaStream_t s);
+cudaError_t launch_ffn_nv(const uint8_t* xq, const uint8_t* xsf, int64_t rows_cap, const int32_t* offsets, int G,
+                          const uint8_t* w1q, const uint8_t* w1sf, const float* g1, const uint8_t* w3q,
+                          const uint8_t* w3sf, const float* g3, const uint8_t* w2q, const uint8_t* w2sf,
+                          const float* g2, int d, int f, uint8_t* hq, uint8_t* hsf, void* y, cudaStream_t s);
 cudaError_t launch_ep_plan(const int32_t* offsets_all, int W, int rank, int N, int32_t* send_splits,
                            int32_t* recv_splits, int32_t* local_offsets, int32_t* regroup_map, int64_t recv_cap,
                            cudaStream_t s);

@@ -168,7 +168,7 @@ class EPMoELayer:
                  exchange=None, update_bias: bool = True, recv_factor: float = 1.0):
         if w.N % world != 0:
             raise ValueError(f"{w.N} experts do not divide over {world} ranks")
-        if w.fp8 or w.mxfp8 or w.expert_choice or w.dtype != "bf16":
+        if w.fp8 or w.mxfp8 or w.nvfp4 or w.expert_choice or w.dtype != "bf16":
             raise ValueError("the expert-parallel layer runs bf16 token-choice routing")
         if not recv_factor > 0:
             raise ValueError("recv_factor must be positive")

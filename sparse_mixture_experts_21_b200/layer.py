@@ -42,24 +42,27 @@ class MoELayer:
         whole group's batch (each rank's sufficient statistics summed over the
         group) and the bias update uses the counts summed over the group, so all
         replicas keep the same selection bias."""
-        if w.expert_choice and (w.fp8 or w.mxfp8):
+        lowp = w.fp8 or w.mxfp8 or w.nvfp4
+        if w.expert_choice and lowp:
             raise ValueError("expert-choice routing runs bf16 or fp32 experts")
-        if (w.fp8 or w.mxfp8) and (w.dtype != "bf16" or w.d % 128 or w.f % 128 or w.f_shared % 128):
+        if lowp and (w.dtype != "bf16" or w.d % 128 or w.f % 128 or w.f_shared % 128):
             raise ValueError("FP8 experts need bf16 inputs and d, d_ff multiples of 128")
+        if w.nvfp4 and (w.d % 256 or w.f % 256 or (w.n_shared * w.f_shared) % 256):
+            raise ValueError("NVFP4 experts need d and d_ff multiples of 256")
         self.w = w
         self.group = group
         # bf16 shared experts on a side stream, concurrently with route and permute (they
         # do not depend on the routing); joined before the combine
-        self.overlap_shared = overlap_shared and not (w.fp8 or w.mxfp8) and w.n_shared > 0
+        self.overlap_shared = overlap_shared and not lowp and w.n_shared > 0
         # gather_rows: bf16 experts read their rows straight from x (moe_grouped_ffn_gather),
         # so the permutation writes no expert-ordered copy of x (T k d elements less
         # memory); off by default: the gathering copies are slower than the copy they save
         self.gather_rows = (gather_rows and w.dtype == "bf16" and w.d % 64 == 0
-                            and not (w.fp8 or w.mxfp8 or w.expert_choice))
+                            and not (lowp or w.expert_choice))
         # fuse_shared: a bf16 shared expert of the routed experts' width runs as one more
         # group inside the routed grouped-FFN launches (moe_grouped_ffn_shared); its rows
         # follow the routed rows in h and y_perm
-        self.fuse_shared = (fuse_shared and w.dtype == "bf16" and not (w.fp8 or w.mxfp8 or w.expert_choice)
+        self.fuse_shared = (fuse_shared and w.dtype == "bf16" and not (lowp or w.expert_choice)
                             and not self.gather_rows and w.n_shared * w.f_shared == w.f and w.N < 512)
         if self.fuse_shared:
             self.overlap_shared = False
@@ -100,7 +103,7 @@ class MoELayer:
                 self.hs = z(max(T, 1), self.fs, dtype=dt)
                 self.ys = z(max(T, 1), d, dtype=dt)
         self.y = z(max(T, 1), d, dtype=dt)
-        if w.fp8 or w.mxfp8:
+        if lowp:
             self._init_fp8(z)
         self.stats = torch.zeros(L.STATS_BYTES, dtype=torch.uint8, device=self.dev)
         self.counts_global = z(N, dtype=torch.int32)
@@ -135,20 +138,32 @@ class MoELayer:
                     self.p_partial, self.margin, ws, stream, shared_w=self.shared_w)
 
     def _init_fp8(self, z):
-        """FP8 experts: quantise the weights once (fine-grained: 128 x 128 blocks with
-        fp32 scales; MXFP8: 1 x 32 blocks along K with E8M0 scales) and hold E4M3
-        buffers for the permuted rows, the hidden rows and the shared experts' input
-        in place of the bf16 ones."""
+        """Low-precision experts: quantise the weights once (fine-grained FP8: 128 x 128
+        blocks with fp32 scales; MXFP8: 1 x 32 blocks along K with E8M0 scales; NVFP4:
+        1 x 16 blocks along K with E4M3 scales and one fp32 scale per expert matrix) and
+        hold code buffers for the permuted rows, the hidden rows and the shared experts'
+        input in place of the bf16 ones."""
         w, W, T, d, N, k = self.w, self.weights, self.w.T, self.w.d, self.w.N, self.w.k
         u8 = torch.uint8
-        mx = w.mxfp8
-        # scales of grouped (permuted) rows: MXFP8 tile atoms need one spare tile per group
-        sfa = (lambda rows, cols, groups=0: L.mx_scales(rows, cols, self.dev, groups)) if mx else \
-            (lambda rows, cols, groups=0: z(rows, cols // 128))
+        mx, nv = w.mxfp8, w.nvfp4
+        # scales of grouped (permuted) rows: tile atoms need one spare tile per group
+        if nv:
+            sfa = lambda rows, cols, groups=0: L.nv_scales(rows, cols, self.dev, groups)  # noqa: E731
+        elif mx:
+            sfa = lambda rows, cols, groups=0: L.mx_scales(rows, cols, self.dev, groups)  # noqa: E731
+        else:
+            sfa = lambda rows, cols, groups=0: z(rows, cols // 128)  # noqa: E731
+        cw = (lambda cols: cols // 2) if nv else (lambda cols: cols)     # code bytes per row
 
         def quant_w(t):
             m = t.reshape(-1, t.shape[-1])
-            q = z(m.shape[0], m.shape[1], dtype=u8)
+            q = z(m.shape[0], cw(m.shape[1]), dtype=u8)
+            if nv:
+                # one tensor scale per expert matrix (t is [experts, rows, cols] or one matrix)
+                per = t.shape[-2]
+                sc, g = L.nv_scales(m.shape[0], m.shape[1], self.dev), z(m.shape[0] // per)
+                L.moe_quantize_nvfp4(m, q, sc, g, tensor_rows=per)
+                return q, sc, g
             if mx:
                 sc = L.mx_scales(m.shape[0], m.shape[1], self.dev)
                 L.moe_quantize_mxfp8(m, q, sc)
@@ -160,18 +175,21 @@ class MoELayer:
         self.wq = {name: quant_w(W[name]) for name in ("w1", "w3", "w2")}
         rows = max(T * k, 1)
         self.x_perm = self.h = None
-        self.xq_perm, self.xs_perm = z(rows, d, dtype=u8), sfa(rows, d, N)
-        self.hq, self.hsc = z(rows, w.f, dtype=u8), sfa(rows, w.f, N)
+        self.xq_perm, self.xs_perm = z(rows, cw(d), dtype=u8), sfa(rows, d, N)
+        self.hq, self.hsc = z(rows, cw(w.f), dtype=u8), sfa(rows, w.f, N)
         if self.fs > 0:
             self.wq.update({name: quant_w(W[name]) for name in ("ws1", "ws3", "ws2")})
-            self.xq, self.xs = z(max(T, 1), d, dtype=u8), sfa(max(T, 1), d)
-            self.hq_sh, self.hsc_sh = z(max(T, 1), self.fs, dtype=u8), sfa(max(T, 1), self.fs)
+            self.xq, self.xs = z(max(T, 1), cw(d), dtype=u8), sfa(max(T, 1), d)
+            self.hq_sh, self.hsc_sh = z(max(T, 1), cw(self.fs), dtype=u8), sfa(max(T, 1), self.fs)
             self.hs = None
 
     def _ffn_fp8(self, c, xq, xs, rows, offsets, G, names, f, hq, hsc, y, s):
-        (w1q, w1s), (w3q, w3s), (w2q, w2s) = (self.wq[n] for n in names)
+        w1, w3, w2 = (self.wq[n] for n in names)
+        if self.w.nvfp4:
+            L.moe_grouped_ffn_nvfp4(c, xq, xs, rows, offsets, G, *w1, *w3, *w2, f, hq, hsc, y, s)
+            return
         fn = L.moe_grouped_ffn_mxfp8 if self.w.mxfp8 else L.moe_grouped_ffn_fp8
-        fn(c, xq, xs, rows, offsets, G, w1q, w1s, w3q, w3s, w2q, w2s, f, hq, hsc, y, s)
+        fn(c, xq, xs, rows, offsets, G, *w1, *w3, *w2, f, hq, hsc, y, s)
 
     # the launches of one layer forward; `x` is [T, d] on the device.  `marks`, if
     # given, is a list of 7 CUDA events recorded between the stages (route, permute,
@@ -200,10 +218,13 @@ class MoELayer:
             join = torch.cuda.Event()
             join.record(side)
         rec(1)
-        fp8 = self.w.fp8 or self.w.mxfp8
+        fp8 = self.w.fp8 or self.w.mxfp8 or self.w.nvfp4
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
                       self.token_of_row, self.x_perm, self.n_dropped, self.ws, s)
-        if self.w.mxfp8:
+        if self.w.nvfp4:
+            L.moe_permute_nvfp4(c, x, self.topk_idx, self.row_of_slot, self.offsets, self.xq_perm, self.xs_perm,
+                                self.xq if self.fs > 0 else None, self.xs if self.fs > 0 else None, s)
+        elif self.w.mxfp8:
             L.moe_permute_mxfp8(c, x, self.topk_idx, self.row_of_slot, self.offsets, self.xq_perm, self.xs_perm,
                                 self.xq if self.fs > 0 else None, self.xs if self.fs > 0 else None, s)
         elif fp8:

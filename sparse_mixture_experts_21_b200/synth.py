@@ -51,6 +51,7 @@ class Workload:
     expert_choice: bool = False         # experts pick their top-C tokens (C = ceil(cf k T / N))
     fp8: bool = False                   # expert matmuls on E4M3 codes with fine-grained block scales
     mxfp8: bool = False                 # expert matmuls in MXFP8 (E4M3, E8M0 scale per 32 along K)
+    nvfp4: bool = False                 # expert matmuls in NVFP4 (E2M1, E4M3 scale per 16, fp32 per tensor)
 
     def with_tokens(self, T: int) -> "Workload":
         return replace(self, T=T)
@@ -80,6 +81,10 @@ WORKLOADS = {
     "deepseek_v3_mxfp8": Workload("deepseek_v3_mxfp8", T=16384, d=7168, N=256, k=8, f=2048, n_shared=1,
                                   f_shared=2048, score="sigmoid", n_groups=8, topk_groups=4,
                                   group_topn=2, bias_std=0.1, mxfp8=True),
+    # the same with NVFP4 experts (block scales applied by the tensor cores)
+    "deepseek_v3_nvfp4": Workload("deepseek_v3_nvfp4", T=16384, d=7168, N=256, k=8, f=2048, n_shared=1,
+                                  f_shared=2048, score="sigmoid", n_groups=8, topk_groups=4,
+                                  group_topn=2, bias_std=0.1, nvfp4=True),
 }
 
 

@@ -179,6 +179,29 @@ def test_fused_shared_ffn_checks(lib):
     assert f(cp, None, 0, ok, 1, None, None, None, 256, None, None, None, 0, None, None, None, None) == L.MOE_OK
 
 
+def test_nvfp4_argument_checks(lib):
+    """NVFP4 entry points reject bad shapes, missing tensor scales and unsupported
+    configurations before anything reaches the GPU."""
+    ok, UN, IA = 0x1000000, L.MOE_ERR_UNSUPPORTED, L.MOE_ERR_INVALID_ARG
+    q = lib.moe_quantize_nvfp4
+    assert q(ok, 128, 96, 0, ok, ok, None, None) == IA           # cols % 64
+    assert q(ok, 130, 128, 64, ok, ok, ok, None) == IA           # rows % tensor_rows
+    assert q(ok, 128, 128, 64, ok, ok, None, None) == IA         # tensor scales need g
+    assert q(ok, 128, 128, 0, ok + 2, ok, None, None) == IA      # codes 4-byte aligned
+    assert q(ok, 0, 128, 0, None, None, None, None) == L.MOE_OK  # nothing to do
+    c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    cp = ctypes.byref(c)
+    ffn = lib.moe_grouped_ffn_nvfp4
+    args = [ok, ok, 1024, ok, 4, ok, ok, ok, ok, ok, ok, ok, ok, ok, 2048, ok, ok, ok, None]
+    assert ffn(cp, *args[:14], 2176, *args[15:]) == UN             # f % 256
+    assert ffn(cp, *args[:4], 0, *args[5:]) == IA                  # G
+    assert ffn(cp, *args[:7], None, *args[8:]) == IA               # g1
+    c32 = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    assert ffn(ctypes.byref(c32), *args) == UN
+    assert lib.moe_permute_nvfp4(ctypes.byref(c32), ok, ok, ok, ok, ok, ok, None, None, None) == UN
+    assert lib.moe_permute_nvfp4(cp, ok, ok, None, ok, ok, ok, None, None, None) == IA   # no row maps, no q
+
+
 def test_route_prepare_checks(lib):
     ok = 0x1000000
     c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
