@@ -104,6 +104,27 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
     if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
   }
 }
+// Order-preserving map of fp32 to uint32 (a larger float gives a larger key; -0 is
+// taken as +0 first, so equal floats give equal keys) and its inverse.
+__device__ __forceinline__ uint32_t f32_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_f32(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+// warp_argmax with the warp's integer reductions (redux.sync): the largest v, ties to
+// the lower index; i >= 0.  Same result as warp_argmax for NaN-free v.
+__device__ __forceinline__ void warp_argmax_redux(float& v, int& i) {
+  const uint32_t key = f32_key(v);
+  const uint32_t mk = __reduce_max_sync(0xffffffffu, key);
+  i = (int)__reduce_min_sync(0xffffffffu, key == mk ? (uint32_t)i : 0xffffffffu);
+  v = key_f32(mk);
+}
+// The largest v over the warp (redux.sync on order-preserving keys).
+__device__ __forceinline__ float warp_max_redux(float v) {
+  return key_f32(__reduce_max_sync(0xffffffffu, f32_key(v)));
+}
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

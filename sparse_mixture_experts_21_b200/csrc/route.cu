@@ -56,6 +56,10 @@ struct RouteArgs {
 template <int NV, int WARPS>
 __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, const RouteArgs& a,
                              float* pwarp) {
+  // each warp takes two tokens at a time (tm and tm + WARPS) through every step, so
+  // the two tokens' dependent chains of warp reductions interleave (one token when a
+  // lane holds more than 8 experts: the state of two would not fit in registers)
+  constexpr int U = NV <= 8 ? 2 : 1;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int N = a.N, k = a.k;
   float pacc[NV];
@@ -75,192 +79,257 @@ __device__ void select_phase(const float* logits, int ld, int TM, int64_t t0, co
   }
   const bool col_groups = a.n_groups > 1 && gsz == 32 && a.group_topn <= 2;
 
-  for (int tm = warp; tm < TM; tm += WARPS) {
-    const int64_t t = t0 + tm;
-    if (t >= a.T) break;
-    float z[NV], s[NV], q[NV];
+  for (int tm0 = warp; tm0 < TM; tm0 += U * WARPS) {
+    int tmu[U];
+    int64_t t[U];
+    bool live[U];
 #pragma unroll
-    for (int i = 0; i < NV; ++i)
-      z[i] = ((valid_m >> i) & 1u) ? logits[tm * ld + lane + 32 * i] + off_r[i] : -INFINITY;
-    // affinity and logsumexp (with the sink, over the N routed logits and the shared one)
-    const float z_sh = a.sink ? logits[tm * ld + N] : -INFINITY;
-    float m = z_sh;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) m = fmaxf(m, z[i]);
-    m = warp_max(m);
-    float ex[NV], se = 0.f;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      ex[i] = ((valid_m >> i) & 1u) ? expf(z[i] - m) : 0.f;
-      se += ex[i];
+    for (int u = 0; u < U; ++u) {
+      tmu[u] = tm0 + u * WARPS;
+      t[u] = t0 + tmu[u];
+      live[u] = tmu[u] < TM && t[u] < a.T;
     }
-    se = warp_sum(se);
-    const float ex_sh = a.sink ? expf(z_sh - m) : 0.f;
-    se += ex_sh;
-    const float lse = m + logf(se);
-    float s_sh = 0.f;
-    if (a.sink) s_sh = a.score_fn == MOE_SCORE_SOFTMAX ? ex_sh / se : 1.f / (1.f + expf(-z_sh));
-    float ssum = 0.f;
+    if (!live[0]) break;
+    float s[U][NV], q[U][NV];
+    float lse[U], s_sh[U], ssum[U];
+    {
+      float z[U][NV], m[U], z_sh[U], se[U];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const bool v = (valid_m >> i) & 1u;
-      if (a.score_fn == MOE_SCORE_SOFTMAX) s[i] = v ? ex[i] / se : 0.f;
-      else s[i] = v ? 1.f / (1.f + expf(-z[i])) : 0.f;
-      ssum += s[i];
-      q[i] = v ? s[i] + bias_r[i] : -INFINITY;
+      for (int u = 0; u < U; ++u) {
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+          z[u][i] = !live[u] ? 0.f
+                  : ((valid_m >> i) & 1u) ? logits[tmu[u] * ld + lane + 32 * i] + off_r[i] : -INFINITY;
+        // affinity and logsumexp (with the sink, over the N routed logits and the shared one)
+        z_sh[u] = (a.sink && live[u]) ? logits[tmu[u] * ld + N] : -INFINITY;
+        m[u] = z_sh[u];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) m[u] = fmaxf(m[u], z[u][i]);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) m[u] = warp_max_redux(m[u]);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        se[u] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          s[u][i] = ((valid_m >> i) & 1u) ? expf(z[u][i] - m[u]) : 0.f;    // exp terms for now
+          se[u] += s[u][i];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) se[u] = warp_sum(se[u]);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float ex_sh = a.sink ? expf(z_sh[u] - m[u]) : 0.f;
+        se[u] += ex_sh;
+        lse[u] = m[u] + logf(se[u]);
+        s_sh[u] = 0.f;
+        if (a.sink) s_sh[u] = a.score_fn == MOE_SCORE_SOFTMAX ? ex_sh / se[u] : 1.f / (1.f + expf(-z_sh[u]));
+        ssum[u] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          const bool v = (valid_m >> i) & 1u;
+          if (a.score_fn == MOE_SCORE_SOFTMAX) s[u][i] = v ? s[u][i] / se[u] : 0.f;
+          else s[u][i] = v ? 1.f / (1.f + expf(-z[u][i])) : 0.f;
+          ssum[u] += s[u][i];
+          q[u][i] = v ? s[u][i] + bias_r[i] : -INFINITY;
+        }
+      }
     }
     // load-balance statistics: routed affinities normalised over the routed experts
     // (softmax probs as they are, or s / sum s)
     if (a.score_fn == MOE_SCORE_SIGMOID || a.sink) {
-      ssum = warp_sum(ssum);
 #pragma unroll
-      for (int i = 0; i < NV; ++i) pacc[i] += s[i] / ssum;
+      for (int u = 0; u < U; ++u) ssum[u] = warp_sum(ssum[u]);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (live[u]) {
+#pragma unroll
+          for (int i = 0; i < NV; ++i) pacc[i] += s[u][i] / ssum[u];
+        }
     } else {
 #pragma unroll
-      for (int i = 0; i < NV; ++i) pacc[i] += s[i];
+      for (int u = 0; u < U; ++u)
+        if (live[u]) {
+#pragma unroll
+          for (int i = 0; i < NV; ++i) pacc[i] += s[u][i];
+        }
     }
 
     if (a.scores) {      // expert-choice routing: the affinity matrix, expert-major
 #pragma unroll
-      for (int i = 0; i < NV; ++i)
-        if ((valid_m >> i) & 1u) a.scores[(int64_t)(lane + 32 * i) * a.T + t] = s[i];
-      if (lane == 0) a.lse[t] = lse;
+      for (int u = 0; u < U; ++u)
+        if (live[u]) {
+#pragma unroll
+          for (int i = 0; i < NV; ++i)
+            if ((valid_m >> i) & 1u) a.scores[(int64_t)(lane + 32 * i) * a.T + t[u]] = s[u][i];
+          if (lane == 0) a.lse[t[u]] = lse[u];
+        }
       continue;
     }
 
-    // group-limited pre-selection: group_keep bit g = group g kept; gmargin = score of
-    // the last kept group minus the best dropped one (ties: lower group index first)
-    uint32_t group_keep = 0xffffffffu;
-    float gmargin = INFINITY;
+    // group-limited pre-selection: keep bit g = group g kept; gmargin = score of the
+    // last kept group minus the best dropped one (ties: lower group index first)
+    uint32_t group_keep[U];
+    float gmargin[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) { group_keep[u] = 0xffffffffu; gmargin[u] = INFINITY; }
     if (a.n_groups > 1) {
-      uint32_t kept_mask = 0;
       if (col_groups) {
-        // each group is one register column: butterfly merge of (best, second) gives
-        // every lane every group's score, and each lane selects the groups itself
-        float gsc[NV];
+        // each group is one register column: its largest and second largest selection
+        // scores (a repeated maximum counts twice) by warp reductions, so every lane
+        // knows every group's score and selects the groups itself
+        // lane g ends up holding group g's score
+        float gl[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) gl[u] = -INFINITY;
 #pragma unroll
         for (int i = 0; i < NV; ++i) {
-          float b1 = q[i], b2 = -INFINITY;
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const float ob1 = __shfl_xor_sync(0xffffffffu, b1, o);
-            const float ob2 = __shfl_xor_sync(0xffffffffu, b2, o);
-            const float hi = fmaxf(b1, ob1), lo = fminf(b1, ob1);
-            b2 = fmaxf(lo, fmaxf(b2, ob2));
-            b1 = hi;
+          for (int u = 0; u < U; ++u) {
+            const uint32_t key = f32_key(q[u][i]);
+            const uint32_t k1 = __reduce_max_sync(0xffffffffu, key);
+            const uint32_t at_max = __ballot_sync(0xffffffffu, key == k1);
+            const uint32_t k2 = __popc(at_max) >= 2 ? k1 : __reduce_max_sync(0xffffffffu, key == k1 ? 0u : key);
+            if (lane == i) gl[u] = a.group_topn == 1 ? key_f32(k1) : key_f32(k1) + key_f32(k2);
           }
-          gsc[i] = a.group_topn == 1 ? b1 : b1 + b2;
         }
-        float last = 0.f;
-        for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
-          float v = -INFINITY;
-          int gi = -1;
+        // the top groups: one warp arg-max per pick over the lanes' group scores (ties
+        // to the lower group index), one more for the margin
 #pragma unroll
-          for (int i = 0; i < NV; ++i)
-            if (i < a.n_groups && !((kept_mask >> i) & 1u) && (gi < 0 || gsc[i] > v)) { v = gsc[i]; gi = i; }
-          if (r < a.topk_groups) {
-            kept_mask |= 1u << gi;
-            last = v;
-          } else {
-            gmargin = last - v;
+        for (int u = 0; u < U; ++u) {
+          uint32_t kept_mask = 0;
+          float last = 0.f;
+          for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
+            float v = (lane < a.n_groups && !((kept_mask >> lane) & 1u)) ? gl[u] : -INFINITY;
+            int gi = lane;
+            warp_argmax_redux(v, gi);
+            if (r < a.topk_groups) {
+              kept_mask |= 1u << gi;
+              last = v;
+            } else {
+              gmargin[u] = last - v;
+            }
           }
+          group_keep[u] = kept_mask;
         }
       } else {
-        float my_gscore = -INFINITY;
-        for (int g = 0; g < a.n_groups; ++g) {
-          uint32_t taken = 0;
-          float gs = 0.f;
-          for (int r = 0; r < a.group_topn; ++r) {
-            float v = -INFINITY;
-            int bi = 0x7fffffff;
 #pragma unroll
-            for (int i = 0; i < NV; ++i) {
-              const int e = lane + 32 * i;
-              if (((valid_m >> i) & 1u) && gid[i] == g && !((taken >> i) & 1u) && (q[i] > v || (q[i] == v && e < bi))) {
-                v = q[i]; bi = e;
+        for (int u = 0; u < U; ++u) {
+          uint32_t kept_mask = 0;
+          float my_gscore = -INFINITY;
+          for (int g = 0; g < a.n_groups; ++g) {
+            uint32_t taken = 0;
+            float gs = 0.f;
+            for (int r = 0; r < a.group_topn; ++r) {
+              float v = -INFINITY;
+              int bi = 0x7fffffff;
+#pragma unroll
+              for (int i = 0; i < NV; ++i) {
+                const int e = lane + 32 * i;
+                if (((valid_m >> i) & 1u) && gid[i] == g && !((taken >> i) & 1u) &&
+                    (q[u][i] > v || (q[u][i] == v && e < bi))) {
+                  v = q[u][i]; bi = e;
+                }
               }
+              warp_argmax_redux(v, bi);
+              gs += v;
+              if (bi != 0x7fffffff && (bi & 31) == lane) taken |= 1u << (bi >> 5);
             }
-            warp_argmax(v, bi);
-            gs += v;
-            if (bi != 0x7fffffff && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (lane == g) my_gscore = gs;
           }
-          if (lane == g) my_gscore = gs;
-        }
-        float last = 0.f;
-        for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
-          const bool cand = lane < a.n_groups && !((kept_mask >> lane) & 1u);
-          float v = cand ? my_gscore : -INFINITY;
-          int gi = cand ? lane : 0x7fffffff;
-          warp_argmax(v, gi);
-          if (r < a.topk_groups) {
-            if (gi != 0x7fffffff) kept_mask |= 1u << gi;
-            last = v;
-          } else {
-            gmargin = last - v;
+          float last = 0.f;
+          for (int r = 0; r <= a.topk_groups && r < a.n_groups; ++r) {
+            const bool cand = lane < a.n_groups && !((kept_mask >> lane) & 1u);
+            float v = cand ? my_gscore : -INFINITY;
+            int gi = cand ? lane : 0x7fffffff;
+            warp_argmax_redux(v, gi);
+            if (r < a.topk_groups) {
+              if (gi != 0x7fffffff) kept_mask |= 1u << gi;
+              last = v;
+            } else {
+              gmargin[u] = last - v;
+            }
           }
+          group_keep[u] = kept_mask;
         }
       }
-      group_keep = kept_mask;
     }
 
-    // this lane's eligible experts, sorted by selection score (stable: the lower
+    // each lane's eligible experts, sorted by selection score (stable: the lower
     // column, hence the lower expert, first among equal scores)
-    float cv[NV];
-    int ci[NV];
+    float cv[U][NV];
+    int ci[U][NV];
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const bool el = ((valid_m >> i) & 1u) && ((group_keep >> gid[i]) & 1u);
-      cv[i] = el ? q[i] : -INFINITY;
-      ci[i] = i;
-    }
+    for (int u = 0; u < U; ++u) {
 #pragma unroll
-    for (int x = 1; x < NV; ++x) {
+      for (int i = 0; i < NV; ++i) {
+        const bool el = ((valid_m >> i) & 1u) && ((group_keep[u] >> gid[i]) & 1u);
+        cv[u][i] = el ? q[u][i] : -INFINITY;
+        ci[u][i] = i;
+      }
 #pragma unroll
-      for (int y = x; y > 0; --y) {
-        const bool sw = cv[y] > cv[y - 1];
-        const float tv = cv[y];
-        const int ti = ci[y];
-        cv[y] = sw ? cv[y - 1] : cv[y];
-        ci[y] = sw ? ci[y - 1] : ci[y];
-        cv[y - 1] = sw ? tv : cv[y - 1];
-        ci[y - 1] = sw ? ti : ci[y - 1];
+      for (int x = 1; x < NV; ++x) {
+#pragma unroll
+        for (int y = x; y > 0; --y) {
+          const bool sw = cv[u][y] > cv[u][y - 1];
+          const float tv = cv[u][y];
+          const int ti = ci[u][y];
+          cv[u][y] = sw ? cv[u][y - 1] : cv[u][y];
+          ci[u][y] = sw ? ci[u][y - 1] : ci[u][y];
+          cv[u][y - 1] = sw ? tv : cv[u][y - 1];
+          ci[u][y - 1] = sw ? ti : ci[u][y - 1];
+        }
       }
     }
-    // k picks, descending, ties to the lower expert index; then the margin
-    int my_idx = 0;
-    float kth_q = 0.f, nv = -INFINITY;
+    // k picks, descending, ties to the lower expert index; then the margin's runner-up
+    int my_idx[U];
+    float kth_q[U], nv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) { my_idx[u] = 0; kth_q[u] = 0.f; nv[u] = -INFINITY; }
     for (int j = 0; j <= k; ++j) {
-      float v = cv[0];
-      int e = v == -INFINITY ? 0x7fffffff : lane + 32 * ci[0];
-      warp_argmax(v, e);
-      if (j == k) { nv = v; break; }
-      if (e != 0x7fffffff && (e & 31) == lane) {       // the winning lane drops its head
 #pragma unroll
-        for (int i = 0; i + 1 < NV; ++i) { cv[i] = cv[i + 1]; ci[i] = ci[i + 1]; }
-        cv[NV - 1] = -INFINITY;
+      for (int u = 0; u < U; ++u) {
+        float v = cv[u][0];
+        int e = v == -INFINITY ? 0x7fffffff : lane + 32 * ci[u][0];
+        warp_argmax_redux(v, e);
+        if (j == k) {
+          nv[u] = v;
+        } else {
+          if (e != 0x7fffffff && (e & 31) == lane) {     // the winning lane drops its head
+#pragma unroll
+            for (int i = 0; i + 1 < NV; ++i) { cv[u][i] = cv[u][i + 1]; ci[u][i] = ci[u][i + 1]; }
+            cv[u][NV - 1] = -INFINITY;
+          }
+          if (lane == j) my_idx[u] = e;
+          kth_q[u] = v;
+        }
       }
-      if (lane == j) my_idx = e;
-      kth_q = v;
     }
-    const float emargin = (nv == -INFINITY) ? INFINITY : kth_q - nv;
-    // the affinity of each lane's pick (lanes j < k)
-    float my_s = 0.f;
-    const int src = lane < k ? (my_idx & 31) : 0;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const float v = __shfl_sync(0xffffffffu, s[i], src);
-      if (lane < k && (my_idx >> 5) == i) my_s = v;
-    }
-
-    const float wsum = warp_sum(lane < k ? my_s : 0.f) + s_sh;
-    if (lane < k) {
-      a.topk_idx[t * k + lane] = my_idx;
-      a.topk_w[t * k + lane] = a.renorm ? my_s / wsum : my_s;
-    }
-    if (lane == 0) {
-      a.lse[t] = lse;
-      if (a.margin) a.margin[t] = fminf(emargin, gmargin);
-      if (a.sink) a.shared_w[t] = a.renorm ? s_sh / wsum : s_sh;
+    for (int u = 0; u < U; ++u) {
+      const float emargin = (nv[u] == -INFINITY) ? INFINITY : kth_q[u] - nv[u];
+      // the affinity of each lane's pick (lanes j < k)
+      float my_s = 0.f;
+      const int src = lane < k ? (my_idx[u] & 31) : 0;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const float v = __shfl_sync(0xffffffffu, s[u][i], src);
+        if (lane < k && (my_idx[u] >> 5) == i) my_s = v;
+      }
+      const float wsum = warp_sum(lane < k ? my_s : 0.f) + s_sh[u];
+      if (live[u]) {
+        if (lane < k) {
+          a.topk_idx[t[u] * k + lane] = my_idx[u];
+          a.topk_w[t[u] * k + lane] = a.renorm ? my_s / wsum : my_s;
+        }
+        if (lane == 0) {
+          a.lse[t[u]] = lse[u];
+          if (a.margin) a.margin[t[u]] = fminf(emargin, gmargin[u]);
+          if (a.sink) a.shared_w[t[u]] = a.renorm ? s_sh[u] / wsum : s_sh[u];
+        }
+      }
     }
   }
 
