@@ -226,6 +226,19 @@ __device__ __forceinline__ T8 decode8(int L, const F8Shared* sh, int G, int tile
 
 __device__ __forceinline__ float silu8(float g) { return g / (1.0f + __expf(-g)); }
 
+// a0 += x0 * s and a1 += x1 * s as one packed two-wide fp32 FMA (each half rounds
+// exactly as fma.rn.f32)
+__device__ __forceinline__ void fma2(float& a0, float& a1, float x0, float x1, float s) {
+  asm("{\n\t.reg .b64 acc, x, sc;\n\t"
+      "mov.b64 acc, {%0, %1};\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 sc, {%4, %4};\n\t"
+      "fma.rn.f32x2 acc, x, sc, acc;\n\t"
+      "mov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(x0), "f"(x1), "f"(s));
+}
+
 // E4M3 x E4M3 -> fp32, both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
@@ -407,7 +420,8 @@ ffn_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tmem_ld_wait();
             const float sc = (MODE == 0 && part >= 2) ? s1 : s0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[32 * part + i] = fmaf(__uint_as_float(v[i]), sc, acc[32 * part + i]);
+            for (int i = 0; i < 32; i += 2)
+              fma2(acc[32 * part + i], acc[32 * part + i + 1], __uint_as_float(v[i]), __uint_as_float(v[i + 1]), sc);
           }
           tc_fence_before();
           __syncwarp();
