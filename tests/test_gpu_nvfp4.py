@@ -241,3 +241,30 @@ def test_nvfp4_layer_forward():
     err = rel_err(f64(lay.y[:w.T]), out["y"])
     print(f"NVFP4 layer: y vs oracle {err:.3e}")
     assert err < TOL_NV
+
+
+def test_nvfp4_deepseek_v3_sampled_tokens():
+    """The DeepSeek-V3-shaped layer with NVFP4 experts, at full size: sampled tokens
+    against the oracle's NVFP4 experts under the GPU's routing."""
+    w = WORKLOADS["deepseek_v3_nvfp4"]
+    inp = make_inputs(w, "cuda")
+    lay = MoELayer(w, inp, "cuda", update_bias=False)
+    lay.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    toks = np.random.default_rng(3).choice(w.T, size=4, replace=False)
+    get = expert_weights_fn(inp)
+    idx, wts = i64(lay.topk_idx), f64(lay.topk_w)
+    x64 = f64(inp["x"])
+    y_gpu = f64(lay.y[torch.tensor(toks, device="cuda")])
+    y_ref = O.swiglu_ffn_nvfp4(x64[toks], *shared_weights(inp))
+    by_expert = {}
+    for i, t in enumerate(toks):
+        for j in range(w.k):
+            by_expert.setdefault(int(idx[t, j]), []).append((i, j))
+    for e, uses in by_expert.items():
+        ye = O.swiglu_ffn_nvfp4(x64[toks[[i for i, _ in uses]]], *get(e))
+        for r_i, (i, j) in enumerate(uses):
+            y_ref[i] += wts[toks[i], j] * ye[r_i]
+    for i, t in enumerate(toks):
+        assert rel_err(y_gpu[i], y_ref[i]) < TOL_NV, (t, rel_err(y_gpu[i], y_ref[i]))
