@@ -2,26 +2,29 @@
 // Every check runs before anything is enqueued, so a rejected call has no effect.
 #include <math.h>
 
+#include <map>
 #include <mutex>
-#include <set>
-#include <tuple>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
 
 namespace moe {
 
+// The attribute is a maximum: setting a smaller value lowers it, so each (kernel,
+// device) keeps the largest size set so far and only ever raises it.
 cudaError_t ensure_smem_attr(const void* func, int bytes) {
   static std::mutex mu;
-  static std::set<std::tuple<const void*, int, int>> done;   // (kernel, device, bytes)
+  static std::map<std::pair<const void*, int>, int> set_to;   // (kernel, device) -> bytes
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_tuple(func, dev, bytes);
-  if (done.count(key)) return cudaSuccess;
+  const auto key = std::make_pair(func, dev);
+  const auto it = set_to.find(key);
+  if (it != set_to.end() && it->second >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done.insert(key);
+  if (e == cudaSuccess) set_to[key] = bytes;
   return e;
 }
 

@@ -198,7 +198,7 @@ cudaError_t launch_permute(const moe_config_t& c, int64_t capacity, const void* 
   if (nblk == 0) return cudaGetLastError();
   pm::permute_place_kernel<<<nblk, 256, N * pm::kWordsPerExpert * sizeof(uint32_t), s>>>(
       topk_idx, c.T, k, N, capacity, blk_counts, offsets, row_of_slot, token_of_row, n_dropped);
-  if (!x_perm) return cudaGetLastError();
+  if (!x_perm || c.T == 0) return cudaGetLastError();
   const size_t eb = c.x_dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const int nvec = (int)((size_t)c.d_model * eb / 16);
   const int64_t want_blocks = (c.T + 7) / 8;   // 8 warps (tokens) per block per sweep

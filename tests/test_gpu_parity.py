@@ -671,3 +671,24 @@ def test_route_with_prepared_split_equals_route_with_weight():
     torch.cuda.synchronize()
     for a, b in zip(*outs):
         assert torch.equal(a, b)
+
+
+def test_permute_row_sizes_in_any_order():
+    """Calls whose rows need different amounts of dynamic shared memory, larger after
+    smaller: a kernel's shared-memory limit is only ever raised, never lowered."""
+    for d in (512, 264, 512, 1024, 264):
+        w = replace(SMALL["mixtral_small"], d=d, T=300)
+        inp = make_inputs(w, "cuda", experts=False)
+        c = make_config(w)
+        T, N, k = w.T, w.N, w.k
+        idx = torch.stack([torch.arange(T, device="cuda") % N, (torch.arange(T, device="cuda") + 3) % N],
+                          1).to(torch.int32).contiguous()
+        z = lambda *s: torch.zeros(*s, dtype=torch.int32, device="cuda")  # noqa: E731
+        counts, offsets, ros, tor, nd = z(N), z(N + 1), z(T, k), z(T * k), z(2)
+        xp = torch.zeros(T * k, d, dtype=torch.bfloat16, device="cuda")
+        ws = torch.zeros(max(L.workspace_size(c), 16), dtype=torch.uint8, device="cuda")
+        L.moe_permute(c, inp["x"], idx, counts, offsets, ros, tor, xp, nd, ws)
+        torch.cuda.synchronize()
+        R = int(offsets[-1])
+        assert R == T * k
+        assert torch.equal(xp[:R], inp["x"][tor[:R].long()])
