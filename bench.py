@@ -173,14 +173,27 @@ def run_reference(args, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": w.name, "T": w.T, "d_model": w.d, "experts": w.N, "top_k": w.k,
-                       "d_ff": w.f, "shared": w.n_shared, "sample_tokens_per_step": sample},
+            "config": dict(workload_config(w, args.gpus), sample_tokens_per_step=sample),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{sample} tokens per step of the {w.name} workload "
                                        f"(full routing, experts, shared expert, combine, stats)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def workload_config(w, world: int = 1) -> dict:
+    """The workload's description, the same in both arms' lines."""
+    return {"workload": w.name, "T": w.T, "d_model": w.d, "experts": w.N, "top_k": w.k, "d_ff": w.f,
+            "shared_experts": w.n_shared,
+            "score": w.score + ("+bias" if w.bias_std > 0 else ""),
+            "groups": f"{w.n_groups} keep {w.topk_groups}" if w.n_groups > 1 else "none",
+            "routing": "expert-choice" if w.expert_choice else "token-choice top-k",
+            "capacity": w.capacity, "parallelism": f"replicas x{world}",
+            "experts_precision": ("E4M3, 1x128 / 128x128 block scales" if w.fp8 else
+                                  "MXFP8: E4M3, E8M0 scale per 32 along K" if w.mxfp8 else
+                                  "NVFP4: E2M1, E4M3 scale per 16 along K, fp32 per expert matrix"
+                                  if w.nvfp4 else "fp32" if w.dtype == "fp32" else "bf16")}
 
 
 # ---------------------------------------------------------------------------- our arm
@@ -536,20 +549,12 @@ def main():
                                                               "fp8-e4m3 experts, fp32 router" if w.fp8 else
                                                               "fp32" if w.dtype == "fp32" else "bf16"),
             "data": "synthetic",
-            "config": {"workload": w.name, "T": T, "d_model": d, "experts": N, "top_k": k, "d_ff": f,
-                       "shared_experts": w.n_shared,
-                       "score": w.score + ("+bias" if w.bias_std > 0 else ""),
-                       "groups": f"{w.n_groups} keep {w.topk_groups}" if w.n_groups > 1 else "none",
-                       "routing": "expert-choice" if w.expert_choice else "token-choice top-k",
-                       "capacity": w.capacity, "rows_R": R, "parallelism": f"replicas x{world}",
-                       "expert_rows": ("read from x by the first grouped GEMM (TMA gather4)" if lay.gather_rows
-                                       else "expert-ordered copy of x written by the permutation"),
-                       "experts_precision": ("E4M3, 1x128 / 128x128 block scales" if w.fp8 else
-                                             "MXFP8: E4M3, E8M0 scale per 32 along K" if w.mxfp8 else
-                                             "NVFP4: E2M1, E4M3 scale per 16 along K, fp32 per expert matrix"
-                                             if w.nvfp4 else "bf16"),
-                       "l2": (f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "
-                              f"{3 * N * d * f * (0.5 if w.nvfp4 else 1 if lowp else eb) / 1e9:.1f} GB); no flush")},
+            "config": dict(workload_config(w, world), rows_R=R,
+                           expert_rows=("read from x by the first grouped GEMM (TMA gather4)" if lay.gather_rows
+                                        else "expert-ordered copy of x written by the permutation"),
+                           l2=(f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "
+                               f"{3 * N * d * f * (0.5 if w.nvfp4 else 1 if lowp else eb) / 1e9:.1f} GB); "
+                               "no flush")),
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
             "roofline": {"kernel": ("grouped SwiGLU FFN, routed + shared experts in one tile list (gate/up + "
                                     "down passes)" if lay.fuse_shared else
