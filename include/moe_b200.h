@@ -503,6 +503,90 @@ int moe_rows_move(const void* src, int64_t row_bytes, const int32_t* map, const 
                   int32_t scatter, void* dst, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * The exchange over NVLink peer memory (the Practice page, "专家并行与 all-to-all":
+ * dispatch to the expert's rank, compute, send back for the weighted combine; its
+ * "通信优化按什么顺序做" asks for the dispatch to be fused with the work around it).
+ * Every rank maps every other rank's receive buffer (moe_peer_export on the owner,
+ * moe_peer_import elsewhere, handles passed by the caller's all-gather).  A rank's
+ * kernels store its rows straight into the owning ranks' receive buffers and read
+ * the results back from there; no kernel waits for another rank.  The caller
+ * separates the phases with a stream-ordered barrier (any collective on the stream):
+ *   moe_ep_peer_plan -> moe_ep_peer_dispatch -> barrier -> local grouped FFN on the
+ *   receive buffer (local_offsets from moe_ep_plan) -> barrier ->
+ *   moe_combine_peer (one round) or moe_ep_peer_collect + moe_combine (rounds)
+ * and, before a receive buffer takes new rows, a barrier after its last readers.
+ * A receive buffer is in local-expert order (local expert major, then source rank,
+ * then row): the rows moe_ep_plan's regroup map would produce, without the regroup.
+ * ------------------------------------------------------------------------- */
+#define MOE_PEER_HANDLE_BYTES 72
+
+/* moe_peer_export -- handle of a device buffer for other processes of the node.
+ *   ptr      device pointer into a cudaMalloc allocation (e.g. from a caching allocator)
+ *   handle   [MOE_PEER_HANDLE_BYTES] host out: the allocation's CUDA IPC handle (64
+ *            bytes), then ptr's byte offset inside the allocation (int64)
+ * The buffer stays owned by the caller and must outlive every import of it.
+ * Errors: MOE_ERR_INVALID_ARG for NULL or a pointer outside any device allocation;
+ * MOE_ERR_CUDA when the allocation cannot be shared (e.g. virtual-memory mapped). */
+int moe_peer_export(const void* ptr, void* handle);
+
+/* moe_peer_import -- map another process's exported buffer into this one.
+ *   handle   [MOE_PEER_HANDLE_BYTES] host: from moe_peer_export in the owner process
+ *   ptr      host out: device pointer to the buffer, valid on the calling thread's
+ *            current device (peer access over NVLink) until moe_peer_close
+ * Importing the same handle again returns the same pointer and counts one more use.
+ * Errors: MOE_ERR_INVALID_ARG for NULL or a negative offset; MOE_ERR_CUDA when the
+ * runtime cannot open the handle (e.g. the owner process is this process). */
+int moe_peer_import(const void* handle, void** ptr);
+
+/* moe_peer_close -- release one import; the mapping goes when its last use does.
+ * Errors: MOE_ERR_INVALID_ARG for a pointer that moe_peer_import did not return. */
+int moe_peer_close(void* ptr);
+
+/* moe_ep_peer_plan -- where each of this rank's rows lands in one round.
+ *   offsets_round [W, N+1] int32 (device): every rank's expert offsets counting only
+ *                 the pieces (source, expert) of this round (a piece is wholly in one
+ *                 round); the same array moe_ep_plan takes
+ *   offsets_own   [N+1] int32 (device): this rank's full offsets from moe_permute
+ *   peer_rows     [W] uint64 (device): address of row 0 of each rank's receive buffer
+ *                 as this rank sees it (its own buffer at [rank])
+ *   row_bytes     bytes per row (d * element size, % 16 == 0); recv_cap rows per buffer
+ *   row_addr      [rows, >= offsets_own[N]] uint64 out: row i's address in the receive
+ *                 buffer of rank e / (N / W), e its expert; 0 for rows outside the round.
+ *                 A row of the round that would land past recv_cap gets 0 and records
+ *                 MOE_ERR_INVALID_ARG in the device status word.
+ * Errors: MOE_ERR_INVALID_ARG for W < 1, rank outside [0, W), N % W != 0, a bad
+ * row_bytes or recv_cap, NULL. */
+int moe_ep_peer_plan(const int32_t* offsets_round, const int32_t* offsets_own, int32_t world, int32_t rank,
+                     int32_t n_experts, const uint64_t* peer_rows, int64_t row_bytes, int64_t recv_cap,
+                     uint64_t* row_addr, void* stream);
+
+/* moe_ep_peer_dispatch -- *row_addr[row_of_slot[t, j]] = x[t] for every slot whose row
+ * is not -1 and whose address is not 0: the permutation's row gather and the
+ * dispatch in one pass, x read once per token (call moe_permute with x_perm = NULL).
+ * The stores are made visible to the whole system before the kernel ends.
+ *   x [T, d] cfg->x_dtype (16-byte aligned); row_of_slot [T, k] from moe_permute;
+ *   row_addr [rows_cap] from moe_ep_peer_plan.  A row at or past rows_cap moves
+ *   nothing and records MOE_ERR_INVALID_ARG in the device status word.
+ * Errors: MOE_ERR_INVALID_ARG for a bad config, rows_cap < 0, NULL or misaligned x. */
+int moe_ep_peer_dispatch(const moe_config_t* cfg, const void* x, const int32_t* row_of_slot,
+                         const uint64_t* row_addr, int64_t rows_cap, void* stream);
+
+/* moe_ep_peer_collect -- y_perm[i] = *row_addr[i] for i < min(*n_rows, rows_cap) with
+ * row_addr[i] != 0: one round's results back into this rank's expert-ordered rows.
+ *   y_perm [rows_cap, d] cfg->x_dtype out (16-byte aligned)
+ * Errors: MOE_ERR_INVALID_ARG for a bad config, NULL or misaligned y_perm. */
+int moe_ep_peer_collect(const moe_config_t* cfg, const uint64_t* row_addr, const int32_t* n_rows, int64_t rows_cap,
+                        void* y_perm, void* stream);
+
+/* moe_combine_peer -- moe_combine with the result of row r read at row_addr[r] (a
+ * peer's receive buffer) instead of y_perm[r]; a row whose address is 0 counts as
+ * dropped.  Same slot order and fp32 accumulation as moe_combine, so the output is
+ * bit-identical to moe_combine over the collected rows.
+ * Errors: as moe_combine. */
+int moe_combine_peer(const moe_config_t* cfg, const uint64_t* row_addr, const int32_t* row_of_slot,
+                     const float* topk_w, const void* shared_out, const float* shared_w, void* y, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_combine -- y[t] = shared[t] + sum_{j: row >= 0} w[t,j] * y_perm[row(t,j)].
  *
  * Defines: llm-compass "稀疏门控与 Top-k 路由" (y = sum_i g_i E_i(x)) and the Practice

@@ -30,7 +30,8 @@ EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_rou
             "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
             "moe_quantize_mxfp8", "moe_permute_mxfp8", "moe_grouped_ffn_mxfp8", "moe_quantize_nvfp4",
             "moe_permute_nvfp4", "moe_grouped_ffn_nvfp4", "moe_ep_plan",
-            "moe_rows_move", "moe_router_stats_partial", "moe_router_stats_finalize",
+            "moe_rows_move", "moe_peer_export", "moe_peer_import", "moe_peer_close", "moe_ep_peer_plan",
+            "moe_ep_peer_dispatch", "moe_ep_peer_collect", "moe_combine_peer", "moe_router_stats_partial", "moe_router_stats_finalize",
             "moe_expert_choice_capacity", "moe_route_prepare_size", "moe_route_prepare",
             "moe_last_cuda_error", "moe_last_cuda_error_string")
 
@@ -118,6 +119,13 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_quantize_mxfp8": [vp, c_int64, c_int32, vp, vp, vp],
         "moe_ep_plan": [vp, c_int32, c_int32, c_int32, vp, vp, vp, vp, c_int64, vp],
         "moe_rows_move": [vp, c_int64, vp, vp, c_int64, c_int32, vp, vp],
+        "moe_peer_export": [vp, vp],
+        "moe_peer_import": [vp, ctypes.POINTER(vp)],
+        "moe_peer_close": [vp],
+        "moe_ep_peer_plan": [vp, vp, c_int32, c_int32, c_int32, vp, c_int64, c_int64, vp, vp],
+        "moe_ep_peer_dispatch": [cfgp, vp, vp, vp, c_int64, vp],
+        "moe_ep_peer_collect": [cfgp, vp, vp, c_int64, vp, vp],
+        "moe_combine_peer": [cfgp, vp, vp, vp, vp, vp, vp, vp],
         "moe_permute_mxfp8": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "moe_grouped_ffn_mxfp8": [cfgp, vp, vp, c_int64, vp, c_int32, vp, vp, vp, vp, vp, vp, c_int32, vp, vp,
                                   vp, vp],
@@ -332,6 +340,60 @@ def moe_rows_move(src, map_, n_rows, dst, scatter=False, rows_cap=None, stream=N
     _check("moe_rows_move", load().moe_rows_move(
         _ptr(src), int(row_bytes), _ptr(map_), _ptr(n_rows), int(map_.shape[0] if rows_cap is None else rows_cap),
         1 if scatter else 0, _ptr(dst), _stream(stream)))
+
+
+PEER_HANDLE_BYTES = 72
+
+
+def moe_peer_export(t: torch.Tensor) -> bytes:
+    """Handle (CUDA IPC handle of t's allocation + t's offset in it) for other processes."""
+    buf = ctypes.create_string_buffer(PEER_HANDLE_BYTES)
+    _check("moe_peer_export", load().moe_peer_export(_ptr(t), buf))
+    return buf.raw
+
+
+def moe_peer_import(handle: bytes) -> int:
+    """Device address of another process's exported buffer (until moe_peer_close)."""
+    if len(handle) != PEER_HANDLE_BYTES:
+        raise ValueError(f"a peer handle has {PEER_HANDLE_BYTES} bytes, not {len(handle)}")
+    out = ctypes.c_void_p()
+    _check("moe_peer_import", load().moe_peer_import(ctypes.create_string_buffer(handle, len(handle)),
+                                                     ctypes.byref(out)))
+    return int(out.value)
+
+
+def moe_peer_close(ptr: int) -> None:
+    _check("moe_peer_close", load().moe_peer_close(ctypes.c_void_p(ptr)))
+
+
+def moe_ep_peer_plan(offsets_round, offsets_own, world, rank, peer_rows, row_bytes, recv_cap, row_addr, stream=None):
+    """row_addr[i]: where row i of this rank lands in its expert's rank's receive buffer
+    this round (0 outside the round).  peer_rows: uint64/int64 [W] device addresses."""
+    _check("moe_ep_peer_plan", load().moe_ep_peer_plan(
+        _ptr(offsets_round), _ptr(offsets_own), int(world), int(rank), int(offsets_own.shape[0]) - 1, _ptr(peer_rows),
+        int(row_bytes), int(recv_cap), _ptr(row_addr), _stream(stream)))
+
+
+def moe_ep_peer_dispatch(cfg, x, row_of_slot, row_addr, rows_cap=None, stream=None):
+    """*row_addr[row_of_slot[t, j]] = x[t] for the slots of this round (the permutation's
+    gather and the dispatch in one pass)."""
+    _check("moe_ep_peer_dispatch", load().moe_ep_peer_dispatch(
+        ctypes.byref(cfg), _ptr(x), _ptr(row_of_slot), _ptr(row_addr),
+        int(row_addr.shape[0] if rows_cap is None else rows_cap), _stream(stream)))
+
+
+def moe_ep_peer_collect(cfg, row_addr, n_rows, y_perm, rows_cap=None, stream=None):
+    """y_perm[i] = *row_addr[i] for the rows of this round."""
+    _check("moe_ep_peer_collect", load().moe_ep_peer_collect(
+        ctypes.byref(cfg), _ptr(row_addr), _ptr(n_rows), int(row_addr.shape[0] if rows_cap is None else rows_cap),
+        _ptr(y_perm), _stream(stream)))
+
+
+def moe_combine_peer(cfg, row_addr, row_of_slot, topk_w, shared_out, y, stream=None, shared_w=None):
+    """moe_combine reading the result of row r at row_addr[r]."""
+    _check("moe_combine_peer", load().moe_combine_peer(
+        ctypes.byref(cfg), _ptr(row_addr), _ptr(row_of_slot), _ptr(topk_w), _ptr(shared_out), _ptr(shared_w),
+        _ptr(y), _stream(stream)))
 
 
 def moe_combine(cfg, y_perm, row_of_slot, topk_w, shared_out, y, stream=None, shared_w=None):

@@ -1,6 +1,7 @@
 // C ABI of the MoE layer library: host-side argument checks and launches.
 // Every check runs before anything is enqueued, so a rejected call has no effect.
 #include <math.h>
+#include <string.h>
 
 #include <map>
 #include <mutex>
@@ -443,6 +444,79 @@ int moe_rows_move(const void* src, int64_t row_bytes, const int32_t* map, const 
   if (!src || !map || !dst || !aligned16(src) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_rows_move(src, row_bytes, map, n_rows, rows_cap, scatter, dst,
                                     static_cast<cudaStream_t>(stream)));
+}
+
+int moe_peer_export(const void* ptr, void* handle) {
+  if (!ptr || !handle) return MOE_ERR_INVALID_ARG;
+  int64_t off = 0;
+  uint8_t* h = static_cast<uint8_t*>(handle);
+  const cudaError_t e = peer_export(ptr, h, &off);
+  if (e == cudaErrorInvalidValue) return MOE_ERR_INVALID_ARG;
+  if (e != cudaSuccess) return from_cuda(e);
+  memcpy(h + MOE_PEER_HANDLE_BYTES - 8, &off, 8);
+  return MOE_OK;
+}
+
+int moe_peer_import(const void* handle, void** ptr) {
+  if (!handle || !ptr) return MOE_ERR_INVALID_ARG;
+  int64_t off = 0;
+  memcpy(&off, static_cast<const uint8_t*>(handle) + MOE_PEER_HANDLE_BYTES - 8, 8);
+  if (off < 0) return MOE_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  return from_cuda(peer_import(static_cast<const uint8_t*>(handle), off, ptr));
+}
+
+int moe_peer_close(void* ptr) {
+  if (!ptr) return MOE_ERR_INVALID_ARG;
+  const int st = peer_close(ptr);
+  if (st == 1) return MOE_ERR_INVALID_ARG;
+  return from_cuda((cudaError_t)st);
+}
+
+int moe_ep_peer_plan(const int32_t* offsets_round, const int32_t* offsets_own, int32_t world, int32_t rank,
+                     int32_t n_experts, const uint64_t* peer_rows, int64_t row_bytes, int64_t recv_cap,
+                     uint64_t* row_addr, void* stream) {
+  if (world < 1 || n_experts < 1 || rank < 0 || rank >= world || (n_experts % world) != 0 || recv_cap < 0 ||
+      row_bytes <= 0 || (row_bytes % 16) != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!offsets_round || !offsets_own || !peer_rows || !row_addr) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_ep_peer_plan(offsets_round, offsets_own, world, rank, n_experts, peer_rows, row_bytes,
+                                       recv_cap, row_addr, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ep_peer_dispatch(const moe_config_t* cfg, const void* x, const int32_t* row_of_slot,
+                         const uint64_t* row_addr, int64_t rows_cap, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (rows_cap < 0) return MOE_ERR_INVALID_ARG;
+  if (rows_cap == 0 || cfg->T == 0) return MOE_OK;
+  if (!x || !aligned16(x) || !row_of_slot || !row_addr) return MOE_ERR_INVALID_ARG;
+  const int64_t row_bytes = (int64_t)cfg->d_model * (cfg->x_dtype == MOE_DTYPE_BF16 ? 2 : 4);
+  return from_cuda(launch_ep_peer_push(x, row_bytes, cfg->T, cfg->top_k, row_of_slot, row_addr, rows_cap,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int moe_ep_peer_collect(const moe_config_t* cfg, const uint64_t* row_addr, const int32_t* n_rows, int64_t rows_cap,
+                        void* y_perm, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (rows_cap < 0) return MOE_ERR_INVALID_ARG;
+  if (rows_cap == 0) return MOE_OK;
+  if (!row_addr || !n_rows || !y_perm || !aligned16(y_perm)) return MOE_ERR_INVALID_ARG;
+  const int64_t row_bytes = (int64_t)cfg->d_model * (cfg->x_dtype == MOE_DTYPE_BF16 ? 2 : 4);
+  return from_cuda(launch_ep_peer_pull(row_bytes, n_rows, rows_cap, row_addr, y_perm,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int moe_combine_peer(const moe_config_t* cfg, const uint64_t* row_addr, const int32_t* row_of_slot,
+                     const float* topk_w, const void* shared_out, const float* shared_w, void* y, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!row_addr || !row_of_slot || !topk_w || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || (shared_out && !aligned16(shared_out))) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_combine(*cfg, nullptr, row_of_slot, topk_w, shared_out, shared_w, y,
+                                  static_cast<cudaStream_t>(stream), row_addr));
 }
 
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const int32_t* row_of_slot,

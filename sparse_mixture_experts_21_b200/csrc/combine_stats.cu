@@ -12,25 +12,34 @@ namespace cs {
 // the always-on output is added).  One warp per token, fp32 accumulation in a
 // fixed order, 16-byte vectors, no atomics.
 // ---------------------------------------------------------------------------
-template <typename XT, int K, int U>
+// ADDR: the result of row r is at row_addr[r] (a peer's buffer under expert
+// parallelism, 0 when the row has none) instead of y_perm + r.
+template <typename XT, int K, int U, bool ADDR = false>
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ row_of_slot,
                const float* __restrict__ topk_w, const uint4* __restrict__ shared_out,
                const float* __restrict__ shared_w, uint4* __restrict__ y, int64_t T, int k,
-               int nvec) {
+               int nvec, const uint64_t* __restrict__ row_addr = nullptr) {
   constexpr int VN = Vec<XT>::N;
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t t = warp0; t < T; t += nwarps) {
-    const int32_t mr = lane < k ? row_of_slot[t * k + lane] : -1;
+    int32_t mr = lane < k ? row_of_slot[t * k + lane] : -1;
     const float mw = lane < k ? topk_w[t * k + lane] : 0.f;
+    uint64_t ma = 0;
+    if constexpr (ADDR) {
+      ma = mr >= 0 ? row_addr[mr] : 0;
+      if (!ma) mr = -1;
+    }
     // a dropped (or padding) slot reads a kept row of the same token with weight 0,
     // so every load below is unconditional and can be issued together
     const unsigned kept = __ballot_sync(0xffffffffu, mr >= 0);
     const float sw = shared_w ? shared_w[t] : 1.f;
-    const int32_t any_row = kept ? __shfl_sync(0xffffffffu, mr, __ffs(kept) - 1) : 0;
+    const int any_lane = kept ? __ffs(kept) - 1 : 0;
+    const int32_t any_row = __shfl_sync(0xffffffffu, mr, any_lane);
     int32_t rows[K];
+    const uint4* src[ADDR ? K : 1];
     float ws[K];
 #pragma unroll
     for (int j = 0; j < K; ++j) {
@@ -38,6 +47,8 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ row
       const float wj = __shfl_sync(0xffffffffu, mw, j);
       rows[j] = r >= 0 ? r : any_row;
       ws[j] = r >= 0 ? wj : 0.f;
+      if constexpr (ADDR)
+        src[j] = reinterpret_cast<const uint4*>(__shfl_sync(0xffffffffu, ma, r >= 0 ? j : any_lane));
     }
     for (int c0 = lane; c0 < nvec; c0 += 32 * U) {
       float acc[U][VN];
@@ -47,7 +58,10 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ row
         const int c = c0 + 32 * u;
         if (c < nvec && kept) {
 #pragma unroll
-          for (int j = 0; j < K; ++j) v[u][j] = ldg_nc16(y_perm + (int64_t)rows[j] * nvec + c);
+          for (int j = 0; j < K; ++j) {
+            if constexpr (ADDR) v[u][j] = ldg16(src[j] + c);
+            else v[u][j] = ldg_nc16(y_perm + (int64_t)rows[j] * nvec + c);
+          }
         }
         if (c < nvec && shared_out) {
           unpack16(ldg_nc16(shared_out + t * nvec + c), acc[u], XT());
@@ -301,16 +315,16 @@ bias_update_seq_kernel(const double* __restrict__ part, int n_seq, float* __rest
 }  // namespace cs
 
 
-template <typename XT>
+template <typename XT, bool ADDR>
 cudaError_t launch_combine_t(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
                              const float* topk_w, const void* shared_out, const float* shared_w,
-                             void* y, int grid, int nvec, cudaStream_t s) {
+                             void* y, int grid, int nvec, cudaStream_t s, const uint64_t* row_addr) {
   auto yp = static_cast<const uint4*>(y_perm);
   auto sh = static_cast<const uint4*>(shared_out);
   auto yo = static_cast<uint4*>(y);
 #define MOE_COMBINE(KK, UU) \
-  cs::combine_kernel<XT, KK, UU><<<grid, 256, 0, s>>>(yp, row_of_slot, topk_w, sh, shared_w, yo, c.T, \
-                                                      c.top_k, nvec)
+  cs::combine_kernel<XT, KK, UU, ADDR><<<grid, 256, 0, s>>>(yp, row_of_slot, topk_w, sh, shared_w, yo, c.T, \
+                                                            c.top_k, nvec, row_addr)
   switch (c.top_k) {
     case 1: MOE_COMBINE(1, 4); break;
     case 2: MOE_COMBINE(2, 4); break;
@@ -328,17 +342,25 @@ cudaError_t launch_combine_t(const moe_config_t& c, const void* y_perm, const in
 
 cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
                            const float* topk_w, const void* shared_out, const float* shared_w,
-                           void* y, cudaStream_t s) {
+                           void* y, cudaStream_t s, const uint64_t* row_addr) {
   if (c.T == 0) return cudaSuccess;
   const size_t eb = c.x_dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const int nvec = (int)((size_t)c.d_model * eb / 16);
   const int64_t want = (c.T + 7) / 8;
   const int64_t cap = (int64_t)sm_count() * 8;
   const int grid = (int)(want < cap ? want : cap);
+  if (row_addr) {
+    if (c.x_dtype == MOE_DTYPE_BF16)
+      return launch_combine_t<__nv_bfloat16, true>(c, nullptr, row_of_slot, topk_w, shared_out, shared_w, y,
+                                                   grid, nvec, s, row_addr);
+    return launch_combine_t<float, true>(c, nullptr, row_of_slot, topk_w, shared_out, shared_w, y, grid, nvec,
+                                         s, row_addr);
+  }
   if (c.x_dtype == MOE_DTYPE_BF16)
-    return launch_combine_t<__nv_bfloat16>(c, y_perm, row_of_slot, topk_w, shared_out, shared_w, y, grid,
-                                           nvec, s);
-  return launch_combine_t<float>(c, y_perm, row_of_slot, topk_w, shared_out, shared_w, y, grid, nvec, s);
+    return launch_combine_t<__nv_bfloat16, false>(c, y_perm, row_of_slot, topk_w, shared_out, shared_w, y,
+                                                  grid, nvec, s, nullptr);
+  return launch_combine_t<float, false>(c, y_perm, row_of_slot, topk_w, shared_out, shared_w, y, grid, nvec, s,
+                                        nullptr);
 }
 
 cudaError_t launch_stats(const moe_config_t& c, int mode, const int32_t* counts, const int32_t* offsets,

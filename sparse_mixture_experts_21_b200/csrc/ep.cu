@@ -96,7 +96,150 @@ rows_move_kernel(const uint4* __restrict__ src, int nvec, const int32_t* __restr
   }
 }
 
+// ---------------------------------------------------------------------------
+// The exchange over peer memory: every rank maps every other rank's receive buffer,
+// its kernels store its rows straight into the ranks that own their experts and load
+// the results back from there.  The caller puts a stream-ordered barrier (a
+// collective) between the phases, so no kernel ever waits for another rank's kernel.
+// A destination's receive buffer is in local-expert order (expert major, then source
+// rank, then row), so its grouped FFN runs on it as it stands -- no regroup pass.
+//
+//   ep_peer_plan   row_addr[i] for this rank's rows i (expert major, moe_permute's
+//                  order): the address of row i in rank d = e / El's receive buffer,
+//                  d's rows of local experts before e's, then of sources before this
+//                  rank for e, then i - offsets[e]; 0 for rows outside this round
+//   ep_peer_push   *row_addr[row_of_slot[t, j]] = x[t]: the permutation's row gather
+//                  and the dispatch in one pass, x read once per token (the
+//                  expert-ordered copy of x is never written)
+//   ep_peer_pull   y_perm[i] = *row_addr[i]
+// ---------------------------------------------------------------------------
+
+// One block per expert e of the N.
+__global__ void __launch_bounds__(256)
+ep_peer_plan_kernel(const int32_t* __restrict__ offsets_round, const int32_t* __restrict__ offsets_own, int W,
+                    int rank, int N, int El, const uint64_t* __restrict__ peer_rows, int64_t row_bytes,
+                    int64_t recv_cap, uint64_t* __restrict__ row_addr) {
+  const int e = blockIdx.x, d = e / El, j = e % El;
+  auto kept = [&](int s2, int e2) -> int64_t {
+    const int32_t* o = offsets_round + (int64_t)s2 * (N + 1);
+    return (int64_t)o[e2 + 1] - o[e2];
+  };
+  __shared__ int64_t s_base, s_cnt;
+  if (threadIdx.x == 0) {
+    int64_t base = 0;
+    for (int j2 = 0; j2 < j; ++j2)
+      for (int s2 = 0; s2 < W; ++s2) base += kept(s2, d * El + j2);
+    for (int s2 = 0; s2 < rank; ++s2) base += kept(s2, e);
+    s_base = base;
+    s_cnt = kept(rank, e);
+  }
+  __syncthreads();
+  const int64_t r0 = offsets_own[e], cnt = (int64_t)offsets_own[e + 1] - r0;
+  const uint64_t p = peer_rows[d];
+  for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+    uint64_t a = 0;
+    if (s_cnt > 0) {
+      const int64_t q = s_base + i;
+      // a piece is wholly in one round and fits the receive buffer (the host plan's
+      // packing); anything else is the caller's error and moves no row
+      if (i < s_cnt && q < recv_cap && p) a = p + (uint64_t)(q * row_bytes);
+      else flag_invalid_index();
+    }
+    row_addr[r0 + i] = a;
+  }
+}
+
+// One warp per token: x[t] is read once and stored to the rows of its slots in
+// this round, *row_addr[row_of_slot[t, j]] = x[t] (row_addr 0 or row -1: no store).
+__global__ void __launch_bounds__(256)
+ep_peer_push_kernel(const uint4* __restrict__ x, int nvec, int64_t T, int k,
+                    const int32_t* __restrict__ row_of_slot, const uint64_t* __restrict__ row_addr,
+                    int64_t rows_cap) {
+  constexpr int U = 2;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t t = warp0; t < T; t += nwarps) {
+    uint64_t a = 0;
+    if (lane < k) {
+      const int32_t row = row_of_slot[t * k + lane];
+      if (row >= 0 && row < rows_cap) a = row_addr[row];
+      else if (row >= rows_cap) flag_invalid_index();
+    }
+    unsigned live = __ballot_sync(0xffffffffu, a != 0);
+    if (!live) continue;
+    const uint4* src = x + t * nvec;
+    for (int c0 = lane; c0 < nvec; c0 += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + 32 * u < nvec) v[u] = ldg_nc16(src + c0 + 32 * u);
+      for (unsigned m = live; m; m &= m - 1) {
+        uint4* dst = reinterpret_cast<uint4*>(__shfl_sync(0xffffffffu, a, __ffs(m) - 1));
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (c0 + 32 * u < nvec) dst[c0 + 32 * u] = v[u];
+      }
+    }
+  }
+  // the stores reach the peers before anything the stream runs after this kernel
+  // (the barrier collective that releases the destinations)
+  __threadfence_system();
+}
+
+// One warp per row: y_perm[r] = *row_addr[r] for r < min(*n_rows, rows_cap), row_addr[r] != 0.
+__global__ void __launch_bounds__(256)
+ep_peer_pull_kernel(int nvec, const int32_t* __restrict__ n_rows, int64_t rows_cap,
+                    const uint64_t* __restrict__ row_addr, uint4* __restrict__ y_perm) {
+  constexpr int U = 4;
+  const int lane = threadIdx.x & 31;
+  const int64_t n = min((int64_t)*n_rows, rows_cap);
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t r = warp0; r < n; r += nwarps) {
+    const uint64_t a = row_addr[r];
+    if (!a) continue;
+    const uint4* src = reinterpret_cast<const uint4*>(a);
+    uint4* dst = y_perm + r * nvec;
+    for (int c0 = lane; c0 < nvec; c0 += 32 * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + 32 * u < nvec) v[u] = ldg16(src + c0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (c0 + 32 * u < nvec) dst[c0 + 32 * u] = v[u];
+    }
+  }
+}
+
 }  // namespace ep
+
+cudaError_t launch_ep_peer_plan(const int32_t* offsets_round, const int32_t* offsets_own, int W, int rank, int N,
+                                const uint64_t* peer_rows, int64_t row_bytes, int64_t recv_cap, uint64_t* row_addr,
+                                cudaStream_t s) {
+  ep::ep_peer_plan_kernel<<<N, 256, 0, s>>>(offsets_round, offsets_own, W, rank, N, N / W, peer_rows, row_bytes,
+                                            recv_cap, row_addr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_peer_push(const void* x, int64_t row_bytes, int64_t T, int k, const int32_t* row_of_slot,
+                                const uint64_t* row_addr, int64_t rows_cap, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int64_t want = (T + 7) / 8, cap = (int64_t)sm_count() * 8;
+  ep::ep_peer_push_kernel<<<(int)(want < cap ? want : cap), 256, 0, s>>>(
+      static_cast<const uint4*>(x), (int)(row_bytes / 16), T, k, row_of_slot, row_addr, rows_cap);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ep_peer_pull(int64_t row_bytes, const int32_t* n_rows, int64_t rows_cap, const uint64_t* row_addr,
+                                void* y_perm, cudaStream_t s) {
+  if (rows_cap == 0) return cudaSuccess;
+  const int64_t want = (rows_cap + 7) / 8, cap = (int64_t)sm_count() * 8;
+  ep::ep_peer_pull_kernel<<<(int)(want < cap ? want : cap), 256, 0, s>>>(
+      (int)(row_bytes / 16), n_rows, rows_cap, row_addr, static_cast<uint4*>(y_perm));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_ep_plan(const int32_t* offsets_all, int W, int rank, int N, int32_t* send_splits,
                            int32_t* recv_splits, int32_t* local_offsets, int32_t* regroup_map, int64_t recv_cap,

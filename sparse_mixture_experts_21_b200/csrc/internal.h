@@ -67,7 +67,7 @@ cudaError_t launch_ffn_f32(const float* x_rows, int64_t rows_cap, const int32_t*
 
 cudaError_t launch_combine(const moe_config_t& c, const void* y_perm, const int32_t* row_of_slot,
                            const float* topk_w, const void* shared_out, const float* shared_w,
-                           void* y, cudaStream_t s);
+                           void* y, cudaStream_t s, const uint64_t* row_addr = nullptr);
 // mode 0: this batch -> stats; 1: this batch -> sufficient statistics (part_out);
 // 2: sufficient statistics (part_in, possibly summed over ranks) -> stats.
 cudaError_t launch_stats(const moe_config_t& c, int mode, const int32_t* counts, const int32_t* offsets,
@@ -117,6 +117,16 @@ cudaError_t launch_ep_plan(const int32_t* offsets_all, int W, int rank, int N, i
                            cudaStream_t s);
 cudaError_t launch_rows_move(const void* src, int64_t row_bytes, const int32_t* map, const int32_t* n_rows,
                              int64_t rows_cap, int scatter, void* dst, cudaStream_t s);
+cudaError_t launch_ep_peer_plan(const int32_t* offsets_round, const int32_t* offsets_own, int W, int rank, int N,
+                                const uint64_t* peer_rows, int64_t row_bytes, int64_t recv_cap, uint64_t* row_addr,
+                                cudaStream_t s);
+cudaError_t launch_ep_peer_push(const void* x, int64_t row_bytes, int64_t T, int k, const int32_t* row_of_slot,
+                                const uint64_t* row_addr, int64_t rows_cap, cudaStream_t s);
+cudaError_t launch_ep_peer_pull(int64_t row_bytes, const int32_t* n_rows, int64_t rows_cap, const uint64_t* row_addr,
+                                void* y_perm, cudaStream_t s);
+cudaError_t peer_export(const void* ptr, uint8_t* handle, int64_t* offset);
+cudaError_t peer_import(const uint8_t* handle, int64_t offset, void** ptr);
+int peer_close(void* ptr);
 int sm_count();
 
 }  // namespace moe

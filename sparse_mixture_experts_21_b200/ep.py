@@ -23,11 +23,26 @@ is issued before round r's expert compute and round r's return right after it, s
 the transfers overlap the grouped GEMMs ([Practice] "通信优化按什么顺序做": overlap
 the dispatch with expert compute).
 
+With peer=True the rows travel over NVLink peer memory instead: every rank maps the
+other ranks' receive buffers once, and per round moe_ep_peer_plan gives each of its
+rows its address in the owning rank's receive buffer (local-expert order, so no
+regroup pass), moe_ep_peer_dispatch stores x rows straight there (the permutation's
+gather and the dispatch in one kernel: the expert-ordered copy of x is never
+written), a barrier, the local grouped FFN in place on the receive buffer (the shared
+expert fused into round 0's launches), a barrier, and the results are read back by
+the owning ranks' kernels: moe_combine_peer loads them from the peers' buffers
+directly when there is one round, moe_ep_peer_collect pulls each round's into y_perm
+otherwise.  No kernel waits for another rank's; the barriers are collectives on the
+compute stream.
+
 The exchange is an object with all_gather(t) -> [W, *t.shape],
 all_to_all(out_list, in_list, async_op) (lists of per-rank tensors; async_op returns
-a handle with wait()) and all_reduce_sum(t); TorchDistExchange runs them with
-torch.distributed (NCCL over NVLink on GPUs).  The phases are separate methods so a
-caller can drive several ranks' layers in lock step.
+a handle with wait()) and all_reduce_sum(t); for peer=True also barrier() (stream
+ordered), peer_addresses(t) -> [W] device addresses of every rank's t (collective;
+t has the same shape everywhere) and release_peer(address).  TorchDistExchange runs
+them with torch.distributed (NCCL over NVLink on GPUs) and the library's CUDA IPC
+mapping.  The phases are separate methods so a caller can drive several ranks'
+layers in lock step.
 """
 from __future__ import annotations
 
@@ -92,6 +107,23 @@ class TorchDistExchange:
     def all_reduce_sum(self, t: torch.Tensor) -> torch.Tensor:
         self.dist.all_reduce(t, group=self.group)
         return t
+
+    def barrier(self) -> None:
+        """Stream-ordered: the current stream's later work on any rank runs after every
+        rank's earlier work (a one-element all-reduce)."""
+        if not hasattr(self, "_flag"):
+            self._flag = torch.zeros(1, dtype=torch.int32, device=torch.cuda.current_device())
+        self.dist.all_reduce(self._flag, group=self.group)
+
+    def peer_addresses(self, t: torch.Tensor) -> List[int]:
+        """Every rank's t as this process addresses it: its own data_ptr, the others
+        through the library's CUDA IPC mapping (handles all-gathered)."""
+        h = torch.frombuffer(bytearray(L.moe_peer_export(t)), dtype=torch.uint8).to(t.device)
+        hs = self.all_gather(h).cpu().numpy()
+        return [t.data_ptr() if r == self.rank else L.moe_peer_import(hs[r].tobytes()) for r in range(self.world)]
+
+    def release_peer(self, address: int) -> None:
+        L.moe_peer_close(address)
 
 
 # ----------------------------------------------------------------------------- host plan
@@ -165,7 +197,7 @@ class EPMoELayer:
     a failure."""
 
     def __init__(self, w: Workload, weights: dict, rank: int, world: int, device="cuda",
-                 exchange=None, update_bias: bool = True, recv_factor: float = 1.0):
+                 exchange=None, update_bias: bool = True, recv_factor: float = 1.0, peer: bool = False):
         if w.N % world != 0:
             raise ValueError(f"{w.N} experts do not divide over {world} ranks")
         if w.fp8 or w.mxfp8 or w.nvfp4 or w.expert_choice or w.dtype != "bf16":
@@ -190,9 +222,18 @@ class EPMoELayer:
         # order), rows regrouped by local expert (later their results), hidden rows;
         # a single rank exchanges nothing and needs none
         nset = 2 if world > 1 else 0
-        self.recv = [z(self.recv_cap, w.d) for _ in range(nset)]
-        self.loc = [z(self.recv_cap, w.d) for _ in range(nset)]
-        self.h_loc = [z(self.recv_cap, w.f) for _ in range(nset)]
+        self.peer = peer and world > 1
+        # peer mode: the FFN runs in place on the receive buffer, and set 0 also holds
+        # the shared expert's T rows after the routed ones when it rides in the same launches
+        self.fuse_shared = (self.peer and self.base.fs > 0 and self.base.fs == w.f
+                            and w.T * (w.k + 1) < 2 ** 31)
+        extra = w.T if self.fuse_shared else 0
+        self.recv = [z(self.recv_cap + (extra if i == 0 else 0), w.d) for i in range(nset)]
+        self.loc = [z(self.recv_cap, w.d) for _ in range(nset)] if not self.peer else []
+        self.h_loc = [z(self.recv_cap + (extra if i == 0 else 0), w.f) for i in range(nset)]
+        self.row_addr = z(w.T * w.k, dtype=torch.int64) if self.peer else None
+        self.peer_rows: List[torch.Tensor] = []            # per buffer set: [W] addresses of every rank's set
+        self._imported: List[int] = []
         self.regroup_map = [z(self.recv_cap, dtype=torch.int32) for _ in range(nset)]
         self.local_offsets = [z(self.El + 1, dtype=torch.int32) for _ in range(nset)]
         self.send_splits = z(world, dtype=torch.int32)
@@ -262,19 +303,24 @@ class EPMoELayer:
                                    margin=b.margin, stream=stream)
         return b.stats_part
 
-    def finish(self, x: torch.Tensor, stream=None, partial_sum: Optional[torch.Tensor] = None) -> torch.Tensor:
-        """Shared experts, combine (base.y_perm holds the returned rows), statistics
-        and bias update.  With partial_sum (the sum over ranks of stats_partial())
-        the statistics are the whole batch's and the bias update uses the summed
-        counts; without it, this rank's statistics and no bias update."""
+    def finish(self, x: torch.Tensor, stream=None, partial_sum: Optional[torch.Tensor] = None,
+               row_addr: Optional[torch.Tensor] = None, shared: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Shared experts, combine (base.y_perm holds the returned rows, or row_addr
+        gives where each row's result is), statistics and bias update.  shared: the
+        shared experts' output when already computed.  With partial_sum (the sum over
+        ranks of stats_partial()) the statistics are the whole batch's and the bias
+        update uses the summed counts; without it, this rank's statistics and no bias
+        update."""
         b, c, w = self.base, self.base.cfg, self.w
         W = b.weights
-        shared = None
-        if b.fs > 0:
+        if shared is None and b.fs > 0:
             L.moe_grouped_ffn(c, x, w.T, b.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], b.fs, b.hs, b.ys,
                               stream)
             shared = b.ys
-        L.moe_combine(c, b.y_perm, b.row_of_slot, b.topk_w, shared, b.y, stream, shared_w=b.shared_w)
+        if row_addr is not None:
+            L.moe_combine_peer(c, row_addr, b.row_of_slot, b.topk_w, shared, b.y, stream, shared_w=b.shared_w)
+        else:
+            L.moe_combine(c, b.y_perm, b.row_of_slot, b.topk_w, shared, b.y, stream, shared_w=b.shared_w)
         if partial_sum is None:
             L.moe_router_stats(c, b.counts, b.offsets, b.p_partial, b.lse, b.n_dropped, W.get("bias"), w.alpha,
                                w.z_coef, b.stats, b.f_out, b.p_out, stream, margin=b.margin)
@@ -307,6 +353,8 @@ class EPMoELayer:
             y = self.finish(x, comp, part)
             rec(3)
             return y
+        if self.peer:
+            return self._forward_peer(x, comp, rec)
         self.dispatch_prepare(x, comp)
         rec(1)
         offsets_all = ex.all_gather(self.base.offsets)
@@ -347,6 +395,61 @@ class EPMoELayer:
         rec(3)
         return y
 
+    # ---------------------------------------------------------------- one rank, peer memory
+    def map_peers(self) -> None:
+        """Every rank's receive buffers as this rank addresses them (collective: every
+        rank calls it, at its first peer forward)."""
+        if self.peer_rows:
+            return
+        for buf in self.recv:
+            addrs = self.exchange.peer_addresses(buf)
+            self._imported += [a for r, a in enumerate(addrs) if r != self.rank]
+            self.peer_rows.append(torch.tensor(addrs, dtype=torch.int64).to(self.dev))
+
+    def close(self) -> None:
+        """Release the peer mappings (every rank; after the last forward has finished
+        on every rank)."""
+        for a in self._imported:
+            self.exchange.release_peer(a)
+        self._imported, self.peer_rows = [], []
+
+    def _forward_peer(self, x: torch.Tensor, comp, rec) -> torch.Tensor:
+        ex, b, c, w = self.exchange, self.base, self.base.cfg, self.w
+        self.map_peers()
+        with torch.cuda.stream(comp):
+            b.route(x, comp)
+            # the permutation without its row gather: the dispatch gathers from x
+            L.moe_permute(c, x, b.topk_idx, b.counts, b.offsets, b.row_of_slot, b.token_of_row, None,
+                          b.n_dropped, b.ws, comp)
+            rec(1)
+            R = self.plan(ex.all_gather(b.offsets), comp)
+            n_rows = b.offsets[w.N:]
+            shared = None
+            Wt = b.weights
+            for r in range(R):
+                i = r % 2
+                self.round_begin(r, comp)
+                L.moe_ep_peer_plan(self.round_offsets[r], b.offsets, self.world, self.rank, self.peer_rows[i],
+                                   w.d * 2, self.recv_cap, self.row_addr, comp)
+                L.moe_ep_peer_dispatch(c, x, b.row_of_slot, self.row_addr, stream=comp)
+                ex.barrier()                  # every rank's rows of round r have landed here
+                if r == 0 and self.fuse_shared:
+                    L.moe_grouped_ffn_shared(c, self.recv[0], self.recv_cap, self.local_offsets[0], self.El,
+                                             self.w1, self.w3, self.w2, w.f, self.h_loc[0], self.recv[0], x, w.T,
+                                             Wt["ws1"], Wt["ws3"], Wt["ws2"], comp)
+                    shared = self.recv[0][self.recv_cap:self.recv_cap + w.T]
+                else:
+                    L.moe_grouped_ffn(c, self.recv[i], self.recv_cap, self.local_offsets[i], self.El, self.w1,
+                                      self.w3, self.w2, w.f, self.h_loc[i], self.recv[i], comp)
+                ex.barrier()                  # every rank's results of round r are ready
+                if R > 1:
+                    L.moe_ep_peer_collect(c, self.row_addr, n_rows, b.y_perm, stream=comp)
+            rec(2)
+            part = ex.all_reduce_sum(self.stats_partial(comp))
+            y = self.finish(x, comp, part, row_addr=self.row_addr if R == 1 else None, shared=shared)
+        rec(3)
+        return y
+
     def kernel_launches(self, rounds: Optional[int] = None) -> int:
         # route, permute (4), combine, stats (2), bias; shared FFN (2)
         n = 1 + 4 + 1 + 2 + (1 if self.update_bias else 0)
@@ -354,4 +457,10 @@ class EPMoELayer:
         if self.world == 1:
             return n + 2                                      # local FFN (2)
         R = len(self.plans) if rounds is None else rounds
+        if self.peer:
+            # permute without its gather (3); per round: two plans, dispatch, FFN (2), and
+            # with several rounds a collect; the shared expert rides in round 0's FFN
+            n -= 1
+            n -= 2 if self.fuse_shared else 0
+            return n + R * (1 + 1 + 1 + 2) + (R if R > 1 else 0)
         return n + R * (1 + 2 + 2)                            # per round: plan, two row moves, FFN (2)

@@ -299,6 +299,41 @@ def test_expert_parallel_argument_checks(lib):
     assert lib.moe_rows_move(ok, 32, ok, None, 0, 0, ok, None) == L.MOE_OK   # no rows
 
 
+def test_peer_exchange_argument_checks(lib):
+    """The peer-memory exchange entry points reject bad arguments before any CUDA call."""
+    ok = 0x1000000
+    IA = L.MOE_ERR_INVALID_ARG
+    c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    handle = ctypes.create_string_buffer(L.PEER_HANDLE_BYTES)
+    out = ctypes.c_void_p()
+    assert lib.moe_peer_export(None, handle) == IA
+    assert lib.moe_peer_export(ok, None) == IA
+    assert lib.moe_peer_import(None, ctypes.byref(out)) == IA
+    assert lib.moe_peer_import(handle, None) == IA
+    neg = ctypes.create_string_buffer(b"\0" * 64 + (-16).to_bytes(8, "little", signed=True), L.PEER_HANDLE_BYTES)
+    assert lib.moe_peer_import(neg, ctypes.byref(out)) == IA                  # negative offset
+    assert lib.moe_peer_close(None) == IA
+    assert lib.moe_peer_close(ok) == IA                                       # never imported
+    # plan: W must divide N, rank in range, rows a multiple of 16 bytes, every pointer given
+    assert lib.moe_ep_peer_plan(ok, ok, 3, 0, 256, ok, 14336, 100, ok, None) == IA
+    assert lib.moe_ep_peer_plan(ok, ok, 4, -1, 256, ok, 14336, 100, ok, None) == IA
+    assert lib.moe_ep_peer_plan(ok, ok, 4, 0, 256, ok, 14330, 100, ok, None) == IA
+    assert lib.moe_ep_peer_plan(ok, ok, 4, 0, 256, ok, 14336, -1, ok, None) == IA
+    assert lib.moe_ep_peer_plan(ok, ok, 4, 0, 256, None, 14336, 100, ok, None) == IA
+    assert lib.moe_ep_peer_plan(ok, ok, 4, 0, 256, ok, 14336, 100, None, None) == IA
+    # dispatch / collect / combine: pointers and alignment
+    assert lib.moe_ep_peer_dispatch(ctypes.byref(c), None, ok, ok, 10, None) == IA
+    assert lib.moe_ep_peer_dispatch(ctypes.byref(c), ok + 8, ok, ok, 10, None) == IA
+    assert lib.moe_ep_peer_dispatch(ctypes.byref(c), ok, ok, None, 10, None) == IA
+    assert lib.moe_ep_peer_dispatch(ctypes.byref(c), ok, ok, ok, -1, None) == IA
+    assert lib.moe_ep_peer_dispatch(ctypes.byref(c), None, None, None, 0, None) == L.MOE_OK   # no rows
+    assert lib.moe_ep_peer_collect(ctypes.byref(c), ok, ok, 10, ok + 8, None) == IA
+    assert lib.moe_ep_peer_collect(ctypes.byref(c), None, ok, 10, ok, None) == IA
+    assert lib.moe_ep_peer_collect(ctypes.byref(c), ok, None, 10, ok, None) == IA
+    assert lib.moe_combine_peer(ctypes.byref(c), None, ok, ok, None, None, ok, None) == IA
+    assert lib.moe_combine_peer(ctypes.byref(c), ok, ok, ok, None, None, ok + 4, None) == IA
+
+
 def test_layer_rejects_unsupported_combinations():
     from dataclasses import replace
     w = synth.WORKLOADS["ec_deepseekmoe_16b"]
