@@ -272,7 +272,8 @@ def run_ep(args, w, world, rank, local, dev, pg):
         pg = dist
     inp = make_inputs(w, dev, seed=0)                       # router and experts: the same on every rank
     x = make_inputs(w, dev, seed=100 + rank, experts=False)["x"]  # this rank's tokens
-    lay = EPMoELayer(w, inp, rank, world, dev, exchange=TorchDistExchange(), recv_factor=args.recv_factor)
+    lay = EPMoELayer(w, inp, rank, world, dev, exchange=TorchDistExchange(), recv_factor=args.recv_factor,
+                     peer=args.ep_exchange == "peer")
     for name in ("w1", "w3", "w2"):                         # only this rank's experts stay resident
         inp[name] = None
     torch.cuda.empty_cache()
@@ -333,6 +334,7 @@ def run_ep(args, w, world, rank, local, dev, pg):
             "config": {"workload": w.name, "T_per_rank": w.T, "d_model": w.d, "experts": w.N, "top_k": w.k,
                        "d_ff": w.f, "shared_experts": w.n_shared, "parallelism": f"ep{world}",
                        "experts_per_rank": w.N // world, "recv_factor": args.recv_factor,
+                       "exchange": args.ep_exchange if world > 1 else "none (one rank)",
                        "rounds_per_step": max(rounds) if rounds else 1,
                        "l2": "inputs larger than L2 (x 235 MB per rank, local expert weights "
                              f"{3 * (w.N // world) * w.d * w.f * 2 / 1e9:.1f} GB); no flush"},
@@ -352,6 +354,9 @@ def run_ep(args, w, world, rank, local, dev, pg):
             "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)
+    torch.cuda.synchronize(dev)
+    pg.barrier()                      # every rank is done with every other rank's buffers
+    lay.close()
     pg.barrier()
     pg.destroy_process_group()
     return 0
@@ -390,6 +395,10 @@ def main():
                          "expert-ordered copy that the permutation writes")
     ap.add_argument("--recv-factor", type=float, default=1.0,
                     help="ep: receive buffer rows as a multiple of T * k (rounds bound it)")
+    ap.add_argument("--ep-exchange", default="peer", choices=["peer", "nccl"],
+                    help="ep: peer -- the library's kernels store rows into the other ranks' receive buffers "
+                         "and read the results back over NVLink peer memory (CUDA IPC mappings); nccl -- "
+                         "batched NCCL point-to-point transfers")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
