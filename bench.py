@@ -391,7 +391,7 @@ def main():
                     help="run the shared expert in launches of its own instead of as one more group of the "
                          "routed grouped-FFN launches")
     ap.add_argument("--gather-rows", action="store_true",
-                    help="bf16: the grouped FFN gathers its rows from x (TMA gather4) instead of reading the "
+                    help="bf16: the grouped FFN gathers its rows from x (cp.async) instead of reading the "
                          "expert-ordered copy that the permutation writes")
     ap.add_argument("--recv-factor", type=float, default=1.0,
                     help="ep: receive buffer rows as a multiple of T * k (rounds bound it)")
@@ -559,7 +559,7 @@ def main():
                                                               "fp32" if w.dtype == "fp32" else "bf16"),
             "data": "synthetic",
             "config": dict(workload_config(w, world), rows_R=R,
-                           expert_rows=("read from x by the first grouped GEMM (TMA gather4)" if lay.gather_rows
+                           expert_rows=("read from x by the first grouped GEMM (cp.async)" if lay.gather_rows
                                         else "expert-ordered copy of x written by the permutation"),
                            l2=(f"inputs larger than L2 (x {T * d * eb / 1e6:.0f} MB, expert weights "
                                f"{3 * N * d * f * (0.5 if w.nvfp4 else 1 if lowp else eb) / 1e9:.1f} GB); "

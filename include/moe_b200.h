@@ -264,23 +264,33 @@ int moe_grouped_ffn_shared(const moe_config_t* cfg, const void* x_rows, int64_t 
  * The same grouped SwiGLU FFN (same sources, same arithmetic, bit-identical
  * output) with row r's input x[token_of_row[r]] fetched by the first GEMM itself,
  * so the expert-ordered copy of x (moe_permute's x_perm) is never written: call
- * moe_permute with x_perm = NULL and pass its token_of_row here.  This trades time
- * for memory: T k d fewer elements held, but the first GEMM's row copies (four rows
- * per TMA gather4) run well below its tiled loads -- on the DeepSeek-V3-shaped layer
- * (T = 16384, d = 7168, 256 experts, k = 8) the first GEMM took 15.7 ms against
- * 6.1 ms, far more than the 0.36 ms row copy it saves.
+ * moe_permute with x_perm = NULL and pass its token_of_row here.  The first GEMM's
+ * producer warp copies the rows with cp.async, 16 bytes per lane, into the same
+ * swizzled tiles a TMA box would give.  This trades time for memory: T k d fewer
+ * elements held, but on the DeepSeek-V3-shaped layer (T = 16384, d = 7168, 256
+ * experts, k = 8, shared expert fused) the grouped FFN took 14.9 ms against 11.6 ms
+ * over the copy, which itself takes 0.4 ms.  With ws1, ws3, ws2 given, the shared expert
+ * over all T tokens rides in the same two launches as one more group, as in
+ * moe_grouped_ffn_shared (its rows read from x in order).
  *   x             [T, d] bf16 (device), the tokens in token order
  *   token_of_row  [rows_cap] int32 (device): token of each row; read for rows
  *                 < offsets[G] only.  An entry outside [0, T) is replaced by token
  *                 0 and recorded as MOE_ERR_INVALID_ARG in the device status word
- *   offsets, w1, w3, w2, f, h_scratch, y_rows, rows_cap: as for moe_grouped_ffn
+ *   offsets, w1, w3, w2, f, rows_cap: as for moe_grouped_ffn
+ *   h_scratch, y_rows  [rows_cap (+ T with the shared expert), f] and [.., d] bf16:
+ *                 the routed rows, then the shared expert's T rows
+ *   ws1, ws3 [f, d], ws2 [d, f] bf16, or all three NULL: the shared expert, of the
+ *                 routed width f
  * Errors: MOE_ERR_UNSUPPORTED unless cfg->x_dtype is bf16 and d % 64 == 0 (the
- * gather moves whole 64-column boxes of x); MOE_ERR_INVALID_ARG as for moe_grouped_ffn, or for T < 0 or a
- * NULL token_of_row.  T = 0 or rows_cap = 0 is a no-op.
+ * rows are moved in whole 64-column steps), or when rows_cap (+ T) exceeds
+ * INT32_MAX; MOE_ERR_INVALID_ARG as for moe_grouped_ffn, or for G > 511, T < 0, a
+ * NULL token_of_row, or only some of ws1, ws3, ws2.  T = 0, or rows_cap = 0 without
+ * the shared expert, is a no-op.
  * ------------------------------------------------------------------------- */
 int moe_grouped_ffn_gather(const moe_config_t* cfg, const void* x, int64_t T, const int32_t* token_of_row,
                            int64_t rows_cap, const int32_t* offsets, int32_t G, const void* w1, const void* w3,
-                           const void* w2, int32_t f, void* h_scratch, void* y_rows, void* stream);
+                           const void* w2, int32_t f, void* h_scratch, void* y_rows, const void* ws1,
+                           const void* ws3, const void* ws2, void* stream);
 
 /* ---------------------------------------------------------------------------
  * FP8 expert compute with fine-grained block scaling.

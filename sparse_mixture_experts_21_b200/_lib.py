@@ -93,7 +93,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_grouped_ffn": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp],
         "moe_grouped_ffn_shared": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp, c_int64, vp, vp,
                                    vp, vp],
-        "moe_grouped_ffn_gather": [cfgp, vp, c_int64, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp],
+        "moe_grouped_ffn_gather": [cfgp, vp, c_int64, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp, vp,
+                                   vp, vp],
         "moe_combine": [cfgp, vp, vp, vp, vp, vp, vp, vp],
         "moe_router_stats": [cfgp, vp, vp, vp, vp, vp, vp, c_float, vp, c_float, c_float, vp, vp, vp, vp],
         "moe_router_stats_partial": [cfgp, vp, vp, vp, vp, vp, vp, c_float, vp, vp],
@@ -239,11 +240,13 @@ def moe_grouped_ffn_shared(cfg, x_rows, rows_cap, offsets, G, w1, w3, w2, f, h_s
 
 
 def moe_grouped_ffn_gather(cfg, x, T, token_of_row, rows_cap, offsets, G, w1, w3, w2, f, h_scratch, y_rows,
-                           stream=None):
-    """moe_grouped_ffn with row r read from x[token_of_row[r]] (bf16 only)."""
+                           stream=None, ws1=None, ws3=None, ws2=None):
+    """moe_grouped_ffn with row r read from x[token_of_row[r]] (bf16 only); with ws1, ws3,
+    ws2 the shared expert over x rides in the same launches (its rows after rows_cap)."""
     _check("moe_grouped_ffn_gather", load().moe_grouped_ffn_gather(
         ctypes.byref(cfg), _ptr(x), int(T), _ptr(token_of_row), int(rows_cap), _ptr(offsets), int(G), _ptr(w1),
-        _ptr(w3), _ptr(w2), int(f), _ptr(h_scratch), _ptr(y_rows), _stream(stream)))
+        _ptr(w3), _ptr(w2), int(f), _ptr(h_scratch), _ptr(y_rows), _ptr(ws1), _ptr(ws3), _ptr(ws2),
+        _stream(stream)))
 
 
 def moe_quantize_fp8(x, block_rows, q, scales, stream=None):

@@ -245,21 +245,26 @@ int moe_grouped_ffn_shared(const moe_config_t* cfg, const void* x_rows, int64_t 
 
 int moe_grouped_ffn_gather(const moe_config_t* cfg, const void* x, int64_t T, const int32_t* token_of_row,
                            int64_t rows_cap, const int32_t* offsets, int32_t G, const void* w1, const void* w3,
-                           const void* w2, int32_t f, void* h_scratch, void* y_rows, void* stream) {
+                           const void* w2, int32_t f, void* h_scratch, void* y_rows, const void* ws1,
+                           const void* ws3, const void* ws2, void* stream) {
   const int st = check_config(cfg);
   if (st != MOE_OK) return st;
-  // every gathered box lies inside x: whole 64-column boxes, ids checked on the device
+  // every gathered row chunk lies inside x: whole 64-column steps, ids checked on the device
   if (cfg->x_dtype != MOE_DTYPE_BF16 || (cfg->d_model % 64) != 0) return MOE_ERR_UNSUPPORTED;
-  if (T < 0 || rows_cap < 0 || G < 1 || G > 512 || f <= 0 || (f % 8) != 0) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || rows_cap < 0 || G < 1 || G > 511 || f <= 0 || (f % 8) != 0) return MOE_ERR_INVALID_ARG;
   if (!offsets || !token_of_row) return MOE_ERR_INVALID_ARG;
-  if (rows_cap == 0 || T == 0) return MOE_OK;
-  if (rows_cap > (int64_t)INT32_MAX || T > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  const bool shared = ws1 || ws3 || ws2;
+  if (shared && (!ws1 || !ws3 || !ws2)) return MOE_ERR_INVALID_ARG;
+  if (T == 0 || (rows_cap == 0 && !shared)) return MOE_OK;
+  if (rows_cap + (shared ? T : 0) > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
   if (!x || !w1 || !w3 || !w2 || !h_scratch || !y_rows) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w1) || !aligned16(w3) || !aligned16(w2) || !aligned16(h_scratch) ||
       !aligned16(y_rows) || (reinterpret_cast<uintptr_t>(token_of_row) & 3u))
     return MOE_ERR_INVALID_ARG;
+  if (shared && (!aligned16(ws1) || !aligned16(ws3) || !aligned16(ws2))) return MOE_ERR_INVALID_ARG;
   return from_cuda(launch_ffn_bf16_gather(x, (int)T, token_of_row, rows_cap, offsets, G, w1, w3, w2,
-                                          cfg->d_model, f, h_scratch, y_rows, static_cast<cudaStream_t>(stream)));
+                                          cfg->d_model, f, h_scratch, y_rows, ws1, ws3, ws2,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 int moe_quantize_fp8(const void* x, int64_t rows, int32_t cols, int32_t block_rows, uint8_t* q,

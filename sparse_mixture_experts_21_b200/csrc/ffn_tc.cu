@@ -266,14 +266,14 @@ __device__ __forceinline__ int32_t token_at(const int32_t* __restrict__ token_of
 // epilogue applies SwiGLU); MODE 1: down (B = one 256-row W2 box, map tmB0).
 // GATHER = false: A rows come from the expert-ordered rows (map tmA, 128-row boxes;
 // tmAt, 16-row boxes for the tails).  GATHER = true (gate/up only): row r of group g
-// is token token_of_row[r] of x [T, K], fetched with tile::gather4 (tmA over x,
-// one-row boxes; tmAt unused), so the expert-ordered copy of x is never written.
+// is token token_of_row[r] of x [T, K] at xsrc, copied by the producer warp with
+// cp.async (tmA, tmAt unused), so the expert-ordered copy of x is never written.
 // The dense extra group (the shared expert run inside the same launches): its
 // input rows are rows a_base .. a_base + rows - 1 of map a (128-row boxes; at: the
 // tail boxes), its weights b0 / b1 (as for the groups); its outputs are rows
-// rows_cap .. rows_cap + rows - 1 of the pass's output.  rows = 0: none.  Only the
-// non-gathering form takes one.  In the tile list it is group G + 1, after an
-// empty group G over the unused rows [offsets[G], rows_cap).
+// rows_cap .. rows_cap + rows - 1 of the pass's output.  rows = 0: none.  In the
+// tile list it is group G + 1, after an empty group G over the unused rows
+// [offsets[G], rows_cap).
 struct ExtraGroup {
   CUtensorMap a, at, b0, b1;
   int a_base;
@@ -286,7 +286,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
               const int32_t* __restrict__ offsets, int G, int K, int n_out, int64_t rows_cap,
               __nv_bfloat16* __restrict__ out, int ctr_slot, const int32_t* __restrict__ token_of_row,
-              int T, const __grid_constant__ ExtraGroup xg) {
+              int T, const uint8_t* __restrict__ xsrc, const __grid_constant__ ExtraGroup xg) {
   static_assert(MODE == 0 || !GATHER, "only the gate/up pass gathers its rows");
   constexpr int BN = MODE == 0 ? 128 : 256;    // output columns per tile
   extern __shared__ uint8_t smem_raw[];
@@ -299,7 +299,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
   const int nkb = (K + BK - 1) / BK;
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&sh->full[s], 1); mbar_init(&sh->empty[s], 1); }
+    // a stage's full barrier: one arrival (with the TMA bytes), or, gathering, one per
+    // lane of the producer warp
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&sh->full[s], GATHER ? 32 : 1); mbar_init(&sh->empty[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&sh->tfull[a], 1); mbar_init(&sh->tempty[a], EPI_WARPS); }
     for (int q = 0; q < TQ; ++q) { mbar_init(&sh->tq_full[q], 1); mbar_init(&sh->tq_empty[q], 1 + EPI_WARPS); }
     mbar_init(&sh->mma_done, 1);
@@ -320,7 +322,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     tmem_alloc(&sh->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  const int rows_x = GATHER ? 0 : xg.rows;
+  const int rows_x = xg.rows;
   if (warp == 2) build_tile_table(sh, offsets, G, rows_x, (int)rows_cap, lane);
   tc_fence_before();
   __syncthreads();
@@ -331,14 +333,30 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
   int32_t* ctr = g_tile_ctr[ctr_slot];
 
   if (warp == 0 && GATHER) {
-    // ---------------- tile claims + gathering TMA producer (whole warp)
-    // Lane l gathers rows 4l .. 4l+3 of each 128-row operand of the tile (the tail:
-    // of its first tn rows), 32 gather4 copies per full sub-tile and K step; the
-    // token ids are read once per tile.  Lane 0 claims tiles, waits for free stages,
-    // arms the stage barrier and loads the weight tile.
+    // ---------------- tile claims + gathering producer (whole warp)
+    // A routed operand's rows are copied from x with cp.async: one instruction moves
+    // 4 rows x 128 bytes (8 lanes per row, a 16-byte chunk each) into the 128-byte
+    // swizzled layout of a TMA box, so 32 instructions fill a 128-row operand per K
+    // step; token ids are read once per tile.  The weight tile, and the extra group's
+    // rows, come by TMA.  A stage's barrier expects the TMA bytes and 32 arrivals, one
+    // per lane, each made by the hardware once that lane's copies have landed; the MMA
+    // warp fences them for the tensor cores' async-proxy reads after its wait.
+    const int cl = lane & 7, rq = lane >> 3;    // 16-byte chunk of a row; row within a group of 4
+    const size_t row_bytes = (size_t)K * 2;
     uint32_t stage = 0, phase = 0;
     int issued = 0;
     bool ok = true;
+    // the lane's rows 4 j + rq of an operand, j < nj, copied into the box at `dst`
+    auto gather = [&](uint32_t dst, const int32_t* ids, int nj, int kb) {
+      const uint8_t* col = xsrc + (size_t)kb * (BK * 2) + cl * 16;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < nj) {
+          const int row = 4 * j + rq;
+          cp_async16(dst + row * (BK * 2) + ((cl ^ (row & 7)) << 4), col + (size_t)ids[j] * row_bytes);
+        }
+      }
+    };
     for (uint32_t i = 0; ok; ++i) {
       const uint32_t qs = i % TQ, qph = (i / TQ) & 1u;
       int L = -1;
@@ -350,44 +368,64 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       L = __shfl_sync(0xffffffffu, L, 0);
       if (L < 0) { ok = false; break; }
       if (L >= total) break;
-      const Tile t = decode_tile(L, sh, Gt, tiles_n, BN);
-      const int brow = t.g * n_out + t.n0;
-      const uint32_t bytes = (t.has0() ? A_BYTES : 0) + (t.kind == K_PAIR ? A_BYTES : 0) +
-                             (t.swap1() ? t.tn * BK * 2 : 0) + W_BYTES;
+      Tile t = decode_tile(L, sh, Gt, tiles_n, BN);
+      // the extra group reads its rows by TMA from its own maps, rows counted from its first row
+      const bool ex = t.g == G + 1;
+      const CUtensorMap* mB0 = ex ? &xg.b0 : &tmB0;
+      const CUtensorMap* mB1 = ex ? &xg.b1 : &tmB1;
+      if (ex) { t.row0 += xg.a_base - (int)rows_cap; t.trow0 += xg.a_base - (int)rows_cap; }
+      const int brow = (ex ? 0 : t.g * n_out) + t.n0;
+      const uint32_t tx = W_BYTES + (ex ? (t.has0() ? A_BYTES : 0) + (t.kind == K_PAIR ? A_BYTES : 0) +
+                                              (t.swap1() ? t.tn * BK * 2 : 0)
+                                         : 0);
       // token ids of this lane's rows; a row at or past `lim` (past the group's tail,
       // or past rows_cap) reads token 0 and feeds output that is never stored
+      int32_t id0[32], id1[32];
       auto ids = [&](int64_t first, int64_t lim, int32_t* r) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int64_t row = first + 4 * lane + j;
+        for (int j = 0; j < 32; ++j) {
+          const int64_t row = first + 4 * j + rq;
           r[j] = row < lim ? token_at(token_of_row, row, T) : 0;
         }
       };
-      int32_t r0[4] = {0, 0, 0, 0}, r1[4] = {0, 0, 0, 0};
-      const bool g1 = t.kind == K_PAIR || (t.swap1() && 4 * lane < t.tn);
-      if (t.has0()) ids(t.row0, rows_cap, r0);
-      if (t.kind == K_PAIR) ids((int64_t)t.row0 + SUB, rows_cap, r1);
-      else if (g1) ids(t.trow0, min((int64_t)t.trow0 + t.tr, rows_cap), r1);
+      const int nj1 = t.kind == K_PAIR ? 32 : (t.swap1() ? t.tn / 4 : 0);
+      if (!ex) {
+        if (t.has0()) ids(t.row0, rows_cap, id0);
+        if (t.kind == K_PAIR) ids((int64_t)t.row0 + SUB, rows_cap, id1);
+        else if (t.swap1()) ids(t.trow0, min((int64_t)t.trow0 + t.tr, rows_cap), id1);
+      }
       for (int kb = 0; kb < nkb; ++kb) {
         const bool w = lane == 0 ? wait_or_abort(&sh->empty[stage], phase ^ 1u, sh) : true;
         if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
         uint8_t* a = smem + (size_t)stage * STAGE_BYTES;
         uint8_t* b = a + 2 * A_BYTES;
-        if (lane == 0) mbar_arrive_expect_tx(&sh->full[stage], bytes);
-        __syncwarp();
-        if (t.has0()) tma_gather4(&tmA, a + lane * 512, &sh->full[stage], kb * BK, r0[0], r0[1], r0[2], r0[3]);
-        if (g1)
-          tma_gather4(&tmA, a + A_BYTES + lane * 512, &sh->full[stage], kb * BK, r1[0], r1[1], r1[2], r1[3]);
         if (lane == 0) {
-          tma_load_2d(&tmB0, b, &sh->full[stage], kb * BK, brow);
-          if (MODE == 0) tma_load_2d(&tmB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
+          mbar_expect_tx(&sh->full[stage], tx);
+          if (ex) {
+            if (t.has0()) tma_load_2d(&xg.a, a, &sh->full[stage], kb * BK, t.row0);
+            if (t.kind == K_PAIR) tma_load_2d(&xg.a, a + A_BYTES, &sh->full[stage], kb * BK, t.row0 + SUB);
+            if (t.swap1())
+              for (int j = 0; j < t.tn / TAIL_BOX; ++j)
+                tma_load_2d(&xg.at, a + A_BYTES + j * TAIL_BOX * BK * 2, &sh->full[stage], kb * BK,
+                            t.trow0 + j * TAIL_BOX);
+          }
+          tma_load_2d(mB0, b, &sh->full[stage], kb * BK, brow);
+          if (MODE == 0) tma_load_2d(mB1, b + W_BYTES / 2, &sh->full[stage], kb * BK, brow);
         }
+        __syncwarp();
+        if (!ex) {
+          if (t.has0()) gather(smem_u32(a), id0, 32, kb);
+          if (nj1) gather(smem_u32(a + A_BYTES), id1, nj1, kb);
+        }
+        cp_async_arrive_noinc(&sh->full[stage]);
         ++issued;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
+    // this lane's copies have landed; after an abort, this CTA's own TMA copies still
+    // in flight are drained before leaving
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (!ok && lane == 0) {
-      // drain this CTA's own copies still in flight before leaving
       for (int i = 1; i <= min(issued, STAGES); ++i) {
         const int s = ((int)stage - i + 2 * STAGES) % STAGES;
         const uint32_t ph = ((int)stage - i < 0) ? (phase ^ 1u) : phase;
@@ -496,6 +534,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         const uint32_t st0 = stage;
         for (int j = 0; j < P; ++j) {
           if (!wait_or_abort(&sh->full[stage], phase, sh)) { ok = false; break; }
+          if (GATHER) fence_proxy_async();     // the cp.async rows, for the tensor cores' reads
           tc_fence_after();
           if (h0) issue(stage, 0, j == 0);
           if (!h1) umma_commit(&sh->empty[stage]);
@@ -514,6 +553,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         }
         for (int kb = P; kb < nkb; ++kb) {
           if (!wait_or_abort(&sh->full[stage], phase, sh)) { ok = false; break; }
+          if (GATHER) fence_proxy_async();
           tc_fence_after();
           if (h0) issue(stage, 0, false);
           if (h1) { if (sw) issue_swapped(stage, t.tn, false); else issue(stage, 1, false); }
@@ -573,13 +613,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ++use;
         const Tile t = decode_tile(L, sh, Gt, tiles_n, BN);
         if (swapped) {
-          store_swapped<MODE>(v, t, half, q, lane, n_out, rows_cap + (GATHER ? 0 : xg.rows), out);
+          store_swapped<MODE>(v, t, half, q, lane, n_out, rows_cap + xg.rows, out);
           continue;
         }
         const int r = sub * SUB + q * 32 + lane;
         const int64_t grow = (int64_t)t.row0 + r;
         // output rows: the groups' rows_cap rows, then the extra group's
-        if (grow < rows_cap + (GATHER ? 0 : xg.rows)) {
+        if (grow < rows_cap + xg.rows) {
           __nv_bfloat16* orow = out + grow * (int64_t)n_out + t.n0;
           constexpr int NC = MODE == 0 ? 64 : 128;     // output columns of this thread
           const int c0 = half * NC;
@@ -628,7 +668,7 @@ template <int MODE, bool GATHER>
 static cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& at, const CUtensorMap& b0,
                                const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
                                int64_t rows_cap, void* out, const int32_t* token_of_row, int T,
-                               const ExtraGroup& xg, cudaStream_t s) {
+                               const void* xsrc, const ExtraGroup& xg, cudaStream_t s) {
   constexpr int BN = MODE == 0 ? 128 : 256;
   const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<MODE, GATHER>, (int)kSmem);
   if (e != cudaSuccess) return e;
@@ -638,7 +678,8 @@ static cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& at, cons
   if (grid <= 0) return cudaSuccess;
   const int slot = (int)(g_next_slot.fetch_add(1) % kCtrSlots);
   ffn_tc_kernel<MODE, GATHER><<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
-                                                           static_cast<__nv_bfloat16*>(out), slot, token_of_row, T, xg);
+                                                           static_cast<__nv_bfloat16*>(out), slot, token_of_row, T,
+                                                           static_cast<const uint8_t*>(xsrc), xg);
   return cudaGetLastError();
 }
 
@@ -658,9 +699,9 @@ cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t*
     return cudaErrorInvalidValue;
   tc::ExtraGroup none{};
   none.a = none.at = none.b0 = none.b1 = mx;
-  cudaError_t e = tc::launch_pass<0, false>(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, nullptr, 0, none, s);
+  cudaError_t e = tc::launch_pass<0, false>(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, nullptr, 0, nullptr, none, s);
   if (e != cudaSuccess) return e;
-  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, none, s);
+  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, nullptr, none, s);
 }
 
 cudaError_t launch_ffn_bf16_shared(const void* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
@@ -689,26 +730,41 @@ cudaError_t launch_ffn_bf16_shared(const void* x_rows, int64_t rows_cap, const i
   g1.b1 = g1.b0;
   g1.a_base = (int)rows_cap;
   g0.rows = g1.rows = Ts;
-  cudaError_t e = tc::launch_pass<0, false>(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, nullptr, 0, g0, s);
+  cudaError_t e = tc::launch_pass<0, false>(mx, mxt, m1, m3, offsets, G, d, f, rows_cap, h, nullptr, 0, nullptr, g0, s);
   if (e != cudaSuccess) return e;
-  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, g1, s);
+  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, nullptr, g1, s);
 }
 
 cudaError_t launch_ffn_bf16_gather(const void* x, int T, const int32_t* token_of_row, int64_t rows_cap,
                                    const int32_t* offsets, int G, const void* w1, const void* w3, const void* w2,
-                                   int d, int f, void* h, void* y, cudaStream_t s) {
-  if (rows_cap == 0 || G == 0 || T == 0) return cudaSuccess;
-  if (G > tc::kMaxGroups) return cudaErrorInvalidValue;
-  CUtensorMap mx, m1, m3, mh, mht, m2;
-  if (!make_map_bf16(&mx, x, (uint64_t)T, d, 1) || !make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) ||
-      !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) || !make_map_bf16(&mh, h, rows_cap, f, tc::SUB) ||
-      !make_map_bf16(&mht, h, rows_cap, f, tc::TAIL_BOX) || !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
+                                   int d, int f, void* h, void* y, const void* ws1, const void* ws3,
+                                   const void* ws2, cudaStream_t s) {
+  if (G > tc::kMaxGroups - 1) return cudaErrorInvalidValue;
+  const int Ts = ws1 ? T : 0;                      // the shared expert over every token, fused
+  if (T == 0 || (rows_cap == 0 && Ts == 0) || G == 0) return cudaSuccess;
+  // h and y hold the groups' rows_cap rows, then (fused) the shared expert's T rows
+  const int64_t hr = rows_cap + Ts;
+  CUtensorMap m1, m3, mh, mht, m2;
+  tc::ExtraGroup g0{}, g1{};
+  if (!make_map_bf16(&m1, w1, (uint64_t)G * f, d, 128) || !make_map_bf16(&m3, w3, (uint64_t)G * f, d, 128) ||
+      !make_map_bf16(&mh, h, hr, f, tc::SUB) || !make_map_bf16(&mht, h, hr, f, tc::TAIL_BOX) ||
+      !make_map_bf16(&m2, w2, (uint64_t)G * d, f, 256))
     return cudaErrorInvalidValue;
-  tc::ExtraGroup none{};
-  none.a = none.at = none.b0 = none.b1 = mh;
-  cudaError_t e = tc::launch_pass<0, true>(mx, mx, m1, m3, offsets, G, d, f, rows_cap, h, token_of_row, T, none, s);
+  g0.a = g0.at = g0.b0 = g0.b1 = g1.a = g1.at = g1.b0 = g1.b1 = mh;
+  if (Ts > 0) {
+    if (!make_map_bf16(&g0.a, x, Ts, d, tc::SUB) || !make_map_bf16(&g0.at, x, Ts, d, tc::TAIL_BOX) ||
+        !make_map_bf16(&g0.b0, ws1, f, d, 128) || !make_map_bf16(&g0.b1, ws3, f, d, 128) ||
+        !make_map_bf16(&g1.b0, ws2, d, f, 256))
+      return cudaErrorInvalidValue;
+    g1.a = mh;
+    g1.at = mht;
+    g1.b1 = g1.b0;
+    g1.a_base = (int)rows_cap;
+  }
+  g0.rows = g1.rows = Ts;
+  cudaError_t e = tc::launch_pass<0, true>(mh, mht, m1, m3, offsets, G, d, f, rows_cap, h, token_of_row, T, x, g0, s);
   if (e != cudaSuccess) return e;
-  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, none, s);
+  return tc::launch_pass<1, false>(mh, mht, m2, m2, offsets, G, f, d, rows_cap, y, nullptr, 0, nullptr, g1, s);
 }
 
 }  // namespace moe

@@ -60,7 +60,8 @@ cudaError_t launch_ffn_bf16_shared(const void* x_rows, int64_t rows_cap, const i
 // The same FFN with row r of group g read from x[token_of_row[r]] (x [T, d] bf16).
 cudaError_t launch_ffn_bf16_gather(const void* x, int T, const int32_t* token_of_row, int64_t rows_cap,
                                    const int32_t* offsets, int G, const void* w1, const void* w3, const void* w2,
-                                   int d, int f, void* h, void* y, cudaStream_t s);
+                                   int d, int f, void* h, void* y, const void* ws1, const void* ws3,
+                                   const void* ws2, cudaStream_t s);
 cudaError_t launch_ffn_f32(const float* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
                            const float* w1, const float* w3, const float* w2, int d, int f,
                            float* h, float* y, cudaStream_t s);

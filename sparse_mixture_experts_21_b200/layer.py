@@ -56,14 +56,16 @@ class MoELayer:
         self.overlap_shared = overlap_shared and not lowp and w.n_shared > 0
         # gather_rows: bf16 experts read their rows straight from x (moe_grouped_ffn_gather),
         # so the permutation writes no expert-ordered copy of x (T k d elements less
-        # memory); off by default: the gathering copies are slower than the copy they save
+        # memory); off by default: the first GEMM's row copies cost more time than the
+        # copy they save
         self.gather_rows = (gather_rows and w.dtype == "bf16" and w.d % 64 == 0
                             and not (lowp or w.expert_choice))
         # fuse_shared: a bf16 shared expert of the routed experts' width runs as one more
-        # group inside the routed grouped-FFN launches (moe_grouped_ffn_shared); its rows
-        # follow the routed rows in h and y_perm
+        # group inside the routed grouped-FFN launches (moe_grouped_ffn_shared, or
+        # moe_grouped_ffn_gather with the shared weights); its rows follow the routed rows
+        # in h and y_perm
         self.fuse_shared = (fuse_shared and w.dtype == "bf16" and not (lowp or w.expert_choice)
-                            and not self.gather_rows and w.n_shared * w.f_shared == w.f and w.N < 512)
+                            and w.n_shared * w.f_shared == w.f and w.N < 512)
         if self.fuse_shared:
             self.overlap_shared = False
         self.dev = torch.device(device)
@@ -234,12 +236,13 @@ class MoELayer:
         if fp8:
             self._ffn_fp8(c, self.xq_perm, self.xs_perm, T * self.w.k, self.offsets, self.w.N,
                           ("w1", "w3", "w2"), self.w.f, self.hq, self.hsc, self.y_perm, s)
+        elif self.gather_rows:
+            sw = (W["ws1"], W["ws3"], W["ws2"]) if self.fuse_shared else (None, None, None)
+            L.moe_grouped_ffn_gather(c, x, T, self.token_of_row, T * self.w.k, self.offsets, self.w.N, W["w1"],
+                                     W["w3"], W["w2"], self.w.f, self.h, self.y_perm, s, *sw)
         elif self.fuse_shared:
             L.moe_grouped_ffn_shared(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
                                      W["w2"], self.w.f, self.h, self.y_perm, x, T, W["ws1"], W["ws3"], W["ws2"], s)
-        elif self.gather_rows:
-            L.moe_grouped_ffn_gather(c, x, T, self.token_of_row, T * self.w.k, self.offsets, self.w.N, W["w1"],
-                                     W["w3"], W["w2"], self.w.f, self.h, self.y_perm, s)
         else:
             L.moe_grouped_ffn(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
                               W["w2"], self.w.f, self.h, self.y_perm, s)

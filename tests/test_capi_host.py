@@ -132,24 +132,31 @@ def test_null_and_misaligned_pointers_rejected(lib):
 
 
 def test_gathering_ffn_checks(lib):
-    """moe_grouped_ffn_gather: bf16 with d % 64 == 0 only; its row map is required;
-    no rows or no tokens is a no-op.  Nothing here reaches the GPU."""
+    """moe_grouped_ffn_gather: bf16 with d % 64 == 0 only; its row map is required; the
+    shared weights come all three or not at all; no rows or no tokens is a no-op.
+    Nothing here reaches the GPU."""
     ok, UN, IA = 0x1000000, L.MOE_ERR_UNSUPPORTED, L.MOE_ERR_INVALID_ARG
     c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
     cp = ctypes.byref(c)
-    f = lib.moe_grouped_ffn_gather
-    assert f(cp, ok, 100, None, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == IA      # token_of_row
-    assert f(cp, ok, 100, ok + 2, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == IA    # misaligned map
-    assert f(cp, ok + 8, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == IA    # misaligned x
-    assert f(cp, ok, -1, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == IA
-    assert f(cp, ok, 100, ok, 800, ok, 0, ok, ok, ok, 2048, ok, ok, None) == IA          # G
-    assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2047, ok, ok, None) == IA        # f % 8
-    assert f(cp, None, 0, ok, 800, ok, 256, None, None, None, 2048, None, None, None) == L.MOE_OK
-    assert f(cp, None, 100, ok, 0, ok, 256, None, None, None, 2048, None, None, None) == L.MOE_OK
+    no = (None, None, None)
+
+    def f(*a, shared=no):
+        return lib.moe_grouped_ffn_gather(*a, *shared, None)
+    assert f(cp, ok, 100, None, 800, ok, 256, ok, ok, ok, 2048, ok, ok) == IA      # token_of_row
+    assert f(cp, ok, 100, ok + 2, 800, ok, 256, ok, ok, ok, 2048, ok, ok) == IA    # misaligned map
+    assert f(cp, ok + 8, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok) == IA    # misaligned x
+    assert f(cp, ok, -1, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok) == IA
+    assert f(cp, ok, 100, ok, 800, ok, 0, ok, ok, ok, 2048, ok, ok) == IA          # G
+    assert f(cp, ok, 100, ok, 800, ok, 512, ok, ok, ok, 2048, ok, ok) == IA        # G: one slot for the shared
+    assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2047, ok, ok) == IA        # f % 8
+    assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, shared=(ok, None, ok)) == IA
+    assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, shared=(ok, ok, ok + 8)) == IA
+    assert f(cp, None, 0, ok, 800, ok, 256, None, None, None, 2048, None, None) == L.MOE_OK
+    assert f(cp, None, 100, ok, 0, ok, 256, None, None, None, 2048, None, None) == L.MOE_OK
     c32 = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
-    assert f(ctypes.byref(c32), ok, 10, ok, 20, ok, 8, ok, ok, ok, 256, ok, ok, None) == UN
+    assert f(ctypes.byref(c32), ok, 10, ok, 20, ok, 8, ok, ok, ok, 256, ok, ok) == UN
     c.d_model = 7168 + 8                                                                    # d % 64 != 0
-    assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok, None) == UN
+    assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok) == UN
 
 
 def test_fused_shared_ffn_checks(lib):

@@ -514,6 +514,41 @@ def test_grouped_ffn_gather_equals_grouped_ffn_on_gathered_rows(d, f, sizes):
     assert torch.equal(y1, y0)
 
 
+@pytest.mark.parametrize("d,f,sizes,T", [
+    (256, 384, [0, 1, 127, 0, 128, 129, 300, 0], 613),
+    (384, 256, [16, 17, 255, 256, 257, 5], 200),
+])
+def test_grouped_ffn_gather_with_shared_expert(d, f, sizes, T):
+    """moe_grouped_ffn_gather with the shared weights equals moe_grouped_ffn_shared on
+    the gathered rows bit for bit: routed rows and the shared expert's T rows after
+    them, every tile kind of both."""
+    G = len(sizes)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    R, cap = int(off[-1]), int(off[-1]) + 40
+    g = torch.Generator(device="cuda").manual_seed(21)
+    x = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+    tor = torch.randint(0, T, (cap,), generator=g, device="cuda", dtype=torch.int32)
+    w1 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w3 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(G, d, f, generator=g, device="cuda") / f ** 0.5).to(torch.bfloat16)
+    ws1 = (torch.randn(f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    ws3 = (torch.randn(f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    ws2 = (torch.randn(d, f, generator=g, device="cuda") / f ** 0.5).to(torch.bfloat16)
+    offs = torch.tensor(off, device="cuda")
+    cfg = make_config(replace(SMALL["mixtral_small"], d=d, f=f, N=G, T=T))
+    xr = torch.zeros(cap, d, dtype=torch.bfloat16, device="cuda")
+    xr[:R] = x[tor[:R].long()]
+    h0, h1 = (torch.empty(cap + T, f, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    y0, y1 = (torch.full((cap + T, d), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    L.moe_device_status()
+    L.moe_grouped_ffn_shared(cfg, xr, cap, offs, G, w1, w3, w2, f, h0, y0, x, T, ws1, ws3, ws2)
+    L.moe_grouped_ffn_gather(cfg, x, T, tor, cap, offs, G, w1, w3, w2, f, h1, y1, ws1=ws1, ws3=ws3, ws2=ws2)
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(h1[:R], h0[:R]) and torch.equal(h1[cap:], h0[cap:])
+    assert torch.equal(y1, y0)
+
+
 def test_grouped_ffn_gather_flags_out_of_range_token_ids():
     """A token id outside [0, T) in a read row is replaced by token 0 and recorded
     as MOE_ERR_INVALID_ARG; the call itself completes."""
