@@ -100,7 +100,12 @@ struct __align__(8) TcShared {
 // than kCtrSlots apart may share a slot (the earlier one has long finished).
 __device__ int32_t g_tile_ctr[kCtrSlots][2];
 
-constexpr size_t kSmem = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(TcShared);
+// Both passes stage their output through shared memory for TMA stores: one 32-row x
+// 32-column bf16 box (2 KB, 64-byte swizzle) per epilogue warp.
+constexpr int OUT_BOX = 2048;
+constexpr size_t kSharedPad = (sizeof(TcShared) + 1023) / 1024 * 1024;
+constexpr size_t kSmem = 1024 + (size_t)STAGES * STAGE_BYTES + kSharedPad + (size_t)EPI_WARPS * OUT_BOX;
+static_assert(kSmem <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, TcShared* sh) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -286,7 +291,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
               const int32_t* __restrict__ offsets, int G, int K, int n_out, int64_t rows_cap,
               __nv_bfloat16* __restrict__ out, int ctr_slot, const int32_t* __restrict__ token_of_row,
-              int T, const uint8_t* __restrict__ xsrc, const __grid_constant__ ExtraGroup xg) {
+              int T, const uint8_t* __restrict__ xsrc, const __grid_constant__ ExtraGroup xg,
+              const __grid_constant__ CUtensorMap tmY) {
   static_assert(MODE == 0 || !GATHER, "only the gate/up pass gathers its rows");
   constexpr int BN = MODE == 0 ? 128 : 256;    // output columns per tile
   extern __shared__ uint8_t smem_raw[];
@@ -311,6 +317,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     prefetch_tmap(&tmAt);
     prefetch_tmap(&tmB0);
     if (MODE == 0) prefetch_tmap(&tmB1);
+    prefetch_tmap(&tmY);
     if (xg.rows > 0) {
       prefetch_tmap(&xg.a);
       prefetch_tmap(&xg.at);
@@ -575,6 +582,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     // so the MMA warp waits for the TMEM copy, not for the global stores.
     const int q = warp & 3;                   // TMEM lane quarter of this warp
     const int half = (warp - 2) >> 2;         // column half (normal) / row or W half (swapped)
+    // this warp's output staging box (1024-aligned, for the 64-byte swizzle)
+    const uint32_t box = smem_u32(smem + (size_t)STAGES * STAGE_BYTES + kSharedPad) + (warp - 2) * OUT_BOX;
+    bool box_busy = false;                    // a TMA store may still be reading the box
     uint32_t use0 = 0, use1 = 0;
     for (uint32_t i = 0;; ++i) {
       // every lane waits (and acquires); the outcome is made warp-uniform
@@ -616,31 +626,46 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
           store_swapped<MODE>(v, t, half, q, lane, n_out, rows_cap + xg.rows, out);
           continue;
         }
-        const int r = sub * SUB + q * 32 + lane;
-        const int64_t grow = (int64_t)t.row0 + r;
-        // output rows: the groups' rows_cap rows, then the extra group's
-        if (grow < rows_cap + xg.rows) {
-          __nv_bfloat16* orow = out + grow * (int64_t)n_out + t.n0;
-          constexpr int NC = MODE == 0 ? 64 : 128;     // output columns of this thread
-          const int c0 = half * NC;
+        // 32 rows (one per lane) x NC output columns (gate/up: h = silu(gate) * up of 64
+        // hidden units; down: 128 columns of y), as NC / 32 boxes of 32 x 32 through
+        // shared memory: lane l writes row l's 64 bytes (16-byte chunk c at slot
+        // c ^ ((l >> 1) & 3), the 64-byte swizzle), the warp fences the writes for the
+        // TMA engine, and lane 0 stores the box, which the TMA store clips at the
+        // output's last row and column
+        constexpr int NC = MODE == 0 ? 64 : 128;
+        const int row = t.row0 + sub * SUB + q * 32;
 #pragma unroll
-          for (int j = 0; j < NC; j += 8) {
+        for (int cc = 0; cc < NC / 32; ++cc) {
+          if (box_busy) {
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int j = cc * 32 + c * 8;
             float o[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               o[i] = MODE == 0 ? silu_f(__uint_as_float(v[j + i])) * __uint_as_float(v[64 + j + i])
                                : __uint_as_float(v[j + i]);
-            if (t.n0 + c0 + j + 8 <= n_out) {
-              uint4 pk;
-              pk.x = pack_bf16x2(o[0], o[1]); pk.y = pack_bf16x2(o[2], o[3]);
-              pk.z = pack_bf16x2(o[4], o[5]); pk.w = pack_bf16x2(o[6], o[7]);
-              stg16(orow + c0 + j, pk);
-            }
+            uint4 pk;
+            pk.x = pack_bf16x2(o[0], o[1]); pk.y = pack_bf16x2(o[2], o[3]);
+            pk.z = pack_bf16x2(o[4], o[5]); pk.w = pack_bf16x2(o[6], o[7]);
+            sts16(box + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), pk);
           }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, box, t.n0 + half * NC + cc * 32, row);
+            bulk_commit();
+          }
+          box_busy = true;
         }
       }
       if (!ok) break;
     }
+    // every output box of this warp is in global memory before the kernel ends
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -669,6 +694,10 @@ static cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& at, cons
                                const CUtensorMap& b1, const int32_t* offsets, int G, int K, int n_out,
                                int64_t rows_cap, void* out, const int32_t* token_of_row, int T,
                                const void* xsrc, const ExtraGroup& xg, cudaStream_t s) {
+  // the output map: rows_cap routed rows, then the extra group's
+  CUtensorMap my;
+  if (!make_map_bf16_store32(&my, out, (uint64_t)(rows_cap + xg.rows), (uint64_t)n_out))
+    return cudaErrorInvalidValue;
   constexpr int BN = MODE == 0 ? 128 : 256;
   const cudaError_t e = ensure_smem_attr((const void*)ffn_tc_kernel<MODE, GATHER>, (int)kSmem);
   if (e != cudaSuccess) return e;
@@ -679,7 +708,7 @@ static cudaError_t launch_pass(const CUtensorMap& a, const CUtensorMap& at, cons
   const int slot = (int)(g_next_slot.fetch_add(1) % kCtrSlots);
   ffn_tc_kernel<MODE, GATHER><<<grid, THREADS, kSmem, s>>>(a, at, b0, b1, offsets, G, K, n_out, rows_cap,
                                                            static_cast<__nv_bfloat16*>(out), slot, token_of_row, T,
-                                                           static_cast<const uint8_t*>(xsrc), xg);
+                                                           static_cast<const uint8_t*>(xsrc), xg, my);
   return cudaGetLastError();
 }
 

@@ -14,6 +14,7 @@ namespace moe {
 // box_rows rows, 128-byte swizzle, zero fill out of bounds.
 bool make_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+bool make_map_bf16_store32(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols);
 
 // Padded expert count, tokens per block and scratch of the fused router.
 int route_np(int n_experts);
