@@ -43,7 +43,7 @@ NCU_TRAFFIC = {
     # reduced case (T = 4096, 64 experts, shared expert in launches of its own), scaled to
     # the full layer: routed bytes x 4, the shared expert's rows x 4 plus its 88 MB of
     # weights once; profiles/ffn_deepseek_v3_reduced.md
-    "deepseek_v3": ({"ffn_tc.cu": "454b3a2c199fd06c22d7bd11968154aa96b151b5"}, 28.6e9),
+    "deepseek_v3": ({"ffn_tc.cu": "2c6f53fa57720d650812402c7e1362c7f837f184"}, 28.7e9),
     "deepseek_v3_mxfp8": ({"ffn_mx.cu": "709e9d80185da2b81c3d48f20340d1eabb0fd4e9"}, 15.07e9),
 }
 
