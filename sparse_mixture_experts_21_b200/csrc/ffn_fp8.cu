@@ -186,7 +186,12 @@ struct __align__(8) F8Shared {
   int32_t tpre[kMaxGroups + 1];
 };
 
-constexpr size_t kSmem = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(F8Shared);
+// The down pass stages its bf16 output through shared memory for TMA stores: one
+// 32-row x 32-column box (2 KB, 64-byte swizzle) per drain warp.
+constexpr int OUT_BOX = 2048;
+constexpr size_t kSharedPad = (sizeof(F8Shared) + 1023) / 1024 * 1024;
+constexpr size_t kSmem = 1024 + (size_t)STAGES * STAGE_BYTES + kSharedPad + (size_t)EPI_WARPS * OUT_BOX;
+static_assert(kSmem <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ bool wait8(uint64_t* bar, uint32_t parity, F8Shared* sh) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -267,7 +272,8 @@ ffn_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tmB1, const float* __restrict__ sa,
                const float* __restrict__ sb0, const float* __restrict__ sb1,
                const int32_t* __restrict__ offsets, int G, int K, int n_out, int64_t rows_cap,
-               uint8_t* __restrict__ out_q, float* __restrict__ out_s, __nv_bfloat16* __restrict__ out) {
+               uint8_t* __restrict__ out_q, float* __restrict__ out_s, __nv_bfloat16* __restrict__ out,
+               const __grid_constant__ CUtensorMap tmY) {
   constexpr int BN = MODE == 0 ? 128 : 256;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -381,6 +387,9 @@ ffn_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int c_lo = MODE == 0 ? half * 64 : half * 128;
+    // down pass: this warp's output staging box (1024-aligned, for the 64-byte swizzle)
+    const uint32_t box = smem_u32(smem + (size_t)STAGES * STAGE_BYTES + kSharedPad) + (warp - 2) * OUT_BOX;
+    bool box_busy = false;                    // a TMA store may still be reading the box
     uint32_t gkb = 0;
     bool ok = true;
     for (int L = blockIdx.x; L < total; L += gridDim.x) {
@@ -459,6 +468,33 @@ ffn_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
           if (half == 0) out_s[grow * (int64_t)(n_out / 128) + t.n0 / 128] = s;
         }
+      } else if (__all_sync(0xffffffffu, ok) && q * 32 + 32 <= t.rows && col_ok) {
+        // all 32 rows of this warp are the group's: four 32 x 32 boxes through shared
+        // memory (lane l writes row l's 64 bytes, 16-byte chunk c at slot c ^ ((l >> 1) & 3),
+        // the 64-byte swizzle), fenced for the TMA engine, stored by lane 0; the store
+        // clips columns past the output.  A group's last, partial tile stores row by row.
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          if (box_busy) {
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float* e = acc + cc * 32 + c * 8;
+            uint4 pk;
+            pk.x = pack_bf16x2(e[0], e[1]); pk.y = pack_bf16x2(e[2], e[3]);
+            pk.z = pack_bf16x2(e[4], e[5]); pk.w = pack_bf16x2(e[6], e[7]);
+            sts16(box + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), pk);
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, box, t.n0 + c_lo + cc * 32, t.row0 + q * 32);
+            bulk_commit();
+          }
+          box_busy = true;
+        }
       } else if (ok && row_ok && col_ok) {
         __nv_bfloat16* orow = out + grow * (int64_t)n_out + t.n0 + c_lo;
 #pragma unroll
@@ -470,6 +506,8 @@ ffn_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
       }
     }
+    // every output box of this warp is in global memory before the kernel ends
+    if (MODE == 1 && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -490,8 +528,12 @@ cudaError_t launch_f8(const CUtensorMap& a, const CUtensorMap& b0, const CUtenso
   const int64_t max_tiles = ((rows_cap + BM - 1) / BM + G) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
+  // the down pass's output map (the gate/up pass writes no bf16 rows and never reads it)
+  CUtensorMap my{};
+  if (MODE == 1 && !make_map_bf16_store32(&my, out, (uint64_t)rows_cap, (uint64_t)n_out))
+    return cudaErrorInvalidValue;
   ffn_fp8_kernel<MODE><<<grid, THREADS, kSmem, s>>>(a, b0, b1, sa, sb0, sb1, offsets, G, K, n_out, rows_cap,
-                                                    out_q, out_s, static_cast<__nv_bfloat16*>(out));
+                                                    out_q, out_s, static_cast<__nv_bfloat16*>(out), my);
   return cudaGetLastError();
 }
 

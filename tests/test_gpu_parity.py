@@ -512,6 +512,7 @@ def test_grouped_ffn_gather_equals_grouped_ffn_on_gathered_rows(d, f, sizes):
     assert L.moe_device_status() == L.MOE_OK
     assert torch.equal(h1[:R], h0[:R])
     assert torch.equal(y1, y0)
+    assert torch.all(y0[R:] == 3.0)                # no output row past the last group is written
 
 
 @pytest.mark.parametrize("d,f,sizes,T", [
