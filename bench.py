@@ -44,7 +44,9 @@ NCU_TRAFFIC = {
     # the full layer: routed bytes x 4, the shared expert's rows x 4 plus its 88 MB of
     # weights once; profiles/ffn_deepseek_v3_reduced.md
     "deepseek_v3": ({"ffn_tc.cu": "2c6f53fa57720d650812402c7e1362c7f837f184"}, 28.7e9),
-    "deepseek_v3_mxfp8": ({"ffn_mx.cu": "709e9d80185da2b81c3d48f20340d1eabb0fd4e9"}, 15.07e9),
+    # reduced case (T = 4096, 64 experts), routed passes only, x 4;
+    # profiles/ffn_mx_traffic_deepseek_v3_mxfp8_reduced.md
+    "deepseek_v3_mxfp8": ({"ffn_mx.cu": "2e97d1168131256a9632d796c2ebb5de99a384a6"}, 15.04e9),
 }
 
 
