@@ -274,8 +274,9 @@ def run_ep(args, w, world, rank, local, dev, pg):
         pg = dist
     inp = make_inputs(w, dev, seed=0)                       # router and experts: the same on every rank
     x = make_inputs(w, dev, seed=100 + rank, experts=False)["x"]  # this rank's tokens
+    peer = args.ep_exchange == "peer"
     lay = EPMoELayer(w, inp, rank, world, dev, exchange=TorchDistExchange(), recv_factor=args.recv_factor,
-                     peer=args.ep_exchange == "peer")
+                     peer=peer, device_plan=peer and args.ep_plan == "device")
     for name in ("w1", "w3", "w2"):                         # only this rank's experts stay resident
         inp[name] = None
     torch.cuda.empty_cache()
@@ -297,7 +298,7 @@ def run_ep(args, w, world, rank, local, dev, pg):
         start.record(stream)
         for i in range(args.steps):
             lay.forward(x, stream, marks[i])
-            rounds.append(len(lay.plans) if world > 1 else 1)
+            rounds.append(len(lay.plans) if world > 1 and not lay.device_plan else 1)
         end.record(stream)
         barrier()
     ms = max_over_ranks(start.elapsed_time(end) / args.steps, dev)
@@ -306,8 +307,7 @@ def run_ep(args, w, world, rank, local, dev, pg):
     t_route_perm, t_expert, t_finish = stage(0, 1), stage(1, 2), stage(2, 3)
     t_expert_max = max_over_ranks(t_expert, dev)
     # rows this rank's experts computed in the last step, and their FLOPs
-    R_local = int(lay.base.offsets[-1].item()) if world == 1 else \
-        sum(sum(p.recv_count) for p in lay.plans)
+    R_local = lay.rows_received()
     flops_local = 6.0 * R_local * w.d * w.f
     peaks = _peaks()
     tflops = flops_local / (t_expert * 1e-3) / 1e12
@@ -335,8 +335,10 @@ def run_ep(args, w, world, rank, local, dev, pg):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "T_per_rank": w.T, "d_model": w.d, "experts": w.N, "top_k": w.k,
                        "d_ff": w.f, "shared_experts": w.n_shared, "parallelism": f"ep{world}",
-                       "experts_per_rank": w.N // world, "recv_factor": args.recv_factor,
+                       "experts_per_rank": w.N // world,
+                       "recv_factor": None if lay.device_plan else args.recv_factor,
                        "exchange": args.ep_exchange if world > 1 else "none (one rank)",
+                       "plan": ("device" if lay.device_plan else "host") if world > 1 else "none (one rank)",
                        "rounds_per_step": max(rounds) if rounds else 1,
                        "l2": "inputs larger than L2 (x 235 MB per rank, local expert weights "
                              f"{3 * (w.N // world) * w.d * w.f * 2 / 1e9:.1f} GB); no flush"},
@@ -397,6 +399,10 @@ def main():
                          "expert-ordered copy that the permutation writes")
     ap.add_argument("--recv-factor", type=float, default=1.0,
                     help="ep: receive buffer rows as a multiple of T * k (rounds bound it)")
+    ap.add_argument("--ep-plan", default="device", choices=["device", "host"],
+                    help="ep with the peer exchange: device -- receive buffers sized for every row a rank can "
+                         "receive, one round, no host synchronisation; host -- rounds bounded by --recv-factor, "
+                         "planned on the host")
     ap.add_argument("--ep-exchange", default="peer", choices=["peer", "nccl"],
                     help="ep: peer -- the library's kernels store rows into the other ranks' receive buffers "
                          "and read the results back over NVLink peer memory (CUDA IPC mappings); nccl -- "

@@ -194,16 +194,24 @@ class EPMoELayer:
 
     recv_factor: the receive buffer holds ceil(recv_factor * T * k) rows (at least T);
     1.0 is what a rank receives on average.  Skewed routing costs more rounds, never
-    a failure."""
+    a failure.
+
+    device_plan (peer exchange only): the receive buffer holds every row a rank can
+    receive, W * T * min(k, N / W) (a token sends a rank at most one row per expert it
+    picks there), so one round always suffices and the plan never leaves the device:
+    a forward makes no host synchronisation (recv_factor is not used)."""
 
     def __init__(self, w: Workload, weights: dict, rank: int, world: int, device="cuda",
-                 exchange=None, update_bias: bool = True, recv_factor: float = 1.0, peer: bool = False):
+                 exchange=None, update_bias: bool = True, recv_factor: float = 1.0, peer: bool = False,
+                 device_plan: bool = False):
         if w.N % world != 0:
             raise ValueError(f"{w.N} experts do not divide over {world} ranks")
         if w.fp8 or w.mxfp8 or w.nvfp4 or w.expert_choice or w.dtype != "bf16":
             raise ValueError("the expert-parallel layer runs bf16 token-choice routing")
         if not recv_factor > 0:
             raise ValueError("recv_factor must be positive")
+        if device_plan and not peer:
+            raise ValueError("the device-side plan needs the peer exchange")
         self.w, self.rank, self.world = w, rank, world
         self.El = w.N // world
         self.exchange = exchange
@@ -216,17 +224,21 @@ class EPMoELayer:
         self.base = MoELayer(w, local, dev, update_bias=False, gather_rows=False, fuse_shared=False)
         self.w1, self.w3, self.w2 = (weights[n][lo:hi].contiguous() for n in ("w1", "w3", "w2"))
         self.update_bias = update_bias and weights.get("bias") is not None
-        self.recv_cap = max(int(math.ceil(recv_factor * w.T * w.k)), w.T, 1)
-        z = lambda *s, dtype=torch.bfloat16: torch.empty(s, dtype=dtype, device=dev)  # noqa: E731
-        # two buffer sets (rounds alternate): received rows (later the results in arrival
-        # order), rows regrouped by local expert (later their results), hidden rows;
-        # a single rank exchanges nothing and needs none
-        nset = 2 if world > 1 else 0
         self.peer = peer and world > 1
+        self.device_plan = device_plan and self.peer
+        if self.device_plan:
+            self.recv_cap = max(world * w.T * min(w.k, self.El), 1)
+        else:
+            self.recv_cap = max(int(math.ceil(recv_factor * w.T * w.k)), w.T, 1)
+        z = lambda *s, dtype=torch.bfloat16: torch.empty(s, dtype=dtype, device=dev)  # noqa: E731
+        # two buffer sets (rounds alternate; one with the device-side plan): received rows
+        # (later the results in arrival order), rows regrouped by local expert (later their
+        # results), hidden rows; a single rank exchanges nothing and needs none
+        nset = (1 if self.device_plan else 2) if world > 1 else 0
         # peer mode: the FFN runs in place on the receive buffer, and set 0 also holds
         # the shared expert's T rows after the routed ones when it rides in the same launches
         self.fuse_shared = (self.peer and self.base.fs > 0 and self.base.fs == w.f
-                            and w.T * (w.k + 1) < 2 ** 31)
+                            and self.recv_cap + w.T < 2 ** 31)
         extra = w.T if self.fuse_shared else 0
         self.recv = [z(self.recv_cap + (extra if i == 0 else 0), w.d) for i in range(nset)]
         self.loc = [z(self.recv_cap, w.d) for _ in range(nset)] if not self.peer else []
@@ -234,7 +246,8 @@ class EPMoELayer:
         self.row_addr = z(w.T * w.k, dtype=torch.int64) if self.peer else None
         self.peer_rows: List[torch.Tensor] = []            # per buffer set: [W] addresses of every rank's set
         self._imported: List[int] = []
-        self.regroup_map = [z(self.recv_cap, dtype=torch.int32) for _ in range(nset)]
+        # the regroup map is the NCCL exchange's (peer rows land in local-expert order)
+        self.regroup_map = [z(0 if self.peer else self.recv_cap, dtype=torch.int32) for _ in range(nset)]
         self.local_offsets = [z(self.El + 1, dtype=torch.int32) for _ in range(nset)]
         self.send_splits = z(world, dtype=torch.int32)
         self.recv_splits = z(world, dtype=torch.int32)
@@ -422,7 +435,14 @@ class EPMoELayer:
             L.moe_permute(c, x, b.topk_idx, b.counts, b.offsets, b.row_of_slot, b.token_of_row, None,
                           b.n_dropped, b.ws, comp)
             rec(1)
-            R = self.plan(ex.all_gather(b.offsets), comp)
+            offsets_all = ex.all_gather(b.offsets)
+            if self.device_plan:
+                # one round: its offsets are the gathered ones, on the device
+                self.plans = []
+                self.round_offsets = offsets_all.unsqueeze(0)
+                R = 1
+            else:
+                R = self.plan(offsets_all, comp)
             n_rows = b.offsets[w.N:]
             shared = None
             Wt = b.weights
@@ -450,13 +470,21 @@ class EPMoELayer:
         rec(3)
         return y
 
+    def rows_received(self) -> int:
+        """Rows this rank's experts computed in the last forward (reads the device)."""
+        if self.world == 1:
+            return int(self.base.offsets[-1].item())
+        if self.device_plan:
+            return int(self.local_offsets[0][self.El].item())
+        return sum(sum(p.recv_count) for p in self.plans)
+
     def kernel_launches(self, rounds: Optional[int] = None) -> int:
         # route, permute (4), combine, stats (2), bias; shared FFN (2)
         n = 1 + 4 + 1 + 2 + (1 if self.update_bias else 0)
         n += 2 if self.base.fs > 0 else 0
         if self.world == 1:
             return n + 2                                      # local FFN (2)
-        R = len(self.plans) if rounds is None else rounds
+        R = (1 if self.device_plan else len(self.plans)) if rounds is None else rounds
         if self.peer:
             # permute without its gather (3); per round: two plans, dispatch, FFN (2), and
             # with several rounds a collect; the shared expert rides in round 0's FFN

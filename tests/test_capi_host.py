@@ -360,6 +360,8 @@ def test_expert_parallel_layer_validation():
         EPMoELayer(replace(w, mxfp8=True), {}, 0, 2, "cpu")  # the exchange carries bf16 rows
     with pytest.raises(ValueError):
         EPMoELayer(synth.WORKLOADS["ec_deepseekmoe_16b"], {}, 0, 2, "cpu")
+    with pytest.raises(ValueError):
+        EPMoELayer(w, {}, 0, 2, "cpu", peer=False, device_plan=True)   # the device plan needs peer memory
 
 
 def test_capture_refuses_replica_mode():

@@ -9,7 +9,8 @@
   every receive buffer in local-expert order, the collect returns every row, and the
   row-address combine equals moe_combine bit for bit;
 * EPMoELayer(peer=True).forward for W ranks run as threads on one GPU: every rank's
-  output equals the single-rank layer's on its tokens, in one round and in several;
+  output equals the single-rank layer's on its tokens, in one round and in several, and
+  with the plan kept on the device (receive buffers for every row a rank can receive);
 * two processes on one GPU with the library's CUDA IPC mapping: each imports the
   other's receive buffers and runs the peer forward, the barriers on the host (gloo
   plus a device synchronisation), so no kernel of one process waits for the other's.
@@ -249,8 +250,9 @@ class _ThreadPeerExchange:
         pass
 
 
-@pytest.mark.parametrize("W,recv_factor", [(2, 4.0), (4, 1.0), (2, 0.4)])
-def test_ep_peer_forward_threads_matches_single_rank(W, recv_factor):
+@pytest.mark.parametrize("W,recv_factor,device_plan", [(2, 4.0, False), (4, 1.0, False), (2, 0.4, False),
+                                                        (2, 1.0, True), (4, 1.0, True)])
+def test_ep_peer_forward_threads_matches_single_rank(W, recv_factor, device_plan):
     w = _case()
     shared = make_inputs(w, "cuda", seed=0)
     xs = [make_inputs(w, "cuda", seed=80 + r, experts=False)["x"] for r in range(W)]
@@ -258,7 +260,7 @@ def test_ep_peer_forward_threads_matches_single_rank(W, recv_factor):
     hub = _Hub(W)
     weights = [dict(shared, bias=bias0.clone()) for _ in range(W)]
     layers = [EPMoELayer(w, weights[r], r, W, "cuda", exchange=_ThreadPeerExchange(hub, r), update_bias=True,
-                         recv_factor=recv_factor, peer=True) for r in range(W)]
+                         recv_factor=recv_factor, peer=True, device_plan=device_plan) for r in range(W)]
     ys, errs = [None] * W, []
 
     def run(r):
@@ -280,10 +282,12 @@ def test_ep_peer_forward_threads_matches_single_rank(W, recv_factor):
     assert not errs, errs
     torch.cuda.synchronize()
     assert L.moe_device_status() == L.MOE_OK
-    R = len(layers[0].plans)
+    R = 1 if device_plan else len(layers[0].plans)
+    if device_plan:
+        assert layers[0].recv_cap == W * w.T * min(w.k, w.N // W) and not layers[0].plans
     if recv_factor >= 4.0:
         assert R == 1                                   # the combine reads the peers' buffers
-    if recv_factor < 1.0:
+    if recv_factor < 1.0 and not device_plan:
         assert R > 1                                    # every round's results are collected
     assert layers[0].fuse_shared
     counts = torch.zeros(w.N, dtype=torch.int64, device="cuda")
@@ -376,20 +380,22 @@ def _ipc_worker(rank, port, out_dir):
         w = _case()
         shared = make_inputs(w, "cuda", seed=0)
         x = make_inputs(w, "cuda", seed=90 + rank, experts=False)["x"]
-        lay = EPMoELayer(w, shared, rank, 2, "cuda", exchange=ex, update_bias=False, recv_factor=1.0, peer=True)
-        for _ in range(2):
-            y = lay.forward(x).clone()
-        torch.cuda.synchronize()
         single = MoELayer(w, dict(shared, x=x), "cuda", update_bias=False)
-        y_ref = single.forward(x)
+        y_ref = single.forward(x).clone()
         torch.cuda.synchronize()
-        ok_fwd = bool(torch.equal(y[:w.T], y_ref[:w.T]))
+        ok_fwd = True
+        for device_plan in (False, True):
+            lay = EPMoELayer(w, shared, rank, 2, "cuda", exchange=ex, update_bias=False, recv_factor=1.0, peer=True,
+                             device_plan=device_plan)
+            for _ in range(2):
+                y = lay.forward(x).clone()
+            torch.cuda.synchronize()
+            ok_fwd = ok_fwd and bool(torch.equal(y[:w.T], y_ref[:w.T]))
+            ex.barrier()
+            lay.close()
+            ex.barrier()
         status = L.moe_device_status()
-        ex.barrier()
-        lay.close()
-        ex.barrier()
-        np.savez(os.path.join(out_dir, f"r{rank}.npz"), ok_map=ok_map, ok_fwd=ok_fwd, status=status,
-                 rounds=len(lay.plans))
+        np.savez(os.path.join(out_dir, f"r{rank}.npz"), ok_map=ok_map, ok_fwd=ok_fwd, status=status)
     finally:
         dist.destroy_process_group()
 
@@ -402,4 +408,3 @@ def test_ep_peer_two_processes_ipc(tmp_path):
         assert bool(z["ok_map"]), r
         assert bool(z["ok_fwd"]), r
         assert int(z["status"]) == L.MOE_OK
-        assert int(z["rounds"]) >= 1
