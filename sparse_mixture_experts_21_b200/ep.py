@@ -70,12 +70,16 @@ class _Works:
 
 
 class TorchDistExchange:
-    def __init__(self, group=None):
+    """device: where barrier() keeps its one-element flag (default: the current CUDA
+    device; "cpu" for a gloo group on the host)."""
+
+    def __init__(self, group=None, device=None):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
+        self.device = device
 
     def all_gather(self, t: torch.Tensor) -> torch.Tensor:
         out = torch.empty(self.world * t.numel(), dtype=t.dtype, device=t.device)
@@ -112,7 +116,8 @@ class TorchDistExchange:
         """Stream-ordered: the current stream's later work on any rank runs after every
         rank's earlier work (a one-element all-reduce)."""
         if not hasattr(self, "_flag"):
-            self._flag = torch.zeros(1, dtype=torch.int32, device=torch.cuda.current_device())
+            dev = self.device if self.device is not None else torch.cuda.current_device()
+            self._flag = torch.zeros(1, dtype=torch.int32, device=dev)
         self.dist.all_reduce(self._flag, group=self.group)
 
     def peer_addresses(self, t: torch.Tensor) -> List[int]:

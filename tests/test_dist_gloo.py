@@ -117,6 +117,51 @@ def test_ep_exchange_two_ranks(tmp_path):
         assert np.array_equal(r[rank]["back"], r[rank]["send"] + 1000.0)
 
 
+def _peer_worker(rank, port, out_dir):
+    """The peer exchange's host side on CPU (gloo): every rank exports a handle of its
+    buffer, the handles are all-gathered, each rank imports the others' and keeps its
+    own address; barrier() is a collective every rank passes; release_peer closes
+    exactly the imported addresses.  The library's CUDA IPC calls are replaced by
+    fakes that encode (rank, address) in the handle."""
+    import sparse_mixture_experts_21_b200.ep as E
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=EP_WORLD)
+    try:
+        closed = []
+        L = E.L
+        L.moe_peer_export = lambda t: (np.array([rank, t.data_ptr()], dtype=np.int64).tobytes()
+                                       + bytes(L.PEER_HANDLE_BYTES - 16))
+        L.moe_peer_import = lambda h: int(np.frombuffer(h[:16], dtype=np.int64)[1]) + 7   # "mapped" address
+        L.moe_peer_close = lambda a: closed.append(a)
+        ex = E.TorchDistExchange(device="cpu")
+        buf = torch.zeros(4, 8)
+        addrs = ex.peer_addresses(buf)
+        ex.barrier()
+        ex.barrier()
+        others = [a for r, a in enumerate(addrs) if r != rank]
+        for a in others:
+            ex.release_peer(a)
+        np.savez(os.path.join(out_dir, f"peer{rank}.npz"), addrs=np.array(addrs, dtype=np.int64),
+                 own=buf.data_ptr(), closed=np.array(closed, dtype=np.int64), flag=ex._flag.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_peer_handles_exchange_two_ranks(tmp_path):
+    mp.start_processes(_peer_worker, args=(_free_port(), str(tmp_path)), nprocs=EP_WORLD, join=True,
+                       start_method="spawn")
+    r = [np.load(tmp_path / f"peer{i}.npz") for i in range(EP_WORLD)]
+    for rank in range(EP_WORLD):
+        addrs = r[rank]["addrs"]
+        assert addrs[rank] == int(r[rank]["own"])                    # its own buffer, not imported
+        for o in range(EP_WORLD):
+            if o != rank:
+                assert addrs[o] == int(r[o]["own"]) + 7              # the other rank's handle, imported
+        assert sorted(r[rank]["closed"].tolist()) == sorted(int(addrs[o]) for o in range(EP_WORLD) if o != rank)
+        assert int(r[rank]["flag"][0]) == 0                          # the barrier's all-reduce of zeros
+
+
 # ----------------------------------------------------------------------------- global router statistics
 ST_N, ST_K, ST_T, ST_D = 16, 3, 120, 12
 
