@@ -248,7 +248,7 @@ nv_quant_scatter_kernel(const uint4* __restrict__ x, int64_t T, int k, int d, in
 // ---------------------------------------------------------------- grouped GEMM
 // One stage = 256 elements of K = 128 bytes of codes per row: A 16 KB, B 32 KB, and
 // twelve scale atoms (A: four chunks; B: two 128-row tiles x four chunks).
-constexpr int BM = 128, BKB = 128, BKE = 256, STAGES = 4;
+constexpr int BM = 128, BKB = 128, BKE = 256, STAGES = 3;
 constexpr int A_BYTES = BM * BKB;                // 16 KB
 constexpr int B_BYTES = 256 * BKB;               // 32 KB
 constexpr int ATOM = 512;
@@ -273,7 +273,11 @@ struct __align__(128) NvShared {
   int32_t tpre[kMaxGroups + 1];
 };
 
-constexpr size_t kSmem = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(NvShared);
+// The down pass stages its bf16 output through shared memory for TMA stores: one
+// 32-row x 32-column box (2 KB, 64-byte swizzle) per epilogue warp.
+constexpr int OUT_BOX = 2048;
+constexpr size_t kSharedPad = (sizeof(NvShared) + 1023) / 1024 * 1024;
+constexpr size_t kSmem = 1024 + (size_t)STAGES * STAGE_BYTES + kSharedPad + (size_t)EPI_WARPS * OUT_BOX;
 static_assert(kSmem <= 227 * 1024, "shared memory of the NVFP4 GEMM");
 
 __device__ __forceinline__ bool waitnv(uint64_t* bar, uint32_t parity, NvShared* sh) {
@@ -376,7 +380,8 @@ ffn_nv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
               const uint8_t* __restrict__ sfb0, const uint8_t* __restrict__ sfb1,
               const float* __restrict__ gb0, const float* __restrict__ gb1,
               const int32_t* __restrict__ offsets, int G, int K, int n_out, int64_t rows_cap,
-              uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_sf, __nv_bfloat16* __restrict__ out) {
+              uint8_t* __restrict__ out_q, uint8_t* __restrict__ out_sf, __nv_bfloat16* __restrict__ out,
+              const __grid_constant__ CUtensorMap tmY) {
   constexpr int BN = MODE == 0 ? 128 : 256;      // output columns per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -508,6 +513,9 @@ ffn_nv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     const int c_lo = MODE == 0 ? half * 64 : half * 128;
+    // down pass: this warp's output staging box (1024-aligned, for the 64-byte swizzle)
+    const uint32_t box = smem_u32(smem + (size_t)STAGES * STAGE_BYTES + kSharedPad) + (warp - 2) * OUT_BOX;
+    bool box_busy = false;                    // a TMA store may still be reading the box
     uint32_t tile_i = 0;
     for (int L = blockIdx.x; L < total; L += gridDim.x, ++tile_i) {
       const Tile t = decode(L, sh, G, tiles_n, BN);
@@ -524,6 +532,35 @@ ffn_nv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh->tempty);        // accumulator free for the next tile
+      if (MODE == 1 && q * 32 + 32 <= t.rows && t.n0 + c_lo < n_out) {
+        // all 32 rows of this warp are the group's: four 32 x 32 boxes through shared
+        // memory (lane l writes row l's 64 bytes, 16-byte chunk c at slot c ^ ((l >> 1) & 3),
+        // the 64-byte swizzle), fenced for the TMA engine, stored by lane 0; the store
+        // clips columns past the output.  A group's last, partial tile stores row by row.
+        const float s2 = gb0[t.g];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          if (box_busy) {
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = __fmul_rn(__uint_as_float(v[cc * 32 + c * 8 + i]), s2);
+            sts16(box + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), pack16(o, __nv_bfloat16()));
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, box, t.n0 + c_lo + cc * 32, t.row0 + q * 32);
+            bulk_commit();
+          }
+          box_busy = true;
+        }
+        continue;
+      }
       const int r = q * 32 + lane;
       const int64_t grow = (int64_t)t.row0 + r;
       if (r >= t.rows || grow >= rows_cap) continue;
@@ -573,6 +610,8 @@ ffn_nv_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         }
       }
     }
+    // every output box of this warp is in global memory before the kernel ends
+    if (MODE == 1 && lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -594,8 +633,12 @@ cudaError_t launch_nv(const CUtensorMap& a, const CUtensorMap& b0, const CUtenso
   const int64_t max_tiles = ((rows_cap + BM - 1) / BM + G) * tiles_n;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
   if (grid <= 0) return cudaSuccess;
+  // the down pass's output map (the gate/up pass writes no bf16 rows and never reads it)
+  CUtensorMap my{};
+  if (MODE == 1 && !make_map_bf16_store32(&my, out, (uint64_t)rows_cap, (uint64_t)n_out))
+    return cudaErrorInvalidValue;
   ffn_nv_kernel<MODE><<<grid, THREADS, kSmem, s>>>(a, b0, b1, sfa, sfb0, sfb1, gb0, gb1, offsets, G, K, n_out,
-                                                   rows_cap, out_q, out_sf, static_cast<__nv_bfloat16*>(out));
+                                                   rows_cap, out_q, out_sf, static_cast<__nv_bfloat16*>(out), my);
   return cudaGetLastError();
 }
 
