@@ -11,6 +11,7 @@
 * EPMoELayer(peer=True).forward for W ranks run as threads on one GPU: every rank's
   output equals the single-rank layer's on its tokens, in one round and in several, and
   with the plan kept on the device (receive buffers for every row a rank can receive);
+  rank 0's output is also within the bf16 bar of the oracle's layer forward;
 * two processes on one GPU with the library's CUDA IPC mapping: each imports the
   other's receive buffers and runs the peer forward, the barriers on the host (gloo
   plus a device synchronisation), so no kernel of one process waits for the other's.
@@ -31,6 +32,7 @@ from sparse_mixture_experts_21_b200 import _lib as L
 from sparse_mixture_experts_21_b200.ep import EPMoELayer, round_plans
 from sparse_mixture_experts_21_b200.layer import MoELayer
 from sparse_mixture_experts_21_b200.synth import WORKLOADS, make_inputs, random_routing
+from tests.parity_util import NEAR_TIE, TOL_BF16, expert_weights_fn, f64, i64, oracle_cfg, rel_err, shared_weights
 
 pytestmark = pytest.mark.gpu
 
@@ -300,6 +302,14 @@ def test_ep_peer_forward_threads_matches_single_rank(W, recv_factor, device_plan
     ref_bias = O.bias_update(bias0.double().cpu().numpy(), counts.cpu().numpy(), rate=w.bias_rate)
     for r in range(W):
         assert np.max(np.abs(weights[r]["bias"].double().cpu().numpy() - ref_bias)) < 1e-7
+    # rank 0's output against the oracle's layer forward on its tokens (dropless: tokens are
+    # independent), within the bf16 bar on the tokens whose expert choice is clear
+    out = O.layer_forward(f64(xs[0]), f64(shared["w_gate"]), oracle_cfg(w), expert_weights_fn(shared),
+                          shared_weights(shared), bias=f64(bias0))
+    clear = out["routing"]["margin"] >= NEAR_TIE
+    assert clear.mean() > 0.95
+    assert np.array_equal(i64(layers[0].base.topk_idx)[clear], out["routing"]["idx"][clear])
+    assert rel_err(f64(ys[0][:w.T])[clear], out["y"][clear]) < TOL_BF16
 
 
 # ----------------------------------------------------------------------------- two processes, CUDA IPC
