@@ -24,18 +24,16 @@
 // on the same stages.
 //
 // No padding rows.  A group of R rows is cut into floor(R / 128) full 128-row
-// sub-tiles (paired two by two; with an even count and a tail, the last two run as a
-// SINGLE and an ST instead) and a ragged tail of r = R mod 128 rows.  The tail
+// sub-tiles (paired two by two) and a ragged tail of r = R mod 128 rows.  The tail
 // is computed transposed ("swapped"): the weight tile already in shared memory is
 // the MMA's A operand (M = 128 weight rows, i.e. output columns) and the r tail rows
 // are its B operand (N = r rounded up to 16), so the tail costs its own MMA work,
 // not that of a 128-row tile, and reuses the weight stages of the group's last full
 // sub-tile.  Kinds of tile:
 //   PAIR   two full sub-tiles;
-//   SINGLE one full sub-tile, no tail (an odd count of full sub-tiles without a tail,
-//          or the first of the last two of an even count with a tail);
+//   SINGLE one full sub-tile (an odd count of full sub-tiles), no tail;
 //   ST     one full sub-tile + the group's tail as sub-tile 1 (swapped);
-//   T      the tail alone (R < 128).
+//   T      the tail alone (an even count of full sub-tiles, or R < 128).
 // The swapped sub-tile writes D^T into accumulator 1: weight rows 0..127 into
 // columns [0, n) and rows 128..255 into columns [128, 128 + n) (gate/up: W1 and W3,
 // so gate and up of one hidden unit share a TMEM lane; down: the two 128-column
@@ -150,26 +148,17 @@ __device__ __forceinline__ Tile decode_tile(int L, const TcShared* sh, int G, in
   const int n_tile = local / per, j = local - n_tile * per;
   const int rows = sh->goff[g + 1] - sh->goff[g];
   const int full = rows / SUB, r = rows - full * SUB;
-  // an even count (>= 2) of full sub-tiles with a tail: the last pair becomes a SINGLE
-  // and an ST, so the tail shares a weight stream with a full sub-tile instead of
-  // streaming the weight tile alone (same tile count)
-  const bool split = !(full & 1) && full >= 2 && r > 0;
-  const int pairs = split ? full / 2 - 1 : full / 2;
   t.g = g;
   t.n0 = n_tile * BN;
-  t.trow0 = 0;
-  t.tr = 0;
-  t.tn = 0;
-  if (j < pairs) {
+  if (j < full / 2) {
     t.kind = K_PAIR;
     t.row0 = sh->goff[g] + j * 2 * SUB;
-  } else if (split && j == pairs) {
-    t.kind = K_SINGLE;
-    t.row0 = sh->goff[g] + (full - 2) * SUB;
+    t.trow0 = 0;
+    t.tr = 0;
+    t.tn = 0;
   } else {
-    // the group's last tile: its last full sub-tile (if any) and its tail (if any)
-    t.kind = full == 0 ? K_T : (r > 0 ? K_ST : K_SINGLE);
-    t.row0 = sh->goff[g] + (full > 0 ? full - 1 : 0) * SUB;
+    t.kind = (full & 1) ? (r > 0 ? K_ST : K_SINGLE) : K_T;
+    t.row0 = sh->goff[g] + (full & ~1) * SUB;
     t.trow0 = sh->goff[g + 1] - r;
     t.tr = r;
     t.tn = (r + TAIL_BOX - 1) / TAIL_BOX * TAIL_BOX;
@@ -177,9 +166,7 @@ __device__ __forceinline__ Tile decode_tile(int L, const TcShared* sh, int G, in
   return t;
 }
 
-// Tiles of a group of `rows` rows per n-tile: floor(full / 2) + 1 with an odd count of
-// full sub-tiles or a tail (the PAIRs, then SINGLE / ST / T as decode_tile assigns them),
-// floor(full / 2) otherwise.
+// Tiles of a group of `rows` rows per n-tile: its PAIR tiles + at most one more.
 __device__ __forceinline__ int group_tiles(int rows) {
   const int full = rows / SUB;
   return full / 2 + (((full & 1) || rows % SUB) ? 1 : 0);
