@@ -312,6 +312,51 @@ def test_ep_peer_forward_threads_matches_single_rank(W, recv_factor, device_plan
     assert rel_err(f64(ys[0][:w.T])[clear], out["y"][clear]) < TOL_BF16
 
 
+@pytest.mark.parametrize("device_plan", [False, True])
+def test_ep_peer_forward_one_rank_receives_nothing(device_plan):
+    """A selection bias that sends every token to rank 0's experts: rank 1's experts get no
+    rows (an empty grouped FFN), rank 1's combine reads every result from rank 0's buffer,
+    and both ranks still equal the single-rank layer."""
+    import threading
+    W = 2
+    w = _case()
+    shared = make_inputs(w, "cuda", seed=0)
+    El = w.N // W
+    bias = torch.zeros_like(shared["bias"])
+    bias[:El] = 10.0                                   # experts of rank 0 win every selection
+    xs = [make_inputs(w, "cuda", seed=120 + r, experts=False)["x"] for r in range(W)]
+    hub = _Hub(W)
+    weights = [dict(shared, bias=bias.clone()) for _ in range(W)]
+    layers = [EPMoELayer(w, weights[r], r, W, "cuda", exchange=_ThreadPeerExchange(hub, r), update_bias=False,
+                         peer=True, device_plan=device_plan) for r in range(W)]
+    ys, errs = [None] * W, []
+
+    def run(r):
+        try:
+            with torch.cuda.stream(torch.cuda.Stream()):
+                ys[r] = layers[r].forward(xs[r]).clone()
+                torch.cuda.current_stream().synchronize()
+        except Exception as e:          # reported below
+            errs.append(e)
+            hub.barrier.abort()
+
+    th = [threading.Thread(target=run, args=(r,)) for r in range(W)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errs, errs
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert int(layers[1].local_offsets[0][El].item()) == 0      # rank 1 computed nothing
+    assert torch.all(layers[0].base.topk_idx < El) and torch.all(layers[1].base.topk_idx < El)
+    for r in range(W):
+        single = MoELayer(w, dict(shared, x=xs[r], bias=bias.clone()), "cuda", update_bias=False)
+        y_ref = single.forward(xs[r])
+        torch.cuda.synchronize()
+        assert torch.equal(ys[r][:w.T], y_ref[:w.T]), r
+
+
 # ----------------------------------------------------------------------------- two processes, CUDA IPC
 def _free_port():
     with socket.socket() as s:
