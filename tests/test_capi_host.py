@@ -30,6 +30,22 @@ def test_library_exports_every_declared_symbol(lib):
         assert getattr(lib, name) is not None
 
 
+def test_header_is_plain_c(tmp_path):
+    """include/moe_b200.h compiles as strict C99 and as C++ (plain pointers and sizes, no
+    torch or CUDA types in the signatures)."""
+    import shutil
+    import subprocess
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "moe_b200.h"\nint main(void) { return 0; }\n')
+    inc = os.path.join(ROOT, "include")
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-I", inc,
+                    str(src)], check=True)
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Werror", "-fsyntax-only", "-I", inc, "-x", "c++", str(src)],
+                   check=True)
+
+
 def test_config_struct_layout():
     assert ctypes.sizeof(L.MoeConfig) == 64
     assert L.MoeConfig.capacity_factor.offset == 56
