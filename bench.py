@@ -50,6 +50,11 @@ NCU_TRAFFIC = {
 }
 
 
+# The shared expert's first pass (its W1/W3 once, its rows x 4 from the same reduced capture):
+# DRAM bytes that leave the grouped-FFN stage when that pass runs on a side stream.
+SPLIT_SHARED_GATE_UP_BYTES = {"deepseek_v3": 0.58e9}
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -394,6 +399,10 @@ def main():
     ap.add_argument("--no-fuse-shared", action="store_true",
                     help="run the shared expert in launches of its own instead of as one more group of the "
                          "routed grouped-FFN launches")
+    ap.add_argument("--no-split-shared", action="store_true",
+                    help="bf16, shared expert fused: run both of its passes inside the routed launches (default: "
+                         "its first pass on a side stream during route and permute, its second pass inside the "
+                         "routed down launch)")
     ap.add_argument("--gather-rows", action="store_true",
                     help="bf16: the grouped FFN gathers its rows from x (cp.async) instead of reading the "
                          "expert-ordered copy that the permutation writes")
@@ -439,7 +448,8 @@ def main():
         return run_ep(args, w, world, rank, local, dev, pg)
     inp = make_inputs(w, dev, seed=rank)
     lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD, overlap_shared=not args.no_overlap_shared,
-                   gather_rows=args.gather_rows, fuse_shared=not args.no_fuse_shared)
+                   gather_rows=args.gather_rows, fuse_shared=not args.no_fuse_shared,
+                   split_shared=not args.no_split_shared)
     x = inp["x"]
     stream = torch.cuda.current_stream(dev)
 
@@ -506,13 +516,19 @@ def main():
         ffn_peak, ffn_bound = 148 * 128 * 2 * 1.965e9 / 1e12, "alu"
         ffn_peak_src = "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1965 MHz"
     # with the shared expert fused into the routed launches, the stage does both
-    flops_ffn = flops_routed + (flops_shared if lay.fuse_shared else 0.0)
+    # (split: the shared expert's first pass runs on a side stream before the stage, its
+    # second pass -- a third of its FLOPs -- inside the stage's down launch)
+    flops_ffn = flops_routed + (flops_shared / 3.0 if lay.split_shared else flops_shared if lay.fuse_shared
+                                else 0.0)
     tflops_ffn = flops_ffn / (t_ffn * 1e-3) / 1e12
     traffic = None
     if w.name in NCU_TRAFFIC:
         srcs, nbytes = NCU_TRAFFIC[w.name]
         if all(_sha1(os.path.join(ROOT, "sparse_mixture_experts_21_b200", "csrc", f)) == h for f, h in srcs.items()):
             traffic = nbytes
+            if lay.split_shared and w.name in SPLIT_SHARED_GATE_UP_BYTES:
+                # the stage no longer holds the shared expert's first pass
+                traffic -= SPLIT_SHARED_GATE_UP_BYTES[w.name]
 
     # the same step replayed from a CUDA graph (one capture, K replays): launch overhead out
     graph = None
@@ -573,7 +589,9 @@ def main():
                                f"{3 * N * d * f * (0.5 if w.nvfp4 else 1 if lowp else eb) / 1e9:.1f} GB); "
                                "no flush")),
             "tflops": (flops_routed + flops_shared + flops_router) / (ms * 1e-3) / 1e12,
-            "roofline": {"kernel": ("grouped SwiGLU FFN, routed + shared experts in one tile list (gate/up + "
+            "roofline": {"kernel": ("grouped SwiGLU FFN, routed gate/up pass + routed and shared down pass"
+                                    if lay.split_shared else
+                                    "grouped SwiGLU FFN, routed + shared experts in one tile list (gate/up + "
                                     "down passes)" if lay.fuse_shared else
                                     "grouped SwiGLU FFN, routed experts (gate/up + down passes)"),
                          "bound": ffn_bound, "achieved": tflops_ffn,
@@ -590,7 +608,9 @@ def main():
             # experts; the main stream's "shared_ffn" stage is then only the join
             "shared_ffn_tflops": (None if (lay.overlap_shared or lay.fuse_shared or lay.fs == 0)
                                   else flops_shared / (t_shared * 1e-3) / 1e12),
-            "shared_experts": ("fused into the routed grouped-FFN launches" if lay.fuse_shared else
+            "shared_experts": ("first pass on a side stream during route and permute, second pass in the "
+                               "routed down launch" if lay.split_shared else
+                               "fused into the routed grouped-FFN launches" if lay.fuse_shared else
                                "side stream (overlapped)" if lay.overlap_shared else
                                "main stream" if lay.fs > 0 else "none"),
             "router_tflops_fp32": flops_router / (t_route * 1e-3) / 1e12,

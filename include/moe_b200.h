@@ -259,6 +259,30 @@ int moe_grouped_ffn_shared(const moe_config_t* cfg, const void* x_rows, int64_t 
                            const void* ws3, const void* ws2, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_grouped_ffn_gate_up, moe_grouped_ffn_down -- the two passes of moe_grouped_ffn
+ * as separate calls (bf16), so a caller can run the shared expert's first pass on
+ * another stream while the router and the permutation run, and its second pass in
+ * the routed second pass's launch.  Same kernels and arithmetic as moe_grouped_ffn
+ * and moe_grouped_ffn_shared: bit-identical results.
+ *
+ * moe_grouped_ffn_gate_up: h_rows[r] = silu(x_rows[r] W1[g]^T) * (x_rows[r] W3[g]^T)
+ *   for the rows r of each group g.  x_rows [rows_cap, d], w1/w3 [G, f, d], h_rows
+ *   [rows_cap, f] (bf16); offsets [G+1] (device).  G <= 512.
+ * moe_grouped_ffn_down: y_rows[r] = h_rows[r] W2[g]^T for the groups' rows; with T > 0
+ *   and ws2 [d, f] also y_rows[rows_cap + t] = h_rows[rows_cap + t] ws2^T for t < T (the
+ *   shared expert's rows, whose first pass the caller ran), in the same launch.  h_rows
+ *   [rows_cap + T, f], y_rows [rows_cap + T, d].  G <= 511.
+ * Errors: MOE_ERR_UNSUPPORTED unless cfg->x_dtype is bf16, or when the rows exceed
+ * INT32_MAX; MOE_ERR_INVALID_ARG for a bad G, f, rows_cap or T, for T > 0 without ws2
+ * (or ws2 with T = 0), or a NULL or misaligned buffer.  No rows is a no-op.
+ * ------------------------------------------------------------------------- */
+int moe_grouped_ffn_gate_up(const moe_config_t* cfg, const void* x_rows, int64_t rows_cap, const int32_t* offsets,
+                            int32_t G, const void* w1, const void* w3, int32_t f, void* h_rows, void* stream);
+int moe_grouped_ffn_down(const moe_config_t* cfg, const void* h_rows, int64_t rows_cap, const int32_t* offsets,
+                         int32_t G, const void* w2, int32_t f, void* y_rows, int64_t T, const void* ws2,
+                         void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_grouped_ffn_gather -- moe_grouped_ffn reading each row straight from x.
  *
  * The same grouped SwiGLU FFN (same sources, same arithmetic, bit-identical

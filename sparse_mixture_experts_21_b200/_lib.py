@@ -24,7 +24,8 @@ DTYPE_F32, DTYPE_BF16 = 0, 1
 CAP_DROPLESS, CAP_CEIL_CF_T_OVER_N, CAP_CF_K_T_OVER_N_FLOOR = 0, 1, 2
 
 EXPORTED = ("moe_capacity", "moe_route_partials", "moe_workspace_size", "moe_route", "moe_permute",
-            "moe_grouped_ffn", "moe_grouped_ffn_shared", "moe_grouped_ffn_gather", "moe_combine", "moe_router_stats", "moe_bias_update",
+            "moe_grouped_ffn", "moe_grouped_ffn_shared", "moe_grouped_ffn_gather", "moe_grouped_ffn_gate_up",
+            "moe_grouped_ffn_down", "moe_combine", "moe_router_stats", "moe_bias_update",
             "moe_device_status", "moe_status_string", "moe_permute_noalloc", "moe_bias_update_ema",
             "moe_bias_update_seq", "moe_route_scores", "moe_expert_choice", "moe_combine_ec",
             "moe_selftest_wait_timeout", "moe_quantize_fp8", "moe_permute_fp8", "moe_grouped_ffn_fp8",
@@ -93,6 +94,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_grouped_ffn": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp],
         "moe_grouped_ffn_shared": [cfgp, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp, c_int64, vp, vp,
                                    vp, vp],
+        "moe_grouped_ffn_gate_up": [cfgp, vp, c_int64, vp, c_int32, vp, vp, c_int32, vp, vp],
+        "moe_grouped_ffn_down": [cfgp, vp, c_int64, vp, c_int32, vp, c_int32, vp, c_int64, vp, vp],
         "moe_grouped_ffn_gather": [cfgp, vp, c_int64, vp, c_int64, vp, c_int32, vp, vp, vp, c_int32, vp, vp, vp, vp,
                                    vp, vp],
         "moe_combine": [cfgp, vp, vp, vp, vp, vp, vp, vp],
@@ -237,6 +240,21 @@ def moe_grouped_ffn_shared(cfg, x_rows, rows_cap, offsets, G, w1, w3, w2, f, h_s
     _check("moe_grouped_ffn_shared", load().moe_grouped_ffn_shared(
         ctypes.byref(cfg), _ptr(x_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1), _ptr(w3), _ptr(w2), int(f),
         _ptr(h_scratch), _ptr(y_rows), _ptr(x), int(T), _ptr(ws1), _ptr(ws3), _ptr(ws2), _stream(stream)))
+
+
+def moe_grouped_ffn_gate_up(cfg, x_rows, rows_cap, offsets, G, w1, w3, f, h_rows, stream=None):
+    """The first pass of moe_grouped_ffn alone (bf16): h = silu(x W1^T) * (x W3^T) per group."""
+    _check("moe_grouped_ffn_gate_up", load().moe_grouped_ffn_gate_up(
+        ctypes.byref(cfg), _ptr(x_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w1), _ptr(w3), int(f),
+        _ptr(h_rows), _stream(stream)))
+
+
+def moe_grouped_ffn_down(cfg, h_rows, rows_cap, offsets, G, w2, f, y_rows, T=0, ws2=None, stream=None):
+    """The second pass alone (bf16): y = h W2^T per group; with T and ws2, also the shared
+    expert's T rows after rows_cap through ws2, in the same launch."""
+    _check("moe_grouped_ffn_down", load().moe_grouped_ffn_down(
+        ctypes.byref(cfg), _ptr(h_rows), int(rows_cap), _ptr(offsets), int(G), _ptr(w2), int(f), _ptr(y_rows),
+        int(T), _ptr(ws2), _stream(stream)))
 
 
 def moe_grouped_ffn_gather(cfg, x, T, token_of_row, rows_cap, offsets, G, w1, w3, w2, f, h_scratch, y_rows,

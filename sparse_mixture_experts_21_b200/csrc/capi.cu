@@ -243,6 +243,37 @@ int moe_grouped_ffn_shared(const moe_config_t* cfg, const void* x_rows, int64_t 
                                           y_rows, x, (int)T, ws1, ws3, ws2, static_cast<cudaStream_t>(stream)));
 }
 
+int moe_grouped_ffn_gate_up(const moe_config_t* cfg, const void* x_rows, int64_t rows_cap, const int32_t* offsets,
+                            int32_t G, const void* w1, const void* w3, int32_t f, void* h_rows, void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->x_dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < 0 || G < 1 || G > 512 || f <= 0 || (f % 8) != 0 || !offsets) return MOE_ERR_INVALID_ARG;
+  if (rows_cap == 0) return MOE_OK;
+  if (rows_cap > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (!x_rows || !w1 || !w3 || !h_rows) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_rows) || !aligned16(w1) || !aligned16(w3) || !aligned16(h_rows)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_ffn_bf16_gate_up(x_rows, rows_cap, offsets, G, w1, w3, cfg->d_model, f, h_rows,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int moe_grouped_ffn_down(const moe_config_t* cfg, const void* h_rows, int64_t rows_cap, const int32_t* offsets,
+                         int32_t G, const void* w2, int32_t f, void* y_rows, int64_t T, const void* ws2,
+                         void* stream) {
+  const int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->x_dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (rows_cap < 0 || T < 0 || G < 1 || G > 511 || f <= 0 || (f % 8) != 0 || !offsets) return MOE_ERR_INVALID_ARG;
+  if ((T > 0) != (ws2 != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (rows_cap + T == 0) return MOE_OK;
+  if (rows_cap + T > (int64_t)INT32_MAX) return MOE_ERR_UNSUPPORTED;
+  if (!h_rows || !w2 || !y_rows) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h_rows) || !aligned16(w2) || !aligned16(y_rows) || (ws2 && !aligned16(ws2)))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(launch_ffn_bf16_down(h_rows, rows_cap, offsets, G, w2, cfg->d_model, f, y_rows, (int)T, ws2,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 int moe_grouped_ffn_gather(const moe_config_t* cfg, const void* x, int64_t T, const int32_t* token_of_row,
                            int64_t rows_cap, const int32_t* offsets, int32_t G, const void* w1, const void* w3,
                            const void* w2, int32_t f, void* h_scratch, void* y_rows, const void* ws1,

@@ -54,6 +54,10 @@ cudaError_t launch_ffn_bf16(const void* x_rows, int64_t rows_cap, const int32_t*
 // The same FFN plus one dense group of Ts rows (xs [Ts, d], its own ws1/ws3 [f, d],
 // ws2 [d, f]) in the same two launches; h [rows_cap + Ts, f] and y [rows_cap + Ts, d]
 // hold its rows after the groups' rows_cap rows.
+cudaError_t launch_ffn_bf16_gate_up(const void* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
+                                    const void* w1, const void* w3, int d, int f, void* h, cudaStream_t s);
+cudaError_t launch_ffn_bf16_down(const void* h, int64_t rows_cap, const int32_t* offsets, int G, const void* w2,
+                                 int d, int f, void* y, int Ts, const void* ws2, cudaStream_t s);
 cudaError_t launch_ffn_bf16_shared(const void* x_rows, int64_t rows_cap, const int32_t* offsets, int G,
                                    const void* w1, const void* w3, const void* w2, int d, int f, void* h, void* y,
                                    const void* xs, int Ts, const void* ws1, const void* ws3, const void* ws2,

@@ -36,7 +36,7 @@ class MoELayer:
 
     def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True,
                  group=None, overlap_shared: bool = True, gather_rows: bool = False,
-                 fuse_shared: bool = True):
+                 fuse_shared: bool = True, split_shared: bool = True):
         """group: a torch.distributed process group when the layer runs as one of
         several data-parallel replicas; the router statistics are then those of the
         whole group's batch (each rank's sufficient statistics summed over the
@@ -68,6 +68,10 @@ class MoELayer:
                             and w.n_shared * w.f_shared == w.f and w.N < 512)
         if self.fuse_shared:
             self.overlap_shared = False
+        # split_shared (with fuse_shared): the shared expert's first pass on a side stream,
+        # concurrently with route and permute; its second pass inside the routed second
+        # pass's launch (moe_grouped_ffn_gate_up / moe_grouped_ffn_down)
+        self.split_shared = split_shared and self.fuse_shared and not self.gather_rows
         self.dev = torch.device(device)
         self.weights = weights
         self.update_bias = update_bias and weights.get("bias") is not None
@@ -205,18 +209,23 @@ class MoELayer:
             return self._forward_ec(x, s, rec, y)
         rec(0)
         join = None
-        if self.overlap_shared:
+        side_work = self.overlap_shared or self.split_shared
+        if side_work:
             fork = torch.cuda.Event()
             fork.record(s)
         self.route(x, s)
-        if self.overlap_shared:
+        if side_work:
             if not hasattr(self, "_side"):
                 self._side = torch.cuda.Stream(self.dev)
             side = self._side
             side.wait_event(fork)
             with torch.cuda.stream(side):
-                L.moe_grouped_ffn(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], self.fs, self.hs,
-                                  self.ys, side)
+                if self.split_shared:
+                    L.moe_grouped_ffn_gate_up(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], self.fs, self.hs,
+                                              side)
+                else:
+                    L.moe_grouped_ffn(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], W["ws2"], self.fs,
+                                      self.hs, self.ys, side)
             join = torch.cuda.Event()
             join.record(side)
         rec(1)
@@ -240,6 +249,13 @@ class MoELayer:
             sw = (W["ws1"], W["ws3"], W["ws2"]) if self.fuse_shared else (None, None, None)
             L.moe_grouped_ffn_gather(c, x, T, self.token_of_row, T * self.w.k, self.offsets, self.w.N, W["w1"],
                                      W["w3"], W["w2"], self.w.f, self.h, self.y_perm, s, *sw)
+        elif self.split_shared:
+            L.moe_grouped_ffn_gate_up(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
+                                      self.w.f, self.h, s)
+            s.wait_event(join)                 # the shared expert's first pass
+            join = None
+            L.moe_grouped_ffn_down(c, self.h, T * self.w.k, self.offsets, self.w.N, W["w2"], self.w.f, self.y_perm,
+                                   T, W["ws2"], s)
         elif self.fuse_shared:
             L.moe_grouped_ffn_shared(c, self.x_perm, T * self.w.k, self.offsets, self.w.N, W["w1"], W["w3"],
                                      W["w2"], self.w.f, self.h, self.y_perm, x, T, W["ws1"], W["ws3"], W["ws2"], s)
@@ -386,6 +402,8 @@ class MoELayer:
             n -= 1                     # no row gather: the grouped FFN reads x itself
         if self.fs > 0 and not self.fuse_shared:
             n += 2
+        if self.split_shared:
+            n += 1                     # the shared expert's first pass in a launch of its own
         if self.update_bias:
             n += 1
         return n

@@ -175,6 +175,29 @@ def test_gathering_ffn_checks(lib):
     assert f(cp, ok, 100, ok, 800, ok, 256, ok, ok, ok, 2048, ok, ok) == UN
 
 
+def test_ffn_pass_entry_checks(lib):
+    """moe_grouped_ffn_gate_up / moe_grouped_ffn_down: bf16 only, G and f in range, the
+    shared rows only with their weights; no rows is a no-op.  Nothing here reaches the GPU."""
+    ok, UN, IA = 0x1000000, L.MOE_ERR_UNSUPPORTED, L.MOE_ERR_INVALID_ARG
+    c = layer.make_config(synth.WORKLOADS["deepseek_v3"])
+    cp = ctypes.byref(c)
+    gu, dn = lib.moe_grouped_ffn_gate_up, lib.moe_grouped_ffn_down
+    assert gu(cp, ok, 100, ok, 0, ok, ok, 2048, ok, None) == IA             # G
+    assert gu(cp, ok, 100, ok, 513, ok, ok, 2048, ok, None) == IA
+    assert gu(cp, ok, 100, ok, 4, ok, ok, 2047, ok, None) == IA             # f % 8
+    assert gu(cp, ok + 8, 100, ok, 4, ok, ok, 2048, ok, None) == IA         # misaligned rows
+    assert gu(cp, None, 0, ok, 4, None, None, 2048, None, None) == L.MOE_OK
+    assert dn(cp, ok, 100, ok, 512, ok, 2048, ok, 0, None, None) == IA      # G: one slot for the shared
+    assert dn(cp, ok, 100, ok, 4, ok, 2048, ok, 10, None, None) == IA       # shared rows without ws2
+    assert dn(cp, ok, 100, ok, 4, ok, 2048, ok, 0, ok, None) == IA          # ws2 without shared rows
+    assert dn(cp, ok, 100, ok, 4, ok, 2048, ok, -1, None, None) == IA
+    assert dn(cp, ok, 100, ok, 4, ok, 2048, ok + 4, 0, None, None) == IA    # misaligned y
+    assert dn(cp, None, 0, ok, 4, None, 2048, None, 0, None, None) == L.MOE_OK
+    c32 = layer.make_config(synth.WORKLOADS["tiny_top2_fp32"])
+    assert gu(ctypes.byref(c32), ok, 10, ok, 8, ok, ok, 256, ok, None) == UN
+    assert dn(ctypes.byref(c32), ok, 10, ok, 8, ok, 256, ok, 0, None, None) == UN
+
+
 def test_fused_shared_ffn_checks(lib):
     """moe_grouped_ffn_shared: bf16 only, G <= 511, every buffer present and aligned;
     no shared rows is moe_grouped_ffn.  Nothing here reaches the GPU."""

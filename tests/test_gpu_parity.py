@@ -478,6 +478,59 @@ def test_layer_fused_shared_expert_equals_separate(name):
     assert torch.equal(a.ys[:w.T], b.ys[:w.T])
 
 
+@pytest.mark.parametrize("name", ["v3_small"])
+def test_layer_split_shared_expert_equals_fused(name):
+    """The shared expert's first pass on a side stream and its second pass inside the
+    routed down launch give the fused layer's output bit for bit."""
+    w = SMALL[name]
+    inp = make_inputs(w, "cuda")
+    a = MoELayer(w, inp, "cuda", update_bias=False, fuse_shared=True, split_shared=False)
+    b = MoELayer(w, inp, "cuda", update_bias=False, fuse_shared=True, split_shared=True)
+    assert b.split_shared and not a.split_shared
+    ya = a.forward(inp["x"]).clone()
+    for _ in range(2):
+        yb = b.forward(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(ya, yb)
+    assert torch.equal(a.ys[:w.T], b.ys[:w.T])
+
+
+@pytest.mark.parametrize("d,f,sizes,T", [
+    (256, 384, [0, 1, 127, 0, 128, 129, 300, 0], 613),
+    (384, 256, [16, 17, 255, 256, 257, 5], 200),
+])
+def test_grouped_ffn_passes_equal_fused_shared(d, f, sizes, T):
+    """moe_grouped_ffn_gate_up on the routed rows and on x (the shared expert), then
+    moe_grouped_ffn_down with the shared weights, equal moe_grouped_ffn_shared bit for bit."""
+    G = len(sizes)
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    R, cap = int(off[-1]), int(off[-1]) + 40
+    g = torch.Generator(device="cuda").manual_seed(31)
+    x = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+    xr = torch.randn(cap, d, generator=g, device="cuda").to(torch.bfloat16)
+    w1 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w3 = (torch.randn(G, f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    w2 = (torch.randn(G, d, f, generator=g, device="cuda") / f ** 0.5).to(torch.bfloat16)
+    ws1 = (torch.randn(f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    ws3 = (torch.randn(f, d, generator=g, device="cuda") / d ** 0.5).to(torch.bfloat16)
+    ws2 = (torch.randn(d, f, generator=g, device="cuda") / f ** 0.5).to(torch.bfloat16)
+    offs = torch.tensor(off, device="cuda")
+    cfg = make_config(replace(SMALL["mixtral_small"], d=d, f=f, N=G, T=T))
+    h0, h1 = (torch.empty(cap + T, f, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    y0, y1 = (torch.full((cap + T, d), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(2))
+    L.moe_device_status()
+    L.moe_grouped_ffn_shared(cfg, xr, cap, offs, G, w1, w3, w2, f, h0, y0, x, T, ws1, ws3, ws2)
+    L.moe_grouped_ffn_gate_up(cfg, x, T, torch.tensor([0, T], dtype=torch.int32, device="cuda"), 1, ws1, ws3, f,
+                              h1[cap:])
+    L.moe_grouped_ffn_gate_up(cfg, xr, cap, offs, G, w1, w3, f, h1)
+    L.moe_grouped_ffn_down(cfg, h1, cap, offs, G, w2, f, y1, T, ws2)
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(h1[:R], h0[:R]) and torch.equal(h1[cap:], h0[cap:])
+    assert torch.equal(y1, y0)
+
+
 @pytest.mark.parametrize("d,f,sizes", [
     (256, 384, [0, 1, 127, 0, 128, 129, 300, 0]),
     (384, 320, [16, 17, 112, 113, 255, 256, 257, 383, 384, 385, 511, 640, 5, 0, 31]),
