@@ -394,8 +394,9 @@ def main():
                     help="replicas: every rank holds every expert; ep: expert parallelism (N / W experts per "
                          "rank, all-to-all dispatch and return)")
     ap.add_argument("--no-overlap-shared", action="store_true",
-                    help="run the shared experts on the main stream after the routed experts (default: on a "
-                         "side stream, concurrently with route and permute)")
+                    help="run the shared experts on the main stream after the routed experts (default: bf16 "
+                         "shared experts that are not fused run on a side stream, concurrently with route and "
+                         "permute; low-precision ones on the main stream)")
     ap.add_argument("--no-fuse-shared", action="store_true",
                     help="run the shared expert in launches of its own instead of as one more group of the "
                          "routed grouped-FFN launches")
@@ -447,7 +448,7 @@ def main():
     if args.parallel == "ep":
         return run_ep(args, w, world, rank, local, dev, pg)
     inp = make_inputs(w, dev, seed=rank)
-    lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD, overlap_shared=not args.no_overlap_shared,
+    lay = MoELayer(w, inp, dev, group=None if pg is None else pg.group.WORLD, overlap_shared=False if args.no_overlap_shared else None,
                    gather_rows=args.gather_rows, fuse_shared=not args.no_fuse_shared,
                    split_shared=not args.no_split_shared)
     x = inp["x"]

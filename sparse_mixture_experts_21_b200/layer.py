@@ -35,7 +35,7 @@ class MoELayer:
     """Holds the weights and the per-call buffers of one layer for up to T tokens."""
 
     def __init__(self, w: Workload, weights: dict, device="cuda", update_bias: bool = True,
-                 group=None, overlap_shared: bool = True, gather_rows: bool = False,
+                 group=None, overlap_shared: Optional[bool] = None, gather_rows: bool = False,
                  fuse_shared: bool = True, split_shared: bool = True):
         """group: a torch.distributed process group when the layer runs as one of
         several data-parallel replicas; the router statistics are then those of the
@@ -51,9 +51,14 @@ class MoELayer:
             raise ValueError("NVFP4 experts need d and d_ff multiples of 256")
         self.w = w
         self.group = group
-        # bf16 shared experts on a side stream, concurrently with route and permute (they
-        # do not depend on the routing); joined before the combine
-        self.overlap_shared = overlap_shared and not lowp and w.n_shared > 0
+        # shared experts on a side stream, concurrently with route and permute (they do not
+        # depend on the routing); joined before the combine.  With low-precision experts the
+        # side stream also quantises x for them (the quantising scatter then writes only
+        # the routed rows).  None: on for bf16 experts, off for low-precision ones, where
+        # it measured no faster (the step is power-bound and the overlap adds no work saved)
+        if overlap_shared is None:
+            overlap_shared = not lowp
+        self.overlap_shared = overlap_shared and w.n_shared > 0 and not w.expert_choice
         # gather_rows: bf16 experts read their rows straight from x (moe_grouped_ffn_gather),
         # so the permutation writes no expert-ordered copy of x (T k d elements less
         # memory); off by default: the first GEMM's row copies cost more time than the
@@ -207,6 +212,7 @@ class MoELayer:
         rec = (lambda i: marks[i].record(s)) if marks is not None else (lambda i: None)
         if self.w.expert_choice:
             return self._forward_ec(x, s, rec, y)
+        lowp = self.w.fp8 or self.w.mxfp8 or self.w.nvfp4
         rec(0)
         join = None
         side_work = self.overlap_shared or self.split_shared
@@ -220,7 +226,16 @@ class MoELayer:
             side = self._side
             side.wait_event(fork)
             with torch.cuda.stream(side):
-                if self.split_shared:
+                if lowp:
+                    if self.w.nvfp4:
+                        L.moe_quantize_nvfp4(x, self.xq, self.xs, stream=side)
+                    elif self.w.mxfp8:
+                        L.moe_quantize_mxfp8(x, self.xq, self.xs, side)
+                    else:
+                        L.moe_quantize_fp8(x, 1, self.xq, self.xs, side)
+                    self._ffn_fp8(c, self.xq, self.xs, T, self.shared_offsets, 1, ("ws1", "ws3", "ws2"), self.fs,
+                                  self.hq_sh, self.hsc_sh, self.ys, side)
+                elif self.split_shared:
                     L.moe_grouped_ffn_gate_up(c, x, T, self.shared_offsets, 1, W["ws1"], W["ws3"], self.fs, self.hs,
                                               side)
                 else:
@@ -229,18 +244,19 @@ class MoELayer:
             join = torch.cuda.Event()
             join.record(side)
         rec(1)
-        fp8 = self.w.fp8 or self.w.mxfp8 or self.w.nvfp4
+        fp8 = lowp
+        tok = self.fs > 0 and not self.overlap_shared     # the shared experts' input, from the scatter
         L.moe_permute(c, x, self.topk_idx, self.counts, self.offsets, self.row_of_slot,
                       self.token_of_row, self.x_perm, self.n_dropped, self.ws, s)
         if self.w.nvfp4:
             L.moe_permute_nvfp4(c, x, self.topk_idx, self.row_of_slot, self.offsets, self.xq_perm, self.xs_perm,
-                                self.xq if self.fs > 0 else None, self.xs if self.fs > 0 else None, s)
+                                self.xq if tok else None, self.xs if tok else None, s)
         elif self.w.mxfp8:
             L.moe_permute_mxfp8(c, x, self.topk_idx, self.row_of_slot, self.offsets, self.xq_perm, self.xs_perm,
-                                self.xq if self.fs > 0 else None, self.xs if self.fs > 0 else None, s)
+                                self.xq if tok else None, self.xs if tok else None, s)
         elif fp8:
             L.moe_permute_fp8(c, x, self.row_of_slot, self.xq_perm, self.xs_perm,
-                              self.xq if self.fs > 0 else None, self.xs if self.fs > 0 else None, s)
+                              self.xq if tok else None, self.xs if tok else None, s)
         rec(2)
         if fp8:
             self._ffn_fp8(c, self.xq_perm, self.xs_perm, T * self.w.k, self.offsets, self.w.N,

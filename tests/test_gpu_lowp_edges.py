@@ -93,3 +93,25 @@ def test_all_tokens_one_expert(mode):
     out = O.layer_forward(f64(inp["x"]), None, oracle_cfg(w), expert_weights_fn(inp), None,
                           routing={"idx": i64(lay.topk_idx), "w": f64(lay.topk_w)}, expert_ffn=ffn)
     assert rel_err(f64(lay.y[:w.T]), out["y"]) < TOL
+
+
+@pytest.mark.parametrize("mode", ["fp8", "mxfp8", "nvfp4"])
+@pytest.mark.parametrize("T", [777, 100])
+def test_shared_expert_on_side_stream_equals_main_stream(mode, T):
+    """Low-precision shared experts quantised and computed on a side stream during route
+    and permute give the same output bit for bit as after the routed experts on the main
+    stream (whose input codes the quantising scatter writes)."""
+    flags = {"fp8": dict(fp8=True), "mxfp8": dict(mxfp8=True), "nvfp4": dict(nvfp4=True)}[mode]
+    w = replace(WORKLOADS["deepseekmoe_16b"], name=f"dsmoe_{mode}_small", T=T, d=512, N=16, k=6, f=256,
+                n_shared=1, f_shared=512, **flags)
+    inp = make_inputs(w, "cuda")
+    a = MoELayer(w, inp, "cuda", update_bias=False, overlap_shared=False)
+    b = MoELayer(w, inp, "cuda", update_bias=False, overlap_shared=True)
+    assert b.overlap_shared and not a.overlap_shared
+    ya = a.forward(inp["x"]).clone()
+    for _ in range(2):
+        yb = b.forward(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert L.moe_device_status() == L.MOE_OK
+    assert torch.equal(ya, yb)
+    assert torch.equal(a.ys[:T], b.ys[:T])
