@@ -246,6 +246,33 @@ def test_round_plan_invariants():
             assert R == 1
 
 
+def test_device_plan_capacity_always_fits_one_round():
+    """The device-side plan's receive buffer, W * T * min(k, N / W) rows, holds every row a
+    rank can receive: random routings, skewed ones and the worst case (every token of every
+    rank picks k experts of one rank) all plan into a single round."""
+    from sparse_mixture_experts_21_b200.ep import plan_rounds
+    from sparse_mixture_experts_21_b200.synth import random_routing
+    rng = np.random.default_rng(5)
+    for W, N, k, T in [(2, 8, 2, 50), (4, 16, 4, 64), (4, 8, 6, 40), (8, 64, 8, 30)]:
+        El = N // W
+        cap = W * T * min(k, El)
+        cases = []
+        for seed in range(3):
+            idx = [random_routing(T, N, k, "cpu", seed=100 * seed + r, hot=(r if seed == 1 else None)).numpy()
+                   for r in range(W)]
+            cases.append(np.stack([np.bincount(i.reshape(-1), minlength=N) for i in idx]))
+        # worst case: every token of every rank picks experts of rank 0 only (min(k, El) of them)
+        worst = np.zeros((W, N), np.int64)
+        worst[:, :min(k, El)] = T
+        cases.append(worst)
+        for kept in cases:
+            recv = [int(kept[:, d * El:(d + 1) * El].sum()) for d in range(W)]
+            assert max(recv) <= cap
+            _, R = plan_rounds(kept, W, cap)
+            assert R == 1
+        assert int(worst[:, :El].sum()) == cap                 # the bound is reached
+
+
 EPR_N, EPR_WORLD, EPR_D, EPR_CAP = 8, 2, 4, 7
 
 
