@@ -10,7 +10,9 @@ Orchestration only; every data-path step runs in the library's kernels:
      receives are bounded by its receive buffer (recv_factor * T * k rows, at
      least T): a destination's (source, expert) pieces are packed, in expert then
      source order, into rounds that each fit the buffer, and every rank runs as
-     many rounds as the busiest destination needs;
+     many rounds as the busiest destination needs.  (With the peer exchange and
+     device_plan=True the buffer holds every row a rank can receive, one round
+     always suffices, and the offsets never leave the device.);
   4. per round: all-to-all of the round's rows; moe_ep_plan + moe_rows_move regroup
      them by local expert; grouped SwiGLU FFN over the local experts; moe_rows_move
      back to arrival order; all-to-all back into the owning ranks' y_perm;
