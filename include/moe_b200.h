@@ -607,8 +607,11 @@ int moe_ep_peer_dispatch(const moe_config_t* cfg, const void* x, const int32_t* 
 
 /* moe_ep_peer_collect -- y_perm[i] = *row_addr[i] for i < min(*n_rows, rows_cap) with
  * row_addr[i] != 0: one round's results back into this rank's expert-ordered rows.
- *   y_perm [rows_cap, d] cfg->x_dtype out (16-byte aligned)
- * Errors: MOE_ERR_INVALID_ARG for a bad config, NULL or misaligned y_perm. */
+ *   row_addr [rows_cap] uint64 (device) from moe_ep_peer_plan
+ *   n_rows   device int32 scalar: this rank's rows (offsets[N] from moe_permute)
+ *   y_perm   [rows_cap, d] cfg->x_dtype out (16-byte aligned)
+ * Errors: MOE_ERR_INVALID_ARG for a bad config, rows_cap < 0, NULL row_addr or n_rows,
+ * NULL or misaligned y_perm. */
 int moe_ep_peer_collect(const moe_config_t* cfg, const uint64_t* row_addr, const int32_t* n_rows, int64_t rows_cap,
                         void* y_perm, void* stream);
 
